@@ -1,0 +1,221 @@
+/*
+ * libsoup — layer-streamed NF4 + LoRA training step on one B200 (sm_100a).
+ *
+ * The method (as described on the pages about the open-source "Soup" trainer):
+ *   - the frozen base model is kept outside GPU memory and fed to the GPU one decoder
+ *     layer at a time: load the layer, compute its activation, drop it, go to the next
+ *     (rug.gal radar "Soup ... layer streaming", section "En detalle"; imasters "Como cabe um
+ *     8B em 4 GB");
+ *   - the base is NF4 4-bit quantised; only the LoRA adapters and the current batch stay on
+ *     the GPU (same sections; soup.yaml example with `stream_layers: true`, `quantization: 4bit`);
+ *   - streamed and resident runs give the same result bit for bit, because streaming only
+ *     reorders when data reaches the GPU (rug.gal "En detalle"; guillermodelpino "El streaming
+ *     de capas, que es el truco de la casa"; imasters "Do SFT para os métodos de preferência");
+ *   - DPO obtains its reference log-probs by re-streaming the same base with the LoRA adapters
+ *     switched off: one set of weights, one stream (rug.gal "En detalle"; imasters "Do SFT ...").
+ *
+ * Conventions for every entry point:
+ *   - every call returns soup_status: SOUP_OK (0) or a negative code; no exception crosses
+ *     the boundary; out-parameters are written only on success;
+ *   - soup_last_error(model) returns a message owned by the model, valid until the next call;
+ *   - "device" pointers are CUDA device addresses on the model's device, "host" pointers are
+ *     CPU addresses; bf16 tensors are passed as their 16-bit patterns;
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream); calls
+ *     enqueue work on it and return without synchronising unless stated; the layer streamer
+ *     uses one internal copy stream fenced with CUDA events;
+ *   - a model is not thread-safe: one host thread at a time per model;
+ *   - shapes: hidden, head_dim*heads, intermediate and lora_r must be multiples of 8;
+ *     head_dim must be 64 or 128; vocab a multiple of 4.  Other shapes -> SOUP_ERR_UNSUPPORTED.
+ */
+#ifndef SOUP_H_
+#define SOUP_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int32_t soup_status;
+#define SOUP_OK 0
+#define SOUP_ERR_INVALID_ARG (-1)  /* null pointer, out-of-range index, bad size */
+#define SOUP_ERR_STATE (-2)        /* wrong call order (e.g. backward without forward, missing weights) */
+#define SOUP_ERR_OOM (-3)          /* host pinned or device allocation failed */
+#define SOUP_ERR_CUDA (-4)         /* a CUDA runtime call failed */
+#define SOUP_ERR_TIMEOUT (-5)      /* a bounded wait (host event or in-kernel barrier) ran out */
+#define SOUP_ERR_DEVICE_CHECK (-6) /* a kernel's bounds check fired (e.g. token id >= vocab) */
+#define SOUP_ERR_UNSUPPORTED (-7)  /* shape outside what the kernels implement */
+
+typedef struct soup_model soup_model;
+
+enum { SOUP_RESIDENT = 0, SOUP_STREAMED = 1 };
+enum { SOUP_PROJ_Q = 0, SOUP_PROJ_K, SOUP_PROJ_V, SOUP_PROJ_O, SOUP_PROJ_GATE, SOUP_PROJ_UP, SOUP_PROJ_DOWN, SOUP_N_PROJ };
+typedef enum { SOUP_LOSS_SFT = 0, SOUP_LOSS_DPO = 1 } soup_loss;
+
+/* Model shape and run options.  Decoder layer = pre-norm Llama block (RMSNorm, GQA attention
+ * with rotate-half RoPE, SwiGLU MLP), LoRA on all seven projections with scale alpha/r. */
+typedef struct soup_model_config {
+  int n_layers, hidden, n_heads, n_kv_heads, head_dim, intermediate, vocab;
+  float rms_eps, rope_theta;
+  int lora_r;
+  float lora_alpha;
+  int mode;            /* SOUP_RESIDENT (every layer on the device) or SOUP_STREAMED */
+  int n_layer_buffers; /* streamed: device layer buffers, >= 2 (the resident-layer budget) */
+  int max_tokens;      /* largest B*S any call will use (sizes the activation storage) */
+  int device;          /* CUDA device ordinal */
+} soup_model_config;
+
+/* Optional device allocator (e.g. routed to PyTorch's caching allocator).  alloc returns
+ * NULL on failure.  With a NULL soup_allocator the library calls cudaMalloc / cudaFree. */
+typedef struct soup_allocator {
+  void* (*alloc)(size_t bytes, void* user);
+  void (*free)(void* ptr, void* user);
+  void* user;
+} soup_allocator;
+
+/* Per-model counters since creation (or the last soup_reset_stats). */
+typedef struct soup_stats {
+  long long layer_loads;      /* host->device layer copies issued by the streamer */
+  long long bytes_h2d;        /* bytes of those copies */
+  long long layer_reuses;     /* layer requests served by an already-resident buffer */
+  long long kernel_launches;  /* kernels this model's calls launched */
+  long long device_bytes;     /* device bytes the model holds (weights buffers, activations, scratch) */
+  long long pinned_bytes;     /* page-locked host bytes holding the NF4 layer stack */
+  long long steps;            /* completed soup_step calls */
+} soup_stats;
+
+/* One training batch.  Token ids are [B, S] row-major int32.
+ * SFT: row t = (b, s) predicts ids[b, s+1]; targets are positions j >= 1 of each sequence,
+ *      optionally filtered by loss_mask[b, j] != 0 (uint8 [B, S]); loss = token mean.
+ * DPO: B = 2 * n_pairs; rows 2p (chosen) and 2p+1 (rejected); response targets are
+ *      j >= prefix_len; loss = -mean_p log sigmoid(beta [(pi_c - ref_c) - (pi_r - ref_r)]),
+ *      pi = summed target log-probs (fp32) with LoRA on, ref = the same with LoRA off.
+ * ids_on_host != 0: ids / loss_mask are host pointers; the library copies them to the device
+ *      on `stream` inside the call (pageable or pinned memory both accepted). */
+typedef struct soup_batch {
+  const int32_t* ids;
+  const uint8_t* loss_mask; /* may be NULL */
+  int B, S;
+  int ids_on_host;
+  int n_pairs, prefix_len;
+  float beta;
+  float lr;            /* AdamW learning rate (betas 0.9/0.999, eps 1e-8, weight decay 0) */
+  int apply_optimizer; /* 0: leave gradients in the grad buffer, do not update */
+} soup_batch;
+
+/* ---- lifecycle -------------------------------------------------------------------------- */
+
+/* Creates a model: validates cfg, computes the NF4 codebook, allocates the page-locked host
+ * layer stack (n_layers blobs), the device layer buffers (n_layers resident, n_layer_buffers
+ * streamed), activation storage for max_tokens and scratch.  Weights are loaded afterwards. */
+soup_status soup_model_create(const soup_model_config* cfg, const soup_allocator* alloc, soup_model** out);
+soup_status soup_model_destroy(soup_model* model);
+
+/* Bytes of one layer's NF4 blob (7 projections: codes, q8 absmax, fp32 group scales, fp32
+ * mean; then the two bf16 RMSNorm gains), each part 256-byte aligned. */
+soup_status soup_layer_blob_bytes(const soup_model_config* cfg, size_t* bytes);
+
+/* Quantises one layer on the device into the model's host layer stack.
+ * w[p]: device fp32 [out_p, in_p] row-major for p = q,k,v,o,gate,up,down; gammas: device bf16
+ * [hidden].  Runs the NF4 + double-quant kernels, then copies the blob to page-locked host
+ * memory (synchronises `stream`).  In resident mode the blob is also kept on the device. */
+soup_status soup_model_quantize_layer(soup_model* model, int layer, const float* const w[7],
+                                      const uint16_t* gamma_attn, const uint16_t* gamma_mlp, void* stream);
+/* Loads / reads back a pre-quantised blob (host memory, soup_layer_blob_bytes bytes). */
+soup_status soup_model_load_layer_nf4(soup_model* model, int layer, const void* blob, size_t bytes);
+soup_status soup_model_read_layer_nf4(soup_model* model, int layer, void* blob, size_t bytes);
+/* Byte offset and size of a part of projection p inside a layer blob; part 0 = codes, 1 = q8
+ * absmax, 2 = group scales, 3 = mean; p = 7 gives the attention gain, p = 8 the MLP gain. */
+soup_status soup_layer_blob_part(const soup_model_config* cfg, int proj, int part, size_t* offset, size_t* bytes);
+
+/* Frozen head weights (device, bf16, caller-owned, kept by pointer): embedding [vocab, hidden],
+ * final RMSNorm gain [hidden], lm_head [vocab, hidden]. */
+soup_status soup_model_set_head(soup_model* model, const void* embed, const void* final_gamma, const void* lm_head);
+
+/* LoRA storage: four caller-owned device fp32 buffers of soup_lora_numel elements each
+ * (parameters, gradients, AdamW first and second moments; moments start at zero).  Layout:
+ * layer-major; inside a layer A_q, A_k, A_v, A_o, A_gate, A_up, A_down (each [r, in]) then
+ * B_q, ..., B_down (each [out, r]), row-major.  soup_lora_offset gives each tensor's place. */
+soup_status soup_lora_numel(const soup_model_config* cfg, size_t* numel);
+soup_status soup_lora_offset(const soup_model_config* cfg, int layer, int proj, int which_b, size_t* offset,
+                             int* rows, int* cols);
+soup_status soup_model_set_lora(soup_model* model, float* params, float* grads, float* adam_m, float* adam_v);
+
+/* LoRA on/off for the forward and backward calls that follow.  Off: the LoRA branch and its
+ * gradients are skipped entirely (not multiplied by zero), which is the DPO reference model. */
+soup_status soup_set_lora_enabled(soup_model* model, int enabled);
+
+/* ---- layer-level calls ------------------------------------------------------------------- */
+
+/* One decoder layer forward: x_out = layer(x_in), device bf16 [B*S, hidden].  Acquires the
+ * layer from the streamer (or the resident copy), keeps the activations needed by
+ * soup_layer_bwd inside the model (per layer), runs every kernel on `stream`. */
+soup_status soup_layer_fwd(soup_model* model, int layer, const void* x_in, void* x_out, int B, int S, void* stream);
+/* Backward of the last soup_layer_fwd of this layer: dx = d(loss)/d(x_in) given
+ * dy = d(loss)/d(x_out) (device bf16 [B*S, hidden]); ACCUMULATES the layer's LoRA gradients
+ * into the grad buffer (callers zero it first).  SOUP_ERR_STATE without a matching forward. */
+soup_status soup_layer_bwd(soup_model* model, int layer, const void* dy, void* dx, int B, int S, void* stream);
+
+/* ---- whole step -------------------------------------------------------------------------- */
+
+/* One training step: embedding, streamed forward over all layers, head and loss, streamed
+ * backward, LoRA gradients (zeroed first) and, if batch->apply_optimizer, the AdamW update.
+ * SFT streams 2L-2 layer loads from a cold streamer (the two top layers are reused at the
+ * forward/backward turnaround); DPO adds a full LoRA-off forward pass, 3L-2 loads.  Layers
+ * still resident from the previous step are reused.  *loss_out (host) receives the loss
+ * after the call synchronises `stream`. */
+soup_status soup_step(soup_model* model, soup_loss loss, const soup_batch* batch, float* loss_out, void* stream);
+/* AdamW update of all LoRA parameters from the grad buffer (step counter kept by the model). */
+soup_status soup_optimizer_step(soup_model* model, float lr, void* stream);
+/* Per-sequence summed target log-probs of the last DPO step (host fp32[B]): policy and ref. */
+soup_status soup_last_logps(soup_model* model, float* pi, float* ref, int n);
+
+/* ---- single operations (each one kernel sequence, for tests and tools) ------------------- */
+
+/* NF4 + double quantisation of one device fp32 tensor of n elements (row-major flattened):
+ * codes [ceil(n/2)] u8, q8 [ceil(n/64)] i8, scales [ceil(n/64/256)] f32, mean [1] f32, all
+ * device; scratch: device f32 [ceil(n/64)] (absmax). */
+soup_status soup_nf4_quantize(const float* w, long long n, uint8_t* codes, int8_t* q8, float* scales, float* mean,
+                              float* scratch, void* stream);
+/* Standalone NF4 -> bf16 dequantiser: out[i] = bf16_rn(c[code_i] * mhat(block(i))). */
+soup_status soup_nf4_dequantize(const uint8_t* codes, const int8_t* q8, const float* scales, const float* mean,
+                                long long n, uint16_t* out, void* stream);
+/* y[M, N] (bf16) = x[M, K] (bf16) . W^T + (residual) for one NF4 tensor W [N, K] (device
+ * parts as produced by soup_nf4_quantize); transpose_w != 0 computes y[M, K] = x[M, N] . W. */
+soup_status soup_nf4_matmul(const void* x, int M, int N, int K, const uint8_t* codes, const int8_t* q8,
+                            const float* scales, const float* mean, int transpose_w, const void* residual, void* y,
+                            void* stream);
+/* The 16 NF4 levels this library uses (host fp32[16]). */
+soup_status soup_nf4_codebook(float* out16);
+
+/* ---- diagnostics ------------------------------------------------------------------------- */
+soup_status soup_get_stats(soup_model* model, soup_stats* out);
+soup_status soup_reset_stats(soup_model* model);
+/* Live per-kernel profile.  While enabled, every launch a model call makes is bracketed by
+ * CUDA events on the stream it runs on (the H2D layer copies on the streamer's copy stream)
+ * and accumulated per category: launches, device milliseconds and the launch's algorithmic
+ * work (flops of the dense contraction, bytes of its inputs and outputs).  Adds one event
+ * pair per launch; soup_get_profile synchronises the recorded events. */
+typedef struct soup_profile_entry {
+  char name[32];
+  long long launches;
+  double total_ms;
+  double flops;
+  double bytes;
+} soup_profile_entry;
+soup_status soup_set_profiling(soup_model* model, int enabled);
+/* Copies up to max_entries categories (those with launches) into out; *n_entries = count.
+ * Clears the accumulated profile when reset != 0. */
+soup_status soup_get_profile(soup_model* model, soup_profile_entry* out, int max_entries, int* n_entries, int reset);
+
+/* Reads (and clears) the device error word; SOUP_ERR_TIMEOUT / SOUP_ERR_DEVICE_CHECK if set. */
+soup_status soup_check_device(soup_model* model, void* stream);
+const char* soup_status_string(soup_status status);
+const char* soup_last_error(const soup_model* model);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SOUP_H_ */

@@ -1,0 +1,470 @@
+// Row and elementwise kernels of the decoder layer and the loss head (sm_100a).
+// Memory-bound: 16-byte vector loads/stores, fp32 math, fixed-order block reductions
+// (warp shuffles + one shared-memory pass) so results are deterministic run to run.
+#include "common.cuh"
+#include "internal.h"
+
+namespace soup {
+
+std::atomic<long long> g_kernel_launches{0};
+
+namespace {
+
+__device__ __forceinline__ void load8(const uint16_t* p, float (&v)[8]) {
+  const uint4 u = *reinterpret_cast<const uint4*>(p);
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float2 f = unpack_bf16x2(w[j]);
+    v[2 * j] = f.x;
+    v[2 * j + 1] = f.y;
+  }
+}
+__device__ __forceinline__ void store8(uint16_t* p, const float (&v)[8]) {
+  *reinterpret_cast<uint4*>(p) =
+      make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+}
+
+// ---------------------------------------------------------------- embedding gather
+__global__ void embed_kernel(const int32_t* __restrict__ ids, const uint16_t* __restrict__ table, int h, int V,
+                             uint16_t* __restrict__ out, int* err) {
+  const int t = blockIdx.x;
+  const int id = ids[t];
+  const bool ok = (id >= 0 && id < V);
+  if (!ok && threadIdx.x == 0) set_dev_error(err, DEVERR_BOUNDS);
+  for (int c = threadIdx.x * 8; c < h; c += blockDim.x * 8) {
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (ok) v = *reinterpret_cast<const uint4*>(table + static_cast<long long>(id) * h + c);
+    *reinterpret_cast<uint4*>(out + static_cast<long long>(t) * h + c) = v;
+  }
+}
+
+// ---------------------------------------------------------------- RMSNorm
+// y = x * rstd * gamma, rstd = 1/sqrt(mean(x^2) + eps); one CTA per row.
+__global__ void rmsnorm_fwd_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ gamma, int h, float eps,
+                                   uint16_t* __restrict__ y, float* __restrict__ rstd) {
+  __shared__ float red[32];
+  const long long row = blockIdx.x;
+  const uint16_t* xr = x + row * h;
+  float ss = 0.f;
+  for (int c = threadIdx.x * 8; c < h; c += blockDim.x * 8) {
+    float v[8];
+    load8(xr + c, v);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) ss += v[j] * v[j];
+  }
+  ss = block_sum(ss, red);
+  const float r = rsqrtf(ss / static_cast<float>(h) + eps);
+  if (threadIdx.x == 0) rstd[row] = r;
+  for (int c = threadIdx.x * 8; c < h; c += blockDim.x * 8) {
+    float v[8], g[8];
+    load8(xr + c, v);
+    load8(gamma + c, g);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] = v[j] * r * g[j];
+    store8(y + row * h + c, v);
+  }
+}
+
+// dx = dres + rstd*gamma*dy - x * rstd^3 * sum(gamma*dy*x)/h
+__global__ void rmsnorm_bwd_kernel(const uint16_t* __restrict__ dy, const uint16_t* __restrict__ x,
+                                   const float* __restrict__ rstd, const uint16_t* __restrict__ gamma,
+                                   const uint16_t* __restrict__ dres, int h, uint16_t* __restrict__ dx) {
+  __shared__ float red[32];
+  const long long row = blockIdx.x;
+  const float r = rstd[row];
+  float dot = 0.f;
+  for (int c = threadIdx.x * 8; c < h; c += blockDim.x * 8) {
+    float a[8], b[8], g[8];
+    load8(dy + row * h + c, a);
+    load8(x + row * h + c, b);
+    load8(gamma + c, g);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) dot += g[j] * a[j] * b[j];
+  }
+  dot = block_sum(dot, red);
+  const float k = r * r * r * dot / static_cast<float>(h);
+  for (int c = threadIdx.x * 8; c < h; c += blockDim.x * 8) {
+    float a[8], b[8], g[8], o[8];
+    load8(dy + row * h + c, a);
+    load8(x + row * h + c, b);
+    load8(gamma + c, g);
+    if (dres) {
+      load8(dres + row * h + c, o);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) o[j] = 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) o[j] += r * g[j] * a[j] - b[j] * k;
+    store8(dx + row * h + c, o);
+  }
+}
+
+// ---------------------------------------------------------------- RoPE (rotate-half, in place)
+// angle = pos * theta^(-2i/d), pos = t mod S. inverse != 0 rotates by -angle (the backward).
+__global__ void rope_kernel(uint16_t* __restrict__ qkv, long long ld, int S, int nheads, int d, double log_theta,
+                            int inverse) {
+  const int t = blockIdx.x;
+  const int half = d / 2;
+  const double pos = static_cast<double>(t % S);
+  uint16_t* row = qkv + static_cast<long long>(t) * ld;
+  for (int idx = threadIdx.x; idx < nheads * half; idx += blockDim.x) {
+    const int hh = idx / half, i = idx % half;
+    const double ang = pos * exp(-log_theta * (2.0 * i) / d);
+    double sd, cd;
+    sincos(ang, &sd, &cd);
+    const float s = inverse ? -static_cast<float>(sd) : static_cast<float>(sd);
+    const float c = static_cast<float>(cd);
+    uint16_t* z = row + hh * d;
+    const float z1 = bf16_to_f32(z[i]), z2 = bf16_to_f32(z[i + half]);
+    const __nv_bfloat16 o1 = __float2bfloat16_rn(z1 * c - z2 * s);
+    const __nv_bfloat16 o2 = __float2bfloat16_rn(z2 * c + z1 * s);
+    z[i] = *reinterpret_cast<const uint16_t*>(&o1);
+    z[i + half] = *reinterpret_cast<const uint16_t*>(&o2);
+  }
+}
+
+// ---------------------------------------------------------------- SwiGLU
+__global__ void swiglu_fwd_kernel(const uint16_t* __restrict__ gu, int I, long long total8, uint16_t* __restrict__ m) {
+  const long long i8 = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i8 >= total8) return;
+  const long long e = i8 * 8;
+  const long long t = e / I, c = e % I;
+  float g[8], u[8], o[8];
+  load8(gu + t * 2 * I + c, g);
+  load8(gu + t * 2 * I + I + c, u);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) o[j] = g[j] / (1.f + expf(-g[j])) * u[j];
+  store8(m + t * I + c, o);
+}
+
+__global__ void swiglu_bwd_kernel(const uint16_t* __restrict__ dm, const uint16_t* __restrict__ gu, int I,
+                                  long long total8, uint16_t* __restrict__ dgu) {
+  const long long i8 = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i8 >= total8) return;
+  const long long e = i8 * 8;
+  const long long t = e / I, c = e % I;
+  float g[8], u[8], d[8], dg[8], du[8];
+  load8(gu + t * 2 * I + c, g);
+  load8(gu + t * 2 * I + I + c, u);
+  load8(dm + t * I + c, d);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const float sg = 1.f / (1.f + expf(-g[j]));
+    du[j] = d[j] * g[j] * sg;
+    dg[j] = d[j] * u[j] * sg * (1.f + g[j] * (1.f - sg));
+  }
+  store8(dgu + t * 2 * I + c, dg);
+  store8(dgu + t * 2 * I + I + c, du);
+}
+
+// ---------------------------------------------------------------- cross-entropy rows
+// Row t (position s of sequence b) predicts ids[b, s+1]. Writes lse[t] and the target logit.
+__global__ void ce_rows_kernel(const float* __restrict__ logits, int V, const int32_t* __restrict__ ids, int S,
+                               float* __restrict__ lse, float* __restrict__ tgt, int* err) {
+  __shared__ float red[32];
+  const long long t = blockIdx.x;
+  const float4* row = reinterpret_cast<const float4*>(logits + t * V);
+  float mx = -INFINITY, sm = 0.f;
+  for (int c = threadIdx.x; c < V / 4; c += blockDim.x) {
+    const float4 v = row[c];
+    const float lm = fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w));
+    if (lm > mx) {
+      sm *= expf(mx - lm);
+      mx = lm;
+    }
+    sm += expf(v.x - mx) + expf(v.y - mx) + expf(v.z - mx) + expf(v.w - mx);
+  }
+  const float M = block_max(mx, red);
+  const float part = (mx == -INFINITY) ? 0.f : sm * expf(mx - M);
+  const float tot = block_sum(part, red);
+  if (threadIdx.x == 0) {
+    lse[t] = M + logf(tot);
+    const int s = static_cast<int>(t % S);
+    float tv = 0.f;
+    if (s + 1 < S) {
+      const int id = ids[t + 1];
+      if (id >= 0 && id < V)
+        tv = logits[t * V + id];
+      else
+        set_dev_error(err, DEVERR_BOUNDS);
+    }
+    tgt[t] = tv;
+  }
+}
+
+// SFT: loss = sum over counted targets (lse - target logit) / N; row weight 1/N for counted rows.
+__global__ void sft_finish_kernel(const float* __restrict__ lse, const float* __restrict__ tgt, int B, int S,
+                                  const uint8_t* __restrict__ mask, float* __restrict__ loss_out,
+                                  float* __restrict__ row_weight) {
+  __shared__ double redd[32];
+  __shared__ int redn[32];
+  const int T = B * S;
+  double acc = 0.0;
+  int cnt = 0;
+  for (int t = threadIdx.x; t < T; t += blockDim.x) {
+    const int s = t % S;
+    const bool valid = (s + 1 < S) && (mask == nullptr || mask[t + 1] != 0);
+    if (valid) {
+      acc += static_cast<double>(lse[t]) - static_cast<double>(tgt[t]);
+      ++cnt;
+    }
+  }
+  // fixed-order reduction
+  for (int o = 16; o > 0; o >>= 1) {
+    acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+  }
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  if (lane == 0) {
+    redd[wid] = acc;
+    redn[wid] = cnt;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double a = 0.0;
+    int n = 0;
+    for (int w = 0; w < nw; ++w) {
+      a += redd[w];
+      n += redn[w];
+    }
+    redd[0] = a;
+    redn[0] = n;
+    loss_out[0] = (n > 0) ? static_cast<float>(a / n) : 0.f;
+  }
+  __syncthreads();
+  const int n = redn[0];
+  const float w = (n > 0) ? 1.f / static_cast<float>(n) : 0.f;
+  for (int t = threadIdx.x; t < T; t += blockDim.x) {
+    const int s = t % S;
+    const bool valid = (s + 1 < S) && (mask == nullptr || mask[t + 1] != 0);
+    row_weight[t] = valid ? w : 0.f;
+  }
+}
+
+// Per-sequence sum of target log-probs over targets j in [max(start,1), S), fp32 accumulation
+// in a fixed order (thread-strided partial sums, then a fixed tree).
+__global__ void seq_logp_kernel(const float* __restrict__ lse, const float* __restrict__ tgt, int S, int start,
+                                float* __restrict__ out) {
+  __shared__ float red[32];
+  const int b = blockIdx.x;
+  const int j0 = start > 1 ? start : 1;
+  float acc = 0.f;
+  for (int j = j0 + threadIdx.x; j < S; j += blockDim.x) {
+    const long long t = static_cast<long long>(b) * S + j - 1;
+    acc += tgt[t] - lse[t];
+  }
+  acc = block_sum(acc, red);
+  if (threadIdx.x == 0) out[b] = acc;
+}
+
+// DPO closed form on P pairs (rows 2p chosen, 2p+1 rejected); row weights = -dL/dpi on the
+// response rows so that dlogits = w * (softmax - onehot).
+__global__ void dpo_finish_kernel(const float* __restrict__ pi, const float* __restrict__ ref, int B, int S, int start,
+                                  int P, float beta, float* __restrict__ loss_out, float* __restrict__ row_weight) {
+  __shared__ float wrow[64];
+  if (threadIdx.x == 0) {
+    double loss = 0.0;
+    for (int p = 0; p < P; ++p) {
+      const double z = static_cast<double>(beta) * ((static_cast<double>(pi[2 * p]) - ref[2 * p]) -
+                                                    (static_cast<double>(pi[2 * p + 1]) - ref[2 * p + 1]));
+      loss += (z > 0) ? log1p(exp(-z)) : (-z + log1p(exp(z)));  // -log sigmoid(z)
+      const double sneg = 1.0 / (1.0 + exp(z));                  // sigmoid(-z)
+      const double dc = -static_cast<double>(beta) * sneg / P;
+      wrow[2 * p] = static_cast<float>(-dc);
+      wrow[2 * p + 1] = static_cast<float>(dc);
+    }
+    loss_out[0] = static_cast<float>(loss / P);
+  }
+  __syncthreads();
+  const int j0 = start > 1 ? start : 1;
+  for (int t = threadIdx.x; t < B * S; t += blockDim.x) {
+    const int b = t / S, j = t % S + 1;
+    row_weight[t] = (j >= j0 && j < S) ? wrow[b] : 0.f;
+  }
+}
+
+// dlogits[t, v] = w_t * (exp(logit - lse_t) - [v == target_t]), rounded to bf16.
+__global__ void ce_grad_kernel(const float* __restrict__ logits, const float* __restrict__ lse,
+                               const int32_t* __restrict__ ids, const float* __restrict__ row_weight, int S, int V,
+                               uint16_t* __restrict__ dl) {
+  const long long t = blockIdx.x;
+  const float w = row_weight[t];
+  const int s = static_cast<int>(t % S);
+  const int target = (s + 1 < S) ? ids[t + 1] : -1;
+  const float l = lse[t];
+  const float4* row = reinterpret_cast<const float4*>(logits + t * V);
+  uint2* out = reinterpret_cast<uint2*>(dl + t * V);
+  for (int c = threadIdx.x; c < V / 4; c += blockDim.x) {
+    float o[4] = {0.f, 0.f, 0.f, 0.f};
+    if (w != 0.f) {
+      const float4 v = row[c];
+      const float x[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        o[j] = w * (expf(x[j] - l) - ((4 * c + j) == target ? 1.f : 0.f));
+      }
+    }
+    out[c] = make_uint2(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]));
+  }
+}
+
+// ---------------------------------------------------------------- AdamW (fp32, bias-corrected)
+__global__ void adamw_kernel(float* __restrict__ p, const float* __restrict__ g, float* __restrict__ m,
+                             float* __restrict__ v, long long n, float lr, float b1, float b2, float eps, float wd,
+                             float bc1, float bc2) {
+  const long long i4 = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i4 * 4 >= n) return;
+  if (i4 * 4 + 4 <= n) {
+    float4 pp = reinterpret_cast<float4*>(p)[i4];
+    const float4 gg = reinterpret_cast<const float4*>(g)[i4];
+    float4 mm = reinterpret_cast<float4*>(m)[i4];
+    float4 vv = reinterpret_cast<float4*>(v)[i4];
+    float* P = &pp.x;
+    const float* G = &gg.x;
+    float* Mv = &mm.x;
+    float* Vv = &vv.x;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      Mv[j] = b1 * Mv[j] + (1.f - b1) * G[j];
+      Vv[j] = b2 * Vv[j] + (1.f - b2) * G[j] * G[j];
+      const float mh = Mv[j] * bc1, vh = Vv[j] * bc2;
+      P[j] = P[j] - lr * (mh / (sqrtf(vh) + eps) + wd * P[j]);
+    }
+    reinterpret_cast<float4*>(p)[i4] = pp;
+    reinterpret_cast<float4*>(m)[i4] = mm;
+    reinterpret_cast<float4*>(v)[i4] = vv;
+  } else {
+    for (long long i = i4 * 4; i < n; ++i) {
+      m[i] = b1 * m[i] + (1.f - b1) * g[i];
+      v[i] = b2 * v[i] + (1.f - b2) * g[i] * g[i];
+      const float mh = m[i] * bc1, vh = v[i] * bc2;
+      p[i] = p[i] - lr * (mh / (sqrtf(vh) + eps) + wd * p[i]);
+    }
+  }
+}
+
+int row_threads(int h) {
+  int t = h / 8;
+  if (t > 512) t = 512;
+  t = ((t + 31) / 32) * 32;
+  return t < 32 ? 32 : t;
+}
+
+}  // namespace
+
+cudaError_t embed_launch(const int32_t* ids, const uint16_t* table, int T, int h, int V, uint16_t* out, int* err,
+                         cudaStream_t st) {
+  if (T <= 0) return cudaSuccess;
+  embed_kernel<<<T, row_threads(h), 0, st>>>(ids, table, h, V, out, err);
+  ++g_kernel_launches;
+  return cudaGetLastError();
+}
+
+cudaError_t rmsnorm_fwd_launch(const uint16_t* x, const uint16_t* gamma, int T, int h, float eps, uint16_t* y,
+                               float* rstd, cudaStream_t st) {
+  if (T <= 0) return cudaSuccess;
+  rmsnorm_fwd_kernel<<<T, row_threads(h), 0, st>>>(x, gamma, h, eps, y, rstd);
+  ++g_kernel_launches;
+  return cudaGetLastError();
+}
+
+cudaError_t rmsnorm_bwd_launch(const uint16_t* dy, const uint16_t* x, const float* rstd, const uint16_t* gamma,
+                               const uint16_t* dres, int T, int h, uint16_t* dx, cudaStream_t st) {
+  if (T <= 0) return cudaSuccess;
+  rmsnorm_bwd_kernel<<<T, row_threads(h), 0, st>>>(dy, x, rstd, gamma, dres, h, dx);
+  ++g_kernel_launches;
+  return cudaGetLastError();
+}
+
+cudaError_t rope_launch(uint16_t* qkv, long long ld, int B, int S, int hq, int hkv, int d, float theta, int inverse,
+                        cudaStream_t st) {
+  const int T = B * S;
+  if (T <= 0) return cudaSuccess;
+  const int nheads = hq + hkv;  // q heads then k heads, contiguous from column 0
+  int thr = nheads * d / 2;
+  thr = thr > 256 ? 256 : ((thr + 31) / 32) * 32;
+  rope_kernel<<<T, thr, 0, st>>>(qkv, ld, S, nheads, d, log(static_cast<double>(theta)), inverse);
+  ++g_kernel_launches;
+  return cudaGetLastError();
+}
+
+cudaError_t swiglu_fwd_launch(const uint16_t* gu, int T, int I, uint16_t* m, cudaStream_t st) {
+  const long long total8 = static_cast<long long>(T) * I / 8;
+  if (total8 <= 0) return cudaSuccess;
+  swiglu_fwd_kernel<<<static_cast<unsigned>((total8 + 255) / 256), 256, 0, st>>>(gu, I, total8, m);
+  ++g_kernel_launches;
+  return cudaGetLastError();
+}
+
+cudaError_t swiglu_bwd_launch(const uint16_t* dm, const uint16_t* gu, int T, int I, uint16_t* dgu, cudaStream_t st) {
+  const long long total8 = static_cast<long long>(T) * I / 8;
+  if (total8 <= 0) return cudaSuccess;
+  swiglu_bwd_kernel<<<static_cast<unsigned>((total8 + 255) / 256), 256, 0, st>>>(dm, gu, I, total8, dgu);
+  ++g_kernel_launches;
+  return cudaGetLastError();
+}
+
+cudaError_t ce_rows_launch(const float* logits, int T, int V, const int32_t* ids, int B, int S, const uint8_t* mask,
+                           int resp_start, float* lse, float* tgt_logit, int* err, cudaStream_t st) {
+  (void)B;
+  (void)mask;
+  (void)resp_start;
+  if (T <= 0) return cudaSuccess;
+  ce_rows_kernel<<<T, 512, 0, st>>>(logits, V, ids, S, lse, tgt_logit, err);
+  ++g_kernel_launches;
+  return cudaGetLastError();
+}
+
+cudaError_t sft_finish_launch(const float* lse, const float* tgt, const int32_t* ids, int B, int S, const uint8_t* mask,
+                              float* loss_out, float* row_weight, cudaStream_t st) {
+  (void)ids;
+  sft_finish_kernel<<<1, 1024, 0, st>>>(lse, tgt, B, S, mask, loss_out, row_weight);
+  ++g_kernel_launches;
+  return cudaGetLastError();
+}
+
+cudaError_t seq_logp_launch(const float* lse, const float* tgt, int B, int S, int resp_start, float* out,
+                            cudaStream_t st) {
+  seq_logp_kernel<<<B, 256, 0, st>>>(lse, tgt, S, resp_start, out);
+  ++g_kernel_launches;
+  return cudaGetLastError();
+}
+
+cudaError_t dpo_finish_launch(const float* lse, const float* tgt, int B, int S, int resp_start, int n_pairs, float beta,
+                              const float* ref_logp, float* pi_out, float* loss_out, float* row_weight,
+                              cudaStream_t st) {
+  cudaError_t e = seq_logp_launch(lse, tgt, B, S, resp_start, pi_out, st);
+  if (e != cudaSuccess) return e;
+  dpo_finish_kernel<<<1, 256, 0, st>>>(pi_out, ref_logp, B, S, resp_start, n_pairs, beta, loss_out, row_weight);
+  ++g_kernel_launches;
+  return cudaGetLastError();
+}
+
+cudaError_t ce_grad_launch(const float* logits, const float* lse, const int32_t* ids, const float* row_weight, int B,
+                           int S, int V, uint16_t* dlogits, cudaStream_t st) {
+  const int T = B * S;
+  if (T <= 0) return cudaSuccess;
+  ce_grad_kernel<<<T, 512, 0, st>>>(logits, lse, ids, row_weight, S, V, dlogits);
+  ++g_kernel_launches;
+  return cudaGetLastError();
+}
+
+cudaError_t adamw_launch(float* p, const float* g, float* m, float* v, long long n, float lr, float b1, float b2,
+                         float eps, float wd, int t, cudaStream_t st) {
+  if (n <= 0) return cudaSuccess;
+  const float bc1 = static_cast<float>(1.0 / (1.0 - pow(static_cast<double>(b1), t)));
+  const float bc2 = static_cast<float>(1.0 / (1.0 - pow(static_cast<double>(b2), t)));
+  const long long n4 = (n + 3) / 4;
+  adamw_kernel<<<static_cast<unsigned>((n4 + 255) / 256), 256, 0, st>>>(p, g, m, v, n, lr, b1, b2, eps, wd, bc1, bc2);
+  ++g_kernel_launches;
+  return cudaGetLastError();
+}
+
+cudaError_t fill_zero_launch(void* p, size_t bytes, cudaStream_t st) {
+  if (bytes == 0) return cudaSuccess;
+  return cudaMemsetAsync(p, 0, bytes, st);
+}
+
+}  // namespace soup

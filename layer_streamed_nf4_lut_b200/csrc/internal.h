@@ -1,0 +1,125 @@
+// Internal declarations shared by the libsoup translation units (not part of the C-ABI).
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stddef.h>
+
+#include <atomic>
+
+namespace soup {
+
+// ----------------------------------------------------------------- NF4 tensor views
+// One NF4 tensor W[rows, cols] (row-major flattened, blocks of 64, DQ groups of 256 blocks)
+// stacked at row `row_begin` of a group that a GEMM sees as one matrix.
+struct NF4Seg {
+  const uint8_t* codes;  // packed codes, element 2i in the low nibble of byte i
+  const int8_t* q8;      // double-quantised absmax, one per 64-element block
+  const float* scales;   // fp32 scale per group of 256 blocks
+  const float* mean;     // fp32 per-tensor mean of the absmax (device scalar)
+  int row_begin;
+  int rows;
+};
+struct NF4Group {
+  NF4Seg seg[3];
+  int nseg;
+  int cols;        // in-dimension shared by the stacked tensors (multiple of 8)
+  int total_rows;  // sum of rows
+};
+
+// ----------------------------------------------------------------- GEMM operands
+// Element (r, k) of an operand that the GEMM reads as "row r, reduction index k".
+enum OpKind : int {
+  OP_BF16_K = 0,   // bf16 at ptr[r*ld + k]
+  OP_BF16_MN = 1,  // bf16 at ptr[k*ld + r]
+  OP_F32_K = 2,    // fp32 at ptr[r*ld + k], times `scale`, rounded to bf16
+  OP_F32_MN = 3,   // fp32 at ptr[k*ld + r], times `scale`, rounded to bf16
+  OP_NF4_K = 4,    // W[r, k] of the GEMM's NF4 group (forward: y = x W^T)
+  OP_NF4_MN = 5,   // W[k, r] of the GEMM's NF4 group (backward: dx = dy W)
+};
+
+struct Operand {
+  int kind;
+  const void* ptr;
+  long long ld;
+  float scale;
+  int row_lo, row_hi;  // rows outside [row_lo, row_hi) read as zero (block-diagonal LoRA)
+};
+
+struct GemmSeg {
+  int K;
+  Operand A;  // rows = GEMM M
+  Operand B;  // rows = GEMM N
+};
+
+constexpr int GEMM_MAX_SEG = 5;
+
+struct GemmParams {
+  int M, N;
+  int nseg;
+  GemmSeg seg[GEMM_MAX_SEG];
+  NF4Group nf4;
+  float lut[16];
+  // epilogue: out[r, c] (or out[c, r] when out_trans) = alpha * acc (+ residual) (+ old out)
+  void* out;
+  long long ldo;
+  int out_f32;
+  int out_trans;
+  float alpha;
+  int accumulate;
+  const void* residual;  // bf16, same layout as out (not with out_trans)
+  long long ldr;
+  int* err;
+};
+
+// Launch C = sum_seg A_seg B_seg^T on the tcgen05 tensor cores. Returns cudaError_t of launch.
+cudaError_t gemm_launch(const GemmParams& p, cudaStream_t st);
+
+// ----------------------------------------------------------------- NF4 quantiser / dequant
+struct LUT16 {
+  float v[16];
+};
+cudaError_t nf4_quantize_launch(const float* w, long long n, uint8_t* codes, int8_t* q8, float* scales, float* mean,
+                                float* absmax_scratch, const LUT16& lut, cudaStream_t st);
+cudaError_t nf4_dequant_launch(const uint8_t* codes, const int8_t* q8, const float* scales, const float* mean,
+                               long long n, uint16_t* out, const LUT16& lut, cudaStream_t st);
+
+// ----------------------------------------------------------------- attention
+struct AttnShape {
+  int B, S, hq, hkv, d;
+  long long ld_qkv;  // row stride (elements) of the [T, (hq+2hkv)d] qkv buffer
+};
+cudaError_t attn_fwd_launch(const AttnShape& s, const uint16_t* qkv, uint16_t* o, float* lse, cudaStream_t st);
+cudaError_t attn_bwd_launch(const AttnShape& s, const uint16_t* qkv, const uint16_t* o, const uint16_t* dout,
+                            const float* lse, float* delta, uint16_t* dqkv, cudaStream_t st);
+
+// ----------------------------------------------------------------- elementwise / row ops
+cudaError_t embed_launch(const int32_t* ids, const uint16_t* table, int T, int h, int V, uint16_t* out, int* err,
+                         cudaStream_t st);
+cudaError_t rmsnorm_fwd_launch(const uint16_t* x, const uint16_t* gamma, int T, int h, float eps, uint16_t* y,
+                               float* rstd, cudaStream_t st);
+cudaError_t rmsnorm_bwd_launch(const uint16_t* dy, const uint16_t* x, const float* rstd, const uint16_t* gamma,
+                               const uint16_t* dres, int T, int h, uint16_t* dx, cudaStream_t st);
+cudaError_t rope_launch(uint16_t* qkv, long long ld, int B, int S, int hq, int hkv, int d, float theta, int inverse,
+                        cudaStream_t st);
+cudaError_t swiglu_fwd_launch(const uint16_t* gu, int T, int I, uint16_t* m, cudaStream_t st);
+cudaError_t swiglu_bwd_launch(const uint16_t* dm, const uint16_t* gu, int T, int I, uint16_t* dgu, cudaStream_t st);
+cudaError_t ce_rows_launch(const float* logits, int T, int V, const int32_t* ids, int B, int S, const uint8_t* mask,
+                           int resp_start, float* lse, float* tgt_logit, int* err, cudaStream_t st);
+cudaError_t sft_finish_launch(const float* lse, const float* tgt, const int32_t* ids, int B, int S, const uint8_t* mask,
+                              float* loss_out, float* row_weight, cudaStream_t st);
+cudaError_t dpo_finish_launch(const float* lse, const float* tgt, int B, int S, int resp_start, int n_pairs, float beta,
+                              const float* ref_logp, float* pi_out, float* loss_out, float* row_weight,
+                              cudaStream_t st);
+cudaError_t seq_logp_launch(const float* lse, const float* tgt, int B, int S, int resp_start, float* out,
+                            cudaStream_t st);
+cudaError_t ce_grad_launch(const float* logits, const float* lse, const int32_t* ids, const float* row_weight, int B,
+                           int S, int V, uint16_t* dlogits, cudaStream_t st);
+cudaError_t adamw_launch(float* p, const float* g, float* m, float* v, long long n, float lr, float b1, float b2,
+                         float eps, float wd, int t, cudaStream_t st);
+cudaError_t fill_zero_launch(void* p, size_t bytes, cudaStream_t st);
+
+// ----------------------------------------------------------------- launch accounting
+// Number of kernels this library has launched (process-wide, monotonically increasing).
+extern std::atomic<long long> g_kernel_launches;
+
+}  // namespace soup

@@ -1,0 +1,1505 @@
+// libsoup host side: model state, NF4 layer stack in page-locked host memory, the
+// double-buffered layer streamer, per-layer forward/backward orchestration, the SFT and
+// DPO steps, and the extern "C" boundary declared in include/soup.h.
+//
+// Streaming (rug.gal radar "Soup ... layer streaming", "En detalle"): the base stays in host
+// RAM; each decoder layer is copied to one of n_layer_buffers device buffers on a side copy
+// stream right before it is needed, so the copy of layer i+1 overlaps the compute of layer i.
+// Fences: the compute stream waits on copy_done[b] before touching buffer b; the copy stream
+// waits on buf_free[b] (recorded after the last kernel that read buffer b) before overwriting.
+// The same kernels with the same launch configurations run in streamed and resident mode,
+// so both produce identical bits (the pages' "difference 0.0").
+#include "../../include/soup.h"
+#include "common.cuh"
+#include "internal.h"
+
+#include <chrono>
+#include <climits>
+#include <cmath>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <string>
+#include <vector>
+#include <algorithm>
+
+namespace soup {
+namespace {
+
+// ------------------------------------------------------------------ NF4 codebook
+// QLoRA's 4-bit NormalFloat levels: N(0,1) quantiles at probabilities evenly spaced from
+// 1 - delta to 1/2 (8 positive, 7 negative, plus 0), delta = (1/30 + 1/32)/2, scaled so the
+// extremes are -1 and +1.  The inverse CDF is solved in float64 by bisection then Newton on
+// Phi(x) = erfc(-x/sqrt 2)/2; the levels are rounded to float32 once.
+double phi_cdf(double x) { return 0.5 * std::erfc(-x / std::sqrt(2.0)); }
+double normal_quantile(double p) {
+  double lo = -40.0, hi = 40.0;
+  for (int i = 0; i < 200 && hi - lo > 1e-300; ++i) {
+    const double mid = 0.5 * (lo + hi);
+    if (phi_cdf(mid) < p) lo = mid; else hi = mid;
+    if (mid == lo && mid == hi) break;
+  }
+  double x = 0.5 * (lo + hi);
+  for (int i = 0; i < 4; ++i) {
+    const double f = phi_cdf(x) - p;
+    const double d = std::exp(-0.5 * x * x) / std::sqrt(2.0 * M_PI);
+    if (d <= 0) break;
+    x -= f / d;
+  }
+  return x;
+}
+void nf4_codebook_compute(float out[16]) {
+  const double delta = 0.5 * (1.0 / 30.0 + 1.0 / 32.0);
+  const double start = 1.0 - delta;
+  std::vector<double> v;
+  const double step_pos = (0.5 - start) / 8.0;  // linspace(start, 0.5, 9)[:8]
+  for (int i = 0; i < 8; ++i) v.push_back(normal_quantile(static_cast<double>(i) * step_pos + start));
+  const double step_neg = (0.5 - start) / 7.0;  // -(linspace(start, 0.5, 8)[:7])
+  for (int i = 0; i < 7; ++i) v.push_back(-normal_quantile(static_cast<double>(i) * step_neg + start));
+  v.push_back(0.0);
+  std::sort(v.begin(), v.end());
+  const double mx = v.back();
+  for (int i = 0; i < 16; ++i) out[i] = static_cast<float>(v[i] / mx);
+}
+const LUT16& codebook() {
+  static LUT16 lut = [] {
+    LUT16 l;
+    nf4_codebook_compute(l.v);
+    return l;
+  }();
+  return lut;
+}
+
+// ------------------------------------------------------------------ shapes and blob layout
+constexpr size_t ALIGN = 256;
+size_t align_up(size_t x) { return (x + ALIGN - 1) / ALIGN * ALIGN; }
+
+struct ProjShape {
+  int out, in;
+};
+void proj_shapes(const soup_model_config& c, ProjShape s[7]) {
+  const int qd = c.n_heads * c.head_dim, kvd = c.n_kv_heads * c.head_dim;
+  s[0] = {qd, c.hidden};
+  s[1] = {kvd, c.hidden};
+  s[2] = {kvd, c.hidden};
+  s[3] = {c.hidden, qd};
+  s[4] = {c.intermediate, c.hidden};
+  s[5] = {c.intermediate, c.hidden};
+  s[6] = {c.hidden, c.intermediate};
+}
+
+struct BlobLayout {
+  size_t off[9][4];
+  size_t sz[9][4];
+  size_t total;
+};
+BlobLayout blob_layout(const soup_model_config& c) {
+  BlobLayout L{};
+  ProjShape s[7];
+  proj_shapes(c, s);
+  size_t o = 0;
+  for (int p = 0; p < 7; ++p) {
+    const long long n = static_cast<long long>(s[p].out) * s[p].in;
+    const long long nb = (n + 63) / 64, ng = (nb + 255) / 256;
+    const size_t sz[4] = {static_cast<size_t>((n + 1) / 2), static_cast<size_t>(nb), static_cast<size_t>(4 * ng), 4};
+    for (int q = 0; q < 4; ++q) {
+      L.off[p][q] = o;
+      L.sz[p][q] = sz[q];
+      o += align_up(sz[q]);
+    }
+  }
+  for (int g = 0; g < 2; ++g) {
+    L.off[7 + g][0] = o;
+    L.sz[7 + g][0] = static_cast<size_t>(c.hidden) * 2;
+    o += align_up(L.sz[7 + g][0]);
+  }
+  L.total = o;
+  return L;
+}
+
+soup_status validate_cfg(const soup_model_config& c, std::string& why) {
+  if (c.n_layers < 1 || c.hidden < 8 || c.n_heads < 1 || c.n_kv_heads < 1 || c.head_dim < 1 || c.intermediate < 8 ||
+      c.vocab < 4 || c.lora_r < 1 || c.max_tokens < 1) {
+    why = "config: sizes must be positive";
+    return SOUP_ERR_INVALID_ARG;
+  }
+  if (!(c.rms_eps > 0.f) || !(c.rope_theta > 0.f) || !(c.lora_alpha == c.lora_alpha)) {
+    why = "config: rms_eps and rope_theta must be > 0";
+    return SOUP_ERR_INVALID_ARG;
+  }
+  if (c.mode != SOUP_RESIDENT && c.mode != SOUP_STREAMED) {
+    why = "config: mode must be SOUP_RESIDENT or SOUP_STREAMED";
+    return SOUP_ERR_INVALID_ARG;
+  }
+  if (c.mode == SOUP_STREAMED && c.n_layer_buffers < 2) {
+    why = "config: streamed mode needs n_layer_buffers >= 2";
+    return SOUP_ERR_INVALID_ARG;
+  }
+  if (c.n_heads % c.n_kv_heads != 0) {
+    why = "config: n_heads must be a multiple of n_kv_heads";
+    return SOUP_ERR_INVALID_ARG;
+  }
+  if (c.head_dim != 64 && c.head_dim != 128) {
+    why = "config: head_dim must be 64 or 128";
+    return SOUP_ERR_UNSUPPORTED;
+  }
+  if (c.hidden % 8 || c.intermediate % 8 || c.lora_r % 8 || c.vocab % 4) {
+    why = "config: hidden, intermediate, lora_r must be multiples of 8 and vocab of 4";
+    return SOUP_ERR_UNSUPPORTED;
+  }
+  return SOUP_OK;
+}
+
+size_t lora_numel_of(const soup_model_config& c) {
+  ProjShape s[7];
+  proj_shapes(c, s);
+  size_t per = 0;
+  for (int p = 0; p < 7; ++p) per += static_cast<size_t>(c.lora_r) * (s[p].in + s[p].out);
+  return per * c.n_layers;
+}
+// offset of A_p (which=0) or B_p (which=1) of a layer in the flat LoRA buffer
+size_t lora_off(const soup_model_config& c, int layer, int proj, int which) {
+  ProjShape s[7];
+  proj_shapes(c, s);
+  size_t per = 0;
+  for (int p = 0; p < 7; ++p) per += static_cast<size_t>(c.lora_r) * (s[p].in + s[p].out);
+  size_t o = per * layer;
+  if (which == 0) {
+    for (int p = 0; p < proj; ++p) o += static_cast<size_t>(c.lora_r) * s[p].in;
+  } else {
+    for (int p = 0; p < 7; ++p) o += static_cast<size_t>(c.lora_r) * s[p].in;
+    for (int p = 0; p < proj; ++p) o += static_cast<size_t>(c.lora_r) * s[p].out;
+  }
+  return o;
+}
+
+// ------------------------------------------------------------------ model
+struct Saved {  // per-layer activations kept for the backward
+  uint16_t *x, *n1, *qkv, *uqkv, *o, *uo, *x1, *n2, *gu, *ugu, *m, *ud;
+  float *rstd1, *rstd2, *lse;
+  int B = 0, S = 0, lora = 0, valid = 0;
+};
+
+struct LayerView {
+  NF4Seg seg[7];
+  const uint16_t* gamma[2];
+};
+
+}  // namespace
+}  // namespace soup
+
+struct soup_model {
+  soup_model_config cfg{};
+  soup_allocator alloc{};
+  bool has_alloc = false;
+  std::string err;
+  soup::BlobLayout layout{};
+  int qkv_cols = 0;
+  float s_lora = 0.f;
+
+  // host NF4 stack (page-locked)
+  std::vector<uint8_t*> host_blob;
+  std::vector<int> host_loaded;
+  // device layer buffers
+  std::vector<uint8_t*> dev_buf;   // resident: n_layers buffers; streamed: n_layer_buffers
+  std::vector<int> buf_layer;      // which layer each buffer holds (-1: none / stale)
+  std::vector<long long> buf_last; // last use tick
+  std::vector<int> buf_inuse;
+  std::vector<cudaEvent_t> copy_done, buf_free;
+  cudaStream_t copy_stream = nullptr;
+  long long tick = 0;
+
+  // head
+  const uint16_t* embed = nullptr;
+  const uint16_t* final_gamma = nullptr;
+  const uint16_t* lm_head = nullptr;
+  // LoRA storage
+  float *lora_p = nullptr, *lora_g = nullptr, *lora_m = nullptr, *lora_v = nullptr;
+  size_t lora_n = 0;
+  int lora_enabled = 1;
+  int adam_t = 0;
+
+  // activations
+  std::vector<soup::Saved> saved;
+  // work buffers
+  uint16_t *xa = nullptr, *xb = nullptr, *dqkv = nullptr, *dgu = nullptr, *dm = nullptr, *da = nullptr,
+           *dn = nullptr, *dx1 = nullptr, *vqkv = nullptr, *vo = nullptr, *vgu = nullptr, *vd = nullptr,
+           *hf = nullptr, *dh = nullptr, *dlogits = nullptr;
+  float *delta = nullptr, *logits = nullptr, *rowlse = nullptr, *rowtgt = nullptr, *roww = nullptr,
+        *rstdf = nullptr, *pi = nullptr, *ref = nullptr;
+  int32_t* ids_dev = nullptr;
+  uint8_t* mask_dev = nullptr;
+  // scalars: [0] loss (f32), [1] device error word (int)
+  int* scal = nullptr;
+  float* quant_scratch = nullptr;  // absmax scratch for the quantiser
+  float* host_scal = nullptr;      // pinned 2-word staging for the loss + error readback
+
+  std::vector<void*> dev_allocs;
+  // live profile: event pairs per launch, resolved into per-category totals
+  int prof = 0;
+  struct ProfRec {
+    int cat;
+    cudaEvent_t a, b;
+    double flops, bytes;
+  };
+  std::vector<ProfRec> prof_pending;
+  std::vector<cudaEvent_t> prof_pool;
+  struct ProfCat {
+    long long launches = 0;
+    double ms = 0, flops = 0, bytes = 0;
+  };
+  std::vector<ProfCat> prof_cats;
+  soup_stats stats{};
+  long long launches_at_reset = 0;
+};
+
+namespace soup {
+namespace {
+
+#define SOUP_CK(call)                                                                \
+  do {                                                                               \
+    cudaError_t e_ = (call);                                                         \
+    if (e_ != cudaSuccess) {                                                         \
+      m->err = std::string(#call) + ": " + cudaGetErrorString(e_);                   \
+      return SOUP_ERR_CUDA;                                                          \
+    }                                                                                \
+  } while (0)
+
+#define SOUP_TRY(st)                       \
+  do {                                     \
+    soup_status s_ = (st);                 \
+    if (s_ != SOUP_OK) return s_;          \
+  } while (0)
+
+void* dev_alloc(soup_model* m, size_t bytes) {
+  bytes = align_up(bytes ? bytes : ALIGN);
+  void* p = nullptr;
+  if (m->has_alloc) {
+    p = m->alloc.alloc(bytes, m->alloc.user);
+  } else if (cudaMalloc(&p, bytes) != cudaSuccess) {
+    p = nullptr;
+  }
+  if (p) {
+    m->dev_allocs.push_back(p);
+    m->stats.device_bytes += static_cast<long long>(bytes);
+  }
+  return p;
+}
+
+template <class T>
+soup_status alloc_into(soup_model* m, T*& out, size_t count) {
+  out = static_cast<T*>(dev_alloc(m, count * sizeof(T)));
+  if (!out) {
+    m->err = "device allocation failed";
+    return SOUP_ERR_OOM;
+  }
+  return SOUP_OK;
+}
+
+unsigned long long wait_limit_ms() {
+  const char* e = std::getenv("SOUP_WAIT_TIMEOUT_MS");
+  if (e) {
+    const long long v = std::atoll(e);
+    if (v > 0) return static_cast<unsigned long long>(v);
+  }
+  return 600000ull;
+}
+
+// Bounded host wait on all work queued on `st` so far.
+soup_status wait_stream(soup_model* m, cudaStream_t st) {
+  cudaEvent_t ev;
+  SOUP_CK(cudaEventCreateWithFlags(&ev, cudaEventDisableTiming));
+  cudaError_t e = cudaEventRecord(ev, st);
+  if (e != cudaSuccess) {
+    cudaEventDestroy(ev);
+    m->err = std::string("cudaEventRecord: ") + cudaGetErrorString(e);
+    return SOUP_ERR_CUDA;
+  }
+  const auto t0 = std::chrono::steady_clock::now();
+  const unsigned long long lim = wait_limit_ms();
+  for (;;) {
+    e = cudaEventQuery(ev);
+    if (e == cudaSuccess) break;
+    if (e != cudaErrorNotReady) {
+      cudaEventDestroy(ev);
+      m->err = std::string("stream error: ") + cudaGetErrorString(e);
+      return SOUP_ERR_CUDA;
+    }
+    const auto ms = std::chrono::duration_cast<std::chrono::milliseconds>(std::chrono::steady_clock::now() - t0).count();
+    if (static_cast<unsigned long long>(ms) > lim) {
+      cudaEventDestroy(ev);
+      m->err = "timed out waiting for the GPU";
+      return SOUP_ERR_TIMEOUT;
+    }
+    if (ms > 2) {
+      struct timespec ts = {0, 200000};
+      nanosleep(&ts, nullptr);
+    }
+  }
+  cudaEventDestroy(ev);
+  return SOUP_OK;
+}
+
+soup_status check_launch(soup_model* m, cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return SOUP_OK;
+  m->err = std::string(what) + ": " + cudaGetErrorString(e);
+  return e == cudaErrorInvalidValue ? SOUP_ERR_UNSUPPORTED : SOUP_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ live profile
+enum ProfCatId : int {
+  CAT_H2D = 0, CAT_NF4_FWD, CAT_NF4_DX, CAT_LORA, CAT_LORA_GRAD, CAT_LMHEAD_FWD, CAT_LMHEAD_DX, CAT_ATTN_FWD,
+  CAT_ATTN_BWD, CAT_RMSNORM, CAT_ROPE, CAT_SWIGLU, CAT_CE, CAT_ADAMW, CAT_EMBED, CAT_D2D, CAT_QUANT, CAT_COUNT
+};
+const char* const kCatNames[CAT_COUNT] = {
+    "h2d_layer_copy", "gemm_nf4_fwd", "gemm_nf4_dx", "gemm_lora", "gemm_lora_grad", "gemm_lm_head_fwd",
+    "gemm_lm_head_dx", "attention_fwd", "attention_bwd", "rmsnorm", "rope", "swiglu", "cross_entropy", "adamw",
+    "embed", "d2d_copy", "nf4_quantize"};
+
+cudaEvent_t prof_event(soup_model* m) {
+  if (!m->prof_pool.empty()) {
+    cudaEvent_t e = m->prof_pool.back();
+    m->prof_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+  return e;
+}
+int prof_begin(soup_model* m, cudaStream_t st) {
+  if (!m->prof) return -1;
+  soup_model::ProfRec r{};
+  r.a = prof_event(m);
+  r.b = prof_event(m);
+  if (!r.a || !r.b) return -1;
+  cudaEventRecord(r.a, st);
+  m->prof_pending.push_back(r);
+  return static_cast<int>(m->prof_pending.size()) - 1;
+}
+void prof_end(soup_model* m, cudaStream_t st, int idx, int cat, double flops, double bytes) {
+  if (idx < 0) return;
+  soup_model::ProfRec& r = m->prof_pending[idx];
+  r.cat = cat;
+  r.flops = flops;
+  r.bytes = bytes;
+  cudaEventRecord(r.b, st);
+}
+void prof_resolve(soup_model* m) {
+  if (m->prof_cats.size() != CAT_COUNT) m->prof_cats.assign(CAT_COUNT, soup_model::ProfCat{});
+  for (auto& r : m->prof_pending) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(r.b) == cudaSuccess && cudaEventElapsedTime(&ms, r.a, r.b) == cudaSuccess) {
+      auto& c = m->prof_cats[r.cat];
+      c.launches += 1;
+      c.ms += ms;
+      c.flops += r.flops;
+      c.bytes += r.bytes;
+    }
+    m->prof_pool.push_back(r.a);
+    m->prof_pool.push_back(r.b);
+  }
+  m->prof_pending.clear();
+}
+template <class F>
+soup_status launch(soup_model* m, cudaStream_t st, int cat, double flops, double bytes, const char* what, F&& f) {
+  const int idx = prof_begin(m, st);
+  const cudaError_t e = f();
+  prof_end(m, st, idx, cat, flops, bytes);
+  return check_launch(m, e, what);
+}
+
+LayerView view_of(const soup_model* m, const uint8_t* base) {
+  LayerView v{};
+  for (int p = 0; p < 7; ++p) {
+    v.seg[p].codes = base + m->layout.off[p][0];
+    v.seg[p].q8 = reinterpret_cast<const int8_t*>(base + m->layout.off[p][1]);
+    v.seg[p].scales = reinterpret_cast<const float*>(base + m->layout.off[p][2]);
+    v.seg[p].mean = reinterpret_cast<const float*>(base + m->layout.off[p][3]);
+  }
+  v.gamma[0] = reinterpret_cast<const uint16_t*>(base + m->layout.off[7][0]);
+  v.gamma[1] = reinterpret_cast<const uint16_t*>(base + m->layout.off[8][0]);
+  return v;
+}
+
+NF4Group group_of(const soup_model* m, const LayerView& v, std::initializer_list<int> projs) {
+  ProjShape s[7];
+  proj_shapes(m->cfg, s);
+  NF4Group g{};
+  int row = 0, k = 0;
+  for (int p : projs) {
+    g.seg[k] = v.seg[p];
+    g.seg[k].row_begin = row;
+    g.seg[k].rows = s[p].out;
+    g.cols = s[p].in;
+    row += s[p].out;
+    ++k;
+  }
+  g.nseg = k;
+  g.total_rows = row;
+  return g;
+}
+
+// ------------------------------------------------------------------ GEMM helpers
+Operand opnd(int kind, const void* ptr, long long ld, float scale = 1.f, int lo = 0, int hi = INT_MAX) {
+  Operand o;
+  o.kind = kind;
+  o.ptr = ptr;
+  o.ld = ld;
+  o.scale = scale;
+  o.row_lo = lo;
+  o.row_hi = hi;
+  return o;
+}
+GemmParams gemm_base(soup_model* m, int M, int N, void* out, long long ldo, int out_f32, float alpha) {
+  GemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.M = M;
+  p.N = N;
+  p.out = out;
+  p.ldo = ldo;
+  p.out_f32 = out_f32;
+  p.alpha = alpha;
+  p.err = m->scal + 1;
+  std::memcpy(p.lut, codebook().v, sizeof(p.lut));
+  return p;
+}
+void add_seg(GemmParams& p, int K, const Operand& A, const Operand& B) {
+  GemmSeg& s = p.seg[p.nseg++];
+  s.K = K;
+  s.A = A;
+  s.B = B;
+}
+double operand_bytes_per_elem(int kind) {
+  switch (kind) {
+    case OP_BF16_K:
+    case OP_BF16_MN:
+      return 2.0;
+    case OP_F32_K:
+    case OP_F32_MN:
+      return 4.0;
+    default:  // NF4: code nibble + q8 absmax per 64 + fp32 scale per 16384
+      return 0.5 + 1.0 / 64.0 + 4.0 / 16384.0;
+  }
+}
+soup_status run_gemm(soup_model* m, const GemmParams& p, cudaStream_t st, const char* what) {
+  double flops = 0, bytes = 0;
+  for (int i = 0; i < p.nseg; ++i) {
+    const GemmSeg& g = p.seg[i];
+    if (g.K <= 0) continue;
+    const int lo = std::max(0, g.B.row_lo), hi = std::min(p.N, g.B.row_hi);
+    const double rows_b = hi > lo ? hi - lo : 0;
+    flops += 2.0 * p.M * rows_b * g.K;
+    bytes += operand_bytes_per_elem(g.A.kind) * p.M * g.K + operand_bytes_per_elem(g.B.kind) * rows_b * g.K;
+  }
+  bytes += static_cast<double>(p.M) * p.N * (p.out_f32 ? 4.0 : 2.0) * (p.accumulate ? 2.0 : 1.0);
+  if (p.residual) bytes += 2.0 * p.M * p.N;
+  int cat = CAT_LORA;
+  const Operand& b0 = p.seg[0].B;
+  if (b0.kind == OP_NF4_K) cat = CAT_NF4_FWD;
+  else if (b0.kind == OP_NF4_MN) cat = CAT_NF4_DX;
+  else if (b0.ptr == m->lm_head) cat = (b0.kind == OP_BF16_K) ? CAT_LMHEAD_FWD : CAT_LMHEAD_DX;
+  else if (p.seg[0].A.kind == OP_BF16_MN) cat = CAT_LORA_GRAD;
+  return launch(m, st, cat, flops, bytes, what, [&] { return gemm_launch(p, st); });
+}
+
+// ------------------------------------------------------------------ streamer
+soup_status streamer_ensure(soup_model* m, int layer, int protect_lo, int protect_hi) {
+  if (m->cfg.mode == SOUP_RESIDENT) return SOUP_OK;
+  const int nb = static_cast<int>(m->dev_buf.size());
+  for (int b = 0; b < nb; ++b)
+    if (m->buf_layer[b] == layer) return SOUP_OK;
+  if (!m->host_loaded[layer]) {
+    m->err = "layer " + std::to_string(layer) + " has no weights loaded";
+    return SOUP_ERR_STATE;
+  }
+  int victim = -1;
+  for (int b = 0; b < nb; ++b) {
+    if (m->buf_inuse[b]) continue;
+    const int L = m->buf_layer[b];
+    if (L >= protect_lo && L <= protect_hi && L >= 0) continue;
+    if (victim < 0 || m->buf_last[b] < m->buf_last[victim]) victim = b;
+  }
+  if (victim < 0) {
+    for (int b = 0; b < nb; ++b)
+      if (!m->buf_inuse[b] && (victim < 0 || m->buf_last[b] < m->buf_last[victim])) victim = b;
+  }
+  if (victim < 0) {
+    m->err = "streamer: every layer buffer is in use";
+    return SOUP_ERR_STATE;
+  }
+  SOUP_CK(cudaStreamWaitEvent(m->copy_stream, m->buf_free[victim], 0));
+  const int pidx = prof_begin(m, m->copy_stream);
+  SOUP_CK(cudaMemcpyAsync(m->dev_buf[victim], m->host_blob[layer], m->layout.total, cudaMemcpyHostToDevice,
+                          m->copy_stream));
+  prof_end(m, m->copy_stream, pidx, CAT_H2D, 0.0, static_cast<double>(m->layout.total));
+  SOUP_CK(cudaEventRecord(m->copy_done[victim], m->copy_stream));
+  m->buf_layer[victim] = layer;
+  m->buf_last[victim] = ++m->tick;
+  m->stats.layer_loads += 1;
+  m->stats.bytes_h2d += static_cast<long long>(m->layout.total);
+  return SOUP_OK;
+}
+
+soup_status streamer_acquire(soup_model* m, int layer, cudaStream_t st, const uint8_t** base, int* buf) {
+  if (m->cfg.mode == SOUP_RESIDENT) {
+    if (!m->host_loaded[layer]) {
+      m->err = "layer " + std::to_string(layer) + " has no weights loaded";
+      return SOUP_ERR_STATE;
+    }
+    *base = m->dev_buf[layer];
+    *buf = -1;
+    return SOUP_OK;
+  }
+  const int nb = static_cast<int>(m->dev_buf.size());
+  int b = -1;
+  for (int i = 0; i < nb; ++i)
+    if (m->buf_layer[i] == layer) b = i;
+  if (b < 0) {
+    SOUP_TRY(streamer_ensure(m, layer, layer, layer));
+    for (int i = 0; i < nb; ++i)
+      if (m->buf_layer[i] == layer) b = i;
+  } else {
+    m->stats.layer_reuses += 1;
+  }
+  SOUP_CK(cudaStreamWaitEvent(st, m->copy_done[b], 0));
+  m->buf_inuse[b] = 1;
+  m->buf_last[b] = ++m->tick;
+  *base = m->dev_buf[b];
+  *buf = b;
+  return SOUP_OK;
+}
+
+soup_status streamer_release(soup_model* m, int buf, cudaStream_t st) {
+  if (buf < 0) return SOUP_OK;
+  SOUP_CK(cudaEventRecord(m->buf_free[buf], st));
+  m->buf_inuse[buf] = 0;
+  return SOUP_OK;
+}
+
+// Issue the copies of the first layers of a schedule (before compute that precedes them).
+soup_status streamer_warm(soup_model* m, int first, int count) {
+  if (m->cfg.mode == SOUP_RESIDENT) return SOUP_OK;
+  const int n = std::min(count, static_cast<int>(m->dev_buf.size()));
+  for (int k = 0; k < n && first + k < m->cfg.n_layers; ++k)
+    SOUP_TRY(streamer_ensure(m, first + k, first, first + n - 1));
+  return SOUP_OK;
+}
+
+// Prefetch the next layers of a schedule (as many as there are spare buffers).
+soup_status streamer_prefetch(soup_model* m, const std::vector<int>& order, size_t pos) {
+  if (m->cfg.mode == SOUP_RESIDENT) return SOUP_OK;
+  const size_t depth = m->dev_buf.size() - 1;
+  int lo = INT_MAX, hi = INT_MIN;
+  for (size_t k = pos; k < order.size() && k <= pos + depth; ++k) {
+    lo = std::min(lo, order[k]);
+    hi = std::max(hi, order[k]);
+  }
+  for (size_t k = pos + 1; k < order.size() && k <= pos + depth; ++k) SOUP_TRY(streamer_ensure(m, order[k], lo, hi));
+  return SOUP_OK;
+}
+
+// ------------------------------------------------------------------ layer forward / backward
+soup_status layer_forward(soup_model* m, int i, const LayerView& L, const uint16_t* x_in, uint16_t* x_out, int B,
+                          int S, cudaStream_t st) {
+  const soup_model_config& c = m->cfg;
+  const int T = B * S, h = c.hidden, r = c.lora_r, I = c.intermediate;
+  const int qd = c.n_heads * c.head_dim, kvd = c.n_kv_heads * c.head_dim, QKV = m->qkv_cols;
+  const float s = m->s_lora;
+  const bool lora = m->lora_enabled && m->lora_p;
+  Saved& A = m->saved[i];
+  A.valid = 0;
+  const double act = 2.0 * T * h;  // bytes of one [T, h] bf16 activation
+  SOUP_TRY(launch(m, st, CAT_D2D, 0, 2 * act, "save x", [&] {
+    return cudaMemcpyAsync(A.x, x_in, static_cast<size_t>(T) * h * 2, cudaMemcpyDeviceToDevice, st);
+  }));
+  SOUP_TRY(launch(m, st, CAT_RMSNORM, 0, 2 * act + 4.0 * T, "rmsnorm",
+                  [&] { return rmsnorm_fwd_launch(A.x, L.gamma[0], T, h, c.rms_eps, A.n1, A.rstd1, st); }));
+  const float* P = m->lora_p;
+  // ---- q | k | v
+  if (lora) {
+    GemmParams p = gemm_base(m, T, 3 * r, A.uqkv, 3 * r, 0, s);
+    add_seg(p, h, opnd(OP_BF16_K, A.n1, h), opnd(OP_F32_K, P + lora_off(c, i, 0, 0), h));
+    SOUP_TRY(run_gemm(m, p, st, "lora u qkv"));
+  }
+  {
+    GemmParams p = gemm_base(m, T, QKV, A.qkv, QKV, 0, 1.f);
+    p.nf4 = group_of(m, L, {0, 1, 2});
+    add_seg(p, h, opnd(OP_BF16_K, A.n1, h), opnd(OP_NF4_K, nullptr, 0));
+    if (lora) {
+      const int lo[3] = {0, qd, qd + kvd}, hi[3] = {qd, qd + kvd, QKV};
+      for (int q = 0; q < 3; ++q)
+        add_seg(p, r, opnd(OP_BF16_K, A.uqkv + q * r, 3 * r), opnd(OP_F32_K, P + lora_off(c, i, 0, 1), r, 1.f, lo[q], hi[q]));
+    }
+    SOUP_TRY(run_gemm(m, p, st, "qkv gemm"));
+  }
+  const double rope_bytes = 4.0 * T * (c.n_heads + c.n_kv_heads) * c.head_dim;
+  SOUP_TRY(launch(m, st, CAT_ROPE, 0, rope_bytes, "rope", [&] {
+    return rope_launch(A.qkv, QKV, B, S, c.n_heads, c.n_kv_heads, c.head_dim, c.rope_theta, 0, st);
+  }));
+  AttnShape as{B, S, c.n_heads, c.n_kv_heads, c.head_dim, QKV};
+  const double attn_flops = 2.0 * B * c.n_heads * c.head_dim * static_cast<double>(S) * (S + 1);
+  SOUP_TRY(launch(m, st, CAT_ATTN_FWD, attn_flops, 2.0 * T * QKV + 2.0 * T * qd + 4.0 * T * c.n_heads, "attention fwd",
+                  [&] { return attn_fwd_launch(as, A.qkv, A.o, A.lse, st); }));
+  // ---- o + residual
+  if (lora) {
+    GemmParams p = gemm_base(m, T, r, A.uo, r, 0, s);
+    add_seg(p, qd, opnd(OP_BF16_K, A.o, qd), opnd(OP_F32_K, P + lora_off(c, i, 3, 0), qd));
+    SOUP_TRY(run_gemm(m, p, st, "lora u o"));
+  }
+  {
+    GemmParams p = gemm_base(m, T, h, A.x1, h, 0, 1.f);
+    p.nf4 = group_of(m, L, {3});
+    p.residual = A.x;
+    p.ldr = h;
+    add_seg(p, qd, opnd(OP_BF16_K, A.o, qd), opnd(OP_NF4_K, nullptr, 0));
+    if (lora) add_seg(p, r, opnd(OP_BF16_K, A.uo, r), opnd(OP_F32_K, P + lora_off(c, i, 3, 1), r));
+    SOUP_TRY(run_gemm(m, p, st, "o gemm"));
+  }
+  SOUP_TRY(launch(m, st, CAT_RMSNORM, 0, 2 * act + 4.0 * T, "rmsnorm",
+                  [&] { return rmsnorm_fwd_launch(A.x1, L.gamma[1], T, h, c.rms_eps, A.n2, A.rstd2, st); }));
+  // ---- gate | up, SwiGLU
+  if (lora) {
+    GemmParams p = gemm_base(m, T, 2 * r, A.ugu, 2 * r, 0, s);
+    add_seg(p, h, opnd(OP_BF16_K, A.n2, h), opnd(OP_F32_K, P + lora_off(c, i, 4, 0), h));
+    SOUP_TRY(run_gemm(m, p, st, "lora u gate/up"));
+  }
+  {
+    GemmParams p = gemm_base(m, T, 2 * I, A.gu, 2 * I, 0, 1.f);
+    p.nf4 = group_of(m, L, {4, 5});
+    add_seg(p, h, opnd(OP_BF16_K, A.n2, h), opnd(OP_NF4_K, nullptr, 0));
+    if (lora) {
+      for (int q = 0; q < 2; ++q)
+        add_seg(p, r, opnd(OP_BF16_K, A.ugu + q * r, 2 * r),
+                opnd(OP_F32_K, P + lora_off(c, i, 4, 1), r, 1.f, q * I, (q + 1) * I));
+    }
+    SOUP_TRY(run_gemm(m, p, st, "gate/up gemm"));
+  }
+  SOUP_TRY(launch(m, st, CAT_SWIGLU, 0, 6.0 * T * I, "swiglu", [&] { return swiglu_fwd_launch(A.gu, T, I, A.m, st); }));
+  // ---- down + residual
+  if (lora) {
+    GemmParams p = gemm_base(m, T, r, A.ud, r, 0, s);
+    add_seg(p, I, opnd(OP_BF16_K, A.m, I), opnd(OP_F32_K, P + lora_off(c, i, 6, 0), I));
+    SOUP_TRY(run_gemm(m, p, st, "lora u down"));
+  }
+  {
+    GemmParams p = gemm_base(m, T, h, x_out, h, 0, 1.f);
+    p.nf4 = group_of(m, L, {6});
+    p.residual = A.x1;
+    p.ldr = h;
+    add_seg(p, I, opnd(OP_BF16_K, A.m, I), opnd(OP_NF4_K, nullptr, 0));
+    if (lora) add_seg(p, r, opnd(OP_BF16_K, A.ud, r), opnd(OP_F32_K, P + lora_off(c, i, 6, 1), r));
+    SOUP_TRY(run_gemm(m, p, st, "down gemm"));
+  }
+  A.B = B;
+  A.S = S;
+  A.lora = lora ? 1 : 0;
+  A.valid = 1;
+  return SOUP_OK;
+}
+
+// LoRA gradient GEMMs for one projection: dB += g^T u_s, dA += v_s^T x  (both fp32, accumulate)
+soup_status lora_grads(soup_model* m, int T, const uint16_t* g, long long ldg, int out, const uint16_t* us,
+                       long long ldu, float* dB, const uint16_t* x, long long ldx, int in, const uint16_t* vs,
+                       long long ldv, int nv, float* dA, cudaStream_t st, bool do_dB, bool do_dA) {
+  const int r = m->cfg.lora_r;
+  if (do_dB) {
+    GemmParams p = gemm_base(m, out, r, dB, r, 1, 1.f);
+    p.accumulate = 1;
+    add_seg(p, T, opnd(OP_BF16_MN, g, ldg), opnd(OP_BF16_MN, us, ldu));
+    SOUP_TRY(run_gemm(m, p, st, "lora dB"));
+  }
+  if (do_dA) {
+    // dA^T [in, nv] = x^T v_s, written transposed into dA [nv, in]
+    GemmParams p = gemm_base(m, in, nv, dA, in, 1, 1.f);
+    p.accumulate = 1;
+    p.out_trans = 1;
+    add_seg(p, T, opnd(OP_BF16_MN, x, ldx), opnd(OP_BF16_MN, vs, ldv));
+    SOUP_TRY(run_gemm(m, p, st, "lora dA"));
+  }
+  return SOUP_OK;
+}
+
+soup_status layer_backward(soup_model* m, int i, const LayerView& L, const uint16_t* dy, uint16_t* dx, int B, int S,
+                           cudaStream_t st) {
+  const soup_model_config& c = m->cfg;
+  Saved& A = m->saved[i];
+  if (!A.valid || A.B != B || A.S != S) {
+    m->err = "layer_bwd: no matching forward for layer " + std::to_string(i);
+    return SOUP_ERR_STATE;
+  }
+  const int T = B * S, h = c.hidden, r = c.lora_r, I = c.intermediate;
+  const int qd = c.n_heads * c.head_dim, kvd = c.n_kv_heads * c.head_dim, QKV = m->qkv_cols;
+  const float s = m->s_lora;
+  const bool lora = A.lora && m->lora_p;
+  const float* P = m->lora_p;
+  float* G = m->lora_g;
+  // ---- down
+  if (lora) {
+    GemmParams p = gemm_base(m, T, r, m->vd, r, 0, s);
+    add_seg(p, h, opnd(OP_BF16_K, dy, h), opnd(OP_F32_MN, P + lora_off(c, i, 6, 1), r));
+    SOUP_TRY(run_gemm(m, p, st, "lora v down"));
+  }
+  {
+    GemmParams p = gemm_base(m, T, I, m->dm, I, 0, 1.f);
+    p.nf4 = group_of(m, L, {6});
+    add_seg(p, h, opnd(OP_BF16_K, dy, h), opnd(OP_NF4_MN, nullptr, 0));
+    if (lora) add_seg(p, r, opnd(OP_BF16_K, m->vd, r), opnd(OP_F32_MN, P + lora_off(c, i, 6, 0), I));
+    SOUP_TRY(run_gemm(m, p, st, "down dX"));
+  }
+  if (lora)
+    SOUP_TRY(lora_grads(m, T, dy, h, h, A.ud, r, G + lora_off(c, i, 6, 1), A.m, I, I, m->vd, r, r,
+                        G + lora_off(c, i, 6, 0), st, true, true));
+  SOUP_TRY(launch(m, st, CAT_SWIGLU, 0, 10.0 * T * I, "swiglu bwd",
+                  [&] { return swiglu_bwd_launch(m->dm, A.gu, T, I, m->dgu, st); }));
+  // ---- gate | up
+  if (lora) {
+    for (int q = 0; q < 2; ++q) {
+      GemmParams p = gemm_base(m, T, r, m->vgu + q * r, 2 * r, 0, s);
+      add_seg(p, I, opnd(OP_BF16_K, m->dgu + q * I, 2 * I), opnd(OP_F32_MN, P + lora_off(c, i, 4 + q, 1), r));
+      SOUP_TRY(run_gemm(m, p, st, "lora v gate/up"));
+    }
+  }
+  {
+    GemmParams p = gemm_base(m, T, h, m->dn, h, 0, 1.f);
+    p.nf4 = group_of(m, L, {4, 5});
+    add_seg(p, 2 * I, opnd(OP_BF16_K, m->dgu, 2 * I), opnd(OP_NF4_MN, nullptr, 0));
+    if (lora)
+      for (int q = 0; q < 2; ++q)
+        add_seg(p, r, opnd(OP_BF16_K, m->vgu + q * r, 2 * r), opnd(OP_F32_MN, P + lora_off(c, i, 4 + q, 0), h));
+    SOUP_TRY(run_gemm(m, p, st, "gate/up dX"));
+  }
+  if (lora) {
+    for (int q = 0; q < 2; ++q)
+      SOUP_TRY(lora_grads(m, T, m->dgu + q * I, 2 * I, I, A.ugu + q * r, 2 * r, G + lora_off(c, i, 4 + q, 1), nullptr,
+                          0, 0, nullptr, 0, 0, nullptr, st, true, false));
+    SOUP_TRY(lora_grads(m, T, nullptr, 0, 0, nullptr, 0, nullptr, A.n2, h, h, m->vgu, 2 * r, 2 * r,
+                        G + lora_off(c, i, 4, 0), st, false, true));
+  }
+  const double act = 2.0 * T * h;
+  SOUP_TRY(launch(m, st, CAT_RMSNORM, 0, 4 * act + 4.0 * T, "rmsnorm bwd",
+                  [&] { return rmsnorm_bwd_launch(m->dn, A.x1, A.rstd2, L.gamma[1], dy, T, h, m->dx1, st); }));
+  // ---- o
+  if (lora) {
+    GemmParams p = gemm_base(m, T, r, m->vo, r, 0, s);
+    add_seg(p, h, opnd(OP_BF16_K, m->dx1, h), opnd(OP_F32_MN, P + lora_off(c, i, 3, 1), r));
+    SOUP_TRY(run_gemm(m, p, st, "lora v o"));
+  }
+  {
+    GemmParams p = gemm_base(m, T, qd, m->da, qd, 0, 1.f);
+    p.nf4 = group_of(m, L, {3});
+    add_seg(p, h, opnd(OP_BF16_K, m->dx1, h), opnd(OP_NF4_MN, nullptr, 0));
+    if (lora) add_seg(p, r, opnd(OP_BF16_K, m->vo, r), opnd(OP_F32_MN, P + lora_off(c, i, 3, 0), qd));
+    SOUP_TRY(run_gemm(m, p, st, "o dX"));
+  }
+  if (lora)
+    SOUP_TRY(lora_grads(m, T, m->dx1, h, h, A.uo, r, G + lora_off(c, i, 3, 1), A.o, qd, qd, m->vo, r, r,
+                        G + lora_off(c, i, 3, 0), st, true, true));
+  // ---- attention, RoPE
+  AttnShape as{B, S, c.n_heads, c.n_kv_heads, c.head_dim, QKV};
+  const double attn_flops = 4.0 * B * c.n_heads * c.head_dim * static_cast<double>(S) * (S + 1);
+  SOUP_TRY(launch(m, st, CAT_ATTN_BWD, attn_flops, 4.0 * T * QKV + 4.0 * T * qd + 8.0 * T * c.n_heads, "attention bwd",
+                  [&] { return attn_bwd_launch(as, A.qkv, A.o, m->da, A.lse, m->delta, m->dqkv, st); }));
+  const double rope_bytes = 4.0 * T * (c.n_heads + c.n_kv_heads) * c.head_dim;
+  SOUP_TRY(launch(m, st, CAT_ROPE, 0, rope_bytes, "rope bwd", [&] {
+    return rope_launch(m->dqkv, QKV, B, S, c.n_heads, c.n_kv_heads, c.head_dim, c.rope_theta, 1, st);
+  }));
+  // ---- q | k | v
+  const int off[3] = {0, qd, qd + kvd}, outs[3] = {qd, kvd, kvd};
+  if (lora) {
+    for (int q = 0; q < 3; ++q) {
+      GemmParams p = gemm_base(m, T, r, m->vqkv + q * r, 3 * r, 0, s);
+      add_seg(p, outs[q], opnd(OP_BF16_K, m->dqkv + off[q], QKV), opnd(OP_F32_MN, P + lora_off(c, i, q, 1), r));
+      SOUP_TRY(run_gemm(m, p, st, "lora v qkv"));
+    }
+  }
+  {
+    GemmParams p = gemm_base(m, T, h, m->dn, h, 0, 1.f);
+    p.nf4 = group_of(m, L, {0, 1, 2});
+    add_seg(p, QKV, opnd(OP_BF16_K, m->dqkv, QKV), opnd(OP_NF4_MN, nullptr, 0));
+    if (lora)
+      for (int q = 0; q < 3; ++q)
+        add_seg(p, r, opnd(OP_BF16_K, m->vqkv + q * r, 3 * r), opnd(OP_F32_MN, P + lora_off(c, i, q, 0), h));
+    SOUP_TRY(run_gemm(m, p, st, "qkv dX"));
+  }
+  if (lora) {
+    for (int q = 0; q < 3; ++q)
+      SOUP_TRY(lora_grads(m, T, m->dqkv + off[q], QKV, outs[q], A.uqkv + q * r, 3 * r, G + lora_off(c, i, q, 1),
+                          nullptr, 0, 0, nullptr, 0, 0, nullptr, st, true, false));
+    SOUP_TRY(lora_grads(m, T, nullptr, 0, 0, nullptr, 0, nullptr, A.n1, h, h, m->vqkv, 3 * r, 3 * r,
+                        G + lora_off(c, i, 0, 0), st, false, true));
+  }
+  SOUP_TRY(launch(m, st, CAT_RMSNORM, 0, 4 * act + 4.0 * T, "rmsnorm bwd",
+                  [&] { return rmsnorm_bwd_launch(m->dn, A.x, A.rstd1, L.gamma[0], m->dx1, T, h, dx, st); }));
+  return SOUP_OK;
+}
+
+// ------------------------------------------------------------------ head
+// logits = RMSNorm(x) W_lm^T (fp32), per-row LSE and target logit.
+soup_status head_forward(soup_model* m, const uint16_t* x, int B, int S, cudaStream_t st) {
+  const soup_model_config& c = m->cfg;
+  const int T = B * S, h = c.hidden, V = c.vocab;
+  SOUP_TRY(launch(m, st, CAT_RMSNORM, 0, 4.0 * T * h + 4.0 * T, "final norm",
+                  [&] { return rmsnorm_fwd_launch(x, m->final_gamma, T, h, c.rms_eps, m->hf, m->rstdf, st); }));
+  GemmParams p = gemm_base(m, T, V, m->logits, V, 1, 1.f);
+  add_seg(p, h, opnd(OP_BF16_K, m->hf, h), opnd(OP_BF16_K, m->lm_head, h));
+  SOUP_TRY(run_gemm(m, p, st, "lm_head"));
+  SOUP_TRY(launch(m, st, CAT_CE, 0, 4.0 * T * V, "ce rows", [&] {
+    return ce_rows_launch(m->logits, T, V, m->ids_dev, B, S, nullptr, 0, m->rowlse, m->rowtgt, m->scal + 1, st);
+  }));
+  return SOUP_OK;
+}
+// dlogits = w_t (softmax - onehot) -> dh = dlogits W_lm -> final-norm backward into dx.
+soup_status head_backward(soup_model* m, const uint16_t* x, int B, int S, uint16_t* dx, cudaStream_t st) {
+  const soup_model_config& c = m->cfg;
+  const int T = B * S, h = c.hidden, V = c.vocab;
+  SOUP_TRY(launch(m, st, CAT_CE, 0, 6.0 * T * V, "ce grad",
+                  [&] { return ce_grad_launch(m->logits, m->rowlse, m->ids_dev, m->roww, B, S, V, m->dlogits, st); }));
+  GemmParams p = gemm_base(m, T, h, m->dh, h, 0, 1.f);
+  add_seg(p, V, opnd(OP_BF16_K, m->dlogits, V), opnd(OP_BF16_MN, m->lm_head, h));
+  SOUP_TRY(run_gemm(m, p, st, "lm_head dX"));
+  SOUP_TRY(launch(m, st, CAT_RMSNORM, 0, 6.0 * T * h + 4.0 * T, "final norm bwd",
+                  [&] { return rmsnorm_bwd_launch(m->dh, x, m->rstdf, m->final_gamma, nullptr, T, h, dx, st); }));
+  return SOUP_OK;
+}
+
+soup_status stream_forward_pass(soup_model* m, int B, int S, cudaStream_t st, uint16_t** x_final) {
+  const int L = m->cfg.n_layers;
+  std::vector<int> order(L);
+  for (int i = 0; i < L; ++i) order[i] = i;
+  uint16_t* cur = m->xa;
+  uint16_t* nxt = m->xb;
+  for (int i = 0; i < L; ++i) {
+    const uint8_t* base;
+    int buf;
+    SOUP_TRY(streamer_acquire(m, i, st, &base, &buf));
+    SOUP_TRY(streamer_prefetch(m, order, i));
+    const LayerView v = view_of(m, base);
+    SOUP_TRY(layer_forward(m, i, v, cur, nxt, B, S, st));
+    SOUP_TRY(streamer_release(m, buf, st));
+    std::swap(cur, nxt);
+  }
+  *x_final = cur;
+  return SOUP_OK;
+}
+
+soup_status stream_backward_pass(soup_model* m, int B, int S, uint16_t* dcur, uint16_t* dnxt, cudaStream_t st) {
+  const int L = m->cfg.n_layers;
+  std::vector<int> order(L);
+  for (int i = 0; i < L; ++i) order[i] = L - 1 - i;
+  for (int k = 0; k < L; ++k) {
+    const int i = order[k];
+    const uint8_t* base;
+    int buf;
+    SOUP_TRY(streamer_acquire(m, i, st, &base, &buf));
+    SOUP_TRY(streamer_prefetch(m, order, k));
+    const LayerView v = view_of(m, base);
+    SOUP_TRY(layer_backward(m, i, v, dcur, dnxt, B, S, st));
+    SOUP_TRY(streamer_release(m, buf, st));
+    std::swap(dcur, dnxt);
+  }
+  return SOUP_OK;
+}
+
+soup_status read_scalars(soup_model* m, cudaStream_t st, float* loss_out) {
+  SOUP_CK(cudaMemcpyAsync(m->host_scal, m->scal, 8, cudaMemcpyDeviceToHost, st));
+  SOUP_TRY(wait_stream(m, st));
+  int errw;
+  std::memcpy(&errw, m->host_scal + 1, 4);
+  if (errw != 0) {
+    SOUP_CK(cudaMemsetAsync(m->scal + 1, 0, 4, st));
+    m->err = errw == DEVERR_TIMEOUT ? "a kernel's bounded wait timed out" : "a kernel bounds check fired";
+    return errw == DEVERR_TIMEOUT ? SOUP_ERR_TIMEOUT : SOUP_ERR_DEVICE_CHECK;
+  }
+  if (loss_out) *loss_out = m->host_scal[0];
+  return SOUP_OK;
+}
+
+soup_status do_step(soup_model* m, soup_loss kind, const soup_batch* bt, float* loss_out, cudaStream_t st) {
+  const soup_model_config& c = m->cfg;
+  if (!m->embed || !m->lm_head || !m->final_gamma) {
+    m->err = "head weights not set";
+    return SOUP_ERR_STATE;
+  }
+  if (!m->lora_p) {
+    m->err = "LoRA storage not set";
+    return SOUP_ERR_STATE;
+  }
+  const int B = bt->B, S = bt->S, T = B * S;
+  if (B < 1 || S < 2 || T > c.max_tokens || !bt->ids) {
+    m->err = "batch: need B >= 1, S >= 2, B*S <= max_tokens and ids";
+    return SOUP_ERR_INVALID_ARG;
+  }
+  if (kind == SOUP_LOSS_DPO && (bt->n_pairs < 1 || 2 * bt->n_pairs != B || bt->prefix_len < 0 || bt->prefix_len >= S)) {
+    m->err = "DPO batch: B must be 2*n_pairs and 0 <= prefix_len < S";
+    return SOUP_ERR_INVALID_ARG;
+  }
+  for (int i = 0; i < c.n_layers; ++i)
+    if (!m->host_loaded[i]) {
+      m->err = "layer " + std::to_string(i) + " has no weights loaded";
+      return SOUP_ERR_STATE;
+    }
+  const long long launches0 = g_kernel_launches.load();
+  // inputs
+  SOUP_CK(cudaMemcpyAsync(m->ids_dev, bt->ids, static_cast<size_t>(T) * 4,
+                          bt->ids_on_host ? cudaMemcpyHostToDevice : cudaMemcpyDeviceToDevice, st));
+  const uint8_t* mask = nullptr;
+  if (bt->loss_mask) {
+    SOUP_CK(cudaMemcpyAsync(m->mask_dev, bt->loss_mask, static_cast<size_t>(T),
+                            bt->ids_on_host ? cudaMemcpyHostToDevice : cudaMemcpyDeviceToDevice, st));
+    mask = m->mask_dev;
+  }
+  SOUP_CK(cudaMemsetAsync(m->lora_g, 0, m->lora_n * sizeof(float), st));
+  const int saved_enabled = m->lora_enabled;
+  uint16_t* xL = nullptr;
+  if (kind == SOUP_LOSS_DPO) {
+    // reference: same streamed base, LoRA off
+    m->lora_enabled = 0;
+    SOUP_TRY(streamer_warm(m, 0, 2));
+    SOUP_TRY(launch(m, st, CAT_EMBED, 0, 4.0 * T * c.hidden, "embed", [&] {
+    return embed_launch(m->ids_dev, m->embed, T, c.hidden, c.vocab, m->xa, m->scal + 1, st);
+  }));
+    soup_status s1 = stream_forward_pass(m, B, S, st, &xL);
+    if (s1 != SOUP_OK) {
+      m->lora_enabled = saved_enabled;
+      return s1;
+    }
+    SOUP_TRY(head_forward(m, xL, B, S, st));
+    SOUP_TRY(check_launch(m, seq_logp_launch(m->rowlse, m->rowtgt, B, S, bt->prefix_len, m->ref, st), "ref logp"));
+    m->lora_enabled = 1;
+  }
+  SOUP_TRY(streamer_warm(m, 0, 2));
+  SOUP_TRY(launch(m, st, CAT_EMBED, 0, 4.0 * T * c.hidden, "embed", [&] {
+    return embed_launch(m->ids_dev, m->embed, T, c.hidden, c.vocab, m->xa, m->scal + 1, st);
+  }));
+  soup_status s2 = stream_forward_pass(m, B, S, st, &xL);
+  m->lora_enabled = saved_enabled;
+  if (s2 != SOUP_OK) return s2;
+  SOUP_TRY(head_forward(m, xL, B, S, st));
+  float* loss_dev = reinterpret_cast<float*>(m->scal);
+  if (kind == SOUP_LOSS_SFT) {
+    SOUP_TRY(check_launch(m, sft_finish_launch(m->rowlse, m->rowtgt, m->ids_dev, B, S, mask, loss_dev, m->roww, st),
+                          "sft loss"));
+  } else {
+    SOUP_TRY(check_launch(m, dpo_finish_launch(m->rowlse, m->rowtgt, B, S, bt->prefix_len, bt->n_pairs, bt->beta,
+                                               m->ref, m->pi, loss_dev, m->roww, st),
+                          "dpo loss"));
+  }
+  uint16_t* other = (xL == m->xa) ? m->xb : m->xa;
+  SOUP_TRY(head_backward(m, xL, B, S, other, st));
+  // backward ping-pongs between `other` and the buffer that held x_L (no longer needed)
+  SOUP_TRY(stream_backward_pass(m, B, S, other, xL, st));
+  if (bt->apply_optimizer) {
+    m->adam_t += 1;
+    SOUP_TRY(launch(m, st, CAT_ADAMW, 0, 28.0 * m->lora_n, "adamw", [&] {
+      return adamw_launch(m->lora_p, m->lora_g, m->lora_m, m->lora_v, static_cast<long long>(m->lora_n), bt->lr, 0.9f,
+                          0.999f, 1e-8f, 0.f, m->adam_t, st);
+    }));
+  }
+  m->stats.kernel_launches += g_kernel_launches.load() - launches0;
+  SOUP_TRY(read_scalars(m, st, loss_out));
+  m->stats.steps += 1;
+  return SOUP_OK;
+}
+
+soup_status destroy_model(soup_model* m) {
+  if (m->copy_stream) cudaStreamSynchronize(m->copy_stream);
+  cudaDeviceSynchronize();
+  for (void* p : m->dev_allocs) {
+    if (m->has_alloc)
+      m->alloc.free(p, m->alloc.user);
+    else
+      cudaFree(p);
+  }
+  for (uint8_t* h : m->host_blob)
+    if (h) cudaFreeHost(h);
+  if (m->host_scal) cudaFreeHost(m->host_scal);
+  for (auto& r : m->prof_pending) {
+    cudaEventDestroy(r.a);
+    cudaEventDestroy(r.b);
+  }
+  for (auto e : m->prof_pool) cudaEventDestroy(e);
+  for (auto e : m->copy_done) cudaEventDestroy(e);
+  for (auto e : m->buf_free) cudaEventDestroy(e);
+  if (m->copy_stream) cudaStreamDestroy(m->copy_stream);
+  delete m;
+  return SOUP_OK;
+}
+
+soup_status create_model(const soup_model_config* cfg, const soup_allocator* alloc, soup_model** out) {
+  soup_model* m = new soup_model();
+  m->cfg = *cfg;
+  std::string why;
+  soup_status vs = validate_cfg(*cfg, why);
+  if (vs != SOUP_OK) {
+    delete m;
+    return vs;
+  }
+  if (alloc && alloc->alloc && alloc->free) {
+    m->alloc = *alloc;
+    m->has_alloc = true;
+  }
+  auto fail = [&](soup_status s) {
+    destroy_model(m);
+    return s;
+  };
+  if (cudaSetDevice(cfg->device) != cudaSuccess) return fail(SOUP_ERR_CUDA);
+  const soup_model_config& c = m->cfg;
+  m->layout = blob_layout(c);
+  m->qkv_cols = (c.n_heads + 2 * c.n_kv_heads) * c.head_dim;
+  m->s_lora = c.lora_alpha / static_cast<float>(c.lora_r);
+  (void)codebook();
+  const int L = c.n_layers;
+  m->host_blob.assign(L, nullptr);
+  m->host_loaded.assign(L, 0);
+  for (int i = 0; i < L; ++i) {
+    if (cudaHostAlloc(reinterpret_cast<void**>(&m->host_blob[i]), m->layout.total, cudaHostAllocDefault) != cudaSuccess)
+      return fail(SOUP_ERR_OOM);
+    m->stats.pinned_bytes += static_cast<long long>(m->layout.total);
+  }
+  if (cudaHostAlloc(reinterpret_cast<void**>(&m->host_scal), 64, cudaHostAllocDefault) != cudaSuccess)
+    return fail(SOUP_ERR_OOM);
+  const int nbuf = (c.mode == SOUP_RESIDENT) ? L : c.n_layer_buffers;
+  for (int b = 0; b < nbuf; ++b) {
+    uint8_t* p = static_cast<uint8_t*>(dev_alloc(m, m->layout.total));
+    if (!p) return fail(SOUP_ERR_OOM);
+    m->dev_buf.push_back(p);
+  }
+  m->buf_layer.assign(nbuf, -1);
+  m->buf_last.assign(nbuf, 0);
+  m->buf_inuse.assign(nbuf, 0);
+  if (cudaStreamCreateWithFlags(&m->copy_stream, cudaStreamNonBlocking) != cudaSuccess) return fail(SOUP_ERR_CUDA);
+  m->copy_done.resize(nbuf);
+  m->buf_free.resize(nbuf);
+  for (int b = 0; b < nbuf; ++b) {
+    if (cudaEventCreateWithFlags(&m->copy_done[b], cudaEventDisableTiming) != cudaSuccess) return fail(SOUP_ERR_CUDA);
+    if (cudaEventCreateWithFlags(&m->buf_free[b], cudaEventDisableTiming) != cudaSuccess) return fail(SOUP_ERR_CUDA);
+  }
+  // activations
+  const size_t T = static_cast<size_t>(c.max_tokens), h = c.hidden, r = c.lora_r, I = c.intermediate;
+  const size_t qd = static_cast<size_t>(c.n_heads) * c.head_dim, QKV = m->qkv_cols;
+  m->saved.resize(L);
+  for (int i = 0; i < L; ++i) {
+    Saved& A = m->saved[i];
+    if (alloc_into(m, A.x, T * h) || alloc_into(m, A.n1, T * h) || alloc_into(m, A.qkv, T * QKV) ||
+        alloc_into(m, A.uqkv, T * 3 * r) || alloc_into(m, A.o, T * qd) || alloc_into(m, A.uo, T * r) ||
+        alloc_into(m, A.x1, T * h) || alloc_into(m, A.n2, T * h) || alloc_into(m, A.gu, T * 2 * I) ||
+        alloc_into(m, A.ugu, T * 2 * r) || alloc_into(m, A.m, T * I) || alloc_into(m, A.ud, T * r) ||
+        alloc_into(m, A.rstd1, T) || alloc_into(m, A.rstd2, T) || alloc_into(m, A.lse, T * c.n_heads))
+      return fail(SOUP_ERR_OOM);
+  }
+  const size_t V = c.vocab;
+  if (alloc_into(m, m->xa, T * h) || alloc_into(m, m->xb, T * h) || alloc_into(m, m->dqkv, T * QKV) ||
+      alloc_into(m, m->dgu, T * 2 * I) || alloc_into(m, m->dm, T * I) || alloc_into(m, m->da, T * qd) ||
+      alloc_into(m, m->dn, T * h) || alloc_into(m, m->dx1, T * h) || alloc_into(m, m->vqkv, T * 3 * r) ||
+      alloc_into(m, m->vo, T * r) || alloc_into(m, m->vgu, T * 2 * r) || alloc_into(m, m->vd, T * r) ||
+      alloc_into(m, m->hf, T * h) || alloc_into(m, m->dh, T * h) || alloc_into(m, m->dlogits, T * V) ||
+      alloc_into(m, m->delta, T * c.n_heads) || alloc_into(m, m->logits, T * V) || alloc_into(m, m->rowlse, T) ||
+      alloc_into(m, m->rowtgt, T) || alloc_into(m, m->roww, T) || alloc_into(m, m->rstdf, T) ||
+      alloc_into(m, m->pi, T) || alloc_into(m, m->ref, T) || alloc_into(m, m->ids_dev, T) ||
+      alloc_into(m, m->mask_dev, T) || alloc_into(m, m->scal, 64))
+    return fail(SOUP_ERR_OOM);
+  if (cudaMemset(m->scal, 0, 64 * sizeof(int)) != cudaSuccess) return fail(SOUP_ERR_CUDA);
+  m->lora_n = lora_numel_of(c);
+  *out = m;
+  return SOUP_OK;
+}
+
+soup_status quantize_layer(soup_model* m, int layer, const float* const w[7], const uint16_t* ga, const uint16_t* gm,
+                           cudaStream_t st) {
+  const soup_model_config& c = m->cfg;
+  ProjShape s[7];
+  proj_shapes(c, s);
+  if (!m->quant_scratch) {
+    long long mx = 0;
+    for (int p = 0; p < 7; ++p) mx = std::max(mx, (static_cast<long long>(s[p].out) * s[p].in + 63) / 64);
+    if (alloc_into(m, m->quant_scratch, static_cast<size_t>(mx))) return SOUP_ERR_OOM;
+  }
+  // quantise into a device buffer (the layer's resident buffer, or a streamer buffer that is
+  // then marked stale), then copy the blob to page-locked host memory
+  uint8_t* dst;
+  int stale_buf = -1;
+  if (c.mode == SOUP_RESIDENT) {
+    dst = m->dev_buf[layer];
+  } else {
+    int b = -1;
+    for (int i = 0; i < static_cast<int>(m->dev_buf.size()); ++i)
+      if (!m->buf_inuse[i] && (b < 0 || m->buf_last[i] < m->buf_last[b])) b = i;
+    if (b < 0) {
+      m->err = "no free layer buffer to quantise into";
+      return SOUP_ERR_STATE;
+    }
+    SOUP_CK(cudaStreamWaitEvent(st, m->buf_free[b], 0));
+    SOUP_CK(cudaStreamWaitEvent(st, m->copy_done[b], 0));
+    dst = m->dev_buf[b];
+    stale_buf = b;
+  }
+  for (int p = 0; p < 7; ++p) {
+    const long long n = static_cast<long long>(s[p].out) * s[p].in;
+    SOUP_TRY(check_launch(m,
+                          nf4_quantize_launch(w[p], n, dst + m->layout.off[p][0],
+                                              reinterpret_cast<int8_t*>(dst + m->layout.off[p][1]),
+                                              reinterpret_cast<float*>(dst + m->layout.off[p][2]),
+                                              reinterpret_cast<float*>(dst + m->layout.off[p][3]), m->quant_scratch,
+                                              codebook(), st),
+                          "nf4 quantize"));
+  }
+  SOUP_CK(cudaMemcpyAsync(dst + m->layout.off[7][0], ga, static_cast<size_t>(c.hidden) * 2, cudaMemcpyDeviceToDevice, st));
+  SOUP_CK(cudaMemcpyAsync(dst + m->layout.off[8][0], gm, static_cast<size_t>(c.hidden) * 2, cudaMemcpyDeviceToDevice, st));
+  SOUP_CK(cudaMemcpyAsync(m->host_blob[layer], dst, m->layout.total, cudaMemcpyDeviceToHost, st));
+  SOUP_TRY(wait_stream(m, st));
+  if (stale_buf >= 0) {
+    m->buf_layer[stale_buf] = -1;
+    SOUP_CK(cudaEventRecord(m->buf_free[stale_buf], st));
+  }
+  // any streamer buffer holding an older copy of this layer is now stale
+  if (c.mode == SOUP_STREAMED)
+    for (size_t b = 0; b < m->buf_layer.size(); ++b)
+      if (m->buf_layer[b] == layer) m->buf_layer[b] = -1;
+  m->host_loaded[layer] = 1;
+  return SOUP_OK;
+}
+
+}  // namespace
+}  // namespace soup
+
+// ====================================================================== C-ABI
+using namespace soup;
+
+#define SOUP_GUARD(body)                                          \
+  try {                                                           \
+    body                                                          \
+  } catch (const std::exception& ex) {                            \
+    if (m) m->err = ex.what();                                    \
+    return SOUP_ERR_INVALID_ARG;                                  \
+  } catch (...) {                                                 \
+    return SOUP_ERR_INVALID_ARG;                                  \
+  }
+
+extern "C" {
+
+const char* soup_status_string(soup_status s) {
+  switch (s) {
+    case SOUP_OK: return "ok";
+    case SOUP_ERR_INVALID_ARG: return "invalid argument";
+    case SOUP_ERR_STATE: return "invalid call order or state";
+    case SOUP_ERR_OOM: return "out of memory";
+    case SOUP_ERR_CUDA: return "CUDA error";
+    case SOUP_ERR_TIMEOUT: return "timed out";
+    case SOUP_ERR_DEVICE_CHECK: return "device bounds check fired";
+    case SOUP_ERR_UNSUPPORTED: return "unsupported shape";
+    default: return "unknown status";
+  }
+}
+
+const char* soup_last_error(const soup_model* m) { return m ? m->err.c_str() : ""; }
+
+soup_status soup_layer_blob_bytes(const soup_model_config* cfg, size_t* bytes) {
+  if (!cfg || !bytes) return SOUP_ERR_INVALID_ARG;
+  std::string why;
+  soup_status s = validate_cfg(*cfg, why);
+  if (s != SOUP_OK) return s;
+  *bytes = blob_layout(*cfg).total;
+  return SOUP_OK;
+}
+
+soup_status soup_layer_blob_part(const soup_model_config* cfg, int proj, int part, size_t* offset, size_t* bytes) {
+  if (!cfg || !offset || !bytes || proj < 0 || proj > 8 || part < 0 || part > 3) return SOUP_ERR_INVALID_ARG;
+  if (proj >= 7 && part != 0) return SOUP_ERR_INVALID_ARG;
+  std::string why;
+  soup_status s = validate_cfg(*cfg, why);
+  if (s != SOUP_OK) return s;
+  const BlobLayout L = blob_layout(*cfg);
+  *offset = L.off[proj][part];
+  *bytes = L.sz[proj][part];
+  return SOUP_OK;
+}
+
+soup_status soup_lora_numel(const soup_model_config* cfg, size_t* numel) {
+  if (!cfg || !numel) return SOUP_ERR_INVALID_ARG;
+  std::string why;
+  soup_status s = validate_cfg(*cfg, why);
+  if (s != SOUP_OK) return s;
+  *numel = lora_numel_of(*cfg);
+  return SOUP_OK;
+}
+
+soup_status soup_lora_offset(const soup_model_config* cfg, int layer, int proj, int which_b, size_t* offset, int* rows,
+                             int* cols) {
+  if (!cfg || !offset || layer < 0 || layer >= cfg->n_layers || proj < 0 || proj >= 7 || which_b < 0 || which_b > 1)
+    return SOUP_ERR_INVALID_ARG;
+  std::string why;
+  soup_status s = validate_cfg(*cfg, why);
+  if (s != SOUP_OK) return s;
+  ProjShape sh[7];
+  proj_shapes(*cfg, sh);
+  *offset = lora_off(*cfg, layer, proj, which_b);
+  if (rows) *rows = which_b ? sh[proj].out : cfg->lora_r;
+  if (cols) *cols = which_b ? cfg->lora_r : sh[proj].in;
+  return SOUP_OK;
+}
+
+soup_status soup_model_create(const soup_model_config* cfg, const soup_allocator* alloc, soup_model** out) {
+  soup_model* m = nullptr;
+  if (!cfg || !out) return SOUP_ERR_INVALID_ARG;
+  SOUP_GUARD(return create_model(cfg, alloc, out);)
+}
+
+soup_status soup_model_destroy(soup_model* m) {
+  if (!m) return SOUP_ERR_INVALID_ARG;
+  SOUP_GUARD(return destroy_model(m);)
+}
+
+soup_status soup_model_quantize_layer(soup_model* m, int layer, const float* const w[7], const uint16_t* gamma_attn,
+                                      const uint16_t* gamma_mlp, void* stream) {
+  if (!m || !w || !gamma_attn || !gamma_mlp || layer < 0 || layer >= m->cfg.n_layers) return SOUP_ERR_INVALID_ARG;
+  for (int p = 0; p < 7; ++p)
+    if (!w[p]) return SOUP_ERR_INVALID_ARG;
+  SOUP_GUARD(return quantize_layer(m, layer, w, gamma_attn, gamma_mlp, static_cast<cudaStream_t>(stream));)
+}
+
+soup_status soup_model_load_layer_nf4(soup_model* m, int layer, const void* blob, size_t bytes) {
+  if (!m || !blob || layer < 0 || layer >= m->cfg.n_layers) return SOUP_ERR_INVALID_ARG;
+  if (bytes != m->layout.total) {
+    m->err = "blob size mismatch";
+    return SOUP_ERR_INVALID_ARG;
+  }
+  SOUP_GUARD({
+    std::memcpy(m->host_blob[layer], blob, bytes);
+    if (m->cfg.mode == SOUP_RESIDENT) {
+      SOUP_CK(cudaMemcpy(m->dev_buf[layer], m->host_blob[layer], bytes, cudaMemcpyHostToDevice));
+    } else {
+      for (size_t b = 0; b < m->buf_layer.size(); ++b)
+        if (m->buf_layer[b] == layer) m->buf_layer[b] = -1;
+    }
+    m->host_loaded[layer] = 1;
+    return SOUP_OK;
+  })
+}
+
+soup_status soup_model_read_layer_nf4(soup_model* m, int layer, void* blob, size_t bytes) {
+  if (!m || !blob || layer < 0 || layer >= m->cfg.n_layers || bytes != m->layout.total) return SOUP_ERR_INVALID_ARG;
+  if (!m->host_loaded[layer]) return SOUP_ERR_STATE;
+  std::memcpy(blob, m->host_blob[layer], bytes);
+  return SOUP_OK;
+}
+
+soup_status soup_model_set_head(soup_model* m, const void* embed, const void* final_gamma, const void* lm_head) {
+  if (!m || !embed || !final_gamma || !lm_head) return SOUP_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(embed) | reinterpret_cast<uintptr_t>(lm_head) |
+       reinterpret_cast<uintptr_t>(final_gamma)) & 15u) {
+    m->err = "head weights must be 16-byte aligned";
+    return SOUP_ERR_INVALID_ARG;
+  }
+  m->embed = static_cast<const uint16_t*>(embed);
+  m->final_gamma = static_cast<const uint16_t*>(final_gamma);
+  m->lm_head = static_cast<const uint16_t*>(lm_head);
+  return SOUP_OK;
+}
+
+soup_status soup_model_set_lora(soup_model* m, float* params, float* grads, float* adam_m, float* adam_v) {
+  if (!m || !params || !grads || !adam_m || !adam_v) return SOUP_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(params) | reinterpret_cast<uintptr_t>(grads) | reinterpret_cast<uintptr_t>(adam_m) |
+       reinterpret_cast<uintptr_t>(adam_v)) & 15u) {
+    m->err = "LoRA buffers must be 16-byte aligned";
+    return SOUP_ERR_INVALID_ARG;
+  }
+  m->lora_p = params;
+  m->lora_g = grads;
+  m->lora_m = adam_m;
+  m->lora_v = adam_v;
+  m->adam_t = 0;
+  for (auto& a : m->saved) a.valid = 0;
+  return SOUP_OK;
+}
+
+soup_status soup_set_lora_enabled(soup_model* m, int enabled) {
+  if (!m) return SOUP_ERR_INVALID_ARG;
+  m->lora_enabled = enabled ? 1 : 0;
+  return SOUP_OK;
+}
+
+soup_status soup_layer_fwd(soup_model* m, int layer, const void* x_in, void* x_out, int B, int S, void* stream) {
+  if (!m || !x_in || !x_out || layer < 0 || layer >= m->cfg.n_layers || B < 1 || S < 1 ||
+      static_cast<long long>(B) * S > m->cfg.max_tokens)
+    return SOUP_ERR_INVALID_ARG;
+  SOUP_GUARD({
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const long long l0 = g_kernel_launches.load();
+    const uint8_t* base;
+    int buf;
+    SOUP_TRY(streamer_acquire(m, layer, st, &base, &buf));
+    soup_status s = layer_forward(m, layer, view_of(m, base), static_cast<const uint16_t*>(x_in),
+                                  static_cast<uint16_t*>(x_out), B, S, st);
+    soup_status s2 = streamer_release(m, buf, st);
+    m->stats.kernel_launches += g_kernel_launches.load() - l0;
+    return s != SOUP_OK ? s : s2;
+  })
+}
+
+soup_status soup_layer_bwd(soup_model* m, int layer, const void* dy, void* dx, int B, int S, void* stream) {
+  if (!m || !dy || !dx || layer < 0 || layer >= m->cfg.n_layers || B < 1 || S < 1) return SOUP_ERR_INVALID_ARG;
+  SOUP_GUARD({
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (!m->saved[layer].valid) {
+      m->err = "layer_bwd before layer_fwd";
+      return SOUP_ERR_STATE;
+    }
+    if (m->saved[layer].lora && !m->lora_g) return SOUP_ERR_STATE;
+    const long long l0 = g_kernel_launches.load();
+    const uint8_t* base;
+    int buf;
+    SOUP_TRY(streamer_acquire(m, layer, st, &base, &buf));
+    soup_status s = layer_backward(m, layer, view_of(m, base), static_cast<const uint16_t*>(dy),
+                                   static_cast<uint16_t*>(dx), B, S, st);
+    soup_status s2 = streamer_release(m, buf, st);
+    m->stats.kernel_launches += g_kernel_launches.load() - l0;
+    return s != SOUP_OK ? s : s2;
+  })
+}
+
+soup_status soup_step(soup_model* m, soup_loss loss, const soup_batch* batch, float* loss_out, void* stream) {
+  if (!m || !batch || (loss != SOUP_LOSS_SFT && loss != SOUP_LOSS_DPO)) return SOUP_ERR_INVALID_ARG;
+  SOUP_GUARD(return do_step(m, loss, batch, loss_out, static_cast<cudaStream_t>(stream));)
+}
+
+soup_status soup_optimizer_step(soup_model* m, float lr, void* stream) {
+  if (!m) return SOUP_ERR_INVALID_ARG;
+  if (!m->lora_p) return SOUP_ERR_STATE;
+  SOUP_GUARD({
+    m->adam_t += 1;
+    const long long l0 = g_kernel_launches.load();
+    soup_status s = check_launch(m, adamw_launch(m->lora_p, m->lora_g, m->lora_m, m->lora_v,
+                                                 static_cast<long long>(m->lora_n), lr, 0.9f, 0.999f, 1e-8f, 0.f,
+                                                 m->adam_t, static_cast<cudaStream_t>(stream)),
+                                 "adamw");
+    m->stats.kernel_launches += g_kernel_launches.load() - l0;
+    return s;
+  })
+}
+
+soup_status soup_last_logps(soup_model* m, float* pi, float* ref, int n) {
+  if (!m || !pi || !ref || n < 1 || n > m->cfg.max_tokens) return SOUP_ERR_INVALID_ARG;
+  SOUP_GUARD({
+    SOUP_CK(cudaMemcpy(pi, m->pi, static_cast<size_t>(n) * 4, cudaMemcpyDeviceToHost));
+    SOUP_CK(cudaMemcpy(ref, m->ref, static_cast<size_t>(n) * 4, cudaMemcpyDeviceToHost));
+    return SOUP_OK;
+  })
+}
+
+soup_status soup_nf4_quantize(const float* w, long long n, uint8_t* codes, int8_t* q8, float* scales, float* mean,
+                              float* scratch, void* stream) {
+  if (!w || n <= 0 || !codes || !q8 || !scales || !mean || !scratch) return SOUP_ERR_INVALID_ARG;
+  cudaError_t e = nf4_quantize_launch(w, n, codes, q8, scales, mean, scratch, codebook(), static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SOUP_OK : SOUP_ERR_CUDA;
+}
+
+soup_status soup_nf4_dequantize(const uint8_t* codes, const int8_t* q8, const float* scales, const float* mean,
+                                long long n, uint16_t* out, void* stream) {
+  if (!codes || !q8 || !scales || !mean || !out || n < 0) return SOUP_ERR_INVALID_ARG;
+  cudaError_t e = nf4_dequant_launch(codes, q8, scales, mean, n, out, codebook(), static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SOUP_OK : SOUP_ERR_CUDA;
+}
+
+soup_status soup_nf4_matmul(const void* x, int M, int N, int K, const uint8_t* codes, const int8_t* q8,
+                            const float* scales, const float* mean, int transpose_w, const void* residual, void* y,
+                            void* stream) {
+  if (!x || !codes || !q8 || !scales || !mean || !y || M < 0 || N <= 0 || K <= 0) return SOUP_ERR_INVALID_ARG;
+  if (N % 8 || K % 8) return SOUP_ERR_UNSUPPORTED;
+  GemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  NF4Group g{};
+  g.nseg = 1;
+  g.seg[0] = NF4Seg{codes, q8, scales, mean, 0, N};
+  g.cols = K;
+  g.total_rows = N;
+  p.nf4 = g;
+  std::memcpy(p.lut, codebook().v, sizeof(p.lut));
+  p.alpha = 1.f;
+  p.out = y;
+  p.nseg = 1;
+  if (!transpose_w) {  // y[M,N] = x[M,K] W^T
+    p.M = M;
+    p.N = N;
+    p.ldo = N;
+    p.seg[0].K = K;
+    p.seg[0].A = Operand{OP_BF16_K, x, K, 1.f, 0, INT_MAX};
+    p.seg[0].B = Operand{OP_NF4_K, nullptr, 0, 1.f, 0, INT_MAX};
+    if (residual) {
+      p.residual = residual;
+      p.ldr = N;
+    }
+  } else {  // y[M,K] = x[M,N] W
+    p.M = M;
+    p.N = K;
+    p.ldo = K;
+    p.seg[0].K = N;
+    p.seg[0].A = Operand{OP_BF16_K, x, N, 1.f, 0, INT_MAX};
+    p.seg[0].B = Operand{OP_NF4_MN, nullptr, 0, 1.f, 0, INT_MAX};
+    if (residual) {
+      p.residual = residual;
+      p.ldr = K;
+    }
+  }
+  cudaError_t e = gemm_launch(p, static_cast<cudaStream_t>(stream));
+  if (e == cudaErrorInvalidValue) return SOUP_ERR_UNSUPPORTED;
+  return e == cudaSuccess ? SOUP_OK : SOUP_ERR_CUDA;
+}
+
+soup_status soup_nf4_codebook(float* out16) {
+  if (!out16) return SOUP_ERR_INVALID_ARG;
+  std::memcpy(out16, codebook().v, 16 * sizeof(float));
+  return SOUP_OK;
+}
+
+soup_status soup_get_stats(soup_model* m, soup_stats* out) {
+  if (!m || !out) return SOUP_ERR_INVALID_ARG;
+  *out = m->stats;
+  return SOUP_OK;
+}
+
+soup_status soup_reset_stats(soup_model* m) {
+  if (!m) return SOUP_ERR_INVALID_ARG;
+  const long long dev = m->stats.device_bytes, pin = m->stats.pinned_bytes;
+  m->stats = soup_stats{};
+  m->stats.device_bytes = dev;
+  m->stats.pinned_bytes = pin;
+  return SOUP_OK;
+}
+
+soup_status soup_set_profiling(soup_model* m, int enabled) {
+  if (!m) return SOUP_ERR_INVALID_ARG;
+  m->prof = enabled ? 1 : 0;
+  return SOUP_OK;
+}
+
+soup_status soup_get_profile(soup_model* m, soup_profile_entry* out, int max_entries, int* n_entries, int reset) {
+  if (!m || !n_entries || (max_entries > 0 && !out)) return SOUP_ERR_INVALID_ARG;
+  SOUP_GUARD({
+    prof_resolve(m);
+    int n = 0;
+    for (int c = 0; c < CAT_COUNT; ++c) {
+      const auto& pc = m->prof_cats[c];
+      if (pc.launches == 0) continue;
+      if (n < max_entries) {
+        soup_profile_entry& e = out[n];
+        std::memset(&e, 0, sizeof(e));
+        std::strncpy(e.name, kCatNames[c], sizeof(e.name) - 1);
+        e.launches = pc.launches;
+        e.total_ms = pc.ms;
+        e.flops = pc.flops;
+        e.bytes = pc.bytes;
+      }
+      ++n;
+    }
+    *n_entries = std::min(n, std::max(max_entries, 0));
+    if (reset) m->prof_cats.assign(CAT_COUNT, soup_model::ProfCat{});
+    return SOUP_OK;
+  })
+}
+
+soup_status soup_check_device(soup_model* m, void* stream) {
+  if (!m) return SOUP_ERR_INVALID_ARG;
+  SOUP_GUARD(return read_scalars(m, static_cast<cudaStream_t>(stream), nullptr);)
+}
+
+}  // extern "C"

@@ -1,0 +1,265 @@
+"""Thin Python front end of libsoup: passes torch device pointers and streams through the
+C-ABI.  PyTorch supplies device memory (through the allocator callback) and streams; every
+step of the computation runs in libsoup's CUDA kernels.
+"""
+from __future__ import annotations
+
+import ctypes
+from ctypes import byref, c_float, c_int, c_size_t, c_void_p
+
+import numpy as np
+import torch
+
+from . import _lib
+from ._lib import PROJ, Batch, ModelConfig, Stats, check, lib
+
+
+def make_config(cfg: dict, mode: str = "streamed", n_layer_buffers: int = 2, max_tokens: int | None = None,
+                device: int = 0) -> ModelConfig:
+    c = ModelConfig()
+    for k in ("n_layers", "hidden", "n_heads", "n_kv_heads", "head_dim", "intermediate", "vocab", "lora_r"):
+        setattr(c, k, int(cfg[k]))
+    c.rms_eps = float(cfg["rms_eps"])
+    c.rope_theta = float(cfg["rope_theta"])
+    c.lora_alpha = float(cfg["lora_alpha"])
+    c.mode = _lib.SOUP_STREAMED if mode == "streamed" else _lib.SOUP_RESIDENT
+    c.n_layer_buffers = int(n_layer_buffers)
+    c.max_tokens = int(max_tokens if max_tokens is not None else cfg["batch"] * cfg["seq"])
+    c.device = int(device)
+    return c
+
+
+def blob_bytes(cfg: dict) -> int:
+    n = c_size_t()
+    check(lib.soup_layer_blob_bytes(byref(make_config(cfg)), byref(n)))
+    return n.value
+
+
+def blob_part(cfg: dict, proj: int, part: int):
+    off, sz = c_size_t(), c_size_t()
+    check(lib.soup_layer_blob_part(byref(make_config(cfg)), proj, part, byref(off), byref(sz)))
+    return off.value, sz.value
+
+
+def lora_numel(cfg: dict) -> int:
+    n = c_size_t()
+    check(lib.soup_lora_numel(byref(make_config(cfg)), byref(n)))
+    return n.value
+
+
+def lora_offset(cfg: dict, layer: int, proj: int, which_b: int):
+    off, r, c = c_size_t(), c_int(), c_int()
+    check(lib.soup_lora_offset(byref(make_config(cfg)), layer, proj, which_b, byref(off), byref(r), byref(c)))
+    return off.value, r.value, c.value
+
+
+def codebook() -> np.ndarray:
+    out = (c_float * 16)()
+    check(lib.soup_nf4_codebook(out))
+    return np.frombuffer(out, dtype=np.float32).copy()
+
+
+def _stream_ptr(stream=None) -> c_void_p:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return c_void_p(s.cuda_stream)
+
+
+def _ptr(t: torch.Tensor | None) -> c_void_p:
+    return c_void_p(t.data_ptr()) if t is not None else c_void_p(None)
+
+
+class _TorchAllocator:
+    """Routes the library's device allocations to PyTorch's caching allocator."""
+
+    def __init__(self, device: int):
+        self.device = device
+
+        def _alloc(nbytes, user):
+            try:
+                return torch.cuda.caching_allocator_alloc(int(nbytes), self.device)
+            except Exception:  # the library reports SOUP_ERR_OOM
+                return None
+
+        def _free(p, user):
+            torch.cuda.caching_allocator_delete(int(p))
+
+        self._alloc = _lib.ALLOC_FN(_alloc)
+        self._free = _lib.FREE_FN(_free)
+        self.struct = _lib.Allocator(self._alloc, self._free, None)
+
+
+class SoupModel:
+    def __init__(self, cfg: dict, mode: str = "streamed", n_layer_buffers: int = 2, max_tokens: int | None = None,
+                 device: int = 0, torch_alloc: bool = True):
+        self.cfg = dict(cfg)
+        self.ccfg = make_config(cfg, mode, n_layer_buffers, max_tokens, device)
+        self.device = torch.device("cuda", device)
+        self._allocator = _TorchAllocator(device) if torch_alloc else None
+        h = c_void_p()
+        check(lib.soup_model_create(byref(self.ccfg), byref(self._allocator.struct) if self._allocator else None,
+                                    byref(h)))
+        self.h = h
+        self.blob_bytes = blob_bytes(cfg)
+        self._keep = {}
+        self.lora_n = lora_numel(cfg)
+
+    # ------------------------------------------------------------------ lifecycle
+    def close(self):
+        if getattr(self, "h", None):
+            torch.cuda.synchronize(self.device)
+            check(lib.soup_model_destroy(self.h))
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def _ck(self, status):
+        check(status, self.h)
+
+    # ------------------------------------------------------------------ weights
+    def quantize_layer(self, layer: int, w: dict, gamma_attn: torch.Tensor, gamma_mlp: torch.Tensor):
+        """w[p]: fp32 cuda tensors [out, in]; gammas: bf16 cuda tensors [hidden]."""
+        ptrs = (c_void_p * 7)(*[w[p].data_ptr() for p in PROJ])
+        self._ck(lib.soup_model_quantize_layer(self.h, layer, ptrs, _ptr(gamma_attn), _ptr(gamma_mlp), _stream_ptr()))
+
+    def load_layer_nf4(self, layer: int, blob: np.ndarray):
+        blob = np.ascontiguousarray(blob, dtype=np.uint8)
+        self._ck(lib.soup_model_load_layer_nf4(self.h, layer, blob.ctypes.data_as(c_void_p), blob.nbytes))
+
+    def read_layer_nf4(self, layer: int) -> np.ndarray:
+        out = np.empty(self.blob_bytes, dtype=np.uint8)
+        self._ck(lib.soup_model_read_layer_nf4(self.h, layer, out.ctypes.data_as(c_void_p), out.nbytes))
+        return out
+
+    def set_head(self, embed: torch.Tensor, final_gamma: torch.Tensor, lm_head: torch.Tensor):
+        self._keep["head"] = (embed, final_gamma, lm_head)
+        self._ck(lib.soup_model_set_head(self.h, _ptr(embed), _ptr(final_gamma), _ptr(lm_head)))
+
+    def set_lora(self, params: torch.Tensor):
+        """params: flat fp32 cuda tensor of lora_numel elements (layout of include/soup.h)."""
+        assert params.numel() == self.lora_n and params.dtype == torch.float32 and params.is_cuda
+        self.lora_params = params
+        self.lora_grads = torch.zeros_like(params)
+        self.adam_m = torch.zeros_like(params)
+        self.adam_v = torch.zeros_like(params)
+        self._ck(lib.soup_model_set_lora(self.h, _ptr(self.lora_params), _ptr(self.lora_grads), _ptr(self.adam_m),
+                                         _ptr(self.adam_v)))
+
+    def lora_view(self, flat: torch.Tensor, layer: int, proj: str, which_b: int) -> torch.Tensor:
+        off, r, c = lora_offset(self.cfg, layer, PROJ.index(proj), which_b)
+        return flat[off:off + r * c].view(r, c)
+
+    def set_lora_enabled(self, enabled: bool):
+        self._ck(lib.soup_set_lora_enabled(self.h, 1 if enabled else 0))
+
+    # ------------------------------------------------------------------ compute
+    def layer_fwd(self, layer: int, x: torch.Tensor, B: int, S: int, out: torch.Tensor | None = None):
+        y = out if out is not None else torch.empty_like(x)
+        self._ck(lib.soup_layer_fwd(self.h, layer, _ptr(x), _ptr(y), B, S, _stream_ptr()))
+        return y
+
+    def layer_bwd(self, layer: int, dy: torch.Tensor, B: int, S: int, out: torch.Tensor | None = None):
+        dx = out if out is not None else torch.empty_like(dy)
+        self._ck(lib.soup_layer_bwd(self.h, layer, _ptr(dy), _ptr(dx), B, S, _stream_ptr()))
+        return dx
+
+    def step(self, ids, loss: str = "sft", mask=None, n_pairs: int = 0, prefix_len: int = 0, beta: float = 0.1,
+             lr: float = 2e-5, apply_optimizer: bool = True) -> float:
+        """ids: int32 [B, S] as a cuda tensor, or as host memory (numpy / cpu tensor: copied by the library)."""
+        b = Batch()
+        on_host = not (isinstance(ids, torch.Tensor) and ids.is_cuda)
+        if on_host:
+            ids_h = ids if isinstance(ids, torch.Tensor) else torch.from_numpy(np.ascontiguousarray(ids, np.int32))
+            ids_h = ids_h.contiguous()
+            assert ids_h.dtype == torch.int32
+            b.ids = ids_h.data_ptr()
+            keep = [ids_h]
+            if mask is not None:
+                m_h = mask if isinstance(mask, torch.Tensor) else torch.from_numpy(np.ascontiguousarray(mask, np.uint8))
+                m_h = m_h.contiguous()
+                keep.append(m_h)
+                b.loss_mask = m_h.data_ptr()
+            B, S = ids_h.shape
+        else:
+            assert ids.dtype == torch.int32
+            b.ids = ids.data_ptr()
+            if mask is not None:
+                b.loss_mask = mask.data_ptr()
+            B, S = ids.shape
+        b.B, b.S = int(B), int(S)
+        b.ids_on_host = 1 if on_host else 0
+        b.n_pairs, b.prefix_len, b.beta = int(n_pairs), int(prefix_len), float(beta)
+        b.lr, b.apply_optimizer = float(lr), 1 if apply_optimizer else 0
+        out = c_float()
+        kind = _lib.SOUP_LOSS_DPO if loss == "dpo" else _lib.SOUP_LOSS_SFT
+        self._ck(lib.soup_step(self.h, kind, byref(b), byref(out), _stream_ptr()))
+        return out.value
+
+    def optimizer_step(self, lr: float):
+        self._ck(lib.soup_optimizer_step(self.h, float(lr), _stream_ptr()))
+
+    def last_logps(self, n: int):
+        pi, ref = (c_float * n)(), (c_float * n)()
+        self._ck(lib.soup_last_logps(self.h, pi, ref, n))
+        return np.array(pi[:]), np.array(ref[:])
+
+    def stats(self) -> dict:
+        s = Stats()
+        self._ck(lib.soup_get_stats(self.h, byref(s)))
+        return {k: getattr(s, k) for k, _ in Stats._fields_}
+
+    def set_profiling(self, enabled: bool):
+        self._ck(lib.soup_set_profiling(self.h, 1 if enabled else 0))
+
+    def profile(self, reset: bool = False) -> dict:
+        arr = (_lib.ProfileEntry * 64)()
+        n = c_int()
+        self._ck(lib.soup_get_profile(self.h, arr, 64, byref(n), 1 if reset else 0))
+        return {arr[i].name.decode(): dict(launches=arr[i].launches, total_ms=arr[i].total_ms, flops=arr[i].flops,
+                                           bytes=arr[i].bytes) for i in range(n.value)}
+
+    def reset_stats(self):
+        self._ck(lib.soup_reset_stats(self.h))
+
+    def check_device(self):
+        self._ck(lib.soup_check_device(self.h, _stream_ptr()))
+
+
+# ---------------------------------------------------------------------- single ops
+def nf4_quantize(w: torch.Tensor) -> dict:
+    """NF4 + double quant of a cuda fp32 tensor; returns device tensors."""
+    n = w.numel()
+    nb = (n + 63) // 64
+    ng = (nb + 255) // 256
+    dev = w.device
+    out = dict(codes=torch.empty((n + 1) // 2, dtype=torch.uint8, device=dev),
+               q8=torch.empty(nb, dtype=torch.int8, device=dev),
+               scales=torch.empty(ng, dtype=torch.float32, device=dev),
+               mean=torch.empty(1, dtype=torch.float32, device=dev))
+    scratch = torch.empty(nb, dtype=torch.float32, device=dev)
+    check(lib.soup_nf4_quantize(_ptr(w), n, _ptr(out["codes"]), _ptr(out["q8"]), _ptr(out["scales"]),
+                                _ptr(out["mean"]), _ptr(scratch), _stream_ptr()))
+    out["n"] = n
+    out["shape"] = tuple(w.shape)
+    return out
+
+
+def nf4_dequantize(q: dict) -> torch.Tensor:
+    """bf16 (as int16 bit patterns viewed as bfloat16) tensor of shape q['shape']."""
+    out = torch.empty(q["n"], dtype=torch.bfloat16, device=q["codes"].device)
+    check(lib.soup_nf4_dequantize(_ptr(q["codes"]), _ptr(q["q8"]), _ptr(q["scales"]), _ptr(q["mean"]), q["n"],
+                                  _ptr(out), _stream_ptr()))
+    return out.view(q["shape"])
+
+
+def nf4_matmul(x: torch.Tensor, q: dict, transpose_w: bool = False, residual: torch.Tensor | None = None):
+    """y = x W^T (W = NF4 tensor [N, K]) or y = x W when transpose_w; bf16 in/out."""
+    N, K = q["shape"]
+    M = x.shape[0]
+    y = torch.empty((M, K if transpose_w else N), dtype=torch.bfloat16, device=x.device)
+    check(lib.soup_nf4_matmul(_ptr(x), M, N, K, _ptr(q["codes"]), _ptr(q["q8"]), _ptr(q["scales"]), _ptr(q["mean"]),
+                              1 if transpose_w else 0, _ptr(residual), _ptr(y), _stream_ptr()))
+    return y

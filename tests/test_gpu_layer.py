@@ -1,0 +1,85 @@
+"""GPU parity of one decoder layer (forward and backward with LoRA) against the float64
+oracle, on the small Llama-style shape (hidden 256, 4/2 heads, head_dim 64, intermediate
+688: ragged K and N tiles) and a ragged token count."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import model as om
+from tests.gpu_util import Pair, bf16_tensor, cosine, rel_err, to64
+
+pytestmark = pytest.mark.gpu
+
+PROJ = synth.PROJ_NAMES
+
+
+@pytest.fixture(scope="module")
+def pair():
+    cfg = dict(synth.TINY)
+    p = Pair(cfg, seed=3, modes=("resident",), max_tokens=2 * 64)
+    yield p
+    p.close()
+
+
+@pytest.mark.parametrize("B,S", [(1, 64), (2, 37)])
+@pytest.mark.parametrize("lora_on", [True, False])
+def test_layer_forward_backward(pair, B, S, lora_on):
+    cfg = pair.cfg
+    gm = pair.models["resident"]
+    gm.set_lora_enabled(lora_on)
+    T, h = B * S, cfg["hidden"]
+    xb = synth.bf16_bits_from_f32(synth.normal(21, T, (T, h), 1.0))
+    dyb = synth.bf16_bits_from_f32(synth.normal(22, T, (T, h), 1.0))
+    x, dy = bf16_tensor(xb), bf16_tensor(dyb)
+    gm.lora_grads.zero_()
+    y = gm.layer_fwd(1, x, B, S)
+    dx = gm.layer_bwd(1, dy, B, S)
+    torch.cuda.synchronize()
+    gm.set_lora_enabled(True)
+    lo = {p: pair.olora[(1, p)] for p in PROJ}
+    y_o, cache = om.layer_forward(cfg, pair.olayers[1], lo, to64(x), B, S, enabled=lora_on)
+    dx_o, g_o = om.layer_backward(cfg, pair.olayers[1], lo, cache, to64(dy), B, S, enabled=lora_on)
+    # compare the layer's update (the residual input dominates the output)
+    assert rel_err(to64(y) - to64(x), y_o - to64(x)) < 2e-2
+    assert rel_err(to64(dx) - to64(dy), dx_o - to64(dy)) < 2e-2
+    grads = pair.gpu_grads("resident")
+    for p in PROJ:
+        gA, gB = grads[(1, p)]
+        if lora_on:
+            assert cosine(gA, g_o[p][0]) > 0.999, p
+            assert cosine(gB, g_o[p][1]) > 0.999, p
+        else:
+            assert np.all(gA == 0) and np.all(gB == 0)
+        assert np.all(grads[(0, p)][0] == 0)  # other layer untouched
+
+
+def test_lora_off_equals_zero_b_bitwise():
+    cfg = dict(synth.TINY)
+    a = Pair(cfg, seed=4, modes=("resident",), want_oracle=False)
+    b = Pair(cfg, seed=4, modes=("resident",), zero_b=True, want_oracle=False)
+    try:
+        T, h = 64, cfg["hidden"]
+        x = bf16_tensor(synth.bf16_bits_from_f32(synth.normal(23, T, (T, h), 1.0)))
+        a.models["resident"].set_lora_enabled(False)
+        ya = a.models["resident"].layer_fwd(0, x, 1, 64)
+        yb = b.models["resident"].layer_fwd(0, x, 1, 64)
+        torch.cuda.synchronize()
+        # B = 0 adds an exact zero to every fp32 accumulator: same bits as LoRA off
+        assert torch.equal(ya.view(torch.int16), yb.view(torch.int16))
+    finally:
+        a.close()
+        b.close()
+
+
+def test_bwd_without_fwd_is_state_error():
+    from layer_streamed_nf4_lut_b200._lib import SoupError
+    cfg = dict(synth.TINY)
+    p = Pair(cfg, seed=5, modes=("streamed",), want_oracle=False)
+    try:
+        dy = torch.zeros(64, cfg["hidden"], dtype=torch.bfloat16, device="cuda")
+        with pytest.raises(SoupError) as ei:
+            p.models["streamed"].layer_bwd(0, dy, 1, 64)
+        assert ei.value.status == -2
+    finally:
+        p.close()
