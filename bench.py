@@ -189,6 +189,7 @@ def h2d_probe(nbytes, device_index, reps=20):
 def run_soup(args, wl, rank, world, local_rank):
     import torch
     import torch.distributed as dist
+    from layer_streamed_nf4_lut_b200 import dp
     from layer_streamed_nf4_lut_b200.model import SoupModel  # noqa: F401  (fails loudly without libsoup.so)
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
@@ -206,10 +207,8 @@ def run_soup(args, wl, rank, world, local_rank):
     def one_step(ids_arg, mask_arg):
         if world == 1:
             return gm.step(ids_arg, **dict(kw, mask=mask_arg), apply_optimizer=True)
-        loss = gm.step(ids_arg, **dict(kw, mask=mask_arg), apply_optimizer=False)
-        dist.all_reduce(gm.lora_grads)
-        gm.lora_grads.mul_(1.0 / world)
-        gm.optimizer_step(2e-5)
+        loss, _ = dp.dp_step(lambda: gm.step(ids_arg, **dict(kw, mask=mask_arg), apply_optimizer=False),
+                             gm.lora_grads, lambda: gm.optimizer_step(2e-5))
         return loss
 
     h2d_gbs = h2d_probe(gm.blob_bytes, local_rank)
@@ -232,9 +231,7 @@ def run_soup(args, wl, rank, world, local_rank):
     ms = e0.elapsed_time(e1)
     st = gm.stats()
     if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+        ms = dp.max_over_ranks(ms, device=dev)
     ms_step = ms / args.steps
     tok_s = world * T * args.steps / (ms * 1e-3)
     loads_per_step = st["layer_loads"] / args.steps
@@ -261,9 +258,7 @@ def run_soup(args, wl, rank, world, local_rank):
     torch.cuda.synchronize(dev)
     e2e_s = time.perf_counter() - t0
     if world > 1:
-        t = torch.tensor([e2e_s], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_s = float(t.item())
+        e2e_s = dp.max_over_ranks(e2e_s, device=dev)
     e2e_tok_s = world * T * args.steps / e2e_s
 
     if rank != 0:

@@ -6,28 +6,36 @@
 //   * backward dx = dy W + s (dy B) A     : the same NF4 weight read transposed;
 //   * LoRA grads, lm_head forward/backward: plain bf16 / fp32 operands.
 //
-// Roles (384 threads, one CTA per 128 x BN output tile):
-//   warps 0-7  producers: global -> registers -> (NF4 LUT dequant | fp32->bf16 | copy) ->
-//              shared memory in the 128-byte-swizzled K-major layout the tensor core reads;
+// Roles (384 threads, one CTA per 128 x BN output tile, or per K-slice of it under split-K):
+//   warps 0-7  producers, two groups of four warps that fill alternate k-blocks so that one
+//              group's global-memory latency overlaps the other's dequantisation.  A K-major
+//              bf16 A tile arrives by TMA (cp.async.bulk.tensor, 128-byte swizzle, no thread
+//              involvement); the B tile is gathered into registers first (codes, q8 absmax,
+//              group scales), then dequantised through a 16-entry shared-memory codebook and
+//              stored in the same 128-byte-swizzled K-major layout;
 //   warp 8     allocates the TMEM accumulator; lane 0 issues tcgen05.mma (M=128, N=BN, K=16)
 //              and tcgen05.commit to release stages;
-//   warps 8-11 epilogue: tcgen05.ld rows out of TMEM, scale, add residual / old value, store.
-// A STAGES-deep ring of (A,B) tiles with full/empty mbarriers overlaps loads with MMAs.
+//   warps 8-11 epilogue: tcgen05.ld rows out of TMEM, scale, add residual / old value, store
+//              (or store an fp32 partial tile under split-K).
 //
 // NF4 decode follows the double-quantised format: mhat = fp32(fp32(q8 * s2) + mean),
-// w = bf16_rn(fp32(code_value * mhat)), one float32 multiply per element, codebook read from
-// a 16-entry shared-memory table.
+// w = bf16_rn(fp32(code_value * mhat)), one float32 multiply per element.
 #include "common.cuh"
 #include "internal.h"
 
+#include <cudaTypedefs.h>
+
+#include <algorithm>
 #include <atomic>
+#include <mutex>
 
 namespace soup {
 
 namespace {
 
 constexpr int GEMM_THREADS = 384;
-constexpr int PRODUCER_THREADS = 256;
+constexpr int GROUPS = 2;
+constexpr int GROUP_THREADS = 128;
 constexpr int BM = 128;
 constexpr int BK = 64;  // 64 bf16 = 128 bytes = one swizzle row
 
@@ -36,12 +44,12 @@ struct GemmCfg {
   static constexpr int A_BYTES = BM * 128;
   static constexpr int B_BYTES = BN * 128;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES = (BN >= 256) ? 4 : (BN >= 128 ? 5 : 6);
+  static constexpr int STAGES = (BN >= 256) ? 4 : (BN >= 128 ? 6 : 8);
   static constexpr int CTRL_BYTES = 512;
   static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + CTRL_BYTES;
 };
 
-// ---------------------------------------------------------------- tcgen05 wrappers
+// ---------------------------------------------------------------- tcgen05 / TMA wrappers
 __device__ __forceinline__ void tmem_alloc(uint32_t* slot, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot)), "r"(ncols)
                : "memory");
@@ -82,6 +90,18 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 }
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+// 2D tiled TMA load (no multicast) into shared memory, completion counted on `bar`.
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
 // Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row core groups 1024 B apart.
 __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t saddr) {
   uint64_t d = 0;
@@ -104,21 +124,35 @@ __device__ __forceinline__ uint32_t idesc_bf16_f32() {
 }
 
 // ---------------------------------------------------------------- operand fetch
-__device__ __forceinline__ float nf4_mhat(const NF4Seg& sg, long long blk) {
-  const float s2 = __ldg(sg.scales + (blk >> 8));
-  const float q = static_cast<float>(__ldg(sg.q8 + blk));
-  return __fadd_rn(__fmul_rn(q, s2), __ldg(sg.mean));
-}
-
-// 8 consecutive columns [wc, wc+8) of NF4 row wr as 8 bf16 (wc multiple of 8, in range).
-__device__ __forceinline__ uint4 nf4_chunk8(const NF4Group& g, const float* lut, int wr, int wc) {
+__device__ __forceinline__ int nf4_seg_of(const NF4Group& g, int wr) {
   int s = 0;
   if (g.nseg > 1 && wr >= g.seg[1].row_begin) s = 1;
   if (g.nseg > 2 && wr >= g.seg[2].row_begin) s = 2;
+  return s;
+}
+
+// Raw gather of one NF4 chunk (8 consecutive columns of W row wr): code word, q8, s2, segment.
+struct NF4Raw {
+  uint32_t code;
+  float s2;
+  int q8;
+  int seg;
+};
+__device__ __forceinline__ NF4Raw nf4_gather(const NF4Group& g, int wr, int wc) {
+  const int s = nf4_seg_of(g, wr);
   const NF4Seg& sg = g.seg[s];
   const long long flat = static_cast<long long>(wr - sg.row_begin) * g.cols + wc;
-  const float mh = nf4_mhat(sg, flat >> 6);
-  const uint32_t c = __ldg(reinterpret_cast<const uint32_t*>(sg.codes + (flat >> 1)));
+  const long long blk = flat >> 6;
+  NF4Raw r;
+  r.code = __ldg(reinterpret_cast<const uint32_t*>(sg.codes + (flat >> 1)));
+  r.q8 = __ldg(sg.q8 + blk);
+  r.s2 = __ldg(sg.scales + (blk >> 8));
+  r.seg = s;
+  return r;
+}
+__device__ __forceinline__ uint4 nf4_decode(const NF4Raw& r, const float* lut, const float* seg_mean) {
+  const float mh = __fadd_rn(__fmul_rn(static_cast<float>(r.q8), r.s2), seg_mean[r.seg]);
+  const uint32_t c = r.code;
   uint4 o;
   o.x = pack_bf16x2(__fmul_rn(lut[c & 15u], mh), __fmul_rn(lut[(c >> 4) & 15u], mh));
   o.y = pack_bf16x2(__fmul_rn(lut[(c >> 8) & 15u], mh), __fmul_rn(lut[(c >> 12) & 15u], mh));
@@ -127,87 +161,118 @@ __device__ __forceinline__ uint4 nf4_chunk8(const NF4Group& g, const float* lut,
   return o;
 }
 
-__device__ __forceinline__ uint4 fetch_kmajor(const Operand& op, const NF4Group& g, const float* lut, int r, int k) {
-  switch (op.kind) {
-    case OP_BF16_K:
-      return __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(op.ptr) + r * op.ld + k));
-    case OP_F32_K: {
-      const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(op.ptr) + r * op.ld + k);
-      const float4 a = __ldg(src), b = __ldg(src + 1);
-      const float s = op.scale;
-      uint4 o;
-      o.x = pack_bf16x2(a.x * s, a.y * s);
-      o.y = pack_bf16x2(a.z * s, a.w * s);
-      o.z = pack_bf16x2(b.x * s, b.y * s);
-      o.w = pack_bf16x2(b.z * s, b.w * s);
-      return o;
-    }
-    default:  // OP_NF4_K
-      return nf4_chunk8(g, lut, r, k);
-  }
+__device__ __forceinline__ uint4 cvt_f32x8(const float* src, float s) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(src)), b = __ldg(reinterpret_cast<const float4*>(src) + 1);
+  uint4 o;
+  o.x = pack_bf16x2(a.x * s, a.y * s);
+  o.y = pack_bf16x2(a.z * s, a.w * s);
+  o.z = pack_bf16x2(b.x * s, b.y * s);
+  o.w = pack_bf16x2(b.z * s, b.w * s);
+  return o;
 }
 
-// 8 consecutive rows [r, r+8) at reduction index k, as 8 bf16 (zero when k >= K).
-__device__ __forceinline__ uint4 fetch_mn8(const Operand& op, const NF4Group& g, const float* lut, int r, int k,
-                                           int K) {
+// 8 consecutive k of row r (K-major, non-NF4 kinds).
+__device__ __forceinline__ uint4 fetch_kmajor(const Operand& op, int r, int k) {
+  if (op.kind == OP_BF16_K)
+    return __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(op.ptr) + r * op.ld + k));
+  return cvt_f32x8(static_cast<const float*>(op.ptr) + r * op.ld + k, op.scale);  // OP_F32_K
+}
+// 8 consecutive rows [r, r+8) at reduction index k (MN-major, non-NF4 kinds), zero past K.
+__device__ __forceinline__ uint4 fetch_mn8(const Operand& op, int r, int k, int K) {
   if (k >= K) return make_uint4(0, 0, 0, 0);
-  switch (op.kind) {
-    case OP_BF16_MN:
-      return __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(op.ptr) + k * op.ld + r));
-    case OP_F32_MN: {
-      const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(op.ptr) + k * op.ld + r);
-      const float4 a = __ldg(src), b = __ldg(src + 1);
-      const float s = op.scale;
-      uint4 o;
-      o.x = pack_bf16x2(a.x * s, a.y * s);
-      o.y = pack_bf16x2(a.z * s, a.w * s);
-      o.z = pack_bf16x2(b.x * s, b.y * s);
-      o.w = pack_bf16x2(b.z * s, b.w * s);
-      return o;
-    }
-    default:  // OP_NF4_MN: W[k, r..r+7]
-      return nf4_chunk8(g, lut, k, r);
-  }
+  if (op.kind == OP_BF16_MN)
+    return __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(op.ptr) + k * op.ld + r));
+  return cvt_f32x8(static_cast<const float*>(op.ptr) + k * op.ld + r, op.scale);  // OP_F32_MN
 }
 
 __device__ __forceinline__ uint32_t swz_off(int r, int chunk) {
   return static_cast<uint32_t>((r >> 3) * 1024 + (r & 7) * 128 + ((chunk ^ (r & 7)) << 4));
 }
 
-// Fill one ROWS x 64 tile of an operand into swizzled shared memory.
+__device__ __forceinline__ void store_mn_pairs(uint8_t* tile, int rr0, int kp, const uint4& x0, const uint4& x1) {
+  const uint32_t a[4] = {x0.x, x0.y, x0.z, x0.w};
+  const uint32_t b[4] = {x1.x, x1.y, x1.z, x1.w};
+  const uint32_t inchunk = (kp & 3) * 4;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t lo = __byte_perm(a[j], b[j], 0x5410);  // row 2j:   (k, k+1)
+    const uint32_t hi = __byte_perm(a[j], b[j], 0x7632);  // row 2j+1: (k, k+1)
+    *reinterpret_cast<uint32_t*>(tile + swz_off(rr0 + 2 * j, kp >> 2) + inchunk) = lo;
+    *reinterpret_cast<uint32_t*>(tile + swz_off(rr0 + 2 * j + 1, kp >> 2) + inchunk) = hi;
+  }
+}
+
+// Fill one ROWS x 64 tile of an operand (group-cooperative, gtid in [0, 128)).
 template <int ROWS>
-__device__ __forceinline__ void load_tile(const Operand& op, const NF4Group& g, const float* lut, int K, int row0,
-                                          int nrows, int k0, uint8_t* tile, int ptid) {
-  const bool kmajor = (op.kind == OP_BF16_K || op.kind == OP_F32_K || op.kind == OP_NF4_K);
-  if (kmajor) {
-#pragma unroll 2
-    for (int c = ptid; c < ROWS * 8; c += PRODUCER_THREADS) {
+__device__ __forceinline__ void load_tile(const Operand& op, const NF4Group& g, const float* lut,
+                                          const float* seg_mean, int K, int row0, int nrows, int k0, uint8_t* tile,
+                                          int gtid) {
+  if (op.kind == OP_NF4_K) {
+    constexpr int CH = ROWS * 8 / GROUP_THREADS;
+    constexpr int BATCH = CH < 8 ? CH : 8;  // chunks gathered before any is decoded
+#pragma unroll
+    for (int b0 = 0; b0 < CH; b0 += BATCH) {
+      NF4Raw raw[BATCH];
+      bool ok[BATCH];
+#pragma unroll
+      for (int i = 0; i < BATCH; ++i) {  // phase 1: issue the global loads of the batch
+        const int c = gtid + (b0 + i) * GROUP_THREADS;
+        const int row = row0 + (c >> 3), k = k0 + (c & 7) * 8;
+        ok[i] = row < nrows && row >= op.row_lo && row < op.row_hi && k < K;
+        if (ok[i]) raw[i] = nf4_gather(g, row, k);
+      }
+#pragma unroll
+      for (int i = 0; i < BATCH; ++i) {  // phase 2: dequantise and store
+        const int c = gtid + (b0 + i) * GROUP_THREADS;
+        const uint4 v = ok[i] ? nf4_decode(raw[i], lut, seg_mean) : make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4*>(tile + swz_off(c >> 3, c & 7)) = v;
+      }
+    }
+  } else if (op.kind == OP_NF4_MN) {
+    constexpr int U = (ROWS / 8) * 32 / GROUP_THREADS;
+    constexpr int BATCH = U < 4 ? U : 4;
+#pragma unroll
+    for (int b0 = 0; b0 < U; b0 += BATCH) {
+      NF4Raw r0[BATCH], r1[BATCH];
+      bool ok0[BATCH], ok1[BATCH];
+#pragma unroll
+      for (int i = 0; i < BATCH; ++i) {
+        const int u = gtid + (b0 + i) * GROUP_THREADS;
+        const int kp = u & 31, row = row0 + (u >> 5) * 8, k = k0 + kp * 2;
+        const bool rows_ok = row < nrows;
+        ok0[i] = rows_ok && k < K;
+        ok1[i] = rows_ok && k + 1 < K;
+        if (ok0[i]) r0[i] = nf4_gather(g, k, row);
+        if (ok1[i]) r1[i] = nf4_gather(g, k + 1, row);
+      }
+#pragma unroll
+      for (int i = 0; i < BATCH; ++i) {
+        const int u = gtid + (b0 + i) * GROUP_THREADS;
+        const uint4 x0 = ok0[i] ? nf4_decode(r0[i], lut, seg_mean) : make_uint4(0, 0, 0, 0);
+        const uint4 x1 = ok1[i] ? nf4_decode(r1[i], lut, seg_mean) : make_uint4(0, 0, 0, 0);
+        store_mn_pairs(tile, (u >> 5) * 8, u & 31, x0, x1);
+      }
+    }
+  } else if (op.kind == OP_BF16_K || op.kind == OP_F32_K) {
+#pragma unroll 4
+    for (int c = gtid; c < ROWS * 8; c += GROUP_THREADS) {
       const int rr = c >> 3, kc = c & 7;
       const int row = row0 + rr, k = k0 + kc * 8;
       uint4 v = make_uint4(0, 0, 0, 0);
-      if (row < nrows && row >= op.row_lo && row < op.row_hi && k < K) v = fetch_kmajor(op, g, lut, row, k);
+      if (row < nrows && row >= op.row_lo && row < op.row_hi && k < K) v = fetch_kmajor(op, row, k);
       *reinterpret_cast<uint4*>(tile + swz_off(rr, kc)) = v;
     }
-  } else {
-    // units of 8 rows x 2 consecutive k; 32 k-pairs per warp pass keep the 4-byte stores conflict-free
-    for (int u = ptid; u < (ROWS / 8) * 32; u += PRODUCER_THREADS) {
-      const int kp = u & 31, grp = u >> 5;
-      const int rr0 = grp * 8, row = row0 + rr0, k = k0 + kp * 2;
+  } else {  // OP_BF16_MN / OP_F32_MN: units of 8 rows x 2 consecutive k
+#pragma unroll 2
+    for (int u = gtid; u < (ROWS / 8) * 32; u += GROUP_THREADS) {
+      const int kp = u & 31, rr0 = (u >> 5) * 8;
+      const int row = row0 + rr0, k = k0 + kp * 2;
       uint4 x0 = make_uint4(0, 0, 0, 0), x1 = make_uint4(0, 0, 0, 0);
       if (row < nrows && row >= op.row_lo && row < op.row_hi) {
-        x0 = fetch_mn8(op, g, lut, row, k, K);
-        x1 = fetch_mn8(op, g, lut, row, k + 1, K);
+        x0 = fetch_mn8(op, row, k, K);
+        x1 = fetch_mn8(op, row, k + 1, K);
       }
-      const uint32_t a[4] = {x0.x, x0.y, x0.z, x0.w};
-      const uint32_t b[4] = {x1.x, x1.y, x1.z, x1.w};
-      const uint32_t inchunk = (kp & 3) * 4;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const uint32_t lo = __byte_perm(a[j], b[j], 0x5410);  // (row 2j: k, k+1)
-        const uint32_t hi = __byte_perm(a[j], b[j], 0x7632);  // (row 2j+1: k, k+1)
-        *reinterpret_cast<uint32_t*>(tile + swz_off(rr0 + 2 * j, kp >> 2) + inchunk) = lo;
-        *reinterpret_cast<uint32_t*>(tile + swz_off(rr0 + 2 * j + 1, kp >> 2) + inchunk) = hi;
-      }
+      store_mn_pairs(tile, rr0, kp, x0, x1);
     }
   }
 }
@@ -215,6 +280,61 @@ __device__ __forceinline__ void load_tile(const Operand& op, const NF4Group& g, 
 __device__ __forceinline__ bool seg_active(const GemmSeg& s, int n0, int bn) {
   if (s.K <= 0) return false;
   return s.B.row_lo < n0 + bn && s.B.row_hi > n0;
+}
+
+// Epilogue store of 8 consecutive columns [col, col+8) of row `row` (value already scaled).
+__device__ __forceinline__ void epilogue_store8(const GemmParams& p, int row, int col, float (&v)[8]) {
+  if (!p.out_trans) {
+    if (p.residual) {
+      const uint4 rv = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.residual) + row * p.ldr + col);
+      const uint32_t rw[4] = {rv.x, rv.y, rv.z, rv.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = unpack_bf16x2(rw[j]);
+        v[2 * j] += f.x;
+        v[2 * j + 1] += f.y;
+      }
+    }
+    if (p.out_f32) {
+      float4* o = reinterpret_cast<float4*>(static_cast<float*>(p.out) + row * p.ldo + col);
+      if (p.accumulate) {
+        const float4 a = o[0], b = o[1];
+        v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w;
+        v[4] += b.x; v[5] += b.y; v[6] += b.z; v[7] += b.w;
+      }
+      o[0] = make_float4(v[0], v[1], v[2], v[3]);
+      o[1] = make_float4(v[4], v[5], v[6], v[7]);
+    } else {
+      uint4* o = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + row * p.ldo + col);
+      if (p.accumulate) {
+        const uint4 a = *o;
+        const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float2 f = unpack_bf16x2(aw[j]);
+          v[2 * j] += f.x;
+          v[2 * j + 1] += f.y;
+        }
+      }
+      *o = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                      pack_bf16x2(v[6], v[7]));
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const long long idx = static_cast<long long>(col + j) * p.ldo + row;
+      if (p.out_f32) {
+        float* o = static_cast<float*>(p.out) + idx;
+        *o = p.accumulate ? (*o + v[j]) : v[j];
+      } else {
+        uint16_t* o = static_cast<uint16_t*>(p.out) + idx;
+        float w = v[j];
+        if (p.accumulate) w += bf16_to_f32(*o);
+        const __nv_bfloat16 b = __float2bfloat16_rn(w);
+        *o = *reinterpret_cast<const uint16_t*>(&b);
+      }
+    }
+  }
 }
 
 // ---------------------------------------------------------------- the kernel
@@ -230,6 +350,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
   uint64_t* done = empty + C::STAGES;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* seg_mean = reinterpret_cast<float*>(tmem_slot + 4);
   float* lut = reinterpret_cast<float*>(ctrl + 256);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -237,7 +358,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(&full[s], PRODUCER_THREADS / 32);
+      mbar_init(&full[s], GROUP_THREADS / 32 + 1);  // 4 producer warps + the TMA / leader arrival
       mbar_init(&empty[s], 1);
     }
     mbar_init(done, 1);
@@ -245,6 +366,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
     mbar_fence_init();
   }
   if (threadIdx.x < 16) lut[threadIdx.x] = p.lut[threadIdx.x];
+  if (threadIdx.x >= 32 && threadIdx.x < 32 + p.nf4.nseg) seg_mean[threadIdx.x - 32] = *p.nf4.seg[threadIdx.x - 32].mean;
   if (warp == 8) {
     tmem_alloc(tmem_slot, BN);
     tmem_relinquish();
@@ -254,22 +376,41 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  // this CTA's slice of the k-block list (all active segments concatenated)
+  int nkb_all = 0;
+  for (int s = 0; s < p.nseg; ++s)
+    if (seg_active(p.seg[s], n0, BN)) nkb_all += (p.seg[s].K + BK - 1) / BK;
+  const int splits = p.splits > 1 ? p.splits : 1;
+  const int kb_lo = static_cast<int>(static_cast<long long>(blockIdx.z) * nkb_all / splits);
+  const int kb_hi = static_cast<int>(static_cast<long long>(blockIdx.z + 1) * nkb_all / splits);
+
   if (warp < 8) {
-    // ------------------------------------------------ producers
-    const int ptid = threadIdx.x;
-    int kb = 0;
+    // ------------------------------------------------ producers (two groups, alternate k-blocks)
+    const int grp = warp >> 2, gtid = threadIdx.x & (GROUP_THREADS - 1);
+    int g = 0;
     for (int s = 0; s < p.nseg; ++s) {
       const GemmSeg& sg = p.seg[s];
       if (!seg_active(sg, n0, BN)) continue;
       const int nk = (sg.K + BK - 1) / BK;
-      for (int kk = 0; kk < nk; ++kk, ++kb) {
+      for (int kk = 0; kk < nk; ++kk, ++g) {
+        if (g < kb_lo || g >= kb_hi) continue;
+        const int kb = g - kb_lo;
+        if ((kb % GROUPS) != grp) continue;
         const int st = kb % C::STAGES;
         const uint32_t ph = static_cast<uint32_t>(kb / C::STAGES) & 1u;
         mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, p.err);
         uint8_t* As = base + st * C::STAGE_BYTES;
         uint8_t* Bs = As + C::A_BYTES;
-        load_tile<BM>(sg.A, p.nf4, lut, sg.K, m0, p.M, kk * BK, As, ptid);
-        load_tile<BN>(sg.B, p.nf4, lut, sg.K, n0, p.N, kk * BK, Bs, ptid);
+        if (gtid == 0) {
+          if (p.a_tma[s]) {
+            mbar_arrive_expect_tx(&full[st], C::A_BYTES);
+            tma_load_2d(As, &p.tmapA[s], kk * BK, m0, &full[st]);
+          } else {
+            mbar_arrive(&full[st]);
+          }
+        }
+        if (!p.a_tma[s]) load_tile<BM>(sg.A, p.nf4, lut, seg_mean, sg.K, m0, p.M, kk * BK, As, gtid);
+        load_tile<BN>(sg.B, p.nf4, lut, seg_mean, sg.K, n0, p.N, kk * BK, Bs, gtid);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&full[st]);
@@ -279,25 +420,19 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
     if (warp == 8 && lane == 0) {
       // ------------------------------------------------ MMA issuer
       const uint32_t idesc = idesc_bf16_f32<BN>();
-      int kb = 0;
-      for (int s = 0; s < p.nseg; ++s) {
-        const GemmSeg& sg = p.seg[s];
-        if (!seg_active(sg, n0, BN)) continue;
-        const int nk = (sg.K + BK - 1) / BK;
-        for (int kk = 0; kk < nk; ++kk, ++kb) {
-          const int st = kb % C::STAGES;
-          const uint32_t ph = static_cast<uint32_t>(kb / C::STAGES) & 1u;
-          mbar_wait_bounded(&full[st], ph, abort_flag, p.err);
-          tc_fence_after();
-          const uint32_t a_addr = smem_u32(base + st * C::STAGE_BYTES);
-          const uint32_t b_addr = a_addr + C::A_BYTES;
+      for (int kb = 0; kb < kb_hi - kb_lo; ++kb) {
+        const int st = kb % C::STAGES;
+        const uint32_t ph = static_cast<uint32_t>(kb / C::STAGES) & 1u;
+        mbar_wait_bounded(&full[st], ph, abort_flag, p.err);
+        tc_fence_after();
+        const uint32_t a_addr = smem_u32(base + st * C::STAGE_BYTES);
+        const uint32_t b_addr = a_addr + C::A_BYTES;
 #pragma unroll
-          for (int j = 0; j < BK / 16; ++j) {
-            tc_mma_f16(tmem, sw128_kmajor_desc(a_addr + j * 32), sw128_kmajor_desc(b_addr + j * 32), idesc,
-                       (kb > 0 || j > 0) ? 1u : 0u);
-          }
-          tc_commit(&empty[st]);
+        for (int j = 0; j < BK / 16; ++j) {
+          tc_mma_f16(tmem, sw128_kmajor_desc(a_addr + j * 32), sw128_kmajor_desc(b_addr + j * 32), idesc,
+                     (kb > 0 || j > 0) ? 1u : 0u);
         }
+        tc_commit(&empty[st]);
       }
       tc_commit(done);
     }
@@ -306,8 +441,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
     const int q = warp - 8;
     mbar_wait_bounded(done, 0u, abort_flag, p.err);
     tc_fence_after();
-    bool any_k = false;
-    for (int s = 0; s < p.nseg; ++s) any_k |= seg_active(p.seg[s], n0, BN);
+    const bool any_k = kb_hi > kb_lo;
     const int row = m0 + q * 32 + lane;
 #pragma unroll 1
     for (int cc = 0; cc < BN; cc += 32) {
@@ -320,59 +454,16 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
         const int col = n0 + cc + g8 * 8;
         if (col >= p.N) break;
         float v[8];
+        if (splits > 1) {
 #pragma unroll
-        for (int j = 0; j < 8; ++j) v[j] = any_k ? p.alpha * __uint_as_float(r[g8 * 8 + j]) : 0.f;
-        if (!p.out_trans) {
-          if (p.residual) {
-            const uint4 rv =
-                *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.residual) + row * p.ldr + col);
-            const uint32_t rw[4] = {rv.x, rv.y, rv.z, rv.w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const float2 f = unpack_bf16x2(rw[j]);
-              v[2 * j] += f.x;
-              v[2 * j + 1] += f.y;
-            }
-          }
-          if (p.out_f32) {
-            float4* o = reinterpret_cast<float4*>(static_cast<float*>(p.out) + row * p.ldo + col);
-            if (p.accumulate) {
-              const float4 a = o[0], b = o[1];
-              v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w;
-              v[4] += b.x; v[5] += b.y; v[6] += b.z; v[7] += b.w;
-            }
-            o[0] = make_float4(v[0], v[1], v[2], v[3]);
-            o[1] = make_float4(v[4], v[5], v[6], v[7]);
-          } else {
-            uint4* o = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + row * p.ldo + col);
-            if (p.accumulate) {
-              const uint4 a = *o;
-              const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
-#pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                const float2 f = unpack_bf16x2(aw[j]);
-                v[2 * j] += f.x;
-                v[2 * j + 1] += f.y;
-              }
-            }
-            *o = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
-                            pack_bf16x2(v[6], v[7]));
-          }
+          for (int j = 0; j < 8; ++j) v[j] = any_k ? __uint_as_float(r[g8 * 8 + j]) : 0.f;
+          float4* o = reinterpret_cast<float4*>(p.workspace + (static_cast<long long>(blockIdx.z) * p.M + row) * p.N + col);
+          o[0] = make_float4(v[0], v[1], v[2], v[3]);
+          o[1] = make_float4(v[4], v[5], v[6], v[7]);
         } else {
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const long long idx = static_cast<long long>(col + j) * p.ldo + row;
-            if (p.out_f32) {
-              float* o = static_cast<float*>(p.out) + idx;
-              *o = p.accumulate ? (*o + v[j]) : v[j];
-            } else {
-              uint16_t* o = static_cast<uint16_t*>(p.out) + idx;
-              float w = v[j];
-              if (p.accumulate) w += bf16_to_f32(*o);
-              const __nv_bfloat16 b = __float2bfloat16_rn(w);
-              *o = *reinterpret_cast<const uint16_t*>(&b);
-            }
-          }
+          for (int j = 0; j < 8; ++j) v[j] = any_k ? p.alpha * __uint_as_float(r[g8 * 8 + j]) : 0.f;
+          epilogue_store8(p, row, col, v);
         }
       }
     }
@@ -386,6 +477,52 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
   }
 }
 
+// Sum of the split-K partial tiles in split order, then the normal epilogue.
+__global__ void splitk_reduce_kernel(const __grid_constant__ GemmParams p) {
+  const long long n8 = p.N / 8;
+  const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= static_cast<long long>(p.M) * n8) return;
+  const int row = static_cast<int>(idx / n8), col = static_cast<int>(idx % n8) * 8;
+  float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  for (int s = 0; s < p.splits; ++s) {
+    const float4* src = reinterpret_cast<const float4*>(p.workspace + (static_cast<long long>(s) * p.M + row) * p.N + col);
+    const float4 a = src[0], b = src[1];
+    v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w;
+    v[4] += b.x; v[5] += b.y; v[6] += b.z; v[7] += b.w;
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) v[j] *= p.alpha;
+  epilogue_store8(p, row, col, v);
+}
+
+// ---------------------------------------------------------------- host side
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+// TMA descriptor for a K-major bf16 operand: dims (K, M), row stride ld elements, 64 x 128 box,
+// 128-byte swizzle (the layout the MMA descriptors expect), zero fill out of bounds.
+bool encode_kmajor_bf16(CUtensorMap* map, const void* ptr, int K, int M, long long ld) {
+  auto fn = tensor_map_encoder();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
+  cuuint32_t box[2] = {BK, BM};
+  cuuint32_t es[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int BN>
 cudaError_t launch_bn(const GemmParams& p, cudaStream_t st) {
   using C = GemmCfg<BN>;
@@ -395,8 +532,13 @@ cudaError_t launch_bn(const GemmParams& p, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     attr_done.store(1);
   }
-  dim3 grid((p.N + BN - 1) / BN, (p.M + BM - 1) / BM);
+  dim3 grid((p.N + BN - 1) / BN, (p.M + BM - 1) / BM, p.splits > 1 ? p.splits : 1);
   gemm_tc_kernel<BN><<<grid, GEMM_THREADS, C::SMEM_BYTES, st>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || p.splits <= 1) return e;
+  const long long work = static_cast<long long>(p.M) * (p.N / 8);
+  splitk_reduce_kernel<<<static_cast<unsigned>((work + 255) / 256), 256, 0, st>>>(p);
+  ++g_kernel_launches;
   return cudaGetLastError();
 }
 
@@ -425,8 +567,9 @@ bool is_mn(int kind) { return kind == OP_BF16_MN || kind == OP_F32_MN || kind ==
 
 }  // namespace
 
-cudaError_t gemm_launch(const GemmParams& p, cudaStream_t st) {
-  if (p.M <= 0 || p.N <= 0) return cudaSuccess;
+cudaError_t gemm_launch(const GemmParams& p_in, cudaStream_t st) {
+  if (p_in.M <= 0 || p_in.N <= 0) return cudaSuccess;
+  GemmParams p = p_in;
   if (p.N % 8 != 0 || p.nseg < 1 || p.nseg > GEMM_MAX_SEG) return cudaErrorInvalidValue;
   if (!aligned16(p.out)) return cudaErrorInvalidValue;
   if (p.out_trans) {
@@ -435,20 +578,35 @@ cudaError_t gemm_launch(const GemmParams& p, cudaStream_t st) {
     if (p.ldo % 8 != 0) return cudaErrorInvalidValue;
     if (p.residual && (!aligned16(p.residual) || p.ldr % 8 != 0)) return cudaErrorInvalidValue;
   }
+  long long nkb = 0;
   for (int s = 0; s < p.nseg; ++s) {
-    const GemmSeg& sg = p.seg[s];
+    GemmSeg& sg = p.seg[s];
+    p.a_tma[s] = 0;
     if (sg.K < 0) return cudaErrorInvalidValue;
     if (sg.K == 0) continue;
     if (!operand_ok(sg.A, sg.K) || !operand_ok(sg.B, sg.K)) return cudaErrorInvalidValue;
     if (is_mn(sg.A.kind) && p.M % 8 != 0) return cudaErrorInvalidValue;
-    if ((sg.A.kind == OP_NF4_K || sg.A.kind == OP_NF4_MN)) return cudaErrorInvalidValue;  // NF4 only as B
+    if (sg.A.kind == OP_NF4_K || sg.A.kind == OP_NF4_MN) return cudaErrorInvalidValue;  // NF4 only as B
     if (sg.B.kind == OP_NF4_K && (p.nf4.cols % 8 != 0 || sg.K > p.nf4.cols)) return cudaErrorInvalidValue;
     if (sg.B.kind == OP_NF4_MN && (p.nf4.cols % 8 != 0 || p.N > p.nf4.cols)) return cudaErrorInvalidValue;
+    if (sg.A.kind == OP_BF16_K) p.a_tma[s] = encode_kmajor_bf16(&p.tmapA[s], sg.A.ptr, sg.K, p.M, sg.A.ld) ? 1 : 0;
+    nkb += (sg.K + BK - 1) / BK;
+  }
+  const int BN = (p.N <= 64) ? 64 : ((p.N <= 128 || static_cast<long long>((p.N + 255) / 256) * ((p.M + 127) / 128) < 148) ? 128 : 256);
+  // split-K for grids that cannot fill the GPU (skinny LoRA GEMMs, long reductions)
+  p.splits = 1;
+  const long long tiles = static_cast<long long>((p.N + BN - 1) / BN) * ((p.M + BM - 1) / BM);
+  if (p.workspace && tiles < 100 && nkb >= 8) {
+    long long sp = (2 * 148 + tiles - 1) / tiles;
+    sp = std::min<long long>(sp, nkb / 4);
+    sp = std::min<long long>(sp, 32);
+    while (sp > 1 && static_cast<unsigned long long>(sp) * p.M * p.N * 4ull > p.ws_bytes) --sp;
+    p.splits = static_cast<int>(sp < 1 ? 1 : sp);
   }
   cudaError_t e;
-  if (p.N <= 64)
+  if (BN == 64)
     e = launch_bn<64>(p, st);
-  else if (p.N <= 128 || static_cast<long long>((p.N + 255) / 256) * ((p.M + 127) / 128) < 148)
+  else if (BN == 128)
     e = launch_bn<128>(p, st);
   else
     e = launch_bn<256>(p, st);

@@ -1,5 +1,6 @@
 // Internal declarations shared by the libsoup translation units (not part of the C-ABI).
 #pragma once
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 #include <stddef.h>
@@ -54,6 +55,8 @@ struct GemmSeg {
 constexpr int GEMM_MAX_SEG = 5;
 
 struct GemmParams {
+  CUtensorMap tmapA[GEMM_MAX_SEG];  // TMA descriptors of K-major bf16 A operands (filled by gemm_launch)
+  int a_tma[GEMM_MAX_SEG];          // 1: segment's A tile arrives by TMA
   int M, N;
   int nseg;
   GemmSeg seg[GEMM_MAX_SEG];
@@ -69,6 +72,11 @@ struct GemmParams {
   const void* residual;  // bf16, same layout as out (not with out_trans)
   long long ldr;
   int* err;
+  // split-K: when workspace is given, gemm_launch may split the K loop over `splits` CTAs that
+  // write fp32 partial tiles to the workspace; a second kernel sums them in split order
+  float* workspace;
+  size_t ws_bytes;
+  int splits;  // set by gemm_launch
 };
 
 // Launch C = sum_seg A_seg B_seg^T on the tcgen05 tensor cores. Returns cudaError_t of launch.

@@ -232,6 +232,8 @@ struct soup_model {
   // scalars: [0] loss (f32), [1] device error word (int)
   int* scal = nullptr;
   float* quant_scratch = nullptr;  // absmax scratch for the quantiser
+  float* gemm_ws = nullptr;        // split-K partial tiles
+  size_t gemm_ws_bytes = 0;
   float* host_scal = nullptr;      // pinned 2-word staging for the loss + error readback
 
   std::vector<void*> dev_allocs;
@@ -460,6 +462,8 @@ GemmParams gemm_base(soup_model* m, int M, int N, void* out, long long ldo, int 
   p.out_f32 = out_f32;
   p.alpha = alpha;
   p.err = m->scal + 1;
+  p.workspace = m->gemm_ws;
+  p.ws_bytes = m->gemm_ws_bytes;
   std::memcpy(p.lut, codebook().v, sizeof(p.lut));
   return p;
 }
@@ -1098,6 +1102,8 @@ soup_status create_model(const soup_model_config* cfg, const soup_allocator* all
       alloc_into(m, m->pi, T) || alloc_into(m, m->ref, T) || alloc_into(m, m->ids_dev, T) ||
       alloc_into(m, m->mask_dev, T) || alloc_into(m, m->scal, 64))
     return fail(SOUP_ERR_OOM);
+  m->gemm_ws_bytes = static_cast<size_t>(64) << 20;
+  if (alloc_into(m, m->gemm_ws, m->gemm_ws_bytes / sizeof(float))) return fail(SOUP_ERR_OOM);
   if (cudaMemset(m->scal, 0, 64 * sizeof(int)) != cudaSuccess) return fail(SOUP_ERR_CUDA);
   m->lora_n = lora_numel_of(c);
   *out = m;

@@ -37,11 +37,11 @@ class Pair:
     """A GPU model and the oracle's float64 weights for the same synthetic inputs."""
 
     def __init__(self, cfg, seed=0, modes=("streamed",), gamma_noise=0.1, zero_b=False, max_tokens=None,
-                 n_layer_buffers=2, want_oracle=True):
+                 n_layer_buffers=2, want_oracle=True, w_std=0.02):
         from layer_streamed_nf4_lut_b200.model import SoupModel
         self.cfg = cfg
         L = cfg["n_layers"]
-        self.weights = [synth.layer_weights(cfg, seed, i, gamma_noise=gamma_noise) for i in range(L)]
+        self.weights = [synth.layer_weights(cfg, seed, i, std=w_std, gamma_noise=gamma_noise) for i in range(L)]
         self.head_bits = synth.head_weights(cfg, seed, gamma_noise=gamma_noise)
         self.lora = synth.lora_weights(cfg, seed, zero_b=zero_b)
         self.gamma_bits = [(synth.bf16_bits_from_f32(w["attn_norm"]), synth.bf16_bits_from_f32(w["mlp_norm"]))

@@ -17,7 +17,9 @@ PROJ = synth.PROJ_NAMES
 @pytest.fixture(scope="module")
 def pair():
     cfg = dict(synth.TINY)
-    p = Pair(cfg, seed=3, modes=("resident",), max_tokens=2 * 64)
+    # larger weights than the workload's 0.02 so that the layer's update is of the same size
+    # as its residual input and the comparison below is not dominated by bf16 output rounding
+    p = Pair(cfg, seed=3, modes=("resident",), max_tokens=2 * 64, w_std=0.08)
     yield p
     p.close()
 
@@ -40,9 +42,12 @@ def test_layer_forward_backward(pair, B, S, lora_on):
     lo = {p: pair.olora[(1, p)] for p in PROJ}
     y_o, cache = om.layer_forward(cfg, pair.olayers[1], lo, to64(x), B, S, enabled=lora_on)
     dx_o, g_o = om.layer_backward(cfg, pair.olayers[1], lo, cache, to64(dy), B, S, enabled=lora_on)
-    # compare the layer's update (the residual input dominates the output)
+    # the layer's update y - x and dx - dy (bf16 activations throughout: ~2^-8 relative per
+    # rounding, a few roundings deep)
+    assert rel_err(to64(y), y_o) < 1e-2
     assert rel_err(to64(y) - to64(x), y_o - to64(x)) < 2e-2
-    assert rel_err(to64(dx) - to64(dy), dx_o - to64(dy)) < 2e-2
+    assert rel_err(to64(dx), dx_o) < 1e-2
+    assert rel_err(to64(dx) - to64(dy), dx_o - to64(dy)) < 3e-2
     grads = pair.gpu_grads("resident")
     for p in PROJ:
         gA, gB = grads[(1, p)]
