@@ -178,6 +178,22 @@ soup_status soup_last_logps(soup_model* model, float* pi, float* ref, int n);
  * device; scratch: device f32 [ceil(n/64)] (absmax). */
 soup_status soup_nf4_quantize(const float* w, long long n, uint8_t* codes, int8_t* q8, float* scales, float* mean,
                               float* scratch, void* stream);
+/* Same quantiser, for callers that cannot call cudaMalloc (for example code running where
+ * device allocation is not allowed, or whose device memory is all owned by another allocator)
+ * and so cannot supply the absmax scratch buffer soup_nf4_quantize needs.  The paper has no
+ * counterpart: this is a deployment convenience.  The scratch is a fixed array inside the
+ * library (4 MiB of device memory on every GPU that loads the library, held until the
+ * process exits), so n may be at most SOUP_NF4_STATIC_MAX_ELEMS (= 64 x 2^20 elements, every
+ * 8B-shape projection); larger n returns SOUP_ERR_INVALID_ARG without launching anything.
+ * The call allocates nothing.  The first call on a device looks up the array's device
+ * address with that device current (make that first call before any stream capture).  All
+ * calls share the one array and it keeps the last call's contents; every entry a call reads
+ * is written earlier in the same call, so nothing needs clearing, but calls whose kernels
+ * overlap on the GPU (different streams, or different host threads) race on it: serialise
+ * them.  Outputs and error behaviour are those of soup_nf4_quantize. */
+#define SOUP_NF4_STATIC_MAX_ELEMS (64LL << 20)
+soup_status soup_nf4_quantize_static(const float* w, long long n, uint8_t* codes, int8_t* q8, float* scales,
+                                     float* mean, void* stream);
 /* Standalone NF4 -> bf16 dequantiser: out[i] = bf16_rn(c[code_i] * mhat(block(i))). */
 soup_status soup_nf4_dequantize(const uint8_t* codes, const int8_t* q8, const float* scales, const float* mean,
                                 long long n, uint16_t* out, void* stream);

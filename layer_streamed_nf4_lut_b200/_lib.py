@@ -79,6 +79,7 @@ SIGNATURES = {
     "soup_optimizer_step": [c_void_p, c_float, c_void_p],
     "soup_last_logps": [c_void_p, POINTER(c_float), POINTER(c_float), c_int],
     "soup_nf4_quantize": [c_void_p, c_longlong, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p],
+    "soup_nf4_quantize_static": [c_void_p, c_longlong, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p],
     "soup_nf4_dequantize": [c_void_p, c_void_p, c_void_p, c_void_p, c_longlong, c_void_p, c_void_p],
     "soup_nf4_matmul": [c_void_p, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_void_p,
                         c_void_p, c_void_p],

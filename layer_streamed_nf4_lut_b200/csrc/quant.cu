@@ -10,8 +10,11 @@
 //   w = bf16_rn(fp32(c_q * mhat)).
 // The integer decisions (codes, q8) are taken in float64 on exact inputs, so they are
 // reproducible bit for bit by any implementation of the same definition.
+#include "../../include/soup.h"
 #include "common.cuh"
 #include "internal.h"
+
+#include <mutex>
 
 namespace soup {
 
@@ -156,3 +159,46 @@ cudaError_t nf4_dequant_launch(const uint8_t* codes, const int8_t* q8, const flo
 }
 
 }  // namespace soup
+
+// ---------------------------------------------------------------- allocation-free variant
+// Absmax scratch for soup_nf4_quantize_static: one block of 64 elements per entry, so the
+// 1 Mi entries (4 MiB) cover tensors of up to 64 Mi elements.  Lives for the process.
+namespace soup {
+namespace {
+constexpr long long kStaticBlocks = 1ll << 20;
+static_assert(kStaticBlocks * 64 == SOUP_NF4_STATIC_MAX_ELEMS, "limit in soup.h");
+static __device__ __align__(256) float g_static_absmax[kStaticBlocks];
+
+// Device address of g_static_absmax per device ordinal (host code may not use the symbol's
+// name as a pointer: that is a host-side stand-in, not a device address).
+std::mutex g_static_mu;
+float* g_static_ptr[64] = {};
+
+soup_status static_scratch(float** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return SOUP_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  if (!g_static_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_absmax) != cudaSuccess || !p) return SOUP_ERR_CUDA;
+    g_static_ptr[dev] = static_cast<float*>(p);
+  }
+  *out = g_static_ptr[dev];
+  return SOUP_OK;
+}
+}  // namespace
+}  // namespace soup
+
+const soup::LUT16& soup_codebook_lut();
+
+extern "C" soup_status soup_nf4_quantize_static(const float* w, long long n, uint8_t* codes, int8_t* q8,
+                                                float* scales, float* mean, void* stream) {
+  if (!w || n <= 0 || !codes || !q8 || !scales || !mean) return SOUP_ERR_INVALID_ARG;
+  if (n > SOUP_NF4_STATIC_MAX_ELEMS) return SOUP_ERR_INVALID_ARG;
+  float* scratch = nullptr;
+  const soup_status s = soup::static_scratch(&scratch);
+  if (s != SOUP_OK) return s;
+  const cudaError_t e = soup::nf4_quantize_launch(w, n, codes, q8, scales, mean, scratch, soup_codebook_lut(),
+                                                  static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SOUP_OK : SOUP_ERR_CUDA;
+}

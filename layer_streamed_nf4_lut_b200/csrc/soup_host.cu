@@ -1451,6 +1451,13 @@ soup_status soup_nf4_matmul(const void* x, int M, int N, int K, const uint8_t* c
   return e == cudaSuccess ? SOUP_OK : SOUP_ERR_CUDA;
 }
 
+}  // extern "C"
+
+// The library's NF4 levels for other translation units.
+const soup::LUT16& soup_codebook_lut() { return soup::codebook(); }
+
+extern "C" {
+
 soup_status soup_nf4_codebook(float* out16) {
   if (!out16) return SOUP_ERR_INVALID_ARG;
   std::memcpy(out16, codebook().v, 16 * sizeof(float));
