@@ -164,28 +164,6 @@ def make_batch(wl, seed):
     return ids, mask
 
 
-def h2d_probe(nbytes, device_index, reps=20):
-    """Pinned host -> device bandwidth for layer-sized copies issued back to back (GB/s)."""
-    import torch
-    dev = torch.device("cuda", device_index)
-    hbuf = torch.empty(nbytes, dtype=torch.uint8, pin_memory=True)
-    hbuf.fill_(1)
-    dbuf = torch.empty(nbytes, dtype=torch.uint8, device=dev)
-    s = torch.cuda.Stream(device=dev)
-    with torch.cuda.stream(s):
-        for _ in range(3):
-            dbuf.copy_(hbuf, non_blocking=True)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(s)
-        for _ in range(reps):
-            dbuf.copy_(hbuf, non_blocking=True)
-        e1.record(s)
-    e1.synchronize()
-    ms = e0.elapsed_time(e1)
-    del hbuf, dbuf
-    return reps * nbytes / (ms * 1e-3) / 1e9
-
-
 def run_soup(args, wl, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -211,7 +189,7 @@ def run_soup(args, wl, rank, world, local_rank):
                              gm.lora_grads, lambda: gm.optimizer_step(2e-5))
         return loss
 
-    h2d_gbs = h2d_probe(gm.blob_bytes, local_rank)
+    h2d_gbs = gm.h2d_probe(20)
     for _ in range(args.warmup):
         loss = one_step(ids, mask)
     torch.cuda.synchronize(dev)

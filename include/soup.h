@@ -206,6 +206,11 @@ soup_status soup_nf4_matmul(const void* x, int M, int N, int K, const uint8_t* c
 soup_status soup_nf4_codebook(float* out16);
 
 /* ---- diagnostics ------------------------------------------------------------------------- */
+/* Host-to-device link probe: copies the model's page-locked layer-0 blob into a device layer
+ * buffer `reps` times back to back on the streamer's copy stream (the exact path the streamer
+ * uses) and returns the achieved GB/s (1e9 bytes/s) in *gbs.  Synchronises; the buffer used is
+ * marked empty afterwards, so the next step reloads whatever it needs. */
+soup_status soup_h2d_probe(soup_model* model, int reps, double* gbs);
 soup_status soup_get_stats(soup_model* model, soup_stats* out);
 soup_status soup_reset_stats(soup_model* model);
 /* Live per-kernel profile.  While enabled, every launch a model call makes is bracketed by

@@ -88,6 +88,7 @@ SIGNATURES = {
     "soup_reset_stats": [c_void_p],
     "soup_check_device": [c_void_p, c_void_p],
     "soup_set_profiling": [c_void_p, c_int],
+    "soup_h2d_probe": [c_void_p, c_int, POINTER(ctypes.c_double)],
     "soup_get_profile": [c_void_p, POINTER(ProfileEntry), c_int, POINTER(c_int), c_int],
 }
 STRING_FUNCS = {"soup_status_string": [c_int32], "soup_last_error": [c_void_p]}

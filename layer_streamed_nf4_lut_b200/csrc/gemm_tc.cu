@@ -27,6 +27,7 @@
 
 #include <algorithm>
 #include <atomic>
+#include <cstdlib>
 #include <mutex>
 
 namespace soup {
@@ -43,8 +44,12 @@ template <int BN>
 struct GemmCfg {
   static constexpr int A_BYTES = BM * 128;
   static constexpr int B_BYTES = BN * 128;
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES = (BN >= 256) ? 4 : (BN >= 128 ? 6 : 8);
+  // raw NF4 staging (TMA): codes BN x 32 B (forward) or 64 x BN/2 B (transposed), q8 absmax
+  // BN x 16 B or 64 x 16 B
+  static constexpr int RAW_CODE_BYTES = BN * 32;
+  static constexpr int RAW_Q8_BYTES = (BN > 64 ? BN : 64) * 16;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + RAW_CODE_BYTES + RAW_Q8_BYTES;
+  static constexpr int STAGES = (BN >= 256) ? 3 : (BN >= 128 ? 5 : 7);
   static constexpr int CTRL_BYTES = 512;
   static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + CTRL_BYTES;
 };
@@ -113,12 +118,26 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t saddr) {
   return d;
 }
 
-// Instruction descriptor, kind::f16: bf16 x bf16 -> f32, both operands K-major, M = 128.
+// Shared-memory matrix descriptor: MN-major, 128-byte swizzle.  Atoms of 8 K-rows x 64 MN
+// elements (1024 B); the next 8 K-rows are 1024 B further (stride byte offset), the next 64
+// MN elements 8192 B further (leading byte offset: one atom column of a 64-deep K block).
+__device__ __forceinline__ uint64_t sw128_mnmajor_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>(8192 >> 4) << 16;  // leading byte offset: next 64 MN elements
+  d |= static_cast<uint64_t>(1024 >> 4) << 32;  // stride byte offset: next 8 K rows
+  d |= static_cast<uint64_t>(1) << 46;
+  d |= static_cast<uint64_t>(2) << 61;
+  return d;
+}
+
+// Instruction descriptor, kind::f16: bf16 x bf16 -> f32, A K-major, B K- or MN-major, M = 128.
 template <int BN>
-__device__ __forceinline__ uint32_t idesc_bf16_f32() {
+__device__ __forceinline__ uint32_t idesc_bf16_f32(bool b_mn_major) {
   return (1u << 4)                                 // D format f32
          | (1u << 7)                               // A format bf16
          | (1u << 10)                              // B format bf16
+         | ((b_mn_major ? 1u : 0u) << 16)          // B major-ness
          | (static_cast<uint32_t>(BN >> 3) << 17)  // N / 8
          | (static_cast<uint32_t>(BM >> 4) << 24); // M / 16
 }
@@ -277,6 +296,64 @@ __device__ __forceinline__ void load_tile(const Operand& op, const NF4Group& g, 
   }
 }
 
+// Dequantise the forward (W[n, k]) B tile from TMA-staged raw codes / q8 absmax.
+// raw_codes: [BN][32] bytes (row n, k0..k0+63); raw_q8: [BN][16] bytes covering k-blocks
+// [16*floor(kbw/16), +16) of each row; the tile lies inside NF4 tensor `s`.
+template <int BN>
+__device__ __forceinline__ void decode_fwd_raw(const NF4Group& g, int s, const float* lut, const float* seg_mean,
+                                               int n0, int N, int kbw, const uint8_t* raw_codes,
+                                               const uint8_t* raw_q8, uint8_t* tile, int gtid) {
+  const NF4Seg& sg = g.seg[s];
+  const long long cpr = g.cols >> 6;  // absmax blocks per row
+  const float mean = seg_mean[s];
+#pragma unroll 4
+  for (int c = gtid; c < BN * 8; c += GROUP_THREADS) {
+    const int r = c >> 3, kc = c & 7;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (n0 + r < N) {
+      NF4Raw raw;
+      raw.code = *reinterpret_cast<const uint32_t*>(raw_codes + r * 32 + kc * 4);
+      raw.q8 = static_cast<int8_t>(raw_q8[r * 16 + (kbw & 15)]);
+      const long long blk = static_cast<long long>(n0 + r - sg.row_begin) * cpr + kbw;
+      raw.s2 = __ldg(sg.scales + (blk >> 8));
+      raw.seg = s;
+      (void)mean;
+      v = nf4_decode(raw, lut, seg_mean);
+    }
+    *reinterpret_cast<uint4*>(tile + swz_off(r, kc)) = v;
+  }
+}
+
+// Dequantise the transposed (dX) B tile: B[n, k] = W[k0 + k, n0 + n] from raw codes
+// [64][BN/2] bytes and raw q8 [64][16] bytes (absmax blocks [xq, xq+16) of each W row), into
+// the MN-major 128-byte-swizzled layout (8 consecutive n of one k = one 16-byte store).
+template <int BN>
+__device__ __forceinline__ void decode_dx_raw(const NF4Group& g, int s, const float* lut, const float* seg_mean,
+                                              int n0, int N, int k0, int xq, const uint8_t* raw_codes,
+                                              const uint8_t* raw_q8, uint8_t* tile, int gtid) {
+  const NF4Seg& sg = g.seg[s];
+  const long long cpr = g.cols >> 6;
+  constexpr int NC = BN / 8;
+#pragma unroll 4
+  for (int u = gtid; u < 64 * NC; u += GROUP_THREADS) {
+    const int nc = u % NC, kr = u / NC;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    const int n = n0 + nc * 8;
+    if (n < N) {
+      NF4Raw raw;
+      raw.code = *reinterpret_cast<const uint32_t*>(raw_codes + kr * (BN / 2) + nc * 4);
+      const int bcol = n >> 6;
+      raw.q8 = static_cast<int8_t>(raw_q8[kr * 16 + (bcol - xq)]);
+      const long long blk = static_cast<long long>(k0 + kr - sg.row_begin) * cpr + bcol;
+      raw.s2 = __ldg(sg.scales + (blk >> 8));
+      raw.seg = s;
+      v = nf4_decode(raw, lut, seg_mean);
+    }
+    const int off = (nc >> 3) * 8192 + (kr >> 3) * 1024 + (kr & 7) * 128 + (((nc & 7) ^ (kr & 7)) << 4);
+    *reinterpret_cast<uint4*>(tile + off) = v;
+  }
+}
+
 __device__ __forceinline__ bool seg_active(const GemmSeg& s, int n0, int bn) {
   if (s.K <= 0) return false;
   return s.B.row_lo < n0 + bn && s.B.row_hi > n0;
@@ -347,7 +424,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
   uint8_t* ctrl = base + C::STAGES * C::STAGE_BYTES;
   uint64_t* full = reinterpret_cast<uint64_t*>(ctrl);
   uint64_t* empty = full + C::STAGES;
-  uint64_t* done = empty + C::STAGES;
+  uint64_t* raw_full = empty + C::STAGES;
+  uint64_t* done = raw_full + C::STAGES;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* seg_mean = reinterpret_cast<float*>(tmem_slot + 4);
@@ -358,8 +436,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(&full[s], GROUP_THREADS / 32 + 1);  // 4 producer warps + the TMA / leader arrival
+      mbar_init(&full[s], GROUP_THREADS / 32 + 1);  // 4 producer warps + the TMA issuer
       mbar_init(&empty[s], 1);
+      mbar_init(&raw_full[s], 1);
     }
     mbar_init(done, 1);
     *abort_flag = 0;
@@ -392,47 +471,107 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
       const GemmSeg& sg = p.seg[s];
       if (!seg_active(sg, n0, BN)) continue;
       const int nk = (sg.K + BK - 1) / BK;
+      const bool raw = (s == 0) && p.raw_tma;
       for (int kk = 0; kk < nk; ++kk, ++g) {
         if (g < kb_lo || g >= kb_hi) continue;
         const int kb = g - kb_lo;
         if ((kb % GROUPS) != grp) continue;
         const int st = kb % C::STAGES;
         const uint32_t ph = static_cast<uint32_t>(kb / C::STAGES) & 1u;
-        mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, p.err);
         uint8_t* As = base + st * C::STAGE_BYTES;
         uint8_t* Bs = As + C::A_BYTES;
-        if (gtid == 0) {
-          if (p.a_tma[s]) {
-            mbar_arrive_expect_tx(&full[st], C::A_BYTES);
-            tma_load_2d(As, &p.tmapA[s], kk * BK, m0, &full[st]);
+        const uint8_t* Rc = Bs + C::B_BYTES;
+        const uint8_t* Rq = Rc + C::RAW_CODE_BYTES;
+        if (raw) {
+          // raw codes / absmax of this k-block have landed (the issuer waited for the slot)
+          mbar_wait_bounded(&raw_full[st], ph, abort_flag, p.err);
+          if (sg.B.kind == OP_NF4_K) {
+            decode_fwd_raw<BN>(p.nf4, nf4_seg_of(p.nf4, n0), lut, seg_mean, n0, p.N, kk, Rc, Rq, Bs, gtid);
           } else {
-            mbar_arrive(&full[st]);
+            const int k0 = kk * BK;
+            decode_dx_raw<BN>(p.nf4, nf4_seg_of(p.nf4, k0), lut, seg_mean, n0, p.N, k0, ((n0 >> 6) >> 4) << 4, Rc,
+                              Rq, Bs, gtid);
           }
+        } else {
+          mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, p.err);
+          load_tile<BN>(sg.B, p.nf4, lut, seg_mean, sg.K, n0, p.N, kk * BK, Bs, gtid);
         }
         if (!p.a_tma[s]) load_tile<BM>(sg.A, p.nf4, lut, seg_mean, sg.K, m0, p.M, kk * BK, As, gtid);
-        load_tile<BN>(sg.B, p.nf4, lut, seg_mean, sg.K, n0, p.N, kk * BK, Bs, gtid);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&full[st]);
       }
     }
   } else {
+    if (warp == 9 && lane == 0) {
+      // ------------------------------------------------ TMA issuer: A tiles and raw NF4 codes / absmax
+      int g = 0;
+      for (int s = 0; s < p.nseg; ++s) {
+        const GemmSeg& sg = p.seg[s];
+        if (!seg_active(sg, n0, BN)) continue;
+        const int nk = (sg.K + BK - 1) / BK;
+        const bool raw = (s == 0) && p.raw_tma;
+        for (int kk = 0; kk < nk; ++kk, ++g) {
+          if (g < kb_lo || g >= kb_hi) continue;
+          const int kb = g - kb_lo;
+          const int st = kb % C::STAGES;
+          const uint32_t ph = static_cast<uint32_t>(kb / C::STAGES) & 1u;
+          mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, p.err);
+          uint8_t* As = base + st * C::STAGE_BYTES;
+          uint8_t* Rc = As + C::A_BYTES + C::B_BYTES;
+          uint8_t* Rq = Rc + C::RAW_CODE_BYTES;
+          if (p.a_tma[s]) {
+            mbar_arrive_expect_tx(&full[st], C::A_BYTES);
+            tma_load_2d(As, &p.tmapA[s], kk * BK, m0, &full[st]);
+          } else {
+            mbar_arrive(&full[st]);
+          }
+          if (raw) {
+            if (sg.B.kind == OP_NF4_K) {
+              const int si = nf4_seg_of(p.nf4, n0);
+              const int y = n0 - p.nf4.seg[si].row_begin;
+              mbar_arrive_expect_tx(&raw_full[st], BN * 32 + BN * 16);
+              tma_load_2d(Rc, &p.tmapCodes[si], kk * (BK / 2), y, &raw_full[st]);
+              tma_load_2d(Rq, &p.tmapQ8[si], (kk >> 4) << 4, y, &raw_full[st]);
+            } else {
+              const int k0 = kk * BK;
+              const int si = nf4_seg_of(p.nf4, k0);
+              const int y = k0 - p.nf4.seg[si].row_begin;
+              mbar_arrive_expect_tx(&raw_full[st], 64 * (BN / 2) + 64 * 16);
+              tma_load_2d(Rc, &p.tmapCodes[si], n0 / 2, y, &raw_full[st]);
+              tma_load_2d(Rq, &p.tmapQ8[si], ((n0 >> 6) >> 4) << 4, y, &raw_full[st]);
+            }
+          } else {
+            mbar_arrive(&raw_full[st]);  // keeps the stage's raw phase in step
+          }
+        }
+      }
+    }
     if (warp == 8 && lane == 0) {
       // ------------------------------------------------ MMA issuer
-      const uint32_t idesc = idesc_bf16_f32<BN>();
-      for (int kb = 0; kb < kb_hi - kb_lo; ++kb) {
-        const int st = kb % C::STAGES;
-        const uint32_t ph = static_cast<uint32_t>(kb / C::STAGES) & 1u;
-        mbar_wait_bounded(&full[st], ph, abort_flag, p.err);
-        tc_fence_after();
-        const uint32_t a_addr = smem_u32(base + st * C::STAGE_BYTES);
-        const uint32_t b_addr = a_addr + C::A_BYTES;
+      int g = 0, kb = 0;
+      for (int s = 0; s < p.nseg; ++s) {
+        const GemmSeg& sg = p.seg[s];
+        if (!seg_active(sg, n0, BN)) continue;
+        const int nk = (sg.K + BK - 1) / BK;
+        const bool b_mn = (s == 0) && p.raw_tma && sg.B.kind == OP_NF4_MN;
+        const uint32_t idesc = idesc_bf16_f32<BN>(b_mn);
+        for (int kk = 0; kk < nk; ++kk, ++g) {
+          if (g < kb_lo || g >= kb_hi) continue;
+          const int st = kb % C::STAGES;
+          const uint32_t ph = static_cast<uint32_t>(kb / C::STAGES) & 1u;
+          mbar_wait_bounded(&full[st], ph, abort_flag, p.err);
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(base + st * C::STAGE_BYTES);
+          const uint32_t b_addr = a_addr + C::A_BYTES;
 #pragma unroll
-        for (int j = 0; j < BK / 16; ++j) {
-          tc_mma_f16(tmem, sw128_kmajor_desc(a_addr + j * 32), sw128_kmajor_desc(b_addr + j * 32), idesc,
-                     (kb > 0 || j > 0) ? 1u : 0u);
+          for (int j = 0; j < BK / 16; ++j) {
+            const uint64_t bd = b_mn ? sw128_mnmajor_desc(b_addr + j * 2048) : sw128_kmajor_desc(b_addr + j * 32);
+            tc_mma_f16(tmem, sw128_kmajor_desc(a_addr + j * 32), bd, idesc, (kb > 0 || j > 0) ? 1u : 0u);
+          }
+          tc_commit(&empty[st]);
+          ++kb;
         }
-        tc_commit(&empty[st]);
       }
       tc_commit(done);
     }
@@ -523,6 +662,57 @@ bool encode_kmajor_bf16(CUtensorMap* map, const void* ptr, int K, int M, long lo
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// TMA descriptor for a 2D uint8 array (raw NF4 codes or q8 absmax), no swizzle, zero fill.
+bool encode_u8_2d(CUtensorMap* map, const void* ptr, unsigned long long w, unsigned long long h,
+                  unsigned long long stride, unsigned box_w, unsigned box_h) {
+  auto fn = tensor_map_encoder();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {w, h};
+  cuuint64_t strides[1] = {stride};
+  cuuint32_t box[2] = {box_w, box_h};
+  cuuint32_t es[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Raw TMA staging of the NF4 operand: rows of 1024-column multiples (so the q8 absmax rows are
+// 16-byte multiples) and tiles that never straddle two stacked tensors.
+bool raw_tma_allowed() {
+  static const bool allowed = [] {
+    const char* e = std::getenv("SOUP_GEMM_RAW_TMA");
+    return !(e && e[0] == '0');
+  }();
+  return allowed;
+}
+
+bool setup_raw_tma(GemmParams& p, int BN) {
+  if (!raw_tma_allowed()) return false;
+  const GemmSeg& s0 = p.seg[0];
+  if (s0.K <= 0 || (s0.B.kind != OP_NF4_K && s0.B.kind != OP_NF4_MN)) return false;
+  const NF4Group& g = p.nf4;
+  if (g.cols % 1024 != 0 || g.nseg < 1) return false;
+  if (s0.B.kind == OP_NF4_K) {
+    for (int i = 1; i < g.nseg; ++i)
+      if (g.seg[i].row_begin % BN != 0) return false;
+  } else {
+    if (p.N != g.cols) return false;
+    for (int i = 1; i < g.nseg; ++i)
+      if (g.seg[i].row_begin % 64 != 0) return false;
+  }
+  const unsigned long long cb = static_cast<unsigned long long>(g.cols) / 2, qb = static_cast<unsigned long long>(g.cols) / 64;
+  for (int i = 0; i < g.nseg; ++i) {
+    const unsigned long long rows = static_cast<unsigned long long>(g.seg[i].rows);
+    const bool ok = (s0.B.kind == OP_NF4_K)
+                        ? (encode_u8_2d(&p.tmapCodes[i], g.seg[i].codes, cb, rows, cb, 32, BN) &&
+                           encode_u8_2d(&p.tmapQ8[i], g.seg[i].q8, qb, rows, qb, 16, BN))
+                        : (encode_u8_2d(&p.tmapCodes[i], g.seg[i].codes, cb, rows, cb, BN / 2, 64) &&
+                           encode_u8_2d(&p.tmapQ8[i], g.seg[i].q8, qb, rows, qb, 16, 64));
+    if (!ok) return false;
+  }
+  return true;
+}
+
 template <int BN>
 cudaError_t launch_bn(const GemmParams& p, cudaStream_t st) {
   using C = GemmCfg<BN>;
@@ -593,6 +783,8 @@ cudaError_t gemm_launch(const GemmParams& p_in, cudaStream_t st) {
     nkb += (sg.K + BK - 1) / BK;
   }
   const int BN = (p.N <= 64) ? 64 : ((p.N <= 128 || static_cast<long long>((p.N + 255) / 256) * ((p.M + 127) / 128) < 148) ? 128 : 256);
+  p.bn = BN;
+  p.raw_tma = setup_raw_tma(p, BN) ? 1 : 0;
   // split-K for grids that cannot fill the GPU (skinny LoRA GEMMs, long reductions)
   p.splits = 1;
   const long long tiles = static_cast<long long>((p.N + BN - 1) / BN) * ((p.M + BM - 1) / BM);

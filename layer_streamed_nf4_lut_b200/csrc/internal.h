@@ -56,7 +56,11 @@ constexpr int GEMM_MAX_SEG = 5;
 
 struct GemmParams {
   CUtensorMap tmapA[GEMM_MAX_SEG];  // TMA descriptors of K-major bf16 A operands (filled by gemm_launch)
+  CUtensorMap tmapCodes[3];         // TMA descriptors of each NF4 tensor's packed codes (raw staging)
+  CUtensorMap tmapQ8[3];            // ... and of its q8 absmax
   int a_tma[GEMM_MAX_SEG];          // 1: segment's A tile arrives by TMA
+  int raw_tma;                      // 1: the NF4 segment's codes / absmax arrive by TMA (filled by gemm_launch)
+  int bn;                           // output tile width chosen by gemm_launch
   int M, N;
   int nseg;
   GemmSeg seg[GEMM_MAX_SEG];

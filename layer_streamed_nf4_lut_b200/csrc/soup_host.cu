@@ -1510,6 +1510,35 @@ soup_status soup_get_profile(soup_model* m, soup_profile_entry* out, int max_ent
   })
 }
 
+soup_status soup_h2d_probe(soup_model* m, int reps, double* gbs) {
+  if (!m || !gbs || reps < 1) return SOUP_ERR_INVALID_ARG;
+  if (!m->host_loaded[0]) return SOUP_ERR_STATE;
+  SOUP_GUARD({
+    const int b = 0;
+    SOUP_CK(cudaStreamWaitEvent(m->copy_stream, m->buf_free[b], 0));
+    cudaEvent_t e0 = nullptr;
+    cudaEvent_t e1 = nullptr;
+    SOUP_CK(cudaEventCreate(&e0));
+    SOUP_CK(cudaEventCreate(&e1));
+    SOUP_CK(cudaMemcpyAsync(m->dev_buf[b], m->host_blob[0], m->layout.total, cudaMemcpyHostToDevice, m->copy_stream));
+    SOUP_CK(cudaEventRecord(e0, m->copy_stream));
+    for (int i = 0; i < reps; ++i)
+      SOUP_CK(cudaMemcpyAsync(m->dev_buf[b], m->host_blob[0], m->layout.total, cudaMemcpyHostToDevice,
+                              m->copy_stream));
+    SOUP_CK(cudaEventRecord(e1, m->copy_stream));
+    SOUP_CK(cudaEventRecord(m->copy_done[b], m->copy_stream));
+    soup_status st = wait_stream(m, m->copy_stream);
+    float ms = 0.f;
+    if (st == SOUP_OK) SOUP_CK(cudaEventElapsedTime(&ms, e0, e1));
+    cudaEventDestroy(e0);
+    cudaEventDestroy(e1);
+    if (st != SOUP_OK) return st;
+    if (m->cfg.mode == SOUP_STREAMED) m->buf_layer[b] = -1;
+    *gbs = static_cast<double>(reps) * m->layout.total / (ms * 1e-3) / 1e9;
+    return SOUP_OK;
+  })
+}
+
 soup_status soup_check_device(soup_model* m, void* stream) {
   if (!m) return SOUP_ERR_INVALID_ARG;
   SOUP_GUARD(return read_scalars(m, static_cast<cudaStream_t>(stream), nullptr);)

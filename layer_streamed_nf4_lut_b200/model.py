@@ -211,6 +211,12 @@ class SoupModel:
         self._ck(lib.soup_get_stats(self.h, byref(s)))
         return {k: getattr(s, k) for k, _ in Stats._fields_}
 
+    def h2d_probe(self, reps: int = 20) -> float:
+        """GB/s of back-to-back layer copies on the streamer's own copy path."""
+        out = ctypes.c_double()
+        self._ck(lib.soup_h2d_probe(self.h, int(reps), byref(out)))
+        return out.value
+
     def set_profiling(self, enabled: bool):
         self._ck(lib.soup_set_profiling(self.h, 1 if enabled else 0))
 

@@ -1,0 +1,116 @@
+"""Full-size checks at the 8B shape in the bench's launch configuration (hidden 4096, 32/8
+heads, intermediate 14336, vocab 128256, 512 tokens, streamed with 2 layer buffers):
+
+* one decoder layer + the full-vocabulary head, SFT step against the float64 oracle (the
+  oracle quantises the same float32 weights itself);
+* the 32-layer model: streamed and resident steps bitwise equal, layer-load counts 2L-2
+  (cold) and 2L-4 (steady state).
+
+The weights are drawn on the GPU with torch's seeded generator (synth.normal_device): drawing
+218M values per layer on the host would take minutes.  They are inputs, copied to the host for
+the oracle; no oracle input comes from libsoup."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import model as om
+from oracle import nf4
+from tests.gpu_util import bf16_tensor, cosine
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+
+PROJ = synth.PROJ_NAMES
+
+
+def _device_layer(cfg, seed, layer):
+    return {p: synth.normal_device(synth.proj_shape(cfg, p), seed * 1009 + 16 * layer + j, 0.02)
+            for j, p in enumerate(PROJ)}
+
+
+def _bits(t: torch.Tensor) -> np.ndarray:
+    return t.view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def _lora_flat(cfg, lora):
+    from layer_streamed_nf4_lut_b200.model import lora_numel, lora_offset
+    flat = np.zeros(lora_numel(cfg), np.float32)
+    for (layer, p), (A, B) in lora.items():
+        j = PROJ.index(p)
+        oa, _, _ = lora_offset(cfg, layer, j, 0)
+        ob, _, _ = lora_offset(cfg, layer, j, 1)
+        flat[oa:oa + A.size] = A.ravel()
+        flat[ob:ob + B.size] = B.ravel()
+    return torch.from_numpy(flat).cuda()
+
+
+def test_full_width_layer_and_head_step_vs_oracle():
+    from layer_streamed_nf4_lut_b200.model import SoupModel
+    cfg = dict(synth.L8B, n_layers=1)
+    B, S = 1, 512
+    w = _device_layer(cfg, 5, 0)
+    g_attn = (1.0 + 0.1 * synth.normal_device((cfg["hidden"],), 77, 1.0)).to(torch.bfloat16)
+    g_mlp = (1.0 + 0.1 * synth.normal_device((cfg["hidden"],), 78, 1.0)).to(torch.bfloat16)
+    emb = synth.normal_device((cfg["vocab"], cfg["hidden"]), 79, 0.02).to(torch.bfloat16)
+    lm = synth.normal_device((cfg["vocab"], cfg["hidden"]), 80, 0.02).to(torch.bfloat16)
+    g_fin = (1.0 + 0.1 * synth.normal_device((cfg["hidden"],), 81, 1.0)).to(torch.bfloat16)
+    lora = synth.lora_weights(cfg, 6)
+    gm = SoupModel(cfg, mode="streamed", n_layer_buffers=2, max_tokens=B * S)
+    try:
+        gm.quantize_layer(0, w, g_attn, g_mlp)
+        gm.set_head(emb, g_fin, lm)
+        gm.set_lora(_lora_flat(cfg, lora))
+        ids = synth.token_ids_uniform(9, 1, B * S, cfg["vocab"]).reshape(B, S)
+        loss = gm.step(torch.from_numpy(ids).cuda(), apply_optimizer=False)
+        grads = {p: (gm.lora_view(gm.lora_grads, 0, p, 0).double().cpu().numpy(),
+                     gm.lora_view(gm.lora_grads, 0, p, 1).double().cpu().numpy()) for p in PROJ}
+        # oracle: its own quantisation of the same float32 weights
+        q = {p: nf4.quantise(w[p].cpu().numpy()) for p in PROJ}
+        q["attn_norm"], q["mlp_norm"] = _bits(g_attn), _bits(g_mlp)
+        del w
+        layers, head = om.model_from_quantised(cfg, [q], (_bits(emb), _bits(lm), _bits(g_fin)))
+        olora = {k: (a.astype(np.float64), b.astype(np.float64)) for k, (a, b) in lora.items()}
+        ol, og, _ = om.sft_step(cfg, layers, olora, head, ids)
+        assert abs(loss - ol) <= 1e-2 * abs(ol), (loss, ol)
+        for p in PROJ:
+            assert cosine(grads[p][0], og[(0, p)][0]) > 0.999, p
+            assert cosine(grads[p][1], og[(0, p)][1]) > 0.999, p
+    finally:
+        gm.close()
+
+
+def test_full_8b_streamed_equals_resident_and_load_counts():
+    from layer_streamed_nf4_lut_b200.model import SoupModel
+    cfg = dict(synth.L8B)
+    L, B, S = cfg["n_layers"], 1, 512
+    models = {m: SoupModel(cfg, mode=m, n_layer_buffers=2, max_tokens=B * S) for m in ("streamed", "resident")}
+    try:
+        ones = torch.ones(cfg["hidden"], dtype=torch.bfloat16, device="cuda")
+        for i in range(L):
+            w = _device_layer(cfg, 11, i)
+            for m in models.values():
+                m.quantize_layer(i, w, ones, ones)
+            del w
+        emb = synth.normal_device((cfg["vocab"], cfg["hidden"]), 12, 0.02).to(torch.bfloat16)
+        lm = synth.normal_device((cfg["vocab"], cfg["hidden"]), 13, 0.02).to(torch.bfloat16)
+        lora = _lora_flat(cfg, synth.lora_weights(cfg, 14))
+        for m in models.values():
+            m.set_head(emb, ones, lm)
+            m.set_lora(lora.clone())
+        ids = torch.from_numpy(synth.token_ids_uniform(15, 1, B * S, cfg["vocab"]).reshape(B, S)).cuda()
+        st = models["streamed"]
+        st.reset_stats()
+        l_s = st.step(ids, apply_optimizer=False)
+        cold = st.stats()["layer_loads"]
+        l_r = models["resident"].step(ids, apply_optimizer=False)
+        assert math.isfinite(l_s) and l_s == l_r
+        assert torch.equal(st.lora_grads.view(torch.int32), models["resident"].lora_grads.view(torch.int32))
+        assert cold == 2 * L - 2
+        st.reset_stats()
+        st.step(ids, apply_optimizer=False)
+        assert st.stats()["layer_loads"] == 2 * L - 4
+    finally:
+        for m in models.values():
+            m.close()
