@@ -141,6 +141,11 @@ soup_status soup_lora_numel(const soup_model_config* cfg, size_t* numel);
 soup_status soup_lora_offset(const soup_model_config* cfg, int layer, int proj, int which_b, size_t* offset,
                              int* rows, int* cols);
 soup_status soup_model_set_lora(soup_model* model, float* params, float* grads, float* adam_m, float* adam_v);
+/* The kernels read the LoRA parameters through a bf16 copy kept by the library (the values
+ * the fp32 parameters round to), refreshed by soup_model_set_lora (synchronous) and by every
+ * optimizer update the library performs.  A caller that changes the fp32 parameters itself
+ * calls soup_model_refresh_lora (enqueued on `stream`) before the next forward. */
+soup_status soup_model_refresh_lora(soup_model* model, void* stream);
 
 /* LoRA on/off for the forward and backward calls that follow.  Off: the LoRA branch and its
  * gradients are skipped entirely (not multiplied by zero), which is the DPO reference model. */

@@ -73,6 +73,7 @@ SIGNATURES = {
     "soup_lora_offset": [POINTER(ModelConfig), c_int, c_int, c_int, POINTER(c_size_t), POINTER(c_int), POINTER(c_int)],
     "soup_model_set_lora": [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p],
     "soup_set_lora_enabled": [c_void_p, c_int],
+    "soup_model_refresh_lora": [c_void_p, c_void_p],
     "soup_layer_fwd": [c_void_p, c_int, c_void_p, c_void_p, c_int, c_int, c_void_p],
     "soup_layer_bwd": [c_void_p, c_int, c_void_p, c_void_p, c_int, c_int, c_void_p],
     "soup_step": [c_void_p, c_int, POINTER(Batch), POINTER(c_float), c_void_p],

@@ -102,26 +102,34 @@ __global__ void rmsnorm_bwd_kernel(const uint16_t* __restrict__ dy, const uint16
 }
 
 // ---------------------------------------------------------------- RoPE (rotate-half, in place)
-// angle = pos * theta^(-2i/d), pos = t mod S. inverse != 0 rotates by -angle (the backward).
-__global__ void rope_kernel(uint16_t* __restrict__ qkv, long long ld, int S, int nheads, int d, double log_theta,
-                            int inverse) {
+// (z_i, z_{i+d/2}) -> (z_i cos - z_{i+d/2} sin, z_{i+d/2} cos + z_i sin) with the angle
+// pos * theta^(-2i/d), pos = t mod S, read from a [S_max, d/2] cos/sin table; inverse != 0
+// rotates by -angle (the backward).  One thread per 8 consecutive i of one head.
+__global__ void rope_kernel(uint16_t* __restrict__ qkv, long long ld, int S, int nheads, int d,
+                            const float* __restrict__ tcos, const float* __restrict__ tsin, int inverse) {
   const int t = blockIdx.x;
-  const int half = d / 2;
-  const double pos = static_cast<double>(t % S);
+  const int half = d / 2, g8 = half / 8;
+  const int pos = t % S;
   uint16_t* row = qkv + static_cast<long long>(t) * ld;
-  for (int idx = threadIdx.x; idx < nheads * half; idx += blockDim.x) {
-    const int hh = idx / half, i = idx % half;
-    const double ang = pos * exp(-log_theta * (2.0 * i) / d);
-    double sd, cd;
-    sincos(ang, &sd, &cd);
-    const float s = inverse ? -static_cast<float>(sd) : static_cast<float>(sd);
-    const float c = static_cast<float>(cd);
+  for (int idx = threadIdx.x; idx < nheads * g8; idx += blockDim.x) {
+    const int hh = idx / g8, i0 = (idx % g8) * 8;
     uint16_t* z = row + hh * d;
-    const float z1 = bf16_to_f32(z[i]), z2 = bf16_to_f32(z[i + half]);
-    const __nv_bfloat16 o1 = __float2bfloat16_rn(z1 * c - z2 * s);
-    const __nv_bfloat16 o2 = __float2bfloat16_rn(z2 * c + z1 * s);
-    z[i] = *reinterpret_cast<const uint16_t*>(&o1);
-    z[i + half] = *reinterpret_cast<const uint16_t*>(&o2);
+    float a[8], b[8], o1[8], o2[8];
+    load8(z + i0, a);
+    load8(z + half + i0, b);
+    const float4* cp = reinterpret_cast<const float4*>(tcos + static_cast<long long>(pos) * half + i0);
+    const float4* sp = reinterpret_cast<const float4*>(tsin + static_cast<long long>(pos) * half + i0);
+    const float4 c0 = cp[0], c1 = cp[1], s0 = sp[0], s1 = sp[1];
+    const float c[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+    float sn[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float sj = inverse ? -sn[j] : sn[j];
+      o1[j] = a[j] * c[j] - b[j] * sj;
+      o2[j] = b[j] * c[j] + a[j] * sj;
+    }
+    store8(z + i0, o1);
+    store8(z + half + i0, o2);
   }
 }
 
@@ -312,8 +320,8 @@ __global__ void ce_grad_kernel(const float* __restrict__ logits, const float* __
 
 // ---------------------------------------------------------------- AdamW (fp32, bias-corrected)
 __global__ void adamw_kernel(float* __restrict__ p, const float* __restrict__ g, float* __restrict__ m,
-                             float* __restrict__ v, long long n, float lr, float b1, float b2, float eps, float wd,
-                             float bc1, float bc2) {
+                             float* __restrict__ v, uint16_t* __restrict__ pb, long long n, float lr, float b1, float b2,
+                             float eps, float wd, float bc1, float bc2) {
   const long long i4 = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i4 * 4 >= n) return;
   if (i4 * 4 + 4 <= n) {
@@ -335,13 +343,26 @@ __global__ void adamw_kernel(float* __restrict__ p, const float* __restrict__ g,
     reinterpret_cast<float4*>(p)[i4] = pp;
     reinterpret_cast<float4*>(m)[i4] = mm;
     reinterpret_cast<float4*>(v)[i4] = vv;
+    if (pb) reinterpret_cast<uint2*>(pb)[i4] = make_uint2(pack_bf16x2(P[0], P[1]), pack_bf16x2(P[2], P[3]));
   } else {
     for (long long i = i4 * 4; i < n; ++i) {
       m[i] = b1 * m[i] + (1.f - b1) * g[i];
       v[i] = b2 * v[i] + (1.f - b2) * g[i] * g[i];
       const float mh = m[i] * bc1, vh = v[i] * bc2;
       p[i] = p[i] - lr * (mh / (sqrtf(vh) + eps) + wd * p[i]);
+      if (pb) {
+        const __nv_bfloat16 b = __float2bfloat16_rn(p[i]);
+        pb[i] = *reinterpret_cast<const uint16_t*>(&b);
+      }
     }
+  }
+}
+
+__global__ void f32_to_bf16_kernel(const float* __restrict__ x, uint16_t* __restrict__ y, long long n) {
+  const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i < n) {
+    const __nv_bfloat16 b = __float2bfloat16_rn(x[i]);
+    y[i] = *reinterpret_cast<const uint16_t*>(&b);
   }
 }
 
@@ -378,14 +399,14 @@ cudaError_t rmsnorm_bwd_launch(const uint16_t* dy, const uint16_t* x, const floa
   return cudaGetLastError();
 }
 
-cudaError_t rope_launch(uint16_t* qkv, long long ld, int B, int S, int hq, int hkv, int d, float theta, int inverse,
-                        cudaStream_t st) {
+cudaError_t rope_launch(uint16_t* qkv, long long ld, int B, int S, int hq, int hkv, int d, const float* tcos,
+                        const float* tsin, int inverse, cudaStream_t st) {
   const int T = B * S;
   if (T <= 0) return cudaSuccess;
   const int nheads = hq + hkv;  // q heads then k heads, contiguous from column 0
-  int thr = nheads * d / 2;
+  int thr = nheads * d / 16;
   thr = thr > 256 ? 256 : ((thr + 31) / 32) * 32;
-  rope_kernel<<<T, thr, 0, st>>>(qkv, ld, S, nheads, d, log(static_cast<double>(theta)), inverse);
+  rope_kernel<<<T, thr, 0, st>>>(qkv, ld, S, nheads, d, tcos, tsin, inverse);
   ++g_kernel_launches;
   return cudaGetLastError();
 }
@@ -451,13 +472,21 @@ cudaError_t ce_grad_launch(const float* logits, const float* lse, const int32_t*
   return cudaGetLastError();
 }
 
-cudaError_t adamw_launch(float* p, const float* g, float* m, float* v, long long n, float lr, float b1, float b2,
-                         float eps, float wd, int t, cudaStream_t st) {
+cudaError_t f32_to_bf16_launch(const float* x, uint16_t* y, long long n, cudaStream_t st) {
+  if (n <= 0) return cudaSuccess;
+  f32_to_bf16_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(x, y, n);
+  ++g_kernel_launches;
+  return cudaGetLastError();
+}
+
+cudaError_t adamw_launch(float* p, const float* g, float* m, float* v, uint16_t* pb, long long n, float lr, float b1,
+                         float b2, float eps, float wd, int t, cudaStream_t st) {
   if (n <= 0) return cudaSuccess;
   const float bc1 = static_cast<float>(1.0 / (1.0 - pow(static_cast<double>(b1), t)));
   const float bc2 = static_cast<float>(1.0 / (1.0 - pow(static_cast<double>(b2), t)));
   const long long n4 = (n + 3) / 4;
-  adamw_kernel<<<static_cast<unsigned>((n4 + 255) / 256), 256, 0, st>>>(p, g, m, v, n, lr, b1, b2, eps, wd, bc1, bc2);
+  adamw_kernel<<<static_cast<unsigned>((n4 + 255) / 256), 256, 0, st>>>(p, g, m, v, pb, n, lr, b1, b2, eps, wd, bc1,
+                                                                          bc2);
   ++g_kernel_launches;
   return cudaGetLastError();
 }

@@ -131,12 +131,13 @@ __device__ __forceinline__ uint64_t sw128_mnmajor_desc(uint32_t saddr) {
   return d;
 }
 
-// Instruction descriptor, kind::f16: bf16 x bf16 -> f32, A K-major, B K- or MN-major, M = 128.
+// Instruction descriptor, kind::f16: bf16 x bf16 -> f32, A and B each K- or MN-major, M = 128.
 template <int BN>
-__device__ __forceinline__ uint32_t idesc_bf16_f32(bool b_mn_major) {
+__device__ __forceinline__ uint32_t idesc_bf16_f32(bool a_mn_major, bool b_mn_major) {
   return (1u << 4)                                 // D format f32
          | (1u << 7)                               // A format bf16
          | (1u << 10)                              // B format bf16
+         | ((a_mn_major ? 1u : 0u) << 15)          // A major-ness
          | ((b_mn_major ? 1u : 0u) << 16)          // B major-ness
          | (static_cast<uint32_t>(BN >> 3) << 17)  // N / 8
          | (static_cast<uint32_t>(BM >> 4) << 24); // M / 16
@@ -494,9 +495,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
           }
         } else {
           mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, p.err);
-          load_tile<BN>(sg.B, p.nf4, lut, seg_mean, sg.K, n0, p.N, kk * BK, Bs, gtid);
+          if (p.b_mode[s] == 0) load_tile<BN>(sg.B, p.nf4, lut, seg_mean, sg.K, n0, p.N, kk * BK, Bs, gtid);
         }
-        if (!p.a_tma[s]) load_tile<BM>(sg.A, p.nf4, lut, seg_mean, sg.K, m0, p.M, kk * BK, As, gtid);
+        if (p.a_mode[s] == 0) load_tile<BM>(sg.A, p.nf4, lut, seg_mean, sg.K, m0, p.M, kk * BK, As, gtid);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&full[st]);
@@ -518,11 +519,26 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
           const uint32_t ph = static_cast<uint32_t>(kb / C::STAGES) & 1u;
           mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, p.err);
           uint8_t* As = base + st * C::STAGE_BYTES;
-          uint8_t* Rc = As + C::A_BYTES + C::B_BYTES;
+          uint8_t* Bs = As + C::A_BYTES;
+          uint8_t* Rc = Bs + C::B_BYTES;
           uint8_t* Rq = Rc + C::RAW_CODE_BYTES;
-          if (p.a_tma[s]) {
-            mbar_arrive_expect_tx(&full[st], C::A_BYTES);
-            tma_load_2d(As, &p.tmapA[s], kk * BK, m0, &full[st]);
+          const int am = p.a_mode[s], bm = raw ? 0 : p.b_mode[s];
+          const uint32_t tx = (am ? C::A_BYTES : 0) + (bm ? C::B_BYTES : 0);
+          if (tx) {
+            mbar_arrive_expect_tx(&full[st], tx);
+            const int k0 = kk * BK;
+            if (am == 1) {
+              tma_load_2d(As, &p.tmapA[s], k0, m0, &full[st]);
+            } else if (am == 2) {
+#pragma unroll
+              for (int i = 0; i < BM / 64; ++i) tma_load_2d(As + i * 8192, &p.tmapA[s], m0 + 64 * i, k0, &full[st]);
+            }
+            if (bm == 1) {
+              tma_load_2d(Bs, &p.tmapB[s], k0, n0 - p.b_row0[s], &full[st]);
+            } else if (bm == 2) {
+#pragma unroll
+              for (int i = 0; i < BN / 64; ++i) tma_load_2d(Bs + i * 8192, &p.tmapB[s], n0 + 64 * i, k0, &full[st]);
+            }
           } else {
             mbar_arrive(&full[st]);
           }
@@ -554,8 +570,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
         const GemmSeg& sg = p.seg[s];
         if (!seg_active(sg, n0, BN)) continue;
         const int nk = (sg.K + BK - 1) / BK;
-        const bool b_mn = (s == 0) && p.raw_tma && sg.B.kind == OP_NF4_MN;
-        const uint32_t idesc = idesc_bf16_f32<BN>(b_mn);
+        const bool b_mn = ((s == 0) && p.raw_tma && sg.B.kind == OP_NF4_MN) || p.b_mode[s] == 2;
+        const bool a_mn = p.a_mode[s] == 2;
+        const uint32_t idesc = idesc_bf16_f32<BN>(a_mn, b_mn);
         for (int kk = 0; kk < nk; ++kk, ++g) {
           if (g < kb_lo || g >= kb_hi) continue;
           const int st = kb % C::STAGES;
@@ -567,7 +584,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
 #pragma unroll
           for (int j = 0; j < BK / 16; ++j) {
             const uint64_t bd = b_mn ? sw128_mnmajor_desc(b_addr + j * 2048) : sw128_kmajor_desc(b_addr + j * 32);
-            tc_mma_f16(tmem, sw128_kmajor_desc(a_addr + j * 32), bd, idesc, (kb > 0 || j > 0) ? 1u : 0u);
+            const uint64_t ad = a_mn ? sw128_mnmajor_desc(a_addr + j * 2048) : sw128_kmajor_desc(a_addr + j * 32);
+            tc_mma_f16(tmem, ad, bd, idesc, (kb > 0 || j > 0) ? 1u : 0u);
           }
           tc_commit(&empty[st]);
           ++kb;
@@ -648,14 +666,28 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// TMA descriptor for a K-major bf16 operand: dims (K, M), row stride ld elements, 64 x 128 box,
-// 128-byte swizzle (the layout the MMA descriptors expect), zero fill out of bounds.
-bool encode_kmajor_bf16(CUtensorMap* map, const void* ptr, int K, int M, long long ld) {
+// TMA descriptor for a K-major bf16 operand: dims (K, rows), row stride ld elements, 64 x
+// box_rows box, 128-byte swizzle (the layout the MMA descriptors expect), zero fill.
+bool encode_kmajor_bf16(CUtensorMap* map, const void* ptr, int K, int rows, long long ld, int box_rows) {
   auto fn = tensor_map_encoder();
-  if (!fn) return false;
-  cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
+  if (!fn || K <= 0 || rows <= 0) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
-  cuuint32_t box[2] = {BK, BM};
+  cuuint32_t box[2] = {BK, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t es[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// TMA descriptor for an MN-major bf16 operand (element (r, k) at ptr[k*ld + r]): dims (rows, K),
+// 64 x 64 boxes with 128-byte swizzle = one MN-major atom column of a 64-deep K block.
+bool encode_mnmajor_bf16(CUtensorMap* map, const void* ptr, int rows, int K, long long ld) {
+  auto fn = tensor_map_encoder();
+  if (!fn || K <= 0 || rows <= 0) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(K)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
+  cuuint32_t box[2] = {64, 64};
   cuuint32_t es[2] = {1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -681,6 +713,15 @@ bool encode_u8_2d(CUtensorMap* map, const void* ptr, unsigned long long w, unsig
 bool raw_tma_allowed() {
   static const bool allowed = [] {
     const char* e = std::getenv("SOUP_GEMM_RAW_TMA");
+    return !(e && e[0] == '0');
+  }();
+  return allowed;
+}
+
+// SOUP_GEMM_TMA_OPERANDS=0 keeps every operand except K-major A on the producer-warp path.
+bool tma_operands_allowed() {
+  static const bool allowed = [] {
+    const char* e = std::getenv("SOUP_GEMM_TMA_OPERANDS");
     return !(e && e[0] == '0');
   }();
   return allowed;
@@ -771,7 +812,9 @@ cudaError_t gemm_launch(const GemmParams& p_in, cudaStream_t st) {
   long long nkb = 0;
   for (int s = 0; s < p.nseg; ++s) {
     GemmSeg& sg = p.seg[s];
-    p.a_tma[s] = 0;
+    p.a_mode[s] = 0;
+    p.b_mode[s] = 0;
+    p.b_row0[s] = 0;
     if (sg.K < 0) return cudaErrorInvalidValue;
     if (sg.K == 0) continue;
     if (!operand_ok(sg.A, sg.K) || !operand_ok(sg.B, sg.K)) return cudaErrorInvalidValue;
@@ -779,12 +822,39 @@ cudaError_t gemm_launch(const GemmParams& p_in, cudaStream_t st) {
     if (sg.A.kind == OP_NF4_K || sg.A.kind == OP_NF4_MN) return cudaErrorInvalidValue;  // NF4 only as B
     if (sg.B.kind == OP_NF4_K && (p.nf4.cols % 8 != 0 || sg.K > p.nf4.cols)) return cudaErrorInvalidValue;
     if (sg.B.kind == OP_NF4_MN && (p.nf4.cols % 8 != 0 || p.N > p.nf4.cols)) return cudaErrorInvalidValue;
-    if (sg.A.kind == OP_BF16_K) p.a_tma[s] = encode_kmajor_bf16(&p.tmapA[s], sg.A.ptr, sg.K, p.M, sg.A.ld) ? 1 : 0;
     nkb += (sg.K + BK - 1) / BK;
   }
   const int BN = (p.N <= 64) ? 64 : ((p.N <= 128 || static_cast<long long>((p.N + 255) / 256) * ((p.M + 127) / 128) < 148) ? 128 : 256);
   p.bn = BN;
   p.raw_tma = setup_raw_tma(p, BN) ? 1 : 0;
+  if (tma_operands_allowed()) {
+    for (int s = 0; s < p.nseg; ++s) {
+      GemmSeg& sg = p.seg[s];
+      if (sg.K <= 0) continue;
+      if (sg.A.kind == OP_BF16_K)
+        p.a_mode[s] = encode_kmajor_bf16(&p.tmapA[s], sg.A.ptr, sg.K, p.M, sg.A.ld, BM) ? 1 : 0;
+      else if (sg.A.kind == OP_BF16_MN)
+        p.a_mode[s] = encode_mnmajor_bf16(&p.tmapA[s], sg.A.ptr, p.M, sg.K, sg.A.ld) ? 2 : 0;
+      if (sg.B.kind == OP_BF16_K) {
+        // a block-diagonal window [row_lo, row_hi) becomes the descriptor's whole extent, so
+        // rows outside it read as zero through the TMA's out-of-bounds fill
+        const int lo = std::max(0, sg.B.row_lo), hi = std::min(p.N, sg.B.row_hi);
+        if (hi > lo) {
+          const void* base = static_cast<const uint16_t*>(sg.B.ptr) + static_cast<long long>(lo) * sg.B.ld;
+          if (encode_kmajor_bf16(&p.tmapB[s], base, sg.K, hi - lo, sg.B.ld, BN)) {
+            p.b_mode[s] = 1;
+            p.b_row0[s] = lo;
+          }
+        }
+      } else if (sg.B.kind == OP_BF16_MN && sg.B.row_lo <= 0 && sg.B.row_hi >= p.N) {
+        p.b_mode[s] = encode_mnmajor_bf16(&p.tmapB[s], sg.B.ptr, p.N, sg.K, sg.B.ld) ? 2 : 0;
+      }
+    }
+  } else {
+    for (int s = 0; s < p.nseg; ++s)
+      if (p.seg[s].K > 0 && p.seg[s].A.kind == OP_BF16_K)
+        p.a_mode[s] = encode_kmajor_bf16(&p.tmapA[s], p.seg[s].A.ptr, p.seg[s].K, p.M, p.seg[s].A.ld, BM) ? 1 : 0;
+  }
   // split-K for grids that cannot fill the GPU (skinny LoRA GEMMs, long reductions)
   p.splits = 1;
   const long long tiles = static_cast<long long>((p.N + BN - 1) / BN) * ((p.M + BM - 1) / BM);

@@ -55,12 +55,16 @@ struct GemmSeg {
 constexpr int GEMM_MAX_SEG = 5;
 
 struct GemmParams {
-  CUtensorMap tmapA[GEMM_MAX_SEG];  // TMA descriptors of K-major bf16 A operands (filled by gemm_launch)
+  // filled by gemm_launch:
+  CUtensorMap tmapA[GEMM_MAX_SEG];  // TMA descriptors of bf16 A operands
+  CUtensorMap tmapB[GEMM_MAX_SEG];  // TMA descriptors of bf16 B operands
   CUtensorMap tmapCodes[3];         // TMA descriptors of each NF4 tensor's packed codes (raw staging)
   CUtensorMap tmapQ8[3];            // ... and of its q8 absmax
-  int a_tma[GEMM_MAX_SEG];          // 1: segment's A tile arrives by TMA
-  int raw_tma;                      // 1: the NF4 segment's codes / absmax arrive by TMA (filled by gemm_launch)
-  int bn;                           // output tile width chosen by gemm_launch
+  int a_mode[GEMM_MAX_SEG];         // 0: producer warps load A; 1: TMA, K-major; 2: TMA, MN-major
+  int b_mode[GEMM_MAX_SEG];         // same for B (bf16 operands only)
+  int b_row0[GEMM_MAX_SEG];         // first operand row of the B descriptor (block-diagonal windows)
+  int raw_tma;                      // 1: the NF4 segment's codes / absmax arrive by TMA
+  int bn;                           // output tile width
   int M, N;
   int nseg;
   GemmSeg seg[GEMM_MAX_SEG];
@@ -111,8 +115,9 @@ cudaError_t rmsnorm_fwd_launch(const uint16_t* x, const uint16_t* gamma, int T, 
                                float* rstd, cudaStream_t st);
 cudaError_t rmsnorm_bwd_launch(const uint16_t* dy, const uint16_t* x, const float* rstd, const uint16_t* gamma,
                                const uint16_t* dres, int T, int h, uint16_t* dx, cudaStream_t st);
-cudaError_t rope_launch(uint16_t* qkv, long long ld, int B, int S, int hq, int hkv, int d, float theta, int inverse,
-                        cudaStream_t st);
+// tcos / tsin: [S_max, d/2] fp32 tables of cos / sin(pos * theta^(-2i/d)).
+cudaError_t rope_launch(uint16_t* qkv, long long ld, int B, int S, int hq, int hkv, int d, const float* tcos,
+                        const float* tsin, int inverse, cudaStream_t st);
 cudaError_t swiglu_fwd_launch(const uint16_t* gu, int T, int I, uint16_t* m, cudaStream_t st);
 cudaError_t swiglu_bwd_launch(const uint16_t* dm, const uint16_t* gu, int T, int I, uint16_t* dgu, cudaStream_t st);
 cudaError_t ce_rows_launch(const float* logits, int T, int V, const int32_t* ids, int B, int S, const uint8_t* mask,
@@ -126,8 +131,10 @@ cudaError_t seq_logp_launch(const float* lse, const float* tgt, int B, int S, in
                             cudaStream_t st);
 cudaError_t ce_grad_launch(const float* logits, const float* lse, const int32_t* ids, const float* row_weight, int B,
                            int S, int V, uint16_t* dlogits, cudaStream_t st);
-cudaError_t adamw_launch(float* p, const float* g, float* m, float* v, long long n, float lr, float b1, float b2,
-                         float eps, float wd, int t, cudaStream_t st);
+// AdamW on fp32 parameters; also writes their bf16 copy `pb` (may be null).
+cudaError_t adamw_launch(float* p, const float* g, float* m, float* v, uint16_t* pb, long long n, float lr, float b1,
+                         float b2, float eps, float wd, int t, cudaStream_t st);
+cudaError_t f32_to_bf16_launch(const float* x, uint16_t* y, long long n, cudaStream_t st);
 cudaError_t fill_zero_launch(void* p, size_t bytes, cudaStream_t st);
 
 // ----------------------------------------------------------------- launch accounting

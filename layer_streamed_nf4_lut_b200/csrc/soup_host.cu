@@ -215,6 +215,7 @@ struct soup_model {
   const uint16_t* lm_head = nullptr;
   // LoRA storage
   float *lora_p = nullptr, *lora_g = nullptr, *lora_m = nullptr, *lora_v = nullptr;
+  uint16_t* lora_bf16 = nullptr;  // bf16 copy of the parameters: the GEMM operands
   size_t lora_n = 0;
   int lora_enabled = 1;
   int adam_t = 0;
@@ -233,6 +234,7 @@ struct soup_model {
   int* scal = nullptr;
   float* quant_scratch = nullptr;  // absmax scratch for the quantiser
   float* gemm_ws = nullptr;        // split-K partial tiles
+  float *rope_cos = nullptr, *rope_sin = nullptr;  // [max_tokens, head_dim/2]
   size_t gemm_ws_bytes = 0;
   float* host_scal = nullptr;      // pinned 2-word staging for the loss + error readback
 
@@ -618,11 +620,11 @@ soup_status layer_forward(soup_model* m, int i, const LayerView& L, const uint16
   }));
   SOUP_TRY(launch(m, st, CAT_RMSNORM, 0, 2 * act + 4.0 * T, "rmsnorm",
                   [&] { return rmsnorm_fwd_launch(A.x, L.gamma[0], T, h, c.rms_eps, A.n1, A.rstd1, st); }));
-  const float* P = m->lora_p;
+  const uint16_t* P = m->lora_bf16;
   // ---- q | k | v
   if (lora) {
     GemmParams p = gemm_base(m, T, 3 * r, A.uqkv, 3 * r, 0, s);
-    add_seg(p, h, opnd(OP_BF16_K, A.n1, h), opnd(OP_F32_K, P + lora_off(c, i, 0, 0), h));
+    add_seg(p, h, opnd(OP_BF16_K, A.n1, h), opnd(OP_BF16_K, P + lora_off(c, i, 0, 0), h));
     SOUP_TRY(run_gemm(m, p, st, "lora u qkv"));
   }
   {
@@ -632,13 +634,13 @@ soup_status layer_forward(soup_model* m, int i, const LayerView& L, const uint16
     if (lora) {
       const int lo[3] = {0, qd, qd + kvd}, hi[3] = {qd, qd + kvd, QKV};
       for (int q = 0; q < 3; ++q)
-        add_seg(p, r, opnd(OP_BF16_K, A.uqkv + q * r, 3 * r), opnd(OP_F32_K, P + lora_off(c, i, 0, 1), r, 1.f, lo[q], hi[q]));
+        add_seg(p, r, opnd(OP_BF16_K, A.uqkv + q * r, 3 * r), opnd(OP_BF16_K, P + lora_off(c, i, 0, 1), r, 1.f, lo[q], hi[q]));
     }
     SOUP_TRY(run_gemm(m, p, st, "qkv gemm"));
   }
   const double rope_bytes = 4.0 * T * (c.n_heads + c.n_kv_heads) * c.head_dim;
   SOUP_TRY(launch(m, st, CAT_ROPE, 0, rope_bytes, "rope", [&] {
-    return rope_launch(A.qkv, QKV, B, S, c.n_heads, c.n_kv_heads, c.head_dim, c.rope_theta, 0, st);
+    return rope_launch(A.qkv, QKV, B, S, c.n_heads, c.n_kv_heads, c.head_dim, m->rope_cos, m->rope_sin, 0, st);
   }));
   AttnShape as{B, S, c.n_heads, c.n_kv_heads, c.head_dim, QKV};
   const double attn_flops = 2.0 * B * c.n_heads * c.head_dim * static_cast<double>(S) * (S + 1);
@@ -647,7 +649,7 @@ soup_status layer_forward(soup_model* m, int i, const LayerView& L, const uint16
   // ---- o + residual
   if (lora) {
     GemmParams p = gemm_base(m, T, r, A.uo, r, 0, s);
-    add_seg(p, qd, opnd(OP_BF16_K, A.o, qd), opnd(OP_F32_K, P + lora_off(c, i, 3, 0), qd));
+    add_seg(p, qd, opnd(OP_BF16_K, A.o, qd), opnd(OP_BF16_K, P + lora_off(c, i, 3, 0), qd));
     SOUP_TRY(run_gemm(m, p, st, "lora u o"));
   }
   {
@@ -656,7 +658,7 @@ soup_status layer_forward(soup_model* m, int i, const LayerView& L, const uint16
     p.residual = A.x;
     p.ldr = h;
     add_seg(p, qd, opnd(OP_BF16_K, A.o, qd), opnd(OP_NF4_K, nullptr, 0));
-    if (lora) add_seg(p, r, opnd(OP_BF16_K, A.uo, r), opnd(OP_F32_K, P + lora_off(c, i, 3, 1), r));
+    if (lora) add_seg(p, r, opnd(OP_BF16_K, A.uo, r), opnd(OP_BF16_K, P + lora_off(c, i, 3, 1), r));
     SOUP_TRY(run_gemm(m, p, st, "o gemm"));
   }
   SOUP_TRY(launch(m, st, CAT_RMSNORM, 0, 2 * act + 4.0 * T, "rmsnorm",
@@ -664,7 +666,7 @@ soup_status layer_forward(soup_model* m, int i, const LayerView& L, const uint16
   // ---- gate | up, SwiGLU
   if (lora) {
     GemmParams p = gemm_base(m, T, 2 * r, A.ugu, 2 * r, 0, s);
-    add_seg(p, h, opnd(OP_BF16_K, A.n2, h), opnd(OP_F32_K, P + lora_off(c, i, 4, 0), h));
+    add_seg(p, h, opnd(OP_BF16_K, A.n2, h), opnd(OP_BF16_K, P + lora_off(c, i, 4, 0), h));
     SOUP_TRY(run_gemm(m, p, st, "lora u gate/up"));
   }
   {
@@ -674,7 +676,7 @@ soup_status layer_forward(soup_model* m, int i, const LayerView& L, const uint16
     if (lora) {
       for (int q = 0; q < 2; ++q)
         add_seg(p, r, opnd(OP_BF16_K, A.ugu + q * r, 2 * r),
-                opnd(OP_F32_K, P + lora_off(c, i, 4, 1), r, 1.f, q * I, (q + 1) * I));
+                opnd(OP_BF16_K, P + lora_off(c, i, 4, 1), r, 1.f, q * I, (q + 1) * I));
     }
     SOUP_TRY(run_gemm(m, p, st, "gate/up gemm"));
   }
@@ -682,7 +684,7 @@ soup_status layer_forward(soup_model* m, int i, const LayerView& L, const uint16
   // ---- down + residual
   if (lora) {
     GemmParams p = gemm_base(m, T, r, A.ud, r, 0, s);
-    add_seg(p, I, opnd(OP_BF16_K, A.m, I), opnd(OP_F32_K, P + lora_off(c, i, 6, 0), I));
+    add_seg(p, I, opnd(OP_BF16_K, A.m, I), opnd(OP_BF16_K, P + lora_off(c, i, 6, 0), I));
     SOUP_TRY(run_gemm(m, p, st, "lora u down"));
   }
   {
@@ -691,7 +693,7 @@ soup_status layer_forward(soup_model* m, int i, const LayerView& L, const uint16
     p.residual = A.x1;
     p.ldr = h;
     add_seg(p, I, opnd(OP_BF16_K, A.m, I), opnd(OP_NF4_K, nullptr, 0));
-    if (lora) add_seg(p, r, opnd(OP_BF16_K, A.ud, r), opnd(OP_F32_K, P + lora_off(c, i, 6, 1), r));
+    if (lora) add_seg(p, r, opnd(OP_BF16_K, A.ud, r), opnd(OP_BF16_K, P + lora_off(c, i, 6, 1), r));
     SOUP_TRY(run_gemm(m, p, st, "down gemm"));
   }
   A.B = B;
@@ -735,19 +737,19 @@ soup_status layer_backward(soup_model* m, int i, const LayerView& L, const uint1
   const int qd = c.n_heads * c.head_dim, kvd = c.n_kv_heads * c.head_dim, QKV = m->qkv_cols;
   const float s = m->s_lora;
   const bool lora = A.lora && m->lora_p;
-  const float* P = m->lora_p;
+  const uint16_t* P = m->lora_bf16;
   float* G = m->lora_g;
   // ---- down
   if (lora) {
     GemmParams p = gemm_base(m, T, r, m->vd, r, 0, s);
-    add_seg(p, h, opnd(OP_BF16_K, dy, h), opnd(OP_F32_MN, P + lora_off(c, i, 6, 1), r));
+    add_seg(p, h, opnd(OP_BF16_K, dy, h), opnd(OP_BF16_MN, P + lora_off(c, i, 6, 1), r));
     SOUP_TRY(run_gemm(m, p, st, "lora v down"));
   }
   {
     GemmParams p = gemm_base(m, T, I, m->dm, I, 0, 1.f);
     p.nf4 = group_of(m, L, {6});
     add_seg(p, h, opnd(OP_BF16_K, dy, h), opnd(OP_NF4_MN, nullptr, 0));
-    if (lora) add_seg(p, r, opnd(OP_BF16_K, m->vd, r), opnd(OP_F32_MN, P + lora_off(c, i, 6, 0), I));
+    if (lora) add_seg(p, r, opnd(OP_BF16_K, m->vd, r), opnd(OP_BF16_MN, P + lora_off(c, i, 6, 0), I));
     SOUP_TRY(run_gemm(m, p, st, "down dX"));
   }
   if (lora)
@@ -759,7 +761,7 @@ soup_status layer_backward(soup_model* m, int i, const LayerView& L, const uint1
   if (lora) {
     for (int q = 0; q < 2; ++q) {
       GemmParams p = gemm_base(m, T, r, m->vgu + q * r, 2 * r, 0, s);
-      add_seg(p, I, opnd(OP_BF16_K, m->dgu + q * I, 2 * I), opnd(OP_F32_MN, P + lora_off(c, i, 4 + q, 1), r));
+      add_seg(p, I, opnd(OP_BF16_K, m->dgu + q * I, 2 * I), opnd(OP_BF16_MN, P + lora_off(c, i, 4 + q, 1), r));
       SOUP_TRY(run_gemm(m, p, st, "lora v gate/up"));
     }
   }
@@ -769,7 +771,7 @@ soup_status layer_backward(soup_model* m, int i, const LayerView& L, const uint1
     add_seg(p, 2 * I, opnd(OP_BF16_K, m->dgu, 2 * I), opnd(OP_NF4_MN, nullptr, 0));
     if (lora)
       for (int q = 0; q < 2; ++q)
-        add_seg(p, r, opnd(OP_BF16_K, m->vgu + q * r, 2 * r), opnd(OP_F32_MN, P + lora_off(c, i, 4 + q, 0), h));
+        add_seg(p, r, opnd(OP_BF16_K, m->vgu + q * r, 2 * r), opnd(OP_BF16_MN, P + lora_off(c, i, 4 + q, 0), h));
     SOUP_TRY(run_gemm(m, p, st, "gate/up dX"));
   }
   if (lora) {
@@ -785,14 +787,14 @@ soup_status layer_backward(soup_model* m, int i, const LayerView& L, const uint1
   // ---- o
   if (lora) {
     GemmParams p = gemm_base(m, T, r, m->vo, r, 0, s);
-    add_seg(p, h, opnd(OP_BF16_K, m->dx1, h), opnd(OP_F32_MN, P + lora_off(c, i, 3, 1), r));
+    add_seg(p, h, opnd(OP_BF16_K, m->dx1, h), opnd(OP_BF16_MN, P + lora_off(c, i, 3, 1), r));
     SOUP_TRY(run_gemm(m, p, st, "lora v o"));
   }
   {
     GemmParams p = gemm_base(m, T, qd, m->da, qd, 0, 1.f);
     p.nf4 = group_of(m, L, {3});
     add_seg(p, h, opnd(OP_BF16_K, m->dx1, h), opnd(OP_NF4_MN, nullptr, 0));
-    if (lora) add_seg(p, r, opnd(OP_BF16_K, m->vo, r), opnd(OP_F32_MN, P + lora_off(c, i, 3, 0), qd));
+    if (lora) add_seg(p, r, opnd(OP_BF16_K, m->vo, r), opnd(OP_BF16_MN, P + lora_off(c, i, 3, 0), qd));
     SOUP_TRY(run_gemm(m, p, st, "o dX"));
   }
   if (lora)
@@ -805,14 +807,14 @@ soup_status layer_backward(soup_model* m, int i, const LayerView& L, const uint1
                   [&] { return attn_bwd_launch(as, A.qkv, A.o, m->da, A.lse, m->delta, m->dqkv, st); }));
   const double rope_bytes = 4.0 * T * (c.n_heads + c.n_kv_heads) * c.head_dim;
   SOUP_TRY(launch(m, st, CAT_ROPE, 0, rope_bytes, "rope bwd", [&] {
-    return rope_launch(m->dqkv, QKV, B, S, c.n_heads, c.n_kv_heads, c.head_dim, c.rope_theta, 1, st);
+    return rope_launch(m->dqkv, QKV, B, S, c.n_heads, c.n_kv_heads, c.head_dim, m->rope_cos, m->rope_sin, 1, st);
   }));
   // ---- q | k | v
   const int off[3] = {0, qd, qd + kvd}, outs[3] = {qd, kvd, kvd};
   if (lora) {
     for (int q = 0; q < 3; ++q) {
       GemmParams p = gemm_base(m, T, r, m->vqkv + q * r, 3 * r, 0, s);
-      add_seg(p, outs[q], opnd(OP_BF16_K, m->dqkv + off[q], QKV), opnd(OP_F32_MN, P + lora_off(c, i, q, 1), r));
+      add_seg(p, outs[q], opnd(OP_BF16_K, m->dqkv + off[q], QKV), opnd(OP_BF16_MN, P + lora_off(c, i, q, 1), r));
       SOUP_TRY(run_gemm(m, p, st, "lora v qkv"));
     }
   }
@@ -822,7 +824,7 @@ soup_status layer_backward(soup_model* m, int i, const LayerView& L, const uint1
     add_seg(p, QKV, opnd(OP_BF16_K, m->dqkv, QKV), opnd(OP_NF4_MN, nullptr, 0));
     if (lora)
       for (int q = 0; q < 3; ++q)
-        add_seg(p, r, opnd(OP_BF16_K, m->vqkv + q * r, 3 * r), opnd(OP_F32_MN, P + lora_off(c, i, q, 0), h));
+        add_seg(p, r, opnd(OP_BF16_K, m->vqkv + q * r, 3 * r), opnd(OP_BF16_MN, P + lora_off(c, i, q, 0), h));
     SOUP_TRY(run_gemm(m, p, st, "qkv dX"));
   }
   if (lora) {
@@ -995,7 +997,7 @@ soup_status do_step(soup_model* m, soup_loss kind, const soup_batch* bt, float* 
   if (bt->apply_optimizer) {
     m->adam_t += 1;
     SOUP_TRY(launch(m, st, CAT_ADAMW, 0, 28.0 * m->lora_n, "adamw", [&] {
-      return adamw_launch(m->lora_p, m->lora_g, m->lora_m, m->lora_v, static_cast<long long>(m->lora_n), bt->lr, 0.9f,
+      return adamw_launch(m->lora_p, m->lora_g, m->lora_m, m->lora_v, m->lora_bf16, static_cast<long long>(m->lora_n), bt->lr, 0.9f,
                           0.999f, 1e-8f, 0.f, m->adam_t, st);
     }));
   }
@@ -1102,10 +1104,25 @@ soup_status create_model(const soup_model_config* cfg, const soup_allocator* all
       alloc_into(m, m->pi, T) || alloc_into(m, m->ref, T) || alloc_into(m, m->ids_dev, T) ||
       alloc_into(m, m->mask_dev, T) || alloc_into(m, m->scal, 64))
     return fail(SOUP_ERR_OOM);
+  {  // RoPE tables: angle = pos * theta^(-2i/d), computed in float64, stored as float32
+    const int half = c.head_dim / 2;
+    std::vector<float> hc(static_cast<size_t>(T) * half), hs(hc.size());
+    for (size_t pos = 0; pos < T; ++pos)
+      for (int i = 0; i < half; ++i) {
+        const double ang = static_cast<double>(pos) * std::pow(static_cast<double>(c.rope_theta), -2.0 * i / c.head_dim);
+        hc[pos * half + i] = static_cast<float>(std::cos(ang));
+        hs[pos * half + i] = static_cast<float>(std::sin(ang));
+      }
+    if (alloc_into(m, m->rope_cos, hc.size()) || alloc_into(m, m->rope_sin, hs.size())) return fail(SOUP_ERR_OOM);
+    if (cudaMemcpy(m->rope_cos, hc.data(), hc.size() * 4, cudaMemcpyHostToDevice) != cudaSuccess ||
+        cudaMemcpy(m->rope_sin, hs.data(), hs.size() * 4, cudaMemcpyHostToDevice) != cudaSuccess)
+      return fail(SOUP_ERR_CUDA);
+  }
   m->gemm_ws_bytes = static_cast<size_t>(64) << 20;
   if (alloc_into(m, m->gemm_ws, m->gemm_ws_bytes / sizeof(float))) return fail(SOUP_ERR_OOM);
   if (cudaMemset(m->scal, 0, 64 * sizeof(int)) != cudaSuccess) return fail(SOUP_ERR_CUDA);
   m->lora_n = lora_numel_of(c);
+  if (alloc_into(m, m->lora_bf16, m->lora_n)) return fail(SOUP_ERR_OOM);
   *out = m;
   return SOUP_OK;
 }
@@ -1315,7 +1332,20 @@ soup_status soup_model_set_lora(soup_model* m, float* params, float* grads, floa
   m->lora_v = adam_v;
   m->adam_t = 0;
   for (auto& a : m->saved) a.valid = 0;
-  return SOUP_OK;
+  SOUP_GUARD({
+    SOUP_TRY(check_launch(m, f32_to_bf16_launch(params, m->lora_bf16, static_cast<long long>(m->lora_n), nullptr),
+                          "lora copy"));
+    SOUP_CK(cudaDeviceSynchronize());
+    return SOUP_OK;
+  })
+}
+
+soup_status soup_model_refresh_lora(soup_model* m, void* stream) {
+  if (!m) return SOUP_ERR_INVALID_ARG;
+  if (!m->lora_p) return SOUP_ERR_STATE;
+  SOUP_GUARD(return check_launch(m, f32_to_bf16_launch(m->lora_p, m->lora_bf16, static_cast<long long>(m->lora_n),
+                                                       static_cast<cudaStream_t>(stream)),
+                                 "lora copy");)
 }
 
 soup_status soup_set_lora_enabled(soup_model* m, int enabled) {
@@ -1374,7 +1404,7 @@ soup_status soup_optimizer_step(soup_model* m, float lr, void* stream) {
   SOUP_GUARD({
     m->adam_t += 1;
     const long long l0 = g_kernel_launches.load();
-    soup_status s = check_launch(m, adamw_launch(m->lora_p, m->lora_g, m->lora_m, m->lora_v,
+    soup_status s = check_launch(m, adamw_launch(m->lora_p, m->lora_g, m->lora_m, m->lora_v, m->lora_bf16,
                                                  static_cast<long long>(m->lora_n), lr, 0.9f, 0.999f, 1e-8f, 0.f,
                                                  m->adam_t, static_cast<cudaStream_t>(stream)),
                                  "adamw");

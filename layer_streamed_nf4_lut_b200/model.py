@@ -148,6 +148,10 @@ class SoupModel:
         self._ck(lib.soup_model_set_lora(self.h, _ptr(self.lora_params), _ptr(self.lora_grads), _ptr(self.adam_m),
                                          _ptr(self.adam_v)))
 
+    def refresh_lora(self):
+        """Call after changing lora_params outside the library (refreshes its bf16 copy)."""
+        self._ck(lib.soup_model_refresh_lora(self.h, _stream_ptr()))
+
     def lora_view(self, flat: torch.Tensor, layer: int, proj: str, which_b: int) -> torch.Tensor:
         off, r, c = lora_offset(self.cfg, layer, PROJ.index(proj), which_b)
         return flat[off:off + r * c].view(r, c)
