@@ -122,13 +122,13 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------------- soup arm
-def build_model(wl, device_index, seed):
+def build_model(wl, device_index, seed, mode="streamed"):
     import torch
     from layer_streamed_nf4_lut_b200.model import SoupModel, lora_offset
     cfg = dict(wl["cfg"])
     B, S = wl["B"], wl["S"]
     dev = torch.device("cuda", device_index)
-    gm = SoupModel(cfg, mode="streamed", n_layer_buffers=2, max_tokens=B * S, device=device_index)
+    gm = SoupModel(cfg, mode=mode, n_layer_buffers=2, max_tokens=B * S, device=device_index)
     ones = torch.ones(cfg["hidden"], dtype=torch.bfloat16, device=dev)
     for i in range(cfg["n_layers"]):
         w = {}
@@ -239,11 +239,34 @@ def run_soup(args, wl, rank, world, local_rank):
         e2e_s = dp.max_over_ranks(e2e_s, device=dev)
     e2e_tok_s = world * T * args.steps / e2e_s
 
+    # compute-only reference (one GPU): the same step with every layer resident, no streaming;
+    # tells apart the kernels' time from the streaming / overlap losses
+    compute_ms = None
+    if world == 1 and not args.no_compute_only:
+        gm.close()
+        del gm
+        torch.cuda.empty_cache()
+        gr = build_model(wl, local_rank, seed=1234, mode="resident")
+        for _ in range(2):
+            gr.step(ids, **kw, apply_optimizer=True)
+        torch.cuda.synchronize(dev)
+        c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        c0.record(stream)
+        for _ in range(args.steps):
+            gr.step(ids, **kw, apply_optimizer=True)
+        c1.record(stream)
+        c1.synchronize()
+        compute_ms = c0.elapsed_time(c1) / args.steps
+        blob_bytes = gr.blob_bytes
+        gr.close()
+    else:
+        blob_bytes = gm.blob_bytes
+
     if rank != 0:
         return None
     pk = peaks()
     flops = step_flops(cfg, B, S, wl["loss"])
-    stream_bytes = loads_per_step * gm.blob_bytes
+    stream_bytes = loads_per_step * blob_bytes
     t_flops = flops / (pk["bf16_sustained"] * 1e12)
     t_h2d = stream_bytes / (h2d_gbs * 1e9)
     t_roof = max(t_flops, t_h2d)
@@ -286,6 +309,7 @@ def run_soup(args, wl, rank, world, local_rank):
                           "stream_bytes_per_step": int(stream_bytes), "layer_loads_per_step": loads_per_step,
                           "flops_per_step": flops, "bf16_peak_tflops": pk["bf16_sustained"],
                           "achieved_h2d_gbs_in_step": round(h2d["bytes"] / (h2d["total_ms"] * 1e-3) / 1e9, 2) if h2d else None},
+        "compute_only_ms_per_step": round(compute_ms, 3) if compute_ms else None,
         "roofline": roofline,
         "profile": profile_summary,
         "e2e": {"value": round(e2e_tok_s, 2), "unit": "tokens/s", "h2d_bytes_per_step": int(ids_bytes + stream_bytes),
@@ -389,6 +413,7 @@ def main():
     ap.add_argument("--workload", default=DEFAULT, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="soup", choices=["soup", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-compute-only", action="store_true", help="skip the resident (no streaming) timing")
     args = ap.parse_args()
     wl = WORKLOADS[args.workload]
     rank = int(os.environ.get("RANK", "0"))

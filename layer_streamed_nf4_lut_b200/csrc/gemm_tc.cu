@@ -28,7 +28,9 @@
 #include <algorithm>
 #include <atomic>
 #include <cstdlib>
+#include <cstring>
 #include <mutex>
+#include <unordered_map>
 
 namespace soup {
 
@@ -297,61 +299,125 @@ __device__ __forceinline__ void load_tile(const Operand& op, const NF4Group& g, 
   }
 }
 
+// Decode the 8 codes of one 32-bit word with the block's reconstructed absmax `mh`:
+// bf16_rn(codebook[q] * mh), element 2i in the low nibble of byte i.
+__device__ __forceinline__ uint4 decode_word(uint32_t c, float mh, const float* lut) {
+  uint4 o;
+  o.x = pack_bf16x2(__fmul_rn(lut[c & 15u], mh), __fmul_rn(lut[(c >> 4) & 15u], mh));
+  o.y = pack_bf16x2(__fmul_rn(lut[(c >> 8) & 15u], mh), __fmul_rn(lut[(c >> 12) & 15u], mh));
+  o.z = pack_bf16x2(__fmul_rn(lut[(c >> 16) & 15u], mh), __fmul_rn(lut[(c >> 20) & 15u], mh));
+  o.w = pack_bf16x2(__fmul_rn(lut[(c >> 24) & 15u], mh), __fmul_rn(lut[c >> 28], mh));
+  return o;
+}
+
+// PTX byte permute in its default mode: each selector nibble's low 3 bits pick one of the 8
+// source bytes; a set bit 3 replicates that byte's sign bit over the result byte.
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+// Per-block decode table: the 16 values bf16_rn(codebook[j] * mh) of one absmax block, kept as
+// 4 words of low bytes (L) and 4 words of high bytes (H), entry j in byte j%4 of word j/4.
+struct BlockLut {
+  uint32_t L[4], H[4];
+};
+__device__ __forceinline__ BlockLut block_lut(const float (&cb)[16], float mh) {
+  uint32_t R[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) R[i] = pack_bf16x2(__fmul_rn(cb[2 * i], mh), __fmul_rn(cb[2 * i + 1], mh));
+  BlockLut t;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    t.L[i] = prmt(R[2 * i], R[2 * i + 1], 0x6420);
+    t.H[i] = prmt(R[2 * i], R[2 * i + 1], 0x7531);
+  }
+  return t;
+}
+// Four table lookups with byte permutes: s holds four 3-bit indices (nibbles), m has 0xFF in
+// the bytes whose code is >= 8 (upper half of the table).  Returns two bf16x2 words.
+__device__ __forceinline__ void lut4(const BlockLut& t, uint32_t s, uint32_t m, uint32_t& o01, uint32_t& o23) {
+  const uint32_t lo = (prmt(t.L[0], t.L[1], s) & ~m) | (prmt(t.L[2], t.L[3], s) & m);
+  const uint32_t hi = (prmt(t.H[0], t.H[1], s) & ~m) | (prmt(t.H[2], t.H[3], s) & m);
+  o01 = prmt(lo, hi, 0x5140);
+  o23 = prmt(lo, hi, 0x7362);
+}
+// The 8 codes of one 32-bit word (element 2i = low nibble of byte i) through the block table.
+__device__ __forceinline__ uint4 decode_word_lut(uint32_t c, const BlockLut& t) {
+  const uint32_t c4 = c << 4;
+  const uint32_t m0 = prmt(c4, c, 0xD9C8);  // sign-replicated bit 3 of nibbles 0..3
+  const uint32_t m1 = prmt(c4, c, 0xFBEA);  // ... of nibbles 4..7
+  uint4 o;
+  lut4(t, c & 0x7777u, m0, o.x, o.y);
+  lut4(t, (c >> 16) & 0x7777u, m1, o.z, o.w);
+  return o;
+}
+
 // Dequantise the forward (W[n, k]) B tile from TMA-staged raw codes / q8 absmax.
-// raw_codes: [BN][32] bytes (row n, k0..k0+63); raw_q8: [BN][16] bytes covering k-blocks
-// [16*floor(kbw/16), +16) of each row; the tile lies inside NF4 tensor `s`.
+// raw_codes: [BN][32] bytes (row n, k0..k0+63 = exactly one absmax block); raw_q8: [BN][16]
+// bytes covering k-blocks [16*floor(kbw/16), +16) of each row; the tile lies inside NF4
+// tensor `s`.  One thread decodes a whole 64-element row block (one absmax, 8 stores).
 template <int BN>
-__device__ __forceinline__ void decode_fwd_raw(const NF4Group& g, int s, const float* lut, const float* seg_mean,
+__device__ __forceinline__ void decode_fwd_raw(const NF4Group& g, int s, const float (&cb)[16], const float* seg_mean,
                                                int n0, int N, int kbw, const uint8_t* raw_codes,
                                                const uint8_t* raw_q8, uint8_t* tile, int gtid) {
   const NF4Seg& sg = g.seg[s];
   const long long cpr = g.cols >> 6;  // absmax blocks per row
   const float mean = seg_mean[s];
-#pragma unroll 4
-  for (int c = gtid; c < BN * 8; c += GROUP_THREADS) {
-    const int r = c >> 3, kc = c & 7;
-    uint4 v = make_uint4(0, 0, 0, 0);
+#pragma unroll 1
+  for (int r = gtid; r < BN; r += GROUP_THREADS) {
     if (n0 + r < N) {
-      NF4Raw raw;
-      raw.code = *reinterpret_cast<const uint32_t*>(raw_codes + r * 32 + kc * 4);
-      raw.q8 = static_cast<int8_t>(raw_q8[r * 16 + (kbw & 15)]);
+      const uint4 w0 = *reinterpret_cast<const uint4*>(raw_codes + r * 32);
+      const uint4 w1 = *reinterpret_cast<const uint4*>(raw_codes + r * 32 + 16);
+      const int q8 = static_cast<int8_t>(raw_q8[r * 16 + (kbw & 15)]);
       const long long blk = static_cast<long long>(n0 + r - sg.row_begin) * cpr + kbw;
-      raw.s2 = __ldg(sg.scales + (blk >> 8));
-      raw.seg = s;
-      (void)mean;
-      v = nf4_decode(raw, lut, seg_mean);
+      const float mh = __fadd_rn(__fmul_rn(static_cast<float>(q8), __ldg(sg.scales + (blk >> 8))), mean);
+      const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+      const BlockLut t = block_lut(cb, mh);
+#pragma unroll
+      for (int kc = 0; kc < 8; ++kc)
+        *reinterpret_cast<uint4*>(tile + swz_off(r, kc)) = decode_word_lut(words[kc], t);
+    } else {
+#pragma unroll
+      for (int kc = 0; kc < 8; ++kc) *reinterpret_cast<uint4*>(tile + swz_off(r, kc)) = make_uint4(0, 0, 0, 0);
     }
-    *reinterpret_cast<uint4*>(tile + swz_off(r, kc)) = v;
   }
 }
 
 // Dequantise the transposed (dX) B tile: B[n, k] = W[k0 + k, n0 + n] from raw codes
 // [64][BN/2] bytes and raw q8 [64][16] bytes (absmax blocks [xq, xq+16) of each W row), into
-// the MN-major 128-byte-swizzled layout (8 consecutive n of one k = one 16-byte store).
+// the MN-major 128-byte-swizzled layout.  One thread decodes one absmax block: 64
+// consecutive n of one k (= one 128-byte swizzle row, 8 conflict-free 16-byte stores).
 template <int BN>
-__device__ __forceinline__ void decode_dx_raw(const NF4Group& g, int s, const float* lut, const float* seg_mean,
+__device__ __forceinline__ void decode_dx_raw(const NF4Group& g, int s, const float (&cb)[16], const float* seg_mean,
                                               int n0, int N, int k0, int xq, const uint8_t* raw_codes,
                                               const uint8_t* raw_q8, uint8_t* tile, int gtid) {
   const NF4Seg& sg = g.seg[s];
   const long long cpr = g.cols >> 6;
-  constexpr int NC = BN / 8;
-#pragma unroll 4
-  for (int u = gtid; u < 64 * NC; u += GROUP_THREADS) {
-    const int nc = u % NC, kr = u / NC;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    const int n = n0 + nc * 8;
+  constexpr int NB = BN / 64;  // absmax blocks per W row in the tile
+  const float mean = seg_mean[s];
+#pragma unroll 1
+  for (int u = gtid; u < 64 * NB; u += GROUP_THREADS) {
+    const int kr = u / NB, b = u % NB;
+    const int n = n0 + b * 64;
+    uint8_t* dst = tile + b * 8192 + (kr >> 3) * 1024 + (kr & 7) * 128;
     if (n < N) {
-      NF4Raw raw;
-      raw.code = *reinterpret_cast<const uint32_t*>(raw_codes + kr * (BN / 2) + nc * 4);
+      const uint4 w0 = *reinterpret_cast<const uint4*>(raw_codes + kr * (BN / 2) + b * 32);
+      const uint4 w1 = *reinterpret_cast<const uint4*>(raw_codes + kr * (BN / 2) + b * 32 + 16);
       const int bcol = n >> 6;
-      raw.q8 = static_cast<int8_t>(raw_q8[kr * 16 + (bcol - xq)]);
+      const int q8 = static_cast<int8_t>(raw_q8[kr * 16 + (bcol - xq)]);
       const long long blk = static_cast<long long>(k0 + kr - sg.row_begin) * cpr + bcol;
-      raw.s2 = __ldg(sg.scales + (blk >> 8));
-      raw.seg = s;
-      v = nf4_decode(raw, lut, seg_mean);
+      const float mh = __fadd_rn(__fmul_rn(static_cast<float>(q8), __ldg(sg.scales + (blk >> 8))), mean);
+      const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+      const BlockLut t = block_lut(cb, mh);
+#pragma unroll
+      for (int nc = 0; nc < 8; ++nc)
+        *reinterpret_cast<uint4*>(dst + ((nc ^ (kr & 7)) << 4)) = decode_word_lut(words[nc], t);
+    } else {
+#pragma unroll
+      for (int nc = 0; nc < 8; ++nc) *reinterpret_cast<uint4*>(dst + ((nc ^ (kr & 7)) << 4)) = make_uint4(0, 0, 0, 0);
     }
-    const int off = (nc >> 3) * 8192 + (kr >> 3) * 1024 + (kr & 7) * 128 + (((nc & 7) ^ (kr & 7)) << 4);
-    *reinterpret_cast<uint4*>(tile + off) = v;
   }
 }
 
@@ -467,6 +533,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
   if (warp < 8) {
     // ------------------------------------------------ producers (two groups, alternate k-blocks)
     const int grp = warp >> 2, gtid = threadIdx.x & (GROUP_THREADS - 1);
+    float cb[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) cb[j] = p.lut[j];
     int g = 0;
     for (int s = 0; s < p.nseg; ++s) {
       const GemmSeg& sg = p.seg[s];
@@ -487,10 +556,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
           // raw codes / absmax of this k-block have landed (the issuer waited for the slot)
           mbar_wait_bounded(&raw_full[st], ph, abort_flag, p.err);
           if (sg.B.kind == OP_NF4_K) {
-            decode_fwd_raw<BN>(p.nf4, nf4_seg_of(p.nf4, n0), lut, seg_mean, n0, p.N, kk, Rc, Rq, Bs, gtid);
+            decode_fwd_raw<BN>(p.nf4, nf4_seg_of(p.nf4, n0), cb, seg_mean, n0, p.N, kk, Rc, Rq, Bs, gtid);
           } else {
             const int k0 = kk * BK;
-            decode_dx_raw<BN>(p.nf4, nf4_seg_of(p.nf4, k0), lut, seg_mean, n0, p.N, k0, ((n0 >> 6) >> 4) << 4, Rc,
+            decode_dx_raw<BN>(p.nf4, nf4_seg_of(p.nf4, k0), cb, seg_mean, n0, p.N, k0, ((n0 >> 6) >> 4) << 4, Rc,
                               Rq, Bs, gtid);
           }
         } else {
@@ -666,46 +735,84 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
+// Encoded descriptors are cached by their arguments: the same activation and weight buffers
+// recur every layer and every step, and encoding costs host time on every GEMM launch.
+struct MapKey {
+  const void* ptr;
+  unsigned long long d0, d1, stride;
+  unsigned b0, b1;
+  int dtype, swizzle;
+  bool operator==(const MapKey& o) const { return std::memcmp(this, &o, sizeof(MapKey)) == 0; }
+};
+struct MapKeyHash {
+  size_t operator()(const MapKey& k) const {
+    const unsigned long long* w = reinterpret_cast<const unsigned long long*>(&k);
+    unsigned long long h = 1469598103934665603ull;
+    for (size_t i = 0; i < sizeof(MapKey) / 8; ++i) h = (h ^ w[i]) * 1099511628211ull;
+    return static_cast<size_t>(h);
+  }
+};
+bool encode_cached(CUtensorMap* map, const void* ptr, CUtensorMapDataType dtype, unsigned long long d0,
+                   unsigned long long d1, unsigned long long stride_bytes, unsigned b0, unsigned b1,
+                   CUtensorMapSwizzle swz) {
+  static std::mutex mu;
+  static std::unordered_map<MapKey, CUtensorMap, MapKeyHash> cache;
+  MapKey key;
+  std::memset(&key, 0, sizeof(key));
+  key.ptr = ptr;
+  key.d0 = d0;
+  key.d1 = d1;
+  key.stride = stride_bytes;
+  key.b0 = b0;
+  key.b1 = b1;
+  key.dtype = static_cast<int>(dtype);
+  key.swizzle = static_cast<int>(swz);
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) {
+      *map = it->second;
+      return true;
+    }
+  }
+  auto fn = tensor_map_encoder();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {d0, d1};
+  cuuint64_t strides[1] = {stride_bytes};
+  cuuint32_t box[2] = {b0, b1};
+  cuuint32_t es[2] = {1, 1};
+  if (fn(map, dtype, 2, const_cast<void*>(ptr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache.size() > 8192) cache.clear();
+  cache.emplace(key, *map);
+  return true;
+}
+
 // TMA descriptor for a K-major bf16 operand: dims (K, rows), row stride ld elements, 64 x
 // box_rows box, 128-byte swizzle (the layout the MMA descriptors expect), zero fill.
 bool encode_kmajor_bf16(CUtensorMap* map, const void* ptr, int K, int rows, long long ld, int box_rows) {
-  auto fn = tensor_map_encoder();
-  if (!fn || K <= 0 || rows <= 0) return false;
-  cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
-  cuuint32_t box[2] = {BK, static_cast<cuuint32_t>(box_rows)};
-  cuuint32_t es[2] = {1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  if (K <= 0 || rows <= 0) return false;
+  return encode_cached(map, ptr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<unsigned long long>(K),
+                       static_cast<unsigned long long>(rows), static_cast<unsigned long long>(ld) * 2, BK,
+                       static_cast<unsigned>(box_rows), CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 // TMA descriptor for an MN-major bf16 operand (element (r, k) at ptr[k*ld + r]): dims (rows, K),
 // 64 x 64 boxes with 128-byte swizzle = one MN-major atom column of a 64-deep K block.
 bool encode_mnmajor_bf16(CUtensorMap* map, const void* ptr, int rows, int K, long long ld) {
-  auto fn = tensor_map_encoder();
-  if (!fn || K <= 0 || rows <= 0) return false;
-  cuuint64_t dims[2] = {static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(K)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
-  cuuint32_t box[2] = {64, 64};
-  cuuint32_t es[2] = {1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  if (K <= 0 || rows <= 0) return false;
+  return encode_cached(map, ptr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<unsigned long long>(rows),
+                       static_cast<unsigned long long>(K), static_cast<unsigned long long>(ld) * 2, 64, 64,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 // TMA descriptor for a 2D uint8 array (raw NF4 codes or q8 absmax), no swizzle, zero fill.
 bool encode_u8_2d(CUtensorMap* map, const void* ptr, unsigned long long w, unsigned long long h,
                   unsigned long long stride, unsigned box_w, unsigned box_h) {
-  auto fn = tensor_map_encoder();
-  if (!fn) return false;
-  cuuint64_t dims[2] = {w, h};
-  cuuint64_t strides[1] = {stride};
-  cuuint32_t box[2] = {box_w, box_h};
-  cuuint32_t es[2] = {1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return encode_cached(map, ptr, CU_TENSOR_MAP_DATA_TYPE_UINT8, w, h, stride, box_w, box_h,
+                       CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
 // Raw TMA staging of the NF4 operand: rows of 1024-column multiples (so the q8 absmax rows are
