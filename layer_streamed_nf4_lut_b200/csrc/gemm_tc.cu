@@ -358,21 +358,56 @@ __device__ __forceinline__ uint4 decode_word_lut(uint32_t c, const BlockLut& t) 
 // raw_codes: [BN][32] bytes (row n, k0..k0+63 = exactly one absmax block); raw_q8: [BN][16]
 // bytes covering k-blocks [16*floor(kbw/16), +16) of each row; the tile lies inside NF4
 // tensor `s`.  One thread decodes a whole 64-element row block (one absmax, 8 stores).
+// Group scales (s2) of the absmax blocks a thread decodes in one k-block, loaded before the
+// thread waits for the raw tile so their latency overlaps the wait.
+template <int BN>
+__device__ __forceinline__ void fwd_scales(const NF4Group& g, int s, int n0, int N, int kbw, int gtid,
+                                           float (&s2)[(BN + GROUP_THREADS - 1) / GROUP_THREADS]) {
+  const NF4Seg& sg = g.seg[s];
+  const long long cpr = g.cols >> 6;
+#pragma unroll
+  for (int i = 0; i < (BN + GROUP_THREADS - 1) / GROUP_THREADS; ++i) {
+    const int r = gtid + i * GROUP_THREADS;
+    s2[i] = 0.f;
+    if (r < BN && n0 + r < N) {
+      const long long blk = static_cast<long long>(n0 + r - sg.row_begin) * cpr + kbw;
+      s2[i] = __ldg(sg.scales + (blk >> 8));
+    }
+  }
+}
+template <int BN>
+__device__ __forceinline__ void dx_scales(const NF4Group& g, int s, int n0, int N, int k0, int gtid,
+                                          float (&s2)[(64 * (BN / 64) + GROUP_THREADS - 1) / GROUP_THREADS]) {
+  const NF4Seg& sg = g.seg[s];
+  const long long cpr = g.cols >> 6;
+  constexpr int NB = BN / 64;
+#pragma unroll
+  for (int i = 0; i < (64 * NB + GROUP_THREADS - 1) / GROUP_THREADS; ++i) {
+    const int u = gtid + i * GROUP_THREADS;
+    s2[i] = 0.f;
+    const int kr = u / NB, b = u % NB;
+    if (u < 64 * NB && n0 + b * 64 < N) {
+      const long long blk = static_cast<long long>(k0 + kr - sg.row_begin) * cpr + ((n0 + b * 64) >> 6);
+      s2[i] = __ldg(sg.scales + (blk >> 8));
+    }
+  }
+}
+
 template <int BN>
 __device__ __forceinline__ void decode_fwd_raw(const NF4Group& g, int s, const float (&cb)[16], const float* seg_mean,
                                                int n0, int N, int kbw, const uint8_t* raw_codes,
-                                               const uint8_t* raw_q8, uint8_t* tile, int gtid) {
-  const NF4Seg& sg = g.seg[s];
-  const long long cpr = g.cols >> 6;  // absmax blocks per row
+                                               const uint8_t* raw_q8, uint8_t* tile, int gtid,
+                                               const float (&s2)[(BN + GROUP_THREADS - 1) / GROUP_THREADS]) {
   const float mean = seg_mean[s];
-#pragma unroll 1
-  for (int r = gtid; r < BN; r += GROUP_THREADS) {
+#pragma unroll
+  for (int i = 0; i < (BN + GROUP_THREADS - 1) / GROUP_THREADS; ++i) {
+    const int r = gtid + i * GROUP_THREADS;
+    if (r >= BN) break;
     if (n0 + r < N) {
       const uint4 w0 = *reinterpret_cast<const uint4*>(raw_codes + r * 32);
       const uint4 w1 = *reinterpret_cast<const uint4*>(raw_codes + r * 32 + 16);
       const int q8 = static_cast<int8_t>(raw_q8[r * 16 + (kbw & 15)]);
-      const long long blk = static_cast<long long>(n0 + r - sg.row_begin) * cpr + kbw;
-      const float mh = __fadd_rn(__fmul_rn(static_cast<float>(q8), __ldg(sg.scales + (blk >> 8))), mean);
+      const float mh = __fadd_rn(__fmul_rn(static_cast<float>(q8), s2[i]), mean);
       const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
       const BlockLut t = block_lut(cb, mh);
 #pragma unroll
@@ -392,13 +427,14 @@ __device__ __forceinline__ void decode_fwd_raw(const NF4Group& g, int s, const f
 template <int BN>
 __device__ __forceinline__ void decode_dx_raw(const NF4Group& g, int s, const float (&cb)[16], const float* seg_mean,
                                               int n0, int N, int k0, int xq, const uint8_t* raw_codes,
-                                              const uint8_t* raw_q8, uint8_t* tile, int gtid) {
-  const NF4Seg& sg = g.seg[s];
-  const long long cpr = g.cols >> 6;
+                                              const uint8_t* raw_q8, uint8_t* tile, int gtid,
+                                              const float (&s2)[(64 * (BN / 64) + GROUP_THREADS - 1) / GROUP_THREADS]) {
   constexpr int NB = BN / 64;  // absmax blocks per W row in the tile
   const float mean = seg_mean[s];
-#pragma unroll 1
-  for (int u = gtid; u < 64 * NB; u += GROUP_THREADS) {
+#pragma unroll
+  for (int i = 0; i < (64 * NB + GROUP_THREADS - 1) / GROUP_THREADS; ++i) {
+    const int u = gtid + i * GROUP_THREADS;
+    if (u >= 64 * NB) break;
     const int kr = u / NB, b = u % NB;
     const int n = n0 + b * 64;
     uint8_t* dst = tile + b * 8192 + (kr >> 3) * 1024 + (kr & 7) * 128;
@@ -407,8 +443,7 @@ __device__ __forceinline__ void decode_dx_raw(const NF4Group& g, int s, const fl
       const uint4 w1 = *reinterpret_cast<const uint4*>(raw_codes + kr * (BN / 2) + b * 32 + 16);
       const int bcol = n >> 6;
       const int q8 = static_cast<int8_t>(raw_q8[kr * 16 + (bcol - xq)]);
-      const long long blk = static_cast<long long>(k0 + kr - sg.row_begin) * cpr + bcol;
-      const float mh = __fadd_rn(__fmul_rn(static_cast<float>(q8), __ldg(sg.scales + (blk >> 8))), mean);
+      const float mh = __fadd_rn(__fmul_rn(static_cast<float>(q8), s2[i]), mean);
       const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
       const BlockLut t = block_lut(cb, mh);
 #pragma unroll
@@ -533,9 +568,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
   if (warp < 8) {
     // ------------------------------------------------ producers (two groups, alternate k-blocks)
     const int grp = warp >> 2, gtid = threadIdx.x & (GROUP_THREADS - 1);
-    float cb[16];
-#pragma unroll
-    for (int j = 0; j < 16; ++j) cb[j] = p.lut[j];
+    const float(&cb)[16] = p.lut;  // kernel-parameter (constant bank) operands, no registers
     int g = 0;
     for (int s = 0; s < p.nseg; ++s) {
       const GemmSeg& sg = p.seg[s];
@@ -553,14 +586,20 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
         const uint8_t* Rc = Bs + C::B_BYTES;
         const uint8_t* Rq = Rc + C::RAW_CODE_BYTES;
         if (raw) {
-          // raw codes / absmax of this k-block have landed (the issuer waited for the slot)
-          mbar_wait_bounded(&raw_full[st], ph, abort_flag, p.err);
           if (sg.B.kind == OP_NF4_K) {
-            decode_fwd_raw<BN>(p.nf4, nf4_seg_of(p.nf4, n0), cb, seg_mean, n0, p.N, kk, Rc, Rq, Bs, gtid);
+            const int si = nf4_seg_of(p.nf4, n0);
+            float s2[(BN + GROUP_THREADS - 1) / GROUP_THREADS];
+            fwd_scales<BN>(p.nf4, si, n0, p.N, kk, gtid, s2);
+            // raw codes / absmax of this k-block have landed (the issuer waited for the slot)
+            mbar_wait_bounded(&raw_full[st], ph, abort_flag, p.err);
+            decode_fwd_raw<BN>(p.nf4, si, cb, seg_mean, n0, p.N, kk, Rc, Rq, Bs, gtid, s2);
           } else {
             const int k0 = kk * BK;
-            decode_dx_raw<BN>(p.nf4, nf4_seg_of(p.nf4, k0), cb, seg_mean, n0, p.N, k0, ((n0 >> 6) >> 4) << 4, Rc,
-                              Rq, Bs, gtid);
+            const int si = nf4_seg_of(p.nf4, k0);
+            float s2[(64 * (BN / 64) + GROUP_THREADS - 1) / GROUP_THREADS];
+            dx_scales<BN>(p.nf4, si, n0, p.N, k0, gtid, s2);
+            mbar_wait_bounded(&raw_full[st], ph, abort_flag, p.err);
+            decode_dx_raw<BN>(p.nf4, si, cb, seg_mean, n0, p.N, k0, ((n0 >> 6) >> 4) << 4, Rc, Rq, Bs, gtid, s2);
           }
         } else {
           mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, p.err);
