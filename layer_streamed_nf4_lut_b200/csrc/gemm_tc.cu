@@ -36,8 +36,10 @@ namespace soup {
 
 namespace {
 
-constexpr int GEMM_THREADS = 384;
-constexpr int GROUPS = 2;
+constexpr int GROUPS = 3;                       // producer groups (4 warps each) on alternate k-blocks
+constexpr int PRODUCER_WARPS = 4 * GROUPS;
+constexpr int EPI_WARP0 = PRODUCER_WARPS;       // first of the 4 epilogue warps (a whole warpgroup)
+constexpr int GEMM_THREADS = 32 * (PRODUCER_WARPS + 4);
 constexpr int GROUP_THREADS = 128;
 constexpr int BM = 128;
 constexpr int BK = 64;  // 64 bf16 = 128 bytes = one swizzle row
@@ -231,7 +233,7 @@ __device__ __forceinline__ void load_tile(const Operand& op, const NF4Group& g, 
                                           int gtid) {
   if (op.kind == OP_NF4_K) {
     constexpr int CH = ROWS * 8 / GROUP_THREADS;
-    constexpr int BATCH = CH < 8 ? CH : 8;  // chunks gathered before any is decoded
+    constexpr int BATCH = CH < 4 ? CH : 4;  // chunks gathered before any is decoded
 #pragma unroll
     for (int b0 = 0; b0 < CH; b0 += BATCH) {
       NF4Raw raw[BATCH];
@@ -252,7 +254,7 @@ __device__ __forceinline__ void load_tile(const Operand& op, const NF4Group& g, 
     }
   } else if (op.kind == OP_NF4_MN) {
     constexpr int U = (ROWS / 8) * 32 / GROUP_THREADS;
-    constexpr int BATCH = U < 4 ? U : 4;
+    constexpr int BATCH = U < 2 ? U : 2;
 #pragma unroll
     for (int b0 = 0; b0 < U; b0 += BATCH) {
       NF4Raw r0[BATCH], r1[BATCH];
@@ -308,6 +310,21 @@ __device__ __forceinline__ uint4 decode_word(uint32_t c, float mh, const float* 
   o.z = pack_bf16x2(__fmul_rn(lut[(c >> 16) & 15u], mh), __fmul_rn(lut[(c >> 20) & 15u], mh));
   o.w = pack_bf16x2(__fmul_rn(lut[(c >> 24) & 15u], mh), __fmul_rn(lut[c >> 28], mh));
   return o;
+}
+
+// Explicit shared-space accesses for the decode path (32-bit shared addresses).
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ int lds_s8(uint32_t a) {
+  int v;
+  asm volatile("ld.shared.s8 %0, [%1];" : "=r"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ void sts128(uint32_t a, const uint4& v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
 }
 
 // PTX byte permute in its default mode: each selector nibble's low 3 bits pick one of the 8
@@ -403,19 +420,20 @@ __device__ __forceinline__ void decode_fwd_raw(const NF4Group& g, int s, const f
   for (int i = 0; i < (BN + GROUP_THREADS - 1) / GROUP_THREADS; ++i) {
     const int r = gtid + i * GROUP_THREADS;
     if (r >= BN) break;
+    const uint32_t trow = smem_u32(tile) + (r >> 3) * 1024 + (r & 7) * 128;
     if (n0 + r < N) {
-      const uint4 w0 = *reinterpret_cast<const uint4*>(raw_codes + r * 32);
-      const uint4 w1 = *reinterpret_cast<const uint4*>(raw_codes + r * 32 + 16);
-      const int q8 = static_cast<int8_t>(raw_q8[r * 16 + (kbw & 15)]);
+      const uint32_t rc = smem_u32(raw_codes) + r * 32;
+      const uint4 w0 = lds128(rc);
+      const uint4 w1 = lds128(rc + 16);
+      const int q8 = lds_s8(smem_u32(raw_q8) + r * 16 + (kbw & 15));
       const float mh = __fadd_rn(__fmul_rn(static_cast<float>(q8), s2[i]), mean);
       const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
       const BlockLut t = block_lut(cb, mh);
 #pragma unroll
-      for (int kc = 0; kc < 8; ++kc)
-        *reinterpret_cast<uint4*>(tile + swz_off(r, kc)) = decode_word_lut(words[kc], t);
+      for (int kc = 0; kc < 8; ++kc) sts128(trow + ((kc ^ (r & 7)) << 4), decode_word_lut(words[kc], t));
     } else {
 #pragma unroll
-      for (int kc = 0; kc < 8; ++kc) *reinterpret_cast<uint4*>(tile + swz_off(r, kc)) = make_uint4(0, 0, 0, 0);
+      for (int kc = 0; kc < 8; ++kc) sts128(trow + ((kc ^ (r & 7)) << 4), make_uint4(0, 0, 0, 0));
     }
   }
 }
@@ -437,21 +455,21 @@ __device__ __forceinline__ void decode_dx_raw(const NF4Group& g, int s, const fl
     if (u >= 64 * NB) break;
     const int kr = u / NB, b = u % NB;
     const int n = n0 + b * 64;
-    uint8_t* dst = tile + b * 8192 + (kr >> 3) * 1024 + (kr & 7) * 128;
+    const uint32_t dst = smem_u32(tile) + b * 8192 + (kr >> 3) * 1024 + (kr & 7) * 128;
     if (n < N) {
-      const uint4 w0 = *reinterpret_cast<const uint4*>(raw_codes + kr * (BN / 2) + b * 32);
-      const uint4 w1 = *reinterpret_cast<const uint4*>(raw_codes + kr * (BN / 2) + b * 32 + 16);
+      const uint32_t rc = smem_u32(raw_codes) + kr * (BN / 2) + b * 32;
+      const uint4 w0 = lds128(rc);
+      const uint4 w1 = lds128(rc + 16);
       const int bcol = n >> 6;
-      const int q8 = static_cast<int8_t>(raw_q8[kr * 16 + (bcol - xq)]);
+      const int q8 = lds_s8(smem_u32(raw_q8) + kr * 16 + (bcol - xq));
       const float mh = __fadd_rn(__fmul_rn(static_cast<float>(q8), s2[i]), mean);
       const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
       const BlockLut t = block_lut(cb, mh);
 #pragma unroll
-      for (int nc = 0; nc < 8; ++nc)
-        *reinterpret_cast<uint4*>(dst + ((nc ^ (kr & 7)) << 4)) = decode_word_lut(words[nc], t);
+      for (int nc = 0; nc < 8; ++nc) sts128(dst + ((nc ^ (kr & 7)) << 4), decode_word_lut(words[nc], t));
     } else {
 #pragma unroll
-      for (int nc = 0; nc < 8; ++nc) *reinterpret_cast<uint4*>(dst + ((nc ^ (kr & 7)) << 4)) = make_uint4(0, 0, 0, 0);
+      for (int nc = 0; nc < 8; ++nc) sts128(dst + ((nc ^ (kr & 7)) << 4), make_uint4(0, 0, 0, 0));
     }
   }
 }
@@ -548,7 +566,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
   }
   if (threadIdx.x < 16) lut[threadIdx.x] = p.lut[threadIdx.x];
   if (threadIdx.x >= 32 && threadIdx.x < 32 + p.nf4.nseg) seg_mean[threadIdx.x - 32] = *p.nf4.seg[threadIdx.x - 32].mean;
-  if (warp == 8) {
+  if (warp == EPI_WARP0) {
     tmem_alloc(tmem_slot, BN);
     tmem_relinquish();
   }
@@ -565,7 +583,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
   const int kb_lo = static_cast<int>(static_cast<long long>(blockIdx.z) * nkb_all / splits);
   const int kb_hi = static_cast<int>(static_cast<long long>(blockIdx.z + 1) * nkb_all / splits);
 
-  if (warp < 8) {
+  if (warp < PRODUCER_WARPS) {
     // ------------------------------------------------ producers (two groups, alternate k-blocks)
     const int grp = warp >> 2, gtid = threadIdx.x & (GROUP_THREADS - 1);
     const float(&cb)[16] = p.lut;  // kernel-parameter (constant bank) operands, no registers
@@ -612,7 +630,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
       }
     }
   } else {
-    if (warp == 9 && lane == 0) {
+    if (warp == EPI_WARP0 + 1 && lane == 0) {
       // ------------------------------------------------ TMA issuer: A tiles and raw NF4 codes / absmax
       int g = 0;
       for (int s = 0; s < p.nseg; ++s) {
@@ -671,7 +689,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
         }
       }
     }
-    if (warp == 8 && lane == 0) {
+    if (warp == EPI_WARP0 && lane == 0) {
       // ------------------------------------------------ MMA issuer
       int g = 0, kb = 0;
       for (int s = 0; s < p.nseg; ++s) {
@@ -703,7 +721,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
     }
     __syncwarp();
     // ------------------------------------------------ epilogue (warps 8..11 = TMEM lane quarters 0..3)
-    const int q = warp - 8;
+    const int q = warp - EPI_WARP0;
     mbar_wait_bounded(done, 0u, abort_flag, p.err);
     tc_fence_after();
     const bool any_k = kb_hi > kb_lo;
@@ -736,7 +754,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 8) {
+  if (warp == EPI_WARP0) {
     tc_fence_after();
     tmem_dealloc(tmem, BN);
   }
