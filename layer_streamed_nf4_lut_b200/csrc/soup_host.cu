@@ -22,6 +22,7 @@
 #include <string>
 #include <vector>
 #include <algorithm>
+#include <unordered_map>
 
 namespace soup {
 namespace {
@@ -239,6 +240,29 @@ struct soup_model {
   float* host_scal = nullptr;      // pinned 2-word staging for the loss + error readback
 
   std::vector<void*> dev_allocs;
+  // per-layer CUDA graphs of the step's layer calls (key: direction, layer, weight buffer,
+  // activation buffers, shapes, LoRA flag)
+  struct GraphKey {
+    int dir, layer, B, S, lora, pad;
+    const void *base, *in, *out;
+    bool operator==(const GraphKey& o) const { return std::memcmp(this, &o, sizeof(GraphKey)) == 0; }
+  };
+  struct GraphKeyHash {
+    size_t operator()(const GraphKey& k) const {
+      const unsigned long long* w = reinterpret_cast<const unsigned long long*>(&k);
+      unsigned long long h = 1469598103934665603ull;
+      for (size_t i = 0; i < sizeof(GraphKey) / 8; ++i) h = (h ^ w[i]) * 1099511628211ull;
+      return static_cast<size_t>(h);
+    }
+  };
+  struct GraphEntry {
+    cudaGraphExec_t exec = nullptr;
+    int seen = 0;
+    long long launches = 0;
+  };
+  std::unordered_map<GraphKey, GraphEntry, GraphKeyHash> graphs;
+  cudaStream_t cap_stream = nullptr;
+  int use_graphs = 1;
   // live profile: event pairs per launch, resolved into per-category totals
   int prof = 0;
   struct ProfRec {
@@ -868,6 +892,71 @@ soup_status head_backward(soup_model* m, const uint16_t* x, int B, int S, uint16
   return SOUP_OK;
 }
 
+// One layer call of a step, replayed from a CUDA graph once its key has been seen twice (the
+// first run is eager so every kernel attribute and TMA descriptor exists before capture).
+soup_status run_layer(soup_model* m, int dir, int i, const uint8_t* base, const uint16_t* in, uint16_t* out, int B,
+                      int S, cudaStream_t st) {
+  const LayerView v = view_of(m, base);
+  if (!m->use_graphs || m->prof) {
+    return dir == 0 ? layer_forward(m, i, v, in, out, B, S, st) : layer_backward(m, i, v, in, out, B, S, st);
+  }
+  Saved& A = m->saved[i];
+  const int lora = (dir == 0) ? ((m->lora_enabled && m->lora_p) ? 1 : 0) : A.lora;
+  if (dir == 1 && (!A.valid || A.B != B || A.S != S)) {
+    m->err = "layer_bwd: no matching forward for layer " + std::to_string(i);
+    return SOUP_ERR_STATE;
+  }
+  soup_model::GraphKey key;
+  std::memset(&key, 0, sizeof(key));
+  key.dir = dir;
+  key.layer = i;
+  key.B = B;
+  key.S = S;
+  key.lora = lora;
+  key.base = base;
+  key.in = in;
+  key.out = out;
+  soup_model::GraphEntry& e = m->graphs[key];
+  if (!e.exec && e.seen == 0) {
+    e.seen = 1;
+    return dir == 0 ? layer_forward(m, i, v, in, out, B, S, st) : layer_backward(m, i, v, in, out, B, S, st);
+  }
+  if (!e.exec) {
+    const long long l0 = g_kernel_launches.load();
+    SOUP_CK(cudaStreamBeginCapture(m->cap_stream, cudaStreamCaptureModeThreadLocal));
+    soup_status s = dir == 0 ? layer_forward(m, i, v, in, out, B, S, m->cap_stream)
+                             : layer_backward(m, i, v, in, out, B, S, m->cap_stream);
+    cudaGraph_t g = nullptr;
+    const cudaError_t ce = cudaStreamEndCapture(m->cap_stream, &g);
+    e.launches = g_kernel_launches.load() - l0;
+    g_kernel_launches -= e.launches;  // captured, not run
+    if (s != SOUP_OK) {
+      if (g) cudaGraphDestroy(g);
+      return s;
+    }
+    if (ce != cudaSuccess) {
+      m->err = std::string("graph capture: ") + cudaGetErrorString(ce);
+      return SOUP_ERR_CUDA;
+    }
+    const cudaError_t ie = cudaGraphInstantiate(&e.exec, g, 0);
+    cudaGraphDestroy(g);
+    if (ie != cudaSuccess) {
+      e.exec = nullptr;
+      m->err = std::string("graph instantiate: ") + cudaGetErrorString(ie);
+      return SOUP_ERR_CUDA;
+    }
+  }
+  SOUP_CK(cudaGraphLaunch(e.exec, st));
+  g_kernel_launches += e.launches;
+  if (dir == 0) {
+    A.B = B;
+    A.S = S;
+    A.lora = lora;
+    A.valid = 1;
+  }
+  return SOUP_OK;
+}
+
 soup_status stream_forward_pass(soup_model* m, int B, int S, cudaStream_t st, uint16_t** x_final) {
   const int L = m->cfg.n_layers;
   std::vector<int> order(L);
@@ -879,8 +968,7 @@ soup_status stream_forward_pass(soup_model* m, int B, int S, cudaStream_t st, ui
     int buf;
     SOUP_TRY(streamer_acquire(m, i, st, &base, &buf));
     SOUP_TRY(streamer_prefetch(m, order, i));
-    const LayerView v = view_of(m, base);
-    SOUP_TRY(layer_forward(m, i, v, cur, nxt, B, S, st));
+    SOUP_TRY(run_layer(m, 0, i, base, cur, nxt, B, S, st));
     SOUP_TRY(streamer_release(m, buf, st));
     std::swap(cur, nxt);
   }
@@ -898,8 +986,7 @@ soup_status stream_backward_pass(soup_model* m, int B, int S, uint16_t* dcur, ui
     int buf;
     SOUP_TRY(streamer_acquire(m, i, st, &base, &buf));
     SOUP_TRY(streamer_prefetch(m, order, k));
-    const LayerView v = view_of(m, base);
-    SOUP_TRY(layer_backward(m, i, v, dcur, dnxt, B, S, st));
+    SOUP_TRY(run_layer(m, 1, i, base, dcur, dnxt, B, S, st));
     SOUP_TRY(streamer_release(m, buf, st));
     std::swap(dcur, dnxt);
   }
@@ -1007,6 +1094,12 @@ soup_status do_step(soup_model* m, soup_loss kind, const soup_batch* bt, float* 
   return SOUP_OK;
 }
 
+void clear_graphs(soup_model* m) {
+  for (auto& kv : m->graphs)
+    if (kv.second.exec) cudaGraphExecDestroy(kv.second.exec);
+  m->graphs.clear();
+}
+
 soup_status destroy_model(soup_model* m) {
   if (m->copy_stream) cudaStreamSynchronize(m->copy_stream);
   cudaDeviceSynchronize();
@@ -1019,6 +1112,8 @@ soup_status destroy_model(soup_model* m) {
   for (uint8_t* h : m->host_blob)
     if (h) cudaFreeHost(h);
   if (m->host_scal) cudaFreeHost(m->host_scal);
+  clear_graphs(m);
+  if (m->cap_stream) cudaStreamDestroy(m->cap_stream);
   for (auto& r : m->prof_pending) {
     cudaEventDestroy(r.a);
     cudaEventDestroy(r.b);
@@ -1074,6 +1169,11 @@ soup_status create_model(const soup_model_config* cfg, const soup_allocator* all
   m->buf_last.assign(nbuf, 0);
   m->buf_inuse.assign(nbuf, 0);
   if (cudaStreamCreateWithFlags(&m->copy_stream, cudaStreamNonBlocking) != cudaSuccess) return fail(SOUP_ERR_CUDA);
+  if (cudaStreamCreateWithFlags(&m->cap_stream, cudaStreamNonBlocking) != cudaSuccess) return fail(SOUP_ERR_CUDA);
+  {
+    const char* e = std::getenv("SOUP_GRAPHS");
+    m->use_graphs = (e && e[0] == '0') ? 0 : 1;
+  }
   m->copy_done.resize(nbuf);
   m->buf_free.resize(nbuf);
   for (int b = 0; b < nbuf; ++b) {
@@ -1326,6 +1426,7 @@ soup_status soup_model_set_lora(soup_model* m, float* params, float* grads, floa
     m->err = "LoRA buffers must be 16-byte aligned";
     return SOUP_ERR_INVALID_ARG;
   }
+  clear_graphs(m);
   m->lora_p = params;
   m->lora_g = grads;
   m->lora_m = adam_m;
