@@ -348,6 +348,34 @@ def adamw(p, g, m, v, t, lr, b1=0.9, b2=0.999, eps=1e-8, wd=0.0):
     return p, m, v
 
 
+def bf16_round_f64(x):
+    """float64 -> nearest bfloat16 value (ties to even) in ONE rounding, as float64.
+
+    Normal-range finite inputs; the significand keeps 8 bits (frexp mantissa in [0.5, 1))."""
+    x = np.asarray(x, dtype=np.float64)
+    m, e = np.frexp(x)
+    return np.ldexp(np.rint(m * 256.0), e - 8)
+
+
+def merge_lora(W, A, B, s):
+    """Merged weight of one projection: the base fused with its LoRA adapter.
+
+    The pages list a merge command that fuses the trained adapter into the base model
+    (guillermodelpino page, the commands of the full cycle: `soup merge --adapter`;
+    imasters page, "O que muda para quem constrói no Brasil": merging the LoRA into the
+    base).  They give no formula; the plainest reading is the LoRA identity (Hu et al.
+    2021): x W'^T = x W^T + s (x A^T) B^T for every x, i.e. W' = W + s B A, stored in the
+    working precision of the weights (bf16).  A and B enter with the precision the training
+    forward gives them (bf16 values); the sum is exact here and rounded once.
+
+    W: [out, in] dequantised base (bf16 values); A: [r, in]; B: [out, r]; s = alpha / r.
+    Returns float64 values that are bf16 numbers."""
+    from .nf4 import bf16_round
+    Ab = bf16_round(np.asarray(A, dtype=np.float32)).astype(np.float64)
+    Bb = bf16_round(np.asarray(B, dtype=np.float32)).astype(np.float64)
+    return bf16_round_f64(np.asarray(W, dtype=np.float64) + s * (Bb @ Ab))
+
+
 def _lora_of(lora, i):
     if lora is None:
         return None
