@@ -6,17 +6,19 @@
 //   * backward dx = dy W + s (dy B) A     : the same NF4 weight read transposed;
 //   * LoRA grads, lm_head forward/backward: plain bf16 / fp32 operands.
 //
-// Roles (384 threads, one CTA per 128 x BN output tile, or per K-slice of it under split-K):
-//   warps 0-7  producers, two groups of four warps that fill alternate k-blocks so that one
-//              group's global-memory latency overlaps the other's dequantisation.  A K-major
-//              bf16 A tile arrives by TMA (cp.async.bulk.tensor, 128-byte swizzle, no thread
-//              involvement); the B tile is gathered into registers first (codes, q8 absmax,
-//              group scales), then dequantised through a 16-entry shared-memory codebook and
-//              stored in the same 128-byte-swizzled K-major layout;
-//   warp 8     allocates the TMEM accumulator; lane 0 issues tcgen05.mma (M=128, N=BN, K=16)
-//              and tcgen05.commit to release stages;
-//   warps 8-11 epilogue: tcgen05.ld rows out of TMEM, scale, add residual / old value, store
-//              (or store an fp32 partial tile under split-K).
+// Roles (512 threads, one CTA per (MT*128) x BN output tile, or per K-slice of it under split-K):
+//   warps 0-11  producers, three groups of four warps that take alternate k-blocks.  On the NF4
+//               path each dequantises one B tile from raw codes / q8 absmax staged by TMA
+//               (per-absmax-block table of bf16 products in registers, byte-permute lookups)
+//               into the 128-byte-swizzled layout the MMA reads; other operands the TMA does
+//               not carry are gathered and converted here;
+//   warp 12     allocates TMEM; lane 0 issues tcgen05.mma (M=128 per half, N=BN, K=16) and
+//               tcgen05.commit to release stages;
+//   warp 13     lane 0 issues the operand TMA loads (A, bf16 B) into the stage ring;
+//   warp 14     lane 0 issues the raw NF4 TMA loads into a ring of their own, so they run
+//               ahead of the operand stages (a raw slot frees when its k-block is decoded);
+//   warps 12-15 epilogue: tcgen05.ld rows out of TMEM, scale, add residual / old value, store
+//               (or store an fp32 partial tile under split-K).
 //
 // NF4 decode follows the double-quantised format: mhat = fp32(fp32(q8 * s2) + mean),
 // w = bf16_rn(fp32(code_value * mhat)), one float32 multiply per element.
@@ -41,21 +43,30 @@ constexpr int PRODUCER_WARPS = 4 * GROUPS;
 constexpr int EPI_WARP0 = PRODUCER_WARPS;       // first of the 4 epilogue warps (a whole warpgroup)
 constexpr int GEMM_THREADS = 32 * (PRODUCER_WARPS + 4);
 constexpr int GROUP_THREADS = 128;
-constexpr int BM = 128;
-constexpr int BK = 64;  // 64 bf16 = 128 bytes = one swizzle row
+constexpr int UM = 128;  // rows of one tcgen05.mma (cta_group::1); a CTA tile stacks MT of them
+constexpr int BK = 64;   // 64 bf16 = 128 bytes = one swizzle row
+constexpr int SMEM_LIMIT = 232448;  // 227 KiB of dynamic shared memory per CTA
 
-template <int BN>
+template <int MT, int BN>
 struct GemmCfg {
+  static constexpr int BM = UM * MT;
   static constexpr int A_BYTES = BM * 128;
   static constexpr int B_BYTES = BN * 128;
-  // raw NF4 staging (TMA): codes BN x 32 B (forward) or 64 x BN/2 B (transposed), q8 absmax
-  // BN x 16 B or 64 x 16 B
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // one k-block of both MMA operands
+  // Raw NF4 staging (TMA) in a ring of its own: codes BN x 32 B (forward) or 64 x BN/2 B
+  // (transposed), q8 absmax BN x 16 B or 64 x 16 B.  A raw slot is released as soon as its
+  // k-block is dequantised, so the raw loads run several k-blocks ahead of the operand stages.
   static constexpr int RAW_CODE_BYTES = BN * 32;
   static constexpr int RAW_Q8_BYTES = (BN > 64 ? BN : 64) * 16;
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + RAW_CODE_BYTES + RAW_Q8_BYTES;
-  static constexpr int STAGES = (BN >= 256) ? 3 : (BN >= 128 ? 5 : 7);
-  static constexpr int CTRL_BYTES = 512;
-  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + CTRL_BYTES;
+  static constexpr int RAW_BYTES = RAW_CODE_BYTES + RAW_Q8_BYTES;
+  static constexpr int CTRL_BYTES = 640;
+  static constexpr int AVAIL = SMEM_LIMIT - 1024 - CTRL_BYTES;
+  static constexpr int STAGES_FIT = (AVAIL - 4 * RAW_BYTES) / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
+  static constexpr int RAW_FIT = (AVAIL - STAGES * STAGE_BYTES) / RAW_BYTES;
+  static constexpr int RAW_SLOTS = RAW_FIT > 16 ? 16 : RAW_FIT;
+  static constexpr int TMEM_COLS = MT * BN;  // one BN-column fp32 accumulator per 128-row half
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + RAW_SLOTS * RAW_BYTES + CTRL_BYTES;
 };
 
 // ---------------------------------------------------------------- tcgen05 / TMA wrappers
@@ -144,7 +155,7 @@ __device__ __forceinline__ uint32_t idesc_bf16_f32(bool a_mn_major, bool b_mn_ma
          | ((a_mn_major ? 1u : 0u) << 15)          // A major-ness
          | ((b_mn_major ? 1u : 0u) << 16)          // B major-ness
          | (static_cast<uint32_t>(BN >> 3) << 17)  // N / 8
-         | (static_cast<uint32_t>(BM >> 4) << 24); // M / 16
+         | (static_cast<uint32_t>(UM >> 4) << 24); // M / 16
 }
 
 // ---------------------------------------------------------------- operand fetch
@@ -535,21 +546,25 @@ __device__ __forceinline__ void epilogue_store8(const GemmParams& p, int row, in
 }
 
 // ---------------------------------------------------------------- the kernel
-template <int BN>
+template <int MT, int BN>
 __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_constant__ GemmParams p) {
-  using C = GemmCfg<BN>;
+  using C = GemmCfg<MT, BN>;
+  constexpr int BM = C::BM;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* base = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
-  uint8_t* ctrl = base + C::STAGES * C::STAGE_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(ctrl);
+  uint8_t* raw_base = base + C::STAGES * C::STAGE_BYTES;
+  uint8_t* ctrl = raw_base + C::RAW_SLOTS * C::RAW_BYTES;
+  float* lut = reinterpret_cast<float*>(ctrl);                       // 16 floats
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl + 64);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(ctrl + 68);
+  float* seg_mean = reinterpret_cast<float*>(ctrl + 80);              // up to 3 NF4 tensors
+  uint64_t* full = reinterpret_cast<uint64_t*>(ctrl + 128);
   uint64_t* empty = full + C::STAGES;
   uint64_t* raw_full = empty + C::STAGES;
-  uint64_t* done = raw_full + C::STAGES;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* seg_mean = reinterpret_cast<float*>(tmem_slot + 4);
-  float* lut = reinterpret_cast<float*>(ctrl + 256);
+  uint64_t* raw_empty = raw_full + C::RAW_SLOTS;
+  uint64_t* done = raw_empty + C::RAW_SLOTS;
+  static_assert(128 + 8 * (2 * C::STAGES + 2 * C::RAW_SLOTS + 1) <= C::CTRL_BYTES, "control block overflow");
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n0 = blockIdx.x * BN, m0 = blockIdx.y * BM;
@@ -558,7 +573,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full[s], GROUP_THREADS / 32 + 1);  // 4 producer warps + the TMA issuer
       mbar_init(&empty[s], 1);
-      mbar_init(&raw_full[s], 1);
+    }
+    for (int r = 0; r < C::RAW_SLOTS; ++r) {
+      mbar_init(&raw_full[r], 1);
+      mbar_init(&raw_empty[r], GROUP_THREADS / 32);  // the 4 warps of the group that decoded it
     }
     mbar_init(done, 1);
     *abort_flag = 0;
@@ -567,7 +585,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
   if (threadIdx.x < 16) lut[threadIdx.x] = p.lut[threadIdx.x];
   if (threadIdx.x >= 32 && threadIdx.x < 32 + p.nf4.nseg) seg_mean[threadIdx.x - 32] = *p.nf4.seg[threadIdx.x - 32].mean;
   if (warp == EPI_WARP0) {
-    tmem_alloc(tmem_slot, BN);
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -582,9 +600,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
   const int splits = p.splits > 1 ? p.splits : 1;
   const int kb_lo = static_cast<int>(static_cast<long long>(blockIdx.z) * nkb_all / splits);
   const int kb_hi = static_cast<int>(static_cast<long long>(blockIdx.z + 1) * nkb_all / splits);
+  // Raw-staged k-blocks (segment 0 when raw_tma) come first in the slice: local k-blocks
+  // [0, n_raw) use raw slot kb % RAW_SLOTS.
+  const bool seg0_raw = p.raw_tma && seg_active(p.seg[0], n0, BN);
+  const int seg0_nk = seg0_raw ? (p.seg[0].K + BK - 1) / BK : 0;
+  const int n_raw = seg0_raw ? max(0, min(seg0_nk, kb_hi) - kb_lo) : 0;
 
   if (warp < PRODUCER_WARPS) {
-    // ------------------------------------------------ producers (two groups, alternate k-blocks)
+    // ------------------------------------------------ producers (groups on alternate k-blocks)
     const int grp = warp >> 2, gtid = threadIdx.x & (GROUP_THREADS - 1);
     const float(&cb)[16] = p.lut;  // kernel-parameter (constant bank) operands, no registers
     int g = 0;
@@ -601,24 +624,29 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
         const uint32_t ph = static_cast<uint32_t>(kb / C::STAGES) & 1u;
         uint8_t* As = base + st * C::STAGE_BYTES;
         uint8_t* Bs = As + C::A_BYTES;
-        const uint8_t* Rc = Bs + C::B_BYTES;
-        const uint8_t* Rq = Rc + C::RAW_CODE_BYTES;
         if (raw) {
+          const int rs = kb % C::RAW_SLOTS;
+          const uint32_t rph = static_cast<uint32_t>(kb / C::RAW_SLOTS) & 1u;
+          const uint8_t* Rc = raw_base + rs * C::RAW_BYTES;
+          const uint8_t* Rq = Rc + C::RAW_CODE_BYTES;
           if (sg.B.kind == OP_NF4_K) {
             const int si = nf4_seg_of(p.nf4, n0);
             float s2[(BN + GROUP_THREADS - 1) / GROUP_THREADS];
             fwd_scales<BN>(p.nf4, si, n0, p.N, kk, gtid, s2);
-            // raw codes / absmax of this k-block have landed (the issuer waited for the slot)
-            mbar_wait_bounded(&raw_full[st], ph, abort_flag, p.err);
+            mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, p.err);
+            mbar_wait_bounded(&raw_full[rs], rph, abort_flag, p.err);
             decode_fwd_raw<BN>(p.nf4, si, cb, seg_mean, n0, p.N, kk, Rc, Rq, Bs, gtid, s2);
           } else {
             const int k0 = kk * BK;
             const int si = nf4_seg_of(p.nf4, k0);
             float s2[(64 * (BN / 64) + GROUP_THREADS - 1) / GROUP_THREADS];
             dx_scales<BN>(p.nf4, si, n0, p.N, k0, gtid, s2);
-            mbar_wait_bounded(&raw_full[st], ph, abort_flag, p.err);
+            mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, p.err);
+            mbar_wait_bounded(&raw_full[rs], rph, abort_flag, p.err);
             decode_dx_raw<BN>(p.nf4, si, cb, seg_mean, n0, p.N, k0, ((n0 >> 6) >> 4) << 4, Rc, Rq, Bs, gtid, s2);
           }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&raw_empty[rs]);  // this warp's reads of the raw slot are done
         } else {
           mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, p.err);
           if (p.b_mode[s] == 0) load_tile<BN>(sg.B, p.nf4, lut, seg_mean, sg.K, n0, p.N, kk * BK, Bs, gtid);
@@ -631,7 +659,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
     }
   } else {
     if (warp == EPI_WARP0 + 1 && lane == 0) {
-      // ------------------------------------------------ TMA issuer: A tiles and raw NF4 codes / absmax
+      // ------------------------------------------------ TMA issuer: operand tiles (A, bf16 B)
       int g = 0;
       for (int s = 0; s < p.nseg; ++s) {
         const GemmSeg& sg = p.seg[s];
@@ -646,8 +674,6 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
           mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, p.err);
           uint8_t* As = base + st * C::STAGE_BYTES;
           uint8_t* Bs = As + C::A_BYTES;
-          uint8_t* Rc = Bs + C::B_BYTES;
-          uint8_t* Rq = Rc + C::RAW_CODE_BYTES;
           const int am = p.a_mode[s], bm = raw ? 0 : p.b_mode[s];
           const uint32_t tx = (am ? C::A_BYTES : 0) + (bm ? C::B_BYTES : 0);
           if (tx) {
@@ -668,24 +694,32 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
           } else {
             mbar_arrive(&full[st]);
           }
-          if (raw) {
-            if (sg.B.kind == OP_NF4_K) {
-              const int si = nf4_seg_of(p.nf4, n0);
-              const int y = n0 - p.nf4.seg[si].row_begin;
-              mbar_arrive_expect_tx(&raw_full[st], BN * 32 + BN * 16);
-              tma_load_2d(Rc, &p.tmapCodes[si], kk * (BK / 2), y, &raw_full[st]);
-              tma_load_2d(Rq, &p.tmapQ8[si], (kk >> 4) << 4, y, &raw_full[st]);
-            } else {
-              const int k0 = kk * BK;
-              const int si = nf4_seg_of(p.nf4, k0);
-              const int y = k0 - p.nf4.seg[si].row_begin;
-              mbar_arrive_expect_tx(&raw_full[st], 64 * (BN / 2) + 64 * 16);
-              tma_load_2d(Rc, &p.tmapCodes[si], n0 / 2, y, &raw_full[st]);
-              tma_load_2d(Rq, &p.tmapQ8[si], ((n0 >> 6) >> 4) << 4, y, &raw_full[st]);
-            }
-          } else {
-            mbar_arrive(&raw_full[st]);  // keeps the stage's raw phase in step
-          }
+        }
+      }
+    }
+    if (warp == EPI_WARP0 + 2 && lane == 0 && n_raw > 0) {
+      // ------------------------------------------------ TMA issuer: raw NF4 codes / absmax
+      const GemmSeg& sg = p.seg[0];
+      for (int kb = 0; kb < n_raw; ++kb) {
+        const int kk = kb_lo + kb;  // k-block index within segment 0
+        const int rs = kb % C::RAW_SLOTS;
+        const uint32_t rph = static_cast<uint32_t>(kb / C::RAW_SLOTS) & 1u;
+        mbar_wait_bounded(&raw_empty[rs], rph ^ 1u, abort_flag, p.err);
+        uint8_t* Rc = raw_base + rs * C::RAW_BYTES;
+        uint8_t* Rq = Rc + C::RAW_CODE_BYTES;
+        if (sg.B.kind == OP_NF4_K) {
+          const int si = nf4_seg_of(p.nf4, n0);
+          const int y = n0 - p.nf4.seg[si].row_begin;
+          mbar_arrive_expect_tx(&raw_full[rs], BN * 32 + BN * 16);
+          tma_load_2d(Rc, &p.tmapCodes[si], kk * (BK / 2), y, &raw_full[rs]);
+          tma_load_2d(Rq, &p.tmapQ8[si], (kk >> 4) << 4, y, &raw_full[rs]);
+        } else {
+          const int k0 = kk * BK;
+          const int si = nf4_seg_of(p.nf4, k0);
+          const int y = k0 - p.nf4.seg[si].row_begin;
+          mbar_arrive_expect_tx(&raw_full[rs], 64 * (BN / 2) + 64 * 16);
+          tma_load_2d(Rc, &p.tmapCodes[si], n0 / 2, y, &raw_full[rs]);
+          tma_load_2d(Rq, &p.tmapQ8[si], ((n0 >> 6) >> 4) << 4, y, &raw_full[rs]);
         }
       }
     }
@@ -710,8 +744,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
 #pragma unroll
           for (int j = 0; j < BK / 16; ++j) {
             const uint64_t bd = b_mn ? sw128_mnmajor_desc(b_addr + j * 2048) : sw128_kmajor_desc(b_addr + j * 32);
-            const uint64_t ad = a_mn ? sw128_mnmajor_desc(a_addr + j * 2048) : sw128_kmajor_desc(a_addr + j * 32);
-            tc_mma_f16(tmem, ad, bd, idesc, (kb > 0 || j > 0) ? 1u : 0u);
+#pragma unroll
+            for (int h = 0; h < MT; ++h) {  // the 128-row halves share the B tile (one dequant)
+              const uint32_t ah = a_addr + h * (UM * 128);
+              const uint64_t ad = a_mn ? sw128_mnmajor_desc(ah + j * 2048) : sw128_kmajor_desc(ah + j * 32);
+              tc_mma_f16(tmem + h * BN, ad, bd, idesc, (kb > 0 || j > 0) ? 1u : 0u);
+            }
           }
           tc_commit(&empty[st]);
           ++kb;
@@ -725,11 +763,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
     mbar_wait_bounded(done, 0u, abort_flag, p.err);
     tc_fence_after();
     const bool any_k = kb_hi > kb_lo;
-    const int row = m0 + q * 32 + lane;
 #pragma unroll 1
-    for (int cc = 0; cc < BN; cc += 32) {
+    for (int hc = 0; hc < MT * BN; hc += 32) {
+      const int h = hc / BN, cc = hc % BN;
+      const int row = m0 + h * UM + q * 32 + lane;
       uint32_t r[32];
-      tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(cc), r);
+      tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(hc), r);
       tmem_ld_wait();
       if (row >= p.M) continue;
 #pragma unroll
@@ -756,7 +795,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
   __syncthreads();
   if (warp == EPI_WARP0) {
     tc_fence_after();
-    tmem_dealloc(tmem, BN);
+    tmem_dealloc(tmem, C::TMEM_COLS);
   }
 }
 
@@ -918,17 +957,19 @@ bool setup_raw_tma(GemmParams& p, int BN) {
   return true;
 }
 
-template <int BN>
-cudaError_t launch_bn(const GemmParams& p, cudaStream_t st) {
-  using C = GemmCfg<BN>;
+template <int MT, int BN>
+cudaError_t launch_tile(const GemmParams& p, cudaStream_t st) {
+  using C = GemmCfg<MT, BN>;
+  static_assert(C::STAGES >= 2, "tile too large for shared memory");
   static std::atomic<int> attr_done{0};
   if (!attr_done.load()) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    cudaError_t e =
+        cudaFuncSetAttribute(gemm_tc_kernel<MT, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_done.store(1);
   }
-  dim3 grid((p.N + BN - 1) / BN, (p.M + BM - 1) / BM, p.splits > 1 ? p.splits : 1);
-  gemm_tc_kernel<BN><<<grid, GEMM_THREADS, C::SMEM_BYTES, st>>>(p);
+  dim3 grid((p.N + BN - 1) / BN, (p.M + C::BM - 1) / C::BM, p.splits > 1 ? p.splits : 1);
+  gemm_tc_kernel<MT, BN><<<grid, GEMM_THREADS, C::SMEM_BYTES, st>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || p.splits <= 1) return e;
   const long long work = static_cast<long long>(p.M) * (p.N / 8);
@@ -988,7 +1029,28 @@ cudaError_t gemm_launch(const GemmParams& p_in, cudaStream_t st) {
     if (sg.B.kind == OP_NF4_MN && (p.nf4.cols % 8 != 0 || p.N > p.nf4.cols)) return cudaErrorInvalidValue;
     nkb += (sg.K + BK - 1) / BK;
   }
-  const int BN = (p.N <= 64) ? 64 : ((p.N <= 128 || static_cast<long long>((p.N + 255) / 256) * ((p.M + 127) / 128) < 148) ? 128 : 256);
+  // Tile choice: MT 128-row halves x BN columns.  Time ~ waves x per-tile time, with the per-tile
+  // time proportional to the k-blocks and a per-k-block cost measured on B200 for each tile
+  // shape (NF4 GEMMs at M = 512 and 2048): 2x128 50, 1x256 60, 1x128 38, 2x64 47, 1x64 36.
+  const int cand[5][2] = {{2, 128}, {1, 256}, {1, 128}, {2, 64}, {1, 64}};
+  const double unit[5] = {50.0, 60.0, 38.0, 47.0, 36.0};
+  int MT = 1, BN = 128;
+  double best = 1e300;
+  for (int ci = 0; ci < 5; ++ci) {
+    const int mt = cand[ci][0], bn = cand[ci][1];
+    if (mt == 2 && p.M <= UM) continue;
+    if (bn > 64 && p.N <= 64) continue;
+    if (bn > 128 && p.N <= 128) continue;
+    const long long tl = static_cast<long long>((p.N + bn - 1) / bn) * ((p.M + UM * mt - 1) / (UM * mt));
+    const long long waves = (tl + 147) / 148;
+    const double cost = static_cast<double>(waves) * (static_cast<double>(nkb) + 2.0) * unit[ci];
+    if (cost < best * 0.999) {
+      best = cost;
+      MT = mt;
+      BN = bn;
+    }
+  }
+  const int BM = UM * MT;
   p.bn = BN;
   p.raw_tma = setup_raw_tma(p, BN) ? 1 : 0;
   if (tma_operands_allowed()) {
@@ -1030,12 +1092,10 @@ cudaError_t gemm_launch(const GemmParams& p_in, cudaStream_t st) {
     p.splits = static_cast<int>(sp < 1 ? 1 : sp);
   }
   cudaError_t e;
-  if (BN == 64)
-    e = launch_bn<64>(p, st);
-  else if (BN == 128)
-    e = launch_bn<128>(p, st);
+  if (MT == 2)
+    e = (BN == 64) ? launch_tile<2, 64>(p, st) : launch_tile<2, 128>(p, st);
   else
-    e = launch_bn<256>(p, st);
+    e = (BN == 64) ? launch_tile<1, 64>(p, st) : (BN == 128 ? launch_tile<1, 128>(p, st) : launch_tile<1, 256>(p, st));
   ++g_kernel_launches;
   return e;
 }
