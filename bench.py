@@ -40,6 +40,19 @@ WORKLOADS = {
     "llama8b-sft-b4-s512-zipf-masked": dict(cfg=synth.L8B_B4, B=4, S=512, loss="sft", zipf=True, mask=True),
     "llama8b-dpo-2pairs-s512": dict(cfg=synth.L8B_DPO, B=4, S=512, loss="dpo", n_pairs=2, prefix_len=256,
                                     beta=0.1),
+    # same DPO step, each layer loaded once for the reference and the policy forward
+    "llama8b-dpo-2pairs-s512-shared-load": dict(cfg=synth.L8B_DPO, B=4, S=512, loss="dpo", n_pairs=2,
+                                                prefix_len=256, beta=0.1, dpo_shared_load=True),
+    # the other preference losses on the same batch shape (KTO: 4 unpaired rows, 2 desirable)
+    "llama8b-kto-4seq-s512": dict(cfg=synth.L8B_DPO, B=4, S=512, loss="kto", n_pairs=2, prefix_len=256, beta=0.1,
+                                  labels=(1, 0, 1, 0)),
+    "llama8b-simpo-2pairs-s512": dict(cfg=synth.L8B_DPO, B=4, S=512, loss="simpo", n_pairs=2, prefix_len=256,
+                                      beta=2.0, gamma=0.5),
+    "llama8b-orpo-2pairs-s512": dict(cfg=synth.L8B_DPO, B=4, S=512, loss="orpo", n_pairs=2, prefix_len=256,
+                                     lambda_or=0.1),
+    # the same SFT step with the layer stack in a file (stream_source = file), read through
+    # page-locked staging slots
+    "llama8b-sft-b1-s512-file": dict(cfg=synth.L8B, B=1, S=512, loss="sft", source="file"),
     "llama70b-sft-b1-s2048": dict(cfg=synth.L70B, B=1, S=2048, loss="sft"),
     "tiny-sft-b1-s64": dict(cfg=synth.TINY, B=1, S=64, loss="sft"),
 }
@@ -63,7 +76,7 @@ def step_flops(cfg, B, S, loss):
     p_layer = h * hq * d + 2 * h * hkv * d + hq * d * h + 3 * h * I
     io = (h + hq * d) + 2 * (h + hkv * d) + (hq * d + h) + 2 * (h + I) + (I + h)
     train = L * (4 * p_layer + 6 * r * io + 6 * S * d * hq) * T + 4 * h * V * T
-    if loss == "dpo":  # plus the LoRA-off reference forward
+    if loss in ("dpo", "kto"):  # plus the LoRA-off reference forward
         train += L * (2 * p_layer + 2 * S * d * hq) * T + 2 * h * V * T
     return float(train)
 
@@ -128,7 +141,18 @@ def build_model(wl, device_index, seed, mode="streamed"):
     cfg = dict(wl["cfg"])
     B, S = wl["B"], wl["S"]
     dev = torch.device("cuda", device_index)
-    gm = SoupModel(cfg, mode=mode, n_layer_buffers=2, max_tokens=B * S, device=device_index)
+    source = wl.get("source", "ram") if mode == "streamed" else "ram"
+    path = None
+    if source == "file":
+        import tempfile
+        import atexit
+        import shutil
+        d = tempfile.mkdtemp(prefix="soup_stack_", dir=os.environ.get("SOUP_STACK_DIR"))
+        atexit.register(shutil.rmtree, d, True)
+        path = os.path.join(d, "stack.soup")
+    gm = SoupModel(cfg, mode=mode, n_layer_buffers=2, max_tokens=B * S, device=device_index, source=source,
+                   stack_path=path)
+    gm.stack_path = path
     ones = torch.ones(cfg["hidden"], dtype=torch.bfloat16, device=dev)
     for i in range(cfg["n_layers"]):
         w = {}
@@ -156,7 +180,7 @@ def build_model(wl, device_index, seed, mode="streamed"):
 
 def make_batch(wl, seed):
     cfg = dict(wl["cfg"], batch=wl["B"], seq=wl["S"])
-    if wl["loss"] == "dpo":
+    if wl["loss"] != "sft":
         ids = synth.preference_batch(dict(cfg, n_pairs=wl["n_pairs"], prefix_len=wl["prefix_len"]), seed)
         return ids, None
     ids = synth.token_batch(cfg, seed, zipf=wl.get("zipf", False))
@@ -179,13 +203,20 @@ def run_soup(args, wl, rank, world, local_rank):
     ids = torch.from_numpy(ids_np).to(dev)
     mask = torch.from_numpy(mask_np).to(dev) if mask_np is not None else None
     kw = dict(loss=wl["loss"], mask=mask, n_pairs=wl.get("n_pairs", 0), prefix_len=wl.get("prefix_len", 0),
-              beta=wl.get("beta", 0.1), lr=2e-5)
+              beta=wl.get("beta", 0.1), lr=2e-5, dpo_shared_load=wl.get("dpo_shared_load", False),
+              gamma=wl.get("gamma", 0.0), lambda_or=wl.get("lambda_or", 0.1),
+              labels=np.array(wl["labels"], np.uint8) if "labels" in wl else None)
     setup_s = time.time() - t_setup
 
+    labels_np = kw.pop("labels")
+    labels_dev = torch.from_numpy(labels_np).to(dev) if labels_np is not None else None
+
     def one_step(ids_arg, mask_arg):
+        # labels (KTO) live where the ids live
+        lab = labels_dev if (isinstance(ids_arg, torch.Tensor) and ids_arg.is_cuda) else labels_np
         if world == 1:
-            return gm.step(ids_arg, **dict(kw, mask=mask_arg), apply_optimizer=True)
-        loss, _ = dp.dp_step(lambda: gm.step(ids_arg, **dict(kw, mask=mask_arg), apply_optimizer=False),
+            return gm.step(ids_arg, **dict(kw, mask=mask_arg, labels=lab), apply_optimizer=True)
+        loss, _ = dp.dp_step(lambda: gm.step(ids_arg, **dict(kw, mask=mask_arg, labels=lab), apply_optimizer=False),
                              gm.lora_grads, lambda: gm.optimizer_step(2e-5))
         return loss
 
@@ -214,6 +245,7 @@ def run_soup(args, wl, rank, world, local_rank):
     tok_s = world * T * args.steps / (ms * 1e-3)
     loads_per_step = st["layer_loads"] / args.steps
     launches = st["kernel_launches"]
+    file_gbs = (st["file_bytes_read"] / (st["file_read_ms"] * 1e-3) / 1e9) if st.get("file_read_ms") else None
 
     # profiled pass (separate from the timed one): per-kernel device time from CUDA events
     gm.set_profiling(True)
@@ -248,12 +280,12 @@ def run_soup(args, wl, rank, world, local_rank):
         torch.cuda.empty_cache()
         gr = build_model(wl, local_rank, seed=1234, mode="resident")
         for _ in range(2):
-            gr.step(ids, **kw, apply_optimizer=True)
+            gr.step(ids, **kw, labels=labels_dev, apply_optimizer=True)
         torch.cuda.synchronize(dev)
         c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         c0.record(stream)
         for _ in range(args.steps):
-            gr.step(ids, **kw, apply_optimizer=True)
+            gr.step(ids, **kw, labels=labels_dev, apply_optimizer=True)
         c1.record(stream)
         c1.synchronize()
         compute_ms = c0.elapsed_time(c1) / args.steps
@@ -294,7 +326,7 @@ def run_soup(args, wl, rank, world, local_rank):
                            "tflops": round(v["flops"] / (v["total_ms"] * 1e-3) / 1e12, 1) if v["flops"] else None,
                            "gbs": round(v["bytes"] / (v["total_ms"] * 1e-3) / 1e9, 1)}
                        for k, v in sorted(prof.items(), key=lambda kv: -kv[1]["total_ms"])}
-    ids_bytes = T * 4 + (T if mask_np is not None else 0)
+    ids_bytes = T * 4 + (T if mask_np is not None else 0) + (B if labels_np is not None else 0)
     out = {
         "metric": METRIC, "value": round(tok_s, 2), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 3), "higher_is_better": True, "scaling": "weak",
@@ -308,7 +340,9 @@ def run_soup(args, wl, rank, world, local_rank):
                           "frac": round(tok_s / world / roof_tok_s, 4), "h2d_gbs_measured": round(h2d_gbs, 2),
                           "stream_bytes_per_step": int(stream_bytes), "layer_loads_per_step": loads_per_step,
                           "flops_per_step": flops, "bf16_peak_tflops": pk["bf16_sustained"],
-                          "achieved_h2d_gbs_in_step": round(h2d["bytes"] / (h2d["total_ms"] * 1e-3) / 1e9, 2) if h2d else None},
+                          "achieved_h2d_gbs_in_step": round(h2d["bytes"] / (h2d["total_ms"] * 1e-3) / 1e9, 2) if h2d else None,
+                          "stream_source": "file" if st.get("stream_source") == 1 else "ram",
+                          "file_read_gbs_in_step": round(file_gbs, 2) if file_gbs else None},
         "compute_only_ms_per_step": round(compute_ms, 3) if compute_ms else None,
         "roofline": roofline,
         "profile": profile_summary,
@@ -374,7 +408,7 @@ def cpu_baseline(wl, budget_layers=1):
     t_layer = min(layer_once() for _ in range(budget_layers))
     t_head = head_once()
     L = wl["cfg"]["n_layers"]
-    mult = 1.5 if wl["loss"] == "dpo" else 1.0  # DPO adds a forward-only pass (~1/3 of fwd+bwd)
+    mult = 1.5 if wl["loss"] in ("dpo", "kto") else 1.0  # the reference adds a forward-only pass (~1/3 of fwd+bwd)
     t_step = L * t_layer * mult + t_head
     T = wl["B"] * wl["S"]
     return {"value": round(T / t_step, 4), "unit": "tokens/s", "cores": threads_used(), "host_cpus": os.cpu_count(),
@@ -387,7 +421,7 @@ def run_reference(args, wl):
     layer_once, head_once = oracle_sample(wl)
     t_head = head_once()
     L = wl["cfg"]["n_layers"]
-    mult = 1.5 if wl["loss"] == "dpo" else 1.0
+    mult = 1.5 if wl["loss"] in ("dpo", "kto") else 1.0
     for _ in range(args.warmup):
         layer_once()
     times = [layer_once() for _ in range(args.steps)]

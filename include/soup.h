@@ -46,12 +46,21 @@ typedef int32_t soup_status;
 #define SOUP_ERR_TIMEOUT (-5)      /* a bounded wait (host event or in-kernel barrier) ran out */
 #define SOUP_ERR_DEVICE_CHECK (-6) /* a kernel's bounds check fired (e.g. token id >= vocab) */
 #define SOUP_ERR_UNSUPPORTED (-7)  /* shape outside what the kernels implement */
+#define SOUP_ERR_IO (-8)           /* the file-backed layer stack failed to read or write */
 
 typedef struct soup_model soup_model;
 
 enum { SOUP_RESIDENT = 0, SOUP_STREAMED = 1 };
+/* Where the NF4 layer stack lives on the host side (the pages' stream_source). */
+enum { SOUP_SOURCE_RAM = 0, SOUP_SOURCE_FILE = 1, SOUP_SOURCE_AUTO = 2 };
 enum { SOUP_PROJ_Q = 0, SOUP_PROJ_K, SOUP_PROJ_V, SOUP_PROJ_O, SOUP_PROJ_GATE, SOUP_PROJ_UP, SOUP_PROJ_DOWN, SOUP_N_PROJ };
-typedef enum { SOUP_LOSS_SFT = 0, SOUP_LOSS_DPO = 1 } soup_loss;
+typedef enum {
+  SOUP_LOSS_SFT = 0,
+  SOUP_LOSS_DPO = 1,
+  SOUP_LOSS_KTO = 2,   /* reference from the LoRA-off re-stream, like DPO */
+  SOUP_LOSS_ORPO = 3,  /* reference-free */
+  SOUP_LOSS_SIMPO = 4  /* reference-free */
+} soup_loss;
 
 /* Model shape and run options.  Decoder layer = pre-norm Llama block (RMSNorm, GQA attention
  * with rotate-half RoPE, SwiGLU MLP), LoRA on all seven projections with scale alpha/r. */
@@ -64,6 +73,13 @@ typedef struct soup_model_config {
   int n_layer_buffers; /* streamed: device layer buffers, >= 2 (the resident-layer budget) */
   int max_tokens;      /* largest B*S any call will use (sizes the activation storage) */
   int device;          /* CUDA device ordinal */
+  int stream_source;   /* SOUP_SOURCE_RAM (0): page-locked host RAM, one blob per layer.
+                          SOUP_SOURCE_FILE: one file at stack_path (created / truncated by
+                          soup_model_create), layer i at i * stride (blob bytes rounded up to
+                          4096); a reader thread fills n_layer_buffers page-locked staging
+                          slots ahead of the copies.  SOUP_SOURCE_AUTO: RAM if the stack fits in
+                          half the host's free physical memory, else FILE (needs stack_path). */
+  const char* stack_path; /* FILE / AUTO: path of the layer stack file; may be NULL for RAM */
 } soup_model_config;
 
 /* Optional device allocator (e.g. routed to PyTorch's caching allocator).  alloc returns
@@ -83,16 +99,28 @@ typedef struct soup_stats {
   long long device_bytes;     /* device bytes the model holds (weights buffers, activations, scratch) */
   long long pinned_bytes;     /* page-locked host bytes holding the NF4 layer stack */
   long long steps;            /* completed soup_step calls */
+  long long file_bytes_read;  /* file source: bytes read from the stack file into staging */
+  double file_read_ms;        /* file source: wall time of those reads (reader thread) */
+  int stream_source;          /* the source in use: SOUP_SOURCE_RAM or SOUP_SOURCE_FILE */
 } soup_stats;
 
 /* One training batch.  Token ids are [B, S] row-major int32.
  * SFT: row t = (b, s) predicts ids[b, s+1]; targets are positions j >= 1 of each sequence,
  *      optionally filtered by loss_mask[b, j] != 0 (uint8 [B, S]); loss = token mean.
- * DPO: B = 2 * n_pairs; rows 2p (chosen) and 2p+1 (rejected); response targets are
- *      j >= prefix_len; loss = -mean_p log sigmoid(beta [(pi_c - ref_c) - (pi_r - ref_r)]),
- *      pi = summed target log-probs (fp32) with LoRA on, ref = the same with LoRA off.
- * ids_on_host != 0: ids / loss_mask are host pointers; the library copies them to the device
- *      on `stream` inside the call (pageable or pinned memory both accepted). */
+ * Preference losses act on per-sequence sums of target log-probs over the response, targets
+ * j >= max(prefix_len, 1): pi with LoRA on (fp32 sums), ref the same with LoRA off; n = S -
+ * max(prefix_len, 1) response targets per row; sigma = logistic function.
+ * DPO (Rafailov et al. 2023): B = 2 * n_pairs; rows 2p (chosen) and 2p+1 (rejected);
+ *      loss = -mean_p log sigma(beta [(pi_c - ref_c) - (pi_r - ref_r)]).
+ * SimPO (Meng et al. 2024): pairs as DPO, no reference; a = pi / n;
+ *      loss = -mean_p log sigma(beta (a_c - a_r) - gamma).
+ * ORPO (Hong et al. 2024): pairs as DPO, no reference; odds(a) = e^a / (1 - e^a);
+ *      loss = mean_p [-a_c - lambda_or log sigma(log odds(a_c) - log odds(a_r))].
+ * KTO (Ethayarajh et al. 2024): B unpaired rows, labels[b] != 0 desirable; r = pi - ref;
+ *      z0 = max(0, mean_b r_b) with no gradient through it; v_b = lambda_d sigma(beta (r_b -
+ *      z0)) if desirable, lambda_u sigma(beta (z0 - r_b)) if not; loss = mean_b (lambda_b - v_b).
+ * ids_on_host != 0: ids / loss_mask / labels are host pointers; the library copies them to
+ *      the device on `stream` inside the call (pageable or pinned memory both accepted). */
 typedef struct soup_batch {
   const int32_t* ids;
   const uint8_t* loss_mask; /* may be NULL */
@@ -102,6 +130,14 @@ typedef struct soup_batch {
   float beta;
   float lr;            /* AdamW learning rate (betas 0.9/0.999, eps 1e-8, weight decay 0) */
   int apply_optimizer; /* 0: leave gradients in the grad buffer, do not update */
+  int dpo_shared_load; /* DPO and KTO.  0: the reference forward re-streams the whole stack
+                          with LoRA off, then the policy forward streams it again (3L-2 loads
+                          from a cold streamer).  1: each layer is loaded once and runs the
+                          LoRA-off and the LoRA-on forward back to back (2L-2 loads); same bits. */
+  const uint8_t* labels; /* KTO: uint8 [B], desirable != 0 (same memory space as ids) */
+  float gamma;           /* SimPO target margin */
+  float lambda_or;       /* ORPO weight of the odds-ratio term */
+  float lambda_d, lambda_u; /* KTO weights of desirable / undesirable rows */
 } soup_batch;
 
 /* ---- lifecycle -------------------------------------------------------------------------- */
@@ -151,6 +187,18 @@ soup_status soup_model_refresh_lora(soup_model* model, void* stream);
  * gradients are skipped entirely (not multiplied by zero), which is the DPO reference model. */
 soup_status soup_set_lora_enabled(soup_model* model, int enabled);
 
+/* Merged weight of one projection: out = bf16(W + (lora_alpha / lora_r) * B * A), device bf16
+ * [out_features, in_features] row-major (the layout of the projection's NF4 tensor, q|k|v and
+ * gate|up NOT stacked), 16-byte aligned, caller-owned.  W is the dequantised NF4 base, A and
+ * B the projection's adapters (their bf16 values, as the training forward uses them); the
+ * product accumulates in fp32 and the sum is rounded once to bf16.  This is the pages' merge
+ * command, which fuses the trained adapter into the base (guillermodelpino page, the commands
+ * of the full cycle; imasters page, "O que muda para quem constrói no Brasil").  The layer is
+ * taken from the streamer like a forward does (a streamed model may load it).  Runs on
+ * `stream`.  SOUP_ERR_STATE before set_lora or before the layer has weights;
+ * SOUP_ERR_INVALID_ARG for a bad layer / proj index or a misaligned `out`. */
+soup_status soup_model_merge_lora(soup_model* model, int layer, int proj, void* out, void* stream);
+
 /* ---- layer-level calls ------------------------------------------------------------------- */
 
 /* One decoder layer forward: x_out = layer(x_in), device bf16 [B*S, hidden].  Acquires the
@@ -167,13 +215,15 @@ soup_status soup_layer_bwd(soup_model* model, int layer, const void* dy, void* d
 /* One training step: embedding, streamed forward over all layers, head and loss, streamed
  * backward, LoRA gradients (zeroed first) and, if batch->apply_optimizer, the AdamW update.
  * SFT streams 2L-2 layer loads from a cold streamer (the two top layers are reused at the
- * forward/backward turnaround); DPO adds a full LoRA-off forward pass, 3L-2 loads.  Layers
+ * forward/backward turnaround); DPO and KTO add a full LoRA-off forward pass, 3L-2 loads
+ * (2L-2 with dpo_shared_load); SimPO and ORPO stream like SFT.  Layers
  * still resident from the previous step are reused.  *loss_out (host) receives the loss
  * after the call synchronises `stream`. */
 soup_status soup_step(soup_model* model, soup_loss loss, const soup_batch* batch, float* loss_out, void* stream);
 /* AdamW update of all LoRA parameters from the grad buffer (step counter kept by the model). */
 soup_status soup_optimizer_step(soup_model* model, float lr, void* stream);
-/* Per-sequence summed target log-probs of the last DPO step (host fp32[B]): policy and ref. */
+/* Per-sequence summed target log-probs of the last preference step (host fp32[B]): policy
+ * and ref (ref is written by DPO and KTO only). */
 soup_status soup_last_logps(soup_model* model, float* pi, float* ref, int n);
 
 /* ---- single operations (each one kernel sequence, for tests and tools) ------------------- */

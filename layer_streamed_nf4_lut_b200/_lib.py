@@ -17,7 +17,9 @@ SOUP_OK = 0
 STATUS = {0: "SOUP_OK", -1: "SOUP_ERR_INVALID_ARG", -2: "SOUP_ERR_STATE", -3: "SOUP_ERR_OOM", -4: "SOUP_ERR_CUDA",
           -5: "SOUP_ERR_TIMEOUT", -6: "SOUP_ERR_DEVICE_CHECK", -7: "SOUP_ERR_UNSUPPORTED"}
 SOUP_RESIDENT, SOUP_STREAMED = 0, 1
-SOUP_LOSS_SFT, SOUP_LOSS_DPO = 0, 1
+SOUP_SOURCE_RAM, SOUP_SOURCE_FILE, SOUP_SOURCE_AUTO = 0, 1, 2
+SOUP_LOSS_SFT, SOUP_LOSS_DPO, SOUP_LOSS_KTO, SOUP_LOSS_ORPO, SOUP_LOSS_SIMPO = 0, 1, 2, 3, 4
+LOSS_KINDS = {"sft": 0, "dpo": 1, "kto": 2, "orpo": 3, "simpo": 4}
 PROJ = ("q", "k", "v", "o", "gate", "up", "down")
 
 
@@ -31,7 +33,8 @@ class ModelConfig(Structure):
     _fields_ = [("n_layers", c_int), ("hidden", c_int), ("n_heads", c_int), ("n_kv_heads", c_int),
                 ("head_dim", c_int), ("intermediate", c_int), ("vocab", c_int), ("rms_eps", c_float),
                 ("rope_theta", c_float), ("lora_r", c_int), ("lora_alpha", c_float), ("mode", c_int),
-                ("n_layer_buffers", c_int), ("max_tokens", c_int), ("device", c_int)]
+                ("n_layer_buffers", c_int), ("max_tokens", c_int), ("device", c_int), ("stream_source", c_int),
+                ("stack_path", ctypes.c_char_p)]
 
 
 ALLOC_FN = CFUNCTYPE(c_void_p, c_size_t, c_void_p)
@@ -45,7 +48,8 @@ class Allocator(Structure):
 class Stats(Structure):
     _fields_ = [("layer_loads", c_longlong), ("bytes_h2d", c_longlong), ("layer_reuses", c_longlong),
                 ("kernel_launches", c_longlong), ("device_bytes", c_longlong), ("pinned_bytes", c_longlong),
-                ("steps", c_longlong)]
+                ("steps", c_longlong), ("file_bytes_read", c_longlong), ("file_read_ms", ctypes.c_double),
+                ("stream_source", c_int)]
 
 
 class ProfileEntry(Structure):
@@ -56,7 +60,8 @@ class ProfileEntry(Structure):
 class Batch(Structure):
     _fields_ = [("ids", c_void_p), ("loss_mask", c_void_p), ("B", c_int), ("S", c_int), ("ids_on_host", c_int),
                 ("n_pairs", c_int), ("prefix_len", c_int), ("beta", c_float), ("lr", c_float),
-                ("apply_optimizer", c_int)]
+                ("apply_optimizer", c_int), ("dpo_shared_load", c_int), ("labels", c_void_p), ("gamma", c_float),
+                ("lambda_or", c_float), ("lambda_d", c_float), ("lambda_u", c_float)]
 
 
 # name -> (restype, argtypes); every function returns soup_status unless stated
@@ -74,6 +79,7 @@ SIGNATURES = {
     "soup_model_set_lora": [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p],
     "soup_set_lora_enabled": [c_void_p, c_int],
     "soup_model_refresh_lora": [c_void_p, c_void_p],
+    "soup_model_merge_lora": [c_void_p, c_int, c_int, c_void_p, c_void_p],
     "soup_layer_fwd": [c_void_p, c_int, c_void_p, c_void_p, c_int, c_int, c_void_p],
     "soup_layer_bwd": [c_void_p, c_int, c_void_p, c_void_p, c_int, c_int, c_void_p],
     "soup_step": [c_void_p, c_int, POINTER(Batch), POINTER(c_float), c_void_p],

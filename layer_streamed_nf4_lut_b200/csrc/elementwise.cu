@@ -271,7 +271,7 @@ __global__ void seq_logp_kernel(const float* __restrict__ lse, const float* __re
 // response rows so that dlogits = w * (softmax - onehot).
 __global__ void dpo_finish_kernel(const float* __restrict__ pi, const float* __restrict__ ref, int B, int S, int start,
                                   int P, float beta, float* __restrict__ loss_out, float* __restrict__ row_weight) {
-  __shared__ float wrow[64];
+  __shared__ float wrow[256];
   if (threadIdx.x == 0) {
     double loss = 0.0;
     for (int p = 0; p < P; ++p) {
@@ -284,6 +284,79 @@ __global__ void dpo_finish_kernel(const float* __restrict__ pi, const float* __r
       wrow[2 * p + 1] = static_cast<float>(dc);
     }
     loss_out[0] = static_cast<float>(loss / P);
+  }
+  __syncthreads();
+  const int j0 = start > 1 ? start : 1;
+  for (int t = threadIdx.x; t < B * S; t += blockDim.x) {
+    const int b = t / S, j = t % S + 1;
+    row_weight[t] = (j >= j0 && j < S) ? wrow[b] : 0.f;
+  }
+}
+
+// SimPO / ORPO / KTO closed forms on the per-sequence sums pi (and ref for KTO); like DPO the
+// row weights are -dL/dpi_b on the response rows.  One thread does the arithmetic in float64
+// (at most a few dozen sequences).  n = response targets per row.
+__device__ __forceinline__ double softplus_neg(double z) {  // -log sigmoid(z)
+  return (z > 0) ? log1p(exp(-z)) : (-z + log1p(exp(z)));
+}
+__device__ __forceinline__ double sigmoid_d(double z) { return 1.0 / (1.0 + exp(-z)); }
+__device__ __forceinline__ double log1mexp_d(double a) {  // log(1 - e^a), a < 0
+  return (a > -0.6931471805599453) ? log(-expm1(a)) : log1p(-exp(a));
+}
+
+__global__ void pref_finish_kernel(int kind, const float* __restrict__ pi, const float* __restrict__ ref,
+                                   const uint8_t* __restrict__ labels, int B, int S, int start, float beta,
+                                   float gamma, float lam_or, float lam_d, float lam_u, float* __restrict__ loss_out,
+                                   float* __restrict__ row_weight) {
+  __shared__ float wrow[256];
+  if (threadIdx.x == 0) {
+    const int j0 = start > 1 ? start : 1;
+    const double n = static_cast<double>(S - j0);
+    const double bt = beta;
+    double loss = 0.0;
+    if (kind == PREF_KTO) {
+      double zsum = 0.0;
+      for (int b = 0; b < B; ++b) zsum += static_cast<double>(pi[b]) - ref[b];
+      const double z0 = fmax(0.0, zsum / B);
+      for (int b = 0; b < B; ++b) {
+        const double r = static_cast<double>(pi[b]) - ref[b];
+        double dpi;
+        if (labels[b]) {
+          const double sg = sigmoid_d(bt * (r - z0));
+          loss += lam_d * (1.0 - sg);
+          dpi = -static_cast<double>(lam_d) * bt * sg * (1.0 - sg) / B;
+        } else {
+          const double sg = sigmoid_d(bt * (z0 - r));
+          loss += lam_u * (1.0 - sg);
+          dpi = static_cast<double>(lam_u) * bt * sg * (1.0 - sg) / B;
+        }
+        wrow[b] = static_cast<float>(-dpi);
+      }
+      loss /= B;
+    } else {
+      const int P = B / 2;
+      for (int p = 0; p < P; ++p) {
+        const double ac = pi[2 * p] / n, ar = pi[2 * p + 1] / n;
+        double dc, dr;
+        if (kind == PREF_SIMPO) {
+          const double z = bt * (ac - ar) - gamma;
+          loss += softplus_neg(z);
+          const double sneg = sigmoid_d(-z);
+          dc = -sneg * bt / n / P;
+          dr = sneg * bt / n / P;
+        } else {  // PREF_ORPO
+          const double z = (ac - log1mexp_d(ac)) - (ar - log1mexp_d(ar));
+          loss += -ac + lam_or * softplus_neg(z);
+          const double sneg = sigmoid_d(-z);
+          dc = (-1.0 - lam_or * sneg / (-expm1(ac))) / n / P;
+          dr = (lam_or * sneg / (-expm1(ar))) / n / P;
+        }
+        wrow[2 * p] = static_cast<float>(-dc);
+        wrow[2 * p + 1] = static_cast<float>(-dr);
+      }
+      loss /= P;
+    }
+    loss_out[0] = static_cast<float>(loss);
   }
   __syncthreads();
   const int j0 = start > 1 ? start : 1;
@@ -456,9 +529,23 @@ cudaError_t seq_logp_launch(const float* lse, const float* tgt, int B, int S, in
 cudaError_t dpo_finish_launch(const float* lse, const float* tgt, int B, int S, int resp_start, int n_pairs, float beta,
                               const float* ref_logp, float* pi_out, float* loss_out, float* row_weight,
                               cudaStream_t st) {
+  if (B < 2 || B > 256) return cudaErrorInvalidValue;
   cudaError_t e = seq_logp_launch(lse, tgt, B, S, resp_start, pi_out, st);
   if (e != cudaSuccess) return e;
   dpo_finish_kernel<<<1, 256, 0, st>>>(pi_out, ref_logp, B, S, resp_start, n_pairs, beta, loss_out, row_weight);
+  ++g_kernel_launches;
+  return cudaGetLastError();
+}
+
+cudaError_t pref_finish_launch(int kind, const float* lse, const float* tgt, int B, int S, int resp_start,
+                               const float* ref_logp, const uint8_t* labels, float beta, float gamma, float lam_or,
+                               float lam_d, float lam_u, float* pi_out, float* loss_out, float* row_weight,
+                               cudaStream_t st) {
+  if (B < 1 || B > 256) return cudaErrorInvalidValue;
+  cudaError_t e = seq_logp_launch(lse, tgt, B, S, resp_start, pi_out, st);
+  if (e != cudaSuccess) return e;
+  pref_finish_kernel<<<1, 256, 0, st>>>(kind, pi_out, ref_logp, labels, B, S, resp_start, beta, gamma, lam_or, lam_d,
+                                        lam_u, loss_out, row_weight);
   ++g_kernel_launches;
   return cudaGetLastError();
 }

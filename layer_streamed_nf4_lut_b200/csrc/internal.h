@@ -127,6 +127,11 @@ cudaError_t sft_finish_launch(const float* lse, const float* tgt, const int32_t*
 cudaError_t dpo_finish_launch(const float* lse, const float* tgt, int B, int S, int resp_start, int n_pairs, float beta,
                               const float* ref_logp, float* pi_out, float* loss_out, float* row_weight,
                               cudaStream_t st);
+enum PrefKind { PREF_KTO = 2, PREF_ORPO = 3, PREF_SIMPO = 4 };  // values of soup_loss
+cudaError_t pref_finish_launch(int kind, const float* lse, const float* tgt, int B, int S, int resp_start,
+                               const float* ref_logp, const uint8_t* labels, float beta, float gamma, float lam_or,
+                               float lam_d, float lam_u, float* pi_out, float* loss_out, float* row_weight,
+                               cudaStream_t st);
 cudaError_t seq_logp_launch(const float* lse, const float* tgt, int B, int S, int resp_start, float* out,
                             cudaStream_t st);
 cudaError_t ce_grad_launch(const float* logits, const float* lse, const int32_t* ids, const float* row_weight, int B,

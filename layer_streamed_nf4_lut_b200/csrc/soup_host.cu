@@ -12,6 +12,9 @@
 #include "../../include/soup.h"
 #include "common.cuh"
 #include "internal.h"
+#include "layer_file.h"
+
+#include <unistd.h>
 
 #include <chrono>
 #include <climits>
@@ -140,6 +143,14 @@ soup_status validate_cfg(const soup_model_config& c, std::string& why) {
     why = "config: n_heads must be a multiple of n_kv_heads";
     return SOUP_ERR_INVALID_ARG;
   }
+  if (c.stream_source < SOUP_SOURCE_RAM || c.stream_source > SOUP_SOURCE_AUTO) {
+    why = "config: stream_source must be SOUP_SOURCE_RAM, _FILE or _AUTO";
+    return SOUP_ERR_INVALID_ARG;
+  }
+  if (c.stream_source == SOUP_SOURCE_FILE && (!c.stack_path || !c.stack_path[0])) {
+    why = "config: the file source needs stack_path";
+    return SOUP_ERR_INVALID_ARG;
+  }
   if (c.head_dim != 64 && c.head_dim != 128) {
     why = "config: head_dim must be 64 or 128";
     return SOUP_ERR_UNSUPPORTED;
@@ -198,9 +209,14 @@ struct soup_model {
   int qkv_cols = 0;
   float s_lora = 0.f;
 
-  // host NF4 stack (page-locked)
+  // host NF4 stack: page-locked RAM (one blob per layer), or a file streamed through
+  // page-locked staging slots
   std::vector<uint8_t*> host_blob;
   std::vector<int> host_loaded;
+  soup::LayerFile file;
+  int use_file = 0;
+  long long file_bytes0 = 0;  // file counters at the last soup_reset_stats
+  double file_ms0 = 0.0;
   // device layer buffers
   std::vector<uint8_t*> dev_buf;   // resident: n_layers buffers; streamed: n_layer_buffers
   std::vector<int> buf_layer;      // which layer each buffer holds (-1: none / stale)
@@ -224,6 +240,7 @@ struct soup_model {
   // activations
   std::vector<soup::Saved> saved;
   // work buffers
+  uint16_t *xra = nullptr, *xrb = nullptr;  // reference-pass hidden states (DPO shared-load schedule)
   uint16_t *xa = nullptr, *xb = nullptr, *dqkv = nullptr, *dgu = nullptr, *dm = nullptr, *da = nullptr,
            *dn = nullptr, *dx1 = nullptr, *vqkv = nullptr, *vo = nullptr, *vgu = nullptr, *vd = nullptr,
            *hf = nullptr, *dh = nullptr, *dlogits = nullptr;
@@ -231,6 +248,7 @@ struct soup_model {
         *rstdf = nullptr, *pi = nullptr, *ref = nullptr;
   int32_t* ids_dev = nullptr;
   uint8_t* mask_dev = nullptr;
+  uint8_t* labels_dev = nullptr;  // KTO labels [B]
   // scalars: [0] loss (f32), [1] device error word (int)
   int* scal = nullptr;
   float* quant_scratch = nullptr;  // absmax scratch for the quantiser
@@ -559,8 +577,12 @@ soup_status streamer_ensure(soup_model* m, int layer, int protect_lo, int protec
   }
   SOUP_CK(cudaStreamWaitEvent(m->copy_stream, m->buf_free[victim], 0));
   const int pidx = prof_begin(m, m->copy_stream);
-  SOUP_CK(cudaMemcpyAsync(m->dev_buf[victim], m->host_blob[layer], m->layout.total, cudaMemcpyHostToDevice,
-                          m->copy_stream));
+  if (m->use_file) {
+    SOUP_CK(m->file.stream_layer(layer, m->dev_buf[victim], m->copy_stream));
+  } else {
+    SOUP_CK(cudaMemcpyAsync(m->dev_buf[victim], m->host_blob[layer], m->layout.total, cudaMemcpyHostToDevice,
+                            m->copy_stream));
+  }
   prof_end(m, m->copy_stream, pidx, CAT_H2D, 0.0, static_cast<double>(m->layout.total));
   SOUP_CK(cudaEventRecord(m->copy_done[victim], m->copy_stream));
   m->buf_layer[victim] = layer;
@@ -976,6 +998,36 @@ soup_status stream_forward_pass(soup_model* m, int B, int S, cudaStream_t st, ui
   return SOUP_OK;
 }
 
+// DPO with one load per layer: LoRA-off (reference) and LoRA-on (policy) forward of layer i
+// back to back.  The reference pass runs first and its saved activations are overwritten by
+// the policy pass, which is the one the backward uses.
+soup_status stream_forward_pass_shared(soup_model* m, int B, int S, cudaStream_t st, uint16_t** x_ref,
+                                       uint16_t** x_pol) {
+  const int L = m->cfg.n_layers;
+  std::vector<int> order(L);
+  for (int i = 0; i < L; ++i) order[i] = i;
+  uint16_t *pc = m->xa, *pn = m->xb, *rc = m->xra, *rn = m->xrb;
+  const int saved_enabled = m->lora_enabled;
+  for (int i = 0; i < L; ++i) {
+    const uint8_t* base;
+    int buf;
+    SOUP_TRY(streamer_acquire(m, i, st, &base, &buf));
+    SOUP_TRY(streamer_prefetch(m, order, i));
+    m->lora_enabled = 0;
+    soup_status s = run_layer(m, 0, i, base, rc, rn, B, S, st);
+    m->lora_enabled = 1;
+    if (s == SOUP_OK) s = run_layer(m, 0, i, base, pc, pn, B, S, st);
+    m->lora_enabled = saved_enabled;
+    SOUP_TRY(s);
+    SOUP_TRY(streamer_release(m, buf, st));
+    std::swap(pc, pn);
+    std::swap(rc, rn);
+  }
+  *x_ref = rc;
+  *x_pol = pc;
+  return SOUP_OK;
+}
+
 soup_status stream_backward_pass(soup_model* m, int B, int S, uint16_t* dcur, uint16_t* dnxt, cudaStream_t st) {
   const int L = m->cfg.n_layers;
   std::vector<int> order(L);
@@ -1003,6 +1055,13 @@ soup_status read_scalars(soup_model* m, cudaStream_t st, float* loss_out) {
     m->err = errw == DEVERR_TIMEOUT ? "a kernel's bounded wait timed out" : "a kernel bounds check fired";
     return errw == DEVERR_TIMEOUT ? SOUP_ERR_TIMEOUT : SOUP_ERR_DEVICE_CHECK;
   }
+  if (m->use_file) {
+    const std::string fe = m->file.take_error();
+    if (!fe.empty()) {
+      m->err = fe;
+      return SOUP_ERR_IO;
+    }
+  }
   if (loss_out) *loss_out = m->host_scal[0];
   return SOUP_OK;
 }
@@ -1022,8 +1081,14 @@ soup_status do_step(soup_model* m, soup_loss kind, const soup_batch* bt, float* 
     m->err = "batch: need B >= 1, S >= 2, B*S <= max_tokens and ids";
     return SOUP_ERR_INVALID_ARG;
   }
-  if (kind == SOUP_LOSS_DPO && (bt->n_pairs < 1 || 2 * bt->n_pairs != B || bt->prefix_len < 0 || bt->prefix_len >= S)) {
-    m->err = "DPO batch: B must be 2*n_pairs and 0 <= prefix_len < S";
+  const bool paired = kind == SOUP_LOSS_DPO || kind == SOUP_LOSS_SIMPO || kind == SOUP_LOSS_ORPO;
+  const bool needs_ref = kind == SOUP_LOSS_DPO || kind == SOUP_LOSS_KTO;
+  if (paired && (bt->n_pairs < 1 || 2 * bt->n_pairs != B || B > 256 || bt->prefix_len < 0 || bt->prefix_len >= S)) {
+    m->err = "preference batch: B must be 2*n_pairs <= 256 and 0 <= prefix_len < S";
+    return SOUP_ERR_INVALID_ARG;
+  }
+  if (kind == SOUP_LOSS_KTO && (!bt->labels || B > 256 || bt->prefix_len < 0 || bt->prefix_len >= S)) {
+    m->err = "KTO batch: labels[B] required, B <= 256 and 0 <= prefix_len < S";
     return SOUP_ERR_INVALID_ARG;
   }
   for (int i = 0; i < c.n_layers; ++i)
@@ -1041,10 +1106,27 @@ soup_status do_step(soup_model* m, soup_loss kind, const soup_batch* bt, float* 
                             bt->ids_on_host ? cudaMemcpyHostToDevice : cudaMemcpyDeviceToDevice, st));
     mask = m->mask_dev;
   }
+  if (kind == SOUP_LOSS_KTO)
+    SOUP_CK(cudaMemcpyAsync(m->labels_dev, bt->labels, static_cast<size_t>(B),
+                            bt->ids_on_host ? cudaMemcpyHostToDevice : cudaMemcpyDeviceToDevice, st));
   SOUP_CK(cudaMemsetAsync(m->lora_g, 0, m->lora_n * sizeof(float), st));
   const int saved_enabled = m->lora_enabled;
   uint16_t* xL = nullptr;
-  if (kind == SOUP_LOSS_DPO) {
+  if (needs_ref && bt->dpo_shared_load) {
+    SOUP_TRY(streamer_warm(m, 0, 2));
+    SOUP_TRY(launch(m, st, CAT_EMBED, 0, 4.0 * T * c.hidden, "embed", [&] {
+      return embed_launch(m->ids_dev, m->embed, T, c.hidden, c.vocab, m->xa, m->scal + 1, st);
+    }));
+    SOUP_TRY(launch(m, st, CAT_D2D, 0, 4.0 * T * c.hidden, "embed copy", [&] {
+      return cudaMemcpyAsync(m->xra, m->xa, static_cast<size_t>(T) * c.hidden * 2, cudaMemcpyDeviceToDevice, st);
+    }));
+    uint16_t* xR = nullptr;
+    SOUP_TRY(stream_forward_pass_shared(m, B, S, st, &xR, &xL));
+    SOUP_TRY(head_forward(m, xR, B, S, st));
+    SOUP_TRY(check_launch(m, seq_logp_launch(m->rowlse, m->rowtgt, B, S, bt->prefix_len, m->ref, st), "ref logp"));
+    SOUP_TRY(head_forward(m, xL, B, S, st));
+  } else {
+  if (needs_ref) {
     // reference: same streamed base, LoRA off
     m->lora_enabled = 0;
     SOUP_TRY(streamer_warm(m, 0, 2));
@@ -1068,14 +1150,20 @@ soup_status do_step(soup_model* m, soup_loss kind, const soup_batch* bt, float* 
   m->lora_enabled = saved_enabled;
   if (s2 != SOUP_OK) return s2;
   SOUP_TRY(head_forward(m, xL, B, S, st));
+  }
   float* loss_dev = reinterpret_cast<float*>(m->scal);
   if (kind == SOUP_LOSS_SFT) {
     SOUP_TRY(check_launch(m, sft_finish_launch(m->rowlse, m->rowtgt, m->ids_dev, B, S, mask, loss_dev, m->roww, st),
                           "sft loss"));
-  } else {
+  } else if (kind == SOUP_LOSS_DPO) {
     SOUP_TRY(check_launch(m, dpo_finish_launch(m->rowlse, m->rowtgt, B, S, bt->prefix_len, bt->n_pairs, bt->beta,
                                                m->ref, m->pi, loss_dev, m->roww, st),
                           "dpo loss"));
+  } else {
+    SOUP_TRY(check_launch(m, pref_finish_launch(static_cast<int>(kind), m->rowlse, m->rowtgt, B, S, bt->prefix_len,
+                                                m->ref, m->labels_dev, bt->beta, bt->gamma, bt->lambda_or,
+                                                bt->lambda_d, bt->lambda_u, m->pi, loss_dev, m->roww, st),
+                          "preference loss"));
   }
   uint16_t* other = (xL == m->xa) ? m->xb : m->xa;
   SOUP_TRY(head_backward(m, xL, B, S, other, st));
@@ -1111,6 +1199,7 @@ soup_status destroy_model(soup_model* m) {
   }
   for (uint8_t* h : m->host_blob)
     if (h) cudaFreeHost(h);
+  m->file.close();
   if (m->host_scal) cudaFreeHost(m->host_scal);
   clear_graphs(m);
   if (m->cap_stream) cudaStreamDestroy(m->cap_stream);
@@ -1152,10 +1241,26 @@ soup_status create_model(const soup_model_config* cfg, const soup_allocator* all
   const int L = c.n_layers;
   m->host_blob.assign(L, nullptr);
   m->host_loaded.assign(L, 0);
-  for (int i = 0; i < L; ++i) {
-    if (cudaHostAlloc(reinterpret_cast<void**>(&m->host_blob[i]), m->layout.total, cudaHostAllocDefault) != cudaSuccess)
-      return fail(SOUP_ERR_OOM);
-    m->stats.pinned_bytes += static_cast<long long>(m->layout.total);
+  m->use_file = c.stream_source == SOUP_SOURCE_FILE;
+  if (c.stream_source == SOUP_SOURCE_AUTO && c.stack_path && c.stack_path[0]) {
+    // RAM when the stack fits in half of the free physical memory, else the file
+    const double free_bytes = static_cast<double>(sysconf(_SC_AVPHYS_PAGES)) * static_cast<double>(sysconf(_SC_PAGESIZE));
+    m->use_file = static_cast<double>(m->layout.total) * L > 0.5 * free_bytes;
+  }
+  if (m->use_file) {
+    const int slots = std::max(2, c.n_layer_buffers);
+    if (!m->file.open(c.stack_path, L, m->layout.total, slots, static_cast<long long>(wait_limit_ms()), m->err)) {
+      std::fprintf(stderr, "libsoup: %s\n", m->err.c_str());
+      return fail(SOUP_ERR_IO);
+    }
+    m->stats.pinned_bytes += static_cast<long long>(m->layout.total) * slots;
+  } else {
+    for (int i = 0; i < L; ++i) {
+      if (cudaHostAlloc(reinterpret_cast<void**>(&m->host_blob[i]), m->layout.total, cudaHostAllocDefault) !=
+          cudaSuccess)
+        return fail(SOUP_ERR_OOM);
+      m->stats.pinned_bytes += static_cast<long long>(m->layout.total);
+    }
   }
   if (cudaHostAlloc(reinterpret_cast<void**>(&m->host_scal), 64, cudaHostAllocDefault) != cudaSuccess)
     return fail(SOUP_ERR_OOM);
@@ -1194,7 +1299,8 @@ soup_status create_model(const soup_model_config* cfg, const soup_allocator* all
       return fail(SOUP_ERR_OOM);
   }
   const size_t V = c.vocab;
-  if (alloc_into(m, m->xa, T * h) || alloc_into(m, m->xb, T * h) || alloc_into(m, m->dqkv, T * QKV) ||
+  if (alloc_into(m, m->xa, T * h) || alloc_into(m, m->xb, T * h) || alloc_into(m, m->xra, T * h) ||
+      alloc_into(m, m->xrb, T * h) || alloc_into(m, m->dqkv, T * QKV) ||
       alloc_into(m, m->dgu, T * 2 * I) || alloc_into(m, m->dm, T * I) || alloc_into(m, m->da, T * qd) ||
       alloc_into(m, m->dn, T * h) || alloc_into(m, m->dx1, T * h) || alloc_into(m, m->vqkv, T * 3 * r) ||
       alloc_into(m, m->vo, T * r) || alloc_into(m, m->vgu, T * 2 * r) || alloc_into(m, m->vd, T * r) ||
@@ -1202,7 +1308,7 @@ soup_status create_model(const soup_model_config* cfg, const soup_allocator* all
       alloc_into(m, m->delta, T * c.n_heads) || alloc_into(m, m->logits, T * V) || alloc_into(m, m->rowlse, T) ||
       alloc_into(m, m->rowtgt, T) || alloc_into(m, m->roww, T) || alloc_into(m, m->rstdf, T) ||
       alloc_into(m, m->pi, T) || alloc_into(m, m->ref, T) || alloc_into(m, m->ids_dev, T) ||
-      alloc_into(m, m->mask_dev, T) || alloc_into(m, m->scal, 64))
+      alloc_into(m, m->mask_dev, T) || alloc_into(m, m->labels_dev, T) || alloc_into(m, m->scal, 64))
     return fail(SOUP_ERR_OOM);
   {  // RoPE tables: angle = pos * theta^(-2i/d), computed in float64, stored as float32
     const int half = c.head_dim / 2;
@@ -1268,8 +1374,15 @@ soup_status quantize_layer(soup_model* m, int layer, const float* const w[7], co
   }
   SOUP_CK(cudaMemcpyAsync(dst + m->layout.off[7][0], ga, static_cast<size_t>(c.hidden) * 2, cudaMemcpyDeviceToDevice, st));
   SOUP_CK(cudaMemcpyAsync(dst + m->layout.off[8][0], gm, static_cast<size_t>(c.hidden) * 2, cudaMemcpyDeviceToDevice, st));
-  SOUP_CK(cudaMemcpyAsync(m->host_blob[layer], dst, m->layout.total, cudaMemcpyDeviceToHost, st));
+  std::vector<uint8_t> staged;
+  if (m->use_file) {
+    staged.resize(m->layout.total);
+    SOUP_CK(cudaMemcpyAsync(staged.data(), dst, m->layout.total, cudaMemcpyDeviceToHost, st));
+  } else {
+    SOUP_CK(cudaMemcpyAsync(m->host_blob[layer], dst, m->layout.total, cudaMemcpyDeviceToHost, st));
+  }
   SOUP_TRY(wait_stream(m, st));
+  if (m->use_file && !m->file.write(layer, staged.data(), m->err)) return SOUP_ERR_IO;
   if (stale_buf >= 0) {
     m->buf_layer[stale_buf] = -1;
     SOUP_CK(cudaEventRecord(m->buf_free[stale_buf], st));
@@ -1310,6 +1423,7 @@ const char* soup_status_string(soup_status s) {
     case SOUP_ERR_TIMEOUT: return "timed out";
     case SOUP_ERR_DEVICE_CHECK: return "device bounds check fired";
     case SOUP_ERR_UNSUPPORTED: return "unsupported shape";
+    case SOUP_ERR_IO: return "layer stack file I/O failed";
     default: return "unknown status";
   }
 }
@@ -1387,9 +1501,13 @@ soup_status soup_model_load_layer_nf4(soup_model* m, int layer, const void* blob
     return SOUP_ERR_INVALID_ARG;
   }
   SOUP_GUARD({
-    std::memcpy(m->host_blob[layer], blob, bytes);
+    if (m->use_file) {
+      if (!m->file.write(layer, blob, m->err)) return SOUP_ERR_IO;
+    } else {
+      std::memcpy(m->host_blob[layer], blob, bytes);
+    }
     if (m->cfg.mode == SOUP_RESIDENT) {
-      SOUP_CK(cudaMemcpy(m->dev_buf[layer], m->host_blob[layer], bytes, cudaMemcpyHostToDevice));
+      SOUP_CK(cudaMemcpy(m->dev_buf[layer], blob, bytes, cudaMemcpyHostToDevice));
     } else {
       for (size_t b = 0; b < m->buf_layer.size(); ++b)
         if (m->buf_layer[b] == layer) m->buf_layer[b] = -1;
@@ -1402,6 +1520,7 @@ soup_status soup_model_load_layer_nf4(soup_model* m, int layer, const void* blob
 soup_status soup_model_read_layer_nf4(soup_model* m, int layer, void* blob, size_t bytes) {
   if (!m || !blob || layer < 0 || layer >= m->cfg.n_layers || bytes != m->layout.total) return SOUP_ERR_INVALID_ARG;
   if (!m->host_loaded[layer]) return SOUP_ERR_STATE;
+  if (m->use_file) return m->file.read(layer, blob, m->err) ? SOUP_OK : SOUP_ERR_IO;
   std::memcpy(blob, m->host_blob[layer], bytes);
   return SOUP_OK;
 }
@@ -1455,6 +1574,45 @@ soup_status soup_set_lora_enabled(soup_model* m, int enabled) {
   return SOUP_OK;
 }
 
+soup_status soup_model_merge_lora(soup_model* m, int layer, int proj, void* out, void* stream) {
+  if (!m || !out || layer < 0 || layer >= m->cfg.n_layers || proj < 0 || proj > 6) return SOUP_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(out) & 15u) return SOUP_ERR_INVALID_ARG;
+  if (!m->lora_p || !m->host_loaded[layer]) return SOUP_ERR_STATE;
+  SOUP_GUARD({
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const long long l0 = g_kernel_launches.load();
+    const uint8_t* base;
+    int buf;
+    SOUP_TRY(streamer_acquire(m, layer, st, &base, &buf));
+    const LayerView v = view_of(m, base);
+    ProjShape sh[7];
+    proj_shapes(m->cfg, sh);
+    const int rows = sh[proj].out;
+    const int cols = sh[proj].in;
+    const int r = m->cfg.lora_r;
+    const NF4Seg& w = v.seg[proj];
+    soup_status s = check_launch(m,
+                                 nf4_dequant_launch(w.codes, w.q8, w.scales, w.mean,
+                                                    static_cast<long long>(rows) * cols, static_cast<uint16_t*>(out),
+                                                    codebook(), st),
+                                 "merge dequant");
+    if (s == SOUP_OK) {
+      // out[rows, cols] += s * B[rows, r] . A[r, cols]: A operand B K-major (ld r), B operand
+      // A^T read MN-major (element (n, k) at A[k * cols + n])
+      const uint16_t* P = m->lora_bf16;
+      GemmParams p = gemm_base(m, rows, cols, out, cols, 0, m->s_lora);
+      p.residual = out;
+      p.ldr = cols;
+      add_seg(p, r, opnd(OP_BF16_K, P + lora_off(m->cfg, layer, proj, 1), r),
+              opnd(OP_BF16_MN, P + lora_off(m->cfg, layer, proj, 0), cols));
+      s = run_gemm(m, p, st, "merge lora");
+    }
+    soup_status s2 = streamer_release(m, buf, st);
+    m->stats.kernel_launches += g_kernel_launches.load() - l0;
+    return s != SOUP_OK ? s : s2;
+  })
+}
+
 soup_status soup_layer_fwd(soup_model* m, int layer, const void* x_in, void* x_out, int B, int S, void* stream) {
   if (!m || !x_in || !x_out || layer < 0 || layer >= m->cfg.n_layers || B < 1 || S < 1 ||
       static_cast<long long>(B) * S > m->cfg.max_tokens)
@@ -1495,7 +1653,7 @@ soup_status soup_layer_bwd(soup_model* m, int layer, const void* dy, void* dx, i
 }
 
 soup_status soup_step(soup_model* m, soup_loss loss, const soup_batch* batch, float* loss_out, void* stream) {
-  if (!m || !batch || (loss != SOUP_LOSS_SFT && loss != SOUP_LOSS_DPO)) return SOUP_ERR_INVALID_ARG;
+  if (!m || !batch || loss < SOUP_LOSS_SFT || loss > SOUP_LOSS_SIMPO) return SOUP_ERR_INVALID_ARG;
   SOUP_GUARD(return do_step(m, loss, batch, loss_out, static_cast<cudaStream_t>(stream));)
 }
 
@@ -1598,6 +1756,11 @@ soup_status soup_nf4_codebook(float* out16) {
 soup_status soup_get_stats(soup_model* m, soup_stats* out) {
   if (!m || !out) return SOUP_ERR_INVALID_ARG;
   *out = m->stats;
+  out->stream_source = m->use_file ? SOUP_SOURCE_FILE : SOUP_SOURCE_RAM;
+  if (m->use_file) {
+    out->file_bytes_read = m->file.bytes_read() - m->file_bytes0;
+    out->file_read_ms = m->file.read_ms() - m->file_ms0;
+  }
   return SOUP_OK;
 }
 
@@ -1607,6 +1770,10 @@ soup_status soup_reset_stats(soup_model* m) {
   m->stats = soup_stats{};
   m->stats.device_bytes = dev;
   m->stats.pinned_bytes = pin;
+  if (m->use_file) {
+    m->file_bytes0 = m->file.bytes_read();
+    m->file_ms0 = m->file.read_ms();
+  }
   return SOUP_OK;
 }
 
@@ -1646,16 +1813,16 @@ soup_status soup_h2d_probe(soup_model* m, int reps, double* gbs) {
   if (!m->host_loaded[0]) return SOUP_ERR_STATE;
   SOUP_GUARD({
     const int b = 0;
+    const uint8_t* src = m->use_file ? m->file.probe_buffer() : m->host_blob[0];
     SOUP_CK(cudaStreamWaitEvent(m->copy_stream, m->buf_free[b], 0));
     cudaEvent_t e0 = nullptr;
     cudaEvent_t e1 = nullptr;
     SOUP_CK(cudaEventCreate(&e0));
     SOUP_CK(cudaEventCreate(&e1));
-    SOUP_CK(cudaMemcpyAsync(m->dev_buf[b], m->host_blob[0], m->layout.total, cudaMemcpyHostToDevice, m->copy_stream));
+    SOUP_CK(cudaMemcpyAsync(m->dev_buf[b], src, m->layout.total, cudaMemcpyHostToDevice, m->copy_stream));
     SOUP_CK(cudaEventRecord(e0, m->copy_stream));
     for (int i = 0; i < reps; ++i)
-      SOUP_CK(cudaMemcpyAsync(m->dev_buf[b], m->host_blob[0], m->layout.total, cudaMemcpyHostToDevice,
-                              m->copy_stream));
+      SOUP_CK(cudaMemcpyAsync(m->dev_buf[b], src, m->layout.total, cudaMemcpyHostToDevice, m->copy_stream));
     SOUP_CK(cudaEventRecord(e1, m->copy_stream));
     SOUP_CK(cudaEventRecord(m->copy_done[b], m->copy_stream));
     soup_status st = wait_stream(m, m->copy_stream);

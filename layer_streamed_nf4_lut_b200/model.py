@@ -15,7 +15,7 @@ from ._lib import PROJ, Batch, ModelConfig, Stats, check, lib
 
 
 def make_config(cfg: dict, mode: str = "streamed", n_layer_buffers: int = 2, max_tokens: int | None = None,
-                device: int = 0) -> ModelConfig:
+                device: int = 0, source: str = "ram", stack_path: str | None = None) -> ModelConfig:
     c = ModelConfig()
     for k in ("n_layers", "hidden", "n_heads", "n_kv_heads", "head_dim", "intermediate", "vocab", "lora_r"):
         setattr(c, k, int(cfg[k]))
@@ -26,6 +26,8 @@ def make_config(cfg: dict, mode: str = "streamed", n_layer_buffers: int = 2, max
     c.n_layer_buffers = int(n_layer_buffers)
     c.max_tokens = int(max_tokens if max_tokens is not None else cfg["batch"] * cfg["seq"])
     c.device = int(device)
+    c.stream_source = {"ram": _lib.SOUP_SOURCE_RAM, "file": _lib.SOUP_SOURCE_FILE, "auto": _lib.SOUP_SOURCE_AUTO}[source]
+    c.stack_path = stack_path.encode() if stack_path else None
     return c
 
 
@@ -90,9 +92,11 @@ class _TorchAllocator:
 
 class SoupModel:
     def __init__(self, cfg: dict, mode: str = "streamed", n_layer_buffers: int = 2, max_tokens: int | None = None,
-                 device: int = 0, torch_alloc: bool = True):
+                 device: int = 0, torch_alloc: bool = True, source: str = "ram", stack_path: str | None = None):
+        """source: "ram" (page-locked host stack), "file" (stack file at stack_path, streamed
+        through page-locked staging) or "auto" (RAM if it fits, else the file)."""
         self.cfg = dict(cfg)
-        self.ccfg = make_config(cfg, mode, n_layer_buffers, max_tokens, device)
+        self.ccfg = make_config(cfg, mode, n_layer_buffers, max_tokens, device, source, stack_path)
         self.device = torch.device("cuda", device)
         self._allocator = _TorchAllocator(device) if torch_alloc else None
         h = c_void_p()
@@ -159,6 +163,22 @@ class SoupModel:
     def set_lora_enabled(self, enabled: bool):
         self._ck(lib.soup_set_lora_enabled(self.h, 1 if enabled else 0))
 
+    def merge_lora(self, layer: int, proj: str, out: torch.Tensor | None = None) -> torch.Tensor:
+        """bf16 [out_features, in_features]: the projection's NF4 base fused with its adapter."""
+        j = PROJ.index(proj)
+        rows, cols = self._proj_shape(j)
+        if out is None:
+            out = torch.empty(rows, cols, dtype=torch.bfloat16, device=self.device)
+        assert out.dtype == torch.bfloat16 and out.is_contiguous() and tuple(out.shape) == (rows, cols)
+        self._ck(lib.soup_model_merge_lora(self.h, layer, j, _ptr(out), _stream_ptr()))
+        return out
+
+    def _proj_shape(self, j: int):
+        c = self.cfg
+        qd, kvd = c["n_heads"] * c["head_dim"], c["n_kv_heads"] * c["head_dim"]
+        h, I = c["hidden"], c["intermediate"]
+        return [(qd, h), (kvd, h), (kvd, h), (h, qd), (I, h), (I, h), (h, I)][j]
+
     # ------------------------------------------------------------------ compute
     def layer_fwd(self, layer: int, x: torch.Tensor, B: int, S: int, out: torch.Tensor | None = None):
         y = out if out is not None else torch.empty_like(x)
@@ -171,35 +191,51 @@ class SoupModel:
         return dx
 
     def step(self, ids, loss: str = "sft", mask=None, n_pairs: int = 0, prefix_len: int = 0, beta: float = 0.1,
-             lr: float = 2e-5, apply_optimizer: bool = True) -> float:
-        """ids: int32 [B, S] as a cuda tensor, or as host memory (numpy / cpu tensor: copied by the library)."""
+             lr: float = 2e-5, apply_optimizer: bool = True, dpo_shared_load: bool = False, labels=None,
+             gamma: float = 0.0, lambda_or: float = 0.1, lambda_d: float = 1.0, lambda_u: float = 1.0) -> float:
+        """ids: int32 [B, S] as a cuda tensor, or as host memory (numpy / cpu tensor: copied by the
+        library); mask (SFT) and labels (KTO, uint8 [B]) in the same memory space as ids."""
         b = Batch()
         on_host = not (isinstance(ids, torch.Tensor) and ids.is_cuda)
+        keep = []
+
+        def _host_u8(a):
+            t = a if isinstance(a, torch.Tensor) else torch.from_numpy(np.ascontiguousarray(a, np.uint8))
+            t = t.contiguous()
+            keep.append(t)
+            return t.data_ptr()
+
         if on_host:
             ids_h = ids if isinstance(ids, torch.Tensor) else torch.from_numpy(np.ascontiguousarray(ids, np.int32))
             ids_h = ids_h.contiguous()
             assert ids_h.dtype == torch.int32
             b.ids = ids_h.data_ptr()
-            keep = [ids_h]
+            keep.append(ids_h)
             if mask is not None:
-                m_h = mask if isinstance(mask, torch.Tensor) else torch.from_numpy(np.ascontiguousarray(mask, np.uint8))
-                m_h = m_h.contiguous()
-                keep.append(m_h)
-                b.loss_mask = m_h.data_ptr()
+                b.loss_mask = _host_u8(mask)
+            if labels is not None:
+                b.labels = _host_u8(labels)
             B, S = ids_h.shape
         else:
             assert ids.dtype == torch.int32
             b.ids = ids.data_ptr()
             if mask is not None:
                 b.loss_mask = mask.data_ptr()
+            if labels is not None:
+                if not (isinstance(labels, torch.Tensor) and labels.is_cuda):
+                    labels = torch.as_tensor(np.ascontiguousarray(labels, np.uint8)).to(ids.device)
+                assert labels.dtype == torch.uint8
+                keep.append(labels)
+                b.labels = labels.data_ptr()
             B, S = ids.shape
         b.B, b.S = int(B), int(S)
         b.ids_on_host = 1 if on_host else 0
         b.n_pairs, b.prefix_len, b.beta = int(n_pairs), int(prefix_len), float(beta)
         b.lr, b.apply_optimizer = float(lr), 1 if apply_optimizer else 0
+        b.dpo_shared_load = 1 if dpo_shared_load else 0
+        b.gamma, b.lambda_or, b.lambda_d, b.lambda_u = float(gamma), float(lambda_or), float(lambda_d), float(lambda_u)
         out = c_float()
-        kind = _lib.SOUP_LOSS_DPO if loss == "dpo" else _lib.SOUP_LOSS_SFT
-        self._ck(lib.soup_step(self.h, kind, byref(b), byref(out), _stream_ptr()))
+        self._ck(lib.soup_step(self.h, _lib.LOSS_KINDS[loss], byref(b), byref(out), _stream_ptr()))
         return out.value
 
     def optimizer_step(self, lr: float):

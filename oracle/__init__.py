@@ -17,14 +17,18 @@ Sources.  The method comes from five web pages about the open-source "Soup" trai
     gráfica" (guillermodelpino.com), sections "El streaming de capas, que es el truco de la
     casa", the soup.yaml example, "Preguntas frecuentes";
   * "Soup promete fine-tuning de modelo 8B em GPU de notebook com 4 GB" (imasters.com.br),
-    sections "Como cabe um 8B em 4 GB" and "Do SFT para os métodos de preferência".
-The pages name NF4, LoRA, the Llama-3.1-8B decoder layer, SFT and DPO but print no
-formula; where they are silent each function states the textbook definition it follows
-(QLoRA, LoRA, Llama, DPO and AdamW papers).
+    sections "Como cabe um 8B em 4 GB", "Do SFT para os métodos de preferência" and "O que
+    muda para quem constrói no Brasil".
+The pages name NF4, LoRA, the Llama-3.1-8B decoder layer, SFT, DPO, KTO, ORPO, SimPO and a
+merge command but print no formula; where they are silent each function states the textbook
+definition it follows (QLoRA, LoRA, Llama, DPO, KTO, ORPO, SimPO and AdamW papers).
+
+Modules: nf4 (codebook, quantise / dequantise, blob sizes), model (decoder layer, LoRA, SFT
+and DPO losses, backward passes, AdamW, LoRA merge), pref (KTO, ORPO, SimPO).
 
 Parity status per function: every function here is pinned by tests/test_oracle_*.py
 (closed forms, library routines, finite differences, a published table).  The composed
 training step's absolute loss on random weights has no printed value to compare with:
 "parity unpinned" beyond the pins of its parts.
 """
-from . import nf4, model  # noqa: F401
+from . import nf4, model, pref  # noqa: F401

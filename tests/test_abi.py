@@ -93,6 +93,18 @@ def test_config_validation(field, value, status):
     assert st == status
 
 
+def test_stream_source_validation():
+    n = ctypes.c_size_t()
+    bad = M.make_config(synth.TINY)
+    bad.stream_source = 7
+    assert _lib.lib.soup_layer_blob_bytes(ctypes.byref(bad), ctypes.byref(n)) == -1
+    nopath = M.make_config(synth.TINY, source="file")
+    assert _lib.lib.soup_layer_blob_bytes(ctypes.byref(nopath), ctypes.byref(n)) == -1
+    ok = M.make_config(synth.TINY, source="file", stack_path="/tmp/x.soup")
+    assert _lib.lib.soup_layer_blob_bytes(ctypes.byref(ok), ctypes.byref(n)) == 0
+    assert _lib.lib.soup_status_string(-8) == b"layer stack file I/O failed"
+
+
 def test_streamed_needs_two_buffers():
     c = M.make_config(synth.TINY, mode="streamed", n_layer_buffers=1)
     h = ctypes.c_void_p()
@@ -106,3 +118,32 @@ def test_null_arguments_rejected():
     assert L.soup_step(None, 0, None, None, None) == -1
     assert L.soup_nf4_codebook(None) == -1
     assert L.soup_status_string(-5) == b"timed out"
+
+
+def test_struct_layouts_match_the_c_compiler(tmp_path):
+    """sizeof / offsetof of every public struct, as gcc lays them out from include/soup.h,
+    against the ctypes mirrors the binding passes across the boundary."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    structs = {"soup_model_config": _lib.ModelConfig, "soup_allocator": _lib.Allocator, "soup_stats": _lib.Stats,
+               "soup_profile_entry": _lib.ProfileEntry, "soup_batch": _lib.Batch}
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "soup.h"', "int main(void) {"]
+    for cname, cls in structs.items():
+        lines.append(f'  printf("{cname} sizeof %zu\\n", sizeof({cname}));')
+        for fname, _ in cls._fields_:
+            lines.append(f'  printf("{cname} {fname} %zu\\n", offsetof({cname}, {fname}));')
+    lines += ["  return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-std=c11", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    got = {}
+    for line in subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.splitlines():
+        s, f, v = line.split()
+        got[(s, f)] = int(v)
+    for cname, cls in structs.items():
+        assert got[(cname, "sizeof")] == ctypes.sizeof(cls), cname
+        for fname, _ in cls._fields_:
+            assert got[(cname, fname)] == getattr(cls, fname).offset, (cname, fname)

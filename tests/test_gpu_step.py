@@ -139,3 +139,29 @@ def test_bad_token_id_reports_device_check():
         assert math.isfinite(loss)
     finally:
         p.close()
+
+
+def test_dpo_shared_load_schedule_same_bits_fewer_loads():
+    p = Pair(TINY4, seed=15, modes=("streamed",), want_oracle=False, max_tokens=4 * 64)
+    try:
+        gm = p.models["streamed"]
+        L = TINY4["n_layers"]
+        cfg = dict(TINY4, batch=4, n_pairs=2, prefix_len=32)
+        ids = torch.from_numpy(synth.preference_batch(cfg, 40)).cuda()
+        kw = dict(loss="dpo", n_pairs=2, prefix_len=32, beta=0.1, apply_optimizer=False)
+        gm.step(ids, **kw)  # warm: layers 0, 1 resident afterwards
+        gm.reset_stats()
+        l_re = gm.step(ids, **kw)
+        loads_re = gm.stats()["layer_loads"]
+        g_re = gm.lora_grads.clone()
+        pi_re, ref_re = gm.last_logps(4)
+        gm.reset_stats()
+        l_sh = gm.step(ids, dpo_shared_load=True, **kw)
+        loads_sh = gm.stats()["layer_loads"]
+        pi_sh, ref_sh = gm.last_logps(4)
+        assert l_sh == l_re
+        assert torch.equal(g_re.view(torch.int32), gm.lora_grads.view(torch.int32))
+        assert np.array_equal(pi_sh, pi_re) and np.array_equal(ref_sh, ref_re)
+        assert loads_re == 3 * L - 4 and loads_sh == 2 * L - 4
+    finally:
+        p.close()
