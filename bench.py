@@ -43,6 +43,9 @@ WORKLOADS = {
     # same DPO step, each layer loaded once for the reference and the policy forward
     "llama8b-dpo-2pairs-s512-shared-load": dict(cfg=synth.L8B_DPO, B=4, S=512, loss="dpo", n_pairs=2,
                                                 prefix_len=256, beta=0.1, dpo_shared_load=True),
+    # one load per layer and each pair's 256-token prefix run once: 1536 rows through the layers
+    "llama8b-dpo-2pairs-s512-shared-prefix": dict(cfg=synth.L8B_DPO, B=4, S=512, loss="dpo", n_pairs=2,
+                                                  prefix_len=256, beta=0.1, dpo_shared_load=True, share_prefix=True),
     # the other preference losses on the same batch shape (KTO: 4 unpaired rows, 2 desirable)
     "llama8b-kto-4seq-s512": dict(cfg=synth.L8B_DPO, B=4, S=512, loss="kto", n_pairs=2, prefix_len=256, beta=0.1,
                                   labels=(1, 0, 1, 0)),
@@ -66,6 +69,22 @@ def peaks():
         return dict(hbm_gbs=d["hbm_gbs"], bf16=d["bf16_tflops"], bf16_sustained=d["bf16_tflops_sustained"],
                     source="measured")
     return dict(hbm_gbs=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+def measured_traffic(kernel):
+    """DRAM bytes per launch of a kernel category from an ncu capture summarised under
+    profiles/, or None when the kernel's sources changed since the capture."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic_per_launch.json")
+    if not os.path.exists(path):
+        return None
+    rec = json.load(open(path)).get(kernel)
+    if not rec:
+        return None
+    h = hashlib.sha256()
+    for f in rec["kernel_sources"]:
+        h.update(open(os.path.join(ROOT, f), "rb").read())
+    return rec["dram_bytes_per_launch"] if h.hexdigest() == rec["kernel_sources_sha256"] else None
 
 
 def step_flops(cfg, B, S, loss):
@@ -204,6 +223,7 @@ def run_soup(args, wl, rank, world, local_rank):
     mask = torch.from_numpy(mask_np).to(dev) if mask_np is not None else None
     kw = dict(loss=wl["loss"], mask=mask, n_pairs=wl.get("n_pairs", 0), prefix_len=wl.get("prefix_len", 0),
               beta=wl.get("beta", 0.1), lr=2e-5, dpo_shared_load=wl.get("dpo_shared_load", False),
+              share_prefix=wl.get("share_prefix", False),
               gamma=wl.get("gamma", 0.0), lambda_or=wl.get("lambda_or", 0.1),
               labels=np.array(wl["labels"], np.uint8) if "labels" in wl else None)
     setup_s = time.time() - t_setup
@@ -297,7 +317,10 @@ def run_soup(args, wl, rank, world, local_rank):
     if rank != 0:
         return None
     pk = peaks()
-    flops = step_flops(cfg, B, S, wl["loss"])
+    if wl.get("share_prefix"):  # each pair runs as one block of 2S - prefix rows
+        flops = step_flops(cfg, wl["n_pairs"], 2 * S - wl["prefix_len"], wl["loss"])
+    else:
+        flops = step_flops(cfg, B, S, wl["loss"])
     stream_bytes = loads_per_step * blob_bytes
     t_flops = flops / (pk["bf16_sustained"] * 1e12)
     t_h2d = stream_bytes / (h2d_gbs * 1e9)
@@ -314,13 +337,14 @@ def run_soup(args, wl, rank, world, local_rank):
             achieved = d["flops"] / d["launches"] / (per_launch_ms * 1e-3) / 1e12
             roofline = {"bound": "tensor", "kernel": dom, "achieved": round(achieved, 2),
                         "peak": pk["bf16_sustained"], "unit": "TFLOP/s", "frac": round(achieved / pk["bf16_sustained"], 4),
-                        "peak_source": pk["source"] + " bf16 sustained", "traffic": None,
+                        "peak_source": pk["source"] + " bf16 sustained", "traffic": measured_traffic(dom),
+                        "algorithmic_bytes_per_launch": round(d["bytes"] / d["launches"]),
                         "avg_launch_ms": round(per_launch_ms, 4), "launches": d["launches"]}
         else:
             achieved = d["bytes"] / d["launches"] / (per_launch_ms * 1e-3) / 1e9
             roofline = {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1), "peak": pk["hbm_gbs"],
                         "unit": "GB/s", "frac": round(achieved / pk["hbm_gbs"], 4), "peak_source": pk["source"],
-                        "traffic": None, "avg_launch_ms": round(per_launch_ms, 4), "launches": d["launches"]}
+                        "traffic": measured_traffic(dom), "avg_launch_ms": round(per_launch_ms, 4), "launches": d["launches"]}
     h2d = prof.get("h2d_layer_copy")
     profile_summary = {k: {"launches": v["launches"] // n_prof, "ms_per_step": round(v["total_ms"] / n_prof, 3),
                            "tflops": round(v["flops"] / (v["total_ms"] * 1e-3) / 1e12, 1) if v["flops"] else None,

@@ -138,6 +138,12 @@ typedef struct soup_batch {
   float gamma;           /* SimPO target margin */
   float lambda_or;       /* ORPO weight of the odds-ratio term */
   float lambda_d, lambda_u; /* KTO weights of desirable / undesirable rows */
+  int share_prefix;      /* DPO, SimPO, ORPO: 1 = each pair's shared prefix (ids[2p][:prefix_len] ==
+                            ids[2p+1][:prefix_len], the caller's promise) runs through the layers
+                            once: the pair becomes one block [prefix | chosen | rejected] in which
+                            the rejected response attends to the prefix and to itself.  Applies
+                            when prefix_len and S - prefix_len are multiples of 64 (else the plain
+                            layout runs); the same loss and gradients up to rounding order. */
 } soup_batch;
 
 /* ---- lifecycle -------------------------------------------------------------------------- */

@@ -61,7 +61,7 @@ class Batch(Structure):
     _fields_ = [("ids", c_void_p), ("loss_mask", c_void_p), ("B", c_int), ("S", c_int), ("ids_on_host", c_int),
                 ("n_pairs", c_int), ("prefix_len", c_int), ("beta", c_float), ("lr", c_float),
                 ("apply_optimizer", c_int), ("dpo_shared_load", c_int), ("labels", c_void_p), ("gamma", c_float),
-                ("lambda_or", c_float), ("lambda_d", c_float), ("lambda_u", c_float)]
+                ("lambda_or", c_float), ("lambda_d", c_float), ("lambda_u", c_float), ("share_prefix", c_int)]
 
 
 # name -> (restype, argtypes); every function returns soup_status unless stated

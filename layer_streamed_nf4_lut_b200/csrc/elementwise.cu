@@ -106,10 +106,11 @@ __global__ void rmsnorm_bwd_kernel(const uint16_t* __restrict__ dy, const uint16
 // pos * theta^(-2i/d), pos = t mod S, read from a [S_max, d/2] cos/sin table; inverse != 0
 // rotates by -angle (the backward).  One thread per 8 consecutive i of one head.
 __global__ void rope_kernel(uint16_t* __restrict__ qkv, long long ld, int S, int nheads, int d,
-                            const float* __restrict__ tcos, const float* __restrict__ tsin, int inverse) {
+                            const float* __restrict__ tcos, const float* __restrict__ tsin, int inverse, int pack_rl) {
   const int t = blockIdx.x;
   const int half = d / 2, g8 = half / 8;
-  const int pos = t % S;
+  int pos = t % S;
+  if (pack_rl > 0 && pos >= S - pack_rl) pos -= pack_rl;  // rejected response of a shared-prefix pair
   uint16_t* row = qkv + static_cast<long long>(t) * ld;
   for (int idx = threadIdx.x; idx < nheads * g8; idx += blockDim.x) {
     const int hh = idx / g8, i0 = (idx % g8) * 8;
@@ -270,7 +271,8 @@ __global__ void seq_logp_kernel(const float* __restrict__ lse, const float* __re
 // DPO closed form on P pairs (rows 2p chosen, 2p+1 rejected); row weights = -dL/dpi on the
 // response rows so that dlogits = w * (softmax - onehot).
 __global__ void dpo_finish_kernel(const float* __restrict__ pi, const float* __restrict__ ref, int B, int S, int start,
-                                  int P, float beta, float* __restrict__ loss_out, float* __restrict__ row_weight) {
+                                  int P, float beta, float* __restrict__ loss_out, float* __restrict__ row_weight,
+                                  float* __restrict__ seq_w) {
   __shared__ float wrow[256];
   if (threadIdx.x == 0) {
     double loss = 0.0;
@@ -286,6 +288,8 @@ __global__ void dpo_finish_kernel(const float* __restrict__ pi, const float* __r
     loss_out[0] = static_cast<float>(loss / P);
   }
   __syncthreads();
+  if (seq_w && threadIdx.x < B) seq_w[threadIdx.x] = wrow[threadIdx.x];
+  if (!row_weight) return;
   const int j0 = start > 1 ? start : 1;
   for (int t = threadIdx.x; t < B * S; t += blockDim.x) {
     const int b = t / S, j = t % S + 1;
@@ -307,7 +311,7 @@ __device__ __forceinline__ double log1mexp_d(double a) {  // log(1 - e^a), a < 0
 __global__ void pref_finish_kernel(int kind, const float* __restrict__ pi, const float* __restrict__ ref,
                                    const uint8_t* __restrict__ labels, int B, int S, int start, float beta,
                                    float gamma, float lam_or, float lam_d, float lam_u, float* __restrict__ loss_out,
-                                   float* __restrict__ row_weight) {
+                                   float* __restrict__ row_weight, float* __restrict__ seq_w) {
   __shared__ float wrow[256];
   if (threadIdx.x == 0) {
     const int j0 = start > 1 ? start : 1;
@@ -359,6 +363,8 @@ __global__ void pref_finish_kernel(int kind, const float* __restrict__ pi, const
     loss_out[0] = static_cast<float>(loss);
   }
   __syncthreads();
+  if (seq_w && threadIdx.x < B) seq_w[threadIdx.x] = wrow[threadIdx.x];
+  if (!row_weight) return;
   const int j0 = start > 1 ? start : 1;
   for (int t = threadIdx.x; t < B * S; t += blockDim.x) {
     const int b = t / S, j = t % S + 1;
@@ -385,6 +391,124 @@ __global__ void ce_grad_kernel(const float* __restrict__ logits, const float* __
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         o[j] = w * (expf(x[j] - l) - ((4 * c + j) == target ? 1.f : 0.f));
+      }
+    }
+    out[c] = make_uint2(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]));
+  }
+}
+
+// ---------------------------------------------------------------- shared-prefix pair blocks
+// A preference pair (rows 2p chosen, 2p+1 rejected of ids [2P, S], sharing ids[.., :pl]) is
+// packed as one block of Sb = pl + 2 rl rows, rl = S - pl: [prefix | chosen response |
+// rejected response].  Row x of a block predicts tgt1[x] (-1: none); the last prefix row also
+// predicts the rejected response's first token (tgt2), the one place where the two sequences
+// of a pair differ in what a shared row predicts.
+__global__ void pair_pack_kernel(const int32_t* __restrict__ ids, int P, int S, int pl, int V,
+                                 int32_t* __restrict__ pids, int32_t* __restrict__ tgt1, int32_t* __restrict__ tgt2,
+                                 int* err) {
+  const int rl = S - pl, Sb = pl + 2 * rl;
+  const long long x_all = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (x_all >= static_cast<long long>(P) * Sb) return;
+  const int p = static_cast<int>(x_all / Sb), x = static_cast<int>(x_all % Sb);
+  const int32_t* ch = ids + static_cast<long long>(2 * p) * S;
+  const int32_t* rj = ch + S;
+  int tok, t1 = -1, t2 = -1;
+  if (x < pl + rl) {  // prefix or chosen response: the chosen sequence's row x
+    tok = ch[x];
+    if (x + 1 < S) t1 = ch[x + 1];
+    if (x == pl - 1) t2 = rj[pl];
+  } else {            // rejected response at position x - rl
+    const int pos = x - rl;
+    tok = rj[pos];
+    if (pos + 1 < S) t1 = rj[pos + 1];
+  }
+  if (tok < 0 || tok >= V || t1 >= V || t2 >= V) set_dev_error(err, DEVERR_BOUNDS);
+  pids[x_all] = tok;
+  tgt1[x_all] = t1;
+  tgt2[x_all] = t2;
+}
+
+// Row LSE and the logits at tgt1 / tgt2 (0 where there is no target).
+__global__ void ce_rows_t_kernel(const float* __restrict__ logits, int V, const int32_t* __restrict__ tgt1,
+                                 const int32_t* __restrict__ tgt2, float* __restrict__ lse, float* __restrict__ rt1,
+                                 float* __restrict__ rt2) {
+  __shared__ float red[32];
+  const long long t = blockIdx.x;
+  const float4* row = reinterpret_cast<const float4*>(logits + t * V);
+  float mx = -INFINITY, sm = 0.f;
+  for (int c = threadIdx.x; c < V / 4; c += blockDim.x) {
+    const float4 v = row[c];
+    const float lm = fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w));
+    if (lm > mx) {
+      sm *= expf(mx - lm);
+      mx = lm;
+    }
+    sm += expf(v.x - mx) + expf(v.y - mx) + expf(v.z - mx) + expf(v.w - mx);
+  }
+  const float M = block_max(mx, red);
+  const float part = (mx == -INFINITY) ? 0.f : sm * expf(mx - M);
+  const float tot = block_sum(part, red);
+  if (threadIdx.x == 0) {
+    lse[t] = M + logf(tot);
+    const int a = tgt1[t], b = tgt2[t];
+    rt1[t] = (a >= 0 && a < V) ? logits[t * V + a] : 0.f;
+    rt2[t] = (b >= 0 && b < V) ? logits[t * V + b] : 0.f;
+  }
+}
+
+// Per pair: pi[2p] = chosen response log-prob (rows pl-1 .. pl+rl-2 with tgt1), pi[2p+1] =
+// rejected (row pl-1 with tgt2, rows pl+rl .. pl+2rl-2 with tgt1); fixed-order sums.
+__global__ void pair_logp_kernel(const float* __restrict__ lse, const float* __restrict__ rt1,
+                                 const float* __restrict__ rt2, int pl, int rl, float* __restrict__ out) {
+  __shared__ float red[32];
+  const int p = blockIdx.x, Sb = pl + 2 * rl;
+  const long long base = static_cast<long long>(p) * Sb;
+  float c = 0.f, r = 0.f;
+  for (int x = pl - 1 + threadIdx.x; x < pl + rl - 1; x += blockDim.x) c += rt1[base + x] - lse[base + x];
+  for (int x = pl + rl + threadIdx.x; x < Sb - 1; x += blockDim.x) r += rt1[base + x] - lse[base + x];
+  c = block_sum(c, red);
+  r = block_sum(r, red);
+  if (threadIdx.x == 0) {
+    out[2 * p] = c;
+    out[2 * p + 1] = r + (rt2[base + pl - 1] - lse[base + pl - 1]);
+  }
+}
+
+// Row weights of a pair block from the per-sequence weights (seq_w = -dL/dpi).
+__global__ void pair_rowweight_kernel(const float* __restrict__ seq_w, int P, int pl, int rl, float* __restrict__ w1,
+                                      float* __restrict__ w2) {
+  const int Sb = pl + 2 * rl;
+  const long long x_all = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (x_all >= static_cast<long long>(P) * Sb) return;
+  const int p = static_cast<int>(x_all / Sb), x = static_cast<int>(x_all % Sb);
+  float a = 0.f, b = 0.f;
+  if (x >= pl - 1 && x < pl + rl - 1) a = seq_w[2 * p];
+  if (x >= pl + rl && x < Sb - 1) a = seq_w[2 * p + 1];
+  if (x == pl - 1) b = seq_w[2 * p + 1];
+  w1[x_all] = a;
+  w2[x_all] = b;
+}
+
+// dlogits[t, v] = (w1 + w2) softmax - w1 [v == tgt1] - w2 [v == tgt2], rounded to bf16.
+__global__ void ce_grad_t_kernel(const float* __restrict__ logits, const float* __restrict__ lse,
+                                 const int32_t* __restrict__ tgt1, const float* __restrict__ w1,
+                                 const int32_t* __restrict__ tgt2, const float* __restrict__ w2, int V,
+                                 uint16_t* __restrict__ dl) {
+  const long long t = blockIdx.x;
+  const float a = w1[t], b = w2[t];
+  const int ta = tgt1[t], tb = tgt2[t];
+  const float l = lse[t];
+  const float4* row = reinterpret_cast<const float4*>(logits + t * V);
+  uint2* out = reinterpret_cast<uint2*>(dl + t * V);
+  for (int c = threadIdx.x; c < V / 4; c += blockDim.x) {
+    float o[4] = {0.f, 0.f, 0.f, 0.f};
+    if (a != 0.f || b != 0.f) {
+      const float4 v = row[c];
+      const float x[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int col = 4 * c + j;
+        o[j] = (a + b) * expf(x[j] - l) - (col == ta ? a : 0.f) - (col == tb ? b : 0.f);
       }
     }
     out[c] = make_uint2(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]));
@@ -473,13 +597,13 @@ cudaError_t rmsnorm_bwd_launch(const uint16_t* dy, const uint16_t* x, const floa
 }
 
 cudaError_t rope_launch(uint16_t* qkv, long long ld, int B, int S, int hq, int hkv, int d, const float* tcos,
-                        const float* tsin, int inverse, cudaStream_t st) {
+                        const float* tsin, int inverse, cudaStream_t st, int pack_rl) {
   const int T = B * S;
   if (T <= 0) return cudaSuccess;
   const int nheads = hq + hkv;  // q heads then k heads, contiguous from column 0
   int thr = nheads * d / 16;
   thr = thr > 256 ? 256 : ((thr + 31) / 32) * 32;
-  rope_kernel<<<T, thr, 0, st>>>(qkv, ld, S, nheads, d, tcos, tsin, inverse);
+  rope_kernel<<<T, thr, 0, st>>>(qkv, ld, S, nheads, d, tcos, tsin, inverse, pack_rl);
   ++g_kernel_launches;
   return cudaGetLastError();
 }
@@ -532,7 +656,27 @@ cudaError_t dpo_finish_launch(const float* lse, const float* tgt, int B, int S, 
   if (B < 2 || B > 256) return cudaErrorInvalidValue;
   cudaError_t e = seq_logp_launch(lse, tgt, B, S, resp_start, pi_out, st);
   if (e != cudaSuccess) return e;
-  dpo_finish_kernel<<<1, 256, 0, st>>>(pi_out, ref_logp, B, S, resp_start, n_pairs, beta, loss_out, row_weight);
+  dpo_finish_kernel<<<1, 256, 0, st>>>(pi_out, ref_logp, B, S, resp_start, n_pairs, beta, loss_out, row_weight,
+                                       nullptr);
+  ++g_kernel_launches;
+  return cudaGetLastError();
+}
+
+cudaError_t dpo_loss_seqw_launch(const float* pi, const float* ref_logp, int n_pairs, float beta, float* loss_out,
+                                 float* seq_w, cudaStream_t st) {
+  if (n_pairs < 1 || n_pairs > 128) return cudaErrorInvalidValue;
+  dpo_finish_kernel<<<1, 256, 0, st>>>(pi, ref_logp, 2 * n_pairs, 1, 0, n_pairs, beta, loss_out, nullptr, seq_w);
+  ++g_kernel_launches;
+  return cudaGetLastError();
+}
+
+cudaError_t pref_loss_seqw_launch(int kind, const float* pi, const float* ref_logp, const uint8_t* labels, int B,
+                                  int n_resp, float beta, float gamma, float lam_or, float lam_d, float lam_u,
+                                  float* loss_out, float* seq_w, cudaStream_t st) {
+  if (B < 1 || B > 256) return cudaErrorInvalidValue;
+  // the kernel derives the response length n from (S, start) as S - max(start, 1)
+  pref_finish_kernel<<<1, 256, 0, st>>>(kind, pi, ref_logp, labels, B, n_resp + 1, 1, beta, gamma, lam_or, lam_d, lam_u,
+                                        loss_out, nullptr, seq_w);
   ++g_kernel_launches;
   return cudaGetLastError();
 }
@@ -545,7 +689,7 @@ cudaError_t pref_finish_launch(int kind, const float* lse, const float* tgt, int
   cudaError_t e = seq_logp_launch(lse, tgt, B, S, resp_start, pi_out, st);
   if (e != cudaSuccess) return e;
   pref_finish_kernel<<<1, 256, 0, st>>>(kind, pi_out, ref_logp, labels, B, S, resp_start, beta, gamma, lam_or, lam_d,
-                                        lam_u, loss_out, row_weight);
+                                        lam_u, loss_out, row_weight, nullptr);
   ++g_kernel_launches;
   return cudaGetLastError();
 }
@@ -574,6 +718,45 @@ cudaError_t adamw_launch(float* p, const float* g, float* m, float* v, uint16_t*
   const long long n4 = (n + 3) / 4;
   adamw_kernel<<<static_cast<unsigned>((n4 + 255) / 256), 256, 0, st>>>(p, g, m, v, pb, n, lr, b1, b2, eps, wd, bc1,
                                                                           bc2);
+  ++g_kernel_launches;
+  return cudaGetLastError();
+}
+
+cudaError_t pair_pack_launch(const int32_t* ids, int P, int S, int pl, int V, int32_t* pids, int32_t* tgt1,
+                             int32_t* tgt2, int* err, cudaStream_t st) {
+  const long long n = static_cast<long long>(P) * (2 * S - pl);
+  if (n <= 0) return cudaSuccess;
+  pair_pack_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(ids, P, S, pl, V, pids, tgt1, tgt2, err);
+  ++g_kernel_launches;
+  return cudaGetLastError();
+}
+
+cudaError_t ce_rows_t_launch(const float* logits, int T, int V, const int32_t* tgt1, const int32_t* tgt2, float* lse,
+                             float* rt1, float* rt2, cudaStream_t st) {
+  if (T <= 0) return cudaSuccess;
+  ce_rows_t_kernel<<<T, 512, 0, st>>>(logits, V, tgt1, tgt2, lse, rt1, rt2);
+  ++g_kernel_launches;
+  return cudaGetLastError();
+}
+
+cudaError_t pair_logp_launch(const float* lse, const float* rt1, const float* rt2, int P, int pl, int rl, float* out,
+                             cudaStream_t st) {
+  pair_logp_kernel<<<P, 256, 0, st>>>(lse, rt1, rt2, pl, rl, out);
+  ++g_kernel_launches;
+  return cudaGetLastError();
+}
+
+cudaError_t pair_rowweight_launch(const float* seq_w, int P, int pl, int rl, float* w1, float* w2, cudaStream_t st) {
+  const long long n = static_cast<long long>(P) * (pl + 2 * rl);
+  pair_rowweight_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(seq_w, P, pl, rl, w1, w2);
+  ++g_kernel_launches;
+  return cudaGetLastError();
+}
+
+cudaError_t ce_grad_t_launch(const float* logits, const float* lse, const int32_t* tgt1, const float* w1,
+                             const int32_t* tgt2, const float* w2, int T, int V, uint16_t* dlogits, cudaStream_t st) {
+  if (T <= 0) return cudaSuccess;
+  ce_grad_t_kernel<<<T, 512, 0, st>>>(logits, lse, tgt1, w1, tgt2, w2, V, dlogits);
   ++g_kernel_launches;
   return cudaGetLastError();
 }

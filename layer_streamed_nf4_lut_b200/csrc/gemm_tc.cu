@@ -18,7 +18,8 @@
 //   warp 14     lane 0 issues the raw NF4 TMA loads into a ring of their own, so they run
 //               ahead of the operand stages (a raw slot frees when its k-block is decoded);
 //   warps 12-15 epilogue: tcgen05.ld rows out of TMEM, scale, add residual / old value, store
-//               (or store an fp32 partial tile under split-K).
+//               (under split-K: store an fp32 partial tile; the tile's last split to finish
+//               sums all partials in split order and runs the normal epilogue).
 //
 // NF4 decode follows the double-quantised format: mhat = fp32(fp32(q8 * s2) + mean),
 // w = bf16_rn(fp32(code_value * mhat)), one float32 multiply per element.
@@ -558,6 +559,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
   float* lut = reinterpret_cast<float*>(ctrl);                       // 16 floats
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl + 64);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(ctrl + 68);
+  volatile int* last_flag = reinterpret_cast<volatile int*>(ctrl + 72);  // split-K: this CTA reduces
   float* seg_mean = reinterpret_cast<float*>(ctrl + 80);              // up to 3 NF4 tensors
   uint64_t* full = reinterpret_cast<uint64_t*>(ctrl + 128);
   uint64_t* empty = full + C::STAGES;
@@ -789,6 +791,45 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
         }
       }
     }
+    if (splits > 1) {
+      // the last split of this tile to finish sums every partial in split order (the same
+      // arithmetic, in the same order, as a separate reduction kernel would do)
+      __threadfence();
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (q == 0 && lane == 0) {
+        const int tile = blockIdx.y * gridDim.x + blockIdx.x;
+        const int old = atomicAdd(&p.tile_counters[tile], 1);
+        const int last = (old == splits - 1) ? 1 : 0;
+        if (last) p.tile_counters[tile] = 0;  // every split has counted: ready for the next launch
+        *last_flag = last;
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (*last_flag) {
+        __threadfence();
+#pragma unroll 1
+        for (int hc = 0; hc < MT * BN; hc += 32) {
+          const int h = hc / BN, cc = hc % BN;
+          const int row = m0 + h * UM + q * 32 + lane;
+          if (row >= p.M) continue;
+#pragma unroll 1
+          for (int g8 = 0; g8 < 4; ++g8) {
+            const int col = n0 + cc + g8 * 8;
+            if (col >= p.N) break;
+            float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            for (int sp = 0; sp < splits; ++sp) {
+              const float4* src =
+                  reinterpret_cast<const float4*>(p.workspace + (static_cast<long long>(sp) * p.M + row) * p.N + col);
+              const float4 a = __ldcg(src), b = __ldcg(src + 1);
+              v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w;
+              v[4] += b.x; v[5] += b.y; v[6] += b.z; v[7] += b.w;
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) v[j] *= p.alpha;
+            epilogue_store8(p, row, col, v);
+          }
+        }
+      }
+    }
   }
 
   tc_fence_before();
@@ -797,24 +838,6 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
-}
-
-// Sum of the split-K partial tiles in split order, then the normal epilogue.
-__global__ void splitk_reduce_kernel(const __grid_constant__ GemmParams p) {
-  const long long n8 = p.N / 8;
-  const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (idx >= static_cast<long long>(p.M) * n8) return;
-  const int row = static_cast<int>(idx / n8), col = static_cast<int>(idx % n8) * 8;
-  float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  for (int s = 0; s < p.splits; ++s) {
-    const float4* src = reinterpret_cast<const float4*>(p.workspace + (static_cast<long long>(s) * p.M + row) * p.N + col);
-    const float4 a = src[0], b = src[1];
-    v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w;
-    v[4] += b.x; v[5] += b.y; v[6] += b.z; v[7] += b.w;
-  }
-#pragma unroll
-  for (int j = 0; j < 8; ++j) v[j] *= p.alpha;
-  epilogue_store8(p, row, col, v);
 }
 
 // ---------------------------------------------------------------- host side
@@ -970,11 +993,6 @@ cudaError_t launch_tile(const GemmParams& p, cudaStream_t st) {
   }
   dim3 grid((p.N + BN - 1) / BN, (p.M + C::BM - 1) / C::BM, p.splits > 1 ? p.splits : 1);
   gemm_tc_kernel<MT, BN><<<grid, GEMM_THREADS, C::SMEM_BYTES, st>>>(p);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess || p.splits <= 1) return e;
-  const long long work = static_cast<long long>(p.M) * (p.N / 8);
-  splitk_reduce_kernel<<<static_cast<unsigned>((work + 255) / 256), 256, 0, st>>>(p);
-  ++g_kernel_launches;
   return cudaGetLastError();
 }
 
@@ -1081,12 +1099,14 @@ cudaError_t gemm_launch(const GemmParams& p_in, cudaStream_t st) {
       if (p.seg[s].K > 0 && p.seg[s].A.kind == OP_BF16_K)
         p.a_mode[s] = encode_kmajor_bf16(&p.tmapA[s], p.seg[s].A.ptr, p.seg[s].K, p.M, p.seg[s].A.ld, BM) ? 1 : 0;
   }
-  // split-K for grids that cannot fill the GPU (skinny LoRA GEMMs, long reductions)
+  // split-K for grids that leave SMs idle (the skinny LoRA GEMMs): at most one wave of CTAs,
+  // at least 16 k-blocks per split (a CTA's fixed cost, prologue + pipeline fill + epilogue, is
+  // worth a few k-blocks).  NF4 GEMMs with raw staging keep whole K: their per-CTA cost is
+  // higher and a partial tile of 256 x 128 fp32 costs more than the idle SMs return.
   p.splits = 1;
   const long long tiles = static_cast<long long>((p.N + BN - 1) / BN) * ((p.M + BM - 1) / BM);
-  if (p.workspace && tiles < 100 && nkb >= 8) {
-    long long sp = (2 * 148 + tiles - 1) / tiles;
-    sp = std::min<long long>(sp, nkb / 4);
+  if (p.workspace && p.tile_counters && !p.raw_tma && tiles <= p.n_counters) {
+    long long sp = std::min<long long>(148 / tiles, nkb / 16);
     sp = std::min<long long>(sp, 32);
     while (sp > 1 && static_cast<unsigned long long>(sp) * p.M * p.N * 4ull > p.ws_bytes) --sp;
     p.splits = static_cast<int>(sp < 1 ? 1 : sp);

@@ -53,6 +53,7 @@ struct GemmSeg {
 };
 
 constexpr int GEMM_MAX_SEG = 5;
+constexpr int GEMM_COUNTERS = 16384;  // split-K tile counters per workspace
 
 struct GemmParams {
   // filled by gemm_launch:
@@ -80,10 +81,13 @@ struct GemmParams {
   const void* residual;  // bf16, same layout as out (not with out_trans)
   long long ldr;
   int* err;
-  // split-K: when workspace is given, gemm_launch may split the K loop over `splits` CTAs that
-  // write fp32 partial tiles to the workspace; a second kernel sums them in split order
+  // split-K: when workspace and tile_counters are given, gemm_launch may split the K loop over
+  // `splits` CTAs that write fp32 partial tiles to the workspace; the last CTA of a tile to
+  // finish (counted in tile_counters, which it resets to 0) sums them in split order
   float* workspace;
   size_t ws_bytes;
+  int* tile_counters;  // n_counters ints, zero between launches
+  int n_counters;
   int splits;  // set by gemm_launch
 };
 
@@ -103,10 +107,18 @@ cudaError_t nf4_dequant_launch(const uint8_t* codes, const int8_t* q8, const flo
 struct AttnShape {
   int B, S, hq, hkv, d;
   long long ld_qkv;  // row stride (elements) of the [T, (hq+2hkv)d] qkv buffer
+  // Shared-prefix pair layout (pl > 0): each of the B blocks of S = pl + 2 rl rows holds one
+  // preference pair as [prefix (pl) | chosen response (rl) | rejected response (rl)]; the
+  // rejected rows sit at positions pl.. and see the prefix and their own earlier rows, never
+  // the chosen ones.  pl and rl are multiples of the 64-row tile.  pl = 0: plain causal rows.
+  int pl, rl;
 };
 cudaError_t attn_fwd_launch(const AttnShape& s, const uint16_t* qkv, uint16_t* o, float* lse, cudaStream_t st);
+// ws: fp32 scratch (16-byte aligned) for per-head-slice dK / dV partials when the kv grid
+// alone cannot fill the GPU; NULL / too small: no head slices.
 cudaError_t attn_bwd_launch(const AttnShape& s, const uint16_t* qkv, const uint16_t* o, const uint16_t* dout,
-                            const float* lse, float* delta, uint16_t* dqkv, cudaStream_t st);
+                            const float* lse, float* delta, uint16_t* dqkv, float* ws, size_t ws_bytes,
+                            cudaStream_t st);
 
 // ----------------------------------------------------------------- elementwise / row ops
 cudaError_t embed_launch(const int32_t* ids, const uint16_t* table, int T, int h, int V, uint16_t* out, int* err,
@@ -116,8 +128,10 @@ cudaError_t rmsnorm_fwd_launch(const uint16_t* x, const uint16_t* gamma, int T, 
 cudaError_t rmsnorm_bwd_launch(const uint16_t* dy, const uint16_t* x, const float* rstd, const uint16_t* gamma,
                                const uint16_t* dres, int T, int h, uint16_t* dx, cudaStream_t st);
 // tcos / tsin: [S_max, d/2] fp32 tables of cos / sin(pos * theta^(-2i/d)).
+// pack_rl > 0: rows of a block past S - pack_rl (the rejected response of a shared-prefix
+// pair block) take position (row - pack_rl).
 cudaError_t rope_launch(uint16_t* qkv, long long ld, int B, int S, int hq, int hkv, int d, const float* tcos,
-                        const float* tsin, int inverse, cudaStream_t st);
+                        const float* tsin, int inverse, cudaStream_t st, int pack_rl = 0);
 cudaError_t swiglu_fwd_launch(const uint16_t* gu, int T, int I, uint16_t* m, cudaStream_t st);
 cudaError_t swiglu_bwd_launch(const uint16_t* dm, const uint16_t* gu, int T, int I, uint16_t* dgu, cudaStream_t st);
 cudaError_t ce_rows_launch(const float* logits, int T, int V, const int32_t* ids, int B, int S, const uint8_t* mask,
@@ -132,6 +146,22 @@ cudaError_t pref_finish_launch(int kind, const float* lse, const float* tgt, int
                                const float* ref_logp, const uint8_t* labels, float beta, float gamma, float lam_or,
                                float lam_d, float lam_u, float* pi_out, float* loss_out, float* row_weight,
                                cudaStream_t st);
+// Loss closed forms on precomputed per-sequence sums, writing seq_w = -dL/dpi per sequence.
+cudaError_t dpo_loss_seqw_launch(const float* pi, const float* ref_logp, int n_pairs, float beta, float* loss_out,
+                                 float* seq_w, cudaStream_t st);
+cudaError_t pref_loss_seqw_launch(int kind, const float* pi, const float* ref_logp, const uint8_t* labels, int B,
+                                  int n_resp, float beta, float gamma, float lam_or, float lam_d, float lam_u,
+                                  float* loss_out, float* seq_w, cudaStream_t st);
+// Shared-prefix pair blocks: packing, two-target rows, per-pair log-prob sums, row weights.
+cudaError_t pair_pack_launch(const int32_t* ids, int P, int S, int pl, int V, int32_t* pids, int32_t* tgt1,
+                             int32_t* tgt2, int* err, cudaStream_t st);
+cudaError_t ce_rows_t_launch(const float* logits, int T, int V, const int32_t* tgt1, const int32_t* tgt2, float* lse,
+                             float* rt1, float* rt2, cudaStream_t st);
+cudaError_t pair_logp_launch(const float* lse, const float* rt1, const float* rt2, int P, int pl, int rl, float* out,
+                             cudaStream_t st);
+cudaError_t pair_rowweight_launch(const float* seq_w, int P, int pl, int rl, float* w1, float* w2, cudaStream_t st);
+cudaError_t ce_grad_t_launch(const float* logits, const float* lse, const int32_t* tgt1, const float* w1,
+                             const int32_t* tgt2, const float* w2, int T, int V, uint16_t* dlogits, cudaStream_t st);
 cudaError_t seq_logp_launch(const float* lse, const float* tgt, int B, int S, int resp_start, float* out,
                             cudaStream_t st);
 cudaError_t ce_grad_launch(const float* logits, const float* lse, const int32_t* ids, const float* row_weight, int B,

@@ -249,6 +249,11 @@ struct soup_model {
   int32_t* ids_dev = nullptr;
   uint8_t* mask_dev = nullptr;
   uint8_t* labels_dev = nullptr;  // KTO labels [B]
+  // shared-prefix pair blocks (preference steps with share_prefix): packed ids, the targets of
+  // each packed row (the last prefix row has two), their logits and row weights
+  int pack_pl = 0, pack_rl = 0;  // non-zero while a packed step runs
+  int32_t *pids = nullptr, *tgt1 = nullptr, *tgt2 = nullptr;
+  float *rowtgt2 = nullptr, *roww2 = nullptr, *seqw = nullptr;
   // scalars: [0] loss (f32), [1] device error word (int)
   int* scal = nullptr;
   float* quant_scratch = nullptr;  // absmax scratch for the quantiser
@@ -261,7 +266,7 @@ struct soup_model {
   // per-layer CUDA graphs of the step's layer calls (key: direction, layer, weight buffer,
   // activation buffers, shapes, LoRA flag)
   struct GraphKey {
-    int dir, layer, B, S, lora, pad;
+    int dir, layer, B, S, lora, pack;  // pack: shared-prefix length of a packed pair step (0: none)
     const void *base, *in, *out;
     bool operator==(const GraphKey& o) const { return std::memcmp(this, &o, sizeof(GraphKey)) == 0; }
   };
@@ -281,6 +286,16 @@ struct soup_model {
   std::unordered_map<GraphKey, GraphEntry, GraphKeyHash> graphs;
   cudaStream_t cap_stream = nullptr;
   int use_graphs = 1;
+  // low-priority stream for the LoRA weight-gradient GEMMs of a layer backward (they run
+  // beside the dX GEMMs), its fork / join events and its own split-K workspace
+  cudaStream_t grad_stream = nullptr;
+  cudaEvent_t fork_ev = nullptr, join_ev = nullptr;
+  float* gemm_ws2 = nullptr;
+  size_t gemm_ws2_bytes = 0;
+  int* gemm_cnt = nullptr;   // split-K tile counters of gemm_ws (zero between launches)
+  int* gemm_cnt2 = nullptr;  // ... of gemm_ws2
+  int concurrent_grads = 1;
+  int grads_forked = 0;
   // live profile: event pairs per launch, resolved into per-category totals
   int prof = 0;
   struct ProfRec {
@@ -508,6 +523,8 @@ GemmParams gemm_base(soup_model* m, int M, int N, void* out, long long ldo, int 
   p.err = m->scal + 1;
   p.workspace = m->gemm_ws;
   p.ws_bytes = m->gemm_ws_bytes;
+  p.tile_counters = m->gemm_cnt;
+  p.n_counters = GEMM_COUNTERS;
   std::memcpy(p.lut, codebook().v, sizeof(p.lut));
   return p;
 }
@@ -686,9 +703,10 @@ soup_status layer_forward(soup_model* m, int i, const LayerView& L, const uint16
   }
   const double rope_bytes = 4.0 * T * (c.n_heads + c.n_kv_heads) * c.head_dim;
   SOUP_TRY(launch(m, st, CAT_ROPE, 0, rope_bytes, "rope", [&] {
-    return rope_launch(A.qkv, QKV, B, S, c.n_heads, c.n_kv_heads, c.head_dim, m->rope_cos, m->rope_sin, 0, st);
+    return rope_launch(A.qkv, QKV, B, S, c.n_heads, c.n_kv_heads, c.head_dim, m->rope_cos, m->rope_sin, 0, st,
+                       m->pack_rl);
   }));
-  AttnShape as{B, S, c.n_heads, c.n_kv_heads, c.head_dim, QKV};
+  AttnShape as{B, S, c.n_heads, c.n_kv_heads, c.head_dim, QKV, m->pack_pl, m->pack_rl};
   const double attn_flops = 2.0 * B * c.n_heads * c.head_dim * static_cast<double>(S) * (S + 1);
   SOUP_TRY(launch(m, st, CAT_ATTN_FWD, attn_flops, 2.0 * T * QKV + 2.0 * T * qd + 4.0 * T * c.n_heads, "attention fwd",
                   [&] { return attn_fwd_launch(as, A.qkv, A.o, A.lse, st); }));
@@ -754,8 +772,14 @@ soup_status lora_grads(soup_model* m, int T, const uint16_t* g, long long ldg, i
                        long long ldu, float* dB, const uint16_t* x, long long ldx, int in, const uint16_t* vs,
                        long long ldv, int nv, float* dA, cudaStream_t st, bool do_dB, bool do_dA) {
   const int r = m->cfg.lora_r;
+  float* ws = (st == m->grad_stream) ? m->gemm_ws2 : m->gemm_ws;
+  const size_t ws_bytes = (st == m->grad_stream) ? m->gemm_ws2_bytes : m->gemm_ws_bytes;
+  int* cnt = (st == m->grad_stream) ? m->gemm_cnt2 : m->gemm_cnt;
   if (do_dB) {
     GemmParams p = gemm_base(m, out, r, dB, r, 1, 1.f);
+    p.workspace = ws;
+    p.ws_bytes = ws_bytes;
+    p.tile_counters = cnt;
     p.accumulate = 1;
     add_seg(p, T, opnd(OP_BF16_MN, g, ldg), opnd(OP_BF16_MN, us, ldu));
     SOUP_TRY(run_gemm(m, p, st, "lora dB"));
@@ -763,6 +787,9 @@ soup_status lora_grads(soup_model* m, int T, const uint16_t* g, long long ldg, i
   if (do_dA) {
     // dA^T [in, nv] = x^T v_s, written transposed into dA [nv, in]
     GemmParams p = gemm_base(m, in, nv, dA, in, 1, 1.f);
+    p.workspace = ws;
+    p.ws_bytes = ws_bytes;
+    p.tile_counters = cnt;
     p.accumulate = 1;
     p.out_trans = 1;
     add_seg(p, T, opnd(OP_BF16_MN, x, ldx), opnd(OP_BF16_MN, vs, ldv));
@@ -771,8 +798,39 @@ soup_status lora_grads(soup_model* m, int T, const uint16_t* g, long long ldg, i
   return SOUP_OK;
 }
 
+// The LoRA weight-gradient GEMMs (dA, dB) of a layer backward read only the main stream's
+// v = g B, g and saved activations, and write grad regions nothing reads before the step
+// ends: they run on a low-priority side stream beside the dX GEMMs, on SMs those leave idle.
+// The side stream forks after each v and joins before the layer call returns (the g buffers
+// are reused by the next layer).  Same kernels, same order per region: same bits.
+soup_status grads_fork(soup_model* m, cudaStream_t st, cudaStream_t* gs) {
+  *gs = st;
+  if (!m->concurrent_grads) return SOUP_OK;
+  SOUP_CK(cudaEventRecord(m->fork_ev, st));
+  SOUP_CK(cudaStreamWaitEvent(m->grad_stream, m->fork_ev, 0));
+  m->grads_forked = 1;
+  *gs = m->grad_stream;
+  return SOUP_OK;
+}
+soup_status grads_join(soup_model* m, cudaStream_t st) {
+  if (!m->grads_forked) return SOUP_OK;
+  m->grads_forked = 0;
+  SOUP_CK(cudaEventRecord(m->join_ev, m->grad_stream));
+  SOUP_CK(cudaStreamWaitEvent(st, m->join_ev, 0));
+  return SOUP_OK;
+}
+
+soup_status layer_backward_body(soup_model* m, int i, const LayerView& L, const uint16_t* dy, uint16_t* dx, int B,
+                                int S, cudaStream_t st);
 soup_status layer_backward(soup_model* m, int i, const LayerView& L, const uint16_t* dy, uint16_t* dx, int B, int S,
                            cudaStream_t st) {
+  const soup_status s1 = layer_backward_body(m, i, L, dy, dx, B, S, st);
+  const soup_status s2 = grads_join(m, st);  // also on errors: a capture must end joined
+  return s1 != SOUP_OK ? s1 : s2;
+}
+
+soup_status layer_backward_body(soup_model* m, int i, const LayerView& L, const uint16_t* dy, uint16_t* dx, int B,
+                                int S, cudaStream_t st) {
   const soup_model_config& c = m->cfg;
   Saved& A = m->saved[i];
   if (!A.valid || A.B != B || A.S != S) {
@@ -798,9 +856,12 @@ soup_status layer_backward(soup_model* m, int i, const LayerView& L, const uint1
     if (lora) add_seg(p, r, opnd(OP_BF16_K, m->vd, r), opnd(OP_BF16_MN, P + lora_off(c, i, 6, 0), I));
     SOUP_TRY(run_gemm(m, p, st, "down dX"));
   }
-  if (lora)
+  cudaStream_t gs = st;
+  if (lora) {
+    SOUP_TRY(grads_fork(m, st, &gs));
     SOUP_TRY(lora_grads(m, T, dy, h, h, A.ud, r, G + lora_off(c, i, 6, 1), A.m, I, I, m->vd, r, r,
-                        G + lora_off(c, i, 6, 0), st, true, true));
+                        G + lora_off(c, i, 6, 0), gs, true, true));
+  }
   SOUP_TRY(launch(m, st, CAT_SWIGLU, 0, 10.0 * T * I, "swiglu bwd",
                   [&] { return swiglu_bwd_launch(m->dm, A.gu, T, I, m->dgu, st); }));
   // ---- gate | up
@@ -821,11 +882,12 @@ soup_status layer_backward(soup_model* m, int i, const LayerView& L, const uint1
     SOUP_TRY(run_gemm(m, p, st, "gate/up dX"));
   }
   if (lora) {
+    SOUP_TRY(grads_fork(m, st, &gs));
     for (int q = 0; q < 2; ++q)
       SOUP_TRY(lora_grads(m, T, m->dgu + q * I, 2 * I, I, A.ugu + q * r, 2 * r, G + lora_off(c, i, 4 + q, 1), nullptr,
-                          0, 0, nullptr, 0, 0, nullptr, st, true, false));
+                          0, 0, nullptr, 0, 0, nullptr, gs, true, false));
     SOUP_TRY(lora_grads(m, T, nullptr, 0, 0, nullptr, 0, nullptr, A.n2, h, h, m->vgu, 2 * r, 2 * r,
-                        G + lora_off(c, i, 4, 0), st, false, true));
+                        G + lora_off(c, i, 4, 0), gs, false, true));
   }
   const double act = 2.0 * T * h;
   SOUP_TRY(launch(m, st, CAT_RMSNORM, 0, 4 * act + 4.0 * T, "rmsnorm bwd",
@@ -843,17 +905,23 @@ soup_status layer_backward(soup_model* m, int i, const LayerView& L, const uint1
     if (lora) add_seg(p, r, opnd(OP_BF16_K, m->vo, r), opnd(OP_BF16_MN, P + lora_off(c, i, 3, 0), qd));
     SOUP_TRY(run_gemm(m, p, st, "o dX"));
   }
-  if (lora)
+  if (lora) {
+    SOUP_TRY(grads_fork(m, st, &gs));
     SOUP_TRY(lora_grads(m, T, m->dx1, h, h, A.uo, r, G + lora_off(c, i, 3, 1), A.o, qd, qd, m->vo, r, r,
-                        G + lora_off(c, i, 3, 0), st, true, true));
+                        G + lora_off(c, i, 3, 0), gs, true, true));
+  }
   // ---- attention, RoPE
-  AttnShape as{B, S, c.n_heads, c.n_kv_heads, c.head_dim, QKV};
+  AttnShape as{B, S, c.n_heads, c.n_kv_heads, c.head_dim, QKV, m->pack_pl, m->pack_rl};
   const double attn_flops = 4.0 * B * c.n_heads * c.head_dim * static_cast<double>(S) * (S + 1);
   SOUP_TRY(launch(m, st, CAT_ATTN_BWD, attn_flops, 4.0 * T * QKV + 4.0 * T * qd + 8.0 * T * c.n_heads, "attention bwd",
-                  [&] { return attn_bwd_launch(as, A.qkv, A.o, m->da, A.lse, m->delta, m->dqkv, st); }));
+                  [&] {
+                    return attn_bwd_launch(as, A.qkv, A.o, m->da, A.lse, m->delta, m->dqkv, m->gemm_ws, m->gemm_ws_bytes,
+                                           st);
+                  }));
   const double rope_bytes = 4.0 * T * (c.n_heads + c.n_kv_heads) * c.head_dim;
   SOUP_TRY(launch(m, st, CAT_ROPE, 0, rope_bytes, "rope bwd", [&] {
-    return rope_launch(m->dqkv, QKV, B, S, c.n_heads, c.n_kv_heads, c.head_dim, m->rope_cos, m->rope_sin, 1, st);
+    return rope_launch(m->dqkv, QKV, B, S, c.n_heads, c.n_kv_heads, c.head_dim, m->rope_cos, m->rope_sin, 1, st,
+                       m->pack_rl);
   }));
   // ---- q | k | v
   const int off[3] = {0, qd, qd + kvd}, outs[3] = {qd, kvd, kvd};
@@ -874,11 +942,12 @@ soup_status layer_backward(soup_model* m, int i, const LayerView& L, const uint1
     SOUP_TRY(run_gemm(m, p, st, "qkv dX"));
   }
   if (lora) {
+    SOUP_TRY(grads_fork(m, st, &gs));
     for (int q = 0; q < 3; ++q)
       SOUP_TRY(lora_grads(m, T, m->dqkv + off[q], QKV, outs[q], A.uqkv + q * r, 3 * r, G + lora_off(c, i, q, 1),
-                          nullptr, 0, 0, nullptr, 0, 0, nullptr, st, true, false));
+                          nullptr, 0, 0, nullptr, 0, 0, nullptr, gs, true, false));
     SOUP_TRY(lora_grads(m, T, nullptr, 0, 0, nullptr, 0, nullptr, A.n1, h, h, m->vqkv, 3 * r, 3 * r,
-                        G + lora_off(c, i, 0, 0), st, false, true));
+                        G + lora_off(c, i, 0, 0), gs, false, true));
   }
   SOUP_TRY(launch(m, st, CAT_RMSNORM, 0, 4 * act + 4.0 * T, "rmsnorm bwd",
                   [&] { return rmsnorm_bwd_launch(m->dn, A.x, A.rstd1, L.gamma[0], m->dx1, T, h, dx, st); }));
@@ -895,6 +964,12 @@ soup_status head_forward(soup_model* m, const uint16_t* x, int B, int S, cudaStr
   GemmParams p = gemm_base(m, T, V, m->logits, V, 1, 1.f);
   add_seg(p, h, opnd(OP_BF16_K, m->hf, h), opnd(OP_BF16_K, m->lm_head, h));
   SOUP_TRY(run_gemm(m, p, st, "lm_head"));
+  if (m->pack_pl > 0) {
+    SOUP_TRY(launch(m, st, CAT_CE, 0, 4.0 * T * V, "ce rows", [&] {
+      return ce_rows_t_launch(m->logits, T, V, m->tgt1, m->tgt2, m->rowlse, m->rowtgt, m->rowtgt2, st);
+    }));
+    return SOUP_OK;
+  }
   SOUP_TRY(launch(m, st, CAT_CE, 0, 4.0 * T * V, "ce rows", [&] {
     return ce_rows_launch(m->logits, T, V, m->ids_dev, B, S, nullptr, 0, m->rowlse, m->rowtgt, m->scal + 1, st);
   }));
@@ -904,8 +979,11 @@ soup_status head_forward(soup_model* m, const uint16_t* x, int B, int S, cudaStr
 soup_status head_backward(soup_model* m, const uint16_t* x, int B, int S, uint16_t* dx, cudaStream_t st) {
   const soup_model_config& c = m->cfg;
   const int T = B * S, h = c.hidden, V = c.vocab;
-  SOUP_TRY(launch(m, st, CAT_CE, 0, 6.0 * T * V, "ce grad",
-                  [&] { return ce_grad_launch(m->logits, m->rowlse, m->ids_dev, m->roww, B, S, V, m->dlogits, st); }));
+  SOUP_TRY(launch(m, st, CAT_CE, 0, 6.0 * T * V, "ce grad", [&] {
+    return m->pack_pl > 0
+               ? ce_grad_t_launch(m->logits, m->rowlse, m->tgt1, m->roww, m->tgt2, m->roww2, T, V, m->dlogits, st)
+               : ce_grad_launch(m->logits, m->rowlse, m->ids_dev, m->roww, B, S, V, m->dlogits, st);
+  }));
   GemmParams p = gemm_base(m, T, h, m->dh, h, 0, 1.f);
   add_seg(p, V, opnd(OP_BF16_K, m->dlogits, V), opnd(OP_BF16_MN, m->lm_head, h));
   SOUP_TRY(run_gemm(m, p, st, "lm_head dX"));
@@ -935,6 +1013,7 @@ soup_status run_layer(soup_model* m, int dir, int i, const uint8_t* base, const 
   key.B = B;
   key.S = S;
   key.lora = lora;
+  key.pack = m->pack_pl;
   key.base = base;
   key.in = in;
   key.out = out;
@@ -1066,7 +1145,14 @@ soup_status read_scalars(soup_model* m, cudaStream_t st, float* loss_out) {
   return SOUP_OK;
 }
 
+soup_status do_step_body(soup_model* m, soup_loss kind, const soup_batch* bt, float* loss_out, cudaStream_t st);
 soup_status do_step(soup_model* m, soup_loss kind, const soup_batch* bt, float* loss_out, cudaStream_t st) {
+  const soup_status s = do_step_body(m, kind, bt, loss_out, st);
+  m->pack_pl = m->pack_rl = 0;
+  return s;
+}
+
+soup_status do_step_body(soup_model* m, soup_loss kind, const soup_batch* bt, float* loss_out, cudaStream_t st) {
   const soup_model_config& c = m->cfg;
   if (!m->embed || !m->lm_head || !m->final_gamma) {
     m->err = "head weights not set";
@@ -1109,50 +1195,82 @@ soup_status do_step(soup_model* m, soup_loss kind, const soup_batch* bt, float* 
   if (kind == SOUP_LOSS_KTO)
     SOUP_CK(cudaMemcpyAsync(m->labels_dev, bt->labels, static_cast<size_t>(B),
                             bt->ids_on_host ? cudaMemcpyHostToDevice : cudaMemcpyDeviceToDevice, st));
+  // Shared-prefix pair blocks: each pair's common prefix runs once, [prefix | chosen |
+  // rejected] (when the prefix and response lengths are multiples of the 64-row attention tile;
+  // otherwise the plain layout).  Bx x Sx are the rows the layers see.
+  const int pl = bt->prefix_len, rl = S - bt->prefix_len;
+  const bool share = bt->share_prefix && paired && pl >= 64 && pl % 64 == 0 && rl % 64 == 0;
+  const int Bx = share ? bt->n_pairs : B, Sx = share ? pl + 2 * rl : S, Tx = Bx * Sx;
+  const int32_t* ids_x = m->ids_dev;
+  if (share) {
+    SOUP_TRY(check_launch(m, pair_pack_launch(m->ids_dev, bt->n_pairs, S, pl, c.vocab, m->pids, m->tgt1, m->tgt2,
+                                              m->scal + 1, st),
+                          "pair pack"));
+    m->pack_pl = pl;
+    m->pack_rl = rl;
+    ids_x = m->pids;
+  }
   SOUP_CK(cudaMemsetAsync(m->lora_g, 0, m->lora_n * sizeof(float), st));
   const int saved_enabled = m->lora_enabled;
   uint16_t* xL = nullptr;
   if (needs_ref && bt->dpo_shared_load) {
     SOUP_TRY(streamer_warm(m, 0, 2));
-    SOUP_TRY(launch(m, st, CAT_EMBED, 0, 4.0 * T * c.hidden, "embed", [&] {
-      return embed_launch(m->ids_dev, m->embed, T, c.hidden, c.vocab, m->xa, m->scal + 1, st);
+    SOUP_TRY(launch(m, st, CAT_EMBED, 0, 4.0 * Tx * c.hidden, "embed", [&] {
+      return embed_launch(ids_x, m->embed, Tx, c.hidden, c.vocab, m->xa, m->scal + 1, st);
     }));
-    SOUP_TRY(launch(m, st, CAT_D2D, 0, 4.0 * T * c.hidden, "embed copy", [&] {
-      return cudaMemcpyAsync(m->xra, m->xa, static_cast<size_t>(T) * c.hidden * 2, cudaMemcpyDeviceToDevice, st);
+    SOUP_TRY(launch(m, st, CAT_D2D, 0, 4.0 * Tx * c.hidden, "embed copy", [&] {
+      return cudaMemcpyAsync(m->xra, m->xa, static_cast<size_t>(Tx) * c.hidden * 2, cudaMemcpyDeviceToDevice, st);
     }));
     uint16_t* xR = nullptr;
-    SOUP_TRY(stream_forward_pass_shared(m, B, S, st, &xR, &xL));
-    SOUP_TRY(head_forward(m, xR, B, S, st));
-    SOUP_TRY(check_launch(m, seq_logp_launch(m->rowlse, m->rowtgt, B, S, bt->prefix_len, m->ref, st), "ref logp"));
-    SOUP_TRY(head_forward(m, xL, B, S, st));
+    SOUP_TRY(stream_forward_pass_shared(m, Bx, Sx, st, &xR, &xL));
+    SOUP_TRY(head_forward(m, xR, Bx, Sx, st));
+    SOUP_TRY(check_launch(m,
+                          share ? pair_logp_launch(m->rowlse, m->rowtgt, m->rowtgt2, Bx, pl, rl, m->ref, st)
+                                : seq_logp_launch(m->rowlse, m->rowtgt, B, S, bt->prefix_len, m->ref, st),
+                          "ref logp"));
+    SOUP_TRY(head_forward(m, xL, Bx, Sx, st));
   } else {
   if (needs_ref) {
     // reference: same streamed base, LoRA off
     m->lora_enabled = 0;
     SOUP_TRY(streamer_warm(m, 0, 2));
-    SOUP_TRY(launch(m, st, CAT_EMBED, 0, 4.0 * T * c.hidden, "embed", [&] {
-    return embed_launch(m->ids_dev, m->embed, T, c.hidden, c.vocab, m->xa, m->scal + 1, st);
-  }));
-    soup_status s1 = stream_forward_pass(m, B, S, st, &xL);
+    SOUP_TRY(launch(m, st, CAT_EMBED, 0, 4.0 * Tx * c.hidden, "embed", [&] {
+      return embed_launch(ids_x, m->embed, Tx, c.hidden, c.vocab, m->xa, m->scal + 1, st);
+    }));
+    soup_status s1 = stream_forward_pass(m, Bx, Sx, st, &xL);
     if (s1 != SOUP_OK) {
       m->lora_enabled = saved_enabled;
       return s1;
     }
-    SOUP_TRY(head_forward(m, xL, B, S, st));
-    SOUP_TRY(check_launch(m, seq_logp_launch(m->rowlse, m->rowtgt, B, S, bt->prefix_len, m->ref, st), "ref logp"));
+    SOUP_TRY(head_forward(m, xL, Bx, Sx, st));
+    SOUP_TRY(check_launch(m,
+                          share ? pair_logp_launch(m->rowlse, m->rowtgt, m->rowtgt2, Bx, pl, rl, m->ref, st)
+                                : seq_logp_launch(m->rowlse, m->rowtgt, B, S, bt->prefix_len, m->ref, st),
+                          "ref logp"));
     m->lora_enabled = 1;
   }
   SOUP_TRY(streamer_warm(m, 0, 2));
-  SOUP_TRY(launch(m, st, CAT_EMBED, 0, 4.0 * T * c.hidden, "embed", [&] {
-    return embed_launch(m->ids_dev, m->embed, T, c.hidden, c.vocab, m->xa, m->scal + 1, st);
+  SOUP_TRY(launch(m, st, CAT_EMBED, 0, 4.0 * Tx * c.hidden, "embed", [&] {
+    return embed_launch(ids_x, m->embed, Tx, c.hidden, c.vocab, m->xa, m->scal + 1, st);
   }));
-  soup_status s2 = stream_forward_pass(m, B, S, st, &xL);
+  soup_status s2 = stream_forward_pass(m, Bx, Sx, st, &xL);
   m->lora_enabled = saved_enabled;
   if (s2 != SOUP_OK) return s2;
-  SOUP_TRY(head_forward(m, xL, B, S, st));
+  SOUP_TRY(head_forward(m, xL, Bx, Sx, st));
   }
   float* loss_dev = reinterpret_cast<float*>(m->scal);
-  if (kind == SOUP_LOSS_SFT) {
+  if (share) {
+    SOUP_TRY(check_launch(m, pair_logp_launch(m->rowlse, m->rowtgt, m->rowtgt2, Bx, pl, rl, m->pi, st), "pair logp"));
+    if (kind == SOUP_LOSS_DPO)
+      SOUP_TRY(check_launch(m, dpo_loss_seqw_launch(m->pi, m->ref, bt->n_pairs, bt->beta, loss_dev, m->seqw, st),
+                            "dpo loss"));
+    else
+      SOUP_TRY(check_launch(m, pref_loss_seqw_launch(static_cast<int>(kind), m->pi, m->ref, m->labels_dev, B, rl,
+                                                     bt->beta, bt->gamma, bt->lambda_or, bt->lambda_d, bt->lambda_u,
+                                                     loss_dev, m->seqw, st),
+                            "preference loss"));
+    SOUP_TRY(check_launch(m, pair_rowweight_launch(m->seqw, Bx, pl, rl, m->roww, m->roww2, st), "pair weights"));
+  } else if (kind == SOUP_LOSS_SFT) {
     SOUP_TRY(check_launch(m, sft_finish_launch(m->rowlse, m->rowtgt, m->ids_dev, B, S, mask, loss_dev, m->roww, st),
                           "sft loss"));
   } else if (kind == SOUP_LOSS_DPO) {
@@ -1166,9 +1284,9 @@ soup_status do_step(soup_model* m, soup_loss kind, const soup_batch* bt, float* 
                           "preference loss"));
   }
   uint16_t* other = (xL == m->xa) ? m->xb : m->xa;
-  SOUP_TRY(head_backward(m, xL, B, S, other, st));
+  SOUP_TRY(head_backward(m, xL, Bx, Sx, other, st));
   // backward ping-pongs between `other` and the buffer that held x_L (no longer needed)
-  SOUP_TRY(stream_backward_pass(m, B, S, other, xL, st));
+  SOUP_TRY(stream_backward_pass(m, Bx, Sx, other, xL, st));
   if (bt->apply_optimizer) {
     m->adam_t += 1;
     SOUP_TRY(launch(m, st, CAT_ADAMW, 0, 28.0 * m->lora_n, "adamw", [&] {
@@ -1203,6 +1321,9 @@ soup_status destroy_model(soup_model* m) {
   if (m->host_scal) cudaFreeHost(m->host_scal);
   clear_graphs(m);
   if (m->cap_stream) cudaStreamDestroy(m->cap_stream);
+  if (m->grad_stream) cudaStreamDestroy(m->grad_stream);
+  if (m->fork_ev) cudaEventDestroy(m->fork_ev);
+  if (m->join_ev) cudaEventDestroy(m->join_ev);
   for (auto& r : m->prof_pending) {
     cudaEventDestroy(r.a);
     cudaEventDestroy(r.b);
@@ -1278,6 +1399,14 @@ soup_status create_model(const soup_model_config* cfg, const soup_allocator* all
   {
     const char* e = std::getenv("SOUP_GRAPHS");
     m->use_graphs = (e && e[0] == '0') ? 0 : 1;
+    const char* g = std::getenv("SOUP_CONCURRENT_GRADS");
+    m->concurrent_grads = (g && g[0] == '0') ? 0 : 1;
+    int least = 0, greatest = 0;
+    if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess) return fail(SOUP_ERR_CUDA);
+    if (cudaStreamCreateWithPriority(&m->grad_stream, cudaStreamNonBlocking, least) != cudaSuccess ||
+        cudaEventCreateWithFlags(&m->fork_ev, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&m->join_ev, cudaEventDisableTiming) != cudaSuccess)
+      return fail(SOUP_ERR_CUDA);
   }
   m->copy_done.resize(nbuf);
   m->buf_free.resize(nbuf);
@@ -1308,7 +1437,9 @@ soup_status create_model(const soup_model_config* cfg, const soup_allocator* all
       alloc_into(m, m->delta, T * c.n_heads) || alloc_into(m, m->logits, T * V) || alloc_into(m, m->rowlse, T) ||
       alloc_into(m, m->rowtgt, T) || alloc_into(m, m->roww, T) || alloc_into(m, m->rstdf, T) ||
       alloc_into(m, m->pi, T) || alloc_into(m, m->ref, T) || alloc_into(m, m->ids_dev, T) ||
-      alloc_into(m, m->mask_dev, T) || alloc_into(m, m->labels_dev, T) || alloc_into(m, m->scal, 64))
+      alloc_into(m, m->mask_dev, T) || alloc_into(m, m->labels_dev, T) || alloc_into(m, m->pids, T) ||
+      alloc_into(m, m->tgt1, T) || alloc_into(m, m->tgt2, T) || alloc_into(m, m->rowtgt2, T) ||
+      alloc_into(m, m->roww2, T) || alloc_into(m, m->seqw, 256) || alloc_into(m, m->scal, 64))
     return fail(SOUP_ERR_OOM);
   {  // RoPE tables: angle = pos * theta^(-2i/d), computed in float64, stored as float32
     const int half = c.head_dim / 2;
@@ -1326,6 +1457,12 @@ soup_status create_model(const soup_model_config* cfg, const soup_allocator* all
   }
   m->gemm_ws_bytes = static_cast<size_t>(64) << 20;
   if (alloc_into(m, m->gemm_ws, m->gemm_ws_bytes / sizeof(float))) return fail(SOUP_ERR_OOM);
+  m->gemm_ws2_bytes = m->gemm_ws_bytes;
+  if (alloc_into(m, m->gemm_ws2, m->gemm_ws2_bytes / sizeof(float))) return fail(SOUP_ERR_OOM);
+  if (alloc_into(m, m->gemm_cnt, GEMM_COUNTERS) || alloc_into(m, m->gemm_cnt2, GEMM_COUNTERS)) return fail(SOUP_ERR_OOM);
+  if (cudaMemset(m->gemm_cnt, 0, GEMM_COUNTERS * sizeof(int)) != cudaSuccess ||
+      cudaMemset(m->gemm_cnt2, 0, GEMM_COUNTERS * sizeof(int)) != cudaSuccess)
+    return fail(SOUP_ERR_CUDA);
   if (cudaMemset(m->scal, 0, 64 * sizeof(int)) != cudaSuccess) return fail(SOUP_ERR_CUDA);
   m->lora_n = lora_numel_of(c);
   if (alloc_into(m, m->lora_bf16, m->lora_n)) return fail(SOUP_ERR_OOM);

@@ -192,7 +192,8 @@ class SoupModel:
 
     def step(self, ids, loss: str = "sft", mask=None, n_pairs: int = 0, prefix_len: int = 0, beta: float = 0.1,
              lr: float = 2e-5, apply_optimizer: bool = True, dpo_shared_load: bool = False, labels=None,
-             gamma: float = 0.0, lambda_or: float = 0.1, lambda_d: float = 1.0, lambda_u: float = 1.0) -> float:
+             gamma: float = 0.0, lambda_or: float = 0.1, lambda_d: float = 1.0, lambda_u: float = 1.0,
+             share_prefix: bool = False) -> float:
         """ids: int32 [B, S] as a cuda tensor, or as host memory (numpy / cpu tensor: copied by the
         library); mask (SFT) and labels (KTO, uint8 [B]) in the same memory space as ids."""
         b = Batch()
@@ -234,6 +235,7 @@ class SoupModel:
         b.lr, b.apply_optimizer = float(lr), 1 if apply_optimizer else 0
         b.dpo_shared_load = 1 if dpo_shared_load else 0
         b.gamma, b.lambda_or, b.lambda_d, b.lambda_u = float(gamma), float(lambda_or), float(lambda_d), float(lambda_u)
+        b.share_prefix = 1 if share_prefix else 0
         out = c_float()
         self._ck(lib.soup_step(self.h, _lib.LOSS_KINDS[loss], byref(b), byref(out), _stream_ptr()))
         return out.value

@@ -165,3 +165,22 @@ def test_dpo_shared_load_schedule_same_bits_fewer_loads():
         assert loads_re == 3 * L - 4 and loads_sh == 2 * L - 4
     finally:
         p.close()
+
+
+def test_side_stream_grads_same_bits(monkeypatch):
+    """LoRA weight gradients computed on the side stream (default) equal those computed in
+    line on the main stream, bit for bit."""
+    cfg = dict(TINY4, batch=4)
+    ids = torch.from_numpy(synth.token_batch(cfg, 48)).cuda()
+    out = {}
+    for flag in ("1", "0"):
+        monkeypatch.setenv("SOUP_CONCURRENT_GRADS", flag)
+        p = Pair(TINY4, seed=19, modes=("streamed",), want_oracle=False, max_tokens=4 * 64)
+        try:
+            gm = p.models["streamed"]
+            losses = [gm.step(ids, apply_optimizer=False) for _ in range(3)]  # eager, capture, replay
+            out[flag] = (losses, gm.lora_grads.clone())
+        finally:
+            p.close()
+    assert out["1"][0] == out["0"][0]
+    assert torch.equal(out["1"][1].view(torch.int32), out["0"][1].view(torch.int32))
