@@ -82,13 +82,16 @@ struct GemmParams {
   long long ldr;
   int* err;
   // split-K: when workspace and tile_counters are given, gemm_launch may split the K loop over
-  // `splits` CTAs that write fp32 partial tiles to the workspace; the last CTA of a tile to
-  // finish (counted in tile_counters, which it resets to 0) sums them in split order
+  // `splits` CTAs that write fp32 partial tiles to the workspace; they are summed in split order
+  // by the last CTA of a tile to finish (counted in tile_counters, which it resets to 0) or by
+  // a second kernel
   float* workspace;
   size_t ws_bytes;
   int* tile_counters;  // n_counters ints, zero between launches
   int n_counters;
-  int splits;  // set by gemm_launch
+  int splits;          // set by gemm_launch
+  int fused_reduce;    // set by gemm_launch: 1 = the tile's last split sums the partials,
+                       // 0 = a second kernel sums them (many splits: the sum runs wide)
 };
 
 // Launch C = sum_seg A_seg B_seg^T on the tcgen05 tensor cores. Returns cudaError_t of launch.
