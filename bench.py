@@ -333,7 +333,8 @@ def run_soup(args, wl, rank, world, local_rank):
     if dom:
         d = kern[dom]
         per_launch_ms = d["total_ms"] / d["launches"]
-        if d["flops"] > 0:
+        ridge = pk["bf16_sustained"] * 1e12 / (pk["hbm_gbs"] * 1e9)  # flop / byte
+        if d["flops"] > 0 and d["flops"] / max(d["bytes"], 1.0) >= ridge:
             achieved = d["flops"] / d["launches"] / (per_launch_ms * 1e-3) / 1e12
             roofline = {"bound": "tensor", "kernel": dom, "achieved": round(achieved, 2),
                         "peak": pk["bf16_sustained"], "unit": "TFLOP/s", "frac": round(achieved / pk["bf16_sustained"], 4),

@@ -1476,8 +1476,28 @@ cudaError_t gemm_launch(const GemmParams& p_in, cudaStream_t st) {
   // Tile choice: MT 128-row halves x BN columns.  Time ~ waves x per-tile time, with the per-tile
   // time proportional to the k-blocks and a per-k-block cost measured on B200 for each tile
   // shape (NF4 GEMMs at M = 512 and 2048): 2x128 50, 1x256 60, 1x128 38, 2x64 47, 1x64 36.
+  // GEMMs without an NF4 operand have no decode: a k-block costs about the issuing thread's
+  // MT x 4 tcgen05.mma instructions whatever N is (~100 cycles each), so wider tiles are
+  // nearly free per k-block; the 1x256 tile keeps 3 stages there, hence its small surcharge.
+  bool has_nf4 = false;
+  for (int s = 0; s < p.nseg; ++s)
+    if (p.seg[s].K > 0 && (p.seg[s].B.kind == OP_NF4_K || p.seg[s].B.kind == OP_NF4_MN)) has_nf4 = true;
   const int cand[5][2] = {{2, 128}, {1, 256}, {1, 128}, {2, 64}, {1, 64}};
-  const double unit[5] = {50.0, 60.0, 38.0, 47.0, 36.0};
+  const double unit_nf4[5] = {50.0, 60.0, 38.0, 47.0, 36.0};
+  const double unit_bf16[5] = {64.0, 40.0, 36.0, 64.0, 36.0};
+  const double* unit = has_nf4 ? unit_nf4 : unit_bf16;
+  // split-K for grids that leave SMs idle (the skinny LoRA GEMMs; never NF4): up to two waves
+  // of CTAs, at least 4 k-blocks per split (a CTA of these runs at the issuing thread's rate,
+  // so spreading K shortens the GEMM).  The cost below includes the split and, past 4 partials,
+  // the wide reduction kernel (~500 units).
+  auto split_for = [&](long long tiles) -> long long {
+    if (!p.workspace || !p.tile_counters || has_nf4 || tiles >= 100 || nkb < 8 || tiles > p.n_counters) return 1;
+    long long sp = (2 * 148 + tiles - 1) / tiles;
+    sp = std::min<long long>(sp, nkb / 4);
+    sp = std::min<long long>(sp, 32);
+    while (sp > 1 && static_cast<unsigned long long>(sp) * p.M * p.N * 4ull > p.ws_bytes) --sp;
+    return sp < 1 ? 1 : sp;
+  };
   int MT = 1, BN = 128;
   double best = 1e300;
   for (int ci = 0; ci < 5; ++ci) {
@@ -1486,8 +1506,10 @@ cudaError_t gemm_launch(const GemmParams& p_in, cudaStream_t st) {
     if (bn > 64 && p.N <= 64) continue;
     if (bn > 128 && p.N <= 128) continue;
     const long long tl = static_cast<long long>((p.N + bn - 1) / bn) * ((p.M + UM * mt - 1) / (UM * mt));
-    const long long waves = (tl + 147) / 148;
-    const double cost = static_cast<double>(waves) * (static_cast<double>(nkb) + 2.0) * unit[ci];
+    const long long sp = split_for(tl);
+    const long long waves = (tl * sp + 147) / 148;
+    const double cost = static_cast<double>(waves) * (static_cast<double>((nkb + sp - 1) / sp) + 2.0) * unit[ci] +
+                        (sp > 4 ? 500.0 : 0.0);
     if (cost < best * 0.999) {
       best = cost;
       MT = mt;
@@ -1544,20 +1566,9 @@ cudaError_t gemm_launch(const GemmParams& p_in, cudaStream_t st) {
       if (p.seg[s].K > 0 && p.seg[s].A.kind == OP_BF16_K)
         p.a_mode[s] = encode_kmajor_bf16(&p.tmapA[s], p.seg[s].A.ptr, p.seg[s].K, p.M, p.seg[s].A.ld, BM) ? 1 : 0;
   }
-  // split-K for grids that leave SMs idle (the skinny LoRA GEMMs).  A CTA of these runs at
-  // the single issuing thread's rate, one tcgen05.mma per ~100 cycles (measured), so a k-block
-  // costs the same few hundred cycles whatever the tile: spreading K over up to two waves of
-  // CTAs (at least 4 k-blocks each) shortens the GEMM.  NF4 GEMMs with raw staging keep whole
-  // K: the 96-tile q|k|v GEMM ran 105 us split four ways against 65 us whole.
-  p.splits = 1;
+  // NF4 GEMMs keep whole K (the 96-tile q|k|v GEMM ran 105 us split four ways, 65 us whole)
   const long long tiles = static_cast<long long>((p.N + BN - 1) / BN) * ((p.M + BM - 1) / BM);
-  if (p.workspace && p.tile_counters && !p.raw_tma && tiles <= p.n_counters && tiles < 100 && nkb >= 8) {
-    long long sp = (2 * 148 + tiles - 1) / tiles;
-    sp = std::min<long long>(sp, nkb / 4);
-    sp = std::min<long long>(sp, 32);
-    while (sp > 1 && static_cast<unsigned long long>(sp) * p.M * p.N * 4ull > p.ws_bytes) --sp;
-    p.splits = static_cast<int>(sp < 1 ? 1 : sp);
-  }
+  p.splits = p.raw_tma ? 1 : static_cast<int>(split_for(tiles));
   // up to 4 partials the tile's last CTA sums them; more run through the wide reduction
   // kernel (measured: 16-32 partials summed by one CTA per tile cost more than the launch)
   p.fused_reduce = p.splits <= 4 ? 1 : 0;

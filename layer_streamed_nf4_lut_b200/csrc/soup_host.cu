@@ -805,7 +805,9 @@ soup_status lora_grads(soup_model* m, int T, const uint16_t* g, long long ldg, i
 // are reused by the next layer).  Same kernels, same order per region: same bits.
 soup_status grads_fork(soup_model* m, cudaStream_t st, cudaStream_t* gs) {
   *gs = st;
-  if (!m->concurrent_grads) return SOUP_OK;
+  // (not while profiling: per-launch event times of overlapping kernels would count each
+  // other's time)
+  if (!m->concurrent_grads || m->prof) return SOUP_OK;
   SOUP_CK(cudaEventRecord(m->fork_ev, st));
   SOUP_CK(cudaStreamWaitEvent(m->grad_stream, m->fork_ev, 0));
   m->grads_forked = 1;
