@@ -888,348 +888,6 @@ __global__ void splitk_reduce_kernel(const __grid_constant__ GemmParams p) {
   epilogue_store8(p, row, col, v);
 }
 
-// ---------------------------------------------------------------- the two-SM kernel
-// A cluster of two CTAs computes one 256 x BN2 tile with tcgen05.mma.cta_group::2: CTA r
-// holds rows [128 r, 128 r + 128) of the A tile and rows [r BN2/2, (r+1) BN2/2) of the B tile
-// in its shared memory, at the same offsets; one instruction of the leader (rank 0) multiplies
-// the whole 256 x BN2 x 16 block on both SMs' tensor cores and each CTA's TMEM receives its
-// 128 output rows.  Against the one-SM kernel an MMA instruction carries 4x the work (M 256,
-// N 256), which matters because a single thread issues them at ~100 cycles apiece, and each
-// SM dequantises only half of the B tile for 256 activation rows.
-//   * both CTAs' producers dequantise their B half and arrive on the LEADER's full barrier
-//     (remote arrive through mapa); both CTAs' operand TMA loads (.cta_group::2) complete
-//     their bytes on the leader's barrier, whose expected count the leader sets for both;
-//   * the leader's commits multicast to both CTAs' empty barriers (and finally to done);
-//   * raw NF4 staging stays per CTA (local TMA into a local ring).
-// Used for NF4 GEMMs (forward and dX) with raw staging, M >= 256; no split-K.
-template <int BN2>
-struct Gemm2Cfg {
-  static constexpr int BNH = BN2 / 2;  // B rows per CTA
-  static constexpr int A_BYTES = UM * 128;
-  static constexpr int B_BYTES = BNH * 128;
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int RAW_CODE_BYTES = BNH * 32;
-  static constexpr int RAW_Q8_BYTES = (BNH > 64 ? BNH : 64) * 16;
-  static constexpr int RAW_BYTES = RAW_CODE_BYTES + RAW_Q8_BYTES;
-  static constexpr int CTRL_BYTES = 640;
-  static constexpr int AVAIL = SMEM_LIMIT - 1024 - CTRL_BYTES;
-  static constexpr int STAGES_FIT = (AVAIL - 4 * RAW_BYTES) / STAGE_BYTES;
-  static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
-  static constexpr int RAW_FIT = (AVAIL - STAGES * STAGE_BYTES) / RAW_BYTES;
-  static constexpr int RAW_SLOTS = RAW_FIT > 16 ? 16 : RAW_FIT;
-  static constexpr int TMEM_COLS = BN2;
-  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + RAW_SLOTS * RAW_BYTES + CTRL_BYTES;
-};
-
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ uint32_t mapa_rank(uint32_t local_addr, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_addr), "r"(rank));
-  return r;
-}
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
-}
-__device__ __forceinline__ void cluster_sync() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_alloc2(uint32_t* slot, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot)), "r"(ncols)
-               : "memory");
-}
-__device__ __forceinline__ void tmem_relinquish2() {
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_dealloc2(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
-}
-__device__ __forceinline__ void tc_mma2_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                            uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-// commit of the leader's MMAs to the barrier at the same offset in both CTAs of the pair
-__device__ __forceinline__ void tc_commit2_both(uint64_t* bar) {
-  asm volatile(
-      "{\n\t.reg .b16 m;\n\t"
-      "mov.b16 m, 3;\n\t"
-      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], m;\n\t}" ::"r"(
-          smem_u32(bar))
-      : "memory");
-}
-// operand TMA load whose bytes complete on the pair leader's barrier (cluster address)
-__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, int x, int y, uint32_t bar_leader) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
-      "[%4];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar_leader)
-      : "memory");
-}
-__device__ __forceinline__ void mbar_arrive_expect_tx_local(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
-}
-
-template <int BN2>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
-    gemm_tc2_kernel(const __grid_constant__ GemmParams p) {
-  using C = Gemm2Cfg<BN2>;
-  constexpr int BNH = C::BNH;
-  extern __shared__ uint8_t smem_raw[];
-  const uint32_t raw_addr = smem_u32(smem_raw);
-  uint8_t* base = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
-  uint8_t* raw_base = base + C::STAGES * C::STAGE_BYTES;
-  uint8_t* ctrl = raw_base + C::RAW_SLOTS * C::RAW_BYTES;
-  float* lut = reinterpret_cast<float*>(ctrl);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl + 64);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(ctrl + 68);
-  float* seg_mean = reinterpret_cast<float*>(ctrl + 80);
-  uint64_t* full = reinterpret_cast<uint64_t*>(ctrl + 128);
-  uint64_t* empty = full + C::STAGES;
-  uint64_t* raw_full = empty + C::STAGES;
-  uint64_t* raw_empty = raw_full + C::RAW_SLOTS;
-  uint64_t* done = raw_empty + C::RAW_SLOTS;
-  static_assert(128 + 8 * (2 * C::STAGES + 2 * C::RAW_SLOTS + 1) <= C::CTRL_BYTES, "control block overflow");
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t rank = cluster_ctarank();
-  const bool leader = rank == 0;
-  const int np0 = (blockIdx.x >> 1) * BN2;        // the pair's first output column
-  const int n0 = np0 + static_cast<int>(rank) * BNH;  // this CTA's B rows
-  const int m0 = blockIdx.y * (2 * UM) + static_cast<int>(rank) * UM;  // this CTA's A / output rows
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(&full[s], 1 + 2 * (GROUP_THREADS / 32));  // leader's TMA issuer + 4 producer warps x 2 CTAs
-      mbar_init(&empty[s], 1);                             // the leader's MMA commit
-    }
-    for (int r = 0; r < C::RAW_SLOTS; ++r) {
-      mbar_init(&raw_full[r], 1);
-      mbar_init(&raw_empty[r], GROUP_THREADS / 32);
-    }
-    mbar_init(done, 1);
-    *abort_flag = 0;
-    mbar_fence_init();
-  }
-  if (threadIdx.x < 16) lut[threadIdx.x] = p.lut[threadIdx.x];
-  if (threadIdx.x >= 32 && threadIdx.x < 32 + p.nf4.nseg) seg_mean[threadIdx.x - 32] = *p.nf4.seg[threadIdx.x - 32].mean;
-  if (warp == EPI_WARP0) {
-    tmem_alloc2(tmem_slot, C::TMEM_COLS);
-    tmem_relinquish2();
-  }
-  tc_fence_before();
-  __syncthreads();
-  cluster_sync();  // the peer's barriers are initialised before any remote arrive
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-
-  // k-block list: segments active for the PAIR's columns (both CTAs walk the same list)
-  int nkb = 0;
-  for (int s = 0; s < p.nseg; ++s)
-    if (seg_active(p.seg[s], np0, BN2)) nkb += (p.seg[s].K + BK - 1) / BK;
-  const bool seg0_raw = seg_active(p.seg[0], np0, BN2);
-  const int n_raw = seg0_raw ? (p.seg[0].K + BK - 1) / BK : 0;
-
-  if (warp < PRODUCER_WARPS) {
-    const int grp = warp >> 2, gtid = threadIdx.x & (GROUP_THREADS - 1);
-    const float(&cb)[16] = p.lut;
-    const uint32_t full_leader0 = mapa_rank(smem_u32(&full[0]), 0);
-    if (n_raw > 0) {
-      // raw NF4 k-blocks of this group; next k-block's group scales loaded during this decode
-      const bool fwd = p.seg[0].B.kind == OP_NF4_K;
-      ScaleRegs<BNH> cur, nxt;
-      if (grp < n_raw) load_scales<BNH>(p, fwd, n0, grp, gtid, nxt);
-      for (int kb = grp; kb < n_raw; kb += GROUPS) {
-        const int kk = kb;
-        cur = nxt;
-        if (kb + GROUPS < n_raw) load_scales<BNH>(p, fwd, n0, kk + GROUPS, gtid, nxt);
-        const int st = kb % C::STAGES;
-        const uint32_t ph = static_cast<uint32_t>(kb / C::STAGES) & 1u;
-        uint8_t* As = base + st * C::STAGE_BYTES;
-        uint8_t* Bs = As + C::A_BYTES;
-        const int rs = kb % C::RAW_SLOTS;
-        const uint32_t rph = static_cast<uint32_t>(kb / C::RAW_SLOTS) & 1u;
-        const uint8_t* Rc = raw_base + rs * C::RAW_BYTES;
-        const uint8_t* Rq = Rc + C::RAW_CODE_BYTES;
-        mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, p.err);
-        mbar_wait_bounded(&raw_full[rs], rph, abort_flag, p.err);
-        if (fwd) {
-          decode_fwd_raw<BNH>(p.nf4, nf4_seg_of(p.nf4, n0), cb, seg_mean, n0, p.N, kk, Rc, Rq, Bs, gtid, cur.v);
-        } else {
-          const int k0 = kk * BK;
-          decode_dx_raw<BNH>(p.nf4, nf4_seg_of(p.nf4, k0), cb, seg_mean, n0, p.N, k0, ((n0 >> 6) >> 4) << 4, Rc, Rq,
-                             Bs, gtid, cur.v);
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&raw_empty[rs]);
-        if (p.a_mode[0] == 0) load_tile<UM>(p.seg[0].A, p.nf4, lut, seg_mean, p.seg[0].K, m0, p.M, kk * BK, As, gtid);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_remote(full_leader0 + 8u * static_cast<uint32_t>(st));
-      }
-    }
-    int kb = 0;
-    for (int s = 0; s < p.nseg; ++s) {
-      const GemmSeg& sg = p.seg[s];
-      if (!seg_active(sg, np0, BN2)) continue;
-      const int nk = (sg.K + BK - 1) / BK;
-      if (s == 0) {  // raw NF4 segment: handled above
-        kb += nk;
-        continue;
-      }
-      for (int kk = 0; kk < nk; ++kk, ++kb) {
-        if ((kb % GROUPS) != grp) continue;
-        const int st = kb % C::STAGES;
-        const uint32_t ph = static_cast<uint32_t>(kb / C::STAGES) & 1u;
-        uint8_t* As = base + st * C::STAGE_BYTES;
-        uint8_t* Bs = As + C::A_BYTES;
-        mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, p.err);
-        if (p.b_mode[s] == 0) load_tile<BNH>(sg.B, p.nf4, lut, seg_mean, sg.K, n0, p.N, kk * BK, Bs, gtid);
-        if (p.a_mode[s] == 0) load_tile<UM>(sg.A, p.nf4, lut, seg_mean, sg.K, m0, p.M, kk * BK, As, gtid);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_remote(full_leader0 + 8u * static_cast<uint32_t>(st));
-      }
-    }
-  } else {
-    if (warp == EPI_WARP0 + 1 && lane == 0) {
-      // operand TMA (both CTAs): bytes complete on the leader's full barrier
-      int kb = 0;
-      for (int s = 0; s < p.nseg; ++s) {
-        const GemmSeg& sg = p.seg[s];
-        if (!seg_active(sg, np0, BN2)) continue;
-        const int nk = (sg.K + BK - 1) / BK;
-        const bool raw = (s == 0);
-        for (int kk = 0; kk < nk; ++kk, ++kb) {
-          const int st = kb % C::STAGES;
-          const uint32_t ph = static_cast<uint32_t>(kb / C::STAGES) & 1u;
-          mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, p.err);
-          uint8_t* As = base + st * C::STAGE_BYTES;
-          uint8_t* Bs = As + C::A_BYTES;
-          const int am = p.a_mode[s], bm = raw ? 0 : p.b_mode[s];
-          const uint32_t tx = (am ? C::A_BYTES : 0) + (bm ? C::B_BYTES : 0);
-          const uint32_t bar_l = mapa_rank(smem_u32(&full[st]), 0);
-          if (leader) {
-            if (tx)
-              mbar_arrive_expect_tx_local(&full[st], 2 * tx);  // both CTAs' bytes
-            else
-              mbar_arrive(&full[st]);
-          }
-          if (tx) {
-            const int k0 = kk * BK;
-            if (am == 1) {
-              tma_load_2d_pair(As, &p.tmapA[s], k0, m0, bar_l);
-            } else if (am == 2) {
-#pragma unroll
-              for (int i = 0; i < UM / 64; ++i) tma_load_2d_pair(As + i * 8192, &p.tmapA[s], m0 + 64 * i, k0, bar_l);
-            }
-            if (bm == 1) {
-              tma_load_2d_pair(Bs, &p.tmapB[s], k0, n0 - p.b_row0[s], bar_l);
-            } else if (bm == 2) {
-#pragma unroll
-              for (int i = 0; i < BNH / 64; ++i) tma_load_2d_pair(Bs + i * 8192, &p.tmapB[s], n0 + 64 * i, k0, bar_l);
-            }
-          }
-        }
-      }
-    }
-    if (warp == EPI_WARP0 + 2 && lane == 0 && n_raw > 0) {
-      // raw NF4 codes / absmax of this CTA's B rows, into the local ring
-      const GemmSeg& sg = p.seg[0];
-      for (int kb = 0; kb < n_raw; ++kb) {
-        const int kk = kb;
-        const int rs = kb % C::RAW_SLOTS;
-        const uint32_t rph = static_cast<uint32_t>(kb / C::RAW_SLOTS) & 1u;
-        mbar_wait_bounded(&raw_empty[rs], rph ^ 1u, abort_flag, p.err);
-        uint8_t* Rc = raw_base + rs * C::RAW_BYTES;
-        uint8_t* Rq = Rc + C::RAW_CODE_BYTES;
-        if (sg.B.kind == OP_NF4_K) {
-          const int si = nf4_seg_of(p.nf4, n0);
-          const int y = n0 - p.nf4.seg[si].row_begin;
-          mbar_arrive_expect_tx(&raw_full[rs], BNH * 32 + BNH * 16);
-          tma_load_2d(Rc, &p.tmapCodes[si], kk * (BK / 2), y, &raw_full[rs]);
-          tma_load_2d(Rq, &p.tmapQ8[si], (kk >> 4) << 4, y, &raw_full[rs]);
-        } else {
-          const int k0 = kk * BK;
-          const int si = nf4_seg_of(p.nf4, k0);
-          const int y = k0 - p.nf4.seg[si].row_begin;
-          mbar_arrive_expect_tx(&raw_full[rs], 64 * (BNH / 2) + 64 * 16);
-          tma_load_2d(Rc, &p.tmapCodes[si], n0 / 2, y, &raw_full[rs]);
-          tma_load_2d(Rq, &p.tmapQ8[si], ((n0 >> 6) >> 4) << 4, y, &raw_full[rs]);
-        }
-      }
-    }
-    if (warp == EPI_WARP0 && lane == 0 && leader) {
-      // MMA issuer (leader only): M = 256 over both CTAs, N = BN2
-      int kb = 0;
-      for (int s = 0; s < p.nseg; ++s) {
-        const GemmSeg& sg = p.seg[s];
-        if (!seg_active(sg, np0, BN2)) continue;
-        const int nk = (sg.K + BK - 1) / BK;
-        const bool b_mn = ((s == 0) && sg.B.kind == OP_NF4_MN) || p.b_mode[s] == 2;
-        const bool a_mn = p.a_mode[s] == 2;
-        const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) |
-                               ((b_mn ? 1u : 0u) << 16) | (static_cast<uint32_t>(BN2 >> 3) << 17) |
-                               (static_cast<uint32_t>((2 * UM) >> 4) << 24);
-        for (int kk = 0; kk < nk; ++kk, ++kb) {
-          const int st = kb % C::STAGES;
-          const uint32_t ph = static_cast<uint32_t>(kb / C::STAGES) & 1u;
-          mbar_wait_bounded(&full[st], ph, abort_flag, p.err);
-          tc_fence_after();
-          const uint32_t a_addr = smem_u32(base + st * C::STAGE_BYTES);
-          const uint32_t b_addr = a_addr + C::A_BYTES;
-#pragma unroll
-          for (int j = 0; j < BK / 16; ++j) {
-            const uint64_t bd = b_mn ? sw128_mnmajor_desc(b_addr + j * 2048) : sw128_kmajor_desc(b_addr + j * 32);
-            const uint64_t ad = a_mn ? sw128_mnmajor_desc(a_addr + j * 2048) : sw128_kmajor_desc(a_addr + j * 32);
-            tc_mma2_f16(tmem, ad, bd, idesc, (kb > 0 || j > 0) ? 1u : 0u);
-          }
-          tc_commit2_both(&empty[st]);
-        }
-      }
-      tc_commit2_both(done);
-    }
-    __syncwarp();
-    // epilogue: this CTA's 128 rows x BN2 columns
-    const int q = warp - EPI_WARP0;
-    mbar_wait_bounded(done, 0u, abort_flag, p.err);
-    tc_fence_after();
-    const bool any_k = nkb > 0;
-#pragma unroll 1
-    for (int hc = 0; hc < BN2; hc += 32) {
-      const int row = m0 + q * 32 + lane;
-      uint32_t r[32];
-      tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(hc), r);
-      tmem_ld_wait();
-      if (row >= p.M) continue;
-#pragma unroll
-      for (int g8 = 0; g8 < 4; ++g8) {
-        const int col = np0 + hc + g8 * 8;
-        if (col >= p.N) break;
-        float v[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) v[j] = any_k ? p.alpha * __uint_as_float(r[g8 * 8 + j]) : 0.f;
-        epilogue_store8(p, row, col, v);
-      }
-    }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  cluster_sync();  // no CTA of the pair leaves while the other may still touch its memory
-  if (warp == EPI_WARP0) {
-    tc_fence_after();
-    tmem_dealloc2(tmem, C::TMEM_COLS);
-  }
-}
-
 // ---------------------------------------------------------------- host side
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -1391,37 +1049,6 @@ cudaError_t launch_tile(const GemmParams& p, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-template <int BN2>
-cudaError_t launch_pair(const GemmParams& p, cudaStream_t st) {
-  using C = Gemm2Cfg<BN2>;
-  static_assert(C::STAGES >= 2, "tile too large for shared memory");
-  static std::atomic<int> attr_done{0};
-  if (!attr_done.load()) {
-    cudaError_t e =
-        cudaFuncSetAttribute(gemm_tc2_kernel<BN2>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    attr_done.store(1);
-  }
-  dim3 grid(2 * ((p.N + BN2 - 1) / BN2), (p.M + 2 * UM - 1) / (2 * UM), 1);
-  gemm_tc2_kernel<BN2><<<grid, GEMM_THREADS, C::SMEM_BYTES, st>>>(p);
-  return cudaGetLastError();
-}
-
-// Per-k-block cost of the two-SM 256 x 256 pair tile in the units of the one-SM table, measured
-// on B200 at M = 512 / 2048 (8B projections): no faster per k-block than the one-SM 256 x 128
-// tile for the same CTA count, so the cost model picks it only where it saves a wave.
-constexpr double PAIR_UNIT = 52.0;
-
-// SOUP_GEMM_2SM=0: never use the two-SM kernel; 1: use it for every eligible GEMM.
-int pair_mode() {
-  static const int mode = [] {
-    const char* e = std::getenv("SOUP_GEMM_2SM");
-    if (!e) return -1;
-    return e[0] == '0' ? 0 : 1;
-  }();
-  return mode;
-}
-
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 bool operand_ok(const Operand& op, int K) {
@@ -1516,26 +1143,8 @@ cudaError_t gemm_launch(const GemmParams& p_in, cudaStream_t st) {
       BN = bn;
     }
   }
-  // Two-SM tiles (256 x 256 per CTA pair) for NF4 GEMMs with raw staging: a tcgen05.mma
-  // carries 4x the work of the one-SM 128 x 128 instruction.  Cost per k-block relative to the
-  // one-SM shapes above: 35 for the pair's 256 x 256 block.
-  bool pair = false;
-  {
-    const GemmSeg& s0 = p.seg[0];
-    const bool nf4 = s0.K > 0 && (s0.B.kind == OP_NF4_K || s0.B.kind == OP_NF4_MN);
-    const int mode = pair_mode();
-    if (nf4 && mode != 0 && p.M >= 2 * UM && p.N >= 256) {
-      GemmParams probe = p;
-      if (setup_raw_tma(probe, 128)) {
-        const long long ctas = 2LL * ((p.N + 255) / 256) * ((p.M + 2 * UM - 1) / (2 * UM));
-        const long long waves = (ctas + 147) / 148;
-        const double cost = static_cast<double>(waves) * (static_cast<double>(nkb) + 2.0) * PAIR_UNIT;
-        pair = (mode == 1) || (mode < 0 && cost < best * 0.999);
-      }
-    }
-  }
-  const int BM = pair ? UM : UM * MT;   // A rows per CTA
-  const int BNB = pair ? 128 : BN;      // B rows per CTA
+  const int BM = UM * MT;  // A rows per CTA
+  const int BNB = BN;      // B rows per CTA
   p.bn = BNB;
   p.raw_tma = setup_raw_tma(p, BNB) ? 1 : 0;
   if (tma_operands_allowed()) {
@@ -1573,12 +1182,6 @@ cudaError_t gemm_launch(const GemmParams& p_in, cudaStream_t st) {
   // kernel (measured: 16-32 partials summed by one CTA per tile cost more than the launch)
   p.fused_reduce = p.splits <= 4 ? 1 : 0;
   cudaError_t e;
-  if (pair) {
-    p.splits = 1;
-    e = launch_pair<256>(p, st);
-    ++g_kernel_launches;
-    return e;
-  }
   if (MT == 2)
     e = (BN == 64) ? launch_tile<2, 64>(p, st) : launch_tile<2, 128>(p, st);
   else

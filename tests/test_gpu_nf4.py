@@ -71,41 +71,3 @@ def test_nf4_matmul_vs_float64(M_, N, K, transpose):
     assert rel_err(got, want) < 4e-3
     assert np.max(np.abs(got - want)) <= 2.0 ** -7 * np.max(np.abs(want)) + 1e-3
 
-
-_PAIR_SCRIPT = r"""
-import sys, numpy as np, torch
-sys.path.insert(0, '.')
-import synth
-from oracle import nf4
-from tests.gpu_util import bf16_tensor, to64, rel_err
-from tests.test_gpu_nf4 import _gpu_quant
-from layer_streamed_nf4_lut_b200 import model as M
-worst = 0.0
-for (M_, N, K, tr) in [(512, 1024, 2048, False), (512, 1024, 2048, True), (300, 768, 1024, False), (256, 2304, 1024, True)]:
-    w = synth.normal(9, N + K, (N, K), 0.02)
-    q = _gpu_quant(w)
-    Wd = nf4.dequant(nf4.quantise(w)).astype(np.float64)
-    kin = N if tr else K
-    x = bf16_tensor(synth.bf16_bits_from_f32(synth.normal(10, M_, (M_, kin), 1.0)))
-    y = M.nf4_matmul(x, q, transpose_w=tr)
-    torch.cuda.synchronize()
-    want = to64(x) @ (Wd if tr else Wd.T)
-    worst = max(worst, rel_err(to64(y), want))
-print("WORST", worst)
-"""
-
-
-@pytest.mark.parametrize("mode", ["1", "0"])
-def test_nf4_matmul_two_sm_and_one_sm_paths(mode):
-    """Both GEMM paths for NF4 weights, forced through the launcher's switch (read once per
-    process, so each runs in a child process), against the float64 reference."""
-    import os
-    import subprocess
-    import sys
-    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-    env = dict(os.environ, SOUP_GEMM_2SM=mode)
-    r = subprocess.run([sys.executable, "-c", _PAIR_SCRIPT], cwd=root, env=env, capture_output=True, text=True,
-                       timeout=300)
-    assert r.returncode == 0, r.stderr[-2000:]
-    worst = float(r.stdout.split("WORST")[-1])
-    assert worst < 4e-3, worst
