@@ -278,7 +278,9 @@ soup_status soup_reset_stats(soup_model* model);
  * CUDA events on the stream it runs on (the H2D layer copies on the streamer's copy stream)
  * and accumulated per category: launches, device milliseconds and the launch's algorithmic
  * work (flops of the dense contraction, bytes of its inputs and outputs).  Adds one event
- * pair per launch; soup_get_profile synchronises the recorded events. */
+ * pair per launch; soup_get_profile synchronises the recorded events.  Every step made while
+ * enabled first times 8 empty launches the same way, reported as category "event_overhead":
+ * the part of each launch's time that is the measurement's own. */
 typedef struct soup_profile_entry {
   char name[32];
   long long launches;
@@ -290,6 +292,30 @@ soup_status soup_set_profiling(soup_model* model, int enabled);
 /* Copies up to max_entries categories (those with launches) into out; *n_entries = count.
  * Clears the accumulated profile when reset != 0. */
 soup_status soup_get_profile(soup_model* model, soup_profile_entry* out, int max_entries, int* n_entries, int reset);
+
+/* Timed categories: brackets every launch of the named profile categories (names soup_get_profile
+ * reports, comma-separated, e.g. "gemm_nf4_fwd,gemm_nf4_dx"; "all" for every category, layer
+ * copies included) with a CUDA
+ * event pair in ordinary model calls, including the CUDA graphs the layer calls replay (the
+ * pair becomes two external event-record nodes of the graph, recorded on the stream the
+ * kernel runs on at every replay).  Unlike soup_set_profiling it changes neither launch order
+ * nor graph use nor stream concurrency, so it times launches as ordinary calls run them; the
+ * event nodes themselves cost some microseconds per pair, measured by one empty launch at the
+ * start of every layer call, bracketed the same way and reported by soup_get_timed_profile as
+ * category "event_overhead" (not counted by soup_get_timed_category).  NULL or "" turns it off; an
+ * unknown name is SOUP_ERR_INVALID_ARG.  Setting it clears the totals; graphs are captured
+ * anew for the new setting (the first two calls of each layer after a change run eagerly /
+ * capture, as at start-up). */
+soup_status soup_set_timed_category(soup_model* model, const char* category);
+/* Totals over the timed launches since the last reset, summed over the timed categories:
+ * launches, device milliseconds (sum of the event pairs), algorithmic flops and bytes.  Waits
+ * for the recorded events.  name holds the setting's first 31 characters ("" when none).
+ * Clears the totals when reset != 0. */
+soup_status soup_get_timed_category(soup_model* model, soup_profile_entry* out, int reset);
+/* The same totals per category, in the layout of soup_get_profile (categories with launches,
+ * up to max_entries; *n_entries = count).  Clears the totals when reset != 0. */
+soup_status soup_get_timed_profile(soup_model* model, soup_profile_entry* out, int max_entries, int* n_entries,
+                                   int reset);
 
 /* Reads (and clears) the device error word; SOUP_ERR_TIMEOUT / SOUP_ERR_DEVICE_CHECK if set. */
 soup_status soup_check_device(soup_model* model, void* stream);

@@ -97,6 +97,9 @@ SIGNATURES = {
     "soup_set_profiling": [c_void_p, c_int],
     "soup_h2d_probe": [c_void_p, c_int, POINTER(ctypes.c_double)],
     "soup_get_profile": [c_void_p, POINTER(ProfileEntry), c_int, POINTER(c_int), c_int],
+    "soup_set_timed_category": [c_void_p, ctypes.c_char_p],
+    "soup_get_timed_category": [c_void_p, POINTER(ProfileEntry), c_int],
+    "soup_get_timed_profile": [c_void_p, POINTER(ProfileEntry), c_int, POINTER(c_int), c_int],
 }
 STRING_FUNCS = {"soup_status_string": [c_int32], "soup_last_error": [c_void_p]}
 

@@ -703,6 +703,30 @@ cudaError_t ce_grad_launch(const float* logits, const float* lse, const int32_t*
   return cudaGetLastError();
 }
 
+// One thread that spins for about `cycles` SM clock cycles (at most 2^22 polls of the clock).
+// The live profile puts one before each timed launch: the GPU is then still busy when the
+// host submits the launch, so the event pair around it times the kernel, not the host's
+// submission gap.
+__global__ void busy_wait_kernel(long long cycles) {
+  const long long t0 = clock64();
+  for (int i = 0; i < (1 << 22); ++i)
+    if (clock64() - t0 >= cycles) break;
+}
+
+cudaError_t busy_wait_launch(long long cycles, cudaStream_t st) {
+  busy_wait_kernel<<<1, 1, 0, st>>>(cycles);
+  return cudaGetLastError();
+}
+
+// An empty launch: what the live profile's event pair measures around a kernel that does no
+// work (its per-launch overhead).
+__global__ void null_kernel() {}
+
+cudaError_t null_launch(cudaStream_t st) {
+  null_kernel<<<1, 32, 0, st>>>();
+  return cudaGetLastError();
+}
+
 cudaError_t f32_to_bf16_launch(const float* x, uint16_t* y, long long n, cudaStream_t st) {
   if (n <= 0) return cudaSuccess;
   f32_to_bf16_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(x, y, n);

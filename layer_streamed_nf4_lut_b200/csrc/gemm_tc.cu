@@ -109,6 +109,15 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       : "r"(taddr)
       : "memory");
 }
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
@@ -487,57 +496,108 @@ __device__ __forceinline__ bool seg_active(const GemmSeg& s, int n0, int bn) {
   return s.B.row_lo < n0 + bn && s.B.row_hi > n0;
 }
 
-// Epilogue store of 8 consecutive columns [col, col+8) of row `row` (value already scaled).
-__device__ __forceinline__ void epilogue_store8(const GemmParams& p, int row, int col, float (&v)[8]) {
+// Epilogue store of NC consecutive columns [col0, col0 + NC) of row `row` (values already
+// scaled; columns at or past N are skipped, N a multiple of 8).  Every load (residual, the
+// old value of an accumulated output) is issued before the first store: a read-modify-write
+// written column by column makes each store wait for its own load, so a warp would wait on
+// memory once per column instead of once per call.
+template <int NC>
+__device__ __forceinline__ void epilogue_store(const GemmParams& p, int row, int col0, float (&v)[NC]) {
+  static_assert(NC % 8 == 0, "columns come in groups of 8");
+  constexpr int G8 = NC / 8;
+  const int nv = p.N - col0;  // columns in range (>= 8)
   if (!p.out_trans) {
     if (p.residual) {
-      const uint4 rv = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.residual) + row * p.ldr + col);
-      const uint32_t rw[4] = {rv.x, rv.y, rv.z, rv.w};
+      const uint16_t* res = static_cast<const uint16_t*>(p.residual) + row * p.ldr + col0;
+      uint4 rv[G8];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float2 f = unpack_bf16x2(rw[j]);
-        v[2 * j] += f.x;
-        v[2 * j + 1] += f.y;
+      for (int g = 0; g < G8; ++g)
+        if (g * 8 < nv) rv[g] = *reinterpret_cast<const uint4*>(res + g * 8);
+#pragma unroll
+      for (int g = 0; g < G8; ++g) {
+        if (g * 8 >= nv) break;
+        const uint32_t rw[4] = {rv[g].x, rv[g].y, rv[g].z, rv[g].w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float2 f = unpack_bf16x2(rw[j]);
+          v[g * 8 + 2 * j] += f.x;
+          v[g * 8 + 2 * j + 1] += f.y;
+        }
       }
     }
     if (p.out_f32) {
-      float4* o = reinterpret_cast<float4*>(static_cast<float*>(p.out) + row * p.ldo + col);
+      float4* o = reinterpret_cast<float4*>(static_cast<float*>(p.out) + row * p.ldo + col0);
       if (p.accumulate) {
-        const float4 a = o[0], b = o[1];
-        v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w;
-        v[4] += b.x; v[5] += b.y; v[6] += b.z; v[7] += b.w;
-      }
-      o[0] = make_float4(v[0], v[1], v[2], v[3]);
-      o[1] = make_float4(v[4], v[5], v[6], v[7]);
-    } else {
-      uint4* o = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + row * p.ldo + col);
-      if (p.accumulate) {
-        const uint4 a = *o;
-        const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
+        float4 a[2 * G8];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const float2 f = unpack_bf16x2(aw[j]);
-          v[2 * j] += f.x;
-          v[2 * j + 1] += f.y;
+        for (int g = 0; g < 2 * G8; ++g)
+          if (g * 4 < nv) a[g] = o[g];
+#pragma unroll
+        for (int g = 0; g < 2 * G8; ++g) {
+          if (g * 4 >= nv) break;
+          v[4 * g] += a[g].x; v[4 * g + 1] += a[g].y; v[4 * g + 2] += a[g].z; v[4 * g + 3] += a[g].w;
         }
       }
-      *o = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
-                      pack_bf16x2(v[6], v[7]));
+#pragma unroll
+      for (int g = 0; g < 2 * G8; ++g)
+        if (g * 4 < nv) o[g] = make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
+    } else {
+      uint4* o = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + row * p.ldo + col0);
+      if (p.accumulate) {
+        uint4 a[G8];
+#pragma unroll
+        for (int g = 0; g < G8; ++g)
+          if (g * 8 < nv) a[g] = o[g];
+#pragma unroll
+        for (int g = 0; g < G8; ++g) {
+          if (g * 8 >= nv) break;
+          const uint32_t aw[4] = {a[g].x, a[g].y, a[g].z, a[g].w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float2 f = unpack_bf16x2(aw[j]);
+            v[g * 8 + 2 * j] += f.x;
+            v[g * 8 + 2 * j + 1] += f.y;
+          }
+        }
+      }
+#pragma unroll
+      for (int g = 0; g < G8; ++g)
+        if (g * 8 < nv)
+          o[g] = make_uint4(pack_bf16x2(v[g * 8], v[g * 8 + 1]), pack_bf16x2(v[g * 8 + 2], v[g * 8 + 3]),
+                            pack_bf16x2(v[g * 8 + 4], v[g * 8 + 5]), pack_bf16x2(v[g * 8 + 6], v[g * 8 + 7]));
     }
   } else {
+    // transposed output: column c of the tile is row c of `out` (a warp's 32 rows are 32
+    // consecutive elements there)
+    if (p.out_f32) {
+      float* o = static_cast<float*>(p.out) + static_cast<long long>(col0) * p.ldo + row;
+      if (p.accumulate) {
+        float a[NC];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const long long idx = static_cast<long long>(col + j) * p.ldo + row;
-      if (p.out_f32) {
-        float* o = static_cast<float*>(p.out) + idx;
-        *o = p.accumulate ? (*o + v[j]) : v[j];
-      } else {
-        uint16_t* o = static_cast<uint16_t*>(p.out) + idx;
-        float w = v[j];
-        if (p.accumulate) w += bf16_to_f32(*o);
-        const __nv_bfloat16 b = __float2bfloat16_rn(w);
-        *o = *reinterpret_cast<const uint16_t*>(&b);
+        for (int j = 0; j < NC; ++j)
+          if (j < nv) a[j] = o[j * p.ldo];
+#pragma unroll
+        for (int j = 0; j < NC; ++j) v[j] += (j < nv) ? a[j] : 0.f;
       }
+#pragma unroll
+      for (int j = 0; j < NC; ++j)
+        if (j < nv) o[j * p.ldo] = v[j];
+    } else {
+      uint16_t* o = static_cast<uint16_t*>(p.out) + static_cast<long long>(col0) * p.ldo + row;
+      if (p.accumulate) {
+        uint16_t a[NC];
+#pragma unroll
+        for (int j = 0; j < NC; ++j)
+          if (j < nv) a[j] = o[j * p.ldo];
+#pragma unroll
+        for (int j = 0; j < NC; ++j) v[j] += (j < nv) ? bf16_to_f32(a[j]) : 0.f;
+      }
+#pragma unroll
+      for (int j = 0; j < NC; ++j)
+        if (j < nv) {
+          const __nv_bfloat16 b = __float2bfloat16_rn(v[j]);
+          o[j * p.ldo] = *reinterpret_cast<const uint16_t*>(&b);
+        }
     }
   }
 }
@@ -756,34 +816,48 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
     }
     if (warp == EPI_WARP0 && lane == 0) {
       // ------------------------------------------------ MMA issuer
-      int g = 0, kb = 0;
+      // One thread; its per-k-block overhead sits between the tensor core's instructions, so
+      // the loop keeps it small: the stage index and phase advance by increments, operand
+      // descriptors by plain adds (the start-address field is the byte address / 16 and
+      // stays inside its 14 bits in shared memory), and the stage's full barrier is probed
+      // with test_wait before the blocking wait.
+      const uint32_t smem0 = smem_u32(base);
+      int g = 0, kb = 0, st = 0;
+      uint32_t ph = 0;
       for (int s = 0; s < p.nseg; ++s) {
         const GemmSeg& sg = p.seg[s];
         if (!seg_active(sg, n0, BN)) continue;
         const int nk = (sg.K + BK - 1) / BK;
+        const int lo = g > kb_lo ? g : kb_lo;
+        const int hi = g + nk < kb_hi ? g + nk : kb_hi;
+        g += nk;
+        if (lo >= hi) continue;
         const bool b_mn = ((s == 0) && p.raw_tma && sg.B.kind == OP_NF4_MN) || p.b_mode[s] == 2;
         const bool a_mn = p.a_mode[s] == 2;
         const uint32_t idesc = idesc_bf16_f32<BN>(a_mn, b_mn);
-        for (int kk = 0; kk < nk; ++kk, ++g) {
-          if (g < kb_lo || g >= kb_hi) continue;
-          const int st = kb % C::STAGES;
-          const uint32_t ph = static_cast<uint32_t>(kb / C::STAGES) & 1u;
-          mbar_wait_bounded(&full[st], ph, abort_flag, p.err);
+        const uint64_t a0 = a_mn ? sw128_mnmajor_desc(smem0) : sw128_kmajor_desc(smem0);
+        const uint64_t b0 = b_mn ? sw128_mnmajor_desc(smem0 + C::A_BYTES) : sw128_kmajor_desc(smem0 + C::A_BYTES);
+        const uint64_t aj = a_mn ? (2048u >> 4) : (32u >> 4);  // one K = 16 step, in 16-byte units
+        const uint64_t bj = b_mn ? (2048u >> 4) : (32u >> 4);
+        for (int it = lo; it < hi; ++it) {
+          if (!mbar_test_wait(&full[st], ph)) mbar_wait_bounded(&full[st], ph, abort_flag, p.err);
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(base + st * C::STAGE_BYTES);
-          const uint32_t b_addr = a_addr + C::A_BYTES;
+          const uint64_t so = static_cast<uint64_t>(st) * (C::STAGE_BYTES >> 4);
 #pragma unroll
           for (int j = 0; j < BK / 16; ++j) {
-            const uint64_t bd = b_mn ? sw128_mnmajor_desc(b_addr + j * 2048) : sw128_kmajor_desc(b_addr + j * 32);
+            const uint64_t bd = b0 + so + j * bj;
 #pragma unroll
             for (int h = 0; h < MT; ++h) {  // the 128-row halves share the B tile (one dequant)
-              const uint32_t ah = a_addr + h * (UM * 128);
-              const uint64_t ad = a_mn ? sw128_mnmajor_desc(ah + j * 2048) : sw128_kmajor_desc(ah + j * 32);
+              const uint64_t ad = a0 + so + h * ((UM * 128) >> 4) + j * aj;
               tc_mma_f16(tmem + h * BN, ad, bd, idesc, (kb > 0 || j > 0) ? 1u : 0u);
             }
           }
           tc_commit(&empty[st]);
           ++kb;
+          if (++st == C::STAGES) {
+            st = 0;
+            ph ^= 1u;
+          }
         }
       }
       tc_commit(done);
@@ -795,29 +869,28 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
     tc_fence_after();
     const bool any_k = kb_hi > kb_lo;
 #pragma unroll 1
-    for (int hc = 0; hc < MT * BN; hc += 32) {
+    for (int hc = 0; hc < MT * BN; hc += 16) {
       const int h = hc / BN, cc = hc % BN;
       const int row = m0 + h * UM + q * 32 + lane;
-      uint32_t r[32];
-      tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(hc), r);
+      uint32_t r[16];
+      tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(hc), r);
       tmem_ld_wait();
-      if (row >= p.M) continue;
+      const int col0 = n0 + cc;
+      if (row >= p.M || col0 >= p.N) continue;
+      if (splits > 1) {
+        float4* o = reinterpret_cast<float4*>(p.workspace + (static_cast<long long>(blockIdx.z) * p.M + row) * p.N + col0);
 #pragma unroll
-      for (int g8 = 0; g8 < 4; ++g8) {
-        const int col = n0 + cc + g8 * 8;
-        if (col >= p.N) break;
-        float v[8];
-        if (splits > 1) {
-#pragma unroll
-          for (int j = 0; j < 8; ++j) v[j] = any_k ? __uint_as_float(r[g8 * 8 + j]) : 0.f;
-          float4* o = reinterpret_cast<float4*>(p.workspace + (static_cast<long long>(blockIdx.z) * p.M + row) * p.N + col);
-          o[0] = make_float4(v[0], v[1], v[2], v[3]);
-          o[1] = make_float4(v[4], v[5], v[6], v[7]);
-        } else {
-#pragma unroll
-          for (int j = 0; j < 8; ++j) v[j] = any_k ? p.alpha * __uint_as_float(r[g8 * 8 + j]) : 0.f;
-          epilogue_store8(p, row, col, v);
+        for (int g = 0; g < 4; ++g) {
+          if (col0 + g * 4 >= p.N) break;
+          o[g] = any_k ? make_float4(__uint_as_float(r[4 * g]), __uint_as_float(r[4 * g + 1]),
+                                     __uint_as_float(r[4 * g + 2]), __uint_as_float(r[4 * g + 3]))
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
         }
+      } else {
+        float v[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) v[j] = any_k ? p.alpha * __uint_as_float(r[j]) : 0.f;
+        epilogue_store<16>(p, row, col0, v);
       }
     }
     if (splits > 1 && p.fused_reduce) {
@@ -841,20 +914,27 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
           const int row = m0 + h * UM + q * 32 + lane;
           if (row >= p.M) continue;
 #pragma unroll 1
-          for (int g8 = 0; g8 < 4; ++g8) {
-            const int col = n0 + cc + g8 * 8;
-            if (col >= p.N) break;
-            float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+          for (int col0 = n0 + cc; col0 < n0 + cc + 32 && col0 < p.N; col0 += 16) {
+            float v[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[j] = 0.f;
+#pragma unroll 1
             for (int sp = 0; sp < splits; ++sp) {
               const float4* src =
-                  reinterpret_cast<const float4*>(p.workspace + (static_cast<long long>(sp) * p.M + row) * p.N + col);
-              const float4 a = __ldcg(src), b = __ldcg(src + 1);
-              v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w;
-              v[4] += b.x; v[5] += b.y; v[6] += b.z; v[7] += b.w;
+                  reinterpret_cast<const float4*>(p.workspace + (static_cast<long long>(sp) * p.M + row) * p.N + col0);
+              float4 a[4];
+#pragma unroll
+              for (int g = 0; g < 4; ++g)
+                if (col0 + g * 4 < p.N) a[g] = __ldcg(src + g);
+#pragma unroll
+              for (int g = 0; g < 4; ++g) {
+                if (col0 + g * 4 >= p.N) break;
+                v[4 * g] += a[g].x; v[4 * g + 1] += a[g].y; v[4 * g + 2] += a[g].z; v[4 * g + 3] += a[g].w;
+              }
             }
 #pragma unroll
-            for (int j = 0; j < 8; ++j) v[j] *= p.alpha;
-            epilogue_store8(p, row, col, v);
+            for (int j = 0; j < 16; ++j) v[j] *= p.alpha;
+            epilogue_store<16>(p, row, col0, v);
           }
         }
       }
@@ -885,7 +965,7 @@ __global__ void splitk_reduce_kernel(const __grid_constant__ GemmParams p) {
   }
 #pragma unroll
   for (int j = 0; j < 8; ++j) v[j] *= p.alpha;
-  epilogue_store8(p, row, col, v);
+  epilogue_store<8>(p, row, col, v);
 }
 
 // ---------------------------------------------------------------- host side
@@ -1104,14 +1184,15 @@ cudaError_t gemm_launch(const GemmParams& p_in, cudaStream_t st) {
   // time proportional to the k-blocks and a per-k-block cost measured on B200 for each tile
   // shape (NF4 GEMMs at M = 512 and 2048): 2x128 50, 1x256 60, 1x128 38, 2x64 47, 1x64 36.
   // GEMMs without an NF4 operand have no decode: a k-block costs about the issuing thread's
-  // MT x 4 tcgen05.mma instructions whatever N is (~100 cycles each), so wider tiles are
-  // nearly free per k-block; the 1x256 tile keeps 3 stages there, hence its small surcharge.
+  // MT x 4 tcgen05.mma instructions (~100 cycles each for N <= 128), so the skinny LoRA GEMMs
+  // (N <= 192) prefer one 128-row tile; the 1x256 tile (N = 256 instructions, 3 stages) ran
+  // the lm_head GEMMs 25 % slower than 2x128, hence its cost.
   bool has_nf4 = false;
   for (int s = 0; s < p.nseg; ++s)
     if (p.seg[s].K > 0 && (p.seg[s].B.kind == OP_NF4_K || p.seg[s].B.kind == OP_NF4_MN)) has_nf4 = true;
   const int cand[5][2] = {{2, 128}, {1, 256}, {1, 128}, {2, 64}, {1, 64}};
   const double unit_nf4[5] = {50.0, 60.0, 38.0, 47.0, 36.0};
-  const double unit_bf16[5] = {64.0, 40.0, 36.0, 64.0, 36.0};
+  const double unit_bf16[5] = {50.0, 60.0, 36.0, 64.0, 36.0};
   const double* unit = has_nf4 ? unit_nf4 : unit_bf16;
   // split-K for grids that leave SMs idle (the skinny LoRA GEMMs; never NF4): up to two waves
   // of CTAs, at least 4 k-blocks per split (a CTA of these runs at the issuing thread's rate,

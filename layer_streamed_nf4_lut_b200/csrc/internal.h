@@ -172,6 +172,8 @@ cudaError_t ce_grad_launch(const float* logits, const float* lse, const int32_t*
 // AdamW on fp32 parameters; also writes their bf16 copy `pb` (may be null).
 cudaError_t adamw_launch(float* p, const float* g, float* m, float* v, uint16_t* pb, long long n, float lr, float b1,
                          float b2, float eps, float wd, int t, cudaStream_t st);
+cudaError_t busy_wait_launch(long long cycles, cudaStream_t st);  // profiling aid, not counted as a launch
+cudaError_t null_launch(cudaStream_t st);                           // profiling aid, not counted as a launch
 cudaError_t f32_to_bf16_launch(const float* x, uint16_t* y, long long n, cudaStream_t st);
 cudaError_t fill_zero_launch(void* p, size_t bytes, cudaStream_t st);
 

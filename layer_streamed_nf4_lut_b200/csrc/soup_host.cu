@@ -265,8 +265,19 @@ struct soup_model {
   std::vector<void*> dev_allocs;
   // per-layer CUDA graphs of the step's layer calls (key: direction, layer, weight buffer,
   // activation buffers, shapes, LoRA flag)
+  // one launch bracketed by CUDA events, and per-category totals of such launches
+  struct ProfRec {
+    int cat;
+    cudaEvent_t a, b;
+    double flops, bytes;
+  };
+  struct ProfCat {
+    long long launches = 0;
+    double ms = 0, flops = 0, bytes = 0;
+  };
   struct GraphKey {
     int dir, layer, B, S, lora, pack;  // pack: shared-prefix length of a packed pair step (0: none)
+    int tcat;                          // mask of the categories whose launches carry event nodes
     const void *base, *in, *out;
     bool operator==(const GraphKey& o) const { return std::memcmp(this, &o, sizeof(GraphKey)) == 0; }
   };
@@ -282,6 +293,8 @@ struct soup_model {
     cudaGraphExec_t exec = nullptr;
     int seen = 0;
     long long launches = 0;
+    std::vector<ProfRec> recs;  // event-record node pairs of the timed category (graph-owned events)
+    int armed = 0;              // replayed since its events were last read
   };
   std::unordered_map<GraphKey, GraphEntry, GraphKeyHash> graphs;
   cudaStream_t cap_stream = nullptr;
@@ -298,18 +311,15 @@ struct soup_model {
   int grads_forked = 0;
   // live profile: event pairs per launch, resolved into per-category totals
   int prof = 0;
-  struct ProfRec {
-    int cat;
-    cudaEvent_t a, b;
-    double flops, bytes;
-  };
   std::vector<ProfRec> prof_pending;
   std::vector<cudaEvent_t> prof_pool;
-  struct ProfCat {
-    long long launches = 0;
-    double ms = 0, flops = 0, bytes = 0;
-  };
   std::vector<ProfCat> prof_cats;
+  // timed categories: event pairs around their launches in ordinary (graph-replayed) calls
+  int tcat = 0;                              // bit c set: category c is timed (0: none)
+  std::string tname;                         // the setting as given
+  std::vector<ProfRec>* cap_recs = nullptr;  // the graph being captured collects its pairs here
+  std::vector<ProfRec> tpending;             // pairs of eager launches and layer copies
+  std::vector<ProfCat> taccs;                // per category
   soup_stats stats{};
   long long launches_at_reset = 0;
 };
@@ -410,12 +420,13 @@ soup_status check_launch(soup_model* m, cudaError_t e, const char* what) {
 // ------------------------------------------------------------------ live profile
 enum ProfCatId : int {
   CAT_H2D = 0, CAT_NF4_FWD, CAT_NF4_DX, CAT_LORA, CAT_LORA_GRAD, CAT_LMHEAD_FWD, CAT_LMHEAD_DX, CAT_ATTN_FWD,
-  CAT_ATTN_BWD, CAT_RMSNORM, CAT_ROPE, CAT_SWIGLU, CAT_CE, CAT_ADAMW, CAT_EMBED, CAT_D2D, CAT_QUANT, CAT_COUNT
+  CAT_ATTN_BWD, CAT_RMSNORM, CAT_ROPE, CAT_SWIGLU, CAT_CE, CAT_ADAMW, CAT_EMBED, CAT_D2D, CAT_QUANT, CAT_NULL,
+  CAT_COUNT
 };
 const char* const kCatNames[CAT_COUNT] = {
     "h2d_layer_copy", "gemm_nf4_fwd", "gemm_nf4_dx", "gemm_lora", "gemm_lora_grad", "gemm_lm_head_fwd",
     "gemm_lm_head_dx", "attention_fwd", "attention_bwd", "rmsnorm", "rope", "swiglu", "cross_entropy", "adamw",
-    "embed", "d2d_copy", "nf4_quantize"};
+    "embed", "d2d_copy", "nf4_quantize", "event_overhead"};
 
 cudaEvent_t prof_event(soup_model* m) {
   if (!m->prof_pool.empty()) {
@@ -461,12 +472,87 @@ void prof_resolve(soup_model* m) {
   }
   m->prof_pending.clear();
 }
+// ~30 us at the B200's 1.965 GHz: longer than the host takes to prepare and submit a launch
+constexpr long long PROF_LEAD_CYCLES = 60000;
+// Timed category: while a model call is captured into a graph the pair becomes two external
+// event-record nodes of that graph (recorded on every replay); otherwise plain records.
+bool timed_begin(soup_model* m, cudaStream_t st, int cat, soup_model::ProfRec* r) {
+  // empty calibration launches are timed whenever any category is
+  const bool want = ((m->tcat >> cat) & 1) != 0 || (cat == CAT_NULL && m->tcat != 0);
+  if (m->prof || !want) return false;
+  r->a = r->b = nullptr;
+  if (cudaEventCreate(&r->a) != cudaSuccess || cudaEventCreate(&r->b) != cudaSuccess) {
+    if (r->a) cudaEventDestroy(r->a);
+    cudaGetLastError();
+    return false;
+  }
+  if ((m->cap_recs ? cudaEventRecordWithFlags(r->a, st, cudaEventRecordExternal) : cudaEventRecord(r->a, st)) !=
+      cudaSuccess) {
+    cudaEventDestroy(r->a);
+    cudaEventDestroy(r->b);
+    cudaGetLastError();
+    return false;
+  }
+  return true;
+}
+void timed_end(soup_model* m, cudaStream_t st, soup_model::ProfRec& r, int cat, double flops, double bytes) {
+  r.cat = cat;
+  r.flops = flops;
+  r.bytes = bytes;
+  if (m->cap_recs)
+    cudaEventRecordWithFlags(r.b, st, cudaEventRecordExternal);
+  else
+    cudaEventRecord(r.b, st);
+  (m->cap_recs ? *m->cap_recs : m->tpending).push_back(r);
+}
+// Adds the recorded durations of `recs` to the timed totals (waits for their end events);
+// destroys the events when `drop`.
+void timed_harvest(soup_model* m, std::vector<soup_model::ProfRec>& recs, bool drop) {
+  if (m->taccs.size() != CAT_COUNT) m->taccs.assign(CAT_COUNT, soup_model::ProfCat{});
+  for (auto& r : recs) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(r.b) == cudaSuccess && cudaEventElapsedTime(&ms, r.a, r.b) == cudaSuccess) {
+      auto& c = m->taccs[r.cat];
+      c.launches += 1;
+      c.ms += ms;
+      c.flops += r.flops;
+      c.bytes += r.bytes;
+    } else {
+      cudaGetLastError();  // not sticky: keep it from surfacing at the next launch check
+    }
+    if (drop) {
+      cudaEventDestroy(r.a);
+      cudaEventDestroy(r.b);
+    }
+  }
+  if (drop) recs.clear();
+}
+void timed_harvest_all(soup_model* m) {
+  for (auto& kv : m->graphs)
+    if (kv.second.armed) {
+      timed_harvest(m, kv.second.recs, false);
+      kv.second.armed = 0;
+    }
+  timed_harvest(m, m->tpending, true);
+}
+
 template <class F>
 soup_status launch(soup_model* m, cudaStream_t st, int cat, double flops, double bytes, const char* what, F&& f) {
+  if (m->prof) busy_wait_launch(PROF_LEAD_CYCLES, st);
   const int idx = prof_begin(m, st);
+  soup_model::ProfRec tr{};
+  const bool timed = timed_begin(m, st, cat, &tr);
   const cudaError_t e = f();
+  if (timed) timed_end(m, st, tr, cat, flops, bytes);
   prof_end(m, st, idx, cat, flops, bytes);
   return check_launch(m, e, what);
+}
+
+// While a category is timed, each layer call starts with one empty launch bracketed like the
+// timed ones (inside the layer's graph): the event pairs' own cost per launch.
+soup_status timed_calibration(soup_model* m, cudaStream_t st) {
+  if (m->tcat == 0 || m->prof) return SOUP_OK;
+  return launch(m, st, CAT_NULL, 0.0, 0.0, "empty launch", [&] { return null_launch(st); });
 }
 
 LayerView view_of(const soup_model* m, const uint8_t* base) {
@@ -594,12 +680,15 @@ soup_status streamer_ensure(soup_model* m, int layer, int protect_lo, int protec
   }
   SOUP_CK(cudaStreamWaitEvent(m->copy_stream, m->buf_free[victim], 0));
   const int pidx = prof_begin(m, m->copy_stream);
+  soup_model::ProfRec tr{};
+  const bool timed = timed_begin(m, m->copy_stream, CAT_H2D, &tr);
   if (m->use_file) {
     SOUP_CK(m->file.stream_layer(layer, m->dev_buf[victim], m->copy_stream));
   } else {
     SOUP_CK(cudaMemcpyAsync(m->dev_buf[victim], m->host_blob[layer], m->layout.total, cudaMemcpyHostToDevice,
                             m->copy_stream));
   }
+  if (timed) timed_end(m, m->copy_stream, tr, CAT_H2D, 0.0, static_cast<double>(m->layout.total));
   prof_end(m, m->copy_stream, pidx, CAT_H2D, 0.0, static_cast<double>(m->layout.total));
   SOUP_CK(cudaEventRecord(m->copy_done[victim], m->copy_stream));
   m->buf_layer[victim] = layer;
@@ -677,6 +766,7 @@ soup_status layer_forward(soup_model* m, int i, const LayerView& L, const uint16
   const bool lora = m->lora_enabled && m->lora_p;
   Saved& A = m->saved[i];
   A.valid = 0;
+  SOUP_TRY(timed_calibration(m, st));
   const double act = 2.0 * T * h;  // bytes of one [T, h] bf16 activation
   SOUP_TRY(launch(m, st, CAT_D2D, 0, 2 * act, "save x", [&] {
     return cudaMemcpyAsync(A.x, x_in, static_cast<size_t>(T) * h * 2, cudaMemcpyDeviceToDevice, st);
@@ -839,6 +929,7 @@ soup_status layer_backward_body(soup_model* m, int i, const LayerView& L, const 
     m->err = "layer_bwd: no matching forward for layer " + std::to_string(i);
     return SOUP_ERR_STATE;
   }
+  SOUP_TRY(timed_calibration(m, st));
   const int T = B * S, h = c.hidden, r = c.lora_r, I = c.intermediate;
   const int qd = c.n_heads * c.head_dim, kvd = c.n_kv_heads * c.head_dim, QKV = m->qkv_cols;
   const float s = m->s_lora;
@@ -1016,6 +1107,7 @@ soup_status run_layer(soup_model* m, int dir, int i, const uint8_t* base, const 
   key.S = S;
   key.lora = lora;
   key.pack = m->pack_pl;
+  key.tcat = m->tcat;
   key.base = base;
   key.in = in;
   key.out = out;
@@ -1026,13 +1118,23 @@ soup_status run_layer(soup_model* m, int dir, int i, const uint8_t* base, const 
   }
   if (!e.exec) {
     const long long l0 = g_kernel_launches.load();
+    timed_harvest(m, e.recs, true);
+    m->cap_recs = &e.recs;
     SOUP_CK(cudaStreamBeginCapture(m->cap_stream, cudaStreamCaptureModeThreadLocal));
     soup_status s = dir == 0 ? layer_forward(m, i, v, in, out, B, S, m->cap_stream)
                              : layer_backward(m, i, v, in, out, B, S, m->cap_stream);
     cudaGraph_t g = nullptr;
     const cudaError_t ce = cudaStreamEndCapture(m->cap_stream, &g);
+    m->cap_recs = nullptr;
     e.launches = g_kernel_launches.load() - l0;
     g_kernel_launches -= e.launches;  // captured, not run
+    if (s != SOUP_OK || ce != cudaSuccess) {
+      for (auto& r : e.recs) {
+        cudaEventDestroy(r.a);
+        cudaEventDestroy(r.b);
+      }
+      e.recs.clear();
+    }
     if (s != SOUP_OK) {
       if (g) cudaGraphDestroy(g);
       return s;
@@ -1049,7 +1151,10 @@ soup_status run_layer(soup_model* m, int dir, int i, const uint8_t* base, const 
       return SOUP_ERR_CUDA;
     }
   }
+  // a graph's event nodes hold its last replay: read them before they are recorded again
+  if (e.armed) timed_harvest(m, e.recs, false);
   SOUP_CK(cudaGraphLaunch(e.exec, st));
+  e.armed = e.recs.empty() ? 0 : 1;
   g_kernel_launches += e.launches;
   if (dir == 0) {
     A.B = B;
@@ -1149,6 +1254,10 @@ soup_status read_scalars(soup_model* m, cudaStream_t st, float* loss_out) {
 
 soup_status do_step_body(soup_model* m, soup_loss kind, const soup_batch* bt, float* loss_out, cudaStream_t st);
 soup_status do_step(soup_model* m, soup_loss kind, const soup_batch* bt, float* loss_out, cudaStream_t st) {
+  if (m->prof) {
+    // the profile's own per-launch overhead: empty launches bracketed like every other one
+    for (int k = 0; k < 8; ++k) SOUP_TRY(launch(m, st, CAT_NULL, 0.0, 0.0, "empty launch", [&] { return null_launch(st); }));
+  }
   const soup_status s = do_step_body(m, kind, bt, loss_out, st);
   m->pack_pl = m->pack_rl = 0;
   return s;
@@ -1303,8 +1412,13 @@ soup_status do_step_body(soup_model* m, soup_loss kind, const soup_batch* bt, fl
 }
 
 void clear_graphs(soup_model* m) {
-  for (auto& kv : m->graphs)
+  for (auto& kv : m->graphs) {
     if (kv.second.exec) cudaGraphExecDestroy(kv.second.exec);
+    for (auto& r : kv.second.recs) {
+      cudaEventDestroy(r.a);
+      cudaEventDestroy(r.b);
+    }
+  }
   m->graphs.clear();
 }
 
@@ -1331,6 +1445,10 @@ soup_status destroy_model(soup_model* m) {
     cudaEventDestroy(r.b);
   }
   for (auto e : m->prof_pool) cudaEventDestroy(e);
+  for (auto& r : m->tpending) {
+    cudaEventDestroy(r.a);
+    cudaEventDestroy(r.b);
+  }
   for (auto e : m->copy_done) cudaEventDestroy(e);
   for (auto e : m->buf_free) cudaEventDestroy(e);
   if (m->copy_stream) cudaStreamDestroy(m->copy_stream);
@@ -1943,6 +2061,80 @@ soup_status soup_get_profile(soup_model* m, soup_profile_entry* out, int max_ent
     }
     *n_entries = std::min(n, std::max(max_entries, 0));
     if (reset) m->prof_cats.assign(CAT_COUNT, soup_model::ProfCat{});
+    return SOUP_OK;
+  })
+}
+
+soup_status soup_set_timed_category(soup_model* m, const char* category) {
+  if (!m) return SOUP_ERR_INVALID_ARG;
+  static_assert(CAT_COUNT <= 31, "category mask");
+  int mask = 0;
+  const std::string spec = category ? category : "";
+  size_t pos = 0;
+  while (pos < spec.size()) {  // comma-separated names, or "all"
+    const size_t end = std::min(spec.find(',', pos), spec.size());
+    const std::string name = spec.substr(pos, end - pos);
+    pos = end + 1;
+    int c = -1;
+    if (name == "all") mask |= ((1 << CAT_COUNT) - 1) & ~(1 << CAT_NULL);
+    for (int k = 0; k < CAT_COUNT; ++k)
+      if (k != CAT_NULL && name == kCatNames[k]) c = k;
+    if (c >= 0) mask |= 1 << c;
+    if (c < 0 && name != "all") {
+      m->err = "unknown kernel category: " + name;
+      return SOUP_ERR_INVALID_ARG;
+    }
+  }
+  SOUP_GUARD({
+    timed_harvest_all(m);
+    m->tcat = mask;
+    m->tname = mask ? spec : std::string();
+    m->taccs.assign(CAT_COUNT, soup_model::ProfCat{});
+    return SOUP_OK;
+  })
+}
+
+soup_status soup_get_timed_category(soup_model* m, soup_profile_entry* out, int reset) {
+  if (!m || !out) return SOUP_ERR_INVALID_ARG;
+  SOUP_GUARD({
+    timed_harvest_all(m);
+    std::memset(out, 0, sizeof(*out));
+    std::strncpy(out->name, m->tname.c_str(), sizeof(out->name) - 1);
+    for (int k = 0; k < static_cast<int>(m->taccs.size()); ++k) {
+      if (k == CAT_NULL) continue;
+      const auto& c = m->taccs[k];
+      out->launches += c.launches;
+      out->total_ms += c.ms;
+      out->flops += c.flops;
+      out->bytes += c.bytes;
+    }
+    if (reset) m->taccs.assign(CAT_COUNT, soup_model::ProfCat{});
+    return SOUP_OK;
+  })
+}
+
+soup_status soup_get_timed_profile(soup_model* m, soup_profile_entry* out, int max_entries, int* n_entries,
+                                   int reset) {
+  if (!m || !n_entries || (max_entries > 0 && !out)) return SOUP_ERR_INVALID_ARG;
+  SOUP_GUARD({
+    timed_harvest_all(m);
+    int n = 0;
+    for (int c = 0; c < CAT_COUNT; ++c) {
+      const auto& pc = m->taccs[c];
+      if (pc.launches == 0) continue;
+      if (n < max_entries) {
+        soup_profile_entry& e = out[n];
+        std::memset(&e, 0, sizeof(e));
+        std::strncpy(e.name, kCatNames[c], sizeof(e.name) - 1);
+        e.launches = pc.launches;
+        e.total_ms = pc.ms;
+        e.flops = pc.flops;
+        e.bytes = pc.bytes;
+      }
+      ++n;
+    }
+    *n_entries = std::min(n, std::max(max_entries, 0));
+    if (reset) m->taccs.assign(CAT_COUNT, soup_model::ProfCat{});
     return SOUP_OK;
   })
 }

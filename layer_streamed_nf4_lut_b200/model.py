@@ -269,6 +269,23 @@ class SoupModel:
         return {arr[i].name.decode(): dict(launches=arr[i].launches, total_ms=arr[i].total_ms, flops=arr[i].flops,
                                            bytes=arr[i].bytes) for i in range(n.value)}
 
+    def set_timed_category(self, name: str | None):
+        """Event pairs around every launch of one profile category ("all": every category) in
+        ordinary (graph-replayed) calls; None turns them off."""
+        self._ck(lib.soup_set_timed_category(self.h, (name or "").encode()))
+
+    def timed_category(self, reset: bool = False) -> dict:
+        e = _lib.ProfileEntry()
+        self._ck(lib.soup_get_timed_category(self.h, byref(e), 1 if reset else 0))
+        return dict(name=e.name.decode(), launches=e.launches, total_ms=e.total_ms, flops=e.flops, bytes=e.bytes)
+
+    def timed_profile(self, reset: bool = False) -> dict:
+        arr = (_lib.ProfileEntry * 64)()
+        n = c_int()
+        self._ck(lib.soup_get_timed_profile(self.h, arr, 64, byref(n), 1 if reset else 0))
+        return {arr[i].name.decode(): dict(launches=arr[i].launches, total_ms=arr[i].total_ms, flops=arr[i].flops,
+                                           bytes=arr[i].bytes) for i in range(n.value)}
+
     def reset_stats(self):
         self._ck(lib.soup_reset_stats(self.h))
 
