@@ -87,6 +87,31 @@ def measured_traffic(kernel):
     return rec["dram_bytes_per_launch"] if h.hexdigest() == rec["kernel_sources_sha256"] else None
 
 
+# one kernel, two launch kinds each: the NF4 GEMM (forward x W^T and dX through the same codes
+# read transposed) and the LoRA GEMMs (u, v on the main stream; dA, dB beside them)
+KERNEL_GROUPS = {"gemm_nf4_fwd,gemm_nf4_dx": ("gemm_nf4_fwd", "gemm_nf4_dx"),
+                 "gemm_lora,gemm_lora_grad": ("gemm_lora", "gemm_lora_grad")}
+
+
+def rank_kernels(prof):
+    """Names the dominant kernel of a live profile (dict category -> launches, total_ms, ...).
+    The pass's own cost per launch (the empty launches of "event_overhead", bracketed like the
+    others) is taken off each category first (net_ms): otherwise categories of many short
+    launches look longer than they run.  Layer copies are not kernels.  Returns (kernel
+    categories, groups, dominant group name, overhead ms per launch); mutates prof."""
+    ov = prof.pop("event_overhead", None)
+    ov_ms = ov["total_ms"] / ov["launches"] if ov and ov["launches"] else 0.0
+    for v in prof.values():
+        v["net_ms"] = max(v["total_ms"] - v["launches"] * ov_ms, 0.0)
+    kern = {k: v for k, v in prof.items() if k != "h2d_layer_copy"}
+    grouped = {k: (k,) for k in kern if not any(k in g for g in KERNEL_GROUPS.values())}
+    grouped.update({name: tuple(c for c in g if c in kern) for name, g in KERNEL_GROUPS.items()})
+    grouped = {k: g for k, g in grouped.items() if g}
+    net = {k: sum(kern[c]["net_ms"] for c in g) for k, g in grouped.items()}
+    dom = max(net, key=net.get) if net else None
+    return kern, grouped, dom, ov_ms
+
+
 def step_flops(cfg, B, S, loss):
     """Algorithmic FLOPs of one step (no recompute counted)."""
     h, I, V, L = cfg["hidden"], cfg["intermediate"], cfg["vocab"], cfg["n_layers"]
@@ -283,22 +308,7 @@ def run_soup(args, wl, rank, world, local_rank):
         one_step(ids, mask)
     prof = gm.profile(reset=True)
     gm.set_profiling(False)
-    # the pass's own cost per launch (empty launches bracketed the same way), taken off each
-    # category before ranking: otherwise categories of many short launches look longer
-    ov = prof.pop("event_overhead", None)
-    ov_ms = ov["total_ms"] / ov["launches"] if ov and ov["launches"] else 0.0
-    for v in prof.values():
-        v["net_ms"] = max(v["total_ms"] - v["launches"] * ov_ms, 0.0)
-    kern = {k: v for k, v in prof.items() if k != "h2d_layer_copy"}
-    # one kernel, two launch kinds each: the NF4 GEMM (forward x W^T and dX through the same
-    # codes read transposed) and the LoRA GEMMs (u, v on the main stream; dA, dB beside them)
-    groups = {"gemm_nf4_fwd,gemm_nf4_dx": ("gemm_nf4_fwd", "gemm_nf4_dx"),
-              "gemm_lora,gemm_lora_grad": ("gemm_lora", "gemm_lora_grad")}
-    grouped = {k: (k,) for k in kern if not any(k in g for g in groups.values())}
-    grouped.update({name: tuple(c for c in g if c in kern) for name, g in groups.items()})
-    grouped = {k: g for k, g in grouped.items() if g}
-    rank = {k: sum(kern[c]["net_ms"] for c in g) for k, g in grouped.items()}
-    dom = max(rank, key=rank.get) if rank else None
+    kern, grouped, dom, ov_ms = rank_kernels(prof)
     timed = {"launches": 0}
     if dom:
         gm.set_timed_category(dom)

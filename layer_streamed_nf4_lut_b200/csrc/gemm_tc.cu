@@ -730,10 +730,15 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
         g += nk;
         continue;
       }
-      for (int kk = 0; kk < nk; ++kk, ++g) {
-        if (g < kb_lo || g >= kb_hi) continue;
-        const int kb = g - kb_lo;
-        if ((kb % GROUPS) != grp) continue;
+      // only this CTA's k-blocks of the segment, and of those only this group's (walking the
+      // whole K and skipping cost ~100 ns per k-block: 20 us on a 224-k-block split GEMM)
+      const int lo = g > kb_lo ? g : kb_lo;
+      const int hi = g + nk < kb_hi ? g + nk : kb_hi;
+      const int first = lo + ((grp - (lo - kb_lo) % GROUPS) + GROUPS) % GROUPS;
+      g += nk;
+      for (int gk = first; gk < hi; gk += GROUPS) {
+        const int kk = gk - (g - nk);
+        const int kb = gk - kb_lo;
         const int st = kb % C::STAGES;
         const uint32_t ph = static_cast<uint32_t>(kb / C::STAGES) & 1u;
         uint8_t* As = base + st * C::STAGE_BYTES;
@@ -757,9 +762,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
         if (!seg_active(sg, n0, BN)) continue;
         const int nk = (sg.K + BK - 1) / BK;
         const bool raw = (s == 0) && p.raw_tma;
-        for (int kk = 0; kk < nk; ++kk, ++g) {
-          if (g < kb_lo || g >= kb_hi) continue;
-          const int kb = g - kb_lo;
+        const int lo = g > kb_lo ? g : kb_lo;
+        const int hi = g + nk < kb_hi ? g + nk : kb_hi;
+        g += nk;
+        for (int gk = lo; gk < hi; ++gk) {
+          const int kk = gk - (g - nk);
+          const int kb = gk - kb_lo;
           const int st = kb % C::STAGES;
           const uint32_t ph = static_cast<uint32_t>(kb / C::STAGES) & 1u;
           mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, p.err);
@@ -893,59 +901,55 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
         epilogue_store<16>(p, row, col0, v);
       }
     }
-    if (splits > 1 && p.fused_reduce) {
-      // the last split of this tile to finish sums every partial in split order (the same
-      // arithmetic, in the same order, as a separate reduction kernel would do)
-      __threadfence();
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      if (q == 0 && lane == 0) {
-        const int tile = blockIdx.y * gridDim.x + blockIdx.x;
-        const int old = atomicAdd(&p.tile_counters[tile], 1);
-        const int last = (old == splits - 1) ? 1 : 0;
-        if (last) p.tile_counters[tile] = 0;  // every split has counted: ready for the next launch
-        *last_flag = last;
-      }
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      if (*last_flag) {
-        __threadfence();
-#pragma unroll 1
-        for (int hc = 0; hc < MT * BN; hc += 32) {
-          const int h = hc / BN, cc = hc % BN;
-          const int row = m0 + h * UM + q * 32 + lane;
-          if (row >= p.M) continue;
-#pragma unroll 1
-          for (int col0 = n0 + cc; col0 < n0 + cc + 32 && col0 < p.N; col0 += 16) {
-            float v[16];
-#pragma unroll
-            for (int j = 0; j < 16; ++j) v[j] = 0.f;
-#pragma unroll 1
-            for (int sp = 0; sp < splits; ++sp) {
-              const float4* src =
-                  reinterpret_cast<const float4*>(p.workspace + (static_cast<long long>(sp) * p.M + row) * p.N + col0);
-              float4 a[4];
-#pragma unroll
-              for (int g = 0; g < 4; ++g)
-                if (col0 + g * 4 < p.N) a[g] = __ldcg(src + g);
-#pragma unroll
-              for (int g = 0; g < 4; ++g) {
-                if (col0 + g * 4 >= p.N) break;
-                v[4 * g] += a[g].x; v[4 * g + 1] += a[g].y; v[4 * g + 2] += a[g].z; v[4 * g + 3] += a[g].w;
-              }
-            }
-#pragma unroll
-            for (int j = 0; j < 16; ++j) v[j] *= p.alpha;
-            epilogue_store<16>(p, row, col0, v);
-          }
-        }
-      }
-    }
   }
 
   tc_fence_before();
+  if (splits > 1 && p.fused_reduce) __threadfence();  // this CTA's partial tile, visible before its ticket
   __syncthreads();
   if (warp == EPI_WARP0) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+  if (splits > 1 && p.fused_reduce) {
+    // The last split of this tile to finish sums every partial in split order (the same
+    // arithmetic, in the same order, as the separate reduction kernel) with all 512 threads:
+    // one (row, 8-column group) per thread at a time, every split's loads issued together.
+    if (threadIdx.x == 0) {
+      const int tile = blockIdx.y * gridDim.x + blockIdx.x;
+      const int old = atomicAdd(&p.tile_counters[tile], 1);
+      const int last = (old == splits - 1) ? 1 : 0;
+      if (last) p.tile_counters[tile] = 0;  // every split has counted: ready for the next launch
+      *last_flag = last;
+    }
+    __syncthreads();
+    if (*last_flag) {
+      __threadfence();
+      constexpr int G8 = BN / 8;
+#pragma unroll 1
+      for (int it = threadIdx.x; it < BM * G8; it += GEMM_THREADS) {
+        const int row = m0 + it / G8, col0 = n0 + (it % G8) * 8;
+        if (row >= p.M || col0 >= p.N) continue;
+        float4 a[4][2];
+#pragma unroll
+        for (int sp = 0; sp < 4; ++sp) {
+          if (sp >= splits) break;
+          const float4* src =
+              reinterpret_cast<const float4*>(p.workspace + (static_cast<long long>(sp) * p.M + row) * p.N + col0);
+          a[sp][0] = __ldcg(src);
+          a[sp][1] = __ldcg(src + 1);
+        }
+        float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int sp = 0; sp < 4; ++sp) {
+          if (sp >= splits) break;
+          v[0] += a[sp][0].x; v[1] += a[sp][0].y; v[2] += a[sp][0].z; v[3] += a[sp][0].w;
+          v[4] += a[sp][1].x; v[5] += a[sp][1].y; v[6] += a[sp][1].z; v[7] += a[sp][1].w;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] *= p.alpha;
+        epilogue_store<8>(p, row, col0, v);
+      }
+    }
   }
 }
 
@@ -957,6 +961,7 @@ __global__ void splitk_reduce_kernel(const __grid_constant__ GemmParams p) {
   if (idx >= static_cast<long long>(p.M) * n8) return;
   const int row = static_cast<int>(idx / n8), col = static_cast<int>(idx % n8) * 8;
   float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
   for (int s = 0; s < p.splits; ++s) {
     const float4* src = reinterpret_cast<const float4*>(p.workspace + (static_cast<long long>(s) * p.M + row) * p.N + col);
     const float4 a = src[0], b = src[1];
@@ -1199,7 +1204,7 @@ cudaError_t gemm_launch(const GemmParams& p_in, cudaStream_t st) {
   // so spreading K shortens the GEMM).  The cost below includes the split and, past 4 partials,
   // the wide reduction kernel (~500 units).
   auto split_for = [&](long long tiles) -> long long {
-    if (!p.workspace || !p.tile_counters || has_nf4 || tiles >= 100 || nkb < 8 || tiles > p.n_counters) return 1;
+    if (!p.workspace || !p.tile_counters || has_nf4 || tiles >= 100 || nkb < 16 || tiles > p.n_counters) return 1;
     long long sp = (2 * 148 + tiles - 1) / tiles;
     sp = std::min<long long>(sp, nkb / 4);
     sp = std::min<long long>(sp, 32);
