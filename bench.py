@@ -71,15 +71,16 @@ def peaks():
     return dict(hbm_gbs=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
 
 
-def measured_traffic(kernel):
+def measured_traffic(kernel, token_rows):
     """DRAM bytes per launch of a kernel category from an ncu capture summarised under
-    profiles/, or None when the kernel's sources changed since the capture."""
+    profiles/, or None when the kernel's sources changed since the capture or the capture's
+    launch shape (token rows) is not the workload's."""
     import hashlib
     path = os.path.join(ROOT, "profiles", "traffic_per_launch.json")
     if not os.path.exists(path):
         return None
     rec = json.load(open(path)).get(kernel)
-    if not rec:
+    if not rec or rec.get("token_rows") != token_rows:
         return None
     h = hashlib.sha256()
     for f in rec["kernel_sources"]:
@@ -387,14 +388,14 @@ def run_soup(args, wl, rank, world, local_rank):
             achieved = d["flops"] / d["launches"] / (per_launch_ms * 1e-3) / 1e12
             roofline = {"bound": "tensor", "kernel": dom, "achieved": round(achieved, 2),
                         "peak": pk["bf16_sustained"], "unit": "TFLOP/s", "frac": round(achieved / pk["bf16_sustained"], 4),
-                        "peak_source": pk["source"] + " bf16 sustained", "traffic": measured_traffic(dom),
+                        "peak_source": pk["source"] + " bf16 sustained", "traffic": measured_traffic(dom, T),
                         "algorithmic_bytes_per_launch": round(d["bytes"] / d["launches"]),
                         "avg_launch_ms": round(per_launch_ms, 4), "launches": d["launches"]}
         else:
             achieved = d["bytes"] / d["launches"] / (per_launch_ms * 1e-3) / 1e9
             roofline = {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1), "peak": pk["hbm_gbs"],
                         "unit": "GB/s", "frac": round(achieved / pk["hbm_gbs"], 4), "peak_source": pk["source"],
-                        "traffic": measured_traffic(dom), "avg_launch_ms": round(per_launch_ms, 4), "launches": d["launches"]}
+                        "traffic": measured_traffic(dom, T), "avg_launch_ms": round(per_launch_ms, 4), "launches": d["launches"]}
         net_ach = (d["flops"] / d["launches"] / (net_launch_ms * 1e-3) / 1e12 if roofline["unit"] == "TFLOP/s" else
                    d["bytes"] / d["launches"] / (net_launch_ms * 1e-3) / 1e9) if net_launch_ms > 0 else None
         roofline["event_overhead_ms"] = round(per_launch_ms - net_launch_ms, 4)
