@@ -259,7 +259,10 @@ soup_status soup_nf4_quantize_static(const float* w, long long n, uint8_t* codes
 soup_status soup_nf4_dequantize(const uint8_t* codes, const int8_t* q8, const float* scales, const float* mean,
                                 long long n, uint16_t* out, void* stream);
 /* y[M, N] (bf16) = x[M, K] (bf16) . W^T + (residual) for one NF4 tensor W [N, K] (device
- * parts as produced by soup_nf4_quantize); transpose_w != 0 computes y[M, K] = x[M, N] . W. */
+ * parts as produced by soup_nf4_quantize); transpose_w != 0 computes y[M, K] = x[M, N] . W.
+ * The first call on a device allocates a 64 MiB workspace and tile counters for the
+ * stream-K schedule, shared by later calls on that device: calls that overlap on the GPU
+ * (different streams) must not be made. */
 soup_status soup_nf4_matmul(const void* x, int M, int N, int K, const uint8_t* codes, const int8_t* q8,
                             const float* scales, const float* mean, int transpose_w, const void* residual, void* y,
                             void* stream);

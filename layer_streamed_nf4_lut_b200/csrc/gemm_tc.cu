@@ -97,18 +97,6 @@ __device__ __forceinline__ void tc_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
                : "memory");
 }
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
-        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
-        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr)
-      : "memory");
-}
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
@@ -619,8 +607,71 @@ __device__ __forceinline__ void load_scales(const GemmParams& p, bool fwd, int n
     dx_scales<BN>(p.nf4, nf4_seg_of(p.nf4, kk * BK), n0, p.N, kk * BK, gtid, r.v);
 }
 
+// ---------------------------------------------------------------- work pieces
+// A CTA's work is a list of pieces: an output tile and a range [kb_lo, kb_hi) of its k-blocks
+// (the active segments' k-blocks concatenated).  Without stream-K: one piece, the tile of
+// (blockIdx.x, blockIdx.y) and split blockIdx.z of `splits`.  With stream-K: the k-blocks of
+// all tiles, flattened tile by tile (M-tiles fastest), are cut into sk_ctas equal ranges, one
+// per CTA; a range holds the tail of one tile, whole tiles, then the head of another.  A tile
+// cut between CTAs is partial: each CTA stores its fp32 share in a workspace slot (slot 2c for
+// CTA c's first piece, 2c + 1 for its last) and the CTA that completes the tile's count sums
+// the shares in k order at its end.
+struct Piece {
+  int m0, n0, kb_lo, kb_hi, tile;
+  int partial;  // the tile's k-blocks are shared with other CTAs (or other splits)
+};
+__device__ __forceinline__ long long sk_bound(const GemmParams& p, int c) {
+  return static_cast<long long>(p.sk_tiles) * p.sk_nkt * c / p.sk_ctas;
+}
+// the CTA whose range holds flattened k-block x
+__device__ __forceinline__ int sk_owner(const GemmParams& p, long long x) {
+  const long long W = static_cast<long long>(p.sk_tiles) * p.sk_nkt;
+  int c = static_cast<int>(x * p.sk_ctas / W);
+  while (c + 1 < p.sk_ctas && sk_bound(p, c + 1) <= x) ++c;
+  while (c > 0 && sk_bound(p, c) > x) --c;
+  return c;
+}
+template <bool SK>
+__device__ __forceinline__ int piece_count(const GemmParams& p) {
+  if (!SK) return 1;
+  const long long lo = sk_bound(p, blockIdx.x), hi = sk_bound(p, blockIdx.x + 1);
+  if (hi <= lo) return 0;
+  return static_cast<int>((hi - 1) / p.sk_nkt - lo / p.sk_nkt + 1);
+}
+template <int BM, int BN, bool SK>
+__device__ __forceinline__ Piece piece_at(const GemmParams& p, int pc) {
+  Piece z;
+  if (!SK) {
+    z.n0 = blockIdx.x * BN;
+    z.m0 = blockIdx.y * BM;
+    z.tile = blockIdx.y * gridDim.x + blockIdx.x;
+    int nkb_all = 0;
+    for (int s = 0; s < p.nseg; ++s)
+      if (seg_active(p.seg[s], z.n0, BN)) nkb_all += (p.seg[s].K + BK - 1) / BK;
+    const int splits = p.splits > 1 ? p.splits : 1;
+    z.kb_lo = static_cast<int>(static_cast<long long>(blockIdx.z) * nkb_all / splits);
+    z.kb_hi = static_cast<int>(static_cast<long long>(blockIdx.z + 1) * nkb_all / splits);
+    z.partial = splits > 1 ? 1 : 0;
+    return z;
+  }
+  const long long lo = sk_bound(p, blockIdx.x), hi = sk_bound(p, blockIdx.x + 1);
+  const int t = static_cast<int>(lo / p.sk_nkt) + pc;
+  const long long t0 = static_cast<long long>(t) * p.sk_nkt;
+  const long long a = lo > t0 ? lo : t0;
+  const long long b = hi < t0 + p.sk_nkt ? hi : t0 + p.sk_nkt;
+  z.tile = t;
+  z.m0 = (t % p.sk_tiles_m) * BM;
+  z.n0 = (t / p.sk_tiles_m) * BN;
+  z.kb_lo = static_cast<int>(a - t0);
+  z.kb_hi = static_cast<int>(b - t0);
+  z.partial = (z.kb_lo == 0 && z.kb_hi == p.sk_nkt) ? 0 : 1;
+  return z;
+}
+
 // ---------------------------------------------------------------- the kernel
-template <int MT, int BN>
+// SK: the stream-K form (p.sk_ctas > 0); the whole-tile / split-K form keeps its own
+// instantiation, with one piece known at compile time.
+template <int MT, int BN, bool SK>
 __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_constant__ GemmParams p) {
   using C = GemmCfg<MT, BN>;
   constexpr int BM = C::BM;
@@ -634,15 +685,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
   volatile int* abort_flag = reinterpret_cast<volatile int*>(ctrl + 68);
   volatile int* last_flag = reinterpret_cast<volatile int*>(ctrl + 72);  // split-K: this CTA reduces
   float* seg_mean = reinterpret_cast<float*>(ctrl + 80);              // up to 3 NF4 tensors
+  volatile int* n_pend = reinterpret_cast<volatile int*>(ctrl + 92);   // stream-K tiles this CTA sums
+  volatile int* pend = reinterpret_cast<volatile int*>(ctrl + 96);     // ... up to 8 of them
   uint64_t* full = reinterpret_cast<uint64_t*>(ctrl + 128);
   uint64_t* empty = full + C::STAGES;
   uint64_t* raw_full = empty + C::STAGES;
   uint64_t* raw_empty = raw_full + C::RAW_SLOTS;
   uint64_t* done = raw_empty + C::RAW_SLOTS;
-  static_assert(128 + 8 * (2 * C::STAGES + 2 * C::RAW_SLOTS + 1) <= C::CTRL_BYTES, "control block overflow");
+  uint64_t* tmem_empty = done + 1;  // the epilogue has read the accumulator out of TMEM
+  static_assert(128 + 8 * (2 * C::STAGES + 2 * C::RAW_SLOTS + 2) <= C::CTRL_BYTES, "control block overflow");
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * BN, m0 = blockIdx.y * BM;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -654,7 +707,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
       mbar_init(&raw_empty[r], GROUP_THREADS / 32);  // the 4 warps of the group that decoded it
     }
     mbar_init(done, 1);
+    mbar_init(tmem_empty, 4);  // one arrival per epilogue warp
     *abort_flag = 0;
+    *n_pend = 0;
     mbar_fence_init();
   }
   if (threadIdx.x < 16) lut[threadIdx.x] = p.lut[threadIdx.x];
@@ -667,239 +722,287 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
-  // this CTA's slice of the k-block list (all active segments concatenated)
-  int nkb_all = 0;
-  for (int s = 0; s < p.nseg; ++s)
-    if (seg_active(p.seg[s], n0, BN)) nkb_all += (p.seg[s].K + BK - 1) / BK;
+  const int n_pieces = piece_count<SK>(p);
   const int splits = p.splits > 1 ? p.splits : 1;
-  const int kb_lo = static_cast<int>(static_cast<long long>(blockIdx.z) * nkb_all / splits);
-  const int kb_hi = static_cast<int>(static_cast<long long>(blockIdx.z + 1) * nkb_all / splits);
-  // Raw-staged k-blocks (segment 0 when raw_tma) come first in the slice: local k-blocks
-  // [0, n_raw) use raw slot kb % RAW_SLOTS.
-  const bool seg0_raw = p.raw_tma && seg_active(p.seg[0], n0, BN);
-  const int seg0_nk = seg0_raw ? (p.seg[0].K + BK - 1) / BK : 0;
-  const int n_raw = seg0_raw ? max(0, min(seg0_nk, kb_hi) - kb_lo) : 0;
 
+  // Every role walks the same pieces in the same order.  Stage and raw-slot indices (and
+  // their phases) run on across pieces: kb_run / raw_run count the k-blocks / raw k-blocks of
+  // this CTA's earlier pieces.  Within a piece, raw-staged k-blocks (segment 0 when raw_tma)
+  // come first: local k-blocks [0, n_raw).
   if (warp < PRODUCER_WARPS) {
     // ------------------------------------------------ producers (groups on alternate k-blocks)
     const int grp = warp >> 2, gtid = threadIdx.x & (GROUP_THREADS - 1);
     const float(&cb)[16] = p.lut;  // kernel-parameter (constant bank) operands, no registers
-    if (n_raw > 0) {
-      // raw-staged NF4 k-blocks of this group: kb = grp, grp + GROUPS, ...  The group scales of
-      // the group's NEXT k-block are loaded while this one decodes, so their L2 latency never
-      // sits between a k-block's raw data arriving and its decode.
-      const bool fwd = p.seg[0].B.kind == OP_NF4_K;
-      ScaleRegs<BN> cur, nxt;
-      if (grp < n_raw) load_scales<BN>(p, fwd, n0, kb_lo + grp, gtid, nxt);
-      for (int kb = grp; kb < n_raw; kb += GROUPS) {
-        const int kk = kb_lo + kb;
-        cur = nxt;
-        if (kb + GROUPS < n_raw) load_scales<BN>(p, fwd, n0, kk + GROUPS, gtid, nxt);
-        const int st = kb % C::STAGES;
-        const uint32_t ph = static_cast<uint32_t>(kb / C::STAGES) & 1u;
-        uint8_t* As = base + st * C::STAGE_BYTES;
-        uint8_t* Bs = As + C::A_BYTES;
-        const int rs = kb % C::RAW_SLOTS;
-        const uint32_t rph = static_cast<uint32_t>(kb / C::RAW_SLOTS) & 1u;
-        const uint8_t* Rc = raw_base + rs * C::RAW_BYTES;
-        const uint8_t* Rq = Rc + C::RAW_CODE_BYTES;
-        mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, p.err);
-        mbar_wait_bounded(&raw_full[rs], rph, abort_flag, p.err);
-        if (fwd) {
-          decode_fwd_raw<BN>(p.nf4, nf4_seg_of(p.nf4, n0), cb, seg_mean, n0, p.N, kk, Rc, Rq, Bs, gtid, cur.v);
-        } else {
-          const int k0 = kk * BK;
-          decode_dx_raw<BN>(p.nf4, nf4_seg_of(p.nf4, k0), cb, seg_mean, n0, p.N, k0, ((n0 >> 6) >> 4) << 4, Rc, Rq,
-                            Bs, gtid, cur.v);
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&raw_empty[rs]);  // this warp's reads of the raw slot are done
-        if (p.a_mode[0] == 0) load_tile<BM>(p.seg[0].A, p.nf4, lut, seg_mean, p.seg[0].K, m0, p.M, kk * BK, As, gtid);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&full[st]);
-      }
-    }
-    int g = 0;
-    for (int s = 0; s < p.nseg; ++s) {
-      const GemmSeg& sg = p.seg[s];
-      if (!seg_active(sg, n0, BN)) continue;
-      const int nk = (sg.K + BK - 1) / BK;
-      if (s == 0 && p.raw_tma) {  // handled above
-        g += nk;
-        continue;
-      }
-      // only this CTA's k-blocks of the segment, and of those only this group's (walking the
-      // whole K and skipping cost ~100 ns per k-block: 20 us on a 224-k-block split GEMM)
-      const int lo = g > kb_lo ? g : kb_lo;
-      const int hi = g + nk < kb_hi ? g + nk : kb_hi;
-      const int first = lo + ((grp - (lo - kb_lo) % GROUPS) + GROUPS) % GROUPS;
-      g += nk;
-      for (int gk = first; gk < hi; gk += GROUPS) {
-        const int kk = gk - (g - nk);
-        const int kb = gk - kb_lo;
-        const int st = kb % C::STAGES;
-        const uint32_t ph = static_cast<uint32_t>(kb / C::STAGES) & 1u;
-        uint8_t* As = base + st * C::STAGE_BYTES;
-        uint8_t* Bs = As + C::A_BYTES;
-        {
+    int kb_run = 0, raw_run = 0;
+    for (int pc = 0; pc < n_pieces; ++pc) {
+      const Piece z = piece_at<BM, BN, SK>(p, pc);
+      const int n0 = z.n0, m0 = z.m0, kb_lo = z.kb_lo, kb_hi = z.kb_hi;
+      const bool seg0_raw = p.raw_tma && seg_active(p.seg[0], n0, BN);
+      const int seg0_nk = seg0_raw ? (p.seg[0].K + BK - 1) / BK : 0;
+      const int n_raw = seg0_raw ? max(0, min(seg0_nk, kb_hi) - kb_lo) : 0;
+      // local k-block kb belongs to group (kb_run + kb) % GROUPS
+      const int kb0 = ((grp - kb_run % GROUPS) + GROUPS) % GROUPS;
+      if (n_raw > 0) {
+        // raw-staged NF4 k-blocks of this group.  The group scales of the group's NEXT k-block
+        // are loaded while this one decodes, so their L2 latency never sits between a
+        // k-block's raw data arriving and its decode.
+        const bool fwd = p.seg[0].B.kind == OP_NF4_K;
+        ScaleRegs<BN> cur, nxt;
+        if (kb0 < n_raw) load_scales<BN>(p, fwd, n0, kb_lo + kb0, gtid, nxt);
+        for (int kb = kb0; kb < n_raw; kb += GROUPS) {
+          const int kk = kb_lo + kb;
+          cur = nxt;
+          if (kb + GROUPS < n_raw) load_scales<BN>(p, fwd, n0, kk + GROUPS, gtid, nxt);
+          const int gb = kb_run + kb, rb = raw_run + kb;
+          const int st = gb % C::STAGES;
+          const uint32_t ph = static_cast<uint32_t>(gb / C::STAGES) & 1u;
+          uint8_t* As = base + st * C::STAGE_BYTES;
+          uint8_t* Bs = As + C::A_BYTES;
+          const int rs = rb % C::RAW_SLOTS;
+          const uint32_t rph = static_cast<uint32_t>(rb / C::RAW_SLOTS) & 1u;
+          const uint8_t* Rc = raw_base + rs * C::RAW_BYTES;
+          const uint8_t* Rq = Rc + C::RAW_CODE_BYTES;
           mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, p.err);
-          if (p.b_mode[s] == 0) load_tile<BN>(sg.B, p.nf4, lut, seg_mean, sg.K, n0, p.N, kk * BK, Bs, gtid);
+          mbar_wait_bounded(&raw_full[rs], rph, abort_flag, p.err);
+          if (fwd) {
+            decode_fwd_raw<BN>(p.nf4, nf4_seg_of(p.nf4, n0), cb, seg_mean, n0, p.N, kk, Rc, Rq, Bs, gtid, cur.v);
+          } else {
+            const int k0 = kk * BK;
+            decode_dx_raw<BN>(p.nf4, nf4_seg_of(p.nf4, k0), cb, seg_mean, n0, p.N, k0, ((n0 >> 6) >> 4) << 4, Rc, Rq,
+                              Bs, gtid, cur.v);
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&raw_empty[rs]);  // this warp's reads of the raw slot are done
+          if (p.a_mode[0] == 0) load_tile<BM>(p.seg[0].A, p.nf4, lut, seg_mean, p.seg[0].K, m0, p.M, kk * BK, As, gtid);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&full[st]);
         }
-        if (p.a_mode[s] == 0) load_tile<BM>(sg.A, p.nf4, lut, seg_mean, sg.K, m0, p.M, kk * BK, As, gtid);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&full[st]);
       }
-    }
-  } else {
-    if (warp == EPI_WARP0 + 1 && lane == 0) {
-      // ------------------------------------------------ TMA issuer: operand tiles (A, bf16 B)
       int g = 0;
       for (int s = 0; s < p.nseg; ++s) {
         const GemmSeg& sg = p.seg[s];
         if (!seg_active(sg, n0, BN)) continue;
         const int nk = (sg.K + BK - 1) / BK;
-        const bool raw = (s == 0) && p.raw_tma;
+        if (s == 0 && p.raw_tma) {  // handled above
+          g += nk;
+          continue;
+        }
+        // only this piece's k-blocks of the segment, and of those only this group's (walking
+        // the whole K and skipping cost ~100 ns per k-block: 20 us on a 224-k-block GEMM)
         const int lo = g > kb_lo ? g : kb_lo;
         const int hi = g + nk < kb_hi ? g + nk : kb_hi;
+        const int first = lo + ((grp - (kb_run + lo - kb_lo) % GROUPS) + GROUPS) % GROUPS;
         g += nk;
-        for (int gk = lo; gk < hi; ++gk) {
+        for (int gk = first; gk < hi; gk += GROUPS) {
           const int kk = gk - (g - nk);
-          const int kb = gk - kb_lo;
-          const int st = kb % C::STAGES;
-          const uint32_t ph = static_cast<uint32_t>(kb / C::STAGES) & 1u;
-          mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, p.err);
+          const int gb = kb_run + (gk - kb_lo);
+          const int st = gb % C::STAGES;
+          const uint32_t ph = static_cast<uint32_t>(gb / C::STAGES) & 1u;
           uint8_t* As = base + st * C::STAGE_BYTES;
           uint8_t* Bs = As + C::A_BYTES;
-          const int am = p.a_mode[s], bm = raw ? 0 : p.b_mode[s];
-          const uint32_t tx = (am ? C::A_BYTES : 0) + (bm ? C::B_BYTES : 0);
-          if (tx) {
-            mbar_arrive_expect_tx(&full[st], tx);
-            const int k0 = kk * BK;
-            if (am == 1) {
-              tma_load_2d(As, &p.tmapA[s], k0, m0, &full[st]);
-            } else if (am == 2) {
+          {
+            mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, p.err);
+            if (p.b_mode[s] == 0) load_tile<BN>(sg.B, p.nf4, lut, seg_mean, sg.K, n0, p.N, kk * BK, Bs, gtid);
+          }
+          if (p.a_mode[s] == 0) load_tile<BM>(sg.A, p.nf4, lut, seg_mean, sg.K, m0, p.M, kk * BK, As, gtid);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&full[st]);
+        }
+      }
+      kb_run += kb_hi > kb_lo ? kb_hi - kb_lo : 0;
+      raw_run += n_raw;
+    }
+  } else {
+    const int q = warp - EPI_WARP0;  // TMEM lane quarter of this epilogue warp
+    int kb_run = 0, raw_run = 0;
+    int mma_st = 0;  // MMA issuer's stage and phase (run on across pieces)
+    uint32_t mma_ph = 0;
+    for (int pc = 0; pc < n_pieces; ++pc) {
+      const Piece z = piece_at<BM, BN, SK>(p, pc);
+      const int n0 = z.n0, m0 = z.m0, kb_lo = z.kb_lo, kb_hi = z.kb_hi;
+      const bool seg0_raw = p.raw_tma && seg_active(p.seg[0], n0, BN);
+      const int seg0_nk = seg0_raw ? (p.seg[0].K + BK - 1) / BK : 0;
+      const int n_raw = seg0_raw ? max(0, min(seg0_nk, kb_hi) - kb_lo) : 0;
+      if (warp == EPI_WARP0 + 1 && lane == 0) {
+        // ---------------------------------------------- TMA issuer: operand tiles (A, bf16 B)
+        int g = 0;
+        for (int s = 0; s < p.nseg; ++s) {
+          const GemmSeg& sg = p.seg[s];
+          if (!seg_active(sg, n0, BN)) continue;
+          const int nk = (sg.K + BK - 1) / BK;
+          const bool raw = (s == 0) && p.raw_tma;
+          const int lo = g > kb_lo ? g : kb_lo;
+          const int hi = g + nk < kb_hi ? g + nk : kb_hi;
+          g += nk;
+          for (int gk = lo; gk < hi; ++gk) {
+            const int kk = gk - (g - nk);
+            const int gb = kb_run + (gk - kb_lo);
+            const int st = gb % C::STAGES;
+            const uint32_t ph = static_cast<uint32_t>(gb / C::STAGES) & 1u;
+            mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, p.err);
+            uint8_t* As = base + st * C::STAGE_BYTES;
+            uint8_t* Bs = As + C::A_BYTES;
+            const int am = p.a_mode[s], bm = raw ? 0 : p.b_mode[s];
+            const uint32_t tx = (am ? C::A_BYTES : 0) + (bm ? C::B_BYTES : 0);
+            if (tx) {
+              mbar_arrive_expect_tx(&full[st], tx);
+              const int k0 = kk * BK;
+              if (am == 1) {
+                tma_load_2d(As, &p.tmapA[s], k0, m0, &full[st]);
+              } else if (am == 2) {
 #pragma unroll
-              for (int i = 0; i < BM / 64; ++i) tma_load_2d(As + i * 8192, &p.tmapA[s], m0 + 64 * i, k0, &full[st]);
-            }
-            if (bm == 1) {
-              tma_load_2d(Bs, &p.tmapB[s], k0, n0 - p.b_row0[s], &full[st]);
-            } else if (bm == 2) {
+                for (int i = 0; i < BM / 64; ++i) tma_load_2d(As + i * 8192, &p.tmapA[s], m0 + 64 * i, k0, &full[st]);
+              }
+              if (bm == 1) {
+                tma_load_2d(Bs, &p.tmapB[s], k0, n0 - p.b_row0[s], &full[st]);
+              } else if (bm == 2) {
 #pragma unroll
-              for (int i = 0; i < BN / 64; ++i) tma_load_2d(Bs + i * 8192, &p.tmapB[s], n0 + 64 * i, k0, &full[st]);
+                for (int i = 0; i < BN / 64; ++i) tma_load_2d(Bs + i * 8192, &p.tmapB[s], n0 + 64 * i, k0, &full[st]);
+              }
+            } else {
+              mbar_arrive(&full[st]);
             }
+          }
+        }
+      }
+      if (warp == EPI_WARP0 + 2 && lane == 0 && n_raw > 0) {
+        // ---------------------------------------------- TMA issuer: raw NF4 codes / absmax
+        const GemmSeg& sg = p.seg[0];
+        for (int kb = 0; kb < n_raw; ++kb) {
+          const int kk = kb_lo + kb;  // k-block index within segment 0
+          const int rb = raw_run + kb;
+          const int rs = rb % C::RAW_SLOTS;
+          const uint32_t rph = static_cast<uint32_t>(rb / C::RAW_SLOTS) & 1u;
+          mbar_wait_bounded(&raw_empty[rs], rph ^ 1u, abort_flag, p.err);
+          uint8_t* Rc = raw_base + rs * C::RAW_BYTES;
+          uint8_t* Rq = Rc + C::RAW_CODE_BYTES;
+          if (sg.B.kind == OP_NF4_K) {
+            const int si = nf4_seg_of(p.nf4, n0);
+            const int y = n0 - p.nf4.seg[si].row_begin;
+            mbar_arrive_expect_tx(&raw_full[rs], BN * 32 + BN * 16);
+            tma_load_2d(Rc, &p.tmapCodes[si], kk * (BK / 2), y, &raw_full[rs]);
+            tma_load_2d(Rq, &p.tmapQ8[si], (kk >> 4) << 4, y, &raw_full[rs]);
           } else {
-            mbar_arrive(&full[st]);
+            const int k0 = kk * BK;
+            const int si = nf4_seg_of(p.nf4, k0);
+            const int y = k0 - p.nf4.seg[si].row_begin;
+            mbar_arrive_expect_tx(&raw_full[rs], 64 * (BN / 2) + 64 * 16);
+            tma_load_2d(Rc, &p.tmapCodes[si], n0 / 2, y, &raw_full[rs]);
+            tma_load_2d(Rq, &p.tmapQ8[si], ((n0 >> 6) >> 4) << 4, y, &raw_full[rs]);
           }
         }
       }
-    }
-    if (warp == EPI_WARP0 + 2 && lane == 0 && n_raw > 0) {
-      // ------------------------------------------------ TMA issuer: raw NF4 codes / absmax
-      const GemmSeg& sg = p.seg[0];
-      for (int kb = 0; kb < n_raw; ++kb) {
-        const int kk = kb_lo + kb;  // k-block index within segment 0
-        const int rs = kb % C::RAW_SLOTS;
-        const uint32_t rph = static_cast<uint32_t>(kb / C::RAW_SLOTS) & 1u;
-        mbar_wait_bounded(&raw_empty[rs], rph ^ 1u, abort_flag, p.err);
-        uint8_t* Rc = raw_base + rs * C::RAW_BYTES;
-        uint8_t* Rq = Rc + C::RAW_CODE_BYTES;
-        if (sg.B.kind == OP_NF4_K) {
-          const int si = nf4_seg_of(p.nf4, n0);
-          const int y = n0 - p.nf4.seg[si].row_begin;
-          mbar_arrive_expect_tx(&raw_full[rs], BN * 32 + BN * 16);
-          tma_load_2d(Rc, &p.tmapCodes[si], kk * (BK / 2), y, &raw_full[rs]);
-          tma_load_2d(Rq, &p.tmapQ8[si], (kk >> 4) << 4, y, &raw_full[rs]);
-        } else {
-          const int k0 = kk * BK;
-          const int si = nf4_seg_of(p.nf4, k0);
-          const int y = k0 - p.nf4.seg[si].row_begin;
-          mbar_arrive_expect_tx(&raw_full[rs], 64 * (BN / 2) + 64 * 16);
-          tma_load_2d(Rc, &p.tmapCodes[si], n0 / 2, y, &raw_full[rs]);
-          tma_load_2d(Rq, &p.tmapQ8[si], ((n0 >> 6) >> 4) << 4, y, &raw_full[rs]);
-        }
-      }
-    }
-    if (warp == EPI_WARP0 && lane == 0) {
-      // ------------------------------------------------ MMA issuer
-      // One thread; its per-k-block overhead sits between the tensor core's instructions, so
-      // the loop keeps it small: the stage index and phase advance by increments, operand
-      // descriptors by plain adds (the start-address field is the byte address / 16 and
-      // stays inside its 14 bits in shared memory), and the stage's full barrier is probed
-      // with test_wait before the blocking wait.
-      const uint32_t smem0 = smem_u32(base);
-      int g = 0, kb = 0, st = 0;
-      uint32_t ph = 0;
-      for (int s = 0; s < p.nseg; ++s) {
-        const GemmSeg& sg = p.seg[s];
-        if (!seg_active(sg, n0, BN)) continue;
-        const int nk = (sg.K + BK - 1) / BK;
-        const int lo = g > kb_lo ? g : kb_lo;
-        const int hi = g + nk < kb_hi ? g + nk : kb_hi;
-        g += nk;
-        if (lo >= hi) continue;
-        const bool b_mn = ((s == 0) && p.raw_tma && sg.B.kind == OP_NF4_MN) || p.b_mode[s] == 2;
-        const bool a_mn = p.a_mode[s] == 2;
-        const uint32_t idesc = idesc_bf16_f32<BN>(a_mn, b_mn);
-        const uint64_t a0 = a_mn ? sw128_mnmajor_desc(smem0) : sw128_kmajor_desc(smem0);
-        const uint64_t b0 = b_mn ? sw128_mnmajor_desc(smem0 + C::A_BYTES) : sw128_kmajor_desc(smem0 + C::A_BYTES);
-        const uint64_t aj = a_mn ? (2048u >> 4) : (32u >> 4);  // one K = 16 step, in 16-byte units
-        const uint64_t bj = b_mn ? (2048u >> 4) : (32u >> 4);
-        for (int it = lo; it < hi; ++it) {
-          if (!mbar_test_wait(&full[st], ph)) mbar_wait_bounded(&full[st], ph, abort_flag, p.err);
-          tc_fence_after();
-          const uint64_t so = static_cast<uint64_t>(st) * (C::STAGE_BYTES >> 4);
+      if (warp == EPI_WARP0 && lane == 0) {
+        // ---------------------------------------------- MMA issuer
+        // One thread; its per-k-block overhead sits between the tensor core's instructions,
+        // so the loop keeps it small: the stage index and phase advance by increments,
+        // operand descriptors by plain adds (the start-address field is the byte address / 16
+        // and stays inside its 14 bits in shared memory), and the stage's full barrier is
+        // probed with test_wait before the blocking wait.  A piece after the first waits until
+        // the epilogue has read the previous piece's accumulator out of TMEM.
+        if (pc > 0) mbar_wait_bounded(tmem_empty, static_cast<uint32_t>(pc - 1) & 1u, abort_flag, p.err);
+        tc_fence_after();
+        const uint32_t smem0 = smem_u32(base);
+        int g = 0, kb = 0;
+        for (int s = 0; s < p.nseg; ++s) {
+          const GemmSeg& sg = p.seg[s];
+          if (!seg_active(sg, n0, BN)) continue;
+          const int nk = (sg.K + BK - 1) / BK;
+          const int lo = g > kb_lo ? g : kb_lo;
+          const int hi = g + nk < kb_hi ? g + nk : kb_hi;
+          g += nk;
+          if (lo >= hi) continue;
+          const bool b_mn = ((s == 0) && p.raw_tma && sg.B.kind == OP_NF4_MN) || p.b_mode[s] == 2;
+          const bool a_mn = p.a_mode[s] == 2;
+          const uint32_t idesc = idesc_bf16_f32<BN>(a_mn, b_mn);
+          const uint64_t a0 = a_mn ? sw128_mnmajor_desc(smem0) : sw128_kmajor_desc(smem0);
+          const uint64_t b0 = b_mn ? sw128_mnmajor_desc(smem0 + C::A_BYTES) : sw128_kmajor_desc(smem0 + C::A_BYTES);
+          const uint64_t aj = a_mn ? (2048u >> 4) : (32u >> 4);  // one K = 16 step, in 16-byte units
+          const uint64_t bj = b_mn ? (2048u >> 4) : (32u >> 4);
+          for (int it = lo; it < hi; ++it) {
+            if (!mbar_test_wait(&full[mma_st], mma_ph)) mbar_wait_bounded(&full[mma_st], mma_ph, abort_flag, p.err);
+            tc_fence_after();
+            const uint64_t so = static_cast<uint64_t>(mma_st) * (C::STAGE_BYTES >> 4);
 #pragma unroll
-          for (int j = 0; j < BK / 16; ++j) {
-            const uint64_t bd = b0 + so + j * bj;
+            for (int j = 0; j < BK / 16; ++j) {
+              const uint64_t bd = b0 + so + j * bj;
 #pragma unroll
-            for (int h = 0; h < MT; ++h) {  // the 128-row halves share the B tile (one dequant)
-              const uint64_t ad = a0 + so + h * ((UM * 128) >> 4) + j * aj;
-              tc_mma_f16(tmem + h * BN, ad, bd, idesc, (kb > 0 || j > 0) ? 1u : 0u);
+              for (int h = 0; h < MT; ++h) {  // the 128-row halves share the B tile (one dequant)
+                const uint64_t ad = a0 + so + h * ((UM * 128) >> 4) + j * aj;
+                tc_mma_f16(tmem + h * BN, ad, bd, idesc, (kb > 0 || j > 0) ? 1u : 0u);
+              }
+            }
+            tc_commit(&empty[mma_st]);
+            ++kb;
+            if (++mma_st == C::STAGES) {
+              mma_st = 0;
+              mma_ph ^= 1u;
             }
           }
-          tc_commit(&empty[st]);
-          ++kb;
-          if (++st == C::STAGES) {
-            st = 0;
-            ph ^= 1u;
+        }
+        tc_commit(done);
+      }
+      __syncwarp();
+      // ---------------------------------------------- epilogue (warps 12..15 = TMEM lane quarters 0..3)
+      mbar_wait_bounded(done, static_cast<uint32_t>(pc) & 1u, abort_flag, p.err);
+      tc_fence_after();
+      const bool any_k = kb_hi > kb_lo;
+      const bool sk_part = SK && z.partial;
+      float* slot = sk_part ? p.workspace + static_cast<long long>(2 * blockIdx.x + (pc == 0 ? 0 : 1)) * (BM * BN)
+                            : nullptr;
+#pragma unroll 1
+      for (int hc = 0; hc < MT * BN; hc += 16) {
+        const int h = hc / BN, cc = hc % BN;
+        const int rl = h * UM + q * 32 + lane;  // row within the tile
+        const int row = m0 + rl;
+        uint32_t r[16];
+        tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(hc), r);
+        tmem_ld_wait();
+        const int col0 = n0 + cc;
+        if (row >= p.M || col0 >= p.N) continue;
+        if (z.partial) {
+          float4* o = sk_part ? reinterpret_cast<float4*>(slot + rl * BN + cc)
+                              : reinterpret_cast<float4*>(p.workspace +
+                                                          (static_cast<long long>(blockIdx.z) * p.M + row) * p.N + col0);
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            if (col0 + g * 4 >= p.N) break;
+            o[g] = any_k ? make_float4(__uint_as_float(r[4 * g]), __uint_as_float(r[4 * g + 1]),
+                                       __uint_as_float(r[4 * g + 2]), __uint_as_float(r[4 * g + 3]))
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+        } else {
+          float v[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) v[j] = any_k ? p.alpha * __uint_as_float(r[j]) : 0.f;
+          epilogue_store<16>(p, row, col0, v);
+        }
+      }
+      // the accumulator is out of TMEM: the next piece's MMAs may overwrite it
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tmem_empty);
+      if (sk_part) {
+        // this CTA's share of the tile is stored: count it; the CTA that completes the count
+        // sums the tile at its end
+        __threadfence();
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (q == 0 && lane == 0) {
+          const long long x0 = static_cast<long long>(z.tile) * p.sk_nkt;
+          const int shares = sk_owner(p, x0 + p.sk_nkt - 1) - sk_owner(p, x0) + 1;
+          const int old = atomicAdd(&p.tile_counters[z.tile], 1);
+          if (old == shares - 1) {
+            p.tile_counters[z.tile] = 0;  // ready for the next launch
+            const int n = *n_pend;
+            if (n < 8) pend[n] = z.tile;
+            *n_pend = n + 1;
           }
         }
       }
-      tc_commit(done);
-    }
-    __syncwarp();
-    // ------------------------------------------------ epilogue (warps 8..11 = TMEM lane quarters 0..3)
-    const int q = warp - EPI_WARP0;
-    mbar_wait_bounded(done, 0u, abort_flag, p.err);
-    tc_fence_after();
-    const bool any_k = kb_hi > kb_lo;
-#pragma unroll 1
-    for (int hc = 0; hc < MT * BN; hc += 16) {
-      const int h = hc / BN, cc = hc % BN;
-      const int row = m0 + h * UM + q * 32 + lane;
-      uint32_t r[16];
-      tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(hc), r);
-      tmem_ld_wait();
-      const int col0 = n0 + cc;
-      if (row >= p.M || col0 >= p.N) continue;
-      if (splits > 1) {
-        float4* o = reinterpret_cast<float4*>(p.workspace + (static_cast<long long>(blockIdx.z) * p.M + row) * p.N + col0);
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          if (col0 + g * 4 >= p.N) break;
-          o[g] = any_k ? make_float4(__uint_as_float(r[4 * g]), __uint_as_float(r[4 * g + 1]),
-                                     __uint_as_float(r[4 * g + 2]), __uint_as_float(r[4 * g + 3]))
-                       : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-      } else {
-        float v[16];
-#pragma unroll
-        for (int j = 0; j < 16; ++j) v[j] = any_k ? p.alpha * __uint_as_float(r[j]) : 0.f;
-        epilogue_store<16>(p, row, col0, v);
-      }
+      kb_run += kb_hi > kb_lo ? kb_hi - kb_lo : 0;
+      raw_run += n_raw;
     }
   }
 
@@ -910,10 +1013,53 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
+  if (SK) {
+    // stream-K: sum the shares of each tile this CTA completed, in k order (CTA order), with
+    // all 512 threads, one (row, 8-column group) per thread at a time
+    const int np = *n_pend < 8 ? *n_pend : 8;
+    if (*n_pend > 8 && threadIdx.x == 0) set_dev_error(p.err, DEVERR_BOUNDS);  // cannot happen: <= 2 per CTA
+    __threadfence();
+    for (int i = 0; i < np; ++i) {
+      const int t = pend[i];
+      const int m0 = (t % p.sk_tiles_m) * BM, n0 = (t / p.sk_tiles_m) * BN;
+      const long long x0 = static_cast<long long>(t) * p.sk_nkt;
+      const int cf = sk_owner(p, x0);
+      const int nsh = min(sk_owner(p, x0 + p.sk_nkt - 1) - cf + 1, 4);  // shares, in k order
+      // the share of CTA cf + k sits in its first-piece slot unless the tile began before its range
+      const float* src0 = p.workspace + static_cast<long long>(2 * cf + (sk_bound(p, cf) >= x0 ? 0 : 1)) * (BM * BN);
+      constexpr int G8 = BN / 8;
+#pragma unroll 1
+      for (int it = threadIdx.x; it < BM * G8; it += GEMM_THREADS) {
+        const int rl = it / G8, cl8 = (it % G8) * 8;
+        const int row = m0 + rl, col0 = n0 + cl8;
+        if (row >= p.M || col0 >= p.N) continue;
+        float4 a[4][2];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          if (k >= nsh) break;
+          const float* sp = k == 0 ? src0 : p.workspace + static_cast<long long>(2 * (cf + k)) * (BM * BN);
+          const float4* src = reinterpret_cast<const float4*>(sp + rl * BN + cl8);
+          a[k][0] = __ldcg(src);
+          a[k][1] = __ldcg(src + 1);
+        }
+        float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          if (k >= nsh) break;
+          v[0] += a[k][0].x; v[1] += a[k][0].y; v[2] += a[k][0].z; v[3] += a[k][0].w;
+          v[4] += a[k][1].x; v[5] += a[k][1].y; v[6] += a[k][1].z; v[7] += a[k][1].w;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] *= p.alpha;
+        epilogue_store<8>(p, row, col0, v);
+      }
+    }
+  }
   if (splits > 1 && p.fused_reduce) {
     // The last split of this tile to finish sums every partial in split order (the same
     // arithmetic, in the same order, as the separate reduction kernel) with all 512 threads:
     // one (row, 8-column group) per thread at a time, every split's loads issued together.
+    const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
     if (threadIdx.x == 0) {
       const int tile = blockIdx.y * gridDim.x + blockIdx.x;
       const int old = atomicAdd(&p.tile_counters[tile], 1);
@@ -1113,19 +1259,20 @@ bool setup_raw_tma(GemmParams& p, int BN) {
   return true;
 }
 
-template <int MT, int BN>
+template <int MT, int BN, bool SK = false>
 cudaError_t launch_tile(const GemmParams& p, cudaStream_t st) {
   using C = GemmCfg<MT, BN>;
   static_assert(C::STAGES >= 2, "tile too large for shared memory");
   static std::atomic<int> attr_done{0};
   if (!attr_done.load()) {
     cudaError_t e =
-        cudaFuncSetAttribute(gemm_tc_kernel<MT, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+        cudaFuncSetAttribute(gemm_tc_kernel<MT, BN, SK>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_done.store(1);
   }
-  dim3 grid((p.N + BN - 1) / BN, (p.M + C::BM - 1) / C::BM, p.splits > 1 ? p.splits : 1);
-  gemm_tc_kernel<MT, BN><<<grid, GEMM_THREADS, C::SMEM_BYTES, st>>>(p);
+  const dim3 grid = p.sk_ctas > 0 ? dim3(p.sk_ctas, 1, 1)
+                                  : dim3((p.N + BN - 1) / BN, (p.M + C::BM - 1) / C::BM, p.splits > 1 ? p.splits : 1);
+  gemm_tc_kernel<MT, BN, SK><<<grid, GEMM_THREADS, C::SMEM_BYTES, st>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || p.splits <= 1 || p.fused_reduce) return e;
   const long long work = static_cast<long long>(p.M) * (p.N / 8);
@@ -1135,6 +1282,27 @@ cudaError_t launch_tile(const GemmParams& p, cudaStream_t st) {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// SMs of the current device (stream-K spreads a GEMM over one CTA per SM)
+int sm_count() {
+  static std::atomic<int> cached[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  int n = cached[dev].load();
+  if (n == 0) {
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    cached[dev].store(n);
+  }
+  return n;
+}
+// SOUP_GEMM_STREAMK=0 keeps every GEMM on whole tiles (for comparisons)
+bool sk_enabled() {
+  static const bool on = [] {
+    const char* e = std::getenv("SOUP_GEMM_STREAMK");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
 
 bool operand_ok(const Operand& op, int K) {
   switch (op.kind) {
@@ -1229,6 +1397,52 @@ cudaError_t gemm_launch(const GemmParams& p_in, cudaStream_t st) {
       BN = bn;
     }
   }
+  // Stream-K for NF4 GEMMs whose whole-tile grid leaves SMs idle (gate|up forward at 512
+  // rows: 448 CTAs = 3.03 waves; its dX: 128 CTAs of 450 k-blocks on 148 SMs): the 256x128
+  // tile (the cheapest per output), every k-block of every tile spread evenly over one CTA per
+  // SM.  Its cost adds ~4 k-blocks per piece (the epilogue between pieces, the pipeline
+  // refill) and ~24 for the partial tiles' shares (stored, then summed by all threads at the
+  // end).  Measured on the 8B projections at 512 rows: gate|up dX 200 -> 155 us, forward
+  // 176 -> 164, down forward 106 -> 97; the short q|k|v and o GEMMs (28-42 k-blocks per CTA)
+  // ran 20-40 % slower, as did every GEMM at 2048 rows, where whole tiles already fill 86-93 %
+  // of the SMs and ran faster per k-block: so at most two 256-row M-tiles.  Only when every
+  // N-tile has the same active segments (the flattened k-block count is then tiles x k-blocks
+  // per tile) and a tile is cut into at most 4 shares.
+  p.sk_ctas = 0;
+  if (has_nf4 && p.workspace && p.tile_counters && sk_enabled() && p.M <= 2 * UM * 2) {
+    const int mt = p.M > UM ? 2 : 1, bn = 128, bm = UM * mt;
+    const int tiles_n = (p.N + bn - 1) / bn, tiles_m = (p.M + bm - 1) / bm;
+    int nkt = -1;
+    bool uniform = true;
+    for (int tn = 0; tn < tiles_n && uniform; ++tn) {
+      int nk = 0;
+      for (int s = 0; s < p.nseg; ++s) {
+        const GemmSeg& sg = p.seg[s];
+        if (sg.K > 0 && sg.B.row_lo < tn * bn + bn && sg.B.row_hi > tn * bn) nk += (sg.K + BK - 1) / BK;
+      }
+      if (nkt < 0) nkt = nk;
+      uniform = nk == nkt;
+    }
+    const int G = sm_count();
+    const long long T = static_cast<long long>(tiles_n) * tiles_m;
+    const long long W = T * (nkt > 0 ? nkt : 0);
+    const long long per = G > 0 ? W / G : 0;
+    const size_t ws_need = static_cast<size_t>(2) * G * bm * bn * sizeof(float);
+    if (uniform && nkt > 0 && per >= 8 && T <= p.n_counters && ws_need <= p.ws_bytes &&
+        nkt <= 3 * per + 1) {  // at most 4 shares per tile
+      const int ci = mt == 2 ? 0 : 2;  // 2x128 or 1x128 in the cost table
+      const long long pieces = (per + nkt - 1) / nkt + 1;
+      const double cost_sk = (static_cast<double>(per) + 2.0 + 4.0 * pieces + 24.0) * unit[ci];
+      if (cost_sk < 0.95 * best) {
+        MT = mt;
+        BN = bn;
+        p.sk_ctas = G;
+        p.sk_tiles = static_cast<int>(T);
+        p.sk_tiles_m = tiles_m;
+        p.sk_nkt = nkt;
+      }
+    }
+  }
   const int BM = UM * MT;  // A rows per CTA
   const int BNB = BN;      // B rows per CTA
   p.bn = BNB;
@@ -1263,12 +1477,14 @@ cudaError_t gemm_launch(const GemmParams& p_in, cudaStream_t st) {
   }
   // NF4 GEMMs keep whole K (the 96-tile q|k|v GEMM ran 105 us split four ways, 65 us whole)
   const long long tiles = static_cast<long long>((p.N + BN - 1) / BN) * ((p.M + BM - 1) / BM);
-  p.splits = p.raw_tma ? 1 : static_cast<int>(split_for(tiles));
+  p.splits = (p.raw_tma || p.sk_ctas > 0) ? 1 : static_cast<int>(split_for(tiles));
   // up to 4 partials the tile's last CTA sums them; more run through the wide reduction
   // kernel (measured: 16-32 partials summed by one CTA per tile cost more than the launch)
   p.fused_reduce = p.splits <= 4 ? 1 : 0;
   cudaError_t e;
-  if (MT == 2)
+  if (p.sk_ctas > 0)
+    e = (MT == 2) ? launch_tile<2, 128, true>(p, st) : launch_tile<1, 128, true>(p, st);
+  else if (MT == 2)
     e = (BN == 64) ? launch_tile<2, 64>(p, st) : launch_tile<2, 128>(p, st);
   else
     e = (BN == 64) ? launch_tile<1, 64>(p, st) : (BN == 128 ? launch_tile<1, 128>(p, st) : launch_tile<1, 256>(p, st));

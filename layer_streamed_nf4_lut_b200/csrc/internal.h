@@ -92,6 +92,13 @@ struct GemmParams {
   int splits;          // set by gemm_launch
   int fused_reduce;    // set by gemm_launch: 1 = the tile's last split sums the partials,
                        // 0 = a second kernel sums them (many splits: the sum runs wide)
+  // stream-K (set by gemm_launch): sk_ctas > 0 spreads the sk_tiles x sk_nkt k-blocks of the
+  // output tiles (M-tiles fastest, sk_tiles_m of them per N-tile) evenly over sk_ctas CTAs;
+  // partial tiles go through the workspace (two slots per CTA) and the tile counters
+  int sk_ctas;
+  int sk_tiles;
+  int sk_tiles_m;
+  int sk_nkt;
 };
 
 // Launch C = sum_seg A_seg B_seg^T on the tcgen05 tensor cores. Returns cudaError_t of launch.

@@ -25,6 +25,7 @@
 #include <string>
 #include <vector>
 #include <algorithm>
+#include <mutex>
 #include <unordered_map>
 
 namespace soup {
@@ -1991,6 +1992,33 @@ soup_status soup_nf4_matmul(const void* x, int M, int N, int K, const uint8_t* c
       p.residual = residual;
       p.ldr = K;
     }
+  }
+  // the stream-K schedule needs a workspace and tile counters: one pair per device, made on
+  // first use and shared by every call on that device
+  static std::mutex ws_mu;
+  static float* ws[64] = {};
+  static int* cnt[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < 64) {
+    std::lock_guard<std::mutex> lk(ws_mu);
+    if (!ws[dev]) {
+      void* a = nullptr;
+      void* b = nullptr;
+      if (cudaMalloc(&a, static_cast<size_t>(64) << 20) == cudaSuccess &&
+          cudaMalloc(&b, GEMM_COUNTERS * sizeof(int)) == cudaSuccess &&
+          cudaMemset(b, 0, GEMM_COUNTERS * sizeof(int)) == cudaSuccess && cudaDeviceSynchronize() == cudaSuccess) {
+        ws[dev] = static_cast<float*>(a);
+        cnt[dev] = static_cast<int*>(b);
+      } else {
+        if (a) cudaFree(a);
+        if (b) cudaFree(b);
+        cudaGetLastError();
+      }
+    }
+    p.workspace = ws[dev];
+    p.ws_bytes = ws[dev] ? static_cast<size_t>(64) << 20 : 0;
+    p.tile_counters = cnt[dev];
+    p.n_counters = cnt[dev] ? GEMM_COUNTERS : 0;
   }
   cudaError_t e = gemm_launch(p, static_cast<cudaStream_t>(stream));
   if (e == cudaErrorInvalidValue) return SOUP_ERR_UNSUPPORTED;

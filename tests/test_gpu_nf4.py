@@ -47,8 +47,12 @@ def test_dequant_bit_exact(shape):
     assert np.array_equal(got, want)
 
 
+# The last two run the stream-K schedule in one orientation each (forward of the first,
+# transposed of the second: k-blocks spread over one CTA per SM, partial tiles summed through
+# the workspace), with ragged M and N tiles
 @pytest.mark.parametrize("M_,N,K", [(64, 1376, 256), (200, 256, 688), (128, 512, 4096), (37, 128, 128),
-                                    (512, 6144, 4096), (300, 768, 1024), (256, 1280, 2048)])
+                                    (512, 6144, 4096), (300, 768, 1024), (256, 1280, 2048), (300, 3208, 8192),
+                                    (300, 12800, 3208)])
 @pytest.mark.parametrize("transpose", [False, True])
 def test_nf4_matmul_vs_float64(M_, N, K, transpose):
     from layer_streamed_nf4_lut_b200 import model as M
