@@ -266,6 +266,30 @@ soup_status soup_nf4_dequantize(const uint8_t* codes, const int8_t* q8, const fl
 soup_status soup_nf4_matmul(const void* x, int M, int N, int K, const uint8_t* codes, const int8_t* q8,
                             const float* scales, const float* mean, int transpose_w, const void* residual, void* y,
                             void* stream);
+/* ---- GEMM scheduling diagnostics (host only: no GPU needed, nothing launched) ----------- */
+/* How the library schedules y[M, N] = x[M, K] . W^T for one operand W: nf4 != 0 for an NF4
+ * weight (transposed != 0: the dX orientation, W read as [K, N]), else bf16; with the
+ * library's own workspace (64 MiB, 16384 tile counters) on a device of `sms` SMs.  mt x bn is
+ * the output tile (mt 128-row halves); splits > 1 splits K over that many CTAs per tile;
+ * stream_k_ctas > 0 spreads stream_k_tiles x stream_k_kblocks k-blocks over that many CTAs
+ * (see soup_gemm_stream_k_piece).  SOUP_ERR_INVALID_ARG for non-positive sizes or N, K not
+ * multiples of 8. */
+typedef struct soup_gemm_plan_info {
+  int mt, bn, splits, fused_reduce;
+  int stream_k_ctas, stream_k_tiles, stream_k_tiles_m, stream_k_kblocks;
+} soup_gemm_plan_info;
+soup_status soup_gemm_plan(int M, int N, int K, int nf4, int transposed, int sms, soup_gemm_plan_info* out);
+/* The stream-K partition: pieces of CTA `cta` (at most max_pieces written; *n_pieces = count):
+ * output tile, k-block range [kb_lo, kb_hi) within it, and the workspace slot a partial piece
+ * stores its share in (-1 when the piece covers its whole tile). */
+soup_status soup_gemm_stream_k_pieces(long long tiles, int kblocks_per_tile, int ctas, int cta, int max_pieces,
+                                      int* tile, int* kb_lo, int* kb_hi, int* slot, int* n_pieces);
+/* The shares of one tile, in k order (at most max_shares written; *n_shares = count): the CTA
+ * that computes each and the workspace slot it is summed from.  A tile computed by one CTA
+ * alone has one share with slot -1. */
+soup_status soup_gemm_stream_k_shares(long long tiles, int kblocks_per_tile, int ctas, int tile, int max_shares,
+                                      int* cta, int* slot, int* n_shares);
+
 /* The 16 NF4 levels this library uses (host fp32[16]). */
 soup_status soup_nf4_codebook(float* out16);
 

@@ -57,6 +57,11 @@ class ProfileEntry(Structure):
                 ("flops", ctypes.c_double), ("bytes", ctypes.c_double)]
 
 
+class GemmPlanInfo(Structure):
+    _fields_ = [("mt", c_int), ("bn", c_int), ("splits", c_int), ("fused_reduce", c_int), ("stream_k_ctas", c_int),
+                ("stream_k_tiles", c_int), ("stream_k_tiles_m", c_int), ("stream_k_kblocks", c_int)]
+
+
 class Batch(Structure):
     _fields_ = [("ids", c_void_p), ("loss_mask", c_void_p), ("B", c_int), ("S", c_int), ("ids_on_host", c_int),
                 ("n_pairs", c_int), ("prefix_len", c_int), ("beta", c_float), ("lr", c_float),
@@ -100,6 +105,11 @@ SIGNATURES = {
     "soup_set_timed_category": [c_void_p, ctypes.c_char_p],
     "soup_get_timed_category": [c_void_p, POINTER(ProfileEntry), c_int],
     "soup_get_timed_profile": [c_void_p, POINTER(ProfileEntry), c_int, POINTER(c_int), c_int],
+    "soup_gemm_plan": [c_int, c_int, c_int, c_int, c_int, c_int, POINTER(GemmPlanInfo)],
+    "soup_gemm_stream_k_pieces": [ctypes.c_longlong, c_int, c_int, c_int, c_int, POINTER(c_int), POINTER(c_int),
+                                  POINTER(c_int), POINTER(c_int), POINTER(c_int)],
+    "soup_gemm_stream_k_shares": [ctypes.c_longlong, c_int, c_int, c_int, c_int, POINTER(c_int), POINTER(c_int),
+                                  POINTER(c_int)],
 }
 STRING_FUNCS = {"soup_status_string": [c_int32], "soup_last_error": [c_void_p]}
 

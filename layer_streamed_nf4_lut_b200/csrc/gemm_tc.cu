@@ -620,23 +620,10 @@ struct Piece {
   int m0, n0, kb_lo, kb_hi, tile;
   int partial;  // the tile's k-blocks are shared with other CTAs (or other splits)
 };
-__device__ __forceinline__ long long sk_bound(const GemmParams& p, int c) {
-  return static_cast<long long>(p.sk_tiles) * p.sk_nkt * c / p.sk_ctas;
-}
-// the CTA whose range holds flattened k-block x
-__device__ __forceinline__ int sk_owner(const GemmParams& p, long long x) {
-  const long long W = static_cast<long long>(p.sk_tiles) * p.sk_nkt;
-  int c = static_cast<int>(x * p.sk_ctas / W);
-  while (c + 1 < p.sk_ctas && sk_bound(p, c + 1) <= x) ++c;
-  while (c > 0 && sk_bound(p, c) > x) --c;
-  return c;
-}
 template <bool SK>
 __device__ __forceinline__ int piece_count(const GemmParams& p) {
   if (!SK) return 1;
-  const long long lo = sk_bound(p, blockIdx.x), hi = sk_bound(p, blockIdx.x + 1);
-  if (hi <= lo) return 0;
-  return static_cast<int>((hi - 1) / p.sk_nkt - lo / p.sk_nkt + 1);
+  return sk_piece_count(p.sk_tiles, p.sk_nkt, p.sk_ctas, blockIdx.x);
 }
 template <int BM, int BN, bool SK>
 __device__ __forceinline__ Piece piece_at(const GemmParams& p, int pc) {
@@ -654,16 +641,9 @@ __device__ __forceinline__ Piece piece_at(const GemmParams& p, int pc) {
     z.partial = splits > 1 ? 1 : 0;
     return z;
   }
-  const long long lo = sk_bound(p, blockIdx.x), hi = sk_bound(p, blockIdx.x + 1);
-  const int t = static_cast<int>(lo / p.sk_nkt) + pc;
-  const long long t0 = static_cast<long long>(t) * p.sk_nkt;
-  const long long a = lo > t0 ? lo : t0;
-  const long long b = hi < t0 + p.sk_nkt ? hi : t0 + p.sk_nkt;
-  z.tile = t;
-  z.m0 = (t % p.sk_tiles_m) * BM;
-  z.n0 = (t / p.sk_tiles_m) * BN;
-  z.kb_lo = static_cast<int>(a - t0);
-  z.kb_hi = static_cast<int>(b - t0);
+  sk_piece(p.sk_tiles, p.sk_nkt, p.sk_ctas, blockIdx.x, pc, &z.tile, &z.kb_lo, &z.kb_hi);
+  z.m0 = (z.tile % p.sk_tiles_m) * BM;
+  z.n0 = (z.tile / p.sk_tiles_m) * BN;
   z.partial = (z.kb_lo == 0 && z.kb_hi == p.sk_nkt) ? 0 : 1;
   return z;
 }
@@ -950,8 +930,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
       tc_fence_after();
       const bool any_k = kb_hi > kb_lo;
       const bool sk_part = SK && z.partial;
-      float* slot = sk_part ? p.workspace + static_cast<long long>(2 * blockIdx.x + (pc == 0 ? 0 : 1)) * (BM * BN)
-                            : nullptr;
+      float* slot = sk_part ? p.workspace + static_cast<long long>(sk_slot(blockIdx.x, pc)) * (BM * BN) : nullptr;
 #pragma unroll 1
       for (int hc = 0; hc < MT * BN; hc += 16) {
         const int h = hc / BN, cc = hc % BN;
@@ -991,7 +970,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
         asm volatile("bar.sync 1, 128;" ::: "memory");
         if (q == 0 && lane == 0) {
           const long long x0 = static_cast<long long>(z.tile) * p.sk_nkt;
-          const int shares = sk_owner(p, x0 + p.sk_nkt - 1) - sk_owner(p, x0) + 1;
+          const int shares = sk_owner(p.sk_tiles, p.sk_nkt, p.sk_ctas, x0 + p.sk_nkt - 1) -
+                             sk_owner(p.sk_tiles, p.sk_nkt, p.sk_ctas, x0) + 1;
           const int old = atomicAdd(&p.tile_counters[z.tile], 1);
           if (old == shares - 1) {
             p.tile_counters[z.tile] = 0;  // ready for the next launch
@@ -1023,10 +1003,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
       const int t = pend[i];
       const int m0 = (t % p.sk_tiles_m) * BM, n0 = (t / p.sk_tiles_m) * BN;
       const long long x0 = static_cast<long long>(t) * p.sk_nkt;
-      const int cf = sk_owner(p, x0);
-      const int nsh = min(sk_owner(p, x0 + p.sk_nkt - 1) - cf + 1, 4);  // shares, in k order
-      // the share of CTA cf + k sits in its first-piece slot unless the tile began before its range
-      const float* src0 = p.workspace + static_cast<long long>(2 * cf + (sk_bound(p, cf) >= x0 ? 0 : 1)) * (BM * BN);
+      const int cf = sk_owner(p.sk_tiles, p.sk_nkt, p.sk_ctas, x0);
+      const int nsh = min(sk_owner(p.sk_tiles, p.sk_nkt, p.sk_ctas, x0 + p.sk_nkt - 1) - cf + 1, 4);  // shares
+      // share 0 sits in CTA cf's last-piece slot when the tile began inside its range, the
+      // others in their CTAs' first-piece slots
+      int c0, sl0;
+      sk_share(p.sk_tiles, p.sk_nkt, p.sk_ctas, t, 0, &c0, &sl0);
+      const float* src0 = p.workspace + static_cast<long long>(sl0) * (BM * BN);
       constexpr int G8 = BN / 8;
 #pragma unroll 1
       for (int it = threadIdx.x; it < BM * G8; it += GEMM_THREADS) {
@@ -1327,32 +1310,12 @@ bool is_mn(int kind) { return kind == OP_BF16_MN || kind == OP_F32_MN || kind ==
 
 }  // namespace
 
-cudaError_t gemm_launch(const GemmParams& p_in, cudaStream_t st) {
-  if (p_in.M <= 0 || p_in.N <= 0) return cudaSuccess;
-  GemmParams p = p_in;
-  if (p.N % 8 != 0 || p.nseg < 1 || p.nseg > GEMM_MAX_SEG) return cudaErrorInvalidValue;
-  if (!aligned16(p.out)) return cudaErrorInvalidValue;
-  if (p.out_trans) {
-    if (p.residual) return cudaErrorInvalidValue;
-  } else {
-    if (p.ldo % 8 != 0) return cudaErrorInvalidValue;
-    if (p.residual && (!aligned16(p.residual) || p.ldr % 8 != 0)) return cudaErrorInvalidValue;
-  }
+GemmPlan gemm_plan(const GemmParams& p, int sms, bool stream_k_allowed) {
+  GemmPlan pl{};
+  if (sms < 1) sms = 148;
   long long nkb = 0;
-  for (int s = 0; s < p.nseg; ++s) {
-    GemmSeg& sg = p.seg[s];
-    p.a_mode[s] = 0;
-    p.b_mode[s] = 0;
-    p.b_row0[s] = 0;
-    if (sg.K < 0) return cudaErrorInvalidValue;
-    if (sg.K == 0) continue;
-    if (!operand_ok(sg.A, sg.K) || !operand_ok(sg.B, sg.K)) return cudaErrorInvalidValue;
-    if (is_mn(sg.A.kind) && p.M % 8 != 0) return cudaErrorInvalidValue;
-    if (sg.A.kind == OP_NF4_K || sg.A.kind == OP_NF4_MN) return cudaErrorInvalidValue;  // NF4 only as B
-    if (sg.B.kind == OP_NF4_K && (p.nf4.cols % 8 != 0 || sg.K > p.nf4.cols)) return cudaErrorInvalidValue;
-    if (sg.B.kind == OP_NF4_MN && (p.nf4.cols % 8 != 0 || p.N > p.nf4.cols)) return cudaErrorInvalidValue;
-    nkb += (sg.K + BK - 1) / BK;
-  }
+  for (int s = 0; s < p.nseg; ++s)
+    if (p.seg[s].K > 0) nkb += (p.seg[s].K + BK - 1) / BK;
   // Tile choice: MT 128-row halves x BN columns.  Time ~ waves x per-tile time, with the per-tile
   // time proportional to the k-blocks and a per-k-block cost measured on B200 for each tile
   // shape (NF4 GEMMs at M = 512 and 2048): 2x128 50, 1x256 60, 1x128 38, 2x64 47, 1x64 36.
@@ -1373,7 +1336,7 @@ cudaError_t gemm_launch(const GemmParams& p_in, cudaStream_t st) {
   // the wide reduction kernel (~500 units).
   auto split_for = [&](long long tiles) -> long long {
     if (!p.workspace || !p.tile_counters || has_nf4 || tiles >= 100 || nkb < 16 || tiles > p.n_counters) return 1;
-    long long sp = (2 * 148 + tiles - 1) / tiles;
+    long long sp = (2 * sms + tiles - 1) / tiles;
     sp = std::min<long long>(sp, nkb / 4);
     sp = std::min<long long>(sp, 32);
     while (sp > 1 && static_cast<unsigned long long>(sp) * p.M * p.N * 4ull > p.ws_bytes) --sp;
@@ -1388,7 +1351,7 @@ cudaError_t gemm_launch(const GemmParams& p_in, cudaStream_t st) {
     if (bn > 128 && p.N <= 128) continue;
     const long long tl = static_cast<long long>((p.N + bn - 1) / bn) * ((p.M + UM * mt - 1) / (UM * mt));
     const long long sp = split_for(tl);
-    const long long waves = (tl * sp + 147) / 148;
+    const long long waves = (tl * sp + sms - 1) / sms;
     const double cost = static_cast<double>(waves) * (static_cast<double>((nkb + sp - 1) / sp) + 2.0) * unit[ci] +
                         (sp > 4 ? 500.0 : 0.0);
     if (cost < best * 0.999) {
@@ -1408,8 +1371,7 @@ cudaError_t gemm_launch(const GemmParams& p_in, cudaStream_t st) {
   // of the SMs and ran faster per k-block: so at most two 256-row M-tiles.  Only when every
   // N-tile has the same active segments (the flattened k-block count is then tiles x k-blocks
   // per tile) and a tile is cut into at most 4 shares.
-  p.sk_ctas = 0;
-  if (has_nf4 && p.workspace && p.tile_counters && sk_enabled() && p.M <= 2 * UM * 2) {
+  if (has_nf4 && p.workspace && p.tile_counters && stream_k_allowed && p.M <= 2 * UM * 2) {
     const int mt = p.M > UM ? 2 : 1, bn = 128, bm = UM * mt;
     const int tiles_n = (p.N + bn - 1) / bn, tiles_m = (p.M + bm - 1) / bm;
     int nkt = -1;
@@ -1423,7 +1385,7 @@ cudaError_t gemm_launch(const GemmParams& p_in, cudaStream_t st) {
       if (nkt < 0) nkt = nk;
       uniform = nk == nkt;
     }
-    const int G = sm_count();
+    const int G = sms;
     const long long T = static_cast<long long>(tiles_n) * tiles_m;
     const long long W = T * (nkt > 0 ? nkt : 0);
     const long long per = G > 0 ? W / G : 0;
@@ -1436,13 +1398,55 @@ cudaError_t gemm_launch(const GemmParams& p_in, cudaStream_t st) {
       if (cost_sk < 0.95 * best) {
         MT = mt;
         BN = bn;
-        p.sk_ctas = G;
-        p.sk_tiles = static_cast<int>(T);
-        p.sk_tiles_m = tiles_m;
-        p.sk_nkt = nkt;
+        pl.sk_ctas = G;
+        pl.sk_tiles = static_cast<int>(T);
+        pl.sk_tiles_m = tiles_m;
+        pl.sk_nkt = nkt;
       }
     }
   }
+  pl.mt = MT;
+  pl.bn = BN;
+  // NF4 GEMMs keep whole K (the 96-tile q|k|v GEMM ran 105 us split four ways, 65 us whole)
+  const int BM = UM * MT;
+  const long long tiles = static_cast<long long>((p.N + BN - 1) / BN) * ((p.M + BM - 1) / BM);
+  pl.splits = (has_nf4 || pl.sk_ctas > 0) ? 1 : static_cast<int>(split_for(tiles));
+  // up to 4 partials the tile's last CTA sums them; more run through the wide reduction
+  // kernel (measured: 16-32 partials summed by one CTA per tile cost more than the launch)
+  pl.fused_reduce = pl.splits <= 4 ? 1 : 0;
+  return pl;
+}
+
+cudaError_t gemm_launch(const GemmParams& p_in, cudaStream_t st) {
+  if (p_in.M <= 0 || p_in.N <= 0) return cudaSuccess;
+  GemmParams p = p_in;
+  if (p.N % 8 != 0 || p.nseg < 1 || p.nseg > GEMM_MAX_SEG) return cudaErrorInvalidValue;
+  if (!aligned16(p.out)) return cudaErrorInvalidValue;
+  if (p.out_trans) {
+    if (p.residual) return cudaErrorInvalidValue;
+  } else {
+    if (p.ldo % 8 != 0) return cudaErrorInvalidValue;
+    if (p.residual && (!aligned16(p.residual) || p.ldr % 8 != 0)) return cudaErrorInvalidValue;
+  }
+  for (int s = 0; s < p.nseg; ++s) {
+    GemmSeg& sg = p.seg[s];
+    p.a_mode[s] = 0;
+    p.b_mode[s] = 0;
+    p.b_row0[s] = 0;
+    if (sg.K < 0) return cudaErrorInvalidValue;
+    if (sg.K == 0) continue;
+    if (!operand_ok(sg.A, sg.K) || !operand_ok(sg.B, sg.K)) return cudaErrorInvalidValue;
+    if (is_mn(sg.A.kind) && p.M % 8 != 0) return cudaErrorInvalidValue;
+    if (sg.A.kind == OP_NF4_K || sg.A.kind == OP_NF4_MN) return cudaErrorInvalidValue;  // NF4 only as B
+    if (sg.B.kind == OP_NF4_K && (p.nf4.cols % 8 != 0 || sg.K > p.nf4.cols)) return cudaErrorInvalidValue;
+    if (sg.B.kind == OP_NF4_MN && (p.nf4.cols % 8 != 0 || p.N > p.nf4.cols)) return cudaErrorInvalidValue;
+  }
+  const GemmPlan pl = gemm_plan(p, sm_count(), sk_enabled());
+  const int MT = pl.mt, BN = pl.bn;
+  p.sk_ctas = pl.sk_ctas;
+  p.sk_tiles = pl.sk_tiles;
+  p.sk_tiles_m = pl.sk_tiles_m;
+  p.sk_nkt = pl.sk_nkt;
   const int BM = UM * MT;  // A rows per CTA
   const int BNB = BN;      // B rows per CTA
   p.bn = BNB;
@@ -1475,12 +1479,8 @@ cudaError_t gemm_launch(const GemmParams& p_in, cudaStream_t st) {
       if (p.seg[s].K > 0 && p.seg[s].A.kind == OP_BF16_K)
         p.a_mode[s] = encode_kmajor_bf16(&p.tmapA[s], p.seg[s].A.ptr, p.seg[s].K, p.M, p.seg[s].A.ld, BM) ? 1 : 0;
   }
-  // NF4 GEMMs keep whole K (the 96-tile q|k|v GEMM ran 105 us split four ways, 65 us whole)
-  const long long tiles = static_cast<long long>((p.N + BN - 1) / BN) * ((p.M + BM - 1) / BM);
-  p.splits = (p.raw_tma || p.sk_ctas > 0) ? 1 : static_cast<int>(split_for(tiles));
-  // up to 4 partials the tile's last CTA sums them; more run through the wide reduction
-  // kernel (measured: 16-32 partials summed by one CTA per tile cost more than the launch)
-  p.fused_reduce = p.splits <= 4 ? 1 : 0;
+  p.splits = pl.splits;
+  p.fused_reduce = pl.fused_reduce;
   cudaError_t e;
   if (p.sk_ctas > 0)
     e = (MT == 2) ? launch_tile<2, 128, true>(p, st) : launch_tile<1, 128, true>(p, st);

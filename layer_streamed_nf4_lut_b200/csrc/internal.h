@@ -104,6 +104,52 @@ struct GemmParams {
 // Launch C = sum_seg A_seg B_seg^T on the tcgen05 tensor cores. Returns cudaError_t of launch.
 cudaError_t gemm_launch(const GemmParams& p, cudaStream_t st);
 
+// How gemm_launch schedules a GEMM (host only, no CUDA calls): tile (mt 128-row halves x bn
+// columns), split-K count, or the stream-K partition over `sms` CTAs.
+struct GemmPlan {
+  int mt, bn, splits, fused_reduce;
+  int sk_ctas, sk_tiles, sk_tiles_m, sk_nkt;
+};
+GemmPlan gemm_plan(const GemmParams& p, int sms, bool stream_k_allowed);
+
+// ---- stream-K partition (host and device).  The k-blocks of `tiles` output tiles, nkt per
+// tile, flattened tile by tile, are cut into `ctas` ranges: CTA c owns [bound(c), bound(c+1)).
+__host__ __device__ inline long long sk_bound(long long tiles, int nkt, int ctas, int c) {
+  return tiles * nkt * c / ctas;
+}
+// the CTA whose range holds flattened k-block x
+__host__ __device__ inline int sk_owner(long long tiles, int nkt, int ctas, long long x) {
+  const long long W = tiles * nkt;
+  int c = static_cast<int>(x * ctas / W);
+  while (c + 1 < ctas && sk_bound(tiles, nkt, ctas, c + 1) <= x) ++c;
+  while (c > 0 && sk_bound(tiles, nkt, ctas, c) > x) --c;
+  return c;
+}
+// pieces of CTA c: its range cut at tile boundaries (piece pc lies in tile first_tile + pc)
+__host__ __device__ inline int sk_piece_count(long long tiles, int nkt, int ctas, int c) {
+  const long long lo = sk_bound(tiles, nkt, ctas, c), hi = sk_bound(tiles, nkt, ctas, c + 1);
+  return hi <= lo ? 0 : static_cast<int>((hi - 1) / nkt - lo / nkt + 1);
+}
+__host__ __device__ inline void sk_piece(long long tiles, int nkt, int ctas, int c, int pc, int* tile, int* kb_lo,
+                                         int* kb_hi) {
+  const long long lo = sk_bound(tiles, nkt, ctas, c), hi = sk_bound(tiles, nkt, ctas, c + 1);
+  const long long t = lo / nkt + pc, t0 = t * nkt;
+  *tile = static_cast<int>(t);
+  *kb_lo = static_cast<int>((lo > t0 ? lo : t0) - t0);
+  *kb_hi = static_cast<int>((hi < t0 + nkt ? hi : t0 + nkt) - t0);
+}
+// workspace slot of a partial piece: 2c for CTA c's first piece, 2c + 1 for its last (a
+// partial tile is only ever cut at the two ends of a range)
+__host__ __device__ inline int sk_slot(int c, int pc) { return 2 * c + (pc == 0 ? 0 : 1); }
+// share k (in k order) of a tile cut between CTAs: its CTA and slot; the count is
+// sk_owner(last k-block) - sk_owner(first) + 1
+__host__ __device__ inline void sk_share(long long tiles, int nkt, int ctas, int tile, int k, int* cta, int* slot) {
+  const long long x0 = static_cast<long long>(tile) * nkt;
+  const int c = sk_owner(tiles, nkt, ctas, x0) + k;
+  *cta = c;
+  *slot = 2 * c + ((k == 0 && sk_bound(tiles, nkt, ctas, c) < x0) ? 1 : 0);
+}
+
 // ----------------------------------------------------------------- NF4 quantiser / dequant
 struct LUT16 {
   float v[16];

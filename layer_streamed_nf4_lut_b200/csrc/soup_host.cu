@@ -2032,6 +2032,65 @@ const soup::LUT16& soup_codebook_lut() { return soup::codebook(); }
 
 extern "C" {
 
+soup_status soup_gemm_plan(int M, int N, int K, int nf4, int transposed, int sms, soup_gemm_plan_info* out) {
+  if (!out || M <= 0 || N <= 0 || K <= 0 || N % 8 || K % 8 || sms < 1) return SOUP_ERR_INVALID_ARG;
+  GemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.M = M;
+  p.N = N;
+  p.nseg = 1;
+  p.seg[0].K = K;
+  p.seg[0].A = Operand{OP_BF16_K, nullptr, K, 1.f, 0, INT_MAX};
+  p.seg[0].B = Operand{nf4 ? (transposed ? OP_NF4_MN : OP_NF4_K) : OP_BF16_K, nullptr, K, 1.f, 0, INT_MAX};
+  // the workspace the model and soup_nf4_matmul hand to their GEMMs (only its presence and
+  // size count here)
+  static float ws_tag;
+  static int cnt_tag;
+  p.workspace = &ws_tag;
+  p.ws_bytes = static_cast<size_t>(64) << 20;
+  p.tile_counters = &cnt_tag;
+  p.n_counters = GEMM_COUNTERS;
+  const GemmPlan pl = gemm_plan(p, sms, true);
+  out->mt = pl.mt;
+  out->bn = pl.bn;
+  out->splits = pl.splits;
+  out->fused_reduce = pl.fused_reduce;
+  out->stream_k_ctas = pl.sk_ctas;
+  out->stream_k_tiles = pl.sk_tiles;
+  out->stream_k_tiles_m = pl.sk_tiles_m;
+  out->stream_k_kblocks = pl.sk_nkt;
+  return SOUP_OK;
+}
+
+soup_status soup_gemm_stream_k_pieces(long long tiles, int nkt, int ctas, int cta, int max_pieces, int* tile,
+                                      int* kb_lo, int* kb_hi, int* slot, int* n_pieces) {
+  if (tiles < 1 || nkt < 1 || ctas < 1 || cta < 0 || cta >= ctas || max_pieces < 0 || !n_pieces ||
+      (max_pieces > 0 && (!tile || !kb_lo || !kb_hi || !slot)))
+    return SOUP_ERR_INVALID_ARG;
+  const int n = sk_piece_count(tiles, nkt, ctas, cta);
+  for (int pc = 0; pc < n && pc < max_pieces; ++pc) {
+    sk_piece(tiles, nkt, ctas, cta, pc, &tile[pc], &kb_lo[pc], &kb_hi[pc]);
+    slot[pc] = (kb_lo[pc] == 0 && kb_hi[pc] == nkt) ? -1 : sk_slot(cta, pc);
+  }
+  *n_pieces = n;
+  return SOUP_OK;
+}
+
+soup_status soup_gemm_stream_k_shares(long long tiles, int nkt, int ctas, int tile, int max_shares, int* cta,
+                                      int* slot, int* n_shares) {
+  if (tiles < 1 || nkt < 1 || ctas < 1 || tile < 0 || tile >= tiles || max_shares < 0 || !n_shares ||
+      (max_shares > 0 && (!cta || !slot)))
+    return SOUP_ERR_INVALID_ARG;
+  const long long x0 = static_cast<long long>(tile) * nkt;
+  const int n = sk_owner(tiles, nkt, ctas, x0 + nkt - 1) - sk_owner(tiles, nkt, ctas, x0) + 1;
+  for (int k = 0; k < n && k < max_shares; ++k) {
+    sk_share(tiles, nkt, ctas, tile, k, &cta[k], &slot[k]);
+    if (n == 1) slot[k] = -1;
+  }
+  *n_shares = n;
+  return SOUP_OK;
+}
+
 soup_status soup_nf4_codebook(float* out16) {
   if (!out16) return SOUP_ERR_INVALID_ARG;
   std::memcpy(out16, codebook().v, 16 * sizeof(float));

@@ -320,6 +320,30 @@ def nf4_dequantize(q: dict) -> torch.Tensor:
     return out.view(q["shape"])
 
 
+def gemm_plan(M: int, N: int, K: int, nf4: bool = True, transposed: bool = False, sms: int = 148) -> dict:
+    """How the library schedules y[M, N] = x[M, K] W^T (host only; see soup_gemm_plan)."""
+    info = _lib.GemmPlanInfo()
+    check(lib.soup_gemm_plan(M, N, K, 1 if nf4 else 0, 1 if transposed else 0, sms, byref(info)))
+    return {f: getattr(info, f) for f, _ in _lib.GemmPlanInfo._fields_}
+
+
+def stream_k_pieces(tiles: int, kblocks_per_tile: int, ctas: int, cta: int) -> list:
+    """(tile, kb_lo, kb_hi, slot) of each piece of one stream-K CTA (slot -1: whole tile)."""
+    cap = 64
+    arrs = [(c_int * cap)() for _ in range(4)]
+    n = c_int()
+    check(lib.soup_gemm_stream_k_pieces(tiles, kblocks_per_tile, ctas, cta, cap, *arrs, byref(n)))
+    return [tuple(a[i] for a in arrs) for i in range(min(n.value, cap))]
+
+
+def stream_k_shares(tiles: int, kblocks_per_tile: int, ctas: int, tile: int) -> list:
+    """(cta, slot) of each share of one stream-K tile, in k order (slot -1: one CTA alone)."""
+    cap = 64
+    cta, slot, n = (c_int * cap)(), (c_int * cap)(), c_int()
+    check(lib.soup_gemm_stream_k_shares(tiles, kblocks_per_tile, ctas, tile, cap, cta, slot, byref(n)))
+    return [(cta[i], slot[i]) for i in range(min(n.value, cap))]
+
+
 def nf4_matmul(x: torch.Tensor, q: dict, transpose_w: bool = False, residual: torch.Tensor | None = None):
     """y = x W^T (W = NF4 tensor [N, K]) or y = x W when transpose_w; bf16 in/out."""
     N, K = q["shape"]
