@@ -310,17 +310,6 @@ __device__ __forceinline__ void load_tile(const Operand& op, const NF4Group& g, 
   }
 }
 
-// Decode the 8 codes of one 32-bit word with the block's reconstructed absmax `mh`:
-// bf16_rn(codebook[q] * mh), element 2i in the low nibble of byte i.
-__device__ __forceinline__ uint4 decode_word(uint32_t c, float mh, const float* lut) {
-  uint4 o;
-  o.x = pack_bf16x2(__fmul_rn(lut[c & 15u], mh), __fmul_rn(lut[(c >> 4) & 15u], mh));
-  o.y = pack_bf16x2(__fmul_rn(lut[(c >> 8) & 15u], mh), __fmul_rn(lut[(c >> 12) & 15u], mh));
-  o.z = pack_bf16x2(__fmul_rn(lut[(c >> 16) & 15u], mh), __fmul_rn(lut[(c >> 20) & 15u], mh));
-  o.w = pack_bf16x2(__fmul_rn(lut[(c >> 24) & 15u], mh), __fmul_rn(lut[c >> 28], mh));
-  return o;
-}
-
 // Explicit shared-space accesses for the decode path (32-bit shared addresses).
 __device__ __forceinline__ uint4 lds128(uint32_t a) {
   uint4 v;
