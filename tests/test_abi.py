@@ -128,7 +128,8 @@ def test_struct_layouts_match_the_c_compiler(tmp_path):
     if shutil.which("gcc") is None:
         pytest.skip("no C compiler")
     structs = {"soup_model_config": _lib.ModelConfig, "soup_allocator": _lib.Allocator, "soup_stats": _lib.Stats,
-               "soup_profile_entry": _lib.ProfileEntry, "soup_batch": _lib.Batch}
+               "soup_profile_entry": _lib.ProfileEntry, "soup_batch": _lib.Batch,
+               "soup_gemm_plan_info": _lib.GemmPlanInfo}
     lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "soup.h"', "int main(void) {"]
     for cname, cls in structs.items():
         lines.append(f'  printf("{cname} sizeof %zu\\n", sizeof({cname}));')
