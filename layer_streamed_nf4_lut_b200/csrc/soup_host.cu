@@ -14,6 +14,8 @@
 #include "internal.h"
 #include "layer_file.h"
 
+#include <nvtx3/nvToolsExt.h>
+
 #include <unistd.h>
 
 #include <chrono>
@@ -418,6 +420,21 @@ soup_status check_launch(soup_model* m, cudaError_t e, const char* what) {
   return e == cudaErrorInvalidValue ? SOUP_ERR_UNSUPPORTED : SOUP_ERR_CUDA;
 }
 
+// ------------------------------------------------------------------ tracing
+// NVTX ranges on the host thread around each layer call, layer copy, head pass and step, for a
+// timeline tool (no cost when none is attached).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  NvtxRange(const char* what, int i) {
+    char b[48];
+    std::snprintf(b, sizeof(b), "%s %d", what, i);
+    nvtxRangePushA(b);
+  }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+
 // ------------------------------------------------------------------ live profile
 enum ProfCatId : int {
   CAT_H2D = 0, CAT_NF4_FWD, CAT_NF4_DX, CAT_LORA, CAT_LORA_GRAD, CAT_LMHEAD_FWD, CAT_LMHEAD_DX, CAT_ATTN_FWD,
@@ -657,6 +674,7 @@ soup_status run_gemm(soup_model* m, const GemmParams& p, cudaStream_t st, const 
 // ------------------------------------------------------------------ streamer
 soup_status streamer_ensure(soup_model* m, int layer, int protect_lo, int protect_hi) {
   if (m->cfg.mode == SOUP_RESIDENT) return SOUP_OK;
+  const NvtxRange trace("layer copy", layer);
   const int nb = static_cast<int>(m->dev_buf.size());
   for (int b = 0; b < nb; ++b)
     if (m->buf_layer[b] == layer) return SOUP_OK;
@@ -1051,6 +1069,7 @@ soup_status layer_backward_body(soup_model* m, int i, const LayerView& L, const 
 // ------------------------------------------------------------------ head
 // logits = RMSNorm(x) W_lm^T (fp32), per-row LSE and target logit.
 soup_status head_forward(soup_model* m, const uint16_t* x, int B, int S, cudaStream_t st) {
+  const NvtxRange trace("head fwd");
   const soup_model_config& c = m->cfg;
   const int T = B * S, h = c.hidden, V = c.vocab;
   SOUP_TRY(launch(m, st, CAT_RMSNORM, 0, 4.0 * T * h + 4.0 * T, "final norm",
@@ -1071,6 +1090,7 @@ soup_status head_forward(soup_model* m, const uint16_t* x, int B, int S, cudaStr
 }
 // dlogits = w_t (softmax - onehot) -> dh = dlogits W_lm -> final-norm backward into dx.
 soup_status head_backward(soup_model* m, const uint16_t* x, int B, int S, uint16_t* dx, cudaStream_t st) {
+  const NvtxRange trace("head bwd");
   const soup_model_config& c = m->cfg;
   const int T = B * S, h = c.hidden, V = c.vocab;
   SOUP_TRY(launch(m, st, CAT_CE, 0, 6.0 * T * V, "ce grad", [&] {
@@ -1090,6 +1110,7 @@ soup_status head_backward(soup_model* m, const uint16_t* x, int B, int S, uint16
 // first run is eager so every kernel attribute and TMA descriptor exists before capture).
 soup_status run_layer(soup_model* m, int dir, int i, const uint8_t* base, const uint16_t* in, uint16_t* out, int B,
                       int S, cudaStream_t st) {
+  const NvtxRange trace(dir == 0 ? "layer fwd" : "layer bwd", i);
   const LayerView v = view_of(m, base);
   if (!m->use_graphs || m->prof) {
     return dir == 0 ? layer_forward(m, i, v, in, out, B, S, st) : layer_backward(m, i, v, in, out, B, S, st);
@@ -1255,6 +1276,7 @@ soup_status read_scalars(soup_model* m, cudaStream_t st, float* loss_out) {
 
 soup_status do_step_body(soup_model* m, soup_loss kind, const soup_batch* bt, float* loss_out, cudaStream_t st);
 soup_status do_step(soup_model* m, soup_loss kind, const soup_batch* bt, float* loss_out, cudaStream_t st) {
+  const NvtxRange trace("step");
   if (m->prof) {
     // the profile's own per-launch overhead: empty launches bracketed like every other one
     for (int k = 0; k < 8; ++k) SOUP_TRY(launch(m, st, CAT_NULL, 0.0, 0.0, "empty launch", [&] { return null_launch(st); }));
