@@ -164,6 +164,18 @@ soup_status soup_layer_blob_bytes(const soup_model_config* cfg, size_t* bytes);
  * memory (synchronises `stream`).  In resident mode the blob is also kept on the device. */
 soup_status soup_model_quantize_layer(soup_model* model, int layer, const float* const w[7],
                                       const uint16_t* gamma_attn, const uint16_t* gamma_mlp, void* stream);
+/* Loads one layer from float32 weights in HOST memory: the library quantises them on the host
+ * (all hardware threads; the same bytes as soup_model_quantize_layer and soup_nf4_quantize_host)
+ * straight into its page-locked layer stack (or the stack file), so a base that never fits on
+ * the GPU in float32 never has to be there (rug.gal radar "Soup ... layer streaming", "En
+ * detalle": the base stays in CPU RAM and reaches the GPU one quantised layer at a time).
+ * w[p]: host fp32 [out_p, in_p] row-major for p = q,k,v,o,gate,up,down; gammas: host bf16
+ * [hidden].  Synchronous: waits for the streamer's copy stream first (it may be reading an older
+ * blob of this layer), returns when the blob is stored; in resident mode the blob is also
+ * copied to the layer's device buffer.  SOUP_ERR_INVALID_ARG for a NULL pointer or a bad layer
+ * index; SOUP_ERR_IO when the stack file cannot be written. */
+soup_status soup_model_load_layer(soup_model* model, int layer, const float* const w[7], const uint16_t* gamma_attn,
+                                  const uint16_t* gamma_mlp);
 /* Loads / reads back a pre-quantised blob (host memory, soup_layer_blob_bytes bytes). */
 soup_status soup_model_load_layer_nf4(soup_model* model, int layer, const void* blob, size_t bytes);
 soup_status soup_model_read_layer_nf4(soup_model* model, int layer, void* blob, size_t bytes);
@@ -183,6 +195,14 @@ soup_status soup_lora_numel(const soup_model_config* cfg, size_t* numel);
 soup_status soup_lora_offset(const soup_model_config* cfg, int layer, int proj, int which_b, size_t* offset,
                              int* rows, int* cols);
 soup_status soup_model_set_lora(soup_model* model, float* params, float* grads, float* adam_m, float* adam_v);
+/* Sets the adapters of one projection: copies A [r, in] and B [out, r] (fp32, row-major, host
+ * or device memory) into the parameter buffer given to soup_model_set_lora, at the place
+ * soup_lora_offset names, and refreshes their bf16 copy; enqueued on `stream`.  The adapters
+ * are the rank-r pair of each adapted projection (guillermodelpino soup.yaml example: r,
+ * alpha; rug.gal "En detalle": only the adapter is trained).  SOUP_ERR_STATE before
+ * soup_model_set_lora; SOUP_ERR_INVALID_ARG for a bad layer or projection index. */
+soup_status soup_model_set_lora_proj(soup_model* model, int layer, int proj, const float* A, const float* B,
+                                     void* stream);
 /* The kernels read the LoRA parameters through a bf16 copy kept by the library (the values
  * the fp32 parameters round to), refreshed by soup_model_set_lora (synchronous) and by every
  * optimizer update the library performs.  A caller that changes the fp32 parameters itself
@@ -246,8 +266,11 @@ soup_status soup_nf4_quantize(const float* w, long long n, uint8_t* codes, int8_
  * library (4 MiB of device memory on every GPU that loads the library, held until the
  * process exits), so n may be at most SOUP_NF4_STATIC_MAX_ELEMS (= 64 x 2^20 elements, every
  * 8B-shape projection); larger n returns SOUP_ERR_INVALID_ARG without launching anything.
- * The call allocates nothing.  The first call on a device looks up the array's device
- * address with that device current (make that first call before any stream capture).  All
+ * The call allocates nothing.  Every call made outside stream capture looks up the array's
+ * device address on the current device (so a context recreated by cudaDeviceReset is picked
+ * up); a call made while `stream` is capturing reuses the address found by the last call
+ * outside capture on that device, and returns SOUP_ERR_STATE if there was none: make the
+ * first call on a device before any stream capture, and again after a cudaDeviceReset.  All
  * calls share the one array and it keeps the last call's contents; every entry a call reads
  * is written earlier in the same call, so nothing needs clearing, but calls whose kernels
  * overlap on the GPU (different streams, or different host threads) race on it: serialise
@@ -255,6 +278,12 @@ soup_status soup_nf4_quantize(const float* w, long long n, uint8_t* codes, int8_
 #define SOUP_NF4_STATIC_MAX_ELEMS (64LL << 20)
 soup_status soup_nf4_quantize_static(const float* w, long long n, uint8_t* codes, int8_t* q8, float* scales,
                                      float* mean, void* stream);
+/* The same quantiser on the host: w and every output are HOST pointers (sizes as for
+ * soup_nf4_quantize); runs on n_threads host threads (<= 0: all hardware threads) and returns
+ * when done.  No GPU is needed.  The NF4 format of the pages' `quantization: 4bit`
+ * (guillermodelpino soup.yaml example; rug.gal "En detalle"). */
+soup_status soup_nf4_quantize_host(const float* w, long long n, uint8_t* codes, int8_t* q8, float* scales, float* mean,
+                                   int n_threads);
 /* Standalone NF4 -> bf16 dequantiser: out[i] = bf16_rn(c[code_i] * mhat(block(i))). */
 soup_status soup_nf4_dequantize(const uint8_t* codes, const int8_t* q8, const float* scales, const float* mean,
                                 long long n, uint16_t* out, void* stream);
@@ -344,6 +373,15 @@ soup_status soup_get_timed_category(soup_model* model, soup_profile_entry* out, 
 soup_status soup_get_timed_profile(soup_model* model, soup_profile_entry* out, int max_entries, int* n_entries,
                                    int reset);
 
+/* Self-test of the failure path of every in-kernel wait.  Each wait of the library's kernels on
+ * a shared-memory barrier is bounded (2 s): when the bound runs out the kernel sets the model's
+ * device error word and runs to its end instead of hanging, and the next call that reads the
+ * word returns SOUP_ERR_TIMEOUT.  This call launches one thread that waits, with the same wait
+ * code, on a barrier that nothing ever arrives on, with a bound of limit_us microseconds (1 ..
+ * 1000000); it returns after enqueueing on `stream`.  A soup_check_device (or the next
+ * soup_step) then reports SOUP_ERR_TIMEOUT once, clears the word, and the model stays usable.
+ * The pages have no counterpart: this is the library's own fault reporting. */
+soup_status soup_selftest_bounded_wait(soup_model* model, int limit_us, void* stream);
 /* Reads (and clears) the device error word; SOUP_ERR_TIMEOUT / SOUP_ERR_DEVICE_CHECK if set. */
 soup_status soup_check_device(soup_model* model, void* stream);
 const char* soup_status_string(soup_status status);

@@ -15,7 +15,7 @@ LIB_PATH = os.path.join(HERE, "libsoup.so")
 
 SOUP_OK = 0
 STATUS = {0: "SOUP_OK", -1: "SOUP_ERR_INVALID_ARG", -2: "SOUP_ERR_STATE", -3: "SOUP_ERR_OOM", -4: "SOUP_ERR_CUDA",
-          -5: "SOUP_ERR_TIMEOUT", -6: "SOUP_ERR_DEVICE_CHECK", -7: "SOUP_ERR_UNSUPPORTED"}
+          -5: "SOUP_ERR_TIMEOUT", -6: "SOUP_ERR_DEVICE_CHECK", -7: "SOUP_ERR_UNSUPPORTED", -8: "SOUP_ERR_IO"}
 SOUP_RESIDENT, SOUP_STREAMED = 0, 1
 SOUP_SOURCE_RAM, SOUP_SOURCE_FILE, SOUP_SOURCE_AUTO = 0, 1, 2
 SOUP_LOSS_SFT, SOUP_LOSS_DPO, SOUP_LOSS_KTO, SOUP_LOSS_ORPO, SOUP_LOSS_SIMPO = 0, 1, 2, 3, 4
@@ -76,6 +76,7 @@ SIGNATURES = {
     "soup_layer_blob_bytes": [POINTER(ModelConfig), POINTER(c_size_t)],
     "soup_layer_blob_part": [POINTER(ModelConfig), c_int, c_int, POINTER(c_size_t), POINTER(c_size_t)],
     "soup_model_quantize_layer": [c_void_p, c_int, POINTER(c_void_p), c_void_p, c_void_p, c_void_p],
+    "soup_model_load_layer": [c_void_p, c_int, POINTER(c_void_p), c_void_p, c_void_p],
     "soup_model_load_layer_nf4": [c_void_p, c_int, c_void_p, c_size_t],
     "soup_model_read_layer_nf4": [c_void_p, c_int, c_void_p, c_size_t],
     "soup_model_set_head": [c_void_p, c_void_p, c_void_p, c_void_p],
@@ -83,6 +84,7 @@ SIGNATURES = {
     "soup_lora_offset": [POINTER(ModelConfig), c_int, c_int, c_int, POINTER(c_size_t), POINTER(c_int), POINTER(c_int)],
     "soup_model_set_lora": [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p],
     "soup_set_lora_enabled": [c_void_p, c_int],
+    "soup_model_set_lora_proj": [c_void_p, c_int, c_int, c_void_p, c_void_p, c_void_p],
     "soup_model_refresh_lora": [c_void_p, c_void_p],
     "soup_model_merge_lora": [c_void_p, c_int, c_int, c_void_p, c_void_p],
     "soup_layer_fwd": [c_void_p, c_int, c_void_p, c_void_p, c_int, c_int, c_void_p],
@@ -92,6 +94,7 @@ SIGNATURES = {
     "soup_last_logps": [c_void_p, POINTER(c_float), POINTER(c_float), c_int],
     "soup_nf4_quantize": [c_void_p, c_longlong, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p],
     "soup_nf4_quantize_static": [c_void_p, c_longlong, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p],
+    "soup_nf4_quantize_host": [c_void_p, c_longlong, c_void_p, c_void_p, c_void_p, c_void_p, c_int],
     "soup_nf4_dequantize": [c_void_p, c_void_p, c_void_p, c_void_p, c_longlong, c_void_p, c_void_p],
     "soup_nf4_matmul": [c_void_p, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_void_p,
                         c_void_p, c_void_p],
@@ -99,6 +102,7 @@ SIGNATURES = {
     "soup_get_stats": [c_void_p, POINTER(Stats)],
     "soup_reset_stats": [c_void_p],
     "soup_check_device": [c_void_p, c_void_p],
+    "soup_selftest_bounded_wait": [c_void_p, c_int, c_void_p],
     "soup_set_profiling": [c_void_p, c_int],
     "soup_h2d_probe": [c_void_p, c_int, POINTER(ctypes.c_double)],
     "soup_get_profile": [c_void_p, POINTER(ProfileEntry), c_int, POINTER(c_int), c_int],

@@ -79,14 +79,14 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
 // Bounded wait. On timeout: sets the device error word and the CTA's abort flag; every
 // later wait in the CTA then returns at once, so the kernel always terminates.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                                  int* err) {
+                                                  int* err, unsigned long long limit_ns = WAIT_LIMIT_NS) {
   if (mbar_test_wait(bar, parity)) return true;
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (globaltimer_ns() - t0 > WAIT_LIMIT_NS) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       *abort_flag = 1;
       set_dev_error(err, DEVERR_TIMEOUT);
       return false;

@@ -718,6 +718,25 @@ cudaError_t busy_wait_launch(long long cycles, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+// Self-test of the bounded in-kernel wait: one thread waits on a shared-memory barrier that
+// expects one arrival which never comes, with the production wait helper and a short limit;
+// when the limit runs out the helper sets the device error word, and the kernel returns.
+__global__ void bounded_wait_selftest_kernel(int* err, unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  mbar_init(&bar, 1);
+  mbar_fence_init();
+  abort_flag = 0;
+  __syncwarp();
+  mbar_wait_bounded(&bar, 0u, &abort_flag, err, limit_ns);
+}
+
+cudaError_t bounded_wait_selftest_launch(int* err, unsigned long long limit_ns, cudaStream_t st) {
+  bounded_wait_selftest_kernel<<<1, 1, 0, st>>>(err, limit_ns);
+  ++g_kernel_launches;
+  return cudaGetLastError();
+}
+
 // An empty launch: what the live profile's event pair measures around a kernel that does no
 // work (its per-launch overhead).
 __global__ void null_kernel() {}

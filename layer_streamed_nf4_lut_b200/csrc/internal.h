@@ -156,6 +156,10 @@ struct LUT16 {
 };
 cudaError_t nf4_quantize_launch(const float* w, long long n, uint8_t* codes, int8_t* q8, float* scales, float* mean,
                                 float* absmax_scratch, const LUT16& lut, cudaStream_t st);
+// Host quantiser (host_quant.cu): the same bytes as nf4_quantize_launch, from host memory,
+// on `threads` host threads (<= 0: all hardware threads).  Returns a soup_status.
+int host_nf4_quantize(const float* w, long long n, uint8_t* codes, int8_t* q8, float* scales, float* mean,
+                      int threads);
 cudaError_t nf4_dequant_launch(const uint8_t* codes, const int8_t* q8, const float* scales, const float* mean,
                                long long n, uint16_t* out, const LUT16& lut, cudaStream_t st);
 
@@ -226,7 +230,9 @@ cudaError_t ce_grad_launch(const float* logits, const float* lse, const int32_t*
 cudaError_t adamw_launch(float* p, const float* g, float* m, float* v, uint16_t* pb, long long n, float lr, float b1,
                          float b2, float eps, float wd, int t, cudaStream_t st);
 cudaError_t busy_wait_launch(long long cycles, cudaStream_t st);  // profiling aid, not counted as a launch
-cudaError_t null_launch(cudaStream_t st);                           // profiling aid, not counted as a launch
+cudaError_t null_launch(cudaStream_t st);
+// one thread waits on a barrier nothing arrives on, limit_ns ns, then sets *err (timeout)
+cudaError_t bounded_wait_selftest_launch(int* err, unsigned long long limit_ns, cudaStream_t st);                           // profiling aid, not counted as a launch
 cudaError_t f32_to_bf16_launch(const float* x, uint16_t* y, long long n, cudaStream_t st);
 cudaError_t fill_zero_launch(void* p, size_t bytes, cudaStream_t st);
 

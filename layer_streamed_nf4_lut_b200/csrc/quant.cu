@@ -170,18 +170,28 @@ static_assert(kStaticBlocks * 64 == SOUP_NF4_STATIC_MAX_ELEMS, "limit in soup.h"
 static __device__ __align__(256) float g_static_absmax[kStaticBlocks];
 
 // Device address of g_static_absmax per device ordinal (host code may not use the symbol's
-// name as a pointer: that is a host-side stand-in, not a device address).
+// name as a pointer: that is a host-side stand-in, not a device address).  The address is
+// looked up again on every call made outside stream capture, so a context recreated after
+// cudaDeviceReset (which reloads the module, possibly elsewhere) is picked up; a call made
+// while `stream` is capturing uses the address found by the last call outside capture.
 std::mutex g_static_mu;
 float* g_static_ptr[64] = {};
 
-soup_status static_scratch(float** out) {
+soup_status static_scratch(cudaStream_t stream, float** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return SOUP_ERR_CUDA;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) return SOUP_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_static_mu);
-  if (!g_static_ptr[dev]) {
+  if (cap == cudaStreamCaptureStatusNone) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_static_absmax) != cudaSuccess || !p) return SOUP_ERR_CUDA;
+    if (cudaGetSymbolAddress(&p, g_static_absmax) != cudaSuccess || !p) {
+      g_static_ptr[dev] = nullptr;
+      return SOUP_ERR_CUDA;
+    }
     g_static_ptr[dev] = static_cast<float*>(p);
+  } else if (!g_static_ptr[dev]) {
+    return SOUP_ERR_STATE;  // no call outside capture has looked the address up on this device
   }
   *out = g_static_ptr[dev];
   return SOUP_OK;
@@ -196,7 +206,7 @@ extern "C" soup_status soup_nf4_quantize_static(const float* w, long long n, uin
   if (!w || n <= 0 || !codes || !q8 || !scales || !mean) return SOUP_ERR_INVALID_ARG;
   if (n > SOUP_NF4_STATIC_MAX_ELEMS) return SOUP_ERR_INVALID_ARG;
   float* scratch = nullptr;
-  const soup_status s = soup::static_scratch(&scratch);
+  const soup_status s = soup::static_scratch(static_cast<cudaStream_t>(stream), &scratch);
   if (s != SOUP_OK) return s;
   const cudaError_t e = soup::nf4_quantize_launch(w, n, codes, q8, scales, mean, scratch, soup_codebook_lut(),
                                                   static_cast<cudaStream_t>(stream));

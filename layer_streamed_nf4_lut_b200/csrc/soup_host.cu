@@ -1797,6 +1797,51 @@ soup_status soup_model_load_layer_nf4(soup_model* m, int layer, const void* blob
   })
 }
 
+soup_status soup_model_load_layer(soup_model* m, int layer, const float* const w[7], const uint16_t* gamma_attn,
+                                  const uint16_t* gamma_mlp) {
+  if (!m || !w || !gamma_attn || !gamma_mlp || layer < 0 || layer >= m->cfg.n_layers) return SOUP_ERR_INVALID_ARG;
+  for (int p = 0; p < 7; ++p)
+    if (!w[p]) return SOUP_ERR_INVALID_ARG;
+  SOUP_GUARD({
+    // the streamer may still be copying an older blob of this layer out of page-locked memory
+    if (m->copy_stream) SOUP_TRY(wait_stream(m, m->copy_stream));
+    std::vector<uint8_t> staged;
+    uint8_t* dst;
+    if (m->use_file) {
+      staged.assign(m->layout.total, 0);
+      dst = staged.data();
+    } else {
+      dst = m->host_blob[layer];
+      std::memset(dst, 0, m->layout.total);
+    }
+    ProjShape s[7];
+    proj_shapes(m->cfg, s);
+    for (int p = 0; p < 7; ++p) {
+      const long long n = static_cast<long long>(s[p].out) * s[p].in;
+      const int st = host_nf4_quantize(w[p], n, dst + m->layout.off[p][0],
+                                       reinterpret_cast<int8_t*>(dst + m->layout.off[p][1]),
+                                       reinterpret_cast<float*>(dst + m->layout.off[p][2]),
+                                       reinterpret_cast<float*>(dst + m->layout.off[p][3]), 0);
+      if (st != SOUP_OK) {
+        m->host_loaded[layer] = 0;
+        m->err = "host NF4 quantiser failed";
+        return st;
+      }
+    }
+    std::memcpy(dst + m->layout.off[7][0], gamma_attn, static_cast<size_t>(m->cfg.hidden) * 2);
+    std::memcpy(dst + m->layout.off[8][0], gamma_mlp, static_cast<size_t>(m->cfg.hidden) * 2);
+    if (m->use_file && !m->file.write(layer, dst, m->err)) return SOUP_ERR_IO;
+    if (m->cfg.mode == SOUP_RESIDENT) {
+      SOUP_CK(cudaMemcpy(m->dev_buf[layer], dst, m->layout.total, cudaMemcpyHostToDevice));
+    } else {
+      for (size_t b = 0; b < m->buf_layer.size(); ++b)
+        if (m->buf_layer[b] == layer) m->buf_layer[b] = -1;
+    }
+    m->host_loaded[layer] = 1;
+    return SOUP_OK;
+  })
+}
+
 soup_status soup_model_read_layer_nf4(soup_model* m, int layer, void* blob, size_t bytes) {
   if (!m || !blob || layer < 0 || layer >= m->cfg.n_layers || bytes != m->layout.total) return SOUP_ERR_INVALID_ARG;
   if (!m->host_loaded[layer]) return SOUP_ERR_STATE;
@@ -1836,6 +1881,33 @@ soup_status soup_model_set_lora(soup_model* m, float* params, float* grads, floa
     SOUP_TRY(check_launch(m, f32_to_bf16_launch(params, m->lora_bf16, static_cast<long long>(m->lora_n), nullptr),
                           "lora copy"));
     SOUP_CK(cudaDeviceSynchronize());
+    return SOUP_OK;
+  })
+}
+
+soup_status soup_model_set_lora_proj(soup_model* m, int layer, int proj, const float* A, const float* B,
+                                     void* stream) {
+  if (!m || !A || !B || layer < 0 || layer >= m->cfg.n_layers || proj < 0 || proj > 6) return SOUP_ERR_INVALID_ARG;
+  if (!m->lora_p) {
+    m->err = "soup_model_set_lora first";
+    return SOUP_ERR_STATE;
+  }
+  SOUP_GUARD({
+    ProjShape s[7];
+    proj_shapes(m->cfg, s);
+    const int r = m->cfg.lora_r;
+    const size_t na = static_cast<size_t>(r) * s[proj].in;
+    const size_t nbb = static_cast<size_t>(s[proj].out) * r;
+    const size_t oa = lora_off(m->cfg, layer, proj, 0);
+    const size_t ob = lora_off(m->cfg, layer, proj, 1);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    SOUP_CK(cudaMemcpyAsync(m->lora_p + oa, A, na * sizeof(float), cudaMemcpyDefault, st));
+    SOUP_CK(cudaMemcpyAsync(m->lora_p + ob, B, nbb * sizeof(float), cudaMemcpyDefault, st));
+    SOUP_TRY(check_launch(m, f32_to_bf16_launch(m->lora_p + oa, m->lora_bf16 + oa, static_cast<long long>(na), st),
+                          "lora copy"));
+    SOUP_TRY(check_launch(m, f32_to_bf16_launch(m->lora_p + ob, m->lora_bf16 + ob, static_cast<long long>(nbb), st),
+                          "lora copy"));
+    for (auto& a : m->saved) a.valid = 0;
     return SOUP_OK;
   })
 }
@@ -2275,6 +2347,14 @@ soup_status soup_h2d_probe(soup_model* m, int reps, double* gbs) {
     *gbs = static_cast<double>(reps) * m->layout.total / (ms * 1e-3) / 1e9;
     return SOUP_OK;
   })
+}
+
+soup_status soup_selftest_bounded_wait(soup_model* m, int limit_us, void* stream) {
+  if (!m || limit_us < 1 || limit_us > 1000000) return SOUP_ERR_INVALID_ARG;
+  SOUP_GUARD(return check_launch(m,
+                                 bounded_wait_selftest_launch(m->scal + 1, 1000ull * static_cast<unsigned>(limit_us),
+                                                              static_cast<cudaStream_t>(stream)),
+                                 "bounded wait self-test");)
 }
 
 soup_status soup_check_device(soup_model* m, void* stream) {

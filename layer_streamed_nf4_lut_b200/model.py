@@ -129,6 +129,16 @@ class SoupModel:
         ptrs = (c_void_p * 7)(*[w[p].data_ptr() for p in PROJ])
         self._ck(lib.soup_model_quantize_layer(self.h, layer, ptrs, _ptr(gamma_attn), _ptr(gamma_mlp), _stream_ptr()))
 
+    def load_layer(self, layer: int, w: dict, gamma_attn: np.ndarray, gamma_mlp: np.ndarray):
+        """w[p]: host fp32 arrays [out, in]; gammas: host bf16 bit patterns (uint16) [hidden].
+        The library quantises on the host into its page-locked layer stack."""
+        arrs = [np.ascontiguousarray(w[p], dtype=np.float32) for p in PROJ]
+        ga = np.ascontiguousarray(gamma_attn, dtype=np.uint16)
+        gm = np.ascontiguousarray(gamma_mlp, dtype=np.uint16)
+        ptrs = (c_void_p * 7)(*[a.ctypes.data for a in arrs])
+        self._ck(lib.soup_model_load_layer(self.h, layer, ptrs, ga.ctypes.data_as(c_void_p),
+                                           gm.ctypes.data_as(c_void_p)))
+
     def load_layer_nf4(self, layer: int, blob: np.ndarray):
         blob = np.ascontiguousarray(blob, dtype=np.uint8)
         self._ck(lib.soup_model_load_layer_nf4(self.h, layer, blob.ctypes.data_as(c_void_p), blob.nbytes))
@@ -151,6 +161,13 @@ class SoupModel:
         self.adam_v = torch.zeros_like(params)
         self._ck(lib.soup_model_set_lora(self.h, _ptr(self.lora_params), _ptr(self.lora_grads), _ptr(self.adam_m),
                                          _ptr(self.adam_v)))
+
+    def set_lora_proj(self, layer: int, proj: str, A: torch.Tensor, B: torch.Tensor):
+        """Copies one projection's fp32 adapters (cuda or cpu tensors) into the parameter buffer."""
+        A = A.to(torch.float32).contiguous()
+        B = B.to(torch.float32).contiguous()
+        self._ck(lib.soup_model_set_lora_proj(self.h, layer, PROJ.index(proj), _ptr(A), _ptr(B), _stream_ptr()))
+        torch.cuda.current_stream().synchronize()
 
     def refresh_lora(self):
         """Call after changing lora_params outside the library (refreshes its bf16 copy)."""
@@ -309,6 +326,20 @@ def nf4_quantize(w: torch.Tensor) -> dict:
                                 _ptr(out["mean"]), _ptr(scratch), _stream_ptr()))
     out["n"] = n
     out["shape"] = tuple(w.shape)
+    return out
+
+
+def nf4_quantize_host(w: np.ndarray, threads: int = 0) -> dict:
+    """NF4 + double quant of a host fp32 array on the host (no GPU); numpy outputs."""
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    n = w.size
+    nb = (n + 63) // 64
+    ng = (nb + 255) // 256
+    out = dict(codes=np.empty((n + 1) // 2, np.uint8), q8=np.empty(nb, np.int8), scales=np.empty(ng, np.float32),
+               mean=np.empty(1, np.float32))
+    p = lambda a: a.ctypes.data_as(c_void_p)
+    check(lib.soup_nf4_quantize_host(p(w), n, p(out["codes"]), p(out["q8"]), p(out["scales"]), p(out["mean"]),
+                                     int(threads)))
     return out
 
 

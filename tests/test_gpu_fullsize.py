@@ -114,3 +114,47 @@ def test_full_8b_streamed_equals_resident_and_load_counts():
     finally:
         for m in models.values():
             m.close()
+
+
+def test_full_width_layer_and_head_dpo_step_vs_oracle():
+    """The DPO step at the 8B width and the workload's batch shape (2 pairs x 512 tokens, shared
+    256-token prefix, beta 0.1; one decoder layer, full vocabulary): reference log-probs from
+    the LoRA-off re-stream, policy log-probs, loss and every LoRA gradient against the oracle."""
+    from layer_streamed_nf4_lut_b200.model import SoupModel
+    cfg = dict(synth.L8B_DPO, n_layers=1)
+    P, S, pre, beta = cfg["n_pairs"], cfg["seq"], cfg["prefix_len"], cfg["beta"]
+    w = _device_layer(cfg, 7, 0)
+    g_attn = (1.0 + 0.1 * synth.normal_device((cfg["hidden"],), 87, 1.0)).to(torch.bfloat16)
+    g_mlp = (1.0 + 0.1 * synth.normal_device((cfg["hidden"],), 88, 1.0)).to(torch.bfloat16)
+    emb = synth.normal_device((cfg["vocab"], cfg["hidden"]), 89, 0.02).to(torch.bfloat16)
+    lm = synth.normal_device((cfg["vocab"], cfg["hidden"]), 90, 0.02).to(torch.bfloat16)
+    g_fin = (1.0 + 0.1 * synth.normal_device((cfg["hidden"],), 91, 1.0)).to(torch.bfloat16)
+    lora = synth.lora_weights(cfg, 8)
+    gm = SoupModel(cfg, mode="streamed", n_layer_buffers=2, max_tokens=2 * P * S)
+    try:
+        gm.quantize_layer(0, w, g_attn, g_mlp)
+        gm.set_head(emb, g_fin, lm)
+        gm.set_lora(_lora_flat(cfg, lora))
+        ids = synth.preference_batch(cfg, 92)
+        loss = gm.step(torch.from_numpy(ids).cuda(), loss="dpo", n_pairs=P, prefix_len=pre, beta=beta,
+                       apply_optimizer=False)
+        pi, ref = gm.last_logps(2 * P)
+        grads = {p: (gm.lora_view(gm.lora_grads, 0, p, 0).double().cpu().numpy(),
+                     gm.lora_view(gm.lora_grads, 0, p, 1).double().cpu().numpy()) for p in PROJ}
+        q = {p: nf4.quantise(w[p].cpu().numpy()) for p in PROJ}
+        q["attn_norm"], q["mlp_norm"] = _bits(g_attn), _bits(g_mlp)
+        del w
+        layers, head = om.model_from_quantised(cfg, [q], (_bits(emb), _bits(lm), _bits(g_fin)))
+        olora = {k: (a.astype(np.float64), b.astype(np.float64)) for k, (a, b) in lora.items()}
+        ol, og, aux = om.dpo_step(dict(cfg, batch=2 * P), layers, olora, head, ids, pre, beta)
+        # sequence log-prob sums of 256 targets each (fp32 sums on the GPU)
+        assert np.max(np.abs(pi - aux["pi"]) / np.abs(aux["pi"])) < 1e-2, (pi, aux["pi"])
+        assert np.max(np.abs(ref - aux["ref"]) / np.abs(aux["ref"])) < 1e-2, (ref, aux["ref"])
+        closed, _ = om.dpo_loss(pi.astype(np.float64), ref.astype(np.float64), beta)
+        assert abs(loss - closed) < 1e-5
+        assert abs(loss - ol) <= 1e-2 * abs(ol), (loss, ol)
+        for p in PROJ:
+            assert cosine(grads[p][0], og[(0, p)][0]) > 0.999, p
+            assert cosine(grads[p][1], og[(0, p)][1]) > 0.999, p
+    finally:
+        gm.close()

@@ -72,7 +72,7 @@ def test_dpo_step_matches_oracle(tiny_pair):
     closed, _ = om.dpo_loss(pi.astype(np.float64), ref.astype(np.float64), 0.1)
     assert abs(loss - closed) < 1e-5
     assert abs(loss - ol) < 1e-2 * abs(ol)
-    _check_grads(tiny_pair, "streamed", og, min_cos=0.99)
+    _check_grads(tiny_pair, "streamed", og)
 
 
 def test_layer_load_counts():
