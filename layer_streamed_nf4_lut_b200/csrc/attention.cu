@@ -1,261 +1,296 @@
-// Causal grouped-query attention, forward and backward, flash-style (sm_100a).
+// Causal grouped-query attention, forward and backward, on the tcgen05 tensor cores (sm_100a).
 //
-// q, k, v live in one [T, (hq + 2 hkv) d] bf16 buffer (the fused q|k|v projection output,
-// RoPE already applied to q and k).  Query head h reads kv head h / (hq / hkv).
-// Scores are scaled by 1/sqrt(d); the softmax runs online over 64-wide kv tiles with
-// quad-shuffle row reductions; the forward saves the natural-log LSE per (b, h, s).
+// One CTA per (128-query tile, query head, sequence).  q, k, v come from the fused
+// [T, (hq + 2 hkv) d] bf16 projection output (RoPE applied) through TMA (128-byte swizzle); query
+// head h reads kv head h / (hq / hkv).  Per 128-key tile j the CTA computes
+//   S_j = Q K_j^T                      tcgen05.mma, both operands K-major in shared memory, fp32 in TMEM
+//   P_j = exp(S_j / sqrt(d) - m)       softmax warps: one thread per query row reads its row of S_j
+//                                      from TMEM, keeps the running max m and sum l, writes P_j back
+//                                      to TMEM as bf16 over the first half of S_j's columns
+//   O  = O * exp(m_old - m) + P_j V_j  the softmax warps rescale O in TMEM when m grows; P_j is the
+//                                      MMA's A operand straight from TMEM, V_j the MN-major B operand
+// and finally out = O / l, lse = m + log l (natural log) per row.  S/P use three TMEM buffers so
+// that S_{j+1} is computed while the softmax of j runs and PV_{j-1} finishes; O takes d columns.
 //
-// Backward (no atomics, deterministic):
-//   delta[t, h] = sum_d dO * O                                      (row kernel)
-//   pass 1, one CTA per (kv tile, kv head): dV += P^T dO, dK += dS^T Q over every query head of
-//           the group and every causal query tile, in a fixed order;
-//   pass 2, one CTA per (query tile, head): dQ += dS K over the causal kv tiles.
-//   P = exp(S - lse), dS = P * (dP - delta), dP = dO V^T.
+// Warp roles (192 threads): warps 0-3 softmax and epilogue (TMEM lane quarters 0-3, thread = query
+// row), warp 4 allocates TMEM and its lane 0 issues the MMAs, warp 5 lane 0 issues the TMA loads
+// (Q once, K/V tiles in a 2-stage ring).  Every wait is bounded (mbar_wait_bounded): on timeout the
+// device error word is set and the kernel runs to its end.
 //
-// Shared-prefix pair blocks (AttnShape.pl > 0): [prefix | chosen | rejected] rows, the rejected
-// response attending to the prefix and to itself only; a rejected query tile skips the chosen
-// kv tiles, a chosen kv tile is read by chosen query tiles only.
-//
-// Tiles are 64 x 64; 4 warps each own 16 rows; bf16 m16n8k16 tensor-core MMAs with fp32
-// accumulators, operands fed from padded shared memory by ldmatrix.
+// Key tiles a query tile reads: those with a visible (query, key) pair (attn_mask.cuh); the plain
+// causal layout reads tiles 0..qt.  Rows at or past S (a ragged last tile) are masked as keys and
+// never stored as queries.
+#include "attn_mask.cuh"
 #include "common.cuh"
 #include "internal.h"
+#include "tc.cuh"
 
 namespace soup {
 
 namespace {
 
-constexpr int AT_BR = 64;
-constexpr int AT_THREADS = 128;
-constexpr float LOG2E = 1.4426950408889634f;
+constexpr int TQ = 128;  // query rows per CTA: one M = 128 accumulator
+constexpr int TK = 128;  // keys per tile
+constexpr int FWD_THREADS = 192;
+constexpr int SOFTMAX_WARPS = 4;
+constexpr int MMA_WARP = 4, TMA_WARP = 5;
+constexpr int N_SBUF = 3;  // TMEM S/P buffers
+constexpr float LOG2E_F = 1.4426950408889634f;
 
 template <int D>
-struct AttnCfg {
-  static constexpr int LDS = D + 8;  // padded row (elements); 16-byte aligned, conflict-free ldmatrix
-  static constexpr int TILE = AT_BR * LDS;
+struct FwdCfg {
+  static constexpr int TILE_BYTES = TQ * D * 2;  // one [128 x D] bf16 tile: D/64 swizzle atoms of 16 KB
+  static constexpr int Q_OFF = 0;
+  static constexpr int K_OFF = TILE_BYTES;       // 2 stages
+  static constexpr int V_OFF = 3 * TILE_BYTES;   // 2 stages
+  static constexpr int BAR_OFF = 5 * TILE_BYTES;
+  static constexpr int SMEM_BYTES = 1024 + BAR_OFF + 256;
+  static constexpr int O_COL = N_SBUF * TK;      // TMEM column of the O accumulator
+  static constexpr int TMEM_COLS = 512;
+  static_assert(O_COL + D <= TMEM_COLS, "TMEM budget");
 };
 
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-__device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+// Key tile j is read by query tile qt.
+__device__ __forceinline__ bool kv_needed(const AttnShape& s, int qt, int j) {
+  if (s.pl == 0) return j <= qt && j * TK < s.S;
+  return block_visible(s, qt * TQ, qt * TQ + TQ, j * TK, j * TK + TK);
 }
 
-// Visibility of key row k to query row q (block-relative).  Plain layout: causal.  Shared-
-// prefix pair layout: segment 0 = prefix, 1 = chosen, 2 = rejected (rows pl + rl ..), position
-// = row, minus rl for the rejected rows; a key is visible if it is in the prefix or in the
-// query's own segment, at a position not after the query's.
-__device__ __forceinline__ int pk_seg(const AttnShape& s, int x) { return x < s.pl ? 0 : (x < s.pl + s.rl ? 1 : 2); }
-__device__ __forceinline__ int pk_pos(const AttnShape& s, int x) { return x < s.pl + s.rl ? x : x - s.rl; }
-__device__ __forceinline__ bool visible(const AttnShape& s, int q, int k) {
-  if (s.pl == 0) return k <= q;
-  const int sk = pk_seg(s, k);
-  return (sk == 0 || sk == pk_seg(s, q)) && pk_pos(s, k) <= pk_pos(s, q);
-}
-// kv tiles a query tile reads, in order: 0..qt, except that a rejected-response query tile
-// skips the chosen response's tiles.  Returns the count; kv tile of step j = j + skip_at(j).
-struct KvRange {
-  int n, jump_from, jump;
-};
-__device__ __forceinline__ KvRange kv_range(const AttnShape& s, int qt) {
-  KvRange r{qt + 1, 1 << 30, 0};
-  if (s.pl > 0 && qt * AT_BR >= s.pl + s.rl) {
-    r.jump_from = s.pl / AT_BR;
-    r.jump = s.rl / AT_BR;
-    r.n = qt + 1 - r.jump;
-  }
-  return r;
-}
-__device__ __forceinline__ int kv_tile(const KvRange& r, int j) { return j >= r.jump_from ? j + r.jump : j; }
+template <int D>
+__global__ void __launch_bounds__(FWD_THREADS, 1)
+    attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap, const AttnShape s, uint16_t* __restrict__ out,
+                       float* __restrict__ lse, int* err) {
+  using C = FwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* base = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + C::BAR_OFF);
+  uint64_t* q_full = bars;          // 1
+  uint64_t* kv_full = bars + 1;     // 2
+  uint64_t* kv_empty = bars + 3;    // 2
+  uint64_t* s_full = bars + 5;      // 3
+  uint64_t* p_full = bars + 8;      // 3
+  uint64_t* o_ready = bars + 11;    // 1
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 13);
 
-// Load a 64 x D tile of rows [r0, r0+64) (rows >= nrows zero-filled) with cp.async.
-template <int D>
-__device__ __forceinline__ void load_tile_async(uint16_t* dst, const uint16_t* src, long long ld, int r0, int nrows) {
-  constexpr int CH = D / 8;
-  for (int c = threadIdx.x; c < AT_BR * CH; c += AT_THREADS) {
-    const int r = c / CH, cc = c % CH;
-    const bool ok = (r0 + r) < nrows;
-    const uint16_t* g = src + static_cast<long long>(ok ? (r0 + r) : r0) * ld + cc * 8;
-    cp_async16(dst + r * AttnCfg<D>::LDS + cc * 8, g, ok);
-  }
-}
-
-// A fragment (16 rows x 16 cols at column k0) of a row-major padded tile, rows [row0, row0+16).
-template <int D>
-__device__ __forceinline__ void lda_frag(const uint16_t* tile, int row0, int k0, uint32_t (&a)[4]) {
-  const int lane = threadIdx.x & 31;
-  const int mi = lane >> 3, ri = lane & 7;
-  const uint16_t* p = tile + (row0 + ri + (mi & 1) * 8) * AttnCfg<D>::LDS + k0 + (mi >> 1) * 8;
-  ldsm_x4(smem_u32(p), a[0], a[1], a[2], a[3]);
-}
-// B fragments for two n8 blocks (rows n0..n0+15 of a [n][k] tile, k chunk k0..k0+15).
-template <int D>
-__device__ __forceinline__ void ldb_nk(const uint16_t* tile, int n0, int k0, uint32_t& b00, uint32_t& b01,
-                                       uint32_t& b10, uint32_t& b11) {
-  const int lane = threadIdx.x & 31;
-  const int mi = lane >> 3, ri = lane & 7;
-  const uint16_t* p = tile + (n0 + (mi >> 1) * 8 + ri) * AttnCfg<D>::LDS + k0 + (mi & 1) * 8;
-  ldsm_x4(smem_u32(p), b00, b01, b10, b11);
-}
-// B fragments for two n8 blocks (columns n0..n0+15 of a [k][n] tile, k rows k0..k0+15).
-template <int D>
-__device__ __forceinline__ void ldb_kn(const uint16_t* tile, int k0, int n0, uint32_t& b00, uint32_t& b01,
-                                       uint32_t& b10, uint32_t& b11) {
-  const int lane = threadIdx.x & 31;
-  const int mi = lane >> 3, ri = lane & 7;
-  const uint16_t* p = tile + (k0 + (mi & 1) * 8 + ri) * AttnCfg<D>::LDS + n0 + (mi >> 1) * 8;
-  ldsm_x4_t(smem_u32(p), b00, b01, b10, b11);
-}
-
-// ---------------------------------------------------------------- forward
-template <int D>
-__global__ void __launch_bounds__(AT_THREADS) attn_fwd_kernel(const AttnShape s, const uint16_t* __restrict__ qkv,
-                                                               uint16_t* __restrict__ out, float* __restrict__ lse) {
-  extern __shared__ __align__(16) uint16_t sm[];
-  using C = AttnCfg<D>;
-  uint16_t* Qs = sm;
-  uint16_t* Ks = sm + C::TILE;      // 2 buffers
-  uint16_t* Vs = sm + 3 * C::TILE;  // 2 buffers
   const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int g = h / (s.hq / s.hkv);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long row_base = static_cast<long long>(b) * s.S;
-  const uint16_t* qsrc = qkv + row_base * s.ld_qkv + h * D;
-  const uint16_t* ksrc = qkv + row_base * s.ld_qkv + (s.hq + g) * D;
-  const uint16_t* vsrc = qkv + row_base * s.ld_qkv + (s.hq + s.hkv + g) * D;
-  const float scale_log2 = LOG2E / sqrtf(static_cast<float>(D));
+  const int ntk = (s.S + TK - 1) / TK;
 
-  const KvRange kr = kv_range(s, qt);
-  const int nkv = kr.n;
-  load_tile_async<D>(Qs, qsrc, s.ld_qkv, qt * AT_BR, s.S);
-  load_tile_async<D>(Ks, ksrc, s.ld_qkv, kv_tile(kr, 0) * AT_BR, s.S);
-  load_tile_async<D>(Vs, vsrc, s.ld_qkv, kv_tile(kr, 0) * AT_BR, s.S);
-  cp_async_commit();
-
-  float oacc[D / 8][4];
-#pragma unroll
-  for (int i = 0; i < D / 8; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.f;
-  float m_r[2] = {-INFINITY, -INFINITY}, l_r[2] = {0.f, 0.f};
-  const int qrow0 = qt * AT_BR + warp * 16 + (lane >> 2);
-
-  for (int j = 0; j < nkv; ++j) {
-    if (j + 1 < nkv) {
-      load_tile_async<D>(Ks + ((j + 1) & 1) * C::TILE, ksrc, s.ld_qkv, kv_tile(kr, j + 1) * AT_BR, s.S);
-      load_tile_async<D>(Vs + ((j + 1) & 1) * C::TILE, vsrc, s.ld_qkv, kv_tile(kr, j + 1) * AT_BR, s.S);
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
     }
-    cp_async_commit();
-    cp_async_wait<1>();
-    __syncthreads();
-    const uint16_t* Kt = Ks + (j & 1) * C::TILE;
-    const uint16_t* Vt = Vs + (j & 1) * C::TILE;
-    const int kt = kv_tile(kr, j);
-    float sacc[8][4];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) sacc[i][0] = sacc[i][1] = sacc[i][2] = sacc[i][3] = 0.f;
-#pragma unroll
-    for (int kc = 0; kc < D / 16; ++kc) {
-      uint32_t a[4];
-      lda_frag<D>(Qs, warp * 16, kc * 16, a);
-#pragma unroll
-      for (int nb2 = 0; nb2 < 4; ++nb2) {
-        uint32_t b00, b01, b10, b11;
-        ldb_nk<D>(Kt, nb2 * 16, kc * 16, b00, b01, b10, b11);
-        mma16816(sacc[2 * nb2], a, b00, b01);
-        mma16816(sacc[2 * nb2 + 1], a, b10, b11);
-      }
+    for (int i = 0; i < N_SBUF; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], SOFTMAX_WARPS);
     }
-    // scale, causal mask, online softmax
-    float mx[2] = {m_r[0], m_r[1]};
-#pragma unroll
-    for (int nb = 0; nb < 8; ++nb) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int kv = kt * AT_BR + nb * 8 + (lane & 3) * 2 + (e & 1);
-        const int qi = qrow0 + (e >> 1) * 8;
-        float v = sacc[nb][e] * scale_log2;
-        if (!visible(s, qi, kv) || kv >= s.S) v = -INFINITY;
-        sacc[nb][e] = v;
-        mx[e >> 1] = fmaxf(mx[e >> 1], v);
-      }
-    }
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 1));
-      mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 2));
-    }
-    float corr[2];
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      corr[r] = (mx[r] == -INFINITY) ? 1.f : exp2f(m_r[r] - mx[r]);
-      m_r[r] = mx[r];
-      l_r[r] *= corr[r];
-    }
-    uint32_t pa[4][4];  // P as A fragments, 4 k16 chunks over the 64 kv columns
-#pragma unroll
-    for (int nb = 0; nb < 8; ++nb) {
-      float p[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float mm = m_r[e >> 1];
-        p[e] = (mm == -INFINITY) ? 0.f : exp2f(sacc[nb][e] - mm);
-        l_r[e >> 1] += p[e];
-      }
-      pa[nb >> 1][(nb & 1) * 2 + 0] = pack_bf16x2(p[0], p[1]);
-      pa[nb >> 1][(nb & 1) * 2 + 1] = pack_bf16x2(p[2], p[3]);
-    }
-#pragma unroll
-    for (int i = 0; i < D / 8; ++i) {
-      oacc[i][0] *= corr[0];
-      oacc[i][1] *= corr[0];
-      oacc[i][2] *= corr[1];
-      oacc[i][3] *= corr[1];
-    }
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const uint32_t a[4] = {pa[c][0], pa[c][1], pa[c][2], pa[c][3]};
-#pragma unroll
-      for (int db = 0; db < D / 8; db += 2) {
-        uint32_t b00, b01, b10, b11;
-        ldb_kn<D>(Vt, c * 16, db * 8, b00, b01, b10, b11);
-        mma16816(oacc[db], a, b00, b01);
-        mma16816(oacc[db + 1], a, b10, b11);
-      }
-    }
-    __syncthreads();
+    mbar_init(o_ready, 1);
+    *abort_flag = 0;
+    mbar_fence_init();
   }
-  // finalize
-#pragma unroll
-  for (int r = 0; r < 2; ++r) {
-    l_r[r] += __shfl_xor_sync(0xffffffffu, l_r[r], 1);
-    l_r[r] += __shfl_xor_sync(0xffffffffu, l_r[r], 2);
+  if (warp == MMA_WARP) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
   }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int row0 = b * s.S;  // first row of this sequence in the qkv buffer
+
+  if (warp == TMA_WARP) {
+    if (lane == 0) {
+      constexpr uint32_t TB = C::TILE_BYTES;
+      mbar_arrive_expect_tx(q_full, TB);
 #pragma unroll
-  for (int r = 0; r < 2; ++r) {
-    const int qi = qrow0 + r * 8;
-    if (qi >= s.S) continue;
-    const float inv = 1.f / l_r[r];
-    uint16_t* orow = out + (row_base + qi) * static_cast<long long>(s.hq * D) + h * D;
+      for (int c = 0; c < D / 64; ++c)
+        tma_load_2d(base + C::Q_OFF + c * 16384, &tmap, h * D + c * 64, row0 + qt * TQ, q_full);
+      int jj = 0;
+      for (int j = 0; j < ntk; ++j) {
+        if (!kv_needed(s, qt, j)) continue;
+        const int st = jj & 1;
+        mbar_wait_bounded(&kv_empty[st], ((jj >> 1) & 1) ^ 1u, abort_flag, err);
+        mbar_arrive_expect_tx(&kv_full[st], 2 * TB);
 #pragma unroll
-    for (int db = 0; db < D / 8; ++db) {
-      const int col = db * 8 + (lane & 3) * 2;
-      *reinterpret_cast<uint32_t*>(orow + col) = pack_bf16x2(oacc[db][2 * r] * inv, oacc[db][2 * r + 1] * inv);
+        for (int c = 0; c < D / 64; ++c) {
+          tma_load_2d(base + C::K_OFF + st * TB + c * 16384, &tmap, (s.hq + g) * D + c * 64, row0 + j * TK,
+                      &kv_full[st]);
+          tma_load_2d(base + C::V_OFF + st * TB + c * 16384, &tmap, (s.hq + s.hkv + g) * D + c * 64, row0 + j * TK,
+                      &kv_full[st]);
+        }
+        ++jj;
+      }
     }
-    if ((lane & 3) == 0)
-      lse[(static_cast<long long>(b) * s.hq + h) * s.S + qi] = (m_r[r] + log2f(l_r[r])) / LOG2E;
+  } else if (warp == MMA_WARP) {
+    if (lane == 0) {
+      const uint32_t sq = smem_u32(base + C::Q_OFF);
+      const uint32_t idesc_qk = idesc_bf16(TQ, TK, false, false);  // S[q, k] = sum_d Q[q, d] K[k, d]
+      const uint32_t idesc_pv = idesc_bf16(TQ, D, false, true);    // O[q, d] += sum_k P[q, k] V[k, d]
+      mbar_wait_bounded(q_full, 0, abort_flag, err);
+      auto issue_pv = [&](int i) {
+        const int st = i & 1, sb = i % N_SBUF;
+        mbar_wait_bounded(&p_full[sb], (i / N_SBUF) & 1, abort_flag, err);
+        tc_fence_after();
+        const uint32_t sv = smem_u32(base + C::V_OFF + st * C::TILE_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < TK / 16; ++kk) {
+          const uint64_t bd = sw128_mnmajor_desc(sv + kk * 2048, TK * 128);
+          tc_mma_f16_ts(tmem + C::O_COL, tmem + sb * TK + kk * 8, bd, idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc_commit(&kv_empty[st]);
+        tc_commit(o_ready);
+      };
+      int jj = 0;
+      for (int j = 0; j < ntk; ++j) {
+        if (!kv_needed(s, qt, j)) continue;
+        const int st = jj & 1, sb = jj % N_SBUF;
+        mbar_wait_bounded(&kv_full[st], (jj >> 1) & 1, abort_flag, err);
+        tc_fence_after();
+        const uint32_t sk = smem_u32(base + C::K_OFF + st * C::TILE_BYTES);
+#pragma unroll
+        for (int kc = 0; kc < D / 16; ++kc) {
+          const uint32_t off = (kc >> 2) * 16384 + (kc & 3) * 32;
+          tc_mma_f16(tmem + sb * TK, sw128_kmajor_desc(sq + off), sw128_kmajor_desc(sk + off), idesc_qk,
+                     kc > 0 ? 1u : 0u);
+        }
+        tc_commit(&s_full[sb]);
+        if (jj > 0) issue_pv(jj - 1);
+        ++jj;
+      }
+      if (jj > 0) issue_pv(jj - 1);
+    }
+  } else {
+    // ------------------------------------------------------ softmax: thread = query row
+    const int r = warp * 32 + lane;
+    const int q = qt * TQ + r;  // row within the sequence
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const float scale_log2 = LOG2E_F / sqrtf(static_cast<float>(D));
+    float m = -INFINITY, l = 0.f;
+    int jj = 0;
+    for (int j = 0; j < ntk; ++j) {
+      if (!kv_needed(s, qt, j)) continue;
+      const int sb = jj % N_SBUF;
+      mbar_wait_bounded(&s_full[sb], (jj / N_SBUF) & 1, abort_flag, err);
+      tc_fence_after();
+      const bool need_mask = s.pl > 0 || j == qt || (j + 1) * TK > s.S;
+      float x[TK];
+      float mx = m;
+#pragma unroll
+      for (int c = 0; c < TK / 32; ++c) {
+        uint32_t raw[32];
+        tmem_ld32(tmem + lane_base + sb * TK + c * 32, raw);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          float v = __uint_as_float(raw[e]) * scale_log2;
+          if (need_mask) {
+            const int k = j * TK + c * 32 + e;
+            if (k >= s.S || !visible(s, q, k)) v = -INFINITY;
+          }
+          x[c * 32 + e] = v;
+          mx = fmaxf(mx, v);
+        }
+      }
+      const bool live = mx != -INFINITY;  // some key of this row visible so far
+      const float alpha = live ? exp2f(m - mx) : 1.f;
+      // P_jj over the first half of the S buffer's columns (two bf16 per column); PV_{jj-1}
+      // reads another buffer, so this may run before it has finished
+      float sum = 0.f;
+#pragma unroll
+      for (int c = 0; c < TK / 32; ++c) {
+        uint32_t pw[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const float p0 = live ? exp2f(x[c * 32 + e] - mx) : 0.f;
+          const float p1 = live ? exp2f(x[c * 32 + e + 1] - mx) : 0.f;
+          sum += p0 + p1;
+          pw[e >> 1] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(tmem + lane_base + sb * TK + c * 16, pw);
+      }
+      l = l * alpha + sum;
+      m = mx;
+      if (jj > 0) {
+        // PV_{jj-1} has finished accumulating into O: rescale it where this row's max grew
+        mbar_wait_bounded(o_ready, (jj - 1) & 1, abort_flag, err);
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+          for (int c = 0; c < D / 16; ++c) {
+            uint32_t o[16];
+            tmem_ld16(tmem + lane_base + C::O_COL + c * 16, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st16(tmem + lane_base + C::O_COL + c * 16, o);
+          }
+        }
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[sb]);
+      ++jj;
+    }
+    // epilogue: O / l in bf16, natural-log LSE
+    if (jj > 0) mbar_wait_bounded(o_ready, (jj - 1) & 1, abort_flag, err);
+    tc_fence_after();
+    const float inv = (l > 0.f) ? 1.f / l : 0.f;
+    uint16_t* orow = out + (static_cast<long long>(row0) + q) * static_cast<long long>(s.hq * D) + h * D;
+#pragma unroll
+    for (int c = 0; c < D / 16; ++c) {
+      uint32_t o[16];
+      tmem_ld16(tmem + lane_base + C::O_COL + c * 16, o);
+      tmem_ld_wait();
+      if (q < s.S) {
+        uint4 w0, w1;
+        w0.x = pack_bf16x2(__uint_as_float(o[0]) * inv, __uint_as_float(o[1]) * inv);
+        w0.y = pack_bf16x2(__uint_as_float(o[2]) * inv, __uint_as_float(o[3]) * inv);
+        w0.z = pack_bf16x2(__uint_as_float(o[4]) * inv, __uint_as_float(o[5]) * inv);
+        w0.w = pack_bf16x2(__uint_as_float(o[6]) * inv, __uint_as_float(o[7]) * inv);
+        w1.x = pack_bf16x2(__uint_as_float(o[8]) * inv, __uint_as_float(o[9]) * inv);
+        w1.y = pack_bf16x2(__uint_as_float(o[10]) * inv, __uint_as_float(o[11]) * inv);
+        w1.z = pack_bf16x2(__uint_as_float(o[12]) * inv, __uint_as_float(o[13]) * inv);
+        w1.w = pack_bf16x2(__uint_as_float(o[14]) * inv, __uint_as_float(o[15]) * inv);
+        *reinterpret_cast<uint4*>(orow + c * 16) = w0;
+        *reinterpret_cast<uint4*>(orow + c * 16 + 8) = w1;
+      }
+    }
+    if (q < s.S) lse[(static_cast<long long>(b) * s.hq + h) * s.S + q] = (m + log2f(l)) / LOG2E_F;
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == MMA_WARP) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
   }
 }
+
+template <int D>
+cudaError_t launch_fwd(const AttnShape& s, const uint16_t* qkv, uint16_t* o, float* lse, int* err, cudaStream_t st) {
+  using C = FwdCfg<D>;
+  CUtensorMap map;
+  const unsigned long long cols = static_cast<unsigned long long>(s.hq + 2 * s.hkv) * D;
+  const unsigned long long rows = static_cast<unsigned long long>(s.B) * s.S;
+  if (!tma_encode_bf16_sw128(&map, qkv, cols, rows, static_cast<unsigned long long>(s.ld_qkv) * 2, 64, TQ))
+    return cudaErrorInvalidValue;
+  static bool attr = false;
+  if (!attr) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(attn_fwd_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  const dim3 grid((s.S + TQ - 1) / TQ, s.hq, s.B);
+  attn_fwd_tc_kernel<D><<<grid, FWD_THREADS, C::SMEM_BYTES, st>>>(map, s, o, lse, err);
+  return cudaGetLastError();
+}
+
 
 // ---------------------------------------------------------------- delta = rowsum(dO * O)
 __global__ void attn_delta_kernel(const uint16_t* __restrict__ o, const uint16_t* __restrict__ dout, int T, int hq,
@@ -275,191 +310,6 @@ __global__ void attn_delta_kernel(const uint16_t* __restrict__ o, const uint16_t
   }
   acc = warp_sum(acc);
   if (lane == 0) delta[t * hq + h] = acc;  // [T, hq]
-}
-
-// ---------------------------------------------------------------- backward pass 1: dK, dV
-// One CTA per (kv tile, kv head, head slice): it loops over the query heads of its slice of
-// the group and over the causal query tiles, with the next (head, query tile) pair's Q / dO
-// tiles loaded while the current one computes.  hsplit = 1: dK / dV go straight to dqkv.
-// hsplit > 1 (too few kv tiles x kv heads to fill the GPU): each slice writes fp32 partial
-// dK (scaled) / dV to part[slice][row][kv head][2D] and attn_dkdv_sum_kernel adds the slices
-// in slice order.
-template <int D>
-__global__ void __launch_bounds__(AT_THREADS) attn_bwd_dkdv_kernel(const AttnShape s, const uint16_t* __restrict__ qkv,
-                                                                    const uint16_t* __restrict__ dout,
-                                                                    const float* __restrict__ lse,
-                                                                    const float* __restrict__ delta,
-                                                                    uint16_t* __restrict__ dqkv, int hsplit,
-                                                                    float* __restrict__ part) {
-  extern __shared__ __align__(16) uint16_t sm[];
-  using C = AttnCfg<D>;
-  uint16_t* Ks = sm;
-  uint16_t* Vs = sm + C::TILE;
-  uint16_t* Qb = sm + 2 * C::TILE;   // 2 buffers
-  uint16_t* dOb = sm + 4 * C::TILE;  // 2 buffers
-  float* lse_b = reinterpret_cast<float*>(sm + 6 * C::TILE);  // 2 x AT_BR
-  float* del_b = lse_b + 2 * AT_BR;                            // 2 x AT_BR
-  const int kt = blockIdx.x, b = blockIdx.z;
-  const int g = blockIdx.y / hsplit, slice = blockIdx.y % hsplit;
-  const int grp = s.hq / s.hkv;
-  const int hper = grp / hsplit;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long row_base = static_cast<long long>(b) * s.S;
-  const long long ldo = static_cast<long long>(s.hq) * D;
-  const float scale = 1.f / sqrtf(static_cast<float>(D));
-  const float scale_log2 = scale * LOG2E;
-  const int nqt = (s.S + AT_BR - 1) / AT_BR;
-  // query tiles that see this kv tile: kt.. to the end, but a chosen-response kv tile of a
-  // shared-prefix pair is seen by the chosen response only
-  const int q_end = (s.pl > 0 && kt * AT_BR >= s.pl && kt * AT_BR < s.pl + s.rl) ? (s.pl + s.rl) / AT_BR : nqt;
-  const int nq = q_end - kt;
-  const int n_it = hper * nq;      // (head, query tile) pairs
-
-  auto issue = [&](int it) {
-    const int h = g * grp + slice * hper + it / nq;
-    const int qt = kt + it % nq;
-    const int buf = it & 1;
-    load_tile_async<D>(Qb + buf * C::TILE, qkv + row_base * s.ld_qkv + h * D, s.ld_qkv, qt * AT_BR, s.S);
-    load_tile_async<D>(dOb + buf * C::TILE, dout + row_base * ldo + h * D, ldo, qt * AT_BR, s.S);
-    for (int i = threadIdx.x; i < AT_BR; i += AT_THREADS) {
-      const int qi = qt * AT_BR + i;
-      const bool ok = qi < s.S;
-      lse_b[buf * AT_BR + i] = ok ? lse[(static_cast<long long>(b) * s.hq + h) * s.S + qi] * LOG2E : 0.f;
-      del_b[buf * AT_BR + i] = ok ? delta[(row_base + qi) * s.hq + h] : 0.f;
-    }
-  };
-
-  load_tile_async<D>(Ks, qkv + row_base * s.ld_qkv + (s.hq + g) * D, s.ld_qkv, kt * AT_BR, s.S);
-  load_tile_async<D>(Vs, qkv + row_base * s.ld_qkv + (s.hq + s.hkv + g) * D, s.ld_qkv, kt * AT_BR, s.S);
-  issue(0);
-  cp_async_commit();
-
-  float dk[D / 8][4], dv[D / 8][4];
-#pragma unroll
-  for (int i = 0; i < D / 8; ++i) {
-    dk[i][0] = dk[i][1] = dk[i][2] = dk[i][3] = 0.f;
-    dv[i][0] = dv[i][1] = dv[i][2] = dv[i][3] = 0.f;
-  }
-  const int kvrow0 = kt * AT_BR + warp * 16 + (lane >> 2);
-
-  for (int it = 0; it < n_it; ++it) {
-    if (it + 1 < n_it) issue(it + 1);
-    cp_async_commit();
-    cp_async_wait<1>();
-    __syncthreads();
-    const int qt = kt + it % nq;
-    const uint16_t* Qs = Qb + (it & 1) * C::TILE;
-    const uint16_t* dOs = dOb + (it & 1) * C::TILE;
-    const float* lse_s = lse_b + (it & 1) * AT_BR;
-    const float* del_s = del_b + (it & 1) * AT_BR;
-    // S^T = K_w Q^T  (rows: kv, cols: q)
-    float st[8][4];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) st[i][0] = st[i][1] = st[i][2] = st[i][3] = 0.f;
-#pragma unroll
-    for (int kc = 0; kc < D / 16; ++kc) {
-      uint32_t a[4];
-      lda_frag<D>(Ks, warp * 16, kc * 16, a);
-#pragma unroll
-      for (int nb2 = 0; nb2 < 4; ++nb2) {
-        uint32_t b00, b01, b10, b11;
-        ldb_nk<D>(Qs, nb2 * 16, kc * 16, b00, b01, b10, b11);
-        mma16816(st[2 * nb2], a, b00, b01);
-        mma16816(st[2 * nb2 + 1], a, b10, b11);
-      }
-    }
-    // P^T
-#pragma unroll
-    for (int nb = 0; nb < 8; ++nb) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int qcol = nb * 8 + (lane & 3) * 2 + (e & 1);
-        const int qi = qt * AT_BR + qcol;
-        const int kv = kvrow0 + (e >> 1) * 8;
-        float p = exp2f(st[nb][e] * scale_log2 - lse_s[qcol]);
-        if (!visible(s, qi, kv) || qi >= s.S || kv >= s.S) p = 0.f;
-        st[nb][e] = p;
-      }
-    }
-    // dV += P^T dO
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const uint32_t a[4] = {pack_bf16x2(st[2 * c][0], st[2 * c][1]), pack_bf16x2(st[2 * c][2], st[2 * c][3]),
-                             pack_bf16x2(st[2 * c + 1][0], st[2 * c + 1][1]),
-                             pack_bf16x2(st[2 * c + 1][2], st[2 * c + 1][3])};
-#pragma unroll
-      for (int db = 0; db < D / 8; db += 2) {
-        uint32_t b00, b01, b10, b11;
-        ldb_kn<D>(dOs, c * 16, db * 8, b00, b01, b10, b11);
-        mma16816(dv[db], a, b00, b01);
-        mma16816(dv[db + 1], a, b10, b11);
-      }
-    }
-    // dP^T = V_w dO^T
-    float dp[8][4];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) dp[i][0] = dp[i][1] = dp[i][2] = dp[i][3] = 0.f;
-#pragma unroll
-    for (int kc = 0; kc < D / 16; ++kc) {
-      uint32_t a[4];
-      lda_frag<D>(Vs, warp * 16, kc * 16, a);
-#pragma unroll
-      for (int nb2 = 0; nb2 < 4; ++nb2) {
-        uint32_t b00, b01, b10, b11;
-        ldb_nk<D>(dOs, nb2 * 16, kc * 16, b00, b01, b10, b11);
-        mma16816(dp[2 * nb2], a, b00, b01);
-        mma16816(dp[2 * nb2 + 1], a, b10, b11);
-      }
-    }
-    // dS^T = P^T * (dP^T - delta), then dK += dS^T Q
-#pragma unroll
-    for (int nb = 0; nb < 8; ++nb) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int qcol = nb * 8 + (lane & 3) * 2 + (e & 1);
-        st[nb][e] = st[nb][e] * (dp[nb][e] - del_s[qcol]);
-      }
-    }
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const uint32_t a[4] = {pack_bf16x2(st[2 * c][0], st[2 * c][1]), pack_bf16x2(st[2 * c][2], st[2 * c][3]),
-                             pack_bf16x2(st[2 * c + 1][0], st[2 * c + 1][1]),
-                             pack_bf16x2(st[2 * c + 1][2], st[2 * c + 1][3])};
-#pragma unroll
-      for (int db = 0; db < D / 8; db += 2) {
-        uint32_t b00, b01, b10, b11;
-        ldb_kn<D>(Qs, c * 16, db * 8, b00, b01, b10, b11);
-        mma16816(dk[db], a, b00, b01);
-        mma16816(dk[db + 1], a, b10, b11);
-      }
-    }
-    __syncthreads();  // this buffer is refilled two iterations later
-  }
-  // store dK (scaled) and dV: into the k / v columns of dqkv, or as fp32 partials
-#pragma unroll
-  for (int r = 0; r < 2; ++r) {
-    const int kv = kvrow0 + r * 8;
-    if (kv >= s.S) continue;
-    if (hsplit == 1) {
-      uint16_t* krow = dqkv + (row_base + kv) * s.ld_qkv + (s.hq + g) * D;
-      uint16_t* vrow = dqkv + (row_base + kv) * s.ld_qkv + (s.hq + s.hkv + g) * D;
-#pragma unroll
-      for (int db = 0; db < D / 8; ++db) {
-        const int col = db * 8 + (lane & 3) * 2;
-        *reinterpret_cast<uint32_t*>(krow + col) = pack_bf16x2(dk[db][2 * r] * scale, dk[db][2 * r + 1] * scale);
-        *reinterpret_cast<uint32_t*>(vrow + col) = pack_bf16x2(dv[db][2 * r], dv[db][2 * r + 1]);
-      }
-    } else {
-      const long long T = static_cast<long long>(s.B) * s.S;
-      float* prow = part + ((static_cast<long long>(slice) * T + row_base + kv) * s.hkv + g) * (2 * D);
-#pragma unroll
-      for (int db = 0; db < D / 8; ++db) {
-        const int col = db * 8 + (lane & 3) * 2;
-        *reinterpret_cast<float2*>(prow + col) = make_float2(dk[db][2 * r] * scale, dk[db][2 * r + 1] * scale);
-        *reinterpret_cast<float2*>(prow + D + col) = make_float2(dv[db][2 * r], dv[db][2 * r + 1]);
-      }
-    }
-  }
 }
 
 // Sum of the head-slice partials in slice order -> bf16 dK / dV columns of dqkv.  One thread
@@ -486,155 +336,456 @@ __global__ void attn_dkdv_sum_kernel(const AttnShape s, int hsplit, const float*
   *o = make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
 }
 
-// ---------------------------------------------------------------- backward pass 2: dQ
+// ---------------------------------------------------------------- backward
+// Two passes, no atomics (the result does not depend on timing), same arithmetic as the
+// forward: P = exp(S / sqrt(d) - lse), dP = dO V^T, dS = P * (dP - delta), delta = rowsum(dO * O).
+//   dK/dV pass, one CTA per (128-key tile, kv head, head slice); thread = key row:
+//     S^T = K Q_i^T and dP^T = V dO_i^T (tcgen05, K-major operands), P^T and dS^T back into TMEM
+//     as bf16 over the first half of their columns, then dV += P^T dO_i and dK += dS^T Q_i with
+//     P^T / dS^T the A operands from TMEM and dO_i / Q_i read MN-major from the same shared tiles;
+//     over the causal query tiles i of every query head of the slice.  One slice writes dK, dV
+//     (bf16); several write fp32 partials that attn_dkdv_sum_kernel adds in slice order.
+//   dQ pass, one CTA per (128-query tile, head); thread = query row:
+//     S = Q K_j^T, dP = dO V_j^T, dS into TMEM, dQ += dS K_j (K_j read MN-major).
+// The MMAs that overwrite S / dP wait until the previous iteration's MMAs reading P / dS from
+// those columns have completed.
 template <int D>
-__global__ void __launch_bounds__(AT_THREADS) attn_bwd_dq_kernel(const AttnShape s, const uint16_t* __restrict__ qkv,
-                                                                  const uint16_t* __restrict__ dout,
-                                                                  const float* __restrict__ lse,
-                                                                  const float* __restrict__ delta,
-                                                                  uint16_t* __restrict__ dqkv) {
-  extern __shared__ __align__(16) uint16_t sm[];
-  using C = AttnCfg<D>;
-  uint16_t* Qs = sm;
-  uint16_t* dOs = sm + C::TILE;
-  uint16_t* Ks = sm + 2 * C::TILE;  // 2 buffers
-  uint16_t* Vs = sm + 4 * C::TILE;  // 2 buffers
+struct BwdCfg {
+  static constexpr int TILE_BYTES = 128 * D * 2;
+  static constexpr int VEC_OFF = 6 * TILE_BYTES;  // two float[128] vectors (dK/dV pass)
+  static constexpr int BAR_OFF = VEC_OFF + 1024;
+  static constexpr int SMEM_BYTES = 1024 + BAR_OFF + 256;
+  static constexpr int S_COL = 0, DP_COL = 128, ACC0 = 256, ACC1 = 256 + D;
+  static constexpr int TMEM_COLS = 512;
+  static_assert(ACC1 + D <= TMEM_COLS, "TMEM budget");
+};
+
+// K-major tile descriptors: 16-deep step kc of a [128 x D] tile (D/64 atoms of 16 KB)
+__device__ __forceinline__ uint64_t kdesc(uint32_t tile, int kc) {
+  return sw128_kmajor_desc(tile + (kc >> 2) * 16384 + (kc & 3) * 32);
+}
+// MN-major view of the same tile: rows are the reduction index, 16 rows per step
+__device__ __forceinline__ uint64_t mndesc(uint32_t tile, int kk) { return sw128_mnmajor_desc(tile + kk * 2048, 128 * 128); }
+
+template <int D>
+__global__ void __launch_bounds__(FWD_THREADS, 1)
+    attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tdo,
+                            const AttnShape s, const float* __restrict__ lse, const float* __restrict__ delta,
+                            uint16_t* __restrict__ dqkv, int hsplit, float* __restrict__ part, int* err) {
+  using C = BwdCfg<D>;
+  constexpr int TB = C::TILE_BYTES;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* base = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+  uint8_t* Ks = base;
+  uint8_t* Vs = base + TB;
+  uint8_t* Qs = base + 2 * TB;   // 2 stages
+  uint8_t* dOs = base + 4 * TB;  // 2 stages
+  float* lsm = reinterpret_cast<float*>(base + C::VEC_OFF);
+  float* dsm = lsm + 128;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + C::BAR_OFF);
+  uint64_t* kv_full = bars;       // 1
+  uint64_t* qd_full = bars + 1;   // 2
+  uint64_t* qd_empty = bars + 3;  // 2
+  uint64_t* s_full = bars + 5;    // 1
+  uint64_t* p_full = bars + 6;    // 1
+  uint64_t* mma_done = bars + 7;  // 1
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 9);
+
+  const int j = blockIdx.x, b = blockIdx.z;
+  const int g = blockIdx.y / hsplit, slice = blockIdx.y % hsplit;
+  const int grp = s.hq / s.hkv, hper = grp / hsplit, h0 = g * grp + slice * hper;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nqt = (s.S + TQ - 1) / TQ;
+  const int row0 = b * s.S;
+  const float scale = 1.f / sqrtf(static_cast<float>(D));
+  const float scale_log2 = scale * LOG2E_F;
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&qd_full[i], 1);
+      mbar_init(&qd_empty[i], 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(p_full, SOFTMAX_WARPS);
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == MMA_WARP) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  // iterations: (head hh of the slice, query tile i that sees key tile j), heads outer
+  auto q_seen = [&](int i) { return block_visible(s, i * TQ, i * TQ + TQ, j * TK, j * TK + TK); };
+
+  if (warp == TMA_WARP) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(kv_full, 2 * TB);
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c) {
+        tma_load_2d(Ks + c * 16384, &tq, (s.hq + g) * D + c * 64, row0 + j * TK, kv_full);
+        tma_load_2d(Vs + c * 16384, &tq, (s.hq + s.hkv + g) * D + c * 64, row0 + j * TK, kv_full);
+      }
+      int it = 0;
+      for (int hh = 0; hh < hper; ++hh)
+        for (int i = 0; i < nqt; ++i) {
+          if (!q_seen(i)) continue;
+          const int h = h0 + hh, st = it & 1;
+          mbar_wait_bounded(&qd_empty[st], ((it >> 1) & 1) ^ 1u, abort_flag, err);
+          mbar_arrive_expect_tx(&qd_full[st], 2 * TB);
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c) {
+            tma_load_2d(Qs + st * TB + c * 16384, &tq, h * D + c * 64, row0 + i * TQ, &qd_full[st]);
+            tma_load_2d(dOs + st * TB + c * 16384, &tdo, h * D + c * 64, row0 + i * TQ, &qd_full[st]);
+          }
+          ++it;
+        }
+    }
+  } else if (warp == MMA_WARP) {
+    if (lane == 0) {
+      const uint32_t idesc_s = idesc_bf16(TK, TQ, false, false);  // [key, query], K = d
+      const uint32_t idesc_a = idesc_bf16(TK, D, false, true);    // [key, d], K = queries
+      const uint32_t sk = smem_u32(Ks), sv = smem_u32(Vs);
+      mbar_wait_bounded(kv_full, 0, abort_flag, err);
+      int it = 0;
+      for (int hh = 0; hh < hper; ++hh)
+        for (int i = 0; i < nqt; ++i) {
+          if (!q_seen(i)) continue;
+          const int st = it & 1;
+          const uint32_t sq = smem_u32(Qs + st * TB), sd = smem_u32(dOs + st * TB);
+          mbar_wait_bounded(&qd_full[st], (it >> 1) & 1, abort_flag, err);
+          if (it > 0) mbar_wait_bounded(mma_done, (it - 1) & 1, abort_flag, err);
+          tc_fence_after();
+#pragma unroll
+          for (int kc = 0; kc < D / 16; ++kc) tc_mma_f16(tmem + C::S_COL, kdesc(sk, kc), kdesc(sq, kc), idesc_s, kc > 0);
+#pragma unroll
+          for (int kc = 0; kc < D / 16; ++kc) tc_mma_f16(tmem + C::DP_COL, kdesc(sv, kc), kdesc(sd, kc), idesc_s, kc > 0);
+          tc_commit(s_full);
+          mbar_wait_bounded(p_full, it & 1, abort_flag, err);
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < TQ / 16; ++kk)
+            tc_mma_f16_ts(tmem + C::ACC0, tmem + C::S_COL + kk * 8, mndesc(sd, kk), idesc_a, (it > 0 || kk > 0));
+#pragma unroll
+          for (int kk = 0; kk < TQ / 16; ++kk)
+            tc_mma_f16_ts(tmem + C::ACC1, tmem + C::DP_COL + kk * 8, mndesc(sq, kk), idesc_a, (it > 0 || kk > 0));
+          tc_commit(&qd_empty[st]);
+          tc_commit(mma_done);
+          ++it;
+        }
+    }
+  } else {
+    // ------------------------------------------------------ thread = key row
+    const int r = warp * 32 + lane;
+    const int k = j * TK + r;
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    int it = 0;
+    for (int hh = 0; hh < hper; ++hh)
+      for (int i = 0; i < nqt; ++i) {
+        if (!q_seen(i)) continue;
+        const int h = h0 + hh;
+        // the query tile's lse (log2 units) and delta, staged for every key row
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        {
+          const int q = i * TQ + r;
+          lsm[r] = q < s.S ? lse[(static_cast<long long>(b) * s.hq + h) * s.S + q] * LOG2E_F : 0.f;
+          dsm[r] = q < s.S ? delta[(static_cast<long long>(row0) + q) * s.hq + h] : 0.f;
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        mbar_wait_bounded(s_full, it & 1, abort_flag, err);
+        tc_fence_after();
+        const bool need_mask = s.pl > 0 || i == j || (i + 1) * TQ > s.S;
+#pragma unroll
+        for (int c = 0; c < TQ / 32; ++c) {
+          uint32_t sr[32], dr[32];
+          tmem_ld32(tmem + lane_base + C::S_COL + c * 32, sr);
+          tmem_ld32(tmem + lane_base + C::DP_COL + c * 32, dr);
+          tmem_ld_wait();
+          uint32_t pw[16], dw[16];
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            float pv[2], dv[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const int qc = c * 32 + e + u;
+              float p = exp2f(__uint_as_float(sr[e + u]) * scale_log2 - lsm[qc]);
+              if (need_mask) {
+                const int q = i * TQ + qc;
+                if (q >= s.S || !visible(s, q, k)) p = 0.f;
+              }
+              pv[u] = p;
+              dv[u] = p * (__uint_as_float(dr[e + u]) - dsm[qc]);
+            }
+            pw[e >> 1] = pack_bf16x2(pv[0], pv[1]);
+            dw[e >> 1] = pack_bf16x2(dv[0], dv[1]);
+          }
+          tmem_st16(tmem + lane_base + C::S_COL + c * 16, pw);
+          tmem_st16(tmem + lane_base + C::DP_COL + c * 16, dw);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full);
+        ++it;
+      }
+    if (it > 0) mbar_wait_bounded(mma_done, (it - 1) & 1, abort_flag, err);
+    tc_fence_after();
+    // epilogue: dK = scale * (dS^T Q), dV = P^T dO for this key row
+    const long long T = static_cast<long long>(s.B) * s.S;
+#pragma unroll
+    for (int c = 0; c < D / 16; ++c) {
+      uint32_t a[16], v[16];
+      tmem_ld16(tmem + lane_base + C::ACC1 + c * 16, a);  // dK
+      tmem_ld16(tmem + lane_base + C::ACC0 + c * 16, v);  // dV
+      tmem_ld_wait();
+      if (k >= s.S) continue;
+      float fk[16], fv[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        fk[e] = it > 0 ? __uint_as_float(a[e]) * scale : 0.f;
+        fv[e] = it > 0 ? __uint_as_float(v[e]) : 0.f;
+      }
+      if (hsplit == 1) {
+        uint16_t* dk = dqkv + (static_cast<long long>(row0) + k) * s.ld_qkv + (s.hq + g) * D + c * 16;
+        uint16_t* dvp = dqkv + (static_cast<long long>(row0) + k) * s.ld_qkv + (s.hq + s.hkv + g) * D + c * 16;
+        uint4 w[4];
+        w[0] = make_uint4(pack_bf16x2(fk[0], fk[1]), pack_bf16x2(fk[2], fk[3]), pack_bf16x2(fk[4], fk[5]),
+                          pack_bf16x2(fk[6], fk[7]));
+        w[1] = make_uint4(pack_bf16x2(fk[8], fk[9]), pack_bf16x2(fk[10], fk[11]), pack_bf16x2(fk[12], fk[13]),
+                          pack_bf16x2(fk[14], fk[15]));
+        w[2] = make_uint4(pack_bf16x2(fv[0], fv[1]), pack_bf16x2(fv[2], fv[3]), pack_bf16x2(fv[4], fv[5]),
+                          pack_bf16x2(fv[6], fv[7]));
+        w[3] = make_uint4(pack_bf16x2(fv[8], fv[9]), pack_bf16x2(fv[10], fv[11]), pack_bf16x2(fv[12], fv[13]),
+                          pack_bf16x2(fv[14], fv[15]));
+        reinterpret_cast<uint4*>(dk)[0] = w[0];
+        reinterpret_cast<uint4*>(dk)[1] = w[1];
+        reinterpret_cast<uint4*>(dvp)[0] = w[2];
+        reinterpret_cast<uint4*>(dvp)[1] = w[3];
+      } else {
+        const int per_row = s.hkv * 2 * D;
+        float* pr = part + (static_cast<long long>(slice) * T + row0 + k) * per_row + g * 2 * D;
+#pragma unroll
+        for (int e = 0; e < 16; e += 4) {
+          *reinterpret_cast<float4*>(pr + c * 16 + e) = make_float4(fk[e], fk[e + 1], fk[e + 2], fk[e + 3]);
+          *reinterpret_cast<float4*>(pr + D + c * 16 + e) = make_float4(fv[e], fv[e + 1], fv[e + 2], fv[e + 3]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == MMA_WARP) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(FWD_THREADS, 1)
+    attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tdo,
+                          const AttnShape s, const float* __restrict__ lse, const float* __restrict__ delta,
+                          uint16_t* __restrict__ dqkv, int* err) {
+  using C = BwdCfg<D>;
+  constexpr int TB = C::TILE_BYTES;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* base = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+  uint8_t* Qs = base;
+  uint8_t* dOs = base + TB;
+  uint8_t* Ks = base + 2 * TB;  // 2 stages
+  uint8_t* Vs = base + 4 * TB;  // 2 stages
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + C::BAR_OFF);
+  uint64_t* q_full = bars;        // 1
+  uint64_t* kv_full = bars + 1;   // 2
+  uint64_t* kv_empty = bars + 3;  // 2
+  uint64_t* s_full = bars + 5;    // 1
+  uint64_t* p_full = bars + 6;    // 1
+  uint64_t* mma_done = bars + 7;  // 1
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 9);
+
   const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int g = h / (s.hq / s.hkv);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long row_base = static_cast<long long>(b) * s.S;
-  const long long ldo = static_cast<long long>(s.hq) * D;
+  const int ntk = (s.S + TK - 1) / TK;
+  const int row0 = b * s.S;
   const float scale = 1.f / sqrtf(static_cast<float>(D));
-  const float scale_log2 = scale * LOG2E;
-  const uint16_t* ksrc = qkv + row_base * s.ld_qkv + (s.hq + g) * D;
-  const uint16_t* vsrc = qkv + row_base * s.ld_qkv + (s.hq + s.hkv + g) * D;
+  const float scale_log2 = scale * LOG2E_F;
 
-  const KvRange kr = kv_range(s, qt);
-  load_tile_async<D>(Qs, qkv + row_base * s.ld_qkv + h * D, s.ld_qkv, qt * AT_BR, s.S);
-  load_tile_async<D>(dOs, dout + row_base * ldo + h * D, ldo, qt * AT_BR, s.S);
-  load_tile_async<D>(Ks, ksrc, s.ld_qkv, kv_tile(kr, 0) * AT_BR, s.S);
-  load_tile_async<D>(Vs, vsrc, s.ld_qkv, kv_tile(kr, 0) * AT_BR, s.S);
-  cp_async_commit();
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(p_full, SOFTMAX_WARPS);
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == MMA_WARP) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
 
-  const int qrow0 = qt * AT_BR + warp * 16 + (lane >> 2);
-  float lse_r[2], del_r[2];
+  if (warp == TMA_WARP) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(q_full, 2 * TB);
 #pragma unroll
-  for (int r = 0; r < 2; ++r) {
-    const int qi = qrow0 + r * 8;
-    const bool ok = qi < s.S;
-    lse_r[r] = ok ? lse[(static_cast<long long>(b) * s.hq + h) * s.S + qi] * LOG2E : 0.f;
-    del_r[r] = ok ? delta[(row_base + qi) * s.hq + h] : 0.f;
+      for (int c = 0; c < D / 64; ++c) {
+        tma_load_2d(Qs + c * 16384, &tq, h * D + c * 64, row0 + qt * TQ, q_full);
+        tma_load_2d(dOs + c * 16384, &tdo, h * D + c * 64, row0 + qt * TQ, q_full);
+      }
+      int jj = 0;
+      for (int j = 0; j < ntk; ++j) {
+        if (!kv_needed(s, qt, j)) continue;
+        const int st = jj & 1;
+        mbar_wait_bounded(&kv_empty[st], ((jj >> 1) & 1) ^ 1u, abort_flag, err);
+        mbar_arrive_expect_tx(&kv_full[st], 2 * TB);
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c) {
+          tma_load_2d(Ks + st * TB + c * 16384, &tq, (s.hq + g) * D + c * 64, row0 + j * TK, &kv_full[st]);
+          tma_load_2d(Vs + st * TB + c * 16384, &tq, (s.hq + s.hkv + g) * D + c * 64, row0 + j * TK, &kv_full[st]);
+        }
+        ++jj;
+      }
+    }
+  } else if (warp == MMA_WARP) {
+    if (lane == 0) {
+      const uint32_t idesc_s = idesc_bf16(TQ, TK, false, false);  // [query, key], K = d
+      const uint32_t idesc_q = idesc_bf16(TQ, D, false, true);    // [query, d], K = keys
+      const uint32_t sq = smem_u32(Qs), sd = smem_u32(dOs);
+      mbar_wait_bounded(q_full, 0, abort_flag, err);
+      int jj = 0;
+      for (int j = 0; j < ntk; ++j) {
+        if (!kv_needed(s, qt, j)) continue;
+        const int st = jj & 1;
+        const uint32_t sk = smem_u32(Ks + st * TB), sv = smem_u32(Vs + st * TB);
+        mbar_wait_bounded(&kv_full[st], (jj >> 1) & 1, abort_flag, err);
+        if (jj > 0) mbar_wait_bounded(mma_done, (jj - 1) & 1, abort_flag, err);
+        tc_fence_after();
+#pragma unroll
+        for (int kc = 0; kc < D / 16; ++kc) tc_mma_f16(tmem + C::S_COL, kdesc(sq, kc), kdesc(sk, kc), idesc_s, kc > 0);
+#pragma unroll
+        for (int kc = 0; kc < D / 16; ++kc) tc_mma_f16(tmem + C::DP_COL, kdesc(sd, kc), kdesc(sv, kc), idesc_s, kc > 0);
+        tc_commit(s_full);
+        mbar_wait_bounded(p_full, jj & 1, abort_flag, err);
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < TK / 16; ++kk)
+          tc_mma_f16_ts(tmem + C::ACC0, tmem + C::S_COL + kk * 8, mndesc(sk, kk), idesc_q, (jj > 0 || kk > 0));
+        tc_commit(&kv_empty[st]);
+        tc_commit(mma_done);
+        ++jj;
+      }
+    }
+  } else {
+    // ------------------------------------------------------ thread = query row
+    const int r = warp * 32 + lane;
+    const int q = qt * TQ + r;
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const float lse2 = q < s.S ? lse[(static_cast<long long>(b) * s.hq + h) * s.S + q] * LOG2E_F : 0.f;
+    const float dl = q < s.S ? delta[(static_cast<long long>(row0) + q) * s.hq + h] : 0.f;
+    int jj = 0;
+    for (int j = 0; j < ntk; ++j) {
+      if (!kv_needed(s, qt, j)) continue;
+      mbar_wait_bounded(s_full, jj & 1, abort_flag, err);
+      tc_fence_after();
+      const bool need_mask = s.pl > 0 || j == qt || (j + 1) * TK > s.S;
+#pragma unroll
+      for (int c = 0; c < TK / 32; ++c) {
+        uint32_t sr[32], dr[32];
+        tmem_ld32(tmem + lane_base + C::S_COL + c * 32, sr);
+        tmem_ld32(tmem + lane_base + C::DP_COL + c * 32, dr);
+        tmem_ld_wait();
+        uint32_t dw[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          float dv[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            float p = exp2f(__uint_as_float(sr[e + u]) * scale_log2 - lse2);
+            if (need_mask) {
+              const int k = j * TK + c * 32 + e + u;
+              if (k >= s.S || !visible(s, q, k)) p = 0.f;
+            }
+            dv[u] = p * (__uint_as_float(dr[e + u]) - dl);
+          }
+          dw[e >> 1] = pack_bf16x2(dv[0], dv[1]);
+        }
+        tmem_st16(tmem + lane_base + C::S_COL + c * 16, dw);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
+      ++jj;
+    }
+    if (jj > 0) mbar_wait_bounded(mma_done, (jj - 1) & 1, abort_flag, err);
+    tc_fence_after();
+    uint16_t* qrow = dqkv + (static_cast<long long>(row0) + q) * s.ld_qkv + h * D;
+#pragma unroll
+    for (int c = 0; c < D / 16; ++c) {
+      uint32_t a[16];
+      tmem_ld16(tmem + lane_base + C::ACC0 + c * 16, a);
+      tmem_ld_wait();
+      if (q >= s.S) continue;
+      float f[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) f[e] = jj > 0 ? __uint_as_float(a[e]) * scale : 0.f;
+      reinterpret_cast<uint4*>(qrow + c * 16)[0] = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
+                                                              pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
+      reinterpret_cast<uint4*>(qrow + c * 16)[1] = make_uint4(pack_bf16x2(f[8], f[9]), pack_bf16x2(f[10], f[11]),
+                                                              pack_bf16x2(f[12], f[13]), pack_bf16x2(f[14], f[15]));
+    }
   }
-  float dq[D / 8][4];
-#pragma unroll
-  for (int i = 0; i < D / 8; ++i) dq[i][0] = dq[i][1] = dq[i][2] = dq[i][3] = 0.f;
-  const int nkv = kr.n;
-  for (int j = 0; j < nkv; ++j) {
-    if (j + 1 < nkv) {
-      load_tile_async<D>(Ks + ((j + 1) & 1) * C::TILE, ksrc, s.ld_qkv, kv_tile(kr, j + 1) * AT_BR, s.S);
-      load_tile_async<D>(Vs + ((j + 1) & 1) * C::TILE, vsrc, s.ld_qkv, kv_tile(kr, j + 1) * AT_BR, s.S);
-    }
-    cp_async_commit();
-    cp_async_wait<1>();
-    __syncthreads();
-    const uint16_t* Kt = Ks + (j & 1) * C::TILE;
-    const uint16_t* Vt = Vs + (j & 1) * C::TILE;
-    const int kt = kv_tile(kr, j);
-    float sc[8][4], dp[8][4];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      sc[i][0] = sc[i][1] = sc[i][2] = sc[i][3] = 0.f;
-      dp[i][0] = dp[i][1] = dp[i][2] = dp[i][3] = 0.f;
-    }
-#pragma unroll
-    for (int kc = 0; kc < D / 16; ++kc) {
-      uint32_t a[4], ad[4];
-      lda_frag<D>(Qs, warp * 16, kc * 16, a);
-      lda_frag<D>(dOs, warp * 16, kc * 16, ad);
-#pragma unroll
-      for (int nb2 = 0; nb2 < 4; ++nb2) {
-        uint32_t b00, b01, b10, b11;
-        ldb_nk<D>(Kt, nb2 * 16, kc * 16, b00, b01, b10, b11);
-        mma16816(sc[2 * nb2], a, b00, b01);
-        mma16816(sc[2 * nb2 + 1], a, b10, b11);
-        ldb_nk<D>(Vt, nb2 * 16, kc * 16, b00, b01, b10, b11);
-        mma16816(dp[2 * nb2], ad, b00, b01);
-        mma16816(dp[2 * nb2 + 1], ad, b10, b11);
-      }
-    }
-#pragma unroll
-    for (int nb = 0; nb < 8; ++nb) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int kv = kt * AT_BR + nb * 8 + (lane & 3) * 2 + (e & 1);
-        const int qi = qrow0 + (e >> 1) * 8;
-        float p = exp2f(sc[nb][e] * scale_log2 - lse_r[e >> 1]);
-        if (!visible(s, qi, kv) || kv >= s.S || qi >= s.S) p = 0.f;
-        sc[nb][e] = p * (dp[nb][e] - del_r[e >> 1]);
-      }
-    }
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const uint32_t a[4] = {pack_bf16x2(sc[2 * c][0], sc[2 * c][1]), pack_bf16x2(sc[2 * c][2], sc[2 * c][3]),
-                             pack_bf16x2(sc[2 * c + 1][0], sc[2 * c + 1][1]),
-                             pack_bf16x2(sc[2 * c + 1][2], sc[2 * c + 1][3])};
-#pragma unroll
-      for (int db = 0; db < D / 8; db += 2) {
-        uint32_t b00, b01, b10, b11;
-        ldb_kn<D>(Kt, c * 16, db * 8, b00, b01, b10, b11);
-        mma16816(dq[db], a, b00, b01);
-        mma16816(dq[db + 1], a, b10, b11);
-      }
-    }
-    __syncthreads();
-  }
-#pragma unroll
-  for (int r = 0; r < 2; ++r) {
-    const int qi = qrow0 + r * 8;
-    if (qi >= s.S) continue;
-    uint16_t* qrow = dqkv + (row_base + qi) * s.ld_qkv + h * D;
-#pragma unroll
-    for (int db = 0; db < D / 8; ++db) {
-      const int col = db * 8 + (lane & 3) * 2;
-      *reinterpret_cast<uint32_t*>(qrow + col) = pack_bf16x2(dq[db][2 * r] * scale, dq[db][2 * r + 1] * scale);
-    }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == MMA_WARP) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
   }
 }
 
 template <int D>
-cudaError_t fwd_d(const AttnShape& s, const uint16_t* qkv, uint16_t* o, float* lse, cudaStream_t st) {
-  const int smem = 5 * AttnCfg<D>::TILE * 2;
+cudaError_t launch_bwd(const AttnShape& s, const uint16_t* qkv, const uint16_t* o, const uint16_t* dout,
+                       const float* lse, float* delta, uint16_t* dqkv, float* ws, size_t ws_bytes, int* err,
+                       cudaStream_t st) {
+  using C = BwdCfg<D>;
+  CUtensorMap tq, tdo;
+  const unsigned long long rows = static_cast<unsigned long long>(s.B) * s.S;
+  if (!tma_encode_bf16_sw128(&tq, qkv, static_cast<unsigned long long>(s.hq + 2 * s.hkv) * D, rows,
+                             static_cast<unsigned long long>(s.ld_qkv) * 2, 64, 128) ||
+      !tma_encode_bf16_sw128(&tdo, dout, static_cast<unsigned long long>(s.hq) * D, rows,
+                             static_cast<unsigned long long>(s.hq) * D * 2, 64, 128))
+    return cudaErrorInvalidValue;
   static bool attr = false;
   if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e =
+        cudaFuncSetAttribute(attn_bwd_dkdv_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    attr = true;
-  }
-  dim3 grid((s.S + AT_BR - 1) / AT_BR, s.hq, s.B);
-  attn_fwd_kernel<D><<<grid, AT_THREADS, smem, st>>>(s, qkv, o, lse);
-  ++g_kernel_launches;
-  return cudaGetLastError();
-}
-
-template <int D>
-cudaError_t bwd_d(const AttnShape& s, const uint16_t* qkv, const uint16_t* o, const uint16_t* dout, const float* lse,
-                  float* delta, uint16_t* dqkv, float* ws, size_t ws_bytes, cudaStream_t st) {
-  const int smem1 = 6 * AttnCfg<D>::TILE * 2 + 4 * AT_BR * 4;
-  const int smem2 = 6 * AttnCfg<D>::TILE * 2;
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(attn_bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem1);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(attn_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem2);
+    e = cudaFuncSetAttribute(attn_bwd_dq_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr = true;
   }
   const int T = s.B * s.S;
-  const long long warps = static_cast<long long>(T) * s.hq;
-  attn_delta_kernel<<<static_cast<unsigned>((warps * 32 + 255) / 256), 256, 0, st>>>(o, dout, T, s.hq, D, delta);
-  // head slices: the largest divisor of the group size that keeps the grid within two CTAs
-  // per SM and whose partials fit the workspace
-  const int nkt = (s.S + AT_BR - 1) / AT_BR;
+  cudaError_t e = attn_delta_launch(o, dout, T, s.hq, D, delta, st);
+  if (e != cudaSuccess) return e;
+  // head slices: the largest divisor of the group size that keeps the grid within two CTAs per
+  // SM and whose fp32 partials fit the workspace
+  const int nkt = (s.S + TK - 1) / TK;
   const long long base = static_cast<long long>(nkt) * s.hkv * s.B;
   const int grp = s.hq / s.hkv;
   const size_t per_slice = static_cast<size_t>(T) * s.hkv * 2 * D * sizeof(float);
@@ -644,42 +795,63 @@ cudaError_t bwd_d(const AttnShape& s, const uint16_t* qkv, const uint16_t* o, co
       hsplit = c;
       break;
     }
-  dim3 g1(nkt, s.hkv * hsplit, s.B);
-  attn_bwd_dkdv_kernel<D><<<g1, AT_THREADS, smem1, st>>>(s, qkv, dout, lse, delta, dqkv, hsplit, ws);
-  g_kernel_launches += 2;
+  attn_bwd_dkdv_tc_kernel<D><<<dim3(nkt, s.hkv * hsplit, s.B), FWD_THREADS, C::SMEM_BYTES, st>>>(
+      tq, tdo, s, lse, delta, dqkv, hsplit, ws, err);
+  g_kernel_launches += 1;
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
   if (hsplit > 1) {
-    const long long n4 = static_cast<long long>(T) * s.hkv * 2 * D / 4;
-    attn_dkdv_sum_kernel<<<static_cast<unsigned>((n4 + 255) / 256), 256, 0, st>>>(s, hsplit, ws, dqkv);
-    ++g_kernel_launches;
+    e = attn_dkdv_sum_launch(s, hsplit, ws, dqkv, st);
+    if (e != cudaSuccess) return e;
   }
-  dim3 g2(nkt, s.hq, s.B);
-  attn_bwd_dq_kernel<D><<<g2, AT_THREADS, smem2, st>>>(s, qkv, dout, lse, delta, dqkv);
+  attn_bwd_dq_tc_kernel<D><<<dim3((s.S + TQ - 1) / TQ, s.hq, s.B), FWD_THREADS, C::SMEM_BYTES, st>>>(tq, tdo, s, lse,
+                                                                                                   delta, dqkv, err);
   ++g_kernel_launches;
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t attn_fwd_launch(const AttnShape& s, const uint16_t* qkv, uint16_t* o, float* lse, cudaStream_t st) {
+cudaError_t attn_fwd_launch(const AttnShape& s, const uint16_t* qkv, uint16_t* o, float* lse, int* err,
+                               cudaStream_t st) {
   if (s.B <= 0 || s.S <= 0) return cudaSuccess;
-  if (s.hkv <= 0 || s.hq % s.hkv != 0 || s.ld_qkv % 8 != 0) return cudaErrorInvalidValue;
-  if (s.pl < 0 || (s.pl > 0 && (s.pl % AT_BR || s.rl <= 0 || s.rl % AT_BR || s.S != s.pl + 2 * s.rl)))
+  if (s.hq % s.hkv != 0 || (s.pl > 0 && (s.pl + 2 * s.rl != s.S))) return cudaErrorInvalidValue;
+  if (s.ld_qkv % 8 != 0) return cudaErrorInvalidValue;
+  cudaError_t e;
+  if (s.d == 128)
+    e = launch_fwd<128>(s, qkv, o, lse, err, st);
+  else if (s.d == 64)
+    e = launch_fwd<64>(s, qkv, o, lse, err, st);
+  else
     return cudaErrorInvalidValue;
-  if (s.d == 128) return fwd_d<128>(s, qkv, o, lse, st);
-  if (s.d == 64) return fwd_d<64>(s, qkv, o, lse, st);
-  return cudaErrorInvalidValue;
+  ++g_kernel_launches;
+  return e;
 }
 
 cudaError_t attn_bwd_launch(const AttnShape& s, const uint16_t* qkv, const uint16_t* o, const uint16_t* dout,
-                            const float* lse, float* delta, uint16_t* dqkv, float* ws, size_t ws_bytes,
-                            cudaStream_t st) {
+                               const float* lse, float* delta, uint16_t* dqkv, float* ws, size_t ws_bytes, int* err,
+                               cudaStream_t st) {
   if (s.B <= 0 || s.S <= 0) return cudaSuccess;
-  if (s.hkv <= 0 || s.hq % s.hkv != 0 || s.ld_qkv % 8 != 0) return cudaErrorInvalidValue;
-  if (s.pl < 0 || (s.pl > 0 && (s.pl % AT_BR || s.rl <= 0 || s.rl % AT_BR || s.S != s.pl + 2 * s.rl)))
-    return cudaErrorInvalidValue;
-  if (s.d == 128) return bwd_d<128>(s, qkv, o, dout, lse, delta, dqkv, ws, ws_bytes, st);
-  if (s.d == 64) return bwd_d<64>(s, qkv, o, dout, lse, delta, dqkv, ws, ws_bytes, st);
+  if (s.hkv <= 0 || s.hq % s.hkv != 0 || (s.pl > 0 && (s.pl + 2 * s.rl != s.S))) return cudaErrorInvalidValue;
+  if (s.ld_qkv % 8 != 0 || (ws && (reinterpret_cast<uintptr_t>(ws) & 15u))) return cudaErrorInvalidValue;
+  if (s.d == 128) return launch_bwd<128>(s, qkv, o, dout, lse, delta, dqkv, ws, ws_bytes, err, st);
+  if (s.d == 64) return launch_bwd<64>(s, qkv, o, dout, lse, delta, dqkv, ws, ws_bytes, err, st);
   return cudaErrorInvalidValue;
+}
+
+cudaError_t attn_delta_launch(const uint16_t* o, const uint16_t* dout, int T, int hq, int d, float* delta,
+                              cudaStream_t st) {
+  const long long warps = static_cast<long long>(T) * hq;
+  attn_delta_kernel<<<static_cast<unsigned>((warps * 32 + 255) / 256), 256, 0, st>>>(o, dout, T, hq, d, delta);
+  ++g_kernel_launches;
+  return cudaGetLastError();
+}
+
+cudaError_t attn_dkdv_sum_launch(const AttnShape& s, int hsplit, const float* part, uint16_t* dqkv, cudaStream_t st) {
+  const long long n4 = static_cast<long long>(s.B) * s.S * s.hkv * 2 * s.d / 4;
+  attn_dkdv_sum_kernel<<<static_cast<unsigned>((n4 + 255) / 256), 256, 0, st>>>(s, hsplit, part, dqkv);
+  ++g_kernel_launches;
+  return cudaGetLastError();
 }
 
 }  // namespace soup

@@ -25,6 +25,7 @@
 // w = bf16_rn(fp32(code_value * mhat)), one float32 multiply per element.
 #include "common.cuh"
 #include "internal.h"
+#include "tc.cuh"
 
 #include <cudaTypedefs.h>
 
@@ -70,90 +71,10 @@ struct GemmCfg {
   static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + RAW_SLOTS * RAW_BYTES + CTRL_BYTES;
 };
 
-// ---------------------------------------------------------------- tcgen05 / TMA wrappers
-__device__ __forceinline__ void tmem_alloc(uint32_t* slot, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot)), "r"(ncols)
-               : "memory");
-}
-__device__ __forceinline__ void tmem_relinquish() {
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
-}
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-__device__ __forceinline__ void tc_mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                           uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-__device__ __forceinline__ void tc_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-               : "memory");
-}
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
-        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr)
-      : "memory");
-}
-__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
-}
-// 2D tiled TMA load (no multicast) into shared memory, completion counted on `bar`.
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
-          smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
-      : "memory");
-}
-
-// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row core groups 1024 B apart.
-__device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t saddr) {
-  uint64_t d = 0;
-  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);  // start address
-  d |= static_cast<uint64_t>(1) << 16;                  // leading byte offset (unused with this swizzle)
-  d |= static_cast<uint64_t>(1024 >> 4) << 32;          // stride byte offset: next 8-row group
-  d |= static_cast<uint64_t>(1) << 46;                  // descriptor version for sm_100
-  d |= static_cast<uint64_t>(2) << 61;                  // swizzle mode: 128 B
-  return d;
-}
-
-// Shared-memory matrix descriptor: MN-major, 128-byte swizzle.  Atoms of 8 K-rows x 64 MN
-// elements (1024 B); the next 8 K-rows are 1024 B further (stride byte offset), the next 64
-// MN elements 8192 B further (leading byte offset: one atom column of a 64-deep K block).
-__device__ __forceinline__ uint64_t sw128_mnmajor_desc(uint32_t saddr) {
-  uint64_t d = 0;
-  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
-  d |= static_cast<uint64_t>(8192 >> 4) << 16;  // leading byte offset: next 64 MN elements
-  d |= static_cast<uint64_t>(1024 >> 4) << 32;  // stride byte offset: next 8 K rows
-  d |= static_cast<uint64_t>(1) << 46;
-  d |= static_cast<uint64_t>(2) << 61;
-  return d;
-}
-
-// Instruction descriptor, kind::f16: bf16 x bf16 -> f32, A and B each K- or MN-major, M = 128.
+// Instruction descriptor of the GEMM's MMAs: M = 128 rows, N = BN.
 template <int BN>
 __device__ __forceinline__ uint32_t idesc_bf16_f32(bool a_mn_major, bool b_mn_major) {
-  return (1u << 4)                                 // D format f32
-         | (1u << 7)                               // A format bf16
-         | (1u << 10)                              // B format bf16
-         | ((a_mn_major ? 1u : 0u) << 15)          // A major-ness
-         | ((b_mn_major ? 1u : 0u) << 16)          // B major-ness
-         | (static_cast<uint32_t>(BN >> 3) << 17)  // N / 8
-         | (static_cast<uint32_t>(UM >> 4) << 24); // M / 16
+  return idesc_bf16(UM, BN, a_mn_major, b_mn_major);
 }
 
 // ---------------------------------------------------------------- operand fetch
@@ -1298,6 +1219,13 @@ bool operand_ok(const Operand& op, int K) {
 bool is_mn(int kind) { return kind == OP_BF16_MN || kind == OP_F32_MN || kind == OP_NF4_MN; }
 
 }  // namespace
+
+bool tma_encode_bf16_sw128(CUtensorMap* map, const void* ptr, unsigned long long inner, unsigned long long outer,
+                           unsigned long long row_bytes, unsigned box_inner, unsigned box_outer) {
+  if (inner == 0 || outer == 0 || (reinterpret_cast<uintptr_t>(ptr) & 15u) || (row_bytes & 15u)) return false;
+  return encode_cached(map, ptr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, inner, outer, row_bytes, box_inner, box_outer,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
+}
 
 GemmPlan gemm_plan(const GemmParams& p, int sms, bool stream_k_allowed) {
   GemmPlan pl{};

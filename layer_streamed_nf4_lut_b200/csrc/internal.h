@@ -101,6 +101,12 @@ struct GemmParams {
   int sk_nkt;
 };
 
+// TMA descriptor of a 2D bf16 array (inner x outer elements, rows row_bytes apart), box
+// box_inner x box_outer, 128-byte swizzle (box_inner * 2 must be 128), zero fill out of bounds.
+// Cached by its arguments.  False if the driver refuses it (alignment, sizes).
+bool tma_encode_bf16_sw128(CUtensorMap* map, const void* ptr, unsigned long long inner, unsigned long long outer,
+                           unsigned long long row_bytes, unsigned box_inner, unsigned box_outer);
+
 // Launch C = sum_seg A_seg B_seg^T on the tcgen05 tensor cores. Returns cudaError_t of launch.
 cudaError_t gemm_launch(const GemmParams& p, cudaStream_t st);
 
@@ -170,15 +176,23 @@ struct AttnShape {
   // Shared-prefix pair layout (pl > 0): each of the B blocks of S = pl + 2 rl rows holds one
   // preference pair as [prefix (pl) | chosen response (rl) | rejected response (rl)]; the
   // rejected rows sit at positions pl.. and see the prefix and their own earlier rows, never
-  // the chosen ones.  pl and rl are multiples of the 64-row tile.  pl = 0: plain causal rows.
+  // the chosen ones.  pl = 0: plain causal rows.
   int pl, rl;
 };
-cudaError_t attn_fwd_launch(const AttnShape& s, const uint16_t* qkv, uint16_t* o, float* lse, cudaStream_t st);
-// ws: fp32 scratch (16-byte aligned) for per-head-slice dK / dV partials when the kv grid
-// alone cannot fill the GPU; NULL / too small: no head slices.
-cudaError_t attn_bwd_launch(const AttnShape& s, const uint16_t* qkv, const uint16_t* o, const uint16_t* dout,
-                            const float* lse, float* delta, uint16_t* dqkv, float* ws, size_t ws_bytes,
+// Forward (attention.cu, tcgen05): o [T, hq d] bf16, lse [B, hq, S] fp32 (natural log); err: the
+// device error word (a bounded in-kernel wait that ran out sets it).
+cudaError_t attn_fwd_launch(const AttnShape& s, const uint16_t* qkv, uint16_t* o, float* lse, int* err,
                             cudaStream_t st);
+// Backward: delta [T, hq] fp32 scratch, dQ / dK / dV written into dqkv (same layout as qkv).  ws:
+// fp32 scratch (16-byte aligned) for per-head-slice dK / dV partials when the kv grid alone
+// cannot fill the GPU; NULL / too small: no head slices.
+cudaError_t attn_bwd_launch(const AttnShape& s, const uint16_t* qkv, const uint16_t* o, const uint16_t* dout,
+                            const float* lse, float* delta, uint16_t* dqkv, float* ws, size_t ws_bytes, int* err,
+                            cudaStream_t st);
+// delta[t, h] = sum_d dO * O, and the slice-order sum of per-head-slice dK / dV partials
+cudaError_t attn_delta_launch(const uint16_t* o, const uint16_t* dout, int T, int hq, int d, float* delta,
+                              cudaStream_t st);
+cudaError_t attn_dkdv_sum_launch(const AttnShape& s, int hsplit, const float* part, uint16_t* dqkv, cudaStream_t st);
 
 // ----------------------------------------------------------------- elementwise / row ops
 cudaError_t embed_launch(const int32_t* ids, const uint16_t* table, int T, int h, int V, uint16_t* out, int* err,

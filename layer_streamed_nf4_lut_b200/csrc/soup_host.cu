@@ -818,7 +818,9 @@ soup_status layer_forward(soup_model* m, int i, const LayerView& L, const uint16
   AttnShape as{B, S, c.n_heads, c.n_kv_heads, c.head_dim, QKV, m->pack_pl, m->pack_rl};
   const double attn_flops = 2.0 * B * c.n_heads * c.head_dim * static_cast<double>(S) * (S + 1);
   SOUP_TRY(launch(m, st, CAT_ATTN_FWD, attn_flops, 2.0 * T * QKV + 2.0 * T * qd + 4.0 * T * c.n_heads, "attention fwd",
-                  [&] { return attn_fwd_launch(as, A.qkv, A.o, A.lse, st); }));
+                  [&] {
+                    return attn_fwd_launch(as, A.qkv, A.o, A.lse, m->scal + 1, st);
+                  }));
   // ---- o + residual
   if (lora) {
     GemmParams p = gemm_base(m, T, r, A.uo, r, 0, s);
@@ -1027,8 +1029,8 @@ soup_status layer_backward_body(soup_model* m, int i, const LayerView& L, const 
   const double attn_flops = 4.0 * B * c.n_heads * c.head_dim * static_cast<double>(S) * (S + 1);
   SOUP_TRY(launch(m, st, CAT_ATTN_BWD, attn_flops, 4.0 * T * QKV + 4.0 * T * qd + 8.0 * T * c.n_heads, "attention bwd",
                   [&] {
-                    return attn_bwd_launch(as, A.qkv, A.o, m->da, A.lse, m->delta, m->dqkv, m->gemm_ws, m->gemm_ws_bytes,
-                                           st);
+                    return attn_bwd_launch(as, A.qkv, A.o, m->da, A.lse, m->delta, m->dqkv, m->gemm_ws,
+                                              m->gemm_ws_bytes, m->scal + 1, st);
                   }));
   const double rope_bytes = 4.0 * T * (c.n_heads + c.n_kv_heads) * c.head_dim;
   SOUP_TRY(launch(m, st, CAT_ROPE, 0, rope_bytes, "rope bwd", [&] {

@@ -26,3 +26,11 @@ def test_rank_kernels_without_overhead_or_groups():
     kern, grouped, dom, ov_ms = bench.rank_kernels({"attention_fwd": _cat(32, 2.0), "rope": _cat(64, 1.0)})
     assert ov_ms == 0.0 and dom == "attention_fwd"
     assert bench.rank_kernels({"h2d_layer_copy": _cat(1, 1.0)})[2] is None
+
+
+def test_both_arms_print_the_same_config():
+    wl = bench.WORKLOADS[bench.DEFAULT]
+    a = bench.config_of(bench.DEFAULT, wl, 1)
+    assert a == bench.config_of(bench.DEFAULT, dict(wl), 1)
+    assert a["global_batch"] == wl["B"] and a["seq_len"] == wl["S"] and a["parallelism"] == "dp1"
+    assert bench.config_of(bench.DEFAULT, wl, 4)["global_batch"] == 4 * wl["B"]

@@ -147,12 +147,19 @@ def test_full_width_layer_and_head_dpo_step_vs_oracle():
         layers, head = om.model_from_quantised(cfg, [q], (_bits(emb), _bits(lm), _bits(g_fin)))
         olora = {k: (a.astype(np.float64), b.astype(np.float64)) for k, (a, b) in lora.items()}
         ol, og, aux = om.dpo_step(dict(cfg, batch=2 * P), layers, olora, head, ids, pre, beta)
-        # sequence log-prob sums of 256 targets each (fp32 sums on the GPU)
-        assert np.max(np.abs(pi - aux["pi"]) / np.abs(aux["pi"])) < 1e-2, (pi, aux["pi"])
-        assert np.max(np.abs(ref - aux["ref"]) / np.abs(aux["ref"])) < 1e-2, (ref, aux["ref"])
+        # sequence log-prob sums of 256 targets each (fp32 sums over bf16 activations): each
+        # within a nat of the float64 oracle on sums of ~3000 nats (measured <= 0.6)
+        dpi, dref = pi - aux["pi"], ref - aux["ref"]
+        assert np.max(np.abs(dpi)) < 1.0 and np.max(np.abs(dref)) < 1.0, (dpi, dref)
         closed, _ = om.dpo_loss(pi.astype(np.float64), ref.astype(np.float64), beta)
         assert abs(loss - closed) < 1e-5
-        assert abs(loss - ol) <= 1e-2 * abs(ol), (loss, ol)
+        # The loss is a function of z = beta ((pi_c - ref_c) - (pi_r - ref_r)) ~ 0.04 here, so it
+        # sits within z/2 of ln 2, and the bf16 spread of the log-prob sums above moves z by
+        # ~0.01-0.04 (an error that no longer shrinks relative to the loss): the stated 1e-2
+        # relative tolerance, or where that is below the rounding floor, the first-order
+        # propagation of the log-prob errors (|dL/dpi| <= beta / P per sequence)
+        floor = beta / P * float(np.sum(np.abs(dpi)) + np.sum(np.abs(dref)))
+        assert abs(loss - ol) <= max(1e-2 * abs(ol), floor), (loss, ol, floor)
         for p in PROJ:
             assert cosine(grads[p][0], og[(0, p)][0]) > 0.999, p
             assert cosine(grads[p][1], og[(0, p)][1]) > 0.999, p
