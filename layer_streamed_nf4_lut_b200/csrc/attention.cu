@@ -367,6 +367,38 @@ __device__ __forceinline__ uint64_t kdesc(uint32_t tile, int kc) {
 // MN-major view of the same tile: rows are the reduction index, 16 rows per step
 __device__ __forceinline__ uint64_t mndesc(uint32_t tile, int kk) { return sw128_mnmajor_desc(tile + kk * 2048, 128 * 128); }
 
+// The RoPE backward on one row of dQ or dK: columns (i0.., i0 + d/2..) of a head rotated back by
+// the angles of the row's position, x1' = x1 cos + x2 sin, x2' = x2 cos - x1 sin (no tables: no
+// rotation).
+template <int D>
+__device__ __forceinline__ void rope_back16(const AttnShape& s, int pos, int i0, float (&x1)[16], float (&x2)[16]) {
+  if (!s.rope_cos) return;
+  const float4* cp = reinterpret_cast<const float4*>(s.rope_cos + static_cast<long long>(pos) * (D / 2) + i0);
+  const float4* sp = reinterpret_cast<const float4*>(s.rope_sin + static_cast<long long>(pos) * (D / 2) + i0);
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    const float4 cv = __ldg(cp + g), sv = __ldg(sp + g);
+    const float c[4] = {cv.x, cv.y, cv.z, cv.w}, sn[4] = {sv.x, sv.y, sv.z, sv.w};
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float a = x1[4 * g + u], b = x2[4 * g + u];
+      x1[4 * g + u] = a * c[u] + b * sn[u];
+      x2[4 * g + u] = b * c[u] - a * sn[u];
+    }
+  }
+}
+
+__device__ __forceinline__ void store_bf16x16(uint16_t* dst, const float (&f)[16]) {
+  reinterpret_cast<uint4*>(dst)[0] = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
+                                                pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
+  reinterpret_cast<uint4*>(dst)[1] = make_uint4(pack_bf16x2(f[8], f[9]), pack_bf16x2(f[10], f[11]),
+                                                pack_bf16x2(f[12], f[13]), pack_bf16x2(f[14], f[15]));
+}
+__device__ __forceinline__ void store_f32x16(float* dst, const float (&f)[16]) {
+#pragma unroll
+  for (int e = 0; e < 16; e += 4) *reinterpret_cast<float4*>(dst + e) = make_float4(f[e], f[e + 1], f[e + 2], f[e + 3]);
+}
+
 template <int D>
 __global__ void __launch_bounds__(FWD_THREADS, 1)
     attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tdo,
@@ -537,45 +569,42 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
       }
     if (it > 0) mbar_wait_bounded(mma_done, (it - 1) & 1, abort_flag, err);
     tc_fence_after();
-    // epilogue: dK = scale * (dS^T Q), dV = P^T dO for this key row
+    // epilogue: dK = scale * (dS^T Q) rotated back by the key's RoPE angles, dV = P^T dO, for
+    // this key row; columns i0.. and i0 + D/2.. of the head together (the rotation pairs them)
     const long long T = static_cast<long long>(s.B) * s.S;
-#pragma unroll
-    for (int c = 0; c < D / 16; ++c) {
-      uint32_t a[16], v[16];
-      tmem_ld16(tmem + lane_base + C::ACC1 + c * 16, a);  // dK
-      tmem_ld16(tmem + lane_base + C::ACC0 + c * 16, v);  // dV
+    const int pos = pk_pos(s, k);
+#pragma unroll 1
+    for (int i0 = 0; i0 < D / 2; i0 += 16) {
+      uint32_t a1[16], a2[16], v1[16], v2[16];
+      tmem_ld16(tmem + lane_base + C::ACC1 + i0, a1);  // dK
+      tmem_ld16(tmem + lane_base + C::ACC1 + i0 + D / 2, a2);
+      tmem_ld16(tmem + lane_base + C::ACC0 + i0, v1);  // dV
+      tmem_ld16(tmem + lane_base + C::ACC0 + i0 + D / 2, v2);
       tmem_ld_wait();
       if (k >= s.S) continue;
-      float fk[16], fv[16];
+      float k1[16], k2[16], w1[16], w2[16];
 #pragma unroll
       for (int e = 0; e < 16; ++e) {
-        fk[e] = it > 0 ? __uint_as_float(a[e]) * scale : 0.f;
-        fv[e] = it > 0 ? __uint_as_float(v[e]) : 0.f;
+        k1[e] = it > 0 ? __uint_as_float(a1[e]) * scale : 0.f;
+        k2[e] = it > 0 ? __uint_as_float(a2[e]) * scale : 0.f;
+        w1[e] = it > 0 ? __uint_as_float(v1[e]) : 0.f;
+        w2[e] = it > 0 ? __uint_as_float(v2[e]) : 0.f;
       }
+      rope_back16<D>(s, pos, i0, k1, k2);
       if (hsplit == 1) {
-        uint16_t* dk = dqkv + (static_cast<long long>(row0) + k) * s.ld_qkv + (s.hq + g) * D + c * 16;
-        uint16_t* dvp = dqkv + (static_cast<long long>(row0) + k) * s.ld_qkv + (s.hq + s.hkv + g) * D + c * 16;
-        uint4 w[4];
-        w[0] = make_uint4(pack_bf16x2(fk[0], fk[1]), pack_bf16x2(fk[2], fk[3]), pack_bf16x2(fk[4], fk[5]),
-                          pack_bf16x2(fk[6], fk[7]));
-        w[1] = make_uint4(pack_bf16x2(fk[8], fk[9]), pack_bf16x2(fk[10], fk[11]), pack_bf16x2(fk[12], fk[13]),
-                          pack_bf16x2(fk[14], fk[15]));
-        w[2] = make_uint4(pack_bf16x2(fv[0], fv[1]), pack_bf16x2(fv[2], fv[3]), pack_bf16x2(fv[4], fv[5]),
-                          pack_bf16x2(fv[6], fv[7]));
-        w[3] = make_uint4(pack_bf16x2(fv[8], fv[9]), pack_bf16x2(fv[10], fv[11]), pack_bf16x2(fv[12], fv[13]),
-                          pack_bf16x2(fv[14], fv[15]));
-        reinterpret_cast<uint4*>(dk)[0] = w[0];
-        reinterpret_cast<uint4*>(dk)[1] = w[1];
-        reinterpret_cast<uint4*>(dvp)[0] = w[2];
-        reinterpret_cast<uint4*>(dvp)[1] = w[3];
+        uint16_t* dk = dqkv + (static_cast<long long>(row0) + k) * s.ld_qkv + (s.hq + g) * D + i0;
+        uint16_t* dvp = dqkv + (static_cast<long long>(row0) + k) * s.ld_qkv + (s.hq + s.hkv + g) * D + i0;
+        store_bf16x16(dk, k1);
+        store_bf16x16(dk + D / 2, k2);
+        store_bf16x16(dvp, w1);
+        store_bf16x16(dvp + D / 2, w2);
       } else {
         const int per_row = s.hkv * 2 * D;
         float* pr = part + (static_cast<long long>(slice) * T + row0 + k) * per_row + g * 2 * D;
-#pragma unroll
-        for (int e = 0; e < 16; e += 4) {
-          *reinterpret_cast<float4*>(pr + c * 16 + e) = make_float4(fk[e], fk[e + 1], fk[e + 2], fk[e + 3]);
-          *reinterpret_cast<float4*>(pr + D + c * 16 + e) = make_float4(fv[e], fv[e + 1], fv[e + 2], fv[e + 3]);
-        }
+        store_f32x16(pr + i0, k1);
+        store_f32x16(pr + i0 + D / 2, k2);
+        store_f32x16(pr + D + i0, w1);
+        store_f32x16(pr + D + i0 + D / 2, w2);
       }
     }
   }
@@ -735,20 +764,25 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
     }
     if (jj > 0) mbar_wait_bounded(mma_done, (jj - 1) & 1, abort_flag, err);
     tc_fence_after();
+    // dQ = scale * (dS K), rotated back by the query's RoPE angles
     uint16_t* qrow = dqkv + (static_cast<long long>(row0) + q) * s.ld_qkv + h * D;
-#pragma unroll
-    for (int c = 0; c < D / 16; ++c) {
-      uint32_t a[16];
-      tmem_ld16(tmem + lane_base + C::ACC0 + c * 16, a);
+    const int pos = pk_pos(s, q);
+#pragma unroll 1
+    for (int i0 = 0; i0 < D / 2; i0 += 16) {
+      uint32_t a1[16], a2[16];
+      tmem_ld16(tmem + lane_base + C::ACC0 + i0, a1);
+      tmem_ld16(tmem + lane_base + C::ACC0 + i0 + D / 2, a2);
       tmem_ld_wait();
       if (q >= s.S) continue;
-      float f[16];
+      float f1[16], f2[16];
 #pragma unroll
-      for (int e = 0; e < 16; ++e) f[e] = jj > 0 ? __uint_as_float(a[e]) * scale : 0.f;
-      reinterpret_cast<uint4*>(qrow + c * 16)[0] = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
-                                                              pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
-      reinterpret_cast<uint4*>(qrow + c * 16)[1] = make_uint4(pack_bf16x2(f[8], f[9]), pack_bf16x2(f[10], f[11]),
-                                                              pack_bf16x2(f[12], f[13]), pack_bf16x2(f[14], f[15]));
+      for (int e = 0; e < 16; ++e) {
+        f1[e] = jj > 0 ? __uint_as_float(a1[e]) * scale : 0.f;
+        f2[e] = jj > 0 ? __uint_as_float(a2[e]) * scale : 0.f;
+      }
+      rope_back16<D>(s, pos, i0, f1, f2);
+      store_bf16x16(qrow + i0, f1);
+      store_bf16x16(qrow + i0 + D / 2, f2);
     }
   }
   tc_fence_before();

@@ -101,39 +101,6 @@ __global__ void rmsnorm_bwd_kernel(const uint16_t* __restrict__ dy, const uint16
   }
 }
 
-// ---------------------------------------------------------------- RoPE (rotate-half, in place)
-// (z_i, z_{i+d/2}) -> (z_i cos - z_{i+d/2} sin, z_{i+d/2} cos + z_i sin) with the angle
-// pos * theta^(-2i/d), pos = t mod S, read from a [S_max, d/2] cos/sin table; inverse != 0
-// rotates by -angle (the backward).  One thread per 8 consecutive i of one head.
-__global__ void rope_kernel(uint16_t* __restrict__ qkv, long long ld, int S, int nheads, int d,
-                            const float* __restrict__ tcos, const float* __restrict__ tsin, int inverse, int pack_rl) {
-  const int t = blockIdx.x;
-  const int half = d / 2, g8 = half / 8;
-  int pos = t % S;
-  if (pack_rl > 0 && pos >= S - pack_rl) pos -= pack_rl;  // rejected response of a shared-prefix pair
-  uint16_t* row = qkv + static_cast<long long>(t) * ld;
-  for (int idx = threadIdx.x; idx < nheads * g8; idx += blockDim.x) {
-    const int hh = idx / g8, i0 = (idx % g8) * 8;
-    uint16_t* z = row + hh * d;
-    float a[8], b[8], o1[8], o2[8];
-    load8(z + i0, a);
-    load8(z + half + i0, b);
-    const float4* cp = reinterpret_cast<const float4*>(tcos + static_cast<long long>(pos) * half + i0);
-    const float4* sp = reinterpret_cast<const float4*>(tsin + static_cast<long long>(pos) * half + i0);
-    const float4 c0 = cp[0], c1 = cp[1], s0 = sp[0], s1 = sp[1];
-    const float c[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-    float sn[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const float sj = inverse ? -sn[j] : sn[j];
-      o1[j] = a[j] * c[j] - b[j] * sj;
-      o2[j] = b[j] * c[j] + a[j] * sj;
-    }
-    store8(z + i0, o1);
-    store8(z + half + i0, o2);
-  }
-}
-
 // ---------------------------------------------------------------- SwiGLU
 __global__ void swiglu_fwd_kernel(const uint16_t* __restrict__ gu, int I, long long total8, uint16_t* __restrict__ m) {
   const long long i8 = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -592,18 +559,6 @@ cudaError_t rmsnorm_bwd_launch(const uint16_t* dy, const uint16_t* x, const floa
                                const uint16_t* dres, int T, int h, uint16_t* dx, cudaStream_t st) {
   if (T <= 0) return cudaSuccess;
   rmsnorm_bwd_kernel<<<T, row_threads(h), 0, st>>>(dy, x, rstd, gamma, dres, h, dx);
-  ++g_kernel_launches;
-  return cudaGetLastError();
-}
-
-cudaError_t rope_launch(uint16_t* qkv, long long ld, int B, int S, int hq, int hkv, int d, const float* tcos,
-                        const float* tsin, int inverse, cudaStream_t st, int pack_rl) {
-  const int T = B * S;
-  if (T <= 0) return cudaSuccess;
-  const int nheads = hq + hkv;  // q heads then k heads, contiguous from column 0
-  int thr = nheads * d / 16;
-  thr = thr > 256 ? 256 : ((thr + 31) / 32) * 32;
-  rope_kernel<<<T, thr, 0, st>>>(qkv, ld, S, nheads, d, tcos, tsin, inverse, pack_rl);
   ++g_kernel_launches;
   return cudaGetLastError();
 }

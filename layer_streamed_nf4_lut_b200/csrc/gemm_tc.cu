@@ -48,6 +48,9 @@ constexpr int GROUP_THREADS = 128;
 constexpr int UM = 128;  // rows of one tcgen05.mma (cta_group::1); a CTA tile stacks MT of them
 constexpr int BK = 64;   // 64 bf16 = 128 bytes = one swizzle row
 constexpr int SMEM_LIMIT = 232448;  // 227 KiB of dynamic shared memory per CTA
+#ifndef SOUP_GEMM_RAWK
+#define SOUP_GEMM_RAWK 4  // k-blocks per raw NF4 slot
+#endif
 
 template <int MT, int BN>
 struct GemmCfg {
@@ -55,15 +58,19 @@ struct GemmCfg {
   static constexpr int A_BYTES = BM * 128;
   static constexpr int B_BYTES = BN * 128;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // one k-block of both MMA operands
-  // Raw NF4 staging (TMA) in a ring of its own: codes BN x 32 B (forward) or 64 x BN/2 B
-  // (transposed), q8 absmax BN x 16 B or 64 x 16 B.  A raw slot is released as soon as its
-  // k-block is dequantised, so the raw loads run several k-blocks ahead of the operand stages.
-  static constexpr int RAW_CODE_BYTES = BN * 32;
-  static constexpr int RAW_Q8_BYTES = (BN > 64 ? BN : 64) * 16;
+  // Raw NF4 staging (TMA) in a ring of its own, RAWK k-blocks per slot: codes BN x 32 RAWK B
+  // (forward) or 64 RAWK x BN/2 B (transposed), q8 absmax BN x 16 B or 64 RAWK x 16 B.  A TMA
+  // copy costs about the same time whatever its size (measured on B200: a 16 KB and a 32 KB
+  // box both take ~280 ns of a SM's copy engine), so the small raw copies are batched: one
+  // codes copy and one absmax copy per RAWK k-blocks.  A slot is released as soon as its
+  // k-blocks are dequantised, so the raw loads run ahead of the operand stages.
+  static constexpr int RAWK = SOUP_GEMM_RAWK;
+  static constexpr int RAW_CODE_BYTES = BN * 32 * RAWK;
+  static constexpr int RAW_Q8_BYTES = (BN > 64 * RAWK ? BN : 64 * RAWK) * 16;
   static constexpr int RAW_BYTES = RAW_CODE_BYTES + RAW_Q8_BYTES;
   static constexpr int CTRL_BYTES = 640;
   static constexpr int AVAIL = SMEM_LIMIT - 1024 - CTRL_BYTES;
-  static constexpr int STAGES_FIT = (AVAIL - 4 * RAW_BYTES) / STAGE_BYTES;
+  static constexpr int STAGES_FIT = (AVAIL - 2 * RAW_BYTES) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
   static constexpr int RAW_FIT = (AVAIL - STAGES * STAGE_BYTES) / RAW_BYTES;
   static constexpr int RAW_SLOTS = RAW_FIT > 16 ? 16 : RAW_FIT;
@@ -329,7 +336,7 @@ __device__ __forceinline__ void dx_scales(const NF4Group& g, int s, int n0, int 
 
 template <int BN>
 __device__ __forceinline__ void decode_fwd_raw(const NF4Group& g, int s, const float (&cb)[16], const float* seg_mean,
-                                               int n0, int N, int kbw, const uint8_t* raw_codes,
+                                               int n0, int N, int kbw, const uint8_t* raw_codes, int code_stride,
                                                const uint8_t* raw_q8, uint8_t* tile, int gtid, const float* s2) {
   const float mean = seg_mean[s];
 #pragma unroll
@@ -338,7 +345,7 @@ __device__ __forceinline__ void decode_fwd_raw(const NF4Group& g, int s, const f
     if (r >= BN) break;
     const uint32_t trow = smem_u32(tile) + (r >> 3) * 1024 + (r & 7) * 128;
     if (n0 + r < N) {
-      const uint32_t rc = smem_u32(raw_codes) + r * 32;
+      const uint32_t rc = smem_u32(raw_codes) + r * code_stride;
       const uint4 w0 = lds128(rc);
       const uint4 w1 = lds128(rc + 16);
       const int q8 = lds_s8(smem_u32(raw_q8) + r * 16 + (kbw & 15));
@@ -500,6 +507,47 @@ __device__ __forceinline__ void epilogue_store(const GemmParams& p, int row, int
   }
 }
 
+// RoPE epilogue of one row: a[16] / b[16] are the accumulator columns i0..i0+15 and
+// i0 + d/2.. of one head (i0 < d/2) whose first column is col_head; rotated by the row's angles
+// (pos * theta^(-2i/d) from the cos / sin tables) after scaling, then rounded to bf16 once.
+__device__ __forceinline__ void rope_store16(const GemmParams& p, int row, int col_head, int i0, const uint32_t (&a)[16],
+                                             const uint32_t (&b)[16]) {
+  const int half = p.rope_d >> 1;
+  int pos = row % p.rope_S;
+  if (p.rope_rl > 0 && pos >= p.rope_S - p.rope_rl) pos -= p.rope_rl;
+  const float4* cp = reinterpret_cast<const float4*>(p.rope_cos + static_cast<long long>(pos) * half + i0);
+  const float4* sp = reinterpret_cast<const float4*>(p.rope_sin + static_cast<long long>(pos) * half + i0);
+  float c[16], sn[16];
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    const float4 cv = __ldg(cp + g), sv = __ldg(sp + g);
+    c[4 * g] = cv.x; c[4 * g + 1] = cv.y; c[4 * g + 2] = cv.z; c[4 * g + 3] = cv.w;
+    sn[4 * g] = sv.x; sn[4 * g + 1] = sv.y; sn[4 * g + 2] = sv.z; sn[4 * g + 3] = sv.w;
+  }
+  uint32_t w1[8], w2[8];
+#pragma unroll
+  for (int j = 0; j < 16; j += 2) {
+    float o1[2], o2[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const float x1 = p.alpha * __uint_as_float(a[j + u]), x2 = p.alpha * __uint_as_float(b[j + u]);
+      o1[u] = x1 * c[j + u] - x2 * sn[j + u];
+      o2[u] = x2 * c[j + u] + x1 * sn[j + u];
+    }
+    w1[j >> 1] = pack_bf16x2(o1[0], o1[1]);
+    w2[j >> 1] = pack_bf16x2(o2[0], o2[1]);
+  }
+  uint16_t* o = static_cast<uint16_t*>(p.out) + static_cast<long long>(row) * p.ldo + col_head + i0;
+  reinterpret_cast<uint4*>(o)[0] = make_uint4(w1[0], w1[1], w1[2], w1[3]);
+  reinterpret_cast<uint4*>(o)[1] = make_uint4(w1[4], w1[5], w1[6], w1[7]);
+  reinterpret_cast<uint4*>(o + half)[0] = make_uint4(w2[0], w2[1], w2[2], w2[3]);
+  reinterpret_cast<uint4*>(o + half)[1] = make_uint4(w2[4], w2[5], w2[6], w2[7]);
+}
+
+__device__ __forceinline__ void mbar_arrive_cnt(uint64_t* bar, uint32_t cnt) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(cnt) : "memory");
+}
+
 // Group-scale registers of one k-block of the NF4 B tile (forward: one per row this thread
 // decodes; dX: one per absmax block).
 template <int BN>
@@ -594,7 +642,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
     }
     for (int r = 0; r < C::RAW_SLOTS; ++r) {
       mbar_init(&raw_full[r], 1);
-      mbar_init(&raw_empty[r], GROUP_THREADS / 32);  // the 4 warps of the group that decoded it
+      mbar_init(&raw_empty[r], (GROUP_THREADS / 32) * p.raw_k);  // 4 warps per k-block decoded from it
     }
     mbar_init(done, 1);
     mbar_init(tmem_empty, 4);  // one arrival per epilogue warp
@@ -639,11 +687,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
         const bool fwd = p.seg[0].B.kind == OP_NF4_K;
         ScaleRegs<BN> cur, nxt;
         if (kb0 < n_raw) load_scales<BN>(p, fwd, n0, kb_lo + kb0, gtid, nxt);
+        const int rk = p.raw_k, ch0 = kb_lo / rk;
         for (int kb = kb0; kb < n_raw; kb += GROUPS) {
           const int kk = kb_lo + kb;
           cur = nxt;
           if (kb + GROUPS < n_raw) load_scales<BN>(p, fwd, n0, kk + GROUPS, gtid, nxt);
-          const int gb = kb_run + kb, rb = raw_run + kb;
+          // raw slot: chunk kk / rk of this piece's chunks (chunks aligned to multiples of rk)
+          const int gb = kb_run + kb, rb = raw_run + (kk / rk - ch0), sub = kk % rk;
           const int st = gb % C::STAGES;
           const uint32_t ph = static_cast<uint32_t>(gb / C::STAGES) & 1u;
           uint8_t* As = base + st * C::STAGE_BYTES;
@@ -655,14 +705,20 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
           mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, p.err);
           mbar_wait_bounded(&raw_full[rs], rph, abort_flag, p.err);
           if (fwd) {
-            decode_fwd_raw<BN>(p.nf4, nf4_seg_of(p.nf4, n0), cb, seg_mean, n0, p.N, kk, Rc, Rq, Bs, gtid, cur.v);
+            decode_fwd_raw<BN>(p.nf4, nf4_seg_of(p.nf4, n0), cb, seg_mean, n0, p.N, kk, Rc + sub * 32, 32 * rk, Rq, Bs,
+                               gtid, cur.v);
           } else {
             const int k0 = kk * BK;
-            decode_dx_raw<BN>(p.nf4, nf4_seg_of(p.nf4, k0), cb, seg_mean, n0, p.N, k0, ((n0 >> 6) >> 4) << 4, Rc, Rq,
-                              Bs, gtid, cur.v);
+            decode_dx_raw<BN>(p.nf4, nf4_seg_of(p.nf4, k0), cb, seg_mean, n0, p.N, k0, ((n0 >> 6) >> 4) << 4,
+                              Rc + sub * 64 * (BN / 2), Rq + sub * 64 * 16, Bs, gtid, cur.v);
           }
           __syncwarp();
-          if (lane == 0) mbar_arrive(&raw_empty[rs]);  // this warp's reads of the raw slot are done
+          // this warp's reads of the raw slot are done; the last k-block of a chunk this piece
+          // only partly uses also counts the chunk's k-blocks outside the piece
+          if (lane == 0) {
+            const int c_lo = max(kb_lo, (kk / rk) * rk), c_hi = min(kb_lo + n_raw, (kk / rk) * rk + rk);
+            mbar_arrive_cnt(&raw_empty[rs], kk == c_hi - 1 ? 1u + static_cast<uint32_t>(rk - (c_hi - c_lo)) : 1u);
+          }
           if (p.a_mode[0] == 0) load_tile<BM>(p.seg[0].A, p.nf4, lut, seg_mean, p.seg[0].K, m0, p.M, kk * BK, As, gtid);
           fence_proxy_async_smem();
           __syncwarp();
@@ -702,7 +758,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
         }
       }
       kb_run += kb_hi > kb_lo ? kb_hi - kb_lo : 0;
-      raw_run += n_raw;
+      raw_run += n_raw > 0 ? (kb_lo + n_raw - 1) / p.raw_k - kb_lo / p.raw_k + 1 : 0;
     }
   } else {
     const int q = warp - EPI_WARP0;  // TMEM lane quarter of this epilogue warp
@@ -759,10 +815,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
       }
       if (warp == EPI_WARP0 + 2 && lane == 0 && n_raw > 0) {
         // ---------------------------------------------- TMA issuer: raw NF4 codes / absmax
+        // one codes copy and one absmax copy per chunk of rk k-blocks (chunks aligned to
+        // multiples of rk; a piece's first and last chunk may reach outside it)
         const GemmSeg& sg = p.seg[0];
-        for (int kb = 0; kb < n_raw; ++kb) {
-          const int kk = kb_lo + kb;  // k-block index within segment 0
-          const int rb = raw_run + kb;
+        const int rk = p.raw_k, ch0 = kb_lo / rk, nch = (kb_lo + n_raw - 1) / rk - ch0 + 1;
+        for (int c = 0; c < nch; ++c) {
+          const int kk0 = (ch0 + c) * rk;  // first k-block of the chunk within segment 0
+          const int rb = raw_run + c;
           const int rs = rb % C::RAW_SLOTS;
           const uint32_t rph = static_cast<uint32_t>(rb / C::RAW_SLOTS) & 1u;
           mbar_wait_bounded(&raw_empty[rs], rph ^ 1u, abort_flag, p.err);
@@ -771,14 +830,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
           if (sg.B.kind == OP_NF4_K) {
             const int si = nf4_seg_of(p.nf4, n0);
             const int y = n0 - p.nf4.seg[si].row_begin;
-            mbar_arrive_expect_tx(&raw_full[rs], BN * 32 + BN * 16);
-            tma_load_2d(Rc, &p.tmapCodes[si], kk * (BK / 2), y, &raw_full[rs]);
-            tma_load_2d(Rq, &p.tmapQ8[si], (kk >> 4) << 4, y, &raw_full[rs]);
+            mbar_arrive_expect_tx(&raw_full[rs], BN * 32 * rk + BN * 16);
+            tma_load_2d(Rc, &p.tmapCodes[si], kk0 * (BK / 2), y, &raw_full[rs]);
+            tma_load_2d(Rq, &p.tmapQ8[si], (kk0 >> 4) << 4, y, &raw_full[rs]);
           } else {
-            const int k0 = kk * BK;
+            const int k0 = kk0 * BK;
             const int si = nf4_seg_of(p.nf4, k0);
             const int y = k0 - p.nf4.seg[si].row_begin;
-            mbar_arrive_expect_tx(&raw_full[rs], 64 * (BN / 2) + 64 * 16);
+            mbar_arrive_expect_tx(&raw_full[rs], 64 * rk * (BN / 2) + 64 * rk * 16);
             tma_load_2d(Rc, &p.tmapCodes[si], n0 / 2, y, &raw_full[rs]);
             tma_load_2d(Rq, &p.tmapQ8[si], ((n0 >> 6) >> 4) << 4, y, &raw_full[rs]);
           }
@@ -841,8 +900,27 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
       const bool any_k = kb_hi > kb_lo;
       const bool sk_part = SK && z.partial;
       float* slot = sk_part ? p.workspace + static_cast<long long>(sk_slot(blockIdx.x, pc)) * (BM * BN) : nullptr;
+      const bool rope_tile = p.rope_cols > 0 && n0 < p.rope_cols && !z.partial && any_k;
+      if (rope_tile) {
+        // head pairs (i, i + d/2) are both in this tile (tiles never straddle a head: see gemm_plan)
+        const int half = p.rope_d >> 1;
 #pragma unroll 1
-      for (int hc = 0; hc < MT * BN; hc += 16) {
+        for (int h = 0; h < MT; ++h)
+#pragma unroll 1
+          for (int hb = 0; hb < BN; hb += p.rope_d)
+#pragma unroll 1
+            for (int i0 = 0; i0 < half; i0 += 16) {
+              const uint32_t tq = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(h * BN + hb + i0);
+              uint32_t a[16], b[16];
+              tmem_ld16(tq, a);
+              tmem_ld16(tq + static_cast<uint32_t>(half), b);
+              tmem_ld_wait();
+              const int row = m0 + h * UM + q * 32 + lane;
+              if (row < p.M) rope_store16(p, row, n0 + hb, i0, a, b);
+            }
+      }
+#pragma unroll 1
+      for (int hc = 0; hc < (rope_tile ? 0 : MT * BN); hc += 16) {
         const int h = hc / BN, cc = hc % BN;
         const int rl = h * UM + q * 32 + lane;  // row within the tile
         const int row = m0 + rl;
@@ -892,7 +970,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
         }
       }
       kb_run += kb_hi > kb_lo ? kb_hi - kb_lo : 0;
-      raw_run += n_raw;
+      raw_run += n_raw > 0 ? (kb_lo + n_raw - 1) / p.raw_k - kb_lo / p.raw_k + 1 : 0;
     }
   }
 
@@ -1125,7 +1203,7 @@ bool tma_operands_allowed() {
   return allowed;
 }
 
-bool setup_raw_tma(GemmParams& p, int BN) {
+bool setup_raw_tma(GemmParams& p, int BN, int rawk_max) {
   if (!raw_tma_allowed()) return false;
   const GemmSeg& s0 = p.seg[0];
   if (s0.K <= 0 || (s0.B.kind != OP_NF4_K && s0.B.kind != OP_NF4_MN)) return false;
@@ -1139,14 +1217,27 @@ bool setup_raw_tma(GemmParams& p, int BN) {
     for (int i = 1; i < g.nseg; ++i)
       if (g.seg[i].row_begin % 64 != 0) return false;
   }
+  // k-blocks per raw chunk: the largest of 4, 2, 1 (up to the slot's room) such that in the
+  // transposed read no chunk straddles two stacked tensors (chunks are aligned to multiples of
+  // rk in the stacked K)
+  int rk = rawk_max;
+  if (s0.B.kind == OP_NF4_MN)
+    while (rk > 1) {
+      bool ok = true;
+      for (int i = 1; i < g.nseg; ++i)
+        if ((g.seg[i].row_begin / BK) % rk != 0) ok = false;
+      if (ok) break;
+      rk >>= 1;
+    }
+  p.raw_k = rk;
   const unsigned long long cb = static_cast<unsigned long long>(g.cols) / 2, qb = static_cast<unsigned long long>(g.cols) / 64;
   for (int i = 0; i < g.nseg; ++i) {
     const unsigned long long rows = static_cast<unsigned long long>(g.seg[i].rows);
     const bool ok = (s0.B.kind == OP_NF4_K)
-                        ? (encode_u8_2d(&p.tmapCodes[i], g.seg[i].codes, cb, rows, cb, 32, BN) &&
+                        ? (encode_u8_2d(&p.tmapCodes[i], g.seg[i].codes, cb, rows, cb, 32 * rk, BN) &&
                            encode_u8_2d(&p.tmapQ8[i], g.seg[i].q8, qb, rows, qb, 16, BN))
-                        : (encode_u8_2d(&p.tmapCodes[i], g.seg[i].codes, cb, rows, cb, BN / 2, 64) &&
-                           encode_u8_2d(&p.tmapQ8[i], g.seg[i].q8, qb, rows, qb, 16, 64));
+                        : (encode_u8_2d(&p.tmapCodes[i], g.seg[i].codes, cb, rows, cb, BN / 2, 64 * rk) &&
+                           encode_u8_2d(&p.tmapQ8[i], g.seg[i].q8, qb, rows, qb, 16, 64 * rk));
     if (!ok) return false;
   }
   return true;
@@ -1243,6 +1334,8 @@ GemmPlan gemm_plan(const GemmParams& p, int sms, bool stream_k_allowed) {
   bool has_nf4 = false;
   for (int s = 0; s < p.nseg; ++s)
     if (p.seg[s].K > 0 && (p.seg[s].B.kind == OP_NF4_K || p.seg[s].B.kind == OP_NF4_MN)) has_nf4 = true;
+  // a RoPE epilogue needs whole tiles that hold whole heads and never straddle the RoPE range
+  const bool rope = p.rope_cols > 0;
   const int cand[5][2] = {{2, 128}, {1, 256}, {1, 128}, {2, 64}, {1, 64}};
   const double unit_nf4[5] = {50.0, 60.0, 38.0, 47.0, 36.0};
   const double unit_bf16[5] = {50.0, 60.0, 36.0, 64.0, 36.0};
@@ -1266,6 +1359,7 @@ GemmPlan gemm_plan(const GemmParams& p, int sms, bool stream_k_allowed) {
     if (mt == 2 && p.M <= UM) continue;
     if (bn > 64 && p.N <= 64) continue;
     if (bn > 128 && p.N <= 128) continue;
+    if (rope && (bn % p.rope_d != 0 || p.rope_cols % bn != 0)) continue;
     const long long tl = static_cast<long long>((p.N + bn - 1) / bn) * ((p.M + UM * mt - 1) / (UM * mt));
     const long long sp = split_for(tl);
     const long long waves = (tl * sp + sms - 1) / sms;
@@ -1288,7 +1382,7 @@ GemmPlan gemm_plan(const GemmParams& p, int sms, bool stream_k_allowed) {
   // of the SMs and ran faster per k-block: so at most two 256-row M-tiles.  Only when every
   // N-tile has the same active segments (the flattened k-block count is then tiles x k-blocks
   // per tile) and a tile is cut into at most 4 shares.
-  if (has_nf4 && p.workspace && p.tile_counters && stream_k_allowed && p.M <= 2 * UM * 2) {
+  if (has_nf4 && !rope && p.workspace && p.tile_counters && stream_k_allowed && p.M <= 2 * UM * 2) {
     const int mt = p.M > UM ? 2 : 1, bn = 128, bm = UM * mt;
     const int tiles_n = (p.N + bn - 1) / bn, tiles_m = (p.M + bm - 1) / bm;
     int nkt = -1;
@@ -1327,7 +1421,7 @@ GemmPlan gemm_plan(const GemmParams& p, int sms, bool stream_k_allowed) {
   // NF4 GEMMs keep whole K (the 96-tile q|k|v GEMM ran 105 us split four ways, 65 us whole)
   const int BM = UM * MT;
   const long long tiles = static_cast<long long>((p.N + BN - 1) / BN) * ((p.M + BM - 1) / BM);
-  pl.splits = (has_nf4 || pl.sk_ctas > 0) ? 1 : static_cast<int>(split_for(tiles));
+  pl.splits = (has_nf4 || rope || pl.sk_ctas > 0) ? 1 : static_cast<int>(split_for(tiles));
   // up to 4 partials the tile's last CTA sums them; more run through the wide reduction
   // kernel (measured: 16-32 partials summed by one CTA per tile cost more than the launch)
   pl.fused_reduce = pl.splits <= 4 ? 1 : 0;
@@ -1339,6 +1433,10 @@ cudaError_t gemm_launch(const GemmParams& p_in, cudaStream_t st) {
   GemmParams p = p_in;
   if (p.N % 8 != 0 || p.nseg < 1 || p.nseg > GEMM_MAX_SEG) return cudaErrorInvalidValue;
   if (!aligned16(p.out)) return cudaErrorInvalidValue;
+  if (p.rope_cols > 0 &&
+      (p.out_f32 || p.out_trans || p.residual || p.accumulate || !p.rope_cos || !p.rope_sin || p.rope_S <= 0 ||
+       (p.rope_d != 64 && p.rope_d != 128) || p.rope_cols % p.rope_d != 0 || p.rope_cols > p.N))
+    return cudaErrorInvalidValue;
   if (p.out_trans) {
     if (p.residual) return cudaErrorInvalidValue;
   } else {
@@ -1367,7 +1465,8 @@ cudaError_t gemm_launch(const GemmParams& p_in, cudaStream_t st) {
   const int BM = UM * MT;  // A rows per CTA
   const int BNB = BN;      // B rows per CTA
   p.bn = BNB;
-  p.raw_tma = setup_raw_tma(p, BNB) ? 1 : 0;
+  p.raw_k = 1;
+  p.raw_tma = setup_raw_tma(p, BNB, SOUP_GEMM_RAWK) ? 1 : 0;
   if (tma_operands_allowed()) {
     for (int s = 0; s < p.nseg; ++s) {
       GemmSeg& sg = p.seg[s];

@@ -65,6 +65,7 @@ struct GemmParams {
   int b_mode[GEMM_MAX_SEG];         // same for B (bf16 operands only)
   int b_row0[GEMM_MAX_SEG];         // first operand row of the B descriptor (block-diagonal windows)
   int raw_tma;                      // 1: the NF4 segment's codes / absmax arrive by TMA
+  int raw_k;                        // k-blocks per raw TMA chunk (1, 2 or 4)
   int bn;                           // output tile width
   int M, N;
   int nseg;
@@ -80,6 +81,14 @@ struct GemmParams {
   int accumulate;
   const void* residual;  // bf16, same layout as out (not with out_trans)
   long long ldr;
+  // RoPE in the epilogue (the q | k columns of a q|k|v projection): output columns [0, rope_cols)
+  // are heads of rope_d columns; each pair (i, i + rope_d/2) of a head is rotated by the angle of
+  // the row's position, read from [positions, rope_d/2] cos / sin tables, on the fp32 result
+  // before it is rounded.  Position of row r: r mod rope_S, less rope_rl for the last rope_rl
+  // rows of each block (the rejected response of a shared-prefix pair block).  rope_cols = 0: off.
+  const float* rope_cos;
+  const float* rope_sin;
+  int rope_cols, rope_d, rope_S, rope_rl;
   int* err;
   // split-K: when workspace and tile_counters are given, gemm_launch may split the K loop over
   // `splits` CTAs that write fp32 partial tiles to the workspace; they are summed in split order
@@ -178,6 +187,10 @@ struct AttnShape {
   // rejected rows sit at positions pl.. and see the prefix and their own earlier rows, never
   // the chosen ones.  pl = 0: plain causal rows.
   int pl, rl;
+  // RoPE cos / sin tables [positions, d/2] (the forward rotation is applied in the q|k|v GEMM):
+  // the backward rotates dQ and dK back by the same angles before writing them; NULL: no rotation
+  const float* rope_cos;
+  const float* rope_sin;
 };
 // Forward (attention.cu, tcgen05): o [T, hq d] bf16, lse [B, hq, S] fp32 (natural log); err: the
 // device error word (a bounded in-kernel wait that ran out sets it).
@@ -201,11 +214,6 @@ cudaError_t rmsnorm_fwd_launch(const uint16_t* x, const uint16_t* gamma, int T, 
                                float* rstd, cudaStream_t st);
 cudaError_t rmsnorm_bwd_launch(const uint16_t* dy, const uint16_t* x, const float* rstd, const uint16_t* gamma,
                                const uint16_t* dres, int T, int h, uint16_t* dx, cudaStream_t st);
-// tcos / tsin: [S_max, d/2] fp32 tables of cos / sin(pos * theta^(-2i/d)).
-// pack_rl > 0: rows of a block past S - pack_rl (the rejected response of a shared-prefix
-// pair block) take position (row - pack_rl).
-cudaError_t rope_launch(uint16_t* qkv, long long ld, int B, int S, int hq, int hkv, int d, const float* tcos,
-                        const float* tsin, int inverse, cudaStream_t st, int pack_rl = 0);
 cudaError_t swiglu_fwd_launch(const uint16_t* gu, int T, int I, uint16_t* m, cudaStream_t st);
 cudaError_t swiglu_bwd_launch(const uint16_t* dm, const uint16_t* gu, int T, int I, uint16_t* dgu, cudaStream_t st);
 cudaError_t ce_rows_launch(const float* logits, int T, int V, const int32_t* ids, int B, int S, const uint8_t* mask,

@@ -808,14 +808,16 @@ soup_status layer_forward(soup_model* m, int i, const LayerView& L, const uint16
       for (int q = 0; q < 3; ++q)
         add_seg(p, r, opnd(OP_BF16_K, A.uqkv + q * r, 3 * r), opnd(OP_BF16_K, P + lora_off(c, i, 0, 1), r, 1.f, lo[q], hi[q]));
     }
+    // RoPE on the q and k columns, in the epilogue (rotate-half, the row's position)
+    p.rope_cos = m->rope_cos;
+    p.rope_sin = m->rope_sin;
+    p.rope_cols = qd + kvd;
+    p.rope_d = c.head_dim;
+    p.rope_S = S;
+    p.rope_rl = m->pack_rl;
     SOUP_TRY(run_gemm(m, p, st, "qkv gemm"));
   }
-  const double rope_bytes = 4.0 * T * (c.n_heads + c.n_kv_heads) * c.head_dim;
-  SOUP_TRY(launch(m, st, CAT_ROPE, 0, rope_bytes, "rope", [&] {
-    return rope_launch(A.qkv, QKV, B, S, c.n_heads, c.n_kv_heads, c.head_dim, m->rope_cos, m->rope_sin, 0, st,
-                       m->pack_rl);
-  }));
-  AttnShape as{B, S, c.n_heads, c.n_kv_heads, c.head_dim, QKV, m->pack_pl, m->pack_rl};
+  AttnShape as{B, S, c.n_heads, c.n_kv_heads, c.head_dim, QKV, m->pack_pl, m->pack_rl, m->rope_cos, m->rope_sin};
   const double attn_flops = 2.0 * B * c.n_heads * c.head_dim * static_cast<double>(S) * (S + 1);
   SOUP_TRY(launch(m, st, CAT_ATTN_FWD, attn_flops, 2.0 * T * QKV + 2.0 * T * qd + 4.0 * T * c.n_heads, "attention fwd",
                   [&] {
@@ -1025,18 +1027,13 @@ soup_status layer_backward_body(soup_model* m, int i, const LayerView& L, const 
                         G + lora_off(c, i, 3, 0), gs, true, true));
   }
   // ---- attention, RoPE
-  AttnShape as{B, S, c.n_heads, c.n_kv_heads, c.head_dim, QKV, m->pack_pl, m->pack_rl};
+  AttnShape as{B, S, c.n_heads, c.n_kv_heads, c.head_dim, QKV, m->pack_pl, m->pack_rl, m->rope_cos, m->rope_sin};
   const double attn_flops = 4.0 * B * c.n_heads * c.head_dim * static_cast<double>(S) * (S + 1);
   SOUP_TRY(launch(m, st, CAT_ATTN_BWD, attn_flops, 4.0 * T * QKV + 4.0 * T * qd + 8.0 * T * c.n_heads, "attention bwd",
                   [&] {
                     return attn_bwd_launch(as, A.qkv, A.o, m->da, A.lse, m->delta, m->dqkv, m->gemm_ws,
                                               m->gemm_ws_bytes, m->scal + 1, st);
                   }));
-  const double rope_bytes = 4.0 * T * (c.n_heads + c.n_kv_heads) * c.head_dim;
-  SOUP_TRY(launch(m, st, CAT_ROPE, 0, rope_bytes, "rope bwd", [&] {
-    return rope_launch(m->dqkv, QKV, B, S, c.n_heads, c.n_kv_heads, c.head_dim, m->rope_cos, m->rope_sin, 1, st,
-                       m->pack_rl);
-  }));
   // ---- q | k | v
   const int off[3] = {0, qd, qd + kvd}, outs[3] = {qd, kvd, kvd};
   if (lora) {
