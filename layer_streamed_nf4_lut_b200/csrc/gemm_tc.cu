@@ -58,16 +58,15 @@ struct GemmCfg {
   static constexpr int A_BYTES = BM * 128;
   static constexpr int B_BYTES = BN * 128;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // one k-block of both MMA operands
-  // Raw NF4 staging (TMA) in a ring of its own, RAWK k-blocks per slot: codes BN x 32 RAWK B
-  // (forward) or 64 RAWK x BN/2 B (transposed), q8 absmax BN x 16 B or 64 RAWK x 16 B.  A TMA
-  // copy costs about the same time whatever its size (measured on B200: a 16 KB and a 32 KB
-  // box both take ~280 ns of a SM's copy engine), so the small raw copies are batched: one
-  // codes copy and one absmax copy per RAWK k-blocks.  A slot is released as soon as its
-  // k-blocks are dequantised, so the raw loads run ahead of the operand stages.
+  // Raw NF4 codes staged by TMA in a ring of their own, RAWK k-blocks per slot: BN x 32 RAWK B
+  // (forward) or 64 RAWK x BN/2 B (transposed).  A TMA copy costs a SM's copy engine about the
+  // same time whatever its size (measured on B200: ~280 ns for a 16 B x 128-row box and for a
+  // 32 KB box alike), so the raw codes come in one copy per RAWK k-blocks and the absmax bytes
+  // by plain loads in the producers, which leaves the copy engine to the activation tiles.  A
+  // slot is released as soon as its k-blocks are dequantised.
   static constexpr int RAWK = SOUP_GEMM_RAWK;
   static constexpr int RAW_CODE_BYTES = BN * 32 * RAWK;
-  static constexpr int RAW_Q8_BYTES = (BN > 64 * RAWK ? BN : 64 * RAWK) * 16;
-  static constexpr int RAW_BYTES = RAW_CODE_BYTES + RAW_Q8_BYTES;
+  static constexpr int RAW_BYTES = RAW_CODE_BYTES;
   static constexpr int CTRL_BYTES = 640;
   static constexpr int AVAIL = SMEM_LIMIT - 1024 - CTRL_BYTES;
   static constexpr int STAGES_FIT = (AVAIL - 2 * RAW_BYTES) / STAGE_BYTES;
@@ -244,11 +243,6 @@ __device__ __forceinline__ uint4 lds128(uint32_t a) {
   asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
   return v;
 }
-__device__ __forceinline__ int lds_s8(uint32_t a) {
-  int v;
-  asm volatile("ld.shared.s8 %0, [%1];" : "=r"(v) : "r"(a));
-  return v;
-}
 __device__ __forceinline__ void sts128(uint32_t a, const uint4& v) {
   asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
 }
@@ -304,21 +298,25 @@ __device__ __forceinline__ uint4 decode_word_lut(uint32_t c, const BlockLut& t) 
 // Group scales (s2) of the absmax blocks a thread decodes in one k-block, loaded before the
 // thread waits for the raw tile so their latency overlaps the wait.
 template <int BN>
-__device__ __forceinline__ void fwd_scales(const NF4Group& g, int s, int n0, int N, int kbw, int gtid, float* s2) {
+__device__ __forceinline__ void fwd_scales(const NF4Group& g, int s, int n0, int N, int kbw, int gtid, float* s2,
+                                           int* q8) {
   const NF4Seg& sg = g.seg[s];
   const long long cpr = g.cols >> 6;
 #pragma unroll
   for (int i = 0; i < (BN + GROUP_THREADS - 1) / GROUP_THREADS; ++i) {
     const int r = gtid + i * GROUP_THREADS;
     s2[i] = 0.f;
+    q8[i] = 0;
     if (r < BN && n0 + r < N) {
       const long long blk = static_cast<long long>(n0 + r - sg.row_begin) * cpr + kbw;
       s2[i] = __ldg(sg.scales + (blk >> 8));
+      q8[i] = __ldg(sg.q8 + blk);
     }
   }
 }
 template <int BN>
-__device__ __forceinline__ void dx_scales(const NF4Group& g, int s, int n0, int N, int k0, int gtid, float* s2) {
+__device__ __forceinline__ void dx_scales(const NF4Group& g, int s, int n0, int N, int k0, int gtid, float* s2,
+                                          int* q8) {
   const NF4Seg& sg = g.seg[s];
   const long long cpr = g.cols >> 6;
   constexpr int NB = BN / 64;
@@ -326,18 +324,20 @@ __device__ __forceinline__ void dx_scales(const NF4Group& g, int s, int n0, int 
   for (int i = 0; i < (64 * NB + GROUP_THREADS - 1) / GROUP_THREADS; ++i) {
     const int u = gtid + i * GROUP_THREADS;
     s2[i] = 0.f;
+    q8[i] = 0;
     const int kr = u / NB, b = u % NB;
     if (u < 64 * NB && n0 + b * 64 < N) {
       const long long blk = static_cast<long long>(k0 + kr - sg.row_begin) * cpr + ((n0 + b * 64) >> 6);
       s2[i] = __ldg(sg.scales + (blk >> 8));
+      q8[i] = __ldg(sg.q8 + blk);
     }
   }
 }
 
 template <int BN>
 __device__ __forceinline__ void decode_fwd_raw(const NF4Group& g, int s, const float (&cb)[16], const float* seg_mean,
-                                               int n0, int N, int kbw, const uint8_t* raw_codes, int code_stride,
-                                               const uint8_t* raw_q8, uint8_t* tile, int gtid, const float* s2) {
+                                               int n0, int N, const uint8_t* raw_codes, int code_stride,
+                                               uint8_t* tile, int gtid, const float* s2, const int* q8r) {
   const float mean = seg_mean[s];
 #pragma unroll
   for (int i = 0; i < (BN + GROUP_THREADS - 1) / GROUP_THREADS; ++i) {
@@ -348,8 +348,7 @@ __device__ __forceinline__ void decode_fwd_raw(const NF4Group& g, int s, const f
       const uint32_t rc = smem_u32(raw_codes) + r * code_stride;
       const uint4 w0 = lds128(rc);
       const uint4 w1 = lds128(rc + 16);
-      const int q8 = lds_s8(smem_u32(raw_q8) + r * 16 + (kbw & 15));
-      const float mh = __fadd_rn(__fmul_rn(static_cast<float>(q8), s2[i]), mean);
+      const float mh = __fadd_rn(__fmul_rn(static_cast<float>(q8r[i]), s2[i]), mean);
       const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
       const BlockLut t = block_lut(cb, mh);
 #pragma unroll
@@ -367,8 +366,8 @@ __device__ __forceinline__ void decode_fwd_raw(const NF4Group& g, int s, const f
 // consecutive n of one k (= one 128-byte swizzle row, 8 conflict-free 16-byte stores).
 template <int BN>
 __device__ __forceinline__ void decode_dx_raw(const NF4Group& g, int s, const float (&cb)[16], const float* seg_mean,
-                                              int n0, int N, int k0, int xq, const uint8_t* raw_codes,
-                                              const uint8_t* raw_q8, uint8_t* tile, int gtid, const float* s2) {
+                                              int n0, int N, int k0, const uint8_t* raw_codes, uint8_t* tile,
+                                              int gtid, const float* s2, const int* q8r) {
   constexpr int NB = BN / 64;  // absmax blocks per W row in the tile
   const float mean = seg_mean[s];
 #pragma unroll
@@ -382,9 +381,7 @@ __device__ __forceinline__ void decode_dx_raw(const NF4Group& g, int s, const fl
       const uint32_t rc = smem_u32(raw_codes) + kr * (BN / 2) + b * 32;
       const uint4 w0 = lds128(rc);
       const uint4 w1 = lds128(rc + 16);
-      const int bcol = n >> 6;
-      const int q8 = lds_s8(smem_u32(raw_q8) + kr * 16 + (bcol - xq));
-      const float mh = __fadd_rn(__fmul_rn(static_cast<float>(q8), s2[i]), mean);
+      const float mh = __fadd_rn(__fmul_rn(static_cast<float>(q8r[i]), s2[i]), mean);
       const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
       const BlockLut t = block_lut(cb, mh);
 #pragma unroll
@@ -555,14 +552,15 @@ struct ScaleRegs {
   static constexpr int NF = (BN + GROUP_THREADS - 1) / GROUP_THREADS;
   static constexpr int ND = (64 * (BN / 64) + GROUP_THREADS - 1) / GROUP_THREADS;
   static constexpr int N = NF > ND ? NF : ND;
-  float v[N];
+  float v[N];  // group scales s2
+  int q[N];    // double-quantised absmax q8
 };
 template <int BN>
 __device__ __forceinline__ void load_scales(const GemmParams& p, bool fwd, int n0, int kk, int gtid, ScaleRegs<BN>& r) {
   if (fwd)
-    fwd_scales<BN>(p.nf4, nf4_seg_of(p.nf4, n0), n0, p.N, kk, gtid, r.v);
+    fwd_scales<BN>(p.nf4, nf4_seg_of(p.nf4, n0), n0, p.N, kk, gtid, r.v, r.q);
   else
-    dx_scales<BN>(p.nf4, nf4_seg_of(p.nf4, kk * BK), n0, p.N, kk * BK, gtid, r.v);
+    dx_scales<BN>(p.nf4, nf4_seg_of(p.nf4, kk * BK), n0, p.N, kk * BK, gtid, r.v, r.q);
 }
 
 // ---------------------------------------------------------------- work pieces
@@ -701,16 +699,15 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
           const int rs = rb % C::RAW_SLOTS;
           const uint32_t rph = static_cast<uint32_t>(rb / C::RAW_SLOTS) & 1u;
           const uint8_t* Rc = raw_base + rs * C::RAW_BYTES;
-          const uint8_t* Rq = Rc + C::RAW_CODE_BYTES;
           mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, p.err);
           mbar_wait_bounded(&raw_full[rs], rph, abort_flag, p.err);
           if (fwd) {
-            decode_fwd_raw<BN>(p.nf4, nf4_seg_of(p.nf4, n0), cb, seg_mean, n0, p.N, kk, Rc + sub * 32, 32 * rk, Rq, Bs,
-                               gtid, cur.v);
+            decode_fwd_raw<BN>(p.nf4, nf4_seg_of(p.nf4, n0), cb, seg_mean, n0, p.N, Rc + sub * 32, 32 * rk, Bs, gtid,
+                               cur.v, cur.q);
           } else {
             const int k0 = kk * BK;
-            decode_dx_raw<BN>(p.nf4, nf4_seg_of(p.nf4, k0), cb, seg_mean, n0, p.N, k0, ((n0 >> 6) >> 4) << 4,
-                              Rc + sub * 64 * (BN / 2), Rq + sub * 64 * 16, Bs, gtid, cur.v);
+            decode_dx_raw<BN>(p.nf4, nf4_seg_of(p.nf4, k0), cb, seg_mean, n0, p.N, k0, Rc + sub * 64 * (BN / 2), Bs,
+                              gtid, cur.v, cur.q);
           }
           __syncwarp();
           // this warp's reads of the raw slot are done; the last k-block of a chunk this piece
@@ -815,8 +812,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
       }
       if (warp == EPI_WARP0 + 2 && lane == 0 && n_raw > 0) {
         // ---------------------------------------------- TMA issuer: raw NF4 codes / absmax
-        // one codes copy and one absmax copy per chunk of rk k-blocks (chunks aligned to
-        // multiples of rk; a piece's first and last chunk may reach outside it)
+        // one codes copy per chunk of rk k-blocks (chunks aligned to multiples of rk; a piece's
+        // first and last chunk may reach outside it); the absmax bytes are loaded by the
+        // producers themselves, a k-block ahead, with the group scales
         const GemmSeg& sg = p.seg[0];
         const int rk = p.raw_k, ch0 = kb_lo / rk, nch = (kb_lo + n_raw - 1) / rk - ch0 + 1;
         for (int c = 0; c < nch; ++c) {
@@ -826,20 +824,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
           const uint32_t rph = static_cast<uint32_t>(rb / C::RAW_SLOTS) & 1u;
           mbar_wait_bounded(&raw_empty[rs], rph ^ 1u, abort_flag, p.err);
           uint8_t* Rc = raw_base + rs * C::RAW_BYTES;
-          uint8_t* Rq = Rc + C::RAW_CODE_BYTES;
           if (sg.B.kind == OP_NF4_K) {
             const int si = nf4_seg_of(p.nf4, n0);
             const int y = n0 - p.nf4.seg[si].row_begin;
-            mbar_arrive_expect_tx(&raw_full[rs], BN * 32 * rk + BN * 16);
+            mbar_arrive_expect_tx(&raw_full[rs], BN * 32 * rk);
             tma_load_2d(Rc, &p.tmapCodes[si], kk0 * (BK / 2), y, &raw_full[rs]);
-            tma_load_2d(Rq, &p.tmapQ8[si], (kk0 >> 4) << 4, y, &raw_full[rs]);
           } else {
             const int k0 = kk0 * BK;
             const int si = nf4_seg_of(p.nf4, k0);
             const int y = k0 - p.nf4.seg[si].row_begin;
-            mbar_arrive_expect_tx(&raw_full[rs], 64 * rk * (BN / 2) + 64 * rk * 16);
+            mbar_arrive_expect_tx(&raw_full[rs], 64 * rk * (BN / 2));
             tma_load_2d(Rc, &p.tmapCodes[si], n0 / 2, y, &raw_full[rs]);
-            tma_load_2d(Rq, &p.tmapQ8[si], ((n0 >> 6) >> 4) << 4, y, &raw_full[rs]);
           }
         }
       }
@@ -1230,14 +1225,12 @@ bool setup_raw_tma(GemmParams& p, int BN, int rawk_max) {
       rk >>= 1;
     }
   p.raw_k = rk;
-  const unsigned long long cb = static_cast<unsigned long long>(g.cols) / 2, qb = static_cast<unsigned long long>(g.cols) / 64;
+  const unsigned long long cb = static_cast<unsigned long long>(g.cols) / 2;
   for (int i = 0; i < g.nseg; ++i) {
     const unsigned long long rows = static_cast<unsigned long long>(g.seg[i].rows);
     const bool ok = (s0.B.kind == OP_NF4_K)
-                        ? (encode_u8_2d(&p.tmapCodes[i], g.seg[i].codes, cb, rows, cb, 32 * rk, BN) &&
-                           encode_u8_2d(&p.tmapQ8[i], g.seg[i].q8, qb, rows, qb, 16, BN))
-                        : (encode_u8_2d(&p.tmapCodes[i], g.seg[i].codes, cb, rows, cb, BN / 2, 64 * rk) &&
-                           encode_u8_2d(&p.tmapQ8[i], g.seg[i].q8, qb, rows, qb, 16, 64 * rk));
+                        ? encode_u8_2d(&p.tmapCodes[i], g.seg[i].codes, cb, rows, cb, 32 * rk, BN)
+                        : encode_u8_2d(&p.tmapCodes[i], g.seg[i].codes, cb, rows, cb, BN / 2, 64 * rk);
     if (!ok) return false;
   }
   return true;

@@ -60,7 +60,6 @@ struct GemmParams {
   CUtensorMap tmapA[GEMM_MAX_SEG];  // TMA descriptors of bf16 A operands
   CUtensorMap tmapB[GEMM_MAX_SEG];  // TMA descriptors of bf16 B operands
   CUtensorMap tmapCodes[3];         // TMA descriptors of each NF4 tensor's packed codes (raw staging)
-  CUtensorMap tmapQ8[3];            // ... and of its q8 absmax
   int a_mode[GEMM_MAX_SEG];         // 0: producer warps load A; 1: TMA, K-major; 2: TMA, MN-major
   int b_mode[GEMM_MAX_SEG];         // same for B (bf16 operands only)
   int b_row0[GEMM_MAX_SEG];         // first operand row of the B descriptor (block-diagonal windows)
