@@ -150,15 +150,23 @@ typedef struct soup_batch {
 
 /* Creates a model: validates cfg, computes the NF4 codebook, allocates the page-locked host
  * layer stack (n_layers blobs), the device layer buffers (n_layers resident, n_layer_buffers
- * streamed), activation storage for max_tokens and scratch.  Weights are loaded afterwards. */
+ * streamed), activation storage for max_tokens and scratch.  Weights are loaded afterwards.
+ * The host-side stack and the few device layer buffers are the pages' layer streaming: the
+ * base lives in CPU RAM (or on disk, stream_source) and the GPU holds one layer at a time
+ * plus the adapters (rug.gal radar "Soup ... layer streaming", "En detalle"; imasters "Como
+ * cabe um 8B em 4 GB").  SOUP_ERR_UNSUPPORTED for shapes outside the kernels, SOUP_ERR_OOM
+ * when an allocation (or the caller's allocator) fails; nothing is leaked on failure.
+ * soup_model_destroy frees everything the model holds (NULL: SOUP_ERR_INVALID_ARG). */
 soup_status soup_model_create(const soup_model_config* cfg, const soup_allocator* alloc, soup_model** out);
 soup_status soup_model_destroy(soup_model* model);
 
 /* Bytes of one layer's NF4 blob (7 projections: codes, q8 absmax, fp32 group scales, fp32
- * mean; then the two bf16 RMSNorm gains), each part 256-byte aligned. */
+ * mean; then the two bf16 RMSNorm gains), each part 256-byte aligned: the unit the streamer
+ * moves (rug.gal "En detalle": one decoder layer is loaded, used and dropped). */
 soup_status soup_layer_blob_bytes(const soup_model_config* cfg, size_t* bytes);
 
-/* Quantises one layer on the device into the model's host layer stack.
+/* Quantises one layer on the device into the model's host layer stack (NF4, the pages'
+ * `quantization: 4bit`: guillermodelpino soup.yaml example; rug.gal "En detalle").
  * w[p]: device fp32 [out_p, in_p] row-major for p = q,k,v,o,gate,up,down; gammas: device bf16
  * [hidden].  Runs the NF4 + double-quant kernels, then copies the blob to page-locked host
  * memory (synchronises `stream`).  In resident mode the blob is also kept on the device. */
@@ -176,7 +184,10 @@ soup_status soup_model_quantize_layer(soup_model* model, int layer, const float*
  * index; SOUP_ERR_IO when the stack file cannot be written. */
 soup_status soup_model_load_layer(soup_model* model, int layer, const float* const w[7], const uint16_t* gamma_attn,
                                   const uint16_t* gamma_mlp);
-/* Loads / reads back a pre-quantised blob (host memory, soup_layer_blob_bytes bytes). */
+/* Loads / reads back a pre-quantised blob (host memory, soup_layer_blob_bytes bytes) into or
+ * out of the model's host layer stack (the CPU-RAM or disk copy the pages stream from: rug.gal
+ * "En detalle"; imasters "Como cabe um 8B em 4 GB").  Synchronous.  SOUP_ERR_INVALID_ARG for
+ * a bad layer index or a size other than soup_layer_blob_bytes; SOUP_ERR_IO on a file error. */
 soup_status soup_model_load_layer_nf4(soup_model* model, int layer, const void* blob, size_t bytes);
 soup_status soup_model_read_layer_nf4(soup_model* model, int layer, void* blob, size_t bytes);
 /* Byte offset and size of a part of projection p inside a layer blob; part 0 = codes, 1 = q8
@@ -184,10 +195,12 @@ soup_status soup_model_read_layer_nf4(soup_model* model, int layer, void* blob, 
 soup_status soup_layer_blob_part(const soup_model_config* cfg, int proj, int part, size_t* offset, size_t* bytes);
 
 /* Frozen head weights (device, bf16, caller-owned, kept by pointer): embedding [vocab, hidden],
- * final RMSNorm gain [hidden], lm_head [vocab, hidden]. */
+ * final RMSNorm gain [hidden], lm_head [vocab, hidden].  They stay resident: the pages stream
+ * the decoder layers only (rug.gal "En detalle"). */
 soup_status soup_model_set_head(soup_model* model, const void* embed, const void* final_gamma, const void* lm_head);
 
-/* LoRA storage: four caller-owned device fp32 buffers of soup_lora_numel elements each
+/* LoRA storage (the trained adapters, which stay in VRAM: rug.gal "En detalle"; guillermodelpino
+ * soup.yaml example, r and alpha): four caller-owned device fp32 buffers of soup_lora_numel elements each
  * (parameters, gradients, AdamW first and second moments; moments start at zero).  Layout:
  * layer-major; inside a layer A_q, A_k, A_v, A_o, A_gate, A_up, A_down (each [r, in]) then
  * B_q, ..., B_down (each [out, r]), row-major.  soup_lora_offset gives each tensor's place. */
@@ -210,7 +223,9 @@ soup_status soup_model_set_lora_proj(soup_model* model, int layer, int proj, con
 soup_status soup_model_refresh_lora(soup_model* model, void* stream);
 
 /* LoRA on/off for the forward and backward calls that follow.  Off: the LoRA branch and its
- * gradients are skipped entirely (not multiplied by zero), which is the DPO reference model. */
+ * gradients are skipped entirely (not multiplied by zero), which is the DPO reference model:
+ * the same base stream with the adapters switched off (rug.gal "En detalle"; imasters "Do SFT
+ * para os métodos de preferência").  Always SOUP_OK for a valid model. */
 soup_status soup_set_lora_enabled(soup_model* model, int enabled);
 
 /* Merged weight of one projection: out = bf16(W + (lora_alpha / lora_r) * B * A), device bf16
@@ -229,32 +244,41 @@ soup_status soup_model_merge_lora(soup_model* model, int layer, int proj, void* 
 
 /* One decoder layer forward: x_out = layer(x_in), device bf16 [B*S, hidden].  Acquires the
  * layer from the streamer (or the resident copy), keeps the activations needed by
- * soup_layer_bwd inside the model (per layer), runs every kernel on `stream`. */
+ * soup_layer_bwd inside the model (per layer), runs every kernel on `stream`.  The layer is
+ * the Llama-3.1-8B decoder layer the pages stream one at a time (rug.gal lead and "En
+ * detalle"; guillermodelpino "El streaming de capas, que es el truco de la casa"). */
 soup_status soup_layer_fwd(soup_model* model, int layer, const void* x_in, void* x_out, int B, int S, void* stream);
 /* Backward of the last soup_layer_fwd of this layer: dx = d(loss)/d(x_in) given
  * dy = d(loss)/d(x_out) (device bf16 [B*S, hidden]); ACCUMULATES the layer's LoRA gradients
- * into the grad buffer (callers zero it first).  SOUP_ERR_STATE without a matching forward. */
+ * into the grad buffer (callers zero it first); the base gets no gradient, it is frozen
+ * (rug.gal "En detalle").  SOUP_ERR_STATE without a matching forward. */
 soup_status soup_layer_bwd(soup_model* model, int layer, const void* dy, void* dx, int B, int S, void* stream);
 
 /* ---- whole step -------------------------------------------------------------------------- */
 
 /* One training step: embedding, streamed forward over all layers, head and loss, streamed
- * backward, LoRA gradients (zeroed first) and, if batch->apply_optimizer, the AdamW update.
+ * backward, LoRA gradients (zeroed first) and, if batch->apply_optimizer, the AdamW update
+ * (the pages' SFT and preference training under layer streaming: rug.gal "En detalle";
+ * imasters "Do SFT para os métodos de preferência"; guillermodelpino soup.yaml example, lr).
  * SFT streams 2L-2 layer loads from a cold streamer (the two top layers are reused at the
  * forward/backward turnaround); DPO and KTO add a full LoRA-off forward pass, 3L-2 loads
  * (2L-2 with dpo_shared_load); SimPO and ORPO stream like SFT.  Layers
  * still resident from the previous step are reused.  *loss_out (host) receives the loss
  * after the call synchronises `stream`. */
 soup_status soup_step(soup_model* model, soup_loss loss, const soup_batch* batch, float* loss_out, void* stream);
-/* AdamW update of all LoRA parameters from the grad buffer (step counter kept by the model). */
+/* AdamW update of all LoRA parameters from the grad buffer (step counter kept by the model);
+ * the pages give only the learning rate (guillermodelpino soup.yaml example). */
 soup_status soup_optimizer_step(soup_model* model, float lr, void* stream);
 /* Per-sequence summed target log-probs of the last preference step (host fp32[B]): policy
- * and ref (ref is written by DPO and KTO only). */
+ * and ref (ref is written by DPO and KTO only; it comes from the LoRA-off re-stream: rug.gal
+ * "En detalle").  Copies the first n entries (1 <= n <= max_tokens, else SOUP_ERR_INVALID_ARG);
+ * synchronous; entries no preference step has written are unspecified. */
 soup_status soup_last_logps(soup_model* model, float* pi, float* ref, int n);
 
 /* ---- single operations (each one kernel sequence, for tests and tools) ------------------- */
 
-/* NF4 + double quantisation of one device fp32 tensor of n elements (row-major flattened):
+/* NF4 + double quantisation (the pages' `quantization: 4bit`: guillermodelpino soup.yaml
+ * example; rug.gal "En detalle") of one device fp32 tensor of n elements (row-major flattened):
  * codes [ceil(n/2)] u8, q8 [ceil(n/64)] i8, scales [ceil(n/64/256)] f32, mean [1] f32, all
  * device; scratch: device f32 [ceil(n/64)] (absmax). */
 soup_status soup_nf4_quantize(const float* w, long long n, uint8_t* codes, int8_t* q8, float* scales, float* mean,
@@ -284,10 +308,12 @@ soup_status soup_nf4_quantize_static(const float* w, long long n, uint8_t* codes
  * (guillermodelpino soup.yaml example; rug.gal "En detalle"). */
 soup_status soup_nf4_quantize_host(const float* w, long long n, uint8_t* codes, int8_t* q8, float* scales, float* mean,
                                    int n_threads);
-/* Standalone NF4 -> bf16 dequantiser: out[i] = bf16_rn(c[code_i] * mhat(block(i))). */
+/* Standalone NF4 -> bf16 dequantiser: out[i] = bf16_rn(c[code_i] * mhat(block(i))), the
+ * decode every streamed GEMM applies to the 4-bit base (rug.gal "En detalle"). */
 soup_status soup_nf4_dequantize(const uint8_t* codes, const int8_t* q8, const float* scales, const float* mean,
                                 long long n, uint16_t* out, void* stream);
-/* y[M, N] (bf16) = x[M, K] (bf16) . W^T + (residual) for one NF4 tensor W [N, K] (device
+/* The streamed layer's projection on its own (rug.gal "En detalle": the 4-bit base is used
+ * as it arrives): y[M, N] (bf16) = x[M, K] (bf16) . W^T + (residual) for one NF4 tensor W [N, K] (device
  * parts as produced by soup_nf4_quantize); transpose_w != 0 computes y[M, K] = x[M, N] . W.
  * The first call on a device allocates a 64 MiB workspace and tile counters for the
  * stream-K schedule, shared by later calls on that device: calls that overlap on the GPU
@@ -319,10 +345,14 @@ soup_status soup_gemm_stream_k_pieces(long long tiles, int kblocks_per_tile, int
 soup_status soup_gemm_stream_k_shares(long long tiles, int kblocks_per_tile, int ctas, int tile, int max_shares,
                                       int* cta, int* slot, int* n_shares);
 
-/* The 16 NF4 levels this library uses (host fp32[16]). */
+/* The 16 NF4 levels this library uses (host fp32[16]): the NormalFloat-4 code of the pages'
+ * `quantization: 4bit` (guillermodelpino soup.yaml example), Dettmers et al. 2023. */
 soup_status soup_nf4_codebook(float* out16);
 
 /* ---- diagnostics ------------------------------------------------------------------------- */
+/* The pages define none of these; they measure the library's own work.  The link the probe
+ * times is the cost the pages name for streaming (guillermodelpino "Cuándo no te compensa":
+ * moving layers costs speed). */
 /* Host-to-device link probe: copies the model's page-locked layer-0 blob into a device layer
  * buffer `reps` times back to back on the streamer's copy stream (the exact path the streamer
  * uses) and returns the achieved GB/s (1e9 bytes/s) in *gbs.  Synchronises; the buffer used is
@@ -382,7 +412,8 @@ soup_status soup_get_timed_profile(soup_model* model, soup_profile_entry* out, i
  * soup_step) then reports SOUP_ERR_TIMEOUT once, clears the word, and the model stays usable.
  * The pages have no counterpart: this is the library's own fault reporting. */
 soup_status soup_selftest_bounded_wait(soup_model* model, int limit_us, void* stream);
-/* Reads (and clears) the device error word; SOUP_ERR_TIMEOUT / SOUP_ERR_DEVICE_CHECK if set. */
+/* Reads (and clears) the device error word; SOUP_ERR_TIMEOUT / SOUP_ERR_DEVICE_CHECK if set.
+ * Synchronises `stream`.  The library's own fault reporting (no page counterpart). */
 soup_status soup_check_device(soup_model* model, void* stream);
 const char* soup_status_string(soup_status status);
 const char* soup_last_error(const soup_model* model);

@@ -14,7 +14,7 @@
 //
 // Warp roles (192 threads): warps 0-3 softmax and epilogue (TMEM lane quarters 0-3, thread = query
 // row), warp 4 allocates TMEM and its lane 0 issues the MMAs, warp 5 lane 0 issues the TMA loads
-// (Q once, K/V tiles in a 2-stage ring).  Every wait is bounded (mbar_wait_bounded): on timeout the
+// (Q once, K/V tiles in a 2-stage ring; one 3D copy per [128 rows x d] tile).  Every wait is bounded (mbar_wait_bounded): on timeout the
 // device error word is set and the kernel runs to its end.
 //
 // Key tiles a query tile reads: those with a visible (query, key) pair (attn_mask.cuh); the plain
@@ -107,22 +107,15 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
     if (lane == 0) {
       constexpr uint32_t TB = C::TILE_BYTES;
       mbar_arrive_expect_tx(q_full, TB);
-#pragma unroll
-      for (int c = 0; c < D / 64; ++c)
-        tma_load_2d(base + C::Q_OFF + c * 16384, &tmap, h * D + c * 64, row0 + qt * TQ, q_full);
+      tma_load_3d(base + C::Q_OFF, &tmap, 0, row0 + qt * TQ, h * (D / 64), q_full);
       int jj = 0;
       for (int j = 0; j < ntk; ++j) {
         if (!kv_needed(s, qt, j)) continue;
         const int st = jj & 1;
         mbar_wait_bounded(&kv_empty[st], ((jj >> 1) & 1) ^ 1u, abort_flag, err);
         mbar_arrive_expect_tx(&kv_full[st], 2 * TB);
-#pragma unroll
-        for (int c = 0; c < D / 64; ++c) {
-          tma_load_2d(base + C::K_OFF + st * TB + c * 16384, &tmap, (s.hq + g) * D + c * 64, row0 + j * TK,
-                      &kv_full[st]);
-          tma_load_2d(base + C::V_OFF + st * TB + c * 16384, &tmap, (s.hq + s.hkv + g) * D + c * 64, row0 + j * TK,
-                      &kv_full[st]);
-        }
+        tma_load_3d(base + C::K_OFF + st * TB, &tmap, 0, row0 + j * TK, (s.hq + g) * (D / 64), &kv_full[st]);
+        tma_load_3d(base + C::V_OFF + st * TB, &tmap, 0, row0 + j * TK, (s.hq + s.hkv + g) * (D / 64), &kv_full[st]);
         ++jj;
       }
     }
@@ -274,10 +267,11 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
 template <int D>
 cudaError_t launch_fwd(const AttnShape& s, const uint16_t* qkv, uint16_t* o, float* lse, int* err, cudaStream_t st) {
   using C = FwdCfg<D>;
+  // one copy per [128 rows x D] tile: the head's D/64 column blocks as the planes of a 3D map
   CUtensorMap map;
-  const unsigned long long cols = static_cast<unsigned long long>(s.hq + 2 * s.hkv) * D;
+  const unsigned long long planes = static_cast<unsigned long long>(s.hq + 2 * s.hkv) * (D / 64);
   const unsigned long long rows = static_cast<unsigned long long>(s.B) * s.S;
-  if (!tma_encode_bf16_sw128(&map, qkv, cols, rows, static_cast<unsigned long long>(s.ld_qkv) * 2, 64, TQ))
+  if (!tma_encode_bf16_sw128_planes(&map, qkv, rows, planes, static_cast<unsigned long long>(s.ld_qkv) * 2, TQ, D / 64))
     return cudaErrorInvalidValue;
   static bool attr = false;
   if (!attr) {
@@ -460,11 +454,8 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
   if (warp == TMA_WARP) {
     if (lane == 0) {
       mbar_arrive_expect_tx(kv_full, 2 * TB);
-#pragma unroll
-      for (int c = 0; c < D / 64; ++c) {
-        tma_load_2d(Ks + c * 16384, &tq, (s.hq + g) * D + c * 64, row0 + j * TK, kv_full);
-        tma_load_2d(Vs + c * 16384, &tq, (s.hq + s.hkv + g) * D + c * 64, row0 + j * TK, kv_full);
-      }
+      tma_load_3d(Ks, &tq, 0, row0 + j * TK, (s.hq + g) * (D / 64), kv_full);
+      tma_load_3d(Vs, &tq, 0, row0 + j * TK, (s.hq + s.hkv + g) * (D / 64), kv_full);
       int it = 0;
       for (int hh = 0; hh < hper; ++hh)
         for (int i = 0; i < nqt; ++i) {
@@ -472,11 +463,8 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
           const int h = h0 + hh, st = it & 1;
           mbar_wait_bounded(&qd_empty[st], ((it >> 1) & 1) ^ 1u, abort_flag, err);
           mbar_arrive_expect_tx(&qd_full[st], 2 * TB);
-#pragma unroll
-          for (int c = 0; c < D / 64; ++c) {
-            tma_load_2d(Qs + st * TB + c * 16384, &tq, h * D + c * 64, row0 + i * TQ, &qd_full[st]);
-            tma_load_2d(dOs + st * TB + c * 16384, &tdo, h * D + c * 64, row0 + i * TQ, &qd_full[st]);
-          }
+          tma_load_3d(Qs + st * TB, &tq, 0, row0 + i * TQ, h * (D / 64), &qd_full[st]);
+          tma_load_3d(dOs + st * TB, &tdo, 0, row0 + i * TQ, h * (D / 64), &qd_full[st]);
           ++it;
         }
     }
@@ -672,22 +660,16 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
   if (warp == TMA_WARP) {
     if (lane == 0) {
       mbar_arrive_expect_tx(q_full, 2 * TB);
-#pragma unroll
-      for (int c = 0; c < D / 64; ++c) {
-        tma_load_2d(Qs + c * 16384, &tq, h * D + c * 64, row0 + qt * TQ, q_full);
-        tma_load_2d(dOs + c * 16384, &tdo, h * D + c * 64, row0 + qt * TQ, q_full);
-      }
+      tma_load_3d(Qs, &tq, 0, row0 + qt * TQ, h * (D / 64), q_full);
+      tma_load_3d(dOs, &tdo, 0, row0 + qt * TQ, h * (D / 64), q_full);
       int jj = 0;
       for (int j = 0; j < ntk; ++j) {
         if (!kv_needed(s, qt, j)) continue;
         const int st = jj & 1;
         mbar_wait_bounded(&kv_empty[st], ((jj >> 1) & 1) ^ 1u, abort_flag, err);
         mbar_arrive_expect_tx(&kv_full[st], 2 * TB);
-#pragma unroll
-        for (int c = 0; c < D / 64; ++c) {
-          tma_load_2d(Ks + st * TB + c * 16384, &tq, (s.hq + g) * D + c * 64, row0 + j * TK, &kv_full[st]);
-          tma_load_2d(Vs + st * TB + c * 16384, &tq, (s.hq + s.hkv + g) * D + c * 64, row0 + j * TK, &kv_full[st]);
-        }
+        tma_load_3d(Ks + st * TB, &tq, 0, row0 + j * TK, (s.hq + g) * (D / 64), &kv_full[st]);
+        tma_load_3d(Vs + st * TB, &tq, 0, row0 + j * TK, (s.hq + s.hkv + g) * (D / 64), &kv_full[st]);
         ++jj;
       }
     }
@@ -800,10 +782,10 @@ cudaError_t launch_bwd(const AttnShape& s, const uint16_t* qkv, const uint16_t* 
   using C = BwdCfg<D>;
   CUtensorMap tq, tdo;
   const unsigned long long rows = static_cast<unsigned long long>(s.B) * s.S;
-  if (!tma_encode_bf16_sw128(&tq, qkv, static_cast<unsigned long long>(s.hq + 2 * s.hkv) * D, rows,
-                             static_cast<unsigned long long>(s.ld_qkv) * 2, 64, 128) ||
-      !tma_encode_bf16_sw128(&tdo, dout, static_cast<unsigned long long>(s.hq) * D, rows,
-                             static_cast<unsigned long long>(s.hq) * D * 2, 64, 128))
+  if (!tma_encode_bf16_sw128_planes(&tq, qkv, rows, static_cast<unsigned long long>(s.hq + 2 * s.hkv) * (D / 64),
+                                    static_cast<unsigned long long>(s.ld_qkv) * 2, 128, D / 64) ||
+      !tma_encode_bf16_sw128_planes(&tdo, dout, rows, static_cast<unsigned long long>(s.hq) * (D / 64),
+                                    static_cast<unsigned long long>(s.hq) * D * 2, 128, D / 64))
     return cudaErrorInvalidValue;
   static bool attr = false;
   if (!attr) {

@@ -48,9 +48,6 @@ constexpr int GROUP_THREADS = 128;
 constexpr int UM = 128;  // rows of one tcgen05.mma (cta_group::1); a CTA tile stacks MT of them
 constexpr int BK = 64;   // 64 bf16 = 128 bytes = one swizzle row
 constexpr int SMEM_LIMIT = 232448;  // 227 KiB of dynamic shared memory per CTA
-#ifndef SOUP_GEMM_RAWK
-#define SOUP_GEMM_RAWK 4  // k-blocks per raw NF4 slot
-#endif
 
 template <int MT, int BN>
 struct GemmCfg {
@@ -58,18 +55,17 @@ struct GemmCfg {
   static constexpr int A_BYTES = BM * 128;
   static constexpr int B_BYTES = BN * 128;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // one k-block of both MMA operands
-  // Raw NF4 codes staged by TMA in a ring of their own, RAWK k-blocks per slot: BN x 32 RAWK B
-  // (forward) or 64 RAWK x BN/2 B (transposed).  A TMA copy costs a SM's copy engine about the
-  // same time whatever its size (measured on B200: ~280 ns for a 16 B x 128-row box and for a
-  // 32 KB box alike), so the raw codes come in one copy per RAWK k-blocks and the absmax bytes
-  // by plain loads in the producers, which leaves the copy engine to the activation tiles.  A
-  // slot is released as soon as its k-blocks are dequantised.
-  static constexpr int RAWK = SOUP_GEMM_RAWK;
-  static constexpr int RAW_CODE_BYTES = BN * 32 * RAWK;
-  static constexpr int RAW_BYTES = RAW_CODE_BYTES;
+  // Raw NF4 staging (TMA) in a ring of its own: codes BN x 32 B (forward) or 64 x BN/2 B
+  // (transposed), q8 absmax BN x 16 B or 64 x 16 B.  A raw slot is released as soon as its
+  // k-block is dequantised, so the raw loads run several k-blocks ahead of the operand stages.
+  // (Batching four k-blocks of codes per copy, with the q8 bytes loaded by the producers,
+  // measured 5-13 % slower on the 8B projection shapes at 512 rows.)
+  static constexpr int RAW_CODE_BYTES = BN * 32;
+  static constexpr int RAW_Q8_BYTES = (BN > 64 ? BN : 64) * 16;
+  static constexpr int RAW_BYTES = RAW_CODE_BYTES + RAW_Q8_BYTES;
   static constexpr int CTRL_BYTES = 640;
   static constexpr int AVAIL = SMEM_LIMIT - 1024 - CTRL_BYTES;
-  static constexpr int STAGES_FIT = (AVAIL - 2 * RAW_BYTES) / STAGE_BYTES;
+  static constexpr int STAGES_FIT = (AVAIL - 4 * RAW_BYTES) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
   static constexpr int RAW_FIT = (AVAIL - STAGES * STAGE_BYTES) / RAW_BYTES;
   static constexpr int RAW_SLOTS = RAW_FIT > 16 ? 16 : RAW_FIT;
@@ -243,6 +239,11 @@ __device__ __forceinline__ uint4 lds128(uint32_t a) {
   asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
   return v;
 }
+__device__ __forceinline__ int lds_s8(uint32_t a) {
+  int v;
+  asm volatile("ld.shared.s8 %0, [%1];" : "=r"(v) : "r"(a));
+  return v;
+}
 __device__ __forceinline__ void sts128(uint32_t a, const uint4& v) {
   asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
 }
@@ -298,25 +299,21 @@ __device__ __forceinline__ uint4 decode_word_lut(uint32_t c, const BlockLut& t) 
 // Group scales (s2) of the absmax blocks a thread decodes in one k-block, loaded before the
 // thread waits for the raw tile so their latency overlaps the wait.
 template <int BN>
-__device__ __forceinline__ void fwd_scales(const NF4Group& g, int s, int n0, int N, int kbw, int gtid, float* s2,
-                                           int* q8) {
+__device__ __forceinline__ void fwd_scales(const NF4Group& g, int s, int n0, int N, int kbw, int gtid, float* s2) {
   const NF4Seg& sg = g.seg[s];
   const long long cpr = g.cols >> 6;
 #pragma unroll
   for (int i = 0; i < (BN + GROUP_THREADS - 1) / GROUP_THREADS; ++i) {
     const int r = gtid + i * GROUP_THREADS;
     s2[i] = 0.f;
-    q8[i] = 0;
     if (r < BN && n0 + r < N) {
       const long long blk = static_cast<long long>(n0 + r - sg.row_begin) * cpr + kbw;
       s2[i] = __ldg(sg.scales + (blk >> 8));
-      q8[i] = __ldg(sg.q8 + blk);
     }
   }
 }
 template <int BN>
-__device__ __forceinline__ void dx_scales(const NF4Group& g, int s, int n0, int N, int k0, int gtid, float* s2,
-                                          int* q8) {
+__device__ __forceinline__ void dx_scales(const NF4Group& g, int s, int n0, int N, int k0, int gtid, float* s2) {
   const NF4Seg& sg = g.seg[s];
   const long long cpr = g.cols >> 6;
   constexpr int NB = BN / 64;
@@ -324,20 +321,18 @@ __device__ __forceinline__ void dx_scales(const NF4Group& g, int s, int n0, int 
   for (int i = 0; i < (64 * NB + GROUP_THREADS - 1) / GROUP_THREADS; ++i) {
     const int u = gtid + i * GROUP_THREADS;
     s2[i] = 0.f;
-    q8[i] = 0;
     const int kr = u / NB, b = u % NB;
     if (u < 64 * NB && n0 + b * 64 < N) {
       const long long blk = static_cast<long long>(k0 + kr - sg.row_begin) * cpr + ((n0 + b * 64) >> 6);
       s2[i] = __ldg(sg.scales + (blk >> 8));
-      q8[i] = __ldg(sg.q8 + blk);
     }
   }
 }
 
 template <int BN>
 __device__ __forceinline__ void decode_fwd_raw(const NF4Group& g, int s, const float (&cb)[16], const float* seg_mean,
-                                               int n0, int N, const uint8_t* raw_codes, int code_stride,
-                                               uint8_t* tile, int gtid, const float* s2, const int* q8r) {
+                                               int n0, int N, int kbw, const uint8_t* raw_codes,
+                                               const uint8_t* raw_q8, uint8_t* tile, int gtid, const float* s2) {
   const float mean = seg_mean[s];
 #pragma unroll
   for (int i = 0; i < (BN + GROUP_THREADS - 1) / GROUP_THREADS; ++i) {
@@ -345,10 +340,11 @@ __device__ __forceinline__ void decode_fwd_raw(const NF4Group& g, int s, const f
     if (r >= BN) break;
     const uint32_t trow = smem_u32(tile) + (r >> 3) * 1024 + (r & 7) * 128;
     if (n0 + r < N) {
-      const uint32_t rc = smem_u32(raw_codes) + r * code_stride;
+      const uint32_t rc = smem_u32(raw_codes) + r * 32;
       const uint4 w0 = lds128(rc);
       const uint4 w1 = lds128(rc + 16);
-      const float mh = __fadd_rn(__fmul_rn(static_cast<float>(q8r[i]), s2[i]), mean);
+      const int q8 = lds_s8(smem_u32(raw_q8) + r * 16 + (kbw & 15));
+      const float mh = __fadd_rn(__fmul_rn(static_cast<float>(q8), s2[i]), mean);
       const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
       const BlockLut t = block_lut(cb, mh);
 #pragma unroll
@@ -366,8 +362,8 @@ __device__ __forceinline__ void decode_fwd_raw(const NF4Group& g, int s, const f
 // consecutive n of one k (= one 128-byte swizzle row, 8 conflict-free 16-byte stores).
 template <int BN>
 __device__ __forceinline__ void decode_dx_raw(const NF4Group& g, int s, const float (&cb)[16], const float* seg_mean,
-                                              int n0, int N, int k0, const uint8_t* raw_codes, uint8_t* tile,
-                                              int gtid, const float* s2, const int* q8r) {
+                                              int n0, int N, int k0, int xq, const uint8_t* raw_codes,
+                                              const uint8_t* raw_q8, uint8_t* tile, int gtid, const float* s2) {
   constexpr int NB = BN / 64;  // absmax blocks per W row in the tile
   const float mean = seg_mean[s];
 #pragma unroll
@@ -381,7 +377,9 @@ __device__ __forceinline__ void decode_dx_raw(const NF4Group& g, int s, const fl
       const uint32_t rc = smem_u32(raw_codes) + kr * (BN / 2) + b * 32;
       const uint4 w0 = lds128(rc);
       const uint4 w1 = lds128(rc + 16);
-      const float mh = __fadd_rn(__fmul_rn(static_cast<float>(q8r[i]), s2[i]), mean);
+      const int bcol = n >> 6;
+      const int q8 = lds_s8(smem_u32(raw_q8) + kr * 16 + (bcol - xq));
+      const float mh = __fadd_rn(__fmul_rn(static_cast<float>(q8), s2[i]), mean);
       const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
       const BlockLut t = block_lut(cb, mh);
 #pragma unroll
@@ -541,10 +539,6 @@ __device__ __forceinline__ void rope_store16(const GemmParams& p, int row, int c
   reinterpret_cast<uint4*>(o + half)[1] = make_uint4(w2[4], w2[5], w2[6], w2[7]);
 }
 
-__device__ __forceinline__ void mbar_arrive_cnt(uint64_t* bar, uint32_t cnt) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(cnt) : "memory");
-}
-
 // Group-scale registers of one k-block of the NF4 B tile (forward: one per row this thread
 // decodes; dX: one per absmax block).
 template <int BN>
@@ -552,15 +546,14 @@ struct ScaleRegs {
   static constexpr int NF = (BN + GROUP_THREADS - 1) / GROUP_THREADS;
   static constexpr int ND = (64 * (BN / 64) + GROUP_THREADS - 1) / GROUP_THREADS;
   static constexpr int N = NF > ND ? NF : ND;
-  float v[N];  // group scales s2
-  int q[N];    // double-quantised absmax q8
+  float v[N];
 };
 template <int BN>
 __device__ __forceinline__ void load_scales(const GemmParams& p, bool fwd, int n0, int kk, int gtid, ScaleRegs<BN>& r) {
   if (fwd)
-    fwd_scales<BN>(p.nf4, nf4_seg_of(p.nf4, n0), n0, p.N, kk, gtid, r.v, r.q);
+    fwd_scales<BN>(p.nf4, nf4_seg_of(p.nf4, n0), n0, p.N, kk, gtid, r.v);
   else
-    dx_scales<BN>(p.nf4, nf4_seg_of(p.nf4, kk * BK), n0, p.N, kk * BK, gtid, r.v, r.q);
+    dx_scales<BN>(p.nf4, nf4_seg_of(p.nf4, kk * BK), n0, p.N, kk * BK, gtid, r.v);
 }
 
 // ---------------------------------------------------------------- work pieces
@@ -640,7 +633,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
     }
     for (int r = 0; r < C::RAW_SLOTS; ++r) {
       mbar_init(&raw_full[r], 1);
-      mbar_init(&raw_empty[r], (GROUP_THREADS / 32) * p.raw_k);  // 4 warps per k-block decoded from it
+      mbar_init(&raw_empty[r], GROUP_THREADS / 32);  // the 4 warps of the group that decoded it
     }
     mbar_init(done, 1);
     mbar_init(tmem_empty, 4);  // one arrival per epilogue warp
@@ -685,13 +678,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
         const bool fwd = p.seg[0].B.kind == OP_NF4_K;
         ScaleRegs<BN> cur, nxt;
         if (kb0 < n_raw) load_scales<BN>(p, fwd, n0, kb_lo + kb0, gtid, nxt);
-        const int rk = p.raw_k, ch0 = kb_lo / rk;
         for (int kb = kb0; kb < n_raw; kb += GROUPS) {
           const int kk = kb_lo + kb;
           cur = nxt;
           if (kb + GROUPS < n_raw) load_scales<BN>(p, fwd, n0, kk + GROUPS, gtid, nxt);
-          // raw slot: chunk kk / rk of this piece's chunks (chunks aligned to multiples of rk)
-          const int gb = kb_run + kb, rb = raw_run + (kk / rk - ch0), sub = kk % rk;
+          const int gb = kb_run + kb, rb = raw_run + kb;
           const int st = gb % C::STAGES;
           const uint32_t ph = static_cast<uint32_t>(gb / C::STAGES) & 1u;
           uint8_t* As = base + st * C::STAGE_BYTES;
@@ -699,23 +690,18 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
           const int rs = rb % C::RAW_SLOTS;
           const uint32_t rph = static_cast<uint32_t>(rb / C::RAW_SLOTS) & 1u;
           const uint8_t* Rc = raw_base + rs * C::RAW_BYTES;
+          const uint8_t* Rq = Rc + C::RAW_CODE_BYTES;
           mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, p.err);
           mbar_wait_bounded(&raw_full[rs], rph, abort_flag, p.err);
           if (fwd) {
-            decode_fwd_raw<BN>(p.nf4, nf4_seg_of(p.nf4, n0), cb, seg_mean, n0, p.N, Rc + sub * 32, 32 * rk, Bs, gtid,
-                               cur.v, cur.q);
+            decode_fwd_raw<BN>(p.nf4, nf4_seg_of(p.nf4, n0), cb, seg_mean, n0, p.N, kk, Rc, Rq, Bs, gtid, cur.v);
           } else {
             const int k0 = kk * BK;
-            decode_dx_raw<BN>(p.nf4, nf4_seg_of(p.nf4, k0), cb, seg_mean, n0, p.N, k0, Rc + sub * 64 * (BN / 2), Bs,
-                              gtid, cur.v, cur.q);
+            decode_dx_raw<BN>(p.nf4, nf4_seg_of(p.nf4, k0), cb, seg_mean, n0, p.N, k0, ((n0 >> 6) >> 4) << 4, Rc, Rq,
+                              Bs, gtid, cur.v);
           }
           __syncwarp();
-          // this warp's reads of the raw slot are done; the last k-block of a chunk this piece
-          // only partly uses also counts the chunk's k-blocks outside the piece
-          if (lane == 0) {
-            const int c_lo = max(kb_lo, (kk / rk) * rk), c_hi = min(kb_lo + n_raw, (kk / rk) * rk + rk);
-            mbar_arrive_cnt(&raw_empty[rs], kk == c_hi - 1 ? 1u + static_cast<uint32_t>(rk - (c_hi - c_lo)) : 1u);
-          }
+          if (lane == 0) mbar_arrive(&raw_empty[rs]);  // this warp's reads of the raw slot are done
           if (p.a_mode[0] == 0) load_tile<BM>(p.seg[0].A, p.nf4, lut, seg_mean, p.seg[0].K, m0, p.M, kk * BK, As, gtid);
           fence_proxy_async_smem();
           __syncwarp();
@@ -755,7 +741,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
         }
       }
       kb_run += kb_hi > kb_lo ? kb_hi - kb_lo : 0;
-      raw_run += n_raw > 0 ? (kb_lo + n_raw - 1) / p.raw_k - kb_lo / p.raw_k + 1 : 0;
+      raw_run += n_raw;
     }
   } else {
     const int q = warp - EPI_WARP0;  // TMEM lane quarter of this epilogue warp
@@ -812,29 +798,28 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
       }
       if (warp == EPI_WARP0 + 2 && lane == 0 && n_raw > 0) {
         // ---------------------------------------------- TMA issuer: raw NF4 codes / absmax
-        // one codes copy per chunk of rk k-blocks (chunks aligned to multiples of rk; a piece's
-        // first and last chunk may reach outside it); the absmax bytes are loaded by the
-        // producers themselves, a k-block ahead, with the group scales
         const GemmSeg& sg = p.seg[0];
-        const int rk = p.raw_k, ch0 = kb_lo / rk, nch = (kb_lo + n_raw - 1) / rk - ch0 + 1;
-        for (int c = 0; c < nch; ++c) {
-          const int kk0 = (ch0 + c) * rk;  // first k-block of the chunk within segment 0
-          const int rb = raw_run + c;
+        for (int kb = 0; kb < n_raw; ++kb) {
+          const int kk = kb_lo + kb;  // k-block index within segment 0
+          const int rb = raw_run + kb;
           const int rs = rb % C::RAW_SLOTS;
           const uint32_t rph = static_cast<uint32_t>(rb / C::RAW_SLOTS) & 1u;
           mbar_wait_bounded(&raw_empty[rs], rph ^ 1u, abort_flag, p.err);
           uint8_t* Rc = raw_base + rs * C::RAW_BYTES;
+          uint8_t* Rq = Rc + C::RAW_CODE_BYTES;
           if (sg.B.kind == OP_NF4_K) {
             const int si = nf4_seg_of(p.nf4, n0);
             const int y = n0 - p.nf4.seg[si].row_begin;
-            mbar_arrive_expect_tx(&raw_full[rs], BN * 32 * rk);
-            tma_load_2d(Rc, &p.tmapCodes[si], kk0 * (BK / 2), y, &raw_full[rs]);
+            mbar_arrive_expect_tx(&raw_full[rs], BN * 32 + BN * 16);
+            tma_load_2d(Rc, &p.tmapCodes[si], kk * (BK / 2), y, &raw_full[rs]);
+            tma_load_2d(Rq, &p.tmapQ8[si], (kk >> 4) << 4, y, &raw_full[rs]);
           } else {
-            const int k0 = kk0 * BK;
+            const int k0 = kk * BK;
             const int si = nf4_seg_of(p.nf4, k0);
             const int y = k0 - p.nf4.seg[si].row_begin;
-            mbar_arrive_expect_tx(&raw_full[rs], 64 * rk * (BN / 2));
+            mbar_arrive_expect_tx(&raw_full[rs], 64 * (BN / 2) + 64 * 16);
             tma_load_2d(Rc, &p.tmapCodes[si], n0 / 2, y, &raw_full[rs]);
+            tma_load_2d(Rq, &p.tmapQ8[si], ((n0 >> 6) >> 4) << 4, y, &raw_full[rs]);
           }
         }
       }
@@ -965,7 +950,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
         }
       }
       kb_run += kb_hi > kb_lo ? kb_hi - kb_lo : 0;
-      raw_run += n_raw > 0 ? (kb_lo + n_raw - 1) / p.raw_k - kb_lo / p.raw_k + 1 : 0;
+      raw_run += n_raw;
     }
   }
 
@@ -1103,8 +1088,8 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 // recur every layer and every step, and encoding costs host time on every GEMM launch.
 struct MapKey {
   const void* ptr;
-  unsigned long long d0, d1, stride;
-  unsigned b0, b1;
+  unsigned long long d0, d1, stride, d2, stride2;  // d2 = 0: a 2D map
+  unsigned b0, b1, b2, pad;
   int dtype, swizzle;
   bool operator==(const MapKey& o) const { return std::memcmp(this, &o, sizeof(MapKey)) == 0; }
 };
@@ -1118,7 +1103,8 @@ struct MapKeyHash {
 };
 bool encode_cached(CUtensorMap* map, const void* ptr, CUtensorMapDataType dtype, unsigned long long d0,
                    unsigned long long d1, unsigned long long stride_bytes, unsigned b0, unsigned b1,
-                   CUtensorMapSwizzle swz) {
+                   CUtensorMapSwizzle swz, unsigned long long d2 = 0, unsigned long long stride2 = 0,
+                   unsigned b2 = 1) {
   static std::mutex mu;
   static std::unordered_map<MapKey, CUtensorMap, MapKeyHash> cache;
   MapKey key;
@@ -1129,6 +1115,9 @@ bool encode_cached(CUtensorMap* map, const void* ptr, CUtensorMapDataType dtype,
   key.stride = stride_bytes;
   key.b0 = b0;
   key.b1 = b1;
+  key.d2 = d2;
+  key.stride2 = stride2;
+  key.b2 = d2 ? b2 : 0;
   key.dtype = static_cast<int>(dtype);
   key.swizzle = static_cast<int>(swz);
   {
@@ -1141,11 +1130,12 @@ bool encode_cached(CUtensorMap* map, const void* ptr, CUtensorMapDataType dtype,
   }
   auto fn = tensor_map_encoder();
   if (!fn) return false;
-  cuuint64_t dims[2] = {d0, d1};
-  cuuint64_t strides[1] = {stride_bytes};
-  cuuint32_t box[2] = {b0, b1};
-  cuuint32_t es[2] = {1, 1};
-  if (fn(map, dtype, 2, const_cast<void*>(ptr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+  const cuuint32_t rank = d2 ? 3 : 2;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {stride_bytes, stride2};
+  cuuint32_t box[3] = {b0, b1, b2};
+  cuuint32_t es[3] = {1, 1, 1};
+  if (fn(map, dtype, rank, const_cast<void*>(ptr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return false;
   std::lock_guard<std::mutex> lock(mu);
@@ -1198,7 +1188,7 @@ bool tma_operands_allowed() {
   return allowed;
 }
 
-bool setup_raw_tma(GemmParams& p, int BN, int rawk_max) {
+bool setup_raw_tma(GemmParams& p, int BN) {
   if (!raw_tma_allowed()) return false;
   const GemmSeg& s0 = p.seg[0];
   if (s0.K <= 0 || (s0.B.kind != OP_NF4_K && s0.B.kind != OP_NF4_MN)) return false;
@@ -1212,25 +1202,14 @@ bool setup_raw_tma(GemmParams& p, int BN, int rawk_max) {
     for (int i = 1; i < g.nseg; ++i)
       if (g.seg[i].row_begin % 64 != 0) return false;
   }
-  // k-blocks per raw chunk: the largest of 4, 2, 1 (up to the slot's room) such that in the
-  // transposed read no chunk straddles two stacked tensors (chunks are aligned to multiples of
-  // rk in the stacked K)
-  int rk = rawk_max;
-  if (s0.B.kind == OP_NF4_MN)
-    while (rk > 1) {
-      bool ok = true;
-      for (int i = 1; i < g.nseg; ++i)
-        if ((g.seg[i].row_begin / BK) % rk != 0) ok = false;
-      if (ok) break;
-      rk >>= 1;
-    }
-  p.raw_k = rk;
-  const unsigned long long cb = static_cast<unsigned long long>(g.cols) / 2;
+  const unsigned long long cb = static_cast<unsigned long long>(g.cols) / 2, qb = static_cast<unsigned long long>(g.cols) / 64;
   for (int i = 0; i < g.nseg; ++i) {
     const unsigned long long rows = static_cast<unsigned long long>(g.seg[i].rows);
     const bool ok = (s0.B.kind == OP_NF4_K)
-                        ? encode_u8_2d(&p.tmapCodes[i], g.seg[i].codes, cb, rows, cb, 32 * rk, BN)
-                        : encode_u8_2d(&p.tmapCodes[i], g.seg[i].codes, cb, rows, cb, BN / 2, 64 * rk);
+                        ? (encode_u8_2d(&p.tmapCodes[i], g.seg[i].codes, cb, rows, cb, 32, BN) &&
+                           encode_u8_2d(&p.tmapQ8[i], g.seg[i].q8, qb, rows, qb, 16, BN))
+                        : (encode_u8_2d(&p.tmapCodes[i], g.seg[i].codes, cb, rows, cb, BN / 2, 64) &&
+                           encode_u8_2d(&p.tmapQ8[i], g.seg[i].q8, qb, rows, qb, 16, 64));
     if (!ok) return false;
   }
   return true;
@@ -1303,6 +1282,13 @@ bool operand_ok(const Operand& op, int K) {
 bool is_mn(int kind) { return kind == OP_BF16_MN || kind == OP_F32_MN || kind == OP_NF4_MN; }
 
 }  // namespace
+
+bool tma_encode_bf16_sw128_planes(CUtensorMap* map, const void* ptr, unsigned long long rows, unsigned long long planes,
+                                  unsigned long long row_bytes, unsigned box_rows, unsigned box_planes) {
+  if (rows == 0 || planes == 0 || (reinterpret_cast<uintptr_t>(ptr) & 15u) || (row_bytes & 15u)) return false;
+  return encode_cached(map, ptr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 64, rows, row_bytes, 64, box_rows,
+                       CU_TENSOR_MAP_SWIZZLE_128B, planes, 128, box_planes);
+}
 
 bool tma_encode_bf16_sw128(CUtensorMap* map, const void* ptr, unsigned long long inner, unsigned long long outer,
                            unsigned long long row_bytes, unsigned box_inner, unsigned box_outer) {
@@ -1458,8 +1444,7 @@ cudaError_t gemm_launch(const GemmParams& p_in, cudaStream_t st) {
   const int BM = UM * MT;  // A rows per CTA
   const int BNB = BN;      // B rows per CTA
   p.bn = BNB;
-  p.raw_k = 1;
-  p.raw_tma = setup_raw_tma(p, BNB, SOUP_GEMM_RAWK) ? 1 : 0;
+  p.raw_tma = setup_raw_tma(p, BNB) ? 1 : 0;
   if (tma_operands_allowed()) {
     for (int s = 0; s < p.nseg; ++s) {
       GemmSeg& sg = p.seg[s];

@@ -60,11 +60,11 @@ struct GemmParams {
   CUtensorMap tmapA[GEMM_MAX_SEG];  // TMA descriptors of bf16 A operands
   CUtensorMap tmapB[GEMM_MAX_SEG];  // TMA descriptors of bf16 B operands
   CUtensorMap tmapCodes[3];         // TMA descriptors of each NF4 tensor's packed codes (raw staging)
+  CUtensorMap tmapQ8[3];            // ... and of its q8 absmax
   int a_mode[GEMM_MAX_SEG];         // 0: producer warps load A; 1: TMA, K-major; 2: TMA, MN-major
   int b_mode[GEMM_MAX_SEG];         // same for B (bf16 operands only)
   int b_row0[GEMM_MAX_SEG];         // first operand row of the B descriptor (block-diagonal windows)
   int raw_tma;                      // 1: the NF4 segment's codes / absmax arrive by TMA
-  int raw_k;                        // k-blocks per raw TMA chunk (1, 2 or 4)
   int bn;                           // output tile width
   int M, N;
   int nseg;
@@ -114,6 +114,13 @@ struct GemmParams {
 // Cached by its arguments.  False if the driver refuses it (alignment, sizes).
 bool tma_encode_bf16_sw128(CUtensorMap* map, const void* ptr, unsigned long long inner, unsigned long long outer,
                            unsigned long long row_bytes, unsigned box_inner, unsigned box_outer);
+
+// The same array seen as 64-element column blocks ("planes", 128 B apart) of `rows` rows: a
+// 3D map (64, rows, planes) whose box (64, box_rows, box_planes) lands in shared memory as
+// box_planes consecutive [box_rows x 128 B] swizzled tiles, i.e. box_planes 64-wide column
+// blocks of a row range in one copy.
+bool tma_encode_bf16_sw128_planes(CUtensorMap* map, const void* ptr, unsigned long long rows, unsigned long long planes,
+                                  unsigned long long row_bytes, unsigned box_rows, unsigned box_planes);
 
 // Launch C = sum_seg A_seg B_seg^T on the tcgen05 tensor cores. Returns cudaError_t of launch.
 cudaError_t gemm_launch(const GemmParams& p, cudaStream_t st);

@@ -982,11 +982,14 @@ soup_status layer_backward_body(soup_model* m, int i, const LayerView& L, const 
                   [&] { return swiglu_bwd_launch(m->dm, A.gu, T, I, m->dgu, st); }));
   // ---- gate | up
   if (lora) {
-    for (int q = 0; q < 2; ++q) {
-      GemmParams p = gemm_base(m, T, r, m->vgu + q * r, 2 * r, 0, s);
-      add_seg(p, I, opnd(OP_BF16_K, m->dgu + q * I, 2 * I), opnd(OP_BF16_MN, P + lora_off(c, i, 4 + q, 1), r));
-      SOUP_TRY(run_gemm(m, p, st, "lora v gate/up"));
-    }
+    // v_gate | v_up = [dgate | dup] . blockdiag(B_gate, B_up): one GEMM, each output block
+    // reading its own projection's B through a row window (zero elsewhere); the operand is
+    // indexed by the output column n, so B_p is addressed from q r columns before its start
+    GemmParams p = gemm_base(m, T, 2 * r, m->vgu, 2 * r, 0, s);
+    for (int q = 0; q < 2; ++q)
+      add_seg(p, I, opnd(OP_BF16_K, m->dgu + q * I, 2 * I),
+              opnd(OP_BF16_MN, P + lora_off(c, i, 4 + q, 1) - q * r, r, 1.f, q * r, (q + 1) * r));
+    SOUP_TRY(run_gemm(m, p, st, "lora v gate/up"));
   }
   {
     GemmParams p = gemm_base(m, T, h, m->dn, h, 0, 1.f);
@@ -1037,11 +1040,12 @@ soup_status layer_backward_body(soup_model* m, int i, const LayerView& L, const 
   // ---- q | k | v
   const int off[3] = {0, qd, qd + kvd}, outs[3] = {qd, kvd, kvd};
   if (lora) {
-    for (int q = 0; q < 3; ++q) {
-      GemmParams p = gemm_base(m, T, r, m->vqkv + q * r, 3 * r, 0, s);
-      add_seg(p, outs[q], opnd(OP_BF16_K, m->dqkv + off[q], QKV), opnd(OP_BF16_MN, P + lora_off(c, i, q, 1), r));
-      SOUP_TRY(run_gemm(m, p, st, "lora v qkv"));
-    }
+    // v_q | v_k | v_v in one GEMM (block-diagonal B through row windows, as for gate | up)
+    GemmParams p = gemm_base(m, T, 3 * r, m->vqkv, 3 * r, 0, s);
+    for (int q = 0; q < 3; ++q)
+      add_seg(p, outs[q], opnd(OP_BF16_K, m->dqkv + off[q], QKV),
+              opnd(OP_BF16_MN, P + lora_off(c, i, q, 1) - q * r, r, 1.f, q * r, (q + 1) * r));
+    SOUP_TRY(run_gemm(m, p, st, "lora v qkv"));
   }
   {
     GemmParams p = gemm_base(m, T, h, m->dn, h, 0, 1.f);
