@@ -14,8 +14,9 @@
 //
 // Warp roles (192 threads): warps 0-3 softmax and epilogue (TMEM lane quarters 0-3, thread = query
 // row), warp 4 allocates TMEM and its lane 0 issues the MMAs, warp 5 lane 0 issues the TMA loads
-// (Q once, K/V tiles in a 2-stage ring; one 3D copy per [128 rows x d] tile).  Every wait is bounded (mbar_wait_bounded): on timeout the
-// device error word is set and the kernel runs to its end.
+// (Q once; K and V tiles each in a 3-stage ring of its own, a K stage freed as soon as its S
+// MMAs retire; one 3D copy per [128 rows x d] tile).  Every wait is bounded (mbar_wait_bounded):
+// on timeout the device error word is set and the kernel runs to its end.
 //
 // Key tiles a query tile reads: those with a visible (query, key) pair (attn_mask.cuh); the plain
 // causal layout reads tiles 0..qt.  Rows at or past S (a ragged last tile) are masked as keys and
@@ -24,6 +25,7 @@
 #include "common.cuh"
 #include "internal.h"
 #include "tc.cuh"
+
 
 namespace soup {
 
@@ -40,15 +42,36 @@ constexpr float LOG2E_F = 1.4426950408889634f;
 template <int D>
 struct FwdCfg {
   static constexpr int TILE_BYTES = TQ * D * 2;  // one [128 x D] bf16 tile: D/64 swizzle atoms of 16 KB
+  static constexpr int KV_STAGES = 3;
   static constexpr int Q_OFF = 0;
-  static constexpr int K_OFF = TILE_BYTES;       // 2 stages
-  static constexpr int V_OFF = 3 * TILE_BYTES;   // 2 stages
-  static constexpr int BAR_OFF = 5 * TILE_BYTES;
+  static constexpr int K_OFF = TILE_BYTES;                    // KV_STAGES stages
+  static constexpr int V_OFF = (1 + KV_STAGES) * TILE_BYTES;  // KV_STAGES stages
+  static constexpr int BAR_OFF = (1 + 2 * KV_STAGES) * TILE_BYTES;
   static constexpr int SMEM_BYTES = 1024 + BAR_OFF + 256;
+  static_assert((1 + 4 * KV_STAGES + 2 * N_SBUF + 1 + 2) * 8 <= 256, "barrier block");
   static constexpr int O_COL = N_SBUF * TK;      // TMEM column of the O accumulator
   static constexpr int TMEM_COLS = 512;
   static_assert(O_COL + D <= TMEM_COLS, "TMEM budget");
 };
+
+// 2^x with the MUFU approximation (PTX ex2.approx.ftz: relative error about 2^-22), results below
+// 2^-126 flushed to zero: a probability that small is zero at bf16 and in the fp32 row sum alike.
+// The softmax rows' exponentials are the attention kernels' most frequent instruction.
+__device__ __forceinline__ float exp2_ftz(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Masks 32 consecutive scores of query row q (keys k0..k0+31) that the row must not see: keys
+// at or past S and keys `visible` rejects become -inf.
+__device__ __forceinline__ void mask_keys32(const AttnShape& s, int q, int k0, uint32_t (&raw)[32]) {
+#pragma unroll
+  for (int e = 0; e < 32; ++e) {
+    const int k = k0 + e;
+    if (k >= s.S || !visible(s, q, k)) raw[e] = 0xff800000u;  // -inf
+  }
+}
 
 // Key tile j is read by query tile qt.
 __device__ __forceinline__ bool kv_needed(const AttnShape& s, int qt, int j) {
@@ -58,32 +81,40 @@ __device__ __forceinline__ bool kv_needed(const AttnShape& s, int qt, int j) {
 
 template <int D>
 __global__ void __launch_bounds__(FWD_THREADS, 1)
-    attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap, const AttnShape s, uint16_t* __restrict__ out,
-                       float* __restrict__ lse, int* err) {
+    attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ CUtensorMap tmap_o,
+                       const AttnShape s, uint16_t* __restrict__ out, float* __restrict__ lse, int* err) {
   using C = FwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* base = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + C::BAR_OFF);
-  uint64_t* q_full = bars;          // 1
-  uint64_t* kv_full = bars + 1;     // 2
-  uint64_t* kv_empty = bars + 3;    // 2
-  uint64_t* s_full = bars + 5;      // 3
-  uint64_t* p_full = bars + 8;      // 3
-  uint64_t* o_ready = bars + 11;    // 1
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 13);
+  // K and V stages have barriers of their own: K_j's stage frees when S_j's MMAs retire, long
+  // before V_j's (after PV_j), so the next K tiles load while the softmax runs
+  constexpr int KS = C::KV_STAGES;
+  uint64_t* q_full = bars;                 // 1
+  uint64_t* k_full = bars + 1;             // KS
+  uint64_t* v_full = k_full + KS;          // KS
+  uint64_t* k_empty = v_full + KS;         // KS
+  uint64_t* v_empty = k_empty + KS;        // KS
+  uint64_t* s_full = v_empty + KS;         // N_SBUF
+  uint64_t* p_full = s_full + N_SBUF;      // N_SBUF
+  uint64_t* o_ready = p_full + N_SBUF;     // 1
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_ready + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(o_ready + 2);
 
-  const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  // the last query tiles see the most keys: they start first (longest work first on the SMs)
+  const int qt = gridDim.x - 1 - blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int g = h / (s.hq / s.hkv);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ntk = (s.S + TK - 1) / TK;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&kv_full[i], 1);
-      mbar_init(&kv_empty[i], 1);
+    for (int i = 0; i < KS; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&v_full[i], 1);
+      mbar_init(&k_empty[i], 1);
+      mbar_init(&v_empty[i], 1);
     }
     for (int i = 0; i < N_SBUF; ++i) {
       mbar_init(&s_full[i], 1);
@@ -111,11 +142,14 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
       int jj = 0;
       for (int j = 0; j < ntk; ++j) {
         if (!kv_needed(s, qt, j)) continue;
-        const int st = jj & 1;
-        mbar_wait_bounded(&kv_empty[st], ((jj >> 1) & 1) ^ 1u, abort_flag, err);
-        mbar_arrive_expect_tx(&kv_full[st], 2 * TB);
-        tma_load_3d(base + C::K_OFF + st * TB, &tmap, 0, row0 + j * TK, (s.hq + g) * (D / 64), &kv_full[st]);
-        tma_load_3d(base + C::V_OFF + st * TB, &tmap, 0, row0 + j * TK, (s.hq + s.hkv + g) * (D / 64), &kv_full[st]);
+        const int st = jj % KS;
+        const uint32_t ph = static_cast<uint32_t>((jj / KS) & 1) ^ 1u;
+        mbar_wait_bounded(&k_empty[st], ph, abort_flag, err);
+        mbar_arrive_expect_tx(&k_full[st], TB);
+        tma_load_3d(base + C::K_OFF + st * TB, &tmap, 0, row0 + j * TK, (s.hq + g) * (D / 64), &k_full[st]);
+        mbar_wait_bounded(&v_empty[st], ph, abort_flag, err);
+        mbar_arrive_expect_tx(&v_full[st], TB);
+        tma_load_3d(base + C::V_OFF + st * TB, &tmap, 0, row0 + j * TK, (s.hq + s.hkv + g) * (D / 64), &v_full[st]);
         ++jj;
       }
     }
@@ -126,7 +160,8 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
       const uint32_t idesc_pv = idesc_bf16(TQ, D, false, true);    // O[q, d] += sum_k P[q, k] V[k, d]
       mbar_wait_bounded(q_full, 0, abort_flag, err);
       auto issue_pv = [&](int i) {
-        const int st = i & 1, sb = i % N_SBUF;
+        const int st = i % KS, sb = i % N_SBUF;
+        mbar_wait_bounded(&v_full[st], (i / KS) & 1, abort_flag, err);
         mbar_wait_bounded(&p_full[sb], (i / N_SBUF) & 1, abort_flag, err);
         tc_fence_after();
         const uint32_t sv = smem_u32(base + C::V_OFF + st * C::TILE_BYTES);
@@ -135,14 +170,14 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
           const uint64_t bd = sw128_mnmajor_desc(sv + kk * 2048, TK * 128);
           tc_mma_f16_ts(tmem + C::O_COL, tmem + sb * TK + kk * 8, bd, idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
         }
-        tc_commit(&kv_empty[st]);
+        tc_commit(&v_empty[st]);
         tc_commit(o_ready);
       };
       int jj = 0;
       for (int j = 0; j < ntk; ++j) {
         if (!kv_needed(s, qt, j)) continue;
-        const int st = jj & 1, sb = jj % N_SBUF;
-        mbar_wait_bounded(&kv_full[st], (jj >> 1) & 1, abort_flag, err);
+        const int st = jj % KS, sb = jj % N_SBUF;
+        mbar_wait_bounded(&k_full[st], (jj / KS) & 1, abort_flag, err);
         tc_fence_after();
         const uint32_t sk = smem_u32(base + C::K_OFF + st * C::TILE_BYTES);
 #pragma unroll
@@ -152,6 +187,7 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
                      kc > 0 ? 1u : 0u);
         }
         tc_commit(&s_full[sb]);
+        tc_commit(&k_empty[st]);  // K_jj's stage is free once S_jj's MMAs retire
         if (jj > 0) issue_pv(jj - 1);
         ++jj;
       }
@@ -171,41 +207,42 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
       mbar_wait_bounded(&s_full[sb], (jj / N_SBUF) & 1, abort_flag, err);
       tc_fence_after();
       const bool need_mask = s.pl > 0 || j == qt || (j + 1) * TK > s.S;
-      float x[TK];
-      float mx = m;
+      const uint32_t srow = tmem + lane_base + sb * TK;
+      // the row's 128 scores come out of TMEM in four loads and one wait; then the tile's max,
+      // and P = exp2(S scale - m) as bf16 over the first half of the buffer's columns (two per
+      // column), the sum kept in four partial sums.  PV_{jj-1} reads another buffer, so this
+      // may run before it has finished.
+      uint32_t raw[TK / 32][32];
 #pragma unroll
-      for (int c = 0; c < TK / 32; ++c) {
-        uint32_t raw[32];
-        tmem_ld32(tmem + lane_base + sb * TK + c * 32, raw);
-        tmem_ld_wait();
+      for (int c = 0; c < TK / 32; ++c) tmem_ld32(srow + c * 32, raw[c]);
+      tmem_ld_wait();
+      if (need_mask) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          float v = __uint_as_float(raw[e]) * scale_log2;
-          if (need_mask) {
-            const int k = j * TK + c * 32 + e;
-            if (k >= s.S || !visible(s, q, k)) v = -INFINITY;
-          }
-          x[c * 32 + e] = v;
-          mx = fmaxf(mx, v);
-        }
+        for (int c = 0; c < TK / 32; ++c) mask_keys32(s, q, j * TK + c * 32, raw[c]);
       }
+      float t[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int c = 0; c < TK / 32; ++c)
+#pragma unroll
+        for (int e = 0; e < 32; ++e) t[e & 3] = fmaxf(t[e & 3], __uint_as_float(raw[c][e]));
+      const float mx = fmaxf(m, fmaxf(fmaxf(t[0], t[1]), fmaxf(t[2], t[3])) * scale_log2);  // scale_log2 > 0
       const bool live = mx != -INFINITY;  // some key of this row visible so far
       const float alpha = live ? exp2f(m - mx) : 1.f;
-      // P_jj over the first half of the S buffer's columns (two bf16 per column); PV_{jj-1}
-      // reads another buffer, so this may run before it has finished
-      float sum = 0.f;
+      float sums[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < TK / 32; ++c) {
         uint32_t pw[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
-          const float p0 = live ? exp2f(x[c * 32 + e] - mx) : 0.f;
-          const float p1 = live ? exp2f(x[c * 32 + e + 1] - mx) : 0.f;
-          sum += p0 + p1;
+          const float p0 = live ? exp2_ftz(__uint_as_float(raw[c][e]) * scale_log2 - mx) : 0.f;
+          const float p1 = live ? exp2_ftz(__uint_as_float(raw[c][e + 1]) * scale_log2 - mx) : 0.f;
+          sums[e & 2] += p0;
+          sums[(e & 2) + 1] += p1;
           pw[e >> 1] = pack_bf16x2(p0, p1);
         }
-        tmem_st16(tmem + lane_base + sb * TK + c * 16, pw);
+        tmem_st16(srow + c * 16, pw);
       }
+      const float sum = (sums[0] + sums[1]) + (sums[2] + sums[3]);
       l = l * alpha + sum;
       m = mx;
       if (jj > 0) {
@@ -213,7 +250,7 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
         mbar_wait_bounded(o_ready, (jj - 1) & 1, abort_flag, err);
         tc_fence_after();
         if (__any_sync(0xffffffffu, alpha != 1.f)) {
-#pragma unroll
+#pragma unroll 2
           for (int c = 0; c < D / 16; ++c) {
             uint32_t o[16];
             tmem_ld16(tmem + lane_base + C::O_COL + c * 16, o);
@@ -230,17 +267,26 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
       if (lane == 0) mbar_arrive(&p_full[sb]);
       ++jj;
     }
-    // epilogue: O / l in bf16, natural-log LSE
+    // epilogue: O / l in bf16, natural-log LSE.  A whole query tile is written into Q's shared
+    // tile (free: every MMA has retired) in the TMA's swizzled layout and leaves in one TMA
+    // store; a ragged last tile (its rows past S belong to the next sequence) stores row by row.
     if (jj > 0) mbar_wait_bounded(o_ready, (jj - 1) & 1, abort_flag, err);
     tc_fence_after();
     const float inv = (l > 0.f) ? 1.f / l : 0.f;
+    const bool whole_tile = qt * TQ + TQ <= s.S;
+    uint8_t* otile = base + C::Q_OFF;
     uint16_t* orow = out + (static_cast<long long>(row0) + q) * static_cast<long long>(s.hq * D) + h * D;
-#pragma unroll
-    for (int c = 0; c < D / 16; ++c) {
-      uint32_t o[16];
-      tmem_ld16(tmem + lane_base + C::O_COL + c * 16, o);
+    // 64 columns of O per TMEM round trip (two loads, one wait), 16 per store step
+#pragma unroll 1
+    for (int c64 = 0; c64 < D / 64; ++c64) {
+      uint32_t ov[2][32];
+      tmem_ld32(tmem + lane_base + C::O_COL + c64 * 64, ov[0]);
+      tmem_ld32(tmem + lane_base + C::O_COL + c64 * 64 + 32, ov[1]);
       tmem_ld_wait();
-      if (q < s.S) {
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        const int c = c64 * 4 + cc;
+        const uint32_t* o = &ov[cc >> 1][(cc & 1) * 16];
         uint4 w0, w1;
         w0.x = pack_bf16x2(__uint_as_float(o[0]) * inv, __uint_as_float(o[1]) * inv);
         w0.y = pack_bf16x2(__uint_as_float(o[2]) * inv, __uint_as_float(o[3]) * inv);
@@ -250,8 +296,29 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
         w1.y = pack_bf16x2(__uint_as_float(o[10]) * inv, __uint_as_float(o[11]) * inv);
         w1.z = pack_bf16x2(__uint_as_float(o[12]) * inv, __uint_as_float(o[13]) * inv);
         w1.w = pack_bf16x2(__uint_as_float(o[14]) * inv, __uint_as_float(o[15]) * inv);
-        *reinterpret_cast<uint4*>(orow + c * 16) = w0;
-        *reinterpret_cast<uint4*>(orow + c * 16 + 8) = w1;
+        if (whole_tile) {
+          // columns 16c.. : plane 16c / 64, 16-byte chunks 2(c % 4) and 2(c % 4) + 1 of row r,
+          // placed by the 128-byte swizzle (chunk index XOR row % 8)
+          const uint32_t rowa = smem_u32(otile) + static_cast<uint32_t>((c >> 2) * (TQ * 128) + r * 128);
+          const uint32_t ch = static_cast<uint32_t>((c & 3) * 2), sw = static_cast<uint32_t>(r & 7);
+          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(rowa + ((ch ^ sw) << 4)), "r"(w0.x),
+                       "r"(w0.y), "r"(w0.z), "r"(w0.w)
+                       : "memory");
+          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(rowa + (((ch + 1) ^ sw) << 4)), "r"(w1.x),
+                       "r"(w1.y), "r"(w1.z), "r"(w1.w)
+                       : "memory");
+        } else if (q < s.S) {
+          *reinterpret_cast<uint4*>(orow + c * 16) = w0;
+          *reinterpret_cast<uint4*>(orow + c * 16 + 8) = w1;
+        }
+      }
+    }
+    if (whole_tile) {
+      fence_proxy_async_smem();  // the tile's generic-proxy writes, visible to the TMA
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (threadIdx.x == 0) {
+        tma_store_3d(&tmap_o, 0, row0 + qt * TQ, h * (D / 64), otile);
+        tma_store_commit_wait_read();
       }
     }
     if (q < s.S) lse[(static_cast<long long>(b) * s.hq + h) * s.S + q] = (m + log2f(l)) / LOG2E_F;
@@ -268,10 +335,14 @@ template <int D>
 cudaError_t launch_fwd(const AttnShape& s, const uint16_t* qkv, uint16_t* o, float* lse, int* err, cudaStream_t st) {
   using C = FwdCfg<D>;
   // one copy per [128 rows x D] tile: the head's D/64 column blocks as the planes of a 3D map
-  CUtensorMap map;
+  CUtensorMap map, map_o;
   const unsigned long long planes = static_cast<unsigned long long>(s.hq + 2 * s.hkv) * (D / 64);
   const unsigned long long rows = static_cast<unsigned long long>(s.B) * s.S;
   if (!tma_encode_bf16_sw128_planes(&map, qkv, rows, planes, static_cast<unsigned long long>(s.ld_qkv) * 2, TQ, D / 64))
+    return cudaErrorInvalidValue;
+  // the output [T, hq d] as the same kind of map: a query tile's head is one [128 x D] box
+  if (!tma_encode_bf16_sw128_planes(&map_o, o, rows, static_cast<unsigned long long>(s.hq) * (D / 64),
+                                    static_cast<unsigned long long>(s.hq) * D * 2, TQ, D / 64))
     return cudaErrorInvalidValue;
   static bool attr = false;
   if (!attr) {
@@ -281,7 +352,7 @@ cudaError_t launch_fwd(const AttnShape& s, const uint16_t* qkv, uint16_t* o, flo
     attr = true;
   }
   const dim3 grid((s.S + TQ - 1) / TQ, s.hq, s.B);
-  attn_fwd_tc_kernel<D><<<grid, FWD_THREADS, C::SMEM_BYTES, st>>>(map, s, o, lse, err);
+  attn_fwd_tc_kernel<D><<<grid, FWD_THREADS, C::SMEM_BYTES, st>>>(map, map_o, s, o, lse, err);
   return cudaGetLastError();
 }
 
@@ -522,7 +593,8 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
         mbar_wait_bounded(s_full, it & 1, abort_flag, err);
         tc_fence_after();
         const bool need_mask = s.pl > 0 || i == j || (i + 1) * TQ > s.S;
-#pragma unroll
+        // 32-column chunks, rolled (a whole row of S and dP would not fit in registers)
+#pragma unroll 1
         for (int c = 0; c < TQ / 32; ++c) {
           uint32_t sr[32], dr[32];
           tmem_ld32(tmem + lane_base + C::S_COL + c * 32, sr);
@@ -535,7 +607,7 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
               const int qc = c * 32 + e + u;
-              float p = exp2f(__uint_as_float(sr[e + u]) * scale_log2 - lsm[qc]);
+              float p = exp2_ftz(__uint_as_float(sr[e + u]) * scale_log2 - lsm[qc]);
               if (need_mask) {
                 const int q = i * TQ + qc;
                 if (q >= s.S || !visible(s, q, k)) p = 0.f;
@@ -628,7 +700,8 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 9);
 
-  const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  // the last query tiles see the most keys: they start first (longest work first on the SMs)
+  const int qt = gridDim.x - 1 - blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int g = h / (s.hq / s.hkv);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ntk = (s.S + TK - 1) / TK;
@@ -715,7 +788,8 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
       mbar_wait_bounded(s_full, jj & 1, abort_flag, err);
       tc_fence_after();
       const bool need_mask = s.pl > 0 || j == qt || (j + 1) * TK > s.S;
-#pragma unroll
+      // 32-column chunks, rolled (a whole row of S and dP would not fit in registers)
+#pragma unroll 1
       for (int c = 0; c < TK / 32; ++c) {
         uint32_t sr[32], dr[32];
         tmem_ld32(tmem + lane_base + C::S_COL + c * 32, sr);
@@ -727,7 +801,7 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
           float dv[2];
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
-            float p = exp2f(__uint_as_float(sr[e + u]) * scale_log2 - lse2);
+            float p = exp2_ftz(__uint_as_float(sr[e + u]) * scale_log2 - lse2);
             if (need_mask) {
               const int k = j * TK + c * 32 + e + u;
               if (k >= s.S || !visible(s, q, k)) p = 0.f;

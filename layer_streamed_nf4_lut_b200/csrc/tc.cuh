@@ -103,6 +103,19 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, i
       : "memory");
 }
 
+// 3D tiled TMA store from shared memory (bulk-group completion).  The box must lie inside the
+// tensor where it is written: out-of-range rows are clipped, never wrapped.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, int x, int y, int z, const void* src) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%1, %2, %3}], [%4];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y), "r"(z), "r"(smem_u32(src))
+               : "memory");
+}
+// Commits this thread's bulk stores and waits until their shared-memory source has been read.
+__device__ __forceinline__ void tma_store_commit_wait_read() {
+  asm volatile("cp.async.bulk.commit_group;\n\tcp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- shared-memory matrix descriptors
 // K-major, 128-byte swizzle: rows of 64 bf16 (128 B), 8-row core groups 1024 B apart.  A K = 16
 // step inside the 64-wide atom advances the start address by 32 B.
