@@ -614,8 +614,6 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
   volatile int* abort_flag = reinterpret_cast<volatile int*>(ctrl + 68);
   volatile int* last_flag = reinterpret_cast<volatile int*>(ctrl + 72);  // split-K: this CTA reduces
   float* seg_mean = reinterpret_cast<float*>(ctrl + 80);              // up to 3 NF4 tensors
-  volatile int* n_pend = reinterpret_cast<volatile int*>(ctrl + 92);   // stream-K tiles this CTA sums
-  volatile int* pend = reinterpret_cast<volatile int*>(ctrl + 96);     // ... up to 8 of them
   uint64_t* full = reinterpret_cast<uint64_t*>(ctrl + 128);
   uint64_t* empty = full + C::STAGES;
   uint64_t* raw_full = empty + C::STAGES;
@@ -638,7 +636,6 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
     mbar_init(done, 1);
     mbar_init(tmem_empty, 4);  // one arrival per epilogue warp
     *abort_flag = 0;
-    *n_pend = 0;
     mbar_fence_init();
   }
   if (threadIdx.x < 16) lut[threadIdx.x] = p.lut[threadIdx.x];
@@ -931,24 +928,6 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tmem_empty);
-      if (sk_part) {
-        // this CTA's share of the tile is stored: count it; the CTA that completes the count
-        // sums the tile at its end
-        __threadfence();
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        if (q == 0 && lane == 0) {
-          const long long x0 = static_cast<long long>(z.tile) * p.sk_nkt;
-          const int shares = sk_owner(p.sk_tiles, p.sk_nkt, p.sk_ctas, x0 + p.sk_nkt - 1) -
-                             sk_owner(p.sk_tiles, p.sk_nkt, p.sk_ctas, x0) + 1;
-          const int old = atomicAdd(&p.tile_counters[z.tile], 1);
-          if (old == shares - 1) {
-            p.tile_counters[z.tile] = 0;  // ready for the next launch
-            const int n = *n_pend;
-            if (n < 8) pend[n] = z.tile;
-            *n_pend = n + 1;
-          }
-        }
-      }
       kb_run += kb_hi > kb_lo ? kb_hi - kb_lo : 0;
       raw_run += n_raw;
     }
@@ -960,51 +939,6 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
   if (warp == EPI_WARP0) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
-  }
-  if (SK) {
-    // stream-K: sum the shares of each tile this CTA completed, in k order (CTA order), with
-    // all 512 threads, one (row, 8-column group) per thread at a time
-    const int np = *n_pend < 8 ? *n_pend : 8;
-    if (*n_pend > 8 && threadIdx.x == 0) set_dev_error(p.err, DEVERR_BOUNDS);  // cannot happen: <= 2 per CTA
-    __threadfence();
-    for (int i = 0; i < np; ++i) {
-      const int t = pend[i];
-      const int m0 = (t % p.sk_tiles_m) * BM, n0 = (t / p.sk_tiles_m) * BN;
-      const long long x0 = static_cast<long long>(t) * p.sk_nkt;
-      const int cf = sk_owner(p.sk_tiles, p.sk_nkt, p.sk_ctas, x0);
-      const int nsh = min(sk_owner(p.sk_tiles, p.sk_nkt, p.sk_ctas, x0 + p.sk_nkt - 1) - cf + 1, 4);  // shares
-      // share 0 sits in CTA cf's last-piece slot when the tile began inside its range, the
-      // others in their CTAs' first-piece slots
-      int c0, sl0;
-      sk_share(p.sk_tiles, p.sk_nkt, p.sk_ctas, t, 0, &c0, &sl0);
-      const float* src0 = p.workspace + static_cast<long long>(sl0) * (BM * BN);
-      constexpr int G8 = BN / 8;
-#pragma unroll 1
-      for (int it = threadIdx.x; it < BM * G8; it += GEMM_THREADS) {
-        const int rl = it / G8, cl8 = (it % G8) * 8;
-        const int row = m0 + rl, col0 = n0 + cl8;
-        if (row >= p.M || col0 >= p.N) continue;
-        float4 a[4][2];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          if (k >= nsh) break;
-          const float* sp = k == 0 ? src0 : p.workspace + static_cast<long long>(2 * (cf + k)) * (BM * BN);
-          const float4* src = reinterpret_cast<const float4*>(sp + rl * BN + cl8);
-          a[k][0] = __ldcg(src);
-          a[k][1] = __ldcg(src + 1);
-        }
-        float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          if (k >= nsh) break;
-          v[0] += a[k][0].x; v[1] += a[k][0].y; v[2] += a[k][0].z; v[3] += a[k][0].w;
-          v[4] += a[k][1].x; v[5] += a[k][1].y; v[6] += a[k][1].z; v[7] += a[k][1].w;
-        }
-#pragma unroll
-        for (int j = 0; j < 8; ++j) v[j] *= p.alpha;
-        epilogue_store<8>(p, row, col0, v);
-      }
-    }
   }
   if (splits > 1 && p.fused_reduce) {
     // The last split of this tile to finish sums every partial in split order (the same
@@ -1068,6 +1002,62 @@ __global__ void splitk_reduce_kernel(const __grid_constant__ GemmParams p) {
 #pragma unroll
   for (int j = 0; j < 8; ++j) v[j] *= p.alpha;
   epilogue_store<8>(p, row, col, v);
+}
+
+// Stream-K: every tile cut between CTAs summed share by share in k order (CTA order, the order
+// a single CTA's k loop would have added them) and written through the normal epilogue, one
+// thread per (row, 8 columns), all cut tiles at once.  A tile one CTA computed whole was
+// written by that CTA.  Block x looks at the boundary between CTAs x and x + 1: the tile it
+// falls in is cut (unless the boundary is a tile boundary) and is summed by the blocks of its
+// first such boundary; blocks y cover the tile's rows.  A separate launch: summed at the end of
+// the CTA that completed a tile, the shares' loads (up to 4 x 128 KB, one SM) added a ~20 us
+// tail to the long GEMMs.
+template <int BM, int BN>
+__global__ void sk_fixup_kernel(const __grid_constant__ GemmParams p) {
+  const int c = blockIdx.x + 1;  // boundary between CTAs c - 1 and c
+  const long long xb = sk_bound(p.sk_tiles, p.sk_nkt, p.sk_ctas, c);
+  if (xb % p.sk_nkt == 0) return;  // not inside a tile
+  const int t = static_cast<int>(xb / p.sk_nkt);
+  const long long xp = sk_bound(p.sk_tiles, p.sk_nkt, p.sk_ctas, c - 1);
+  if (c > 1 && xp / p.sk_nkt == t && xp % p.sk_nkt != 0) return;  // an earlier boundary cut this tile
+  const long long x0 = static_cast<long long>(t) * p.sk_nkt;
+  const int cf = sk_owner(p.sk_tiles, p.sk_nkt, p.sk_ctas, x0);
+  const int nsh = sk_owner(p.sk_tiles, p.sk_nkt, p.sk_ctas, x0 + p.sk_nkt - 1) - cf + 1;
+  if (nsh < 2) return;
+  if (nsh > 4) {  // the planner cuts a tile into at most 4 shares
+    if (threadIdx.x == 0 && blockIdx.y == 0) set_dev_error(p.err, DEVERR_BOUNDS);
+    return;
+  }
+  constexpr int G8 = BN / 8;
+  const int it = blockIdx.y * blockDim.x + threadIdx.x;
+  if (it >= BM * G8) return;
+  const int m0 = (t % p.sk_tiles_m) * BM, n0 = (t / p.sk_tiles_m) * BN;
+  const int rl = it / G8, cl8 = (it % G8) * 8;
+  const int row = m0 + rl, col0 = n0 + cl8;
+  if (row >= p.M || col0 >= p.N) return;
+  // share 0 sits in CTA cf's last-piece slot when the tile began inside its range, the others
+  // in their CTAs' first-piece slots
+  int c0, sl0;
+  sk_share(p.sk_tiles, p.sk_nkt, p.sk_ctas, t, 0, &c0, &sl0);
+  float4 a[4][2];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    if (k >= nsh) break;
+    const long long slot = k == 0 ? sl0 : 2LL * (cf + k);
+    const float4* src = reinterpret_cast<const float4*>(p.workspace + slot * (BM * BN) + rl * BN + cl8);
+    a[k][0] = __ldcg(src);
+    a[k][1] = __ldcg(src + 1);
+  }
+  float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    if (k >= nsh) break;
+    v[0] += a[k][0].x; v[1] += a[k][0].y; v[2] += a[k][0].z; v[3] += a[k][0].w;
+    v[4] += a[k][1].x; v[5] += a[k][1].y; v[6] += a[k][1].z; v[7] += a[k][1].w;
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) v[j] *= p.alpha;
+  epilogue_store<8>(p, row, col0, v);
 }
 
 // ---------------------------------------------------------------- host side
@@ -1230,7 +1220,16 @@ cudaError_t launch_tile(const GemmParams& p, cudaStream_t st) {
                                   : dim3((p.N + BN - 1) / BN, (p.M + C::BM - 1) / C::BM, p.splits > 1 ? p.splits : 1);
   gemm_tc_kernel<MT, BN, SK><<<grid, GEMM_THREADS, C::SMEM_BYTES, st>>>(p);
   cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess || p.splits <= 1 || p.fused_reduce) return e;
+  if (e != cudaSuccess) return e;
+  if (SK) {
+    // the cut tiles' shares, summed by a wide second kernel
+    constexpr int ITEMS = C::BM * BN / 8;
+    if (p.sk_ctas > 1)
+      sk_fixup_kernel<C::BM, BN><<<dim3(static_cast<unsigned>(p.sk_ctas - 1), (ITEMS + 511) / 512), 512, 0, st>>>(p);
+    ++g_kernel_launches;
+    return cudaGetLastError();
+  }
+  if (p.splits <= 1 || p.fused_reduce) return e;
   const long long work = static_cast<long long>(p.M) * (p.N / 8);
   splitk_reduce_kernel<<<static_cast<unsigned>((work + 255) / 256), 256, 0, st>>>(p);
   ++g_kernel_launches;
