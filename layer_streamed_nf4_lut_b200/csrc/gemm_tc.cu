@@ -1320,15 +1320,38 @@ GemmPlan gemm_plan(const GemmParams& p, int sms, bool stream_k_allowed) {
   const double* unit = has_nf4 ? unit_nf4 : unit_bf16;
   // split-K for grids that leave SMs idle (the skinny LoRA GEMMs; never NF4): up to two waves
   // of CTAs, at least 4 k-blocks per split (a CTA of these runs at the issuing thread's rate,
-  // so spreading K shortens the GEMM).  The cost below includes the split and, past 4 partials,
-  // the wide reduction kernel (~500 units).
-  auto split_for = [&](long long tiles) -> long long {
+  // so spreading K shortens the GEMM).  The cost below includes the split and the sum of the
+  // partials (the tile's last CTA for up to 4, else the wide reduction kernel).
+  auto split_cost = [&](long long tiles, long long sp, double u) {
+    const long long waves = (tiles * sp + sms - 1) / sms;
+    return static_cast<double>(waves) * (static_cast<double>((nkb + sp - 1) / sp) + 2.0) * u +
+           (sp > 4 ? 360.0 : (sp > 1 ? 130.0 : 0.0));
+  };
+  // the split count: the cheapest of 1..4 (summed by the tile's last CTA) and the widest
+  // allowed (summed by the reduction kernel).  The sums' costs are fitted to the LoRA shapes
+  // timed on B200 (k-block ~1 us at these tiles): the reduction kernel ~10 us, the last CTA's
+  // sum of up to 4 partials ~4 us; u of q|k|v (N 192, K 4096) at 512 rows ran 17.5 us with 16
+  // splits and 23.5 with 4, at 2048 rows 35.5 with 10 and 23.6 with 4
+  auto split_for = [&](long long tiles, double u) -> long long {
     if (!p.workspace || !p.tile_counters || has_nf4 || tiles >= 100 || nkb < 16 || tiles > p.n_counters) return 1;
-    long long sp = (2 * sms + tiles - 1) / tiles;
-    sp = std::min<long long>(sp, nkb / 4);
-    sp = std::min<long long>(sp, 32);
-    while (sp > 1 && static_cast<unsigned long long>(sp) * p.M * p.N * 4ull > p.ws_bytes) --sp;
-    return sp < 1 ? 1 : sp;
+    long long mx = (2 * sms + tiles - 1) / tiles;
+    mx = std::min<long long>(mx, nkb / 4);
+    mx = std::min<long long>(mx, 32);
+    while (mx > 1 && static_cast<unsigned long long>(mx) * p.M * p.N * 4ull > p.ws_bytes) --mx;
+    if (mx < 1) mx = 1;
+    long long best_sp = 1;
+    double best_c = split_cost(tiles, 1, u);
+    const long long cands[5] = {2, 3, 4, mx, 0};
+    for (int i = 0; cands[i] > 0; ++i) {
+      const long long sp = cands[i];
+      if (sp > mx) continue;
+      const double c = split_cost(tiles, sp, u);
+      if (c < best_c * 0.999) {
+        best_c = c;
+        best_sp = sp;
+      }
+    }
+    return best_sp;
   };
   int MT = 1, BN = 128;
   double best = 1e300;
@@ -1339,10 +1362,8 @@ GemmPlan gemm_plan(const GemmParams& p, int sms, bool stream_k_allowed) {
     if (bn > 128 && p.N <= 128) continue;
     if (rope && (bn % p.rope_d != 0 || p.rope_cols % bn != 0)) continue;
     const long long tl = static_cast<long long>((p.N + bn - 1) / bn) * ((p.M + UM * mt - 1) / (UM * mt));
-    const long long sp = split_for(tl);
-    const long long waves = (tl * sp + sms - 1) / sms;
-    const double cost = static_cast<double>(waves) * (static_cast<double>((nkb + sp - 1) / sp) + 2.0) * unit[ci] +
-                        (sp > 4 ? 500.0 : 0.0);
+    const long long sp = split_for(tl, unit[ci]);
+    const double cost = split_cost(tl, sp, unit[ci]);
     if (cost < best * 0.999) {
       best = cost;
       MT = mt;
@@ -1399,7 +1420,10 @@ GemmPlan gemm_plan(const GemmParams& p, int sms, bool stream_k_allowed) {
   // NF4 GEMMs keep whole K (the 96-tile q|k|v GEMM ran 105 us split four ways, 65 us whole)
   const int BM = UM * MT;
   const long long tiles = static_cast<long long>((p.N + BN - 1) / BN) * ((p.M + BM - 1) / BM);
-  pl.splits = (has_nf4 || rope || pl.sk_ctas > 0) ? 1 : static_cast<int>(split_for(tiles));
+  int ci_chosen = 0;
+  for (int ci = 0; ci < 5; ++ci)
+    if (cand[ci][0] == MT && cand[ci][1] == BN) ci_chosen = ci;
+  pl.splits = (has_nf4 || rope || pl.sk_ctas > 0) ? 1 : static_cast<int>(split_for(tiles, unit[ci_chosen]));
   // up to 4 partials the tile's last CTA sums them; more run through the wide reduction
   // kernel (measured: 16-32 partials summed by one CTA per tile cost more than the launch)
   pl.fused_reduce = pl.splits <= 4 ? 1 : 0;
