@@ -1209,6 +1209,12 @@ template <int MT, int BN, bool SK = false>
 cudaError_t launch_tile(const GemmParams& p, cudaStream_t st) {
   using C = GemmCfg<MT, BN>;
   static_assert(C::STAGES >= 2, "tile too large for shared memory");
+  // Producer group g fills the k-blocks g, g + GROUPS, ...; when it waits for a stage to free,
+  // the stage's barrier must be at most one phase behind the one it needs, which holds when its
+  // own previous k-block (GROUPS back) already required the MMAs of that stage's previous use:
+  // STAGES >= GROUPS.  (With fewer stages a group can pass a parity check two phases early and
+  // arrive on a barrier that is still collecting the previous k-block.)
+  static_assert(C::STAGES >= GROUPS, "each producer group needs a stage of its own in flight");
   static std::atomic<int> attr_done{0};
   if (!attr_done.load()) {
     cudaError_t e =
