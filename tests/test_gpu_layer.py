@@ -68,6 +68,38 @@ def test_layer_forward_backward(pair, B, S, lora_on):
         assert np.all(grads[(0, p)][0] == 0)  # other layer untouched
 
 
+@pytest.mark.parametrize("B,S", [(1, 512), (2, 256)])
+def test_layer_whole_query_tiles(B, S):
+    """Sequences of whole 128-row query tiles at head_dim 64: the attention forward's O tiles
+    leave through its TMA store (a ragged last tile stores row by row), the K / V rings wrap
+    (four key tiles over three stages at S = 512), and the causal diagonal falls inside tiles."""
+    cfg = dict(synth.TINY)
+    p = Pair(cfg, seed=6, modes=("resident",), max_tokens=B * S, w_std=0.08)
+    try:
+        gm = p.models["resident"]
+        T, h = B * S, cfg["hidden"]
+        x = bf16_tensor(synth.bf16_bits_from_f32(synth.normal(31, T, (T, h), 1.0)))
+        dy = bf16_tensor(synth.bf16_bits_from_f32(synth.normal(32, T, (T, h), 1.0)))
+        gm.lora_grads.zero_()
+        y = gm.layer_fwd(1, x, B, S)
+        dx = gm.layer_bwd(1, dy, B, S)
+        torch.cuda.synchronize()
+        lo = {q: p.olora[(1, q)] for q in PROJ}
+        y_o, cache = om.layer_forward(cfg, p.olayers[1], lo, to64(x), B, S, enabled=True)
+        dx_o, g_o = om.layer_backward(cfg, p.olayers[1], lo, cache, to64(dy), B, S, enabled=True)
+        for got, want, base in ((to64(y), y_o, to64(x)), (to64(dx), dx_o, to64(dy))):
+            upd = float(np.sqrt(np.mean((want - base) ** 2)))
+            bound = 2.0 ** -7 * np.abs(want) + 0.1 * upd
+            worst = np.unravel_index(np.argmax(np.abs(got - want) - bound), want.shape)
+            assert np.all(np.abs(got - want) <= bound), (worst, got[worst], want[worst], upd)
+        grads = p.gpu_grads("resident")
+        for q in PROJ:
+            assert cosine(grads[(1, q)][0], g_o[q][0]) > 0.999, q
+            assert cosine(grads[(1, q)][1], g_o[q][1]) > 0.999, q
+    finally:
+        p.close()
+
+
 def test_lora_off_equals_zero_b_bitwise():
     cfg = dict(synth.TINY)
     a = Pair(cfg, seed=4, modes=("resident",), want_oracle=False)
