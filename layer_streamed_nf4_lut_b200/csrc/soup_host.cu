@@ -914,6 +914,8 @@ soup_status lora_grads(soup_model* m, int T, const uint16_t* g, long long ldg, i
 // The LoRA weight-gradient GEMMs (dA, dB) of a layer backward read only the main stream's
 // v = g B, g and saved activations, and write grad regions nothing reads before the step
 // ends: they run on a low-priority side stream beside the dX GEMMs, on SMs those leave idle.
+// Each group forks as soon as its v GEMM is done, before the projection's dX GEMM, so that the
+// last group of a layer (q|k|v) overlaps that GEMM instead of the layer's end.
 // The side stream forks after each v and joins before the layer call returns (the g buffers
 // are reused by the next layer).  Same kernels, same order per region: same bits.
 soup_status grads_fork(soup_model* m, cudaStream_t st, cudaStream_t* gs) {
@@ -965,18 +967,18 @@ soup_status layer_backward_body(soup_model* m, int i, const LayerView& L, const 
     add_seg(p, h, opnd(OP_BF16_K, dy, h), opnd(OP_BF16_MN, P + lora_off(c, i, 6, 1), r));
     SOUP_TRY(run_gemm(m, p, st, "lora v down"));
   }
+  cudaStream_t gs = st;
+  if (lora) {
+    SOUP_TRY(grads_fork(m, st, &gs));
+    SOUP_TRY(lora_grads(m, T, dy, h, h, A.ud, r, G + lora_off(c, i, 6, 1), A.m, I, I, m->vd, r, r,
+                        G + lora_off(c, i, 6, 0), gs, true, true));
+  }
   {
     GemmParams p = gemm_base(m, T, I, m->dm, I, 0, 1.f);
     p.nf4 = group_of(m, L, {6});
     add_seg(p, h, opnd(OP_BF16_K, dy, h), opnd(OP_NF4_MN, nullptr, 0));
     if (lora) add_seg(p, r, opnd(OP_BF16_K, m->vd, r), opnd(OP_BF16_MN, P + lora_off(c, i, 6, 0), I));
     SOUP_TRY(run_gemm(m, p, st, "down dX"));
-  }
-  cudaStream_t gs = st;
-  if (lora) {
-    SOUP_TRY(grads_fork(m, st, &gs));
-    SOUP_TRY(lora_grads(m, T, dy, h, h, A.ud, r, G + lora_off(c, i, 6, 1), A.m, I, I, m->vd, r, r,
-                        G + lora_off(c, i, 6, 0), gs, true, true));
   }
   SOUP_TRY(launch(m, st, CAT_SWIGLU, 0, 10.0 * T * I, "swiglu bwd",
                   [&] { return swiglu_bwd_launch(m->dm, A.gu, T, I, m->dgu, st); }));
@@ -991,6 +993,14 @@ soup_status layer_backward_body(soup_model* m, int i, const LayerView& L, const 
               opnd(OP_BF16_MN, P + lora_off(c, i, 4 + q, 1) - q * r, r, 1.f, q * r, (q + 1) * r));
     SOUP_TRY(run_gemm(m, p, st, "lora v gate/up"));
   }
+  if (lora) {
+    SOUP_TRY(grads_fork(m, st, &gs));
+    for (int q = 0; q < 2; ++q)
+      SOUP_TRY(lora_grads(m, T, m->dgu + q * I, 2 * I, I, A.ugu + q * r, 2 * r, G + lora_off(c, i, 4 + q, 1), nullptr,
+                          0, 0, nullptr, 0, 0, nullptr, gs, true, false));
+    SOUP_TRY(lora_grads(m, T, nullptr, 0, 0, nullptr, 0, nullptr, A.n2, h, h, m->vgu, 2 * r, 2 * r,
+                        G + lora_off(c, i, 4, 0), gs, false, true));
+  }
   {
     GemmParams p = gemm_base(m, T, h, m->dn, h, 0, 1.f);
     p.nf4 = group_of(m, L, {4, 5});
@@ -999,14 +1009,6 @@ soup_status layer_backward_body(soup_model* m, int i, const LayerView& L, const 
       for (int q = 0; q < 2; ++q)
         add_seg(p, r, opnd(OP_BF16_K, m->vgu + q * r, 2 * r), opnd(OP_BF16_MN, P + lora_off(c, i, 4 + q, 0), h));
     SOUP_TRY(run_gemm(m, p, st, "gate/up dX"));
-  }
-  if (lora) {
-    SOUP_TRY(grads_fork(m, st, &gs));
-    for (int q = 0; q < 2; ++q)
-      SOUP_TRY(lora_grads(m, T, m->dgu + q * I, 2 * I, I, A.ugu + q * r, 2 * r, G + lora_off(c, i, 4 + q, 1), nullptr,
-                          0, 0, nullptr, 0, 0, nullptr, gs, true, false));
-    SOUP_TRY(lora_grads(m, T, nullptr, 0, 0, nullptr, 0, nullptr, A.n2, h, h, m->vgu, 2 * r, 2 * r,
-                        G + lora_off(c, i, 4, 0), gs, false, true));
   }
   const double act = 2.0 * T * h;
   SOUP_TRY(launch(m, st, CAT_RMSNORM, 0, 4 * act + 4.0 * T, "rmsnorm bwd",
@@ -1017,17 +1019,17 @@ soup_status layer_backward_body(soup_model* m, int i, const LayerView& L, const 
     add_seg(p, h, opnd(OP_BF16_K, m->dx1, h), opnd(OP_BF16_MN, P + lora_off(c, i, 3, 1), r));
     SOUP_TRY(run_gemm(m, p, st, "lora v o"));
   }
+  if (lora) {
+    SOUP_TRY(grads_fork(m, st, &gs));
+    SOUP_TRY(lora_grads(m, T, m->dx1, h, h, A.uo, r, G + lora_off(c, i, 3, 1), A.o, qd, qd, m->vo, r, r,
+                        G + lora_off(c, i, 3, 0), gs, true, true));
+  }
   {
     GemmParams p = gemm_base(m, T, qd, m->da, qd, 0, 1.f);
     p.nf4 = group_of(m, L, {3});
     add_seg(p, h, opnd(OP_BF16_K, m->dx1, h), opnd(OP_NF4_MN, nullptr, 0));
     if (lora) add_seg(p, r, opnd(OP_BF16_K, m->vo, r), opnd(OP_BF16_MN, P + lora_off(c, i, 3, 0), qd));
     SOUP_TRY(run_gemm(m, p, st, "o dX"));
-  }
-  if (lora) {
-    SOUP_TRY(grads_fork(m, st, &gs));
-    SOUP_TRY(lora_grads(m, T, m->dx1, h, h, A.uo, r, G + lora_off(c, i, 3, 1), A.o, qd, qd, m->vo, r, r,
-                        G + lora_off(c, i, 3, 0), gs, true, true));
   }
   // ---- attention, RoPE
   AttnShape as{B, S, c.n_heads, c.n_kv_heads, c.head_dim, QKV, m->pack_pl, m->pack_rl, m->rope_cos, m->rope_sin};
@@ -1047,6 +1049,14 @@ soup_status layer_backward_body(soup_model* m, int i, const LayerView& L, const 
               opnd(OP_BF16_MN, P + lora_off(c, i, q, 1) - q * r, r, 1.f, q * r, (q + 1) * r));
     SOUP_TRY(run_gemm(m, p, st, "lora v qkv"));
   }
+  if (lora) {
+    SOUP_TRY(grads_fork(m, st, &gs));
+    for (int q = 0; q < 3; ++q)
+      SOUP_TRY(lora_grads(m, T, m->dqkv + off[q], QKV, outs[q], A.uqkv + q * r, 3 * r, G + lora_off(c, i, q, 1),
+                          nullptr, 0, 0, nullptr, 0, 0, nullptr, gs, true, false));
+    SOUP_TRY(lora_grads(m, T, nullptr, 0, 0, nullptr, 0, nullptr, A.n1, h, h, m->vqkv, 3 * r, 3 * r,
+                        G + lora_off(c, i, 0, 0), gs, false, true));
+  }
   {
     GemmParams p = gemm_base(m, T, h, m->dn, h, 0, 1.f);
     p.nf4 = group_of(m, L, {0, 1, 2});
@@ -1055,14 +1065,6 @@ soup_status layer_backward_body(soup_model* m, int i, const LayerView& L, const 
       for (int q = 0; q < 3; ++q)
         add_seg(p, r, opnd(OP_BF16_K, m->vqkv + q * r, 3 * r), opnd(OP_BF16_MN, P + lora_off(c, i, q, 0), h));
     SOUP_TRY(run_gemm(m, p, st, "qkv dX"));
-  }
-  if (lora) {
-    SOUP_TRY(grads_fork(m, st, &gs));
-    for (int q = 0; q < 3; ++q)
-      SOUP_TRY(lora_grads(m, T, m->dqkv + off[q], QKV, outs[q], A.uqkv + q * r, 3 * r, G + lora_off(c, i, q, 1),
-                          nullptr, 0, 0, nullptr, 0, 0, nullptr, gs, true, false));
-    SOUP_TRY(lora_grads(m, T, nullptr, 0, 0, nullptr, 0, nullptr, A.n1, h, h, m->vqkv, 3 * r, 3 * r,
-                        G + lora_off(c, i, 0, 0), gs, false, true));
   }
   SOUP_TRY(launch(m, st, CAT_RMSNORM, 0, 4 * act + 4.0 * T, "rmsnorm bwd",
                   [&] { return rmsnorm_bwd_launch(m->dn, A.x, A.rstd1, L.gamma[0], m->dx1, T, h, dx, st); }));
