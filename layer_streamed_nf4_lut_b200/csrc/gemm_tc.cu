@@ -985,19 +985,32 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
 }
 
 // Sum of the split-K partial tiles in split order, then the normal epilogue (the wide form
-// for many splits: one thread per 8 outputs instead of one CTA per tile).
+// for many splits: one thread per 8 outputs instead of one CTA per tile, 128-thread blocks so
+// that the few thousand threads of a LoRA-sized output spread over more SMs).
 __global__ void splitk_reduce_kernel(const __grid_constant__ GemmParams p) {
   const long long n8 = p.N / 8;
   const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (idx >= static_cast<long long>(p.M) * n8) return;
   const int row = static_cast<int>(idx / n8), col = static_cast<int>(idx % n8) * 8;
   float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
-  for (int s = 0; s < p.splits; ++s) {
-    const float4* src = reinterpret_cast<const float4*>(p.workspace + (static_cast<long long>(s) * p.M + row) * p.N + col);
-    const float4 a = src[0], b = src[1];
-    v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w;
-    v[4] += b.x; v[5] += b.y; v[6] += b.z; v[7] += b.w;
+  // eight splits' loads in flight at a time, added in split order
+#pragma unroll 1
+  for (int s0 = 0; s0 < p.splits; s0 += 8) {
+    float4 a[8][2];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (s0 + u >= p.splits) break;
+      const float4* src =
+          reinterpret_cast<const float4*>(p.workspace + (static_cast<long long>(s0 + u) * p.M + row) * p.N + col);
+      a[u][0] = __ldcg(src);
+      a[u][1] = __ldcg(src + 1);
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (s0 + u >= p.splits) break;
+      v[0] += a[u][0].x; v[1] += a[u][0].y; v[2] += a[u][0].z; v[3] += a[u][0].w;
+      v[4] += a[u][1].x; v[5] += a[u][1].y; v[6] += a[u][1].z; v[7] += a[u][1].w;
+    }
   }
 #pragma unroll
   for (int j = 0; j < 8; ++j) v[j] *= p.alpha;
@@ -1237,7 +1250,7 @@ cudaError_t launch_tile(const GemmParams& p, cudaStream_t st) {
   }
   if (p.splits <= 1 || p.fused_reduce) return e;
   const long long work = static_cast<long long>(p.M) * (p.N / 8);
-  splitk_reduce_kernel<<<static_cast<unsigned>((work + 255) / 256), 256, 0, st>>>(p);
+  splitk_reduce_kernel<<<static_cast<unsigned>((work + 127) / 128), 128, 0, st>>>(p);
   ++g_kernel_launches;
   return cudaGetLastError();
 }
