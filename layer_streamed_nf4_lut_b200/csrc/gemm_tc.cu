@@ -63,9 +63,15 @@ struct GemmCfg {
   static constexpr int RAW_CODE_BYTES = BN * 32;
   static constexpr int RAW_Q8_BYTES = (BN > 64 ? BN : 64) * 16;
   static constexpr int RAW_BYTES = RAW_CODE_BYTES + RAW_Q8_BYTES;
+  // Every operand stage comes with at least one raw slot (RAW_SLOTS >= STAGES): a producer that
+  // waits for raw k-block kb has seen the MMAs of kb - STAGES retire, so every raw k-block up
+  // to kb - STAGES has landed and been decoded; with RAW_SLOTS >= STAGES that covers kb -
+  // RAW_SLOTS, the previous use of kb's slot, and the slot's parity wait cannot alias it.
+  // (With more stages than raw slots only the order in which TMA loads complete keeps the
+  // phases apart.)
   static constexpr int CTRL_BYTES = 640;
   static constexpr int AVAIL = SMEM_LIMIT - 1024 - CTRL_BYTES;
-  static constexpr int STAGES_FIT = (AVAIL - 4 * RAW_BYTES) / STAGE_BYTES;
+  static constexpr int STAGES_FIT = AVAIL / (STAGE_BYTES + RAW_BYTES);
   static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
   static constexpr int RAW_FIT = (AVAIL - STAGES * STAGE_BYTES) / RAW_BYTES;
   static constexpr int RAW_SLOTS = RAW_FIT > 16 ? 16 : RAW_FIT;
@@ -1228,6 +1234,7 @@ cudaError_t launch_tile(const GemmParams& p, cudaStream_t st) {
   // STAGES >= GROUPS.  (With fewer stages a group can pass a parity check two phases early and
   // arrive on a barrier that is still collecting the previous k-block.)
   static_assert(C::STAGES >= GROUPS, "each producer group needs a stage of its own in flight");
+  static_assert(C::RAW_SLOTS >= C::STAGES, "a raw slot's parity wait needs a slot per operand stage");
   static std::atomic<int> attr_done{0};
   if (!attr_done.load()) {
     cudaError_t e =
