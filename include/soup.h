@@ -258,6 +258,9 @@ soup_status soup_layer_bwd(soup_model* model, int layer, const void* dy, void* d
 
 /* One training step: embedding, streamed forward over all layers, head and loss, streamed
  * backward, LoRA gradients (zeroed first) and, if batch->apply_optimizer, the AdamW update
+ * (each layer's LoRA slice is updated during the backward pass, as soon as its gradients are
+ * complete, with the same arithmetic as soup_optimizer_step; a step that fails part-way may
+ * leave some slices updated)
  * (the pages' SFT and preference training under layer streaming: rug.gal "En detalle";
  * imasters "Do SFT para os métodos de preferência"; guillermodelpino soup.yaml example, lr).
  * SFT streams 2L-2 layer loads from a cold streamer (the two top layers are reused at the

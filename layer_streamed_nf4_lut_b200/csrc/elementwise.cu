@@ -485,9 +485,14 @@ __global__ void ce_grad_t_kernel(const float* __restrict__ logits, const float* 
 // ---------------------------------------------------------------- AdamW (fp32, bias-corrected)
 __global__ void adamw_kernel(float* __restrict__ p, const float* __restrict__ g, float* __restrict__ m,
                              float* __restrict__ v, uint16_t* __restrict__ pb, long long n, float lr, float b1, float b2,
-                             float eps, float wd, float bc1, float bc2) {
+                             float eps, float wd, float bc1, float bc2, const float* __restrict__ hp) {
   const long long i4 = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i4 * 4 >= n) return;
+  if (hp) {  // lr and the bias corrections of this step, written to device memory by the host
+    lr = hp[0];
+    bc1 = hp[1];
+    bc2 = hp[2];
+  }
   if (i4 * 4 + 4 <= n) {
     float4 pp = reinterpret_cast<float4*>(p)[i4];
     const float4 gg = reinterpret_cast<const float4*>(g)[i4];
@@ -708,14 +713,29 @@ cudaError_t f32_to_bf16_launch(const float* x, uint16_t* y, long long n, cudaStr
   return cudaGetLastError();
 }
 
+void adamw_bias_corrections(float b1, float b2, int t, float* bc1, float* bc2) {
+  *bc1 = static_cast<float>(1.0 / (1.0 - pow(static_cast<double>(b1), t)));
+  *bc2 = static_cast<float>(1.0 / (1.0 - pow(static_cast<double>(b2), t)));
+}
+
 cudaError_t adamw_launch(float* p, const float* g, float* m, float* v, uint16_t* pb, long long n, float lr, float b1,
                          float b2, float eps, float wd, int t, cudaStream_t st) {
   if (n <= 0) return cudaSuccess;
-  const float bc1 = static_cast<float>(1.0 / (1.0 - pow(static_cast<double>(b1), t)));
-  const float bc2 = static_cast<float>(1.0 / (1.0 - pow(static_cast<double>(b2), t)));
+  float bc1, bc2;
+  adamw_bias_corrections(b1, b2, t, &bc1, &bc2);
   const long long n4 = (n + 3) / 4;
   adamw_kernel<<<static_cast<unsigned>((n4 + 255) / 256), 256, 0, st>>>(p, g, m, v, pb, n, lr, b1, b2, eps, wd, bc1,
-                                                                          bc2);
+                                                                          bc2, nullptr);
+  ++g_kernel_launches;
+  return cudaGetLastError();
+}
+
+cudaError_t adamw_hp_launch(float* p, const float* g, float* m, float* v, uint16_t* pb, long long n, float b1,
+                            float b2, float eps, float wd, const float* hp, cudaStream_t st) {
+  if (n <= 0) return cudaSuccess;
+  const long long n4 = (n + 3) / 4;
+  adamw_kernel<<<static_cast<unsigned>((n4 + 255) / 256), 256, 0, st>>>(p, g, m, v, pb, n, 0.f, b1, b2, eps, wd, 1.f,
+                                                                          1.f, hp);
   ++g_kernel_launches;
   return cudaGetLastError();
 }

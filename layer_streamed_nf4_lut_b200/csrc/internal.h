@@ -257,6 +257,12 @@ cudaError_t ce_grad_launch(const float* logits, const float* lse, const int32_t*
 // AdamW on fp32 parameters; also writes their bf16 copy `pb` (may be null).
 cudaError_t adamw_launch(float* p, const float* g, float* m, float* v, uint16_t* pb, long long n, float lr, float b1,
                          float b2, float eps, float wd, int t, cudaStream_t st);
+// The same update with lr and the bias corrections read from device memory (hp[0] = lr,
+// hp[1] = 1/(1-b1^t), hp[2] = 1/(1-b2^t)), so that a captured graph applies each step's values.
+cudaError_t adamw_hp_launch(float* p, const float* g, float* m, float* v, uint16_t* pb, long long n, float b1,
+                            float b2, float eps, float wd, const float* hp, cudaStream_t st);
+// 1/(1-b1^t) and 1/(1-b2^t) as the update uses them
+void adamw_bias_corrections(float b1, float b2, int t, float* bc1, float* bc2);
 cudaError_t busy_wait_launch(long long cycles, cudaStream_t st);  // profiling aid, not counted as a launch
 cudaError_t null_launch(cudaStream_t st);
 // one thread waits on a barrier nothing arrives on, limit_ns ns, then sets *err (timeout)

@@ -172,6 +172,8 @@ size_t lora_numel_of(const soup_model_config& c) {
   for (int p = 0; p < 7; ++p) per += static_cast<size_t>(c.lora_r) * (s[p].in + s[p].out);
   return per * c.n_layers;
 }
+// LoRA parameters of one layer (a contiguous slice of the flat buffer, starting at lora_off(c, l, 0, 0))
+size_t lora_layer_numel(const soup_model_config& c) { return lora_numel_of(c) / c.n_layers; }
 // offset of A_p (which=0) or B_p (which=1) of a layer in the flat LoRA buffer
 size_t lora_off(const soup_model_config& c, int layer, int proj, int which) {
   ProjShape s[7];
@@ -239,6 +241,12 @@ struct soup_model {
   size_t lora_n = 0;
   int lora_enabled = 1;
   int adam_t = 0;
+  // Set while soup_step's backward pass runs with the optimizer on: the backward call of layer
+  // i then also applies AdamW to layer i+1's LoRA slice (its gradients are complete and nothing
+  // reads its parameters again this step), on the gradient side stream; lr and the bias
+  // corrections come from device memory (scal + ADAM_HP_WORD) so that captured graphs replay
+  // each step's values.
+  int adam_in_bwd = 0;
 
   // activations
   std::vector<soup::Saved> saved;
@@ -263,7 +271,7 @@ struct soup_model {
   float* gemm_ws = nullptr;        // split-K partial tiles
   float *rope_cos = nullptr, *rope_sin = nullptr;  // [max_tokens, head_dim/2]
   size_t gemm_ws_bytes = 0;
-  float* host_scal = nullptr;      // pinned 2-word staging for the loss + error readback
+  float* host_scal = nullptr;      // pinned staging: words 0-1 loss + error readback, 4-6 AdamW lr + bias corrections
 
   std::vector<void*> dev_allocs;
   // per-layer CUDA graphs of the step's layer calls (key: direction, layer, weight buffer,
@@ -281,6 +289,7 @@ struct soup_model {
   struct GraphKey {
     int dir, layer, B, S, lora, pack;  // pack: shared-prefix length of a packed pair step (0: none)
     int tcat;                          // mask of the categories whose launches carry event nodes
+    int adam;                          // backward call that also updates layer + 1's LoRA slice
     const void *base, *in, *out;
     bool operator==(const GraphKey& o) const { return std::memcmp(this, &o, sizeof(GraphKey)) == 0; }
   };
@@ -937,6 +946,24 @@ soup_status grads_join(soup_model* m, cudaStream_t st) {
   return SOUP_OK;
 }
 
+// Word offset in `scal` of the AdamW hyper-parameters of the running step (lr, 1/(1-b1^t),
+// 1/(1-b2^t)).
+constexpr int ADAM_HP_WORD = 8;
+constexpr float ADAM_B1 = 0.9f, ADAM_B2 = 0.999f, ADAM_EPS = 1e-8f, ADAM_WD = 0.f;
+
+bool adam_after(const soup_model* m, int i) { return m->adam_in_bwd && m->lora_p && i + 1 < m->cfg.n_layers; }
+
+// AdamW on layer l's LoRA slice with the step's hyper-parameters from device memory.
+soup_status adamw_layer(soup_model* m, int l, cudaStream_t st) {
+  const size_t off = lora_off(m->cfg, l, 0, 0), n = lora_layer_numel(m->cfg);
+  const float* hp = reinterpret_cast<const float*>(m->scal + ADAM_HP_WORD);
+  return launch(m, st, CAT_ADAMW, 0, 28.0 * static_cast<double>(n), "adamw", [&] {
+    return adamw_hp_launch(m->lora_p + off, m->lora_g + off, m->lora_m + off, m->lora_v + off,
+                           m->lora_bf16 ? m->lora_bf16 + off : nullptr, static_cast<long long>(n), ADAM_B1, ADAM_B2,
+                           ADAM_EPS, ADAM_WD, hp, st);
+  });
+}
+
 soup_status layer_backward_body(soup_model* m, int i, const LayerView& L, const uint16_t* dy, uint16_t* dx, int B,
                                 int S, cudaStream_t st);
 soup_status layer_backward(soup_model* m, int i, const LayerView& L, const uint16_t* dy, uint16_t* dx, int B, int S,
@@ -955,6 +982,13 @@ soup_status layer_backward_body(soup_model* m, int i, const LayerView& L, const 
     return SOUP_ERR_STATE;
   }
   SOUP_TRY(timed_calibration(m, st));
+  if (adam_after(m, i)) {
+    // layer i+1's update, beside this layer's backward: its last readers (the backward call of
+    // layer i+1, joined at that call's end) are done
+    cudaStream_t gs;
+    SOUP_TRY(grads_fork(m, st, &gs));
+    SOUP_TRY(adamw_layer(m, i + 1, gs));
+  }
   const int T = B * S, h = c.hidden, r = c.lora_r, I = c.intermediate;
   const int qd = c.n_heads * c.head_dim, kvd = c.n_kv_heads * c.head_dim, QKV = m->qkv_cols;
   const float s = m->s_lora;
@@ -1135,6 +1169,7 @@ soup_status run_layer(soup_model* m, int dir, int i, const uint8_t* base, const 
   key.lora = lora;
   key.pack = m->pack_pl;
   key.tcat = m->tcat;
+  key.adam = (dir == 1 && adam_after(m, i)) ? 1 : 0;
   key.base = base;
   key.in = in;
   key.out = out;
@@ -1424,15 +1459,22 @@ soup_status do_step_body(soup_model* m, soup_loss kind, const soup_batch* bt, fl
   }
   uint16_t* other = (xL == m->xa) ? m->xb : m->xa;
   SOUP_TRY(head_backward(m, xL, Bx, Sx, other, st));
-  // backward ping-pongs between `other` and the buffer that held x_L (no longer needed)
-  SOUP_TRY(stream_backward_pass(m, Bx, Sx, other, xL, st));
   if (bt->apply_optimizer) {
+    // this step's lr and bias corrections, for the AdamW launches inside the backward pass
+    // (the pinned staging words are free: the previous step's read-back has completed)
     m->adam_t += 1;
-    SOUP_TRY(launch(m, st, CAT_ADAMW, 0, 28.0 * m->lora_n, "adamw", [&] {
-      return adamw_launch(m->lora_p, m->lora_g, m->lora_m, m->lora_v, m->lora_bf16, static_cast<long long>(m->lora_n), bt->lr, 0.9f,
-                          0.999f, 1e-8f, 0.f, m->adam_t, st);
-    }));
+    float* hp = m->host_scal + 4;
+    hp[0] = bt->lr;
+    adamw_bias_corrections(ADAM_B1, ADAM_B2, m->adam_t, &hp[1], &hp[2]);
+    SOUP_CK(cudaMemcpyAsync(m->scal + ADAM_HP_WORD, hp, 3 * sizeof(float), cudaMemcpyHostToDevice, st));
+    m->adam_in_bwd = 1;
   }
+  // backward ping-pongs between `other` and the buffer that held x_L (no longer needed); with
+  // the optimizer on, layer i's call also updates layer i+1's LoRA slice
+  const soup_status sb = stream_backward_pass(m, Bx, Sx, other, xL, st);
+  m->adam_in_bwd = 0;
+  SOUP_TRY(sb);
+  if (bt->apply_optimizer) SOUP_TRY(adamw_layer(m, 0, st));  // the last slice
   m->stats.kernel_launches += g_kernel_launches.load() - launches0;
   SOUP_TRY(read_scalars(m, st, loss_out));
   m->stats.steps += 1;
@@ -2021,8 +2063,8 @@ soup_status soup_optimizer_step(soup_model* m, float lr, void* stream) {
     m->adam_t += 1;
     const long long l0 = g_kernel_launches.load();
     soup_status s = check_launch(m, adamw_launch(m->lora_p, m->lora_g, m->lora_m, m->lora_v, m->lora_bf16,
-                                                 static_cast<long long>(m->lora_n), lr, 0.9f, 0.999f, 1e-8f, 0.f,
-                                                 m->adam_t, static_cast<cudaStream_t>(stream)),
+                                                 static_cast<long long>(m->lora_n), lr, ADAM_B1, ADAM_B2, ADAM_EPS,
+                                                 ADAM_WD, m->adam_t, static_cast<cudaStream_t>(stream)),
                                  "adamw");
     m->stats.kernel_launches += g_kernel_launches.load() - l0;
     return s;
