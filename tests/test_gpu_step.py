@@ -190,26 +190,32 @@ def test_per_layer_adamw_in_backward_same_bits_as_whole_update():
     """With the optimizer on, soup_step updates each layer's LoRA slice during the backward pass
     (layer i+1's slice beside layer i's backward, layer 0's at the end); parameters, both AdamW
     moments and the losses equal, bit for bit, steps without the optimizer each followed by the
-    whole-vector soup_optimizer_step, over eager, captured and replayed steps."""
+    whole-vector soup_optimizer_step, over eager, captured and replayed steps, with lr changing
+    between steps and the two forms interleaved."""
     cfg = dict(TINY4, batch=2)
     ids = torch.from_numpy(synth.token_batch(cfg, 52)).cuda()
     out = {}
-    for mode in ("in_backward", "after"):
+    # the mixed schedule alternates the two forms, so each layer's backward graph is captured
+    # and replayed both with and without the update, and lr changes between steps
+    schedules = {"in_backward": [True] * 5, "after": [False] * 5, "mixed": [True, False, True, True, False]}
+    lrs = [1e-3, 2e-3, 1e-3, 5e-4, 1e-3]
+    for mode, sched in schedules.items():
         p = Pair(TINY4, seed=29, modes=("streamed",), want_oracle=False, max_tokens=2 * 64)
         try:
             gm = p.models["streamed"]
             losses = []
-            for _ in range(4):
-                if mode == "in_backward":
-                    losses.append(gm.step(ids, lr=1e-3, apply_optimizer=True))
+            for in_bwd, lr in zip(sched, lrs):
+                if in_bwd:
+                    losses.append(gm.step(ids, lr=lr, apply_optimizer=True))
                 else:
-                    losses.append(gm.step(ids, lr=1e-3, apply_optimizer=False))
-                    gm.optimizer_step(1e-3)
+                    losses.append(gm.step(ids, lr=lr, apply_optimizer=False))
+                    gm.optimizer_step(lr)
             torch.cuda.synchronize()
             out[mode] = (losses, gm.lora_params.clone(), gm.adam_m.clone(), gm.adam_v.clone())
         finally:
             p.close()
-    a, b = out["in_backward"], out["after"]
-    assert a[0] == b[0]
-    for x, y in zip(a[1:], b[1:]):
-        assert torch.equal(x.view(torch.int32), y.view(torch.int32))
+    for other in ("after", "mixed"):
+        a, b = out["in_backward"], out[other]
+        assert a[0] == b[0], other
+        for x, y in zip(a[1:], b[1:]):
+            assert torch.equal(x.view(torch.int32), y.view(torch.int32)), other
