@@ -990,6 +990,254 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
   }
 }
 
+// ---------------------------------------------------------------- the TMEM-A forward kernel
+// NF4 forward GEMMs with enough output tiles (y = x W^T (+ LoRA K-blocks), no residual): the
+// tile is transposed, D^T[w, t] = W[w, :] . x[t, :], 128 weight rows (TMEM lanes) x 256 tokens.
+// The producers put the dequantised weight tile straight into tensor memory (tcgen05.st, one
+// weight row per thread) and tcgen05.mma reads it there as its A operand; only the activation
+// tile (TMA) and the raw NF4 bytes pass through shared memory.  Against the shared-memory form
+// (activations and decoded weights both staged in shared memory and both read by every MMA)
+// this moves ~76 KB of shared memory per 4.2 MFLOP k-block instead of ~124 KB.  LoRA segments
+// are further K-blocks: the producers copy the LoRA-B rows of the tile (bf16, zero outside the
+// segment's row window) into tensor memory and the u tile comes by TMA.
+struct TsCfg {
+  static constexpr int BW = 128;  // weight rows (output columns) per CTA
+  static constexpr int BT = 256;  // tokens (output rows) per CTA: the MMA's N
+  static constexpr int STAGES = 5;
+  static constexpr int RAW_SLOTS = 6;
+  static constexpr int X_BYTES = BT * 128;
+  static constexpr int RAW_CODE_BYTES = BW * 32, RAW_Q8_BYTES = BW * 16;
+  static constexpr int RAW_BYTES = RAW_CODE_BYTES + RAW_Q8_BYTES;
+  static constexpr int CTRL_BYTES = 512;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * X_BYTES + RAW_SLOTS * RAW_BYTES + CTRL_BYTES;
+  static constexpr int ACC_COL = 0, W_COL = BT, TMEM_COLS = 512;
+};
+static_assert(TsCfg::W_COL + TsCfg::STAGES * 32 <= TsCfg::TMEM_COLS, "TMEM budget");
+static_assert(TsCfg::RAW_SLOTS >= TsCfg::STAGES && TsCfg::STAGES >= GROUPS, "ring invariants");
+static_assert(TsCfg::SMEM_BYTES <= SMEM_LIMIT, "shared memory");
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]),
+      "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
+      "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+__global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_ts_kernel(const __grid_constant__ GemmParams p) {
+  using C = TsCfg;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* base = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+  uint8_t* raw_base = base + C::STAGES * C::X_BYTES;
+  uint8_t* ctrl = raw_base + C::RAW_SLOTS * C::RAW_BYTES;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(ctrl + 4);
+  float* seg_mean = reinterpret_cast<float*>(ctrl + 16);  // up to 3 NF4 tensors
+  uint64_t* full = reinterpret_cast<uint64_t*>(ctrl + 64);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* raw_full = empty + C::STAGES;
+  uint64_t* raw_empty = raw_full + C::RAW_SLOTS;
+  uint64_t* done = raw_empty + C::RAW_SLOTS;
+  static_assert(64 + 8 * (2 * C::STAGES + 2 * C::RAW_SLOTS + 1) <= C::CTRL_BYTES, "control block overflow");
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n0 = blockIdx.x * C::BW;  // first weight row = output column
+  const int m0 = blockIdx.y * C::BT;  // first token = output row
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], GROUP_THREADS / 32 + 1);  // 4 producer warps + the activation TMA issuer
+      mbar_init(&empty[s], 1);
+    }
+    for (int r = 0; r < C::RAW_SLOTS; ++r) {
+      mbar_init(&raw_full[r], 1);
+      mbar_init(&raw_empty[r], GROUP_THREADS / 32);
+    }
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (threadIdx.x >= 32 && threadIdx.x < 32 + p.nf4.nseg) seg_mean[threadIdx.x - 32] = *p.nf4.seg[threadIdx.x - 32].mean;
+  if (warp == EPI_WARP0) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  // segment 0: the NF4 weight (raw-staged); then the active LoRA segments, one after another
+  const int nk0 = p.seg[0].K / BK;  // a multiple of 16 k-blocks (raw staging needs it)
+
+  if (warp < PRODUCER_WARPS) {
+    // ---------------------------------------------- producers: weight row r of the tile = TMEM lane r
+    const int grp = warp >> 2, r = threadIdx.x & (GROUP_THREADS - 1);
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const float(&cb)[16] = p.lut;
+    const int w = n0 + r;
+    const int si = nf4_seg_of(p.nf4, n0);
+    const NF4Seg& ns = p.nf4.seg[si];
+    const long long cpr = p.nf4.cols >> 6;
+    int kb = 0;
+    for (int s = 0; s < p.nseg; ++s) {
+      const GemmSeg& sg = p.seg[s];
+      if (!seg_active(sg, n0, C::BW)) continue;
+      const int nk = (sg.K + BK - 1) / BK;
+      const int first = kb + ((grp - kb % GROUPS) + GROUPS) % GROUPS;
+      for (int g = first; g < kb + nk; g += GROUPS) {
+        const int kk = g - kb;  // k-block within the segment
+        const int st = g % C::STAGES;
+        const uint32_t ph = static_cast<uint32_t>(g / C::STAGES) & 1u;
+        uint32_t o[32];
+        if (s == 0) {
+          const int rs = g % C::RAW_SLOTS;
+          const uint32_t rph = static_cast<uint32_t>(g / C::RAW_SLOTS) & 1u;
+          const float s2 = (w < p.N) ? __ldg(ns.scales + ((static_cast<long long>(w - ns.row_begin) * cpr + kk) >> 8))
+                                     : 0.f;
+          mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, p.err);
+          mbar_wait_bounded(&raw_full[rs], rph, abort_flag, p.err);
+          const uint32_t rc = smem_u32(raw_base + rs * C::RAW_BYTES) + r * 32;
+          const uint4 w0 = lds128(rc), w1 = lds128(rc + 16);
+          const int q8 = lds_s8(smem_u32(raw_base + rs * C::RAW_BYTES + C::RAW_CODE_BYTES) + r * 16 + (kk & 15));
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&raw_empty[rs]);  // this warp's reads of the raw slot are done
+          const float mh = __fadd_rn(__fmul_rn(static_cast<float>(q8), s2), seg_mean[si]);
+          const BlockLut t = block_lut(cb, mh);
+          const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+          for (int kc = 0; kc < 8; ++kc) {
+            const uint4 v = decode_word_lut(words[kc], t);
+            o[4 * kc] = v.x;
+            o[4 * kc + 1] = v.y;
+            o[4 * kc + 2] = v.z;
+            o[4 * kc + 3] = v.w;
+          }
+          if (w >= p.N) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) o[j] = 0u;
+          }
+        } else {
+          // LoRA-B row w (bf16, K-major): columns kk*64 .. +64 of K, zero outside the row window
+          const bool in = w < p.N && w >= sg.B.row_lo && w < sg.B.row_hi;
+          const int k0 = kk * BK;
+          const uint16_t* src = static_cast<const uint16_t*>(sg.B.ptr) + static_cast<long long>(w) * sg.B.ld + k0;
+          uint4 v[8];
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            v[c] = (in && k0 + c * 8 < sg.K) ? *reinterpret_cast<const uint4*>(src + c * 8) : make_uint4(0, 0, 0, 0);
+          mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, p.err);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            o[4 * c] = v[c].x;
+            o[4 * c + 1] = v[c].y;
+            o[4 * c + 2] = v[c].z;
+            o[4 * c + 3] = v[c].w;
+          }
+        }
+        tmem_st32(tmem + lane_base + C::W_COL + st * 32, o);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&full[st]);
+      }
+      kb += nk;
+    }
+  } else {
+    const int q = warp - EPI_WARP0;  // TMEM lane quarter of this epilogue warp
+    if (warp == EPI_WARP0 + 1 && lane == 0) {
+      // ---------------------------------------------- TMA issuer: the token tiles (x, then u)
+      int kb = 0;
+      for (int s = 0; s < p.nseg; ++s) {
+        const GemmSeg& sg = p.seg[s];
+        if (!seg_active(sg, n0, C::BW)) continue;
+        const int nk = (sg.K + BK - 1) / BK;
+        for (int kk = 0; kk < nk; ++kk, ++kb) {
+          const int st = kb % C::STAGES;
+          const uint32_t ph = static_cast<uint32_t>(kb / C::STAGES) & 1u;
+          mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, p.err);
+          mbar_arrive_expect_tx(&full[st], C::X_BYTES);
+          tma_load_2d(base + st * C::X_BYTES, &p.tmapA[s], kk * BK, m0, &full[st]);
+        }
+      }
+    }
+    if (warp == EPI_WARP0 + 2 && lane == 0) {
+      // ---------------------------------------------- TMA issuer: raw NF4 codes / absmax
+      const int si = nf4_seg_of(p.nf4, n0);
+      const int y = n0 - p.nf4.seg[si].row_begin;
+      for (int kb = 0; kb < nk0; ++kb) {
+        const int rs = kb % C::RAW_SLOTS;
+        const uint32_t rph = static_cast<uint32_t>(kb / C::RAW_SLOTS) & 1u;
+        mbar_wait_bounded(&raw_empty[rs], rph ^ 1u, abort_flag, p.err);
+        uint8_t* Rc = raw_base + rs * C::RAW_BYTES;
+        mbar_arrive_expect_tx(&raw_full[rs], C::RAW_BYTES);
+        tma_load_2d(Rc, &p.tmapCodes[si], kb * (BK / 2), y, &raw_full[rs]);
+        tma_load_2d(Rc + C::RAW_CODE_BYTES, &p.tmapQ8[si], (kb >> 4) << 4, y, &raw_full[rs]);
+      }
+    }
+    if (warp == EPI_WARP0 && lane == 0) {
+      // ---------------------------------------------- MMA issuer: A (weights) from TMEM
+      const uint32_t idesc = idesc_bf16(C::BW, C::BT, false, false);
+      const uint32_t x0 = smem_u32(base);
+      int st = 0, kb = 0;
+      uint32_t ph = 0;
+      for (int s = 0; s < p.nseg; ++s) {
+        const GemmSeg& sg = p.seg[s];
+        if (!seg_active(sg, n0, C::BW)) continue;
+        const int nk = (sg.K + BK - 1) / BK;
+        for (int kk = 0; kk < nk; ++kk, ++kb) {
+          if (!mbar_test_wait(&full[st], ph)) mbar_wait_bounded(&full[st], ph, abort_flag, p.err);
+          tc_fence_after();
+#pragma unroll
+          for (int j = 0; j < BK / 16; ++j)
+            tc_mma_f16_ts(tmem + C::ACC_COL, tmem + C::W_COL + st * 32 + j * 8,
+                          sw128_kmajor_desc(x0 + st * C::X_BYTES + j * 32), idesc, (kb > 0 || j > 0) ? 1u : 0u);
+          tc_commit(&empty[st]);
+          if (++st == C::STAGES) {
+            st = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+      tc_commit(done);
+    }
+    __syncwarp();
+    // ------------------------------------------------ epilogue: thread = output column w
+    mbar_wait_bounded(done, 0u, abort_flag, p.err);
+    tc_fence_after();
+    const int w = n0 + q * 32 + lane;
+    uint16_t* out = static_cast<uint16_t*>(p.out);
+#pragma unroll 1
+    for (int tc = 0; tc < C::BT; tc += 16) {
+      uint32_t acc[16];
+      tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + C::ACC_COL + tc, acc);
+      tmem_ld_wait();
+      float v[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) v[j] = p.alpha * __uint_as_float(acc[j]);
+      if (w < p.N) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int t = m0 + tc + j;
+          if (t < p.M) {
+            const __nv_bfloat16 b = __float2bfloat16_rn(v[j]);
+            out[static_cast<long long>(t) * p.ldo + w] = *reinterpret_cast<const uint16_t*>(&b);
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == EPI_WARP0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
 // Sum of the split-K partial tiles in split order, then the normal epilogue (the wide form
 // for many splits: one thread per 8 outputs instead of one CTA per tile, 128-thread blocks so
 // that the few thousand threads of a LoRA-sized output spread over more SMs).
@@ -1264,6 +1512,63 @@ cudaError_t launch_tile(const GemmParams& p, cudaStream_t st) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// The TMEM-A forward kernel (gemm_ts_kernel) serves forward NF4 GEMMs without residual, RoPE,
+// accumulation or fp32 / transposed output, whose LoRA segments are plain bf16 operands, when
+// they have at least TS_MIN_TILES 128 x 256 output tiles (fewer tiles leave SMs idle: the
+// shared-memory kernel's 128-column tiles, split-K or stream-K serve those).  RoPE stays on the
+// shared-memory kernel: in the transposed tile a thread holds one column for 16 tokens, so the
+// rotation's cos / sin come one token (one L2 round trip) at a time; measured in the 8B step,
+// that epilogue made the q|k|v launch 182 us against 58.  SOUP_GEMM_TS=0 turns it off (read
+// per launch).
+constexpr int TS_MIN_TILES = 96;
+bool ts_enabled() {
+  const char* e = std::getenv("SOUP_GEMM_TS");
+  return !(e && e[0] == '0');
+}
+bool ts_applicable(const GemmParams& p) {
+  if (!ts_enabled() || !tma_operands_allowed() || !raw_tma_allowed()) return false;
+  if (p.nseg < 1 || p.seg[0].K <= 0 || p.seg[0].B.kind != OP_NF4_K || p.seg[0].A.kind != OP_BF16_K) return false;
+  if (p.residual || p.accumulate || p.out_f32 || p.out_trans) return false;
+  if (p.seg[0].K % 1024 != 0 || p.seg[0].B.row_lo > 0 || p.seg[0].B.row_hi < p.N) return false;
+  if (p.rope_cols > 0) return false;
+  for (int s = 0; s < p.nseg; ++s) {
+    const GemmSeg& sg = p.seg[s];
+    if (sg.A.scale != 1.f || sg.B.scale != 1.f) return false;
+    if (s == 0) continue;
+    if (sg.K <= 0 || sg.K % 8 != 0 || sg.A.kind != OP_BF16_K || sg.B.kind != OP_BF16_K) return false;
+    if (sg.B.ld % 8 != 0 || !aligned16(sg.B.ptr)) return false;
+  }
+  const long long tiles = static_cast<long long>((p.N + TsCfg::BW - 1) / TsCfg::BW) * ((p.M + TsCfg::BT - 1) / TsCfg::BT);
+  return tiles >= TS_MIN_TILES;
+}
+// Sets up the descriptors and launches gemm_ts_kernel; false (nothing launched) when a
+// descriptor cannot be encoded, so the caller takes the shared-memory kernel.
+bool launch_ts(GemmParams& p, cudaStream_t st, cudaError_t* err) {
+  if (!setup_raw_tma(p, TsCfg::BW)) return false;
+  for (int s = 0; s < p.nseg; ++s) {
+    const GemmSeg& sg = p.seg[s];
+    if (sg.K > 0 && !encode_kmajor_bf16(&p.tmapA[s], sg.A.ptr, sg.K, p.M, sg.A.ld, TsCfg::BT)) return false;
+  }
+  p.raw_tma = 1;
+  p.bn = TsCfg::BW;
+  p.splits = 1;
+  p.sk_ctas = 0;
+  static std::atomic<int> attr_done{0};
+  if (!attr_done.load()) {
+    const cudaError_t e = cudaFuncSetAttribute(gemm_ts_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               TsCfg::SMEM_BYTES);
+    if (e != cudaSuccess) {
+      *err = e;
+      return true;
+    }
+    attr_done.store(1);
+  }
+  const dim3 grid((p.N + TsCfg::BW - 1) / TsCfg::BW, (p.M + TsCfg::BT - 1) / TsCfg::BT, 1);
+  gemm_ts_kernel<<<grid, GEMM_THREADS, TsCfg::SMEM_BYTES, st>>>(p);
+  *err = cudaGetLastError();
+  return true;
+}
+
 // SMs of the current device (stream-K spreads a GEMM over one CTA per SM)
 int sm_count() {
   static std::atomic<int> cached[64];
@@ -1483,6 +1788,13 @@ cudaError_t gemm_launch(const GemmParams& p_in, cudaStream_t st) {
     if (sg.A.kind == OP_NF4_K || sg.A.kind == OP_NF4_MN) return cudaErrorInvalidValue;  // NF4 only as B
     if (sg.B.kind == OP_NF4_K && (p.nf4.cols % 8 != 0 || sg.K > p.nf4.cols)) return cudaErrorInvalidValue;
     if (sg.B.kind == OP_NF4_MN && (p.nf4.cols % 8 != 0 || p.N > p.nf4.cols)) return cudaErrorInvalidValue;
+  }
+  if (ts_applicable(p)) {
+    cudaError_t e = cudaSuccess;
+    if (launch_ts(p, st, &e)) {
+      ++g_kernel_launches;
+      return e;
+    }
   }
   const GemmPlan pl = gemm_plan(p, sm_count(), sk_enabled());
   const int MT = pl.mt, BN = pl.bn;

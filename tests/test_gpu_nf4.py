@@ -75,3 +75,29 @@ def test_nf4_matmul_vs_float64(M_, N, K, transpose):
     assert rel_err(got, want) < 4e-3
     assert np.max(np.abs(got - want)) <= 2.0 ** -7 * np.max(np.abs(want)) + 1e-3
 
+
+
+# Forward GEMMs without a residual and with at least 96 output tiles of 128 weight rows x 256
+# tokens take the kernel whose dequantised weight tile lives in tensor memory (the MMA's A
+# operand); the second shape has a ragged last weight tile and a ragged last token tile.
+@pytest.mark.parametrize("M_,N,K", [(512, 6144, 4096), (300, 12352, 1024)])
+def test_nf4_matmul_tmem_weight_form_vs_float64(M_, N, K, monkeypatch):
+    from layer_streamed_nf4_lut_b200 import model as M
+    from tests.gpu_util import bf16_tensor
+    w = synth.normal(19, N + K, (N, K), 0.02)
+    q = _gpu_quant(w)
+    Wd = nf4.dequant(nf4.quantise(w)).astype(np.float64)
+    x = bf16_tensor(synth.bf16_bits_from_f32(synth.normal(20, M_, (M_, K), 1.0)))
+    want = to64(x) @ Wd.T
+    outs = {}
+    for flag in ("1", "0"):  # the tensor-memory form, then the shared-memory kernel
+        monkeypatch.setenv("SOUP_GEMM_TS", flag)
+        y = M.nf4_matmul(x, q)
+        torch.cuda.synchronize()
+        got = to64(y)
+        assert rel_err(got, want) < 4e-3
+        assert np.max(np.abs(got - want)) <= 2.0 ** -7 * np.max(np.abs(want)) + 1e-3
+        outs[flag] = y
+    if M_ % 256 == 0 and N % 128 == 0:
+        # whole tiles on both sides: the same products summed in the same k order
+        assert torch.equal(outs["1"], outs["0"])
