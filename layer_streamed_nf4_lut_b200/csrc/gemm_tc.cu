@@ -991,15 +991,21 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc_kernel(const __grid_c
 }
 
 // ---------------------------------------------------------------- the TMEM-A forward kernel
-// NF4 forward GEMMs with enough output tiles (y = x W^T (+ LoRA K-blocks), no residual): the
-// tile is transposed, D^T[w, t] = W[w, :] . x[t, :], 128 weight rows (TMEM lanes) x 256 tokens.
+// NF4 forward GEMMs with enough output tiles (y = x W^T (+ LoRA K-blocks) (+ residual), RoPE on
+// the q | k columns): the tile is transposed, D^T[w, t] = W[w, :] . x[t, :], 128 weight rows
+// (TMEM lanes) x 256 tokens.
 // The producers put the dequantised weight tile straight into tensor memory (tcgen05.st, one
 // weight row per thread) and tcgen05.mma reads it there as its A operand; only the activation
 // tile (TMA) and the raw NF4 bytes pass through shared memory.  Against the shared-memory form
 // (activations and decoded weights both staged in shared memory and both read by every MMA)
 // this moves ~76 KB of shared memory per 4.2 MFLOP k-block instead of ~124 KB.  LoRA segments
 // are further K-blocks: the producers copy the LoRA-B rows of the tile (bf16, zero outside the
-// segment's row window) into tensor memory and the u tile comes by TMA.
+// segment's row window) into tensor memory and the u tile comes by TMA.  The epilogue's
+// per-(token, column) inputs, the residual block or the tile's 256 positions' cos / sin rows,
+// come by TMA as further entries of the activation ring, into the stages the last k-blocks
+// free first, and are read from shared memory: in the transposed tile a thread walks tokens,
+// and fetching those values from global memory one token at a time made the q|k|v launch 182 us
+// against 58 in the 8B step.
 struct TsCfg {
   static constexpr int BW = 128;  // weight rows (output columns) per CTA
   static constexpr int BT = 256;  // tokens (output rows) per CTA: the MMA's N
@@ -1043,7 +1049,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_ts_kernel(const __grid_c
   uint64_t* raw_full = empty + C::STAGES;
   uint64_t* raw_empty = raw_full + C::RAW_SLOTS;
   uint64_t* done = raw_empty + C::RAW_SLOTS;
-  static_assert(64 + 8 * (2 * C::STAGES + 2 * C::RAW_SLOTS + 1) <= C::CTRL_BYTES, "control block overflow");
+  uint64_t* res_full = done + 1;
+  static_assert(64 + 8 * (2 * C::STAGES + 2 * C::RAW_SLOTS + 2) <= C::CTRL_BYTES, "control block overflow");
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n0 = blockIdx.x * C::BW;  // first weight row = output column
@@ -1058,6 +1065,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_ts_kernel(const __grid_c
       mbar_init(&raw_empty[r], GROUP_THREADS / 32);
     }
     mbar_init(done, 1);
+    mbar_init(res_full, 1);
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -1163,6 +1171,28 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_ts_kernel(const __grid_c
           tma_load_2d(base + st * C::X_BYTES, &p.tmapA[s], kk * BK, m0, &full[st]);
         }
       }
+      if (p.residual) {
+        // residual rows [m0, m0 + 128) and [m0 + 128, m0 + 256) into the stages that ring
+        // entries kb and kb + 1 would use (free once the MMAs five entries back retire)
+        mbar_arrive_expect_tx(res_full, 2 * 128 * C::BW * 2);
+        for (int h = 0; h < 2; ++h) {
+          const int g = kb + h, st = g % C::STAGES;
+          const uint32_t ph = static_cast<uint32_t>(g / C::STAGES) & 1u;
+          mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, p.err);
+          tma_load_2d(base + st * C::X_BYTES, &p.tmapB[0], n0, m0 + 128 * h, res_full);
+        }
+      } else if (p.rope_cols > 0 && n0 < p.rope_cols) {
+        // cos rows of positions [pos0, pos0 + 128), [pos0 + 128, +256), then the sin rows, as
+        // ring entries kb .. kb + 3 (the tile's tokens have consecutive positions)
+        const int pos0 = m0 % p.rope_S;
+        mbar_arrive_expect_tx(res_full, 4 * 128 * 64 * 4);
+        for (int e = 0; e < 4; ++e) {
+          const int g = kb + e, st = g % C::STAGES;
+          const uint32_t ph = static_cast<uint32_t>(g / C::STAGES) & 1u;
+          mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, p.err);
+          tma_load_2d(base + st * C::X_BYTES, &p.tmapB[1 + (e >> 1)], 0, pos0 + 128 * (e & 1), res_full);
+        }
+      }
     }
     if (warp == EPI_WARP0 + 2 && lane == 0) {
       // ---------------------------------------------- TMA issuer: raw NF4 codes / absmax
@@ -1210,6 +1240,21 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_ts_kernel(const __grid_c
     tc_fence_after();
     const int w = n0 + q * 32 + lane;
     uint16_t* out = static_cast<uint16_t*>(p.out);
+    int nkb_all = 0;
+    for (int s = 0; s < p.nseg; ++s)
+      if (seg_active(p.seg[s], n0, C::BW)) nkb_all += (p.seg[s].K + BK - 1) / BK;
+    const bool rope_tile = !p.residual && p.rope_cols > 0 && n0 < p.rope_cols;
+    if (p.residual || rope_tile) mbar_wait_bounded(res_full, 0u, abort_flag, p.err);
+    const uint8_t* rs0 = base + (nkb_all % C::STAGES) * C::X_BYTES;
+    const uint8_t* rs1 = base + ((nkb_all + 1) % C::STAGES) * C::X_BYTES;
+    const float* cos0 = reinterpret_cast<const float*>(rs0);
+    const float* cos1 = reinterpret_cast<const float*>(rs1);
+    const float* sin0 = reinterpret_cast<const float*>(base + ((nkb_all + 2) % C::STAGES) * C::X_BYTES);
+    const float* sin1 = reinterpret_cast<const float*>(base + ((nkb_all + 3) % C::STAGES) * C::X_BYTES);
+    // the pair exchange in the stage of the last k-block (ring entry nkb_all - 1 = nkb_all + 4)
+    float* xch = reinterpret_cast<float*>(base + ((nkb_all + 4) % C::STAGES) * C::X_BYTES);
+    const int dr = q * 32 + lane, pdr = dr ^ 64, ci = dr & 63;
+    const bool first = dr < 64;
 #pragma unroll 1
     for (int tc = 0; tc < C::BT; tc += 16) {
       uint32_t acc[16];
@@ -1218,6 +1263,27 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_ts_kernel(const __grid_c
       float v[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) v[j] = p.alpha * __uint_as_float(acc[j]);
+      if (p.residual) {
+        const uint8_t* rb = (tc < 128 ? rs0 : rs1) + (tc & 127) * (C::BW * 2) + (q * 32 + lane) * 2;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) v[j] += bf16_to_f32(*reinterpret_cast<const uint16_t*>(rb + j * C::BW * 2));
+      }
+      if (rope_tile) {
+        // rows dr and dr ^ 64 of the tile are the pair (i, i + 64) of one head
+#pragma unroll
+        for (int j = 0; j < 16; ++j) xch[dr * 17 + j] = v[j];
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        const float* ct = (tc < 128 ? cos0 : cos1) + (tc & 127) * 64 + ci;
+        const float* stb = (tc < 128 ? sin0 : sin1) + (tc & 127) * 64 + ci;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const float other = xch[pdr * 17 + j];
+          const float c = ct[j * 64], sn = stb[j * 64];
+          const float x1 = first ? v[j] : other, x2 = first ? other : v[j];
+          v[j] = first ? x1 * c - x2 * sn : x2 * c + x1 * sn;
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+      }
       if (w < p.N) {
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
@@ -1512,14 +1578,12 @@ cudaError_t launch_tile(const GemmParams& p, cudaStream_t st) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// The TMEM-A forward kernel (gemm_ts_kernel) serves forward NF4 GEMMs without residual, RoPE,
-// accumulation or fp32 / transposed output, whose LoRA segments are plain bf16 operands, when
-// they have at least TS_MIN_TILES 128 x 256 output tiles (fewer tiles leave SMs idle: the
-// shared-memory kernel's 128-column tiles, split-K or stream-K serve those).  RoPE stays on the
-// shared-memory kernel: in the transposed tile a thread holds one column for 16 tokens, so the
-// rotation's cos / sin come one token (one L2 round trip) at a time; measured in the 8B step,
-// that epilogue made the q|k|v launch 182 us against 58.  SOUP_GEMM_TS=0 turns it off (read
-// per launch).
+// The TMEM-A forward kernel (gemm_ts_kernel) serves forward NF4 GEMMs without accumulation or
+// fp32 / transposed output, whose LoRA segments are plain bf16 operands, when they have at least
+// TS_MIN_TILES 128 x 256 output tiles (fewer tiles leave SMs idle: the shared-memory kernel's
+// 128-column tiles, split-K or stream-K serve those).  A residual is a bf16 block of the output's
+// shape; RoPE needs 128-column heads, whole 256-token tiles of consecutive positions and no
+// shared-prefix pair layout.  SOUP_GEMM_TS=0 turns it off (read per launch).
 constexpr int TS_MIN_TILES = 96;
 bool ts_enabled() {
   const char* e = std::getenv("SOUP_GEMM_TS");
@@ -1528,9 +1592,12 @@ bool ts_enabled() {
 bool ts_applicable(const GemmParams& p) {
   if (!ts_enabled() || !tma_operands_allowed() || !raw_tma_allowed()) return false;
   if (p.nseg < 1 || p.seg[0].K <= 0 || p.seg[0].B.kind != OP_NF4_K || p.seg[0].A.kind != OP_BF16_K) return false;
-  if (p.residual || p.accumulate || p.out_f32 || p.out_trans) return false;
+  if (p.accumulate || p.out_f32 || p.out_trans) return false;
+  if (p.residual && (p.ldr % 8 != 0 || !aligned16(p.residual))) return false;
   if (p.seg[0].K % 1024 != 0 || p.seg[0].B.row_lo > 0 || p.seg[0].B.row_hi < p.N) return false;
-  if (p.rope_cols > 0) return false;
+  if (p.rope_cols > 0 && (p.residual || p.rope_d != 128 || p.rope_rl != 0 || p.rope_S % TsCfg::BT != 0 ||
+                         p.M % TsCfg::BT != 0 || p.rope_cols % TsCfg::BW != 0))
+    return false;
   for (int s = 0; s < p.nseg; ++s) {
     const GemmSeg& sg = p.seg[s];
     if (sg.A.scale != 1.f || sg.B.scale != 1.f) return false;
@@ -1548,6 +1615,16 @@ bool launch_ts(GemmParams& p, cudaStream_t st, cudaError_t* err) {
   for (int s = 0; s < p.nseg; ++s) {
     const GemmSeg& sg = p.seg[s];
     if (sg.K > 0 && !encode_kmajor_bf16(&p.tmapA[s], sg.A.ptr, sg.K, p.M, sg.A.ld, TsCfg::BT)) return false;
+  }
+  if (p.residual && !encode_cached(&p.tmapB[0], p.residual, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                                   static_cast<unsigned long long>(p.N), static_cast<unsigned long long>(p.M),
+                                   static_cast<unsigned long long>(p.ldr) * 2, TsCfg::BW, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return false;
+  if (p.rope_cols > 0) {
+    for (int t = 0; t < 2; ++t)
+      if (!encode_cached(&p.tmapB[1 + t], t ? p.rope_sin : p.rope_cos, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 64,
+                         static_cast<unsigned long long>(p.rope_S), 64 * 4, 64, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return false;
   }
   p.raw_tma = 1;
   p.bn = TsCfg::BW;
